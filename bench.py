@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Throughput of the gated delta-rule chunked forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one gdr_fwd_chunked call over the whole workload (every chunk's
+UT/WY transform, the state scan, the outputs and the final state), on
+synthetic seeded inputs already resident in HBM. The default workload is the
+nanochat-scale GDN layer: B=8, T=2048, Hk=Hv=16, Dk=Dv=128, bf16 q/k/v/o,
+fp32 scalar gates, beta and state, h0 ~ 0.02 N(0,1).
+
+Prints one JSON line (rank 0). ``value`` is B*T*Hv head-tokens per second over
+all ranks (each rank runs its own full workload: weak scaling, no data-path
+collective), timed on the device with CUDA events, max over ranks. ``e2e`` is
+the same metric through the public Python API with pinned host buffers, the
+host<->device copies of every step's inputs and results inside the timed
+region. ``roofline`` compares algorithmic HBM bytes per launch with the
+measured HBM copy bandwidth. ``cpu_baseline`` times the fp64 CPU oracle on a
+bounded sample of the same workload on this host's cores.
+
+``--impl reference`` times that oracle alone (the reference arm): each step is
+a bounded sample of the workload on the host cores.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta fwd tokens/s (B·T·Hv per sec) bf16 d=128; % of roofline"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="gdn_bf16")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+# ----------------------------------------------------------------------------- accounting
+def algorithmic_bytes(w):
+    """HBM bytes the method must move per call: q, k, v, o, g, beta, h0 and hT."""
+    es = 2 if w.dtype == "bf16" else 4
+    qk = 2 * w.B * w.T * w.Hk * w.Dk * es
+    vo = 2 * w.B * w.T * w.Hv * w.Dv * es
+    g = w.B * w.T * w.Hv * (w.Dk if w.gate == "channel" else 1) * 4
+    beta = w.B * w.T * w.Hv * 4
+    states = (2 if w.h0_std > 0 else 1) * w.B * w.Hv * w.Dk * w.Dv * 4
+    return qk + vo + g + beta + states
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_sha():
+    csrc = os.path.join(ROOT, "gated_delta_rule_68_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh", ".h")):
+            h.update(n.encode())
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from a committed ncu capture, if the kernels are unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)[workload]
+    except Exception:
+        return None, None
+    if d.get("kernel_sources_sha256") != kernel_sources_sha():
+        return None, d.get("kernel")
+    return float(d["dram_bytes_per_launch"]), d.get("kernel")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML every few ms while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples, self.reasons = [], set()
+        self.ok = False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML unavailable: report that instead of clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(s)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(w, target_s=12.0, seed_rank=0):
+    """Time the fp64 oracle on a bounded sample of the workload: whole sequences of some
+    (b, h) units, chosen so the run takes about target_s seconds on this host."""
+    import oracle
+    from gated_delta_rule_68_b200.workloads import make_inputs
+
+    small = w.with_(B=1, Hk=1, Hv=1)
+    inp = make_inputs(small.with_(seed=w.seed + seed_rank), "cpu")
+    cores = oracle.threads_used(0, 1 << 30)
+    t0 = time.perf_counter()
+    oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], nthreads=1)
+    t_unit = time.perf_counter() - t0
+    units = max(cores, min(w.B * w.Hv, int(target_s * cores / max(t_unit, 1e-6))))
+    units = min(units, w.B * w.Hv)
+    sample = w.with_(B=units, Hk=1, Hv=1)
+    inp = make_inputs(sample, "cpu")
+    q, k, v, g, beta, h0 = (inp[n] for n in ("q", "k", "v", "g", "beta", "h0"))
+    qd, kd, vd, gd, bd = (x.double().numpy() for x in (q, k, v, g, beta))
+    hd = None if h0 is None else h0.double().numpy()
+    t0 = time.perf_counter()
+    oracle.recurrent(qd, kd, vd, gd, bd, hd, nthreads=0)
+    dt = time.perf_counter() - t0
+    return {
+        "value": units * w.T / dt, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+        "kind": "oracle",
+        "sample": f"{units} whole (batch row, value head) sequences of T={w.T}, Dk=Dv={w.Dk}, "
+                  f"{w.gate} gate, fp64 token recurrence; {dt:.1f} s",
+        "seconds": dt,
+    }
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    from gated_delta_rule_68_b200.workloads import make_inputs
+
+    cores = oracle.threads_used(0, 1 << 30)
+    units = max(cores, 8)
+    sample = w.with_(B=units, Hk=1, Hv=1)
+    inp = make_inputs(sample, "cpu")
+    arrs = [None if inp[n] is None else inp[n].double().numpy()
+            for n in ("q", "k", "v", "g", "beta", "h0")]
+    times = []
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.recurrent(*arrs, nthreads=0)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            times.append(dt)
+    per_step = sum(times) / len(times)
+    value = units * w.T / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same recipe as the GPU arm)",
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+                         "kind": "oracle",
+                         "sample": f"each step: {units} whole (batch row, value head) sequences of "
+                                   f"T={w.T} of the workload, fp64 token recurrence"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world):
+    ab = algorithmic_bytes(w)
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "Dk": w.Dk, "Dv": w.Dv,
+            "gate": w.gate, "chunk": 64, "global_batch": w.B * world,
+            "parallelism": f"dp{world} (independent batch shards, no collective)",
+            "l2": ("inputs exceed L2, no flush" if ab > L2_BYTES else "L2 flushed between steps")}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from gated_delta_rule_68_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import gated_delta_rule_68_b200 as gdr
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    wr = w.with_(seed=w.seed + rank)
+    inp_cpu = make_inputs(wr, "cpu")
+    inp = {n: (None if t is None else t.to(dev)) for n, t in inp_cpu.items()}
+    o = torch.empty((w.B, w.T, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)
+    hT = torch.empty((w.B, w.Hv, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+    need = gdr.gdr_fwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, w.gate_mode,
+                                      gdr.GDR_BF16 if w.dtype == "bf16" else gdr.GDR_FP32)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    flush = None if algorithmic_bytes(w) > L2_BYTES else torch.empty(256 * 2 ** 20, dtype=torch.uint8,
+                                                                      device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if flush is not None:
+            flush.add_(1)
+        gdr.gdr_fwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], o=o, hT=hT,
+                            workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = gdr.gdr_kernel_launches()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    launches = gdr.gdr_kernel_launches() - n0
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {n: (None if x is None else x.pin_memory()) for n, x in inp_cpu.items()}
+        dbuf = {n: (None if x is None else torch.empty_like(x, device=dev)) for n, x in inp_cpu.items()}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hT_h = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
+        d2h = o_h.numel() * o_h.element_size() + hT_h.numel() * hT_h.element_size()
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            for n, x in host.items():
+                if x is not None:
+                    dbuf[n].copy_(x, non_blocking=True)
+            gdr.gdr_fwd_chunked(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["h0"], o=o,
+                                hT=hT, workspace=ws, stream=stream)
+            o_h.copy_(o, non_blocking=True)
+            hT_h.copy_(hT, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * w.head_tokens / (float(te.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": float(te.item())}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(w)
+    achieved = alg / (ms / 1e3) / 1e9
+    traffic, traffic_kernel = recorded_traffic(w.name)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(w)
+    line = {
+        "metric": METRIC,
+        "value": world * w.head_tokens / (ms_max / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded CPU generator; q,k L2-normalised N(0,1); v N(0,1); "
+                "g logsigmoid(N(3,1)); beta sigmoid(N(0,1)); h0 0.02 N(0,1))",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg,
+                     "traffic": traffic, "traffic_kernel": traffic_kernel,
+                     "kernel": "gdr_fwd_chunked step"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "launches_per_step": launches / args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

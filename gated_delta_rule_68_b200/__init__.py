@@ -1,0 +1,161 @@
+"""Python binding of libgdr, the B200 (sm_100a) gated delta-rule library.
+
+The functions here carry the C ABI's names (include/gdr.h) and only marshal
+arguments: they check dtypes and shapes, take raw device pointers from torch
+tensors, pass the current CUDA stream, and turn a non-zero status into a
+``GdrError``. Every step of the computation runs in the library's CUDA kernels;
+there is no CPU fallback. If libgdr.so is missing the first call raises.
+
+Layouts (row-major, contiguous): q,k [B,T,Hk,Dk]; v,o [B,T,Hv,Dv]; g [B,T,Hv]
+(scalar gate) or [B,T,Hv,Dk] (per-channel gate) in fp32; beta [B,T,Hv] fp32;
+h0, hT, state [B,Hv,Dk,Dv] fp32. Decode drops the T axis.
+"""
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgdr.so")
+
+GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_MISALIGNED, GDR_ERR_WORKSPACE, GDR_ERR_CUDA = range(6)
+GDR_GATE_SCALAR, GDR_GATE_CHANNEL = 0, 1
+GDR_BF16, GDR_FP32 = 0, 1
+
+# Every symbol include/gdr.h declares.
+EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
+           "gdr_fwd_chunked", "gdr_decode_step")
+
+_lib = None
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"libgdr status {status}: {message}")
+        self.status = status
+
+
+def lib():
+    """Load libgdr.so (built in-tree by ``python -m gated_delta_rule_68_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m gated_delta_rule_68_b200.build` (no fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.gdr_version.restype = i
+        L.gdr_version.argtypes = []
+        L.gdr_last_error.restype = ctypes.c_char_p
+        L.gdr_last_error.argtypes = []
+        L.gdr_kernel_launches.restype = ctypes.c_ulonglong
+        L.gdr_kernel_launches.argtypes = []
+        L.gdr_fwd_workspace_size.restype = sz
+        L.gdr_fwd_workspace_size.argtypes = [i] * 8
+        L.gdr_fwd_chunked.restype = i
+        L.gdr_fwd_chunked.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp] + [i] * 8 + [vp, sz, vp]
+        L.gdr_decode_step.restype = i
+        L.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [i] * 7 + [vp]
+        _lib = L
+    return _lib
+
+
+def gdr_version() -> int:
+    return int(lib().gdr_version())
+
+
+def gdr_last_error() -> str:
+    return lib().gdr_last_error().decode()
+
+
+def gdr_kernel_launches() -> int:
+    return int(lib().gdr_kernel_launches())
+
+
+def _check(status):
+    if status != GDR_OK:
+        raise GdrError(status, gdr_last_error())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return GDR_BF16
+    if t.dtype == torch.float32:
+        return GDR_FP32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def gdr_fwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
+    return int(lib().gdr_fwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype))
+
+
+def gdr_fwd_chunked(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True,
+                    workspace=None, stream=None):
+    """Chunked forward. Returns (o, hT); hT is None when want_hT is False and no hT is given."""
+    B, T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    dt = _dtype_code(q)
+    gate_mode = GDR_GATE_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    _need(q, "q", q.dtype)
+    _need(k, "k", q.dtype, q.shape)
+    _need(v, "v", q.dtype, (B, T, Hv, Dv))
+    _need(g, "g", torch.float32, (B, T, Hv) if gate_mode == 0 else (B, T, Hv, Dk))
+    _need(beta, "beta", torch.float32, (B, T, Hv))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (B, Hv, Dk, Dv))
+    if o is None:
+        o = torch.empty((B, T, Hv, Dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, T, Hv, Dv))
+    if hT is None and want_hT:
+        hT = torch.empty((B, Hv, Dk, Dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _need(hT, "hT", torch.float32, (B, Hv, Dk, Dv))
+    need = gdr_fwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dt)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().gdr_fwd_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+                                 _ptr(hT), B, T, Hk, Hv, Dk, Dv, gate_mode, dt, _ptr(workspace),
+                                 ws_bytes, _stream(stream)))
+    return o, hT
+
+
+def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One decode step; ``state`` is updated in place. Returns o [B,Hv,Dv]."""
+    B, Hk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    dt = _dtype_code(q)
+    gate_mode = GDR_GATE_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
+    _need(q, "q", q.dtype)
+    _need(k, "k", q.dtype, q.shape)
+    _need(v, "v", q.dtype, (B, Hv, Dv))
+    _need(g, "g", torch.float32, (B, Hv) if gate_mode == 0 else (B, Hv, Dk))
+    _need(beta, "beta", torch.float32, (B, Hv))
+    _need(state, "state", torch.float32, (B, Hv, Dk, Dv))
+    if o is None:
+        o = torch.empty((B, Hv, Dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, Hv, Dv))
+    _check(lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o),
+                                 B, Hk, Hv, Dk, Dv, gate_mode, dt, _stream(stream)))
+    return o

@@ -1,0 +1,142 @@
+// C ABI of libgdr: argument checks, workspace sizing and kernel dispatch.
+// The contract of every entry point is documented in include/gdr.h.
+#include <stdarg.h>
+#include <atomic>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/gdr.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "no error";
+std::atomic<unsigned long long> g_launches{0};
+
+int fail(int status, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool supported_dim(int d) { return d == 64 || d == 128; }
+
+int check_common(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype)
+{
+    if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0)
+        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d Hk=%d Hv=%d Dk=%d Dv=%d)",
+                    B, T, Hk, Hv, Dk, Dv);
+    if (Hv % Hk != 0)
+        return fail(GDR_ERR_INVALID_ARG, "Hv (%d) must be a multiple of Hk (%d)", Hv, Hk);
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL)
+        return fail(GDR_ERR_INVALID_ARG, "gate_mode must be GDR_GATE_SCALAR or GDR_GATE_CHANNEL (got %d)", gate_mode);
+    if (dtype != GDR_BF16 && dtype != GDR_FP32)
+        return fail(GDR_ERR_INVALID_ARG, "dtype must be GDR_BF16 or GDR_FP32 (got %d)", dtype);
+    if (!supported_dim(Dk) || !supported_dim(Dv))
+        return fail(GDR_ERR_UNSUPPORTED, "Dk and Dv must each be 64 or 128 (got Dk=%d Dv=%d)", Dk, Dv);
+    if ((long long)B * Hv > (1LL << 31) - 1)
+        return fail(GDR_ERR_INVALID_ARG, "B*Hv too large");
+    return GDR_OK;
+}
+
+gdr::FwdArgs make_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      const float *h0, void *o, float *hT, int B, int T, int Hk, int Hv, int Dk, int Dv,
+                      int gate_mode, int dtype)
+{
+    gdr::FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0; a.o = o; a.hT = hT;
+    a.B = B; a.T = T; a.Hk = Hk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv;
+    a.gate_mode = gate_mode; a.dtype = dtype;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr_version(void) { return 100; }
+
+const char *gdr_last_error(void) { return g_err; }
+
+unsigned long long gdr_kernel_launches(void) { return g_launches.load(); }
+
+size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype)
+{
+    if (check_common(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) != GDR_OK) return 0;
+    if (B == 0 || T == 0) return 0;
+    const gdr::FwdArgs a = make_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                    nullptr, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    return gdr::simt_workspace_size(a);
+}
+
+int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    const float *h0, void *o, float *hT, int B, int T, int Hk, int Hv, int Dk, int Dv,
+                    int gate_mode, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int st = check_common(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (st != GDR_OK) return st;
+    const bool work = B > 0 && T > 0;
+    if (work && (!q || !k || !v || !g || !beta || !o))
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta and o must be non-NULL");
+    const void *ptrs[] = {q, k, v, g, beta, h0, o, hT};
+    const char *names[] = {"q", "k", "v", "g", "beta", "h0", "o", "hT"};
+    for (int i = 0; i < 8; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if (workspace && ((uintptr_t)workspace & 255u))
+        return fail(GDR_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (o && (o == q || o == k || o == v))
+        return fail(GDR_ERR_INVALID_ARG, "o must not alias q, k or v");
+    cudaStream_t s = (cudaStream_t)stream;
+
+    if (!work) {  // empty input: hT = h0 (or zeros)
+        if (hT) {
+            const size_t bytes = (size_t)B * Hv * Dk * Dv * sizeof(float);
+            cudaError_t e = h0 ? (h0 == hT ? cudaSuccess
+                                           : cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, s))
+                               : cudaMemsetAsync(hT, 0, bytes, s);
+            if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA: %s", cudaGetErrorString(e));
+        }
+        return GDR_OK;
+    }
+
+    const gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    const size_t need = gdr::simt_workspace_size(a);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, workspace_bytes,
+                    workspace ? "" : " (NULL)");
+    cudaError_t e = gdr::launch_fwd_simt(a, workspace, s);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += 3;
+    return GDR_OK;
+}
+
+int gdr_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    float *state, void *o, int B, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype,
+                    void *stream)
+{
+    int st = check_common(B, 1, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (st != GDR_OK) return st;
+    if (B == 0) return GDR_OK;
+    if (!q || !k || !v || !g || !beta || !state || !o)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, state and o must be non-NULL");
+    const void *ptrs[] = {q, k, v, g, beta, state, o};
+    const char *names[] = {"q", "k", "v", "g", "beta", "state", "o"};
+    for (int i = 0; i < 7; ++i)
+        if (!aligned16(ptrs[i])) return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    gdr::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.o = o;
+    a.B = B; a.Hk = Hk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.gate_mode = gate_mode; a.dtype = dtype;
+    cudaError_t e = gdr::launch_decode(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += 1;
+    return GDR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,30 @@
+// Internal launch interface between the C ABI (gdr_api.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdr {
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    float *state;
+    void *o;
+    int B, Hk, Hv, Dk, Dv, gate_mode, dtype;
+};
+
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *g, *beta, *h0;
+    void *o;
+    float *hT;
+    int B, T, Hk, Hv, Dk, Dv, gate_mode, dtype;
+};
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+
+// fp32 CUDA-core chunked forward (three kernels). Needs simt_workspace_size() bytes.
+size_t simt_workspace_size(const FwdArgs &a);
+cudaError_t launch_fwd_simt(const FwdArgs &a, void *ws, cudaStream_t st);
+
+}  // namespace gdr

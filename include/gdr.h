@@ -1,0 +1,134 @@
+/*
+ * gdr.h - C ABI of libgdr, a B200 (sm_100a) library for the gated delta rule.
+ *
+ * The operation (NextTransformer, "Source notes", section "Linear attention",
+ * rows gdn and kda; Frontier-model atlas, items 01, 03 and 08):
+ *
+ *   for each batch row b and value head h (key head hk = h / (Hv / Hk)):
+ *     S_t = (I - beta_t k_t k_t^T) diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * S is the Dk x Dv ("K x V") state, stored row-major as [Dk][Dv] in fp32.
+ * g_t <= 0 is the log of the decay alpha_t: one scalar per head (Gated
+ * DeltaNet, GDR_GATE_SCALAR) or one value per key channel (Kimi Delta
+ * Attention, GDR_GATE_CHANNEL); in both cases the decay acts before the delta
+ * update. beta_t in (0,1) is the write strength. The readout uses the state
+ * after the update and no scale (scale = 1, "Backend and numerical limits" on
+ * the same page). q and k are used as given: the library does not normalise them.
+ * DeltaNet is the special case g = 0.
+ *
+ * Layouts (all row-major and contiguous; "bf16 or fp32" follows `dtype`):
+ *   q, k      [B, T, Hk, Dk]   bf16 or fp32
+ *   v, o      [B, T, Hv, Dv]   bf16 or fp32
+ *   g         [B, T, Hv]       fp32 (GDR_GATE_SCALAR)
+ *             [B, T, Hv, Dk]   fp32 (GDR_GATE_CHANNEL)
+ *   beta      [B, T, Hv]       fp32
+ *   h0, hT    [B, Hv, Dk, Dv]  fp32
+ * Decode uses the same layouts with T = 1 ([B, H, D]) and an fp32 state.
+ *
+ * Grouped value heads: Hv must be a multiple of Hk; value head h reads key
+ * head h / (Hv / Hk) (contiguous groups, as repeat-interleaving q and k).
+ *
+ * Ownership and execution: every pointer is device memory owned by the
+ * caller. The library never allocates, frees or synchronises; all work is
+ * enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy default
+ * stream) and GDR_OK means "enqueued". Pointers must be 16-byte aligned.
+ * h0 and hT may be the same buffer (in-place state update); o must not alias
+ * any input. No C++ exception crosses this boundary.
+ *
+ * Errors: arguments are checked on the host before anything is launched.
+ * A non-zero status means nothing was enqueued (except GDR_ERR_CUDA, which
+ * reports a launch failure) and gdr_last_error() returns a message for the
+ * calling thread.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,   /* bad size, Hv % Hk != 0, NULL required pointer, bad enum */
+    GDR_ERR_UNSUPPORTED = 2,   /* Dk or Dv not 64 or 128 */
+    GDR_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    GDR_ERR_WORKSPACE = 4,     /* workspace missing or smaller than gdr_fwd_workspace_size() */
+    GDR_ERR_CUDA = 5           /* a CUDA launch or runtime call failed */
+} gdr_status;
+
+enum { GDR_GATE_SCALAR = 0, GDR_GATE_CHANNEL = 1 };
+enum { GDR_BF16 = 0, GDR_FP32 = 1 };
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDR_API int gdr_version(void);
+
+/* Message describing the last non-GDR_OK status returned on the calling thread. */
+GDR_API const char *gdr_last_error(void);
+
+/* Number of kernels this library has enqueued so far in this process (all
+ * threads and devices); lets a caller count the launches inside a timed region. */
+GDR_API unsigned long long gdr_kernel_launches(void);
+
+/*
+ * Bytes of device workspace gdr_fwd_chunked needs for these sizes (0 when it
+ * needs none). Returns 0 for invalid arguments as well; gdr_fwd_chunked then
+ * reports the actual error.
+ */
+GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv,
+                              int gate_mode, int dtype);
+
+/*
+ * Chunked forward over whole sequences (chunks of 64 tokens; the last chunk
+ * of a sequence may be partial).
+ *
+ * Computes o_t for every t in [0, T) and, if hT != NULL, the state after the
+ * last token. h0 == NULL means a zero initial state. The result equals the
+ * token recurrence above (exact chunkwise form; SinkProbe (Attention-Sink)
+ * README, description of its delta-rule layer): per 64-token chunk a UT/WY
+ * transform A = tril(diag(beta)(K*Gamma)(K/Gamma)^T, -1), T = (I + A)^-1,
+ * W = T diag(beta)(K*Gamma), U = T diag(beta) V, then the state scan
+ * U' = U - W S, S <- diag(Gamma_C) S + (K*Gamma_C/Gamma)^T U', and the output
+ * O = (Q*Gamma) S + tril((Q*Gamma)(K/Gamma)^T) U'.
+ *
+ * bf16 inputs run on the tcgen05 tensor cores with fp32 accumulation and an
+ * fp32 carried state; fp32 inputs run in fp32 throughout.
+ * B == 0 or T == 0 is a valid no-op that still writes hT = h0 (or zeros).
+ *
+ * workspace: device buffer of at least gdr_fwd_workspace_size(...) bytes,
+ * 256-byte aligned, owned by the caller; may be NULL when that size is 0.
+ * Its contents on entry are ignored. Two calls that overlap in time on the
+ * GPU must not share one workspace.
+ */
+GDR_API int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, const float *h0, void *o, float *hT,
+                    int B, int T, int Hk, int Hv, int Dk, int Dv,
+                    int gate_mode, int dtype,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step for B independent sequences (the recurrence with T = 1):
+ *   S' = diag(exp(g)) S;  u = beta (v - S'^T k);  S <- S' + k u^T;  o = S^T q.
+ * state [B, Hv, Dk, Dv] fp32 is read and overwritten in place; q, k [B, Hk, Dk],
+ * v, o [B, Hv, Dv] in `dtype`; g [B, Hv] or [B, Hv, Dk] fp32; beta [B, Hv] fp32.
+ * Needs no workspace. Frontier-model atlas, item 03: decay, memory
+ * prediction, delta correction and recurrent read, in that order.
+ */
+GDR_API int gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, float *state, void *o,
+                    int B, int Hk, int Hv, int Dk, int Dv,
+                    int gate_mode, int dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

