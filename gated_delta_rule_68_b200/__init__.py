@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libgdr.so")
 
 GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_MISALIGNED, GDR_ERR_WORKSPACE, GDR_ERR_CUDA = range(6)
 GDR_GATE_SCALAR, GDR_GATE_CHANNEL = 0, 1
-GDR_BF16, GDR_FP32 = 0, 1
+GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
@@ -77,12 +77,15 @@ def _check(status):
         raise GdrError(status, gdr_last_error())
 
 
-def _dtype_code(t):
+def _dtype_code(t, out_dtype):
     if t.dtype == torch.bfloat16:
-        return GDR_BF16
-    if t.dtype == torch.float32:
-        return GDR_FP32
-    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+        if out_dtype in (None, torch.bfloat16):
+            return GDR_BF16, torch.bfloat16
+        if out_dtype == torch.float32:
+            return GDR_BF16_OUT_F32, torch.float32
+    elif t.dtype == torch.float32 and out_dtype in (None, torch.float32):
+        return GDR_FP32, torch.float32
+    raise TypeError(f"unsupported q/k/v dtype {t.dtype} with output dtype {out_dtype}")
 
 
 def _ptr(t):
@@ -111,11 +114,14 @@ def gdr_fwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
 
 
 def gdr_fwd_chunked(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True,
-                    workspace=None, stream=None):
-    """Chunked forward. Returns (o, hT); hT is None when want_hT is False and no hT is given."""
+                    workspace=None, stream=None, out_dtype=None):
+    """Chunked forward. Returns (o, hT); hT is None when want_hT is False and no hT is given.
+    o has q's dtype unless out_dtype=torch.float32 is asked for with bf16 inputs."""
     B, T, Hk, Dk = q.shape
     Hv, Dv = v.shape[2], v.shape[3]
-    dt = _dtype_code(q)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt, odt = _dtype_code(q, out_dtype)
     gate_mode = GDR_GATE_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
     _need(q, "q", q.dtype)
     _need(k, "k", q.dtype, q.shape)
@@ -125,8 +131,8 @@ def gdr_fwd_chunked(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True,
     if h0 is not None:
         _need(h0, "h0", torch.float32, (B, Hv, Dk, Dv))
     if o is None:
-        o = torch.empty((B, T, Hv, Dv), dtype=q.dtype, device=q.device)
-    _need(o, "o", q.dtype, (B, T, Hv, Dv))
+        o = torch.empty((B, T, Hv, Dv), dtype=odt, device=q.device)
+    _need(o, "o", odt, (B, T, Hv, Dv))
     if hT is None and want_hT:
         hT = torch.empty((B, Hv, Dk, Dv), dtype=torch.float32, device=q.device)
     if hT is not None:
@@ -141,11 +147,13 @@ def gdr_fwd_chunked(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True,
     return o, hT
 
 
-def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None, out_dtype=None):
     """One decode step; ``state`` is updated in place. Returns o [B,Hv,Dv]."""
     B, Hk, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
-    dt = _dtype_code(q)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt, odt = _dtype_code(q, out_dtype)
     gate_mode = GDR_GATE_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
     _need(q, "q", q.dtype)
     _need(k, "k", q.dtype, q.shape)
@@ -154,8 +162,8 @@ def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
     _need(beta, "beta", torch.float32, (B, Hv))
     _need(state, "state", torch.float32, (B, Hv, Dk, Dv))
     if o is None:
-        o = torch.empty((B, Hv, Dv), dtype=q.dtype, device=q.device)
-    _need(o, "o", q.dtype, (B, Hv, Dv))
+        o = torch.empty((B, Hv, Dv), dtype=odt, device=q.device)
+    _need(o, "o", odt, (B, Hv, Dv))
     _check(lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o),
                                  B, Hk, Hv, Dk, Dv, gate_mode, dt, _stream(stream)))
     return o

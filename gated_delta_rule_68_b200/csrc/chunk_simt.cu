@@ -327,7 +327,7 @@ struct OutSmem {
     static constexpr size_t bytes = (size_t)(C * (DK + 1) + DK * DV + C * (C + 1) + C * (DV + 1)) * 4;
 };
 
-template <typename TIn, int DK, int DV, int GATE>
+template <typename TIn, typename TOut, int DK, int DV, int GATE>
 __global__ void __launch_bounds__(NT) out_kernel(FwdArgs a, Work w, int NC)
 {
     constexpr int LDK = DK + 1, LDV = DV + 1, LDC = C + 1;
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(NT) out_kernel(FwdArgs a, Work w, int NC)
     for (int idx = tid; idx < C * DV; idx += NT) Up[(idx / DV) * LDV + idx % DV] = Ug[idx];
     __syncthreads();
 
-    TIn *og = (TIn *)a.o;
+    TOut *og = (TOut *)a.o;
     for (int idx = tid; idx < C * DV; idx += NT) {
         const int r = idx / DV, j = idx % DV;
         if (r >= n) continue;
@@ -373,11 +373,11 @@ __global__ void __launch_bounds__(NT) out_kernel(FwdArgs a, Work w, int NC)
 #pragma unroll 8
         for (int c = 0; c < DK; ++c) s += QG[r * LDK + c] * Ss[c * DV + j];
         for (int i = 0; i <= r; ++i) s += Ms[r * LDC + i] * Up[i * LDV + j];
-        In<TIn>::store(og + (((long)b * a.T + t0 + r) * a.Hv + h) * DV + j, s);
+        In<TOut>::store(og + (((long)b * a.T + t0 + r) * a.Hv + h) * DV + j, s);
     }
 }
 
-template <typename TIn, int DK, int DV, int GATE>
+template <typename TIn, typename TOut, int DK, int DV, int GATE>
 cudaError_t launch_t(const FwdArgs &a, const Work &w, cudaStream_t st)
 {
     const int NC = (a.T + C - 1) / C;
@@ -387,27 +387,28 @@ cudaError_t launch_t(const FwdArgs &a, const Work &w, cudaStream_t st)
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1))) return e;
     if ((e = cudaFuncSetAttribute(scan_kernel<TIn, DK, DV, GATE>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2))) return e;
-    if ((e = cudaFuncSetAttribute(out_kernel<TIn, DK, DV, GATE>,
+    if ((e = cudaFuncSetAttribute(out_kernel<TIn, TOut, DK, DV, GATE>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3))) return e;
     prep_kernel<TIn, DK, DV, GATE><<<dim3(NC, a.Hv, a.B), NT, s1, st>>>(a, w, NC);
     scan_kernel<TIn, DK, DV, GATE><<<dim3(DV / DVS, a.Hv, a.B), NT, s2, st>>>(a, w, NC);
-    out_kernel<TIn, DK, DV, GATE><<<dim3(NC, a.Hv, a.B), NT, s3, st>>>(a, w, NC);
+    out_kernel<TIn, TOut, DK, DV, GATE><<<dim3(NC, a.Hv, a.B), NT, s3, st>>>(a, w, NC);
     return cudaGetLastError();
 }
 
-template <typename TIn, int DK, int DV>
+template <typename TIn, typename TOut, int DK, int DV>
 cudaError_t launch_g(const FwdArgs &a, const Work &w, cudaStream_t st)
 {
-    return a.gate_mode == 0 ? launch_t<TIn, DK, DV, 0>(a, w, st) : launch_t<TIn, DK, DV, 1>(a, w, st);
+    return a.gate_mode == 0 ? launch_t<TIn, TOut, DK, DV, 0>(a, w, st)
+                            : launch_t<TIn, TOut, DK, DV, 1>(a, w, st);
 }
 
-template <typename TIn>
+template <typename TIn, typename TOut>
 cudaError_t launch_d(const FwdArgs &a, const Work &w, cudaStream_t st)
 {
-    if (a.Dk == 128 && a.Dv == 128) return launch_g<TIn, 128, 128>(a, w, st);
-    if (a.Dk == 128 && a.Dv == 64) return launch_g<TIn, 128, 64>(a, w, st);
-    if (a.Dk == 64 && a.Dv == 128) return launch_g<TIn, 64, 128>(a, w, st);
-    return launch_g<TIn, 64, 64>(a, w, st);
+    if (a.Dk == 128 && a.Dv == 128) return launch_g<TIn, TOut, 128, 128>(a, w, st);
+    if (a.Dk == 128 && a.Dv == 64) return launch_g<TIn, TOut, 128, 64>(a, w, st);
+    if (a.Dk == 64 && a.Dv == 128) return launch_g<TIn, TOut, 64, 128>(a, w, st);
+    return launch_g<TIn, TOut, 64, 64>(a, w, st);
 }
 
 }  // namespace
@@ -423,7 +424,9 @@ cudaError_t launch_fwd_simt(const FwdArgs &a, void *ws, cudaStream_t st)
 {
     size_t total = 0;
     const Work w = carve(a, ws, &total);
-    return a.dtype == 0 ? launch_d<__nv_bfloat16>(a, w, st) : launch_d<float>(a, w, st);
+    if (!in_bf16(a.dtype)) return launch_d<float, float>(a, w, st);
+    return out_f32(a.dtype) ? launch_d<__nv_bfloat16, float>(a, w, st)
+                            : launch_d<__nv_bfloat16, __nv_bfloat16>(a, w, st);
 }
 
 }  // namespace gdr

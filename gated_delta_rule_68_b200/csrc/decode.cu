@@ -24,7 +24,7 @@ template <int CL> struct Vec;
 template <> struct Vec<4> { using T = float4; };
 template <> struct Vec<2> { using T = float2; };
 
-template <typename TIn, int DK, int DV, int GATE>
+template <typename TIn, typename TOut, int DK, int DV, int GATE>
 __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
 {
     constexpr int NW = 8, RW = DK / NW, CL = DV / 32;
@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
         for (int ww = 0; ww < NW; ++ww) { kS += red_k[ww][tid]; qS += red_q[ww][tid]; }
         const float u = beta * (vs[tid] - kS);
         us[tid] = u;
-        In<TIn>::store((TIn *)a.o + bh * DV + tid, qS + qk_s * u);
+        In<TOut>::store((TOut *)a.o + bh * DV + tid, qS + qk_s * u);
     }
     __syncthreads();
     float u[CL];
@@ -109,27 +109,29 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
     }
 }
 
-template <typename TIn, int DK, int DV>
+template <typename TIn, typename TOut, int DK, int DV>
 static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t st)
 {
     dim3 grid((unsigned)((long)a.B * a.Hv));
-    if (a.gate_mode == 0) decode_kernel<TIn, DK, DV, 0><<<grid, 256, 0, st>>>(a);
-    else decode_kernel<TIn, DK, DV, 1><<<grid, 256, 0, st>>>(a);
+    if (a.gate_mode == 0) decode_kernel<TIn, TOut, DK, DV, 0><<<grid, 256, 0, st>>>(a);
+    else decode_kernel<TIn, TOut, DK, DV, 1><<<grid, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 
-template <typename TIn>
+template <typename TIn, typename TOut>
 static cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t st)
 {
-    if (a.Dk == 128 && a.Dv == 128) return launch_decode_t<TIn, 128, 128>(a, st);
-    if (a.Dk == 128 && a.Dv == 64) return launch_decode_t<TIn, 128, 64>(a, st);
-    if (a.Dk == 64 && a.Dv == 128) return launch_decode_t<TIn, 64, 128>(a, st);
-    return launch_decode_t<TIn, 64, 64>(a, st);
+    if (a.Dk == 128 && a.Dv == 128) return launch_decode_t<TIn, TOut, 128, 128>(a, st);
+    if (a.Dk == 128 && a.Dv == 64) return launch_decode_t<TIn, TOut, 128, 64>(a, st);
+    if (a.Dk == 64 && a.Dv == 128) return launch_decode_t<TIn, TOut, 64, 128>(a, st);
+    return launch_decode_t<TIn, TOut, 64, 64>(a, st);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st)
 {
-    return a.dtype == 0 ? launch_decode_d<__nv_bfloat16>(a, st) : launch_decode_d<float>(a, st);
+    if (!in_bf16(a.dtype)) return launch_decode_d<float, float>(a, st);
+    return out_f32(a.dtype) ? launch_decode_d<__nv_bfloat16, float>(a, st)
+                            : launch_decode_d<__nv_bfloat16, __nv_bfloat16>(a, st);
 }
 
 }  // namespace gdr

@@ -36,8 +36,9 @@ int check_common(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, in
         return fail(GDR_ERR_INVALID_ARG, "Hv (%d) must be a multiple of Hk (%d)", Hv, Hk);
     if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL)
         return fail(GDR_ERR_INVALID_ARG, "gate_mode must be GDR_GATE_SCALAR or GDR_GATE_CHANNEL (got %d)", gate_mode);
-    if (dtype != GDR_BF16 && dtype != GDR_FP32)
-        return fail(GDR_ERR_INVALID_ARG, "dtype must be GDR_BF16 or GDR_FP32 (got %d)", dtype);
+    if (dtype != GDR_BF16 && dtype != GDR_FP32 && dtype != GDR_BF16_OUT_F32)
+        return fail(GDR_ERR_INVALID_ARG, "dtype must be GDR_BF16, GDR_FP32 or GDR_BF16_OUT_F32 (got %d)",
+                    dtype);
     if (!supported_dim(Dk) || !supported_dim(Dv))
         return fail(GDR_ERR_UNSUPPORTED, "Dk and Dv must each be 64 or 128 (got Dk=%d Dv=%d)", Dk, Dv);
     if ((long long)B * Hv > (1LL << 31) - 1)
@@ -126,10 +127,16 @@ int gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
     if (B == 0) return GDR_OK;
     if (!q || !k || !v || !g || !beta || !state || !o)
         return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, state and o must be non-NULL");
-    const void *ptrs[] = {q, k, v, g, beta, state, o};
-    const char *names[] = {"q", "k", "v", "g", "beta", "state", "o"};
-    for (int i = 0; i < 7; ++i)
-        if (!aligned16(ptrs[i])) return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    // The state is streamed with 128-bit accesses; every other operand is read or
+    // written one element at a time and needs only its element's alignment.
+    if (!aligned16(state)) return fail(GDR_ERR_MISALIGNED, "state is not 16-byte aligned");
+    const uintptr_t in_es = dtype == GDR_FP32 ? 4 : 2, out_es = dtype == GDR_BF16 ? 2 : 4;
+    const void *ptrs[] = {q, k, v, g, beta, o};
+    const uintptr_t need[] = {in_es, in_es, in_es, 4, 4, out_es};
+    const char *names[] = {"q", "k", "v", "g", "beta", "o"};
+    for (int i = 0; i < 6; ++i)
+        if ((uintptr_t)ptrs[i] % need[i])
+            return fail(GDR_ERR_MISALIGNED, "%s is not aligned to its element size", names[i]);
     gdr::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.o = o;
     a.B = B; a.Hk = Hk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.gate_mode = gate_mode; a.dtype = dtype;

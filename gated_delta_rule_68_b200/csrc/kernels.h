@@ -5,6 +5,10 @@
 
 namespace gdr {
 
+// dtype codes (include/gdr.h): 0 bf16 in/out, 1 fp32 in/out, 2 bf16 in / fp32 out.
+inline bool in_bf16(int dtype) { return dtype != 1; }
+inline bool out_f32(int dtype) { return dtype != 0; }
+
 struct DecodeArgs {
     const void *q, *k, *v;
     const float *g, *beta;

@@ -19,7 +19,8 @@
  *
  * Layouts (all row-major and contiguous; "bf16 or fp32" follows `dtype`):
  *   q, k      [B, T, Hk, Dk]   bf16 or fp32
- *   v, o      [B, T, Hv, Dv]   bf16 or fp32
+ *   v         [B, T, Hv, Dv]   bf16 or fp32
+ *   o         [B, T, Hv, Dv]   bf16 or fp32 (fp32 for GDR_BF16_OUT_F32)
  *   g         [B, T, Hv]       fp32 (GDR_GATE_SCALAR)
  *             [B, T, Hv, Dk]   fp32 (GDR_GATE_CHANNEL)
  *   beta      [B, T, Hv]       fp32
@@ -32,7 +33,9 @@
  * Ownership and execution: every pointer is device memory owned by the
  * caller. The library never allocates, frees or synchronises; all work is
  * enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy default
- * stream) and GDR_OK means "enqueued". Pointers must be 16-byte aligned.
+ * stream) and GDR_OK means "enqueued". gdr_fwd_chunked needs every pointer
+ * 16-byte aligned; gdr_decode_step needs the state 16-byte aligned and the
+ * other pointers aligned to their element size.
  * h0 and hT may be the same buffer (in-place state update); o must not alias
  * any input. No C++ exception crosses this boundary.
  *
@@ -66,7 +69,12 @@ typedef enum {
 } gdr_status;
 
 enum { GDR_GATE_SCALAR = 0, GDR_GATE_CHANNEL = 1 };
-enum { GDR_BF16 = 0, GDR_FP32 = 1 };
+/* dtype of q, k, v and o: */
+enum {
+    GDR_BF16 = 0,          /* q, k, v, o bf16 */
+    GDR_FP32 = 1,          /* q, k, v, o fp32 */
+    GDR_BF16_OUT_F32 = 2   /* q, k, v bf16; o fp32 */
+};
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 GDR_API int gdr_version(void);

@@ -110,6 +110,8 @@ def test_workspace_size_rules(L):
     (dict(Dk=32), gdr.GDR_ERR_UNSUPPORTED),
     (dict(state=0), gdr.GDR_ERR_INVALID_ARG),
     (dict(state=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(g=A + 2), gdr.GDR_ERR_MISALIGNED),
+    (dict(q=A + 1), gdr.GDR_ERR_MISALIGNED),
     (dict(gate=5), gdr.GDR_ERR_INVALID_ARG),
 ])
 def test_decode_rejects(L, kw, status):

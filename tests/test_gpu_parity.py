@@ -13,7 +13,7 @@ import torch
 import gated_delta_rule_68_b200 as gdr
 import oracle
 from gated_delta_rule_68_b200.workloads import WORKLOADS, make_inputs
-from tests.gpu_util import TOL, oracle_units, rel_err, sample_units
+from tests.gpu_util import TOL, oracle_units, rel_err, rel_err_excess, sample_units
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -23,19 +23,22 @@ def run_fwd(inp, **kw):
     return gdr.gdr_fwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], **kw)
 
 
-def full_check(w, tol=None):
+def full_check(w, tol=None, plain=False):
+    """Every element of o and hT against the oracle. The five workloads use the plain
+    metric; smaller cases allow the bf16 rounding of o on top (rel_err_excess)."""
     inp = make_inputs(w, DEV)
     o, hT = run_fwd(inp)
     torch.cuda.synchronize()
     o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
     tol = tol or TOL[w.dtype]
-    eo, es = rel_err(o, o_ref), rel_err(hT, s_ref)
+    eo = rel_err(o, o_ref) if plain else rel_err_excess(o, o_ref, w.dtype)
+    es = rel_err(hT, s_ref)
     assert eo <= tol and es <= tol, (w, eo, es)
     return eo, es
 
 
 def test_tiny_gdn_fp32_workload():
-    full_check(WORKLOADS["tiny_gdn_fp32"])
+    full_check(WORKLOADS["tiny_gdn_fp32"], plain=True)
 
 
 SMALL = []
@@ -64,7 +67,7 @@ def test_no_h0_and_no_hT():
     o, hT = run_fwd(inp, want_hT=False)
     assert hT is None
     o_ref, _ = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None)
-    assert rel_err(o, o_ref) <= TOL["bf16"]
+    assert rel_err_excess(o, o_ref, "bf16") <= TOL["bf16"]
 
 
 def test_empty_sequence_writes_h0_to_hT():
@@ -125,28 +128,36 @@ def test_bad_workspace_raises():
 # ------------------------------------------------------------------ full-size workloads
 @pytest.mark.parametrize("name,n_units", [("gdn_bf16", 6), ("gva_gdn_bf16", 6), ("kda_bf16", 3)])
 def test_full_workload_sampled(name, n_units):
+    """The workload exactly as bench.py launches it (bf16 o), and the same call with an
+    fp32 o. The fp32-o outputs and the final state meet max|d|/rms <= 2e-2 against the
+    oracle on sampled (b, h) units; the bf16 o is bit for bit the round-to-nearest bf16
+    of the fp32 o, so storing o in bf16 is the only difference between the two."""
     w = WORKLOADS[name]
     inp_cpu = make_inputs(w, "cpu")
     inp = {n: (None if t is None else t.to(DEV)) for n, t in inp_cpu.items()}
-    o, hT = run_fwd(inp)
+    o16, hT16 = run_fwd(inp)
+    o32, hT = run_fwd(inp, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16 and torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(hT16, hT)
     units = sample_units(w.B, w.Hv, n_units, seed=w.seed)
     o_ref, s_ref = oracle_units(inp_cpu, units)
     for i, (b, h) in enumerate(units):
-        eo = rel_err(o[b, :, h], o_ref[i])
+        eo = rel_err(o32[b, :, h], o_ref[i])
         es = rel_err(hT[b, h], s_ref[i])
-        assert eo <= TOL["bf16"] and es <= TOL["bf16"], (name, b, h, eo, es)
-    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+        eo16 = rel_err_excess(o16[b, :, h], o_ref[i], "bf16")
+        assert eo <= TOL["bf16"] and es <= TOL["bf16"] and eo16 <= TOL["bf16"], (name, b, h, eo, es, eo16)
+    assert torch.isfinite(o32).all() and torch.isfinite(hT).all()
 
 
 # ------------------------------------------------------------------ decode
-def run_decode(inp, steps=None):
+def run_decode(inp, steps=None, out_dtype=None):
     state = inp["h0"].clone()
     steps = steps or inp["q"].shape[0]
     outs = []
     for s in range(steps):
         outs.append(gdr.gdr_decode_step(inp["q"][s], inp["k"][s], inp["v"][s], inp["g"][s],
-                                        inp["beta"][s], state))
+                                        inp["beta"][s], state, out_dtype=out_dtype))
     return torch.stack(outs), state
 
 
@@ -156,10 +167,14 @@ def test_decode_workload_sampled_rows():
     inp = {n: t.to(DEV) for n, t in inp_cpu.items()}
     o, state = run_decode(inp)
     torch.cuda.synchronize()
+    o32, state32 = run_decode(inp, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o32.to(torch.bfloat16)) and torch.equal(state, state32)
     rows = [0, 137, w.B - 1]
     sub = {n: (t[:, rows] if n != "h0" else t[rows]) for n, t in inp_cpu.items()}
     o_ref, s_ref = oracle.decode_steps(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["h0"])
-    assert rel_err(o[:, rows], o_ref) <= TOL["bf16"]
+    assert rel_err(o32[:, rows], o_ref) <= TOL["bf16"]
+    assert rel_err_excess(o[:, rows], o_ref, "bf16") <= TOL["bf16"]
     assert rel_err(state[rows], s_ref) <= TOL["bf16"]
 
 
@@ -174,7 +189,7 @@ def test_decode_small(dtype, gate, D):
     torch.cuda.synchronize()
     o_ref, s_ref = oracle.decode_steps(inp_cpu["q"], inp_cpu["k"], inp_cpu["v"], inp_cpu["g"],
                                        inp_cpu["beta"], inp_cpu["h0"])
-    assert rel_err(o, o_ref) <= TOL[dtype] and rel_err(state, s_ref) <= TOL[dtype]
+    assert rel_err_excess(o, o_ref, dtype) <= TOL[dtype] and rel_err(state, s_ref) <= TOL[dtype]
 
 
 def test_decode_equals_chunked_forward():
