@@ -24,7 +24,10 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
-           "gdr_fwd_chunked", "gdr_decode_step")
+           "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc")
+
+# Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
+GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -56,6 +59,8 @@ def lib():
         L.gdr_fwd_chunked.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp] + [i] * 8 + [vp, sz, vp]
         L.gdr_decode_step.restype = i
         L.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [i] * 7 + [vp]
+        L.gdr_fwd_chunked_noalloc.restype = i
+        L.gdr_fwd_chunked_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp] + [i] * 8 + [vp]
         _lib = L
     return _lib
 
@@ -167,3 +172,34 @@ def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None, out_dtype=N
     _check(lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o),
                                  B, Hk, Hv, Dk, Dv, gate_mode, dt, _stream(stream)))
     return o
+
+
+def gdr_fwd_chunked_noalloc(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True, stream=None,
+                            out_dtype=None):
+    """Chunked forward on the library's own fixed scratch (no workspace, no allocation by the
+    library). For callers that must not allocate device memory; see include/gdr.h. Outputs o
+    and hT are allocated here by torch only when the caller does not pass them."""
+    B, T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt, odt = _dtype_code(q, out_dtype)
+    gate_mode = GDR_GATE_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    _need(q, "q", q.dtype)
+    _need(k, "k", q.dtype, q.shape)
+    _need(v, "v", q.dtype, (B, T, Hv, Dv))
+    _need(g, "g", torch.float32, (B, T, Hv) if gate_mode == 0 else (B, T, Hv, Dk))
+    _need(beta, "beta", torch.float32, (B, T, Hv))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (B, Hv, Dk, Dv))
+    if o is None:
+        o = torch.empty((B, T, Hv, Dv), dtype=odt, device=q.device)
+    _need(o, "o", odt, (B, T, Hv, Dv))
+    if hT is None and want_hT:
+        hT = torch.empty((B, Hv, Dk, Dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _need(hT, "hT", torch.float32, (B, Hv, Dk, Dv))
+    _check(lib().gdr_fwd_chunked_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                         _ptr(o), _ptr(hT), B, T, Hk, Hv, Dk, Dv, gate_mode, dt,
+                                         _stream(stream)))
+    return o, hT

@@ -59,6 +59,11 @@ gdr::FwdArgs make_fwd(const void *q, const void *k, const void *v, const float *
 
 }  // namespace
 
+namespace gdr {
+// Records a failure message for gdr_last_error() from another translation unit.
+int set_failure(int status, const char *msg) { return fail(status, "%s", msg); }
+}  // namespace gdr
+
 extern "C" {
 
 int gdr_version(void) { return 100; }

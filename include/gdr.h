@@ -135,6 +135,35 @@ GDR_API int gdr_decode_step(const void *q, const void *k, const void *v, const f
                     int B, int Hk, int Hv, int Dk, int Dv,
                     int gate_mode, int dtype, void *stream);
 
+/*
+ * Chunked forward for callers that cannot allocate device memory. The source
+ * pages have no counterpart to this entry point; it exists for users of the
+ * library, not for the method.
+ *
+ * Who needs it: code that may not call cudaMalloc - an engine that owns all
+ * device memory through its own pool and forbids side allocations, or a
+ * latency-bound serving loop where allocating (and the device
+ * synchronisation cudaMalloc/cudaFree can trigger) is not allowed after
+ * start-up. Such a caller cannot provide gdr_fwd_chunked's workspace.
+ *
+ * Same arguments and results as gdr_fwd_chunked without the workspace. The
+ * scratch is a fixed array of GDR_NOALLOC_SCRATCH_BYTES in the library's own
+ * device memory; sizes whose gdr_fwd_workspace_size() exceeds it are
+ * rejected with GDR_ERR_WORKSPACE before anything runs. The array is reserved
+ * on every GPU where the library's no-allocation code is loaded and stays
+ * reserved until the process exits. The first call on a device looks up the
+ * array's address on that device: make that first call before any stream
+ * capture. Every call shares the one array and it keeps the previous call's
+ * contents (each call writes every part it reads before reading it), so
+ * calls that overlap in time on one GPU race and must be serialised by the
+ * caller. Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define GDR_NOALLOC_SCRATCH_BYTES (64u << 20)
+GDR_API int gdr_fwd_chunked_noalloc(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *h0, void *o, float *hT,
+                                    int B, int T, int Hk, int Hv, int Dk, int Dv,
+                                    int gate_mode, int dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
