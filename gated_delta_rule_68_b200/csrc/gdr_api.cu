@@ -78,7 +78,7 @@ size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int 
     if (B == 0 || T == 0) return 0;
     const gdr::FwdArgs a = make_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                     nullptr, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
-    return gdr::simt_workspace_size(a);
+    return gdr::fused_supported(a) ? 0 : gdr::simt_workspace_size(a);
 }
 
 int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g, const float *beta,
@@ -113,6 +113,12 @@ int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
     }
 
     const gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (gdr::fused_supported(a)) {
+        cudaError_t e = gdr::launch_fwd_fused(a, s);
+        if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+        g_launches += 1;
+        return GDR_OK;
+    }
     const size_t need = gdr::simt_workspace_size(a);
     if (need > 0 && (!workspace || workspace_bytes < need))
         return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, workspace_bytes,

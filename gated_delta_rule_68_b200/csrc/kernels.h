@@ -27,6 +27,11 @@ struct FwdArgs {
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 
+// Fused chunked forward on the warp-level tensor cores (scalar gate, bf16 inputs,
+// Dk = Dv = 128): one kernel, no workspace.
+bool fused_supported(const FwdArgs &a);
+cudaError_t launch_fwd_fused(const FwdArgs &a, cudaStream_t st);
+
 // fp32 CUDA-core chunked forward (three kernels). Needs simt_workspace_size() bytes.
 size_t simt_workspace_size(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a, void *ws, cudaStream_t st);

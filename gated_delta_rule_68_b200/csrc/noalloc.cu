@@ -5,9 +5,10 @@
 // device memory through its own pool and forbids side allocations, or a
 // latency-bound serving loop where an allocation (and the synchronisation
 // cudaMalloc/cudaFree can cause) is not allowed after start-up. For them this
-// entry point runs the CUDA-core chunked forward on GDR_NOALLOC_SCRATCH_BYTES
-// of scratch reserved in a file-scope __device__ array. The caller still
-// passes every input and output.
+// entry point runs the chunked forward with its workspace placed in
+// GDR_NOALLOC_SCRATCH_BYTES of scratch reserved in a file-scope __device__
+// array; sizes served by the fused single-kernel path need no workspace and
+// leave the array untouched. The caller still passes every input and output.
 //
 // The array is allocated by the CUDA runtime when this file's device code is
 // loaded on a GPU and stays reserved on every GPU that loaded it until the

@@ -80,12 +80,13 @@ def test_fwd_rejects(L, kw, status):
 
 
 def test_fwd_rejects_small_workspace(L):
-    need = L.gdr_fwd_workspace_size(2, 200, 1, 2, 128, 128, 0, 0)
+    need = L.gdr_fwd_workspace_size(2, 200, 1, 2, 128, 128, 0, gdr.GDR_FP32)
     assert need > 0
     st = fwd(L, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480, B=2, T=200, Hv=2,
-             ws=A + 1 << 24, ws_bytes=need - 1)
+             dtype=gdr.GDR_FP32, ws=A + 1 << 24, ws_bytes=need - 1)
     assert st == gdr.GDR_ERR_WORKSPACE
-    st = fwd(L, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480, B=2, T=200, Hv=2)
+    st = fwd(L, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480, B=2, T=200, Hv=2,
+             dtype=gdr.GDR_FP32)
     assert st == gdr.GDR_ERR_WORKSPACE
 
 
@@ -97,7 +98,8 @@ def test_empty_inputs_are_a_no_op(L):
 
 
 def test_workspace_size_rules(L):
-    assert L.gdr_fwd_workspace_size(1, 64, 1, 3, 128, 128, 0, 0) == 0 or True
+    assert L.gdr_fwd_workspace_size(1, 64, 1, 3, 128, 128, 0, gdr.GDR_BF16) == 0   # tensor-core path
+    assert L.gdr_fwd_workspace_size(1, 64, 1, 3, 64, 64, 0, gdr.GDR_BF16) > 0      # CUDA-core path
     assert L.gdr_fwd_workspace_size(1, 64, 2, 3, 128, 128, 0, 0) == 0    # invalid -> 0
     assert L.gdr_fwd_workspace_size(0, 64, 1, 1, 128, 128, 0, 0) == 0    # empty -> 0
     a = L.gdr_fwd_workspace_size(1, 64, 1, 1, 128, 128, 0, 1)
