@@ -49,11 +49,18 @@ constexpr int SZ_C = C * LDC * 2;               // one [64][64] fp16 tile
 constexpr int OFF_M = OFF_S + D * LDD * 2;      // M [r][i]
 constexpr int OFF_TB = OFF_M + SZ_C;            // T diag(beta) [r][i]
 constexpr int OFF_TG = OFF_TB + SZ_C;           // T diag(beta Gamma) [r][i]
-constexpr int OFF_A = OFF_TG + SZ_C;            // fp32 A [64][65]
-constexpr int OFF_T = OFF_A + C * LDF * 4;      // fp32 T [64][65]
-constexpr int OFF_X = OFF_T + C * LDF * 4;      // fp32 [16][48]
-constexpr int OFF_VEC = OFF_X + 16 * 48 * 4;    // G, exp(G), exp(G_C - G), beta: 64 fp32 each
+constexpr int OFF_STG = OFF_TG + SZ_C;          // next chunk's K, Q, V as loaded (bf16 [3][64][128])
+constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32 [2][64])
+constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta: 64 fp32 each
 constexpr int SMEM_BYTES = OFF_VEC + 4 * 64 * 4;
+// The fp32 scratch of the inverse reuses tiles that are dead while it is live:
+// A and T sit in the U' / diag(e) U' tiles, the block-row buffer in the -W tile.
+constexpr int OFF_A = OFF_U;                    // fp32 A [64][65]
+constexpr int OFF_T = OFF_A + C * LDF * 4;      // fp32 T [64][65]
+constexpr int OFF_X = OFF_W;                    // fp32 [16][48]
+static_assert(OFF_T + C * LDF * 4 <= OFF_S, "A and T must fit in the U' tiles");
+static_assert(16 * 48 * 4 <= SZ_D, "block-row buffer must fit in the W tile");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -100,6 +107,18 @@ __device__ __forceinline__ uint32_t b_kn(uint32_t base, int ld, int n0, int k0, 
 {
     return base + ((k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * ld + n0 + (lane >> 4) * 8) * 2;
 }
+
+// Asynchronous global -> shared copies; bytes past src_bytes are filled with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void st_h2(__half *p, float x, float y)
 {
@@ -149,6 +168,9 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
     const uint32_t aTB = smem_u32(sTB), aTG = smem_u32(sTG);
+    const uint4 *sStg = reinterpret_cast<const uint4 *>(sm + OFF_STG);
+    const float *sGst = reinterpret_cast<const float *>(sm + OFF_GST);   // [64] g, then [64] beta
+    const uint32_t aStg = smem_u32(sm + OFF_STG), aGst = smem_u32(sm + OFF_GST);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     const int bh = blockIdx.x;
@@ -179,15 +201,39 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
         }
     }
 
+    // Chunk c's K, Q, V rows, g and beta -> staging buffers, asynchronously (rows past
+    // the end of the sequence are zero-filled).
+    auto issue_loads = [&](int c) {
+        const int t0 = c * C, n = min(C, T - t0);
+#pragma unroll 4
+        for (int idx = tid; idx < 3 * C * 16; idx += NT) {
+            const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
+            const uint4 *src = which == 0 ? kg : (which == 1 ? qg : vg);
+            if (r < n) {
+                const long row = which == 2 ? (((long)b * T + t0 + r) * a.Hv + h) : (((long)b * T + t0 + r) * a.Hk + hk);
+                src += ((row * D) >> 3) + c16;
+            }
+            cp_async16(aStg + idx * 16, src, r < n ? 16u : 0u);
+        }
+        if (tid < 2 * C) {
+            const int r = tid & (C - 1);
+            const float *src = tid < C ? a.g : a.beta;
+            if (r < n) src += ((long)b * T + t0 + r) * a.Hv + h;
+            cp_async4(aGst + tid * 4, src, r < n ? 4u : 0u);
+        }
+        cp_async_commit();
+    };
+    if (NC > 0) issue_loads(0);
+
 #pragma unroll 1
     for (int ch = 0; ch < NC; ++ch) {
         const int t0 = ch * C, n = min(C, T - t0);
+        cp_async_wait_all();
+        __syncthreads();
 
         // ---------------- gate prefix G, exp(G), exp(G_C - G) (warp 0); beta (warps 2, 3)
         if (w == 0) {
-            const long base = ((long)b * T + t0) * a.Hv + h;
-            const float x0 = (2 * lane < n) ? a.g[base + (long)(2 * lane) * a.Hv] : 0.f;
-            const float x1 = (2 * lane + 1 < n) ? a.g[base + (long)(2 * lane + 1) * a.Hv] : 0.f;
+            const float x0 = sGst[2 * lane], x1 = sGst[2 * lane + 1];
             float s = x0 + x1;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -203,25 +249,18 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
             sEt[2 * lane] = expf(gc - e0);
             sEt[2 * lane + 1] = expf(gc - e1);
         } else if (w == 2 || w == 3) {
-            const int r = tid - 64;
-            sBeta[r] = r < n ? a.beta[((long)b * T + t0 + r) * a.Hv + h] : 0.f;
+            sBeta[tid - 64] = sGst[C + tid - 64];
         }
 
-        // ---------------- K, Q, V chunk tiles -> fp16 (rows past the end of the sequence are zero)
+        // ---------------- staged bf16 K, Q, V -> fp16 tiles
 #pragma unroll 4
         for (int idx = tid; idx < 3 * C * 16; idx += NT) {
             const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
-            uint4 u = make_uint4(0, 0, 0, 0);
-            if (r < n) {
-                if (which == 2)
-                    u = __ldg(vg + ((((long)b * T + t0 + r) * a.Hv + h) * D >> 3) + c16);
-                else
-                    u = __ldg((which ? qg : kg) + ((((long)b * T + t0 + r) * a.Hk + hk) * D >> 3) + c16);
-            }
             __half *dst = which == 0 ? sK : (which == 1 ? sQ : sV);
-            *reinterpret_cast<uint4 *>(dst + r * LDD + c16 * 8) = bf16x8_to_f16x8(u);
+            *reinterpret_cast<uint4 *>(dst + r * LDD + c16 * 8) = bf16x8_to_f16x8(sStg[idx]);
         }
         __syncthreads();
+        if (ch + 1 < NC) issue_loads(ch + 1);
 
         // ---------------- Gram [K ; Q] K^T: warps 0-3 rows of K, warps 4-7 rows of Q
         {
