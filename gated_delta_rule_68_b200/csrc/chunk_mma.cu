@@ -53,13 +53,18 @@ constexpr int OFF_STG = OFF_TG + SZ_C;          // next chunk's K, Q, V as loade
 constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32 [2][64])
 constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta: 64 fp32 each
 constexpr int SMEM_BYTES = OFF_VEC + 4 * 64 * 4;
-// The fp32 scratch of the inverse reuses tiles that are dead while it is live:
-// A and T sit in the U' / diag(e) U' tiles, the block-row buffer in the -W tile.
+// The scratch of the inverse reuses tiles that are dead while it is live: fp32
+// A and T sit in the U' / diag(e) U' tiles, their fp16 copies (the tensor-core
+// operands of the block-row products) in the T diag(beta) / T diag(beta Gamma)
+// tiles, and each warp's 16 x 16 block-row product in the -W tile.
 constexpr int OFF_A = OFF_U;                    // fp32 A [64][65]
 constexpr int OFF_T = OFF_A + C * LDF * 4;      // fp32 T [64][65]
-constexpr int OFF_X = OFF_W;                    // fp32 [16][48]
+constexpr int OFF_AH = OFF_TB;                  // fp16 A [64][72]
+constexpr int OFF_TH = OFF_TG;                  // fp16 T [64][72]
+constexpr int LDX = 24;                         // fp16 row stride of a warp's 16 x 16 product
+constexpr int OFF_X = OFF_W;                    // fp16 [8 warps][16][24]
 static_assert(OFF_T + C * LDF * 4 <= OFF_S, "A and T must fit in the U' tiles");
-static_assert(16 * 48 * 4 <= SZ_D, "block-row buffer must fit in the W tile");
+static_assert(8 * 16 * LDX * 2 <= SZ_D, "block-row products must fit in the W tile");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -160,19 +165,21 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
     __half *sTB = reinterpret_cast<__half *>(sm + OFF_TB), *sTG = reinterpret_cast<__half *>(sm + OFF_TG);
     float *sA = reinterpret_cast<float *>(sm + OFF_A);
     float *sT = reinterpret_cast<float *>(sm + OFF_T);
-    float *sX = reinterpret_cast<float *>(sm + OFF_X);
+    __half *sAh = reinterpret_cast<__half *>(sm + OFF_AH), *sTh = reinterpret_cast<__half *>(sm + OFF_TH);
     float *sG = reinterpret_cast<float *>(sm + OFF_VEC);  // [64] G_r
     float *sEg = sG + 64;                                  // [64] exp(G_r)
     float *sEt = sG + 128;                                 // [64] exp(G_C - G_r)
     float *sBeta = sG + 192;                               // [64]
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
-    const uint32_t aTB = smem_u32(sTB), aTG = smem_u32(sTG);
+    const uint32_t aTB = smem_u32(sTB), aTG = smem_u32(sTG), aAh = smem_u32(sAh), aTh = smem_u32(sTh);
     const uint4 *sStg = reinterpret_cast<const uint4 *>(sm + OFF_STG);
     const float *sGst = reinterpret_cast<const float *>(sm + OFF_GST);   // [64] g, then [64] beta
     const uint32_t aStg = smem_u32(sm + OFF_STG), aGst = smem_u32(sm + OFF_GST);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+    __half *sXw = reinterpret_cast<__half *>(sm + OFF_X) + w * 16 * LDX;   // this warp's 16 x 16 tile
+    const uint32_t aXw = smem_u32(sXw);
     const int bh = blockIdx.x;
     const int b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, NC = (T + C - 1) / C;
@@ -290,8 +297,11 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
                     const int i = 8 * j + 2 * t4;
                     const float d0 = acc[j][2 * hh], d1 = acc[j][2 * hh + 1];
                     if (w < 4) {
-                        sA[r * LDF + i] = i < r ? br * expf(gr - sG[i]) * d0 : 0.f;
-                        sA[r * LDF + i + 1] = i + 1 < r ? br * expf(gr - sG[i + 1]) * d1 : 0.f;
+                        const float x0 = i < r ? br * expf(gr - sG[i]) * d0 : 0.f;
+                        const float x1 = i + 1 < r ? br * expf(gr - sG[i + 1]) * d1 : 0.f;
+                        sA[r * LDF + i] = x0;
+                        sA[r * LDF + i + 1] = x1;
+                        st_h2(sAh + r * LDC + i, x0, x1);
                     } else {
                         st_h2(sM + r * LDC + i, i <= r ? expf(gr - sG[i]) * d0 : 0.f,
                               i + 1 <= r ? expf(gr - sG[i + 1]) * d1 : 0.f);
@@ -299,12 +309,13 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
                 }
             }
         }
-        for (int idx = tid; idx < C * LDF; idx += NT) sT[idx] = 0.f;
         __syncthreads();
 
-        // ---------------- T = (I + A)^-1: 16x16 diagonal blocks by forward
-        // substitution, then block rows bi = 1..3:
-        //   T_{bi,bj} = -T_{bi,bi} sum_{m=bj}^{bi-1} A_{bi,m} T_{m,bj}
+        // ---------------- T = (I + A)^-1 (entries above the diagonal are never
+        // written and read as zero). The 16x16 diagonal blocks by forward
+        // substitution in fp32; then block rows bi = 1..3 on tensor cores, one
+        // warp per block (bi, bj):
+        //   X = sum_{m=bj}^{bi-1} A_{bi,m} T_{m,bj},   T_{bi,bj} = -T_{bi,bi} X
         if (tid < 64) {
             const int base = (tid >> 4) * 16, col = tid & 15;
             float tv[16];
@@ -316,31 +327,56 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
                 tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -s);
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sT[(base + r) * LDF + base + col] = tv[r];
+            for (int r = 0; r < 16; ++r) {
+                sT[(base + r) * LDF + base + col] = tv[r];
+                sTh[(base + r) * LDC + base + col] = __float2half_rn(tv[r]);
+            }
         }
         __syncthreads();
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {
-            for (int e = tid; e < bi * 256; e += NT) {
-                const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                float s = 0.f;
-                for (int x = 16 * bj; x < 16 * bi; ++x) s += sA[(16 * bi + r) * LDF + x] * sT[x * LDF + 16 * bj + c];
-                sX[r * 48 + bj * 16 + c] = s;
-            }
-            __syncthreads();
-            for (int e = tid; e < bi * 256; e += NT) {
-                const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                float s = 0.f;
+            if (w < bi) {
+                const int bj = w;
+                float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int m = bj; m < bi; ++m) {
+                    uint32_t af[4], bf[4];
+                    ldsm(af, a_rm(aAh, LDC, 16 * bi, 16 * m, lane));
+                    ldsm_t(bf, b_kn(aTh, LDC, 16 * bj, 16 * m, lane));
+                    mma(x[0], af, bf[0], bf[1]);
+                    mma(x[1], af, bf[2], bf[3]);
+                }
 #pragma unroll
-                for (int x = 0; x < 16; ++x) s += sT[(16 * bi + r) * LDF + 16 * bi + x] * sX[x * 48 + bj * 16 + c];
-                sT[(16 * bi + r) * LDF + 16 * bj + c] = -s;
+                for (int j = 0; j < 2; ++j) {
+                    st_h2(sXw + g * LDX + 8 * j + 2 * t4, x[j][0], x[j][1]);
+                    st_h2(sXw + (g + 8) * LDX + 8 * j + 2 * t4, x[j][2], x[j][3]);
+                }
+                __syncwarp();
+                float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                {
+                    uint32_t af[4], bf[4];
+                    ldsm(af, a_rm(aTh, LDC, 16 * bi, 16 * bi, lane));
+                    ldsm_t(bf, b_kn(aXw, LDX, 0, 0, lane));
+                    mma(y[0], af, bf[0], bf[1]);
+                    mma(y[1], af, bf[2], bf[3]);
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r0 = 16 * bi + g, c = 16 * bj + 8 * j + 2 * t4;
+                    sT[r0 * LDF + c] = -y[j][0];
+                    sT[r0 * LDF + c + 1] = -y[j][1];
+                    sT[(r0 + 8) * LDF + c] = -y[j][2];
+                    sT[(r0 + 8) * LDF + c + 1] = -y[j][3];
+                    st_h2(sTh + r0 * LDC + c, -y[j][0], -y[j][1]);
+                    st_h2(sTh + (r0 + 8) * LDC + c, -y[j][2], -y[j][3]);
+                }
             }
             __syncthreads();
         }
         // T diag(beta) and T diag(beta Gamma) -> fp16 [r][i]
         for (int idx = tid; idx < C * (C / 2); idx += NT) {
             const int r = idx >> 5, i = (idx & 31) * 2;
-            const float t0v = sT[r * LDF + i] * sBeta[i], t1v = sT[r * LDF + i + 1] * sBeta[i + 1];
+            const float t0v = i <= r ? sT[r * LDF + i] * sBeta[i] : 0.f;
+            const float t1v = i + 1 <= r ? sT[r * LDF + i + 1] * sBeta[i + 1] : 0.f;
             st_h2(sTB + r * LDC + i, t0v, t1v);
             st_h2(sTG + r * LDC + i, t0v * sEg[i], t1v * sEg[i + 1]);
         }
