@@ -54,17 +54,17 @@ constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32
 constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta: 64 fp32 each
 constexpr int SMEM_BYTES = OFF_VEC + 4 * 64 * 4;
 // The scratch of the inverse reuses tiles that are dead while it is live: fp32
-// A and T sit in the U' / diag(e) U' tiles, their fp16 copies (the tensor-core
-// operands of the block-row products) in the T diag(beta) / T diag(beta Gamma)
-// tiles, and each warp's 16 x 16 block-row product in the -W tile.
+// A sits in the U' tile, the fp16 inverse T in the diag(e) U' tile, and the
+// fp16 copy of A (an operand of the block-row products) after each warp's
+// 16 x 16 block-row product in the -W tile.
 constexpr int OFF_A = OFF_U;                    // fp32 A [64][65]
-constexpr int OFF_T = OFF_A + C * LDF * 4;      // fp32 T [64][65]
-constexpr int OFF_AH = OFF_TB;                  // fp16 A [64][72]
-constexpr int OFF_TH = OFF_TG;                  // fp16 T [64][72]
+constexpr int OFF_TH = OFF_UE;                  // fp16 T [64][72]
 constexpr int LDX = 24;                         // fp16 row stride of a warp's 16 x 16 product
 constexpr int OFF_X = OFF_W;                    // fp16 [8 warps][16][24]
-static_assert(OFF_T + C * LDF * 4 <= OFF_S, "A and T must fit in the U' tiles");
-static_assert(8 * 16 * LDX * 2 <= SZ_D, "block-row products must fit in the W tile");
+constexpr int OFF_AH = OFF_X + 8 * 16 * LDX * 2;// fp16 A [64][72]
+static_assert(C * LDF * 4 <= SZ_D, "A must fit in the U' tile");
+static_assert(C * LDC * 2 <= SZ_D, "T must fit in the diag(e) U' tile");
+static_assert(8 * 16 * LDX * 2 + C * LDC * 2 <= SZ_D, "block-row products and A must fit in the W tile");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -164,7 +164,6 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
     __half *sS = reinterpret_cast<__half *>(sm + OFF_S), *sM = reinterpret_cast<__half *>(sm + OFF_M);
     __half *sTB = reinterpret_cast<__half *>(sm + OFF_TB), *sTG = reinterpret_cast<__half *>(sm + OFF_TG);
     float *sA = reinterpret_cast<float *>(sm + OFF_A);
-    float *sT = reinterpret_cast<float *>(sm + OFF_T);
     __half *sAh = reinterpret_cast<__half *>(sm + OFF_AH), *sTh = reinterpret_cast<__half *>(sm + OFF_TH);
     float *sG = reinterpret_cast<float *>(sm + OFF_VEC);  // [64] G_r
     float *sEg = sG + 64;                                  // [64] exp(G_r)
@@ -321,16 +320,29 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
             float tv[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float s = 0.f;
+                float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < r; ++i) s += sA[(base + r) * LDF + base + i] * tv[i];
-                tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -s);
+                for (int i = 0; i < r; i += 2) {
+                    s0 += sA[(base + r) * LDF + base + i] * tv[i];
+                    if (i + 1 < r) s1 += sA[(base + r) * LDF + base + i + 1] * tv[i + 1];
+                }
+                tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -(s0 + s1));
             }
+            const float bc = sBeta[base + col], bgc = bc * sEg[base + col];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                sT[(base + r) * LDF + base + col] = tv[r];
-                sTh[(base + r) * LDC + base + col] = __float2half_rn(tv[r]);
+                const int o = (base + r) * LDC + base + col;
+                sTh[o] = __float2half_rn(tv[r]);
+                sTB[o] = __float2half_rn(tv[r] * bc);
+                sTG[o] = __float2half_rn(tv[r] * bgc);
             }
+        } else {
+            // zeros in the six blocks above the diagonal of T diag(beta), T diag(beta Gamma)
+            const int e = tid - 64, blk = e >> 5, row = (e >> 1) & 15, hf = e & 1;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
+            *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
         }
         __syncthreads();
 #pragma unroll 1
@@ -359,28 +371,22 @@ __global__ void __launch_bounds__(NT, 1) fused_fwd_gdn_kernel(FwdArgs a)
                     mma(y[0], af, bf[0], bf[1]);
                     mma(y[1], af, bf[2], bf[3]);
                 }
+                // T_{bi,bj} = -y, and its columns scaled by beta and by beta Gamma
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r0 = 16 * bi + g, c = 16 * bj + 8 * j + 2 * t4;
-                    sT[r0 * LDF + c] = -y[j][0];
-                    sT[r0 * LDF + c + 1] = -y[j][1];
-                    sT[(r0 + 8) * LDF + c] = -y[j][2];
-                    sT[(r0 + 8) * LDF + c + 1] = -y[j][3];
+                    const float b0 = sBeta[c], b1 = sBeta[c + 1];
+                    const float e0 = b0 * sEg[c], e1 = b1 * sEg[c + 1];
                     st_h2(sTh + r0 * LDC + c, -y[j][0], -y[j][1]);
                     st_h2(sTh + (r0 + 8) * LDC + c, -y[j][2], -y[j][3]);
+                    st_h2(sTB + r0 * LDC + c, -y[j][0] * b0, -y[j][1] * b1);
+                    st_h2(sTB + (r0 + 8) * LDC + c, -y[j][2] * b0, -y[j][3] * b1);
+                    st_h2(sTG + r0 * LDC + c, -y[j][0] * e0, -y[j][1] * e1);
+                    st_h2(sTG + (r0 + 8) * LDC + c, -y[j][2] * e0, -y[j][3] * e1);
                 }
             }
             __syncthreads();
         }
-        // T diag(beta) and T diag(beta Gamma) -> fp16 [r][i]
-        for (int idx = tid; idx < C * (C / 2); idx += NT) {
-            const int r = idx >> 5, i = (idx & 31) * 2;
-            const float t0v = i <= r ? sT[r * LDF + i] * sBeta[i] : 0.f;
-            const float t1v = i + 1 <= r ? sT[r * LDF + i + 1] * sBeta[i + 1] : 0.f;
-            st_h2(sTB + r * LDC + i, t0v, t1v);
-            st_h2(sTG + r * LDC + i, t0v * sEg[i], t1v * sEg[i + 1]);
-        }
-        __syncthreads();
 
         // ---------------- W = T diag(beta Gamma) K,  U = T diag(beta) V  (warp tile 16 x 64)
         float accU[8][4];
