@@ -55,7 +55,7 @@ def build(force: bool = False, extra=(), verbose: bool = False) -> str:
             if log:
                 print(log)
     objs = [o for o, _ in results]
-    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", LIB + ".tmp", *objs, "-lcuda"]
+    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", LIB + ".tmp", *objs]
     subprocess.check_call(cmd)
     os.replace(LIB + ".tmp", LIB)
     return LIB
