@@ -54,8 +54,14 @@ def parse_args(argv=None):
 
 # ----------------------------------------------------------------------------- accounting
 def algorithmic_bytes(w):
-    """HBM bytes the method must move per call: q, k, v, o, g, beta, h0 and hT."""
+    """HBM bytes the method must move per call: q, k, v, o, g, beta, h0 and hT. For the
+    decode workload, per step: the state read and written once, and one token's inputs
+    and output for every (batch row, value head)."""
     es = 2 if w.dtype == "bf16" else 4
+    if w.decode:
+        tok = w.B * (2 * w.Hk * w.Dk * es + 2 * w.Hv * w.Dv * es
+                     + w.Hv * (w.Dk if w.gate == "channel" else 1) * 4 + w.Hv * 4)
+        return 2 * w.B * w.Hv * w.Dk * w.Dv * 4 + tok
     qk = 2 * w.B * w.T * w.Hk * w.Dk * es
     vo = 2 * w.B * w.T * w.Hv * w.Dv * es
     g = w.B * w.T * w.Hv * (w.Dk if w.gate == "channel" else 1) * 4
@@ -96,6 +102,27 @@ def recorded_traffic(workload):
     if d.get("kernel_sources_sha256") != kernel_sources_sha():
         return None, d.get("kernel")
     return float(d["dram_bytes_per_launch"]), d.get("kernel")
+
+
+# ----------------------------------------------------------------------------- ranks
+def rank_workload(w, rank):
+    """Each rank runs the whole workload on its own inputs: the seed is offset by the rank."""
+    return w.with_(seed=w.seed + rank)
+
+
+def max_over_ranks(x, device=None):
+    """The largest of every rank's value (the step time the job is judged by)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(units_per_rank, world, ms_max):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -176,14 +203,17 @@ def cpu_oracle_sample(w, target_s=12.0, seed_rank=0):
     q, k, v, g, beta, h0 = (inp[n] for n in ("q", "k", "v", "g", "beta", "h0"))
     qd, kd, vd, gd, bd = (x.double().numpy() for x in (q, k, v, g, beta))
     hd = None if h0 is None else h0.double().numpy()
-    t0 = time.perf_counter()
-    oracle.recurrent(qd, kd, vd, gd, bd, hd, nthreads=0)
-    dt = time.perf_counter() - t0
+    reps, dt = 0, 0.0
+    while reps == 0 or (dt < target_s and reps < 1000):
+        t0 = time.perf_counter()
+        oracle.recurrent(qd, kd, vd, gd, bd, hd, nthreads=0)
+        dt += time.perf_counter() - t0
+        reps += 1
     return {
-        "value": units * w.T / dt, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+        "value": reps * units * w.T / dt, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
         "kind": "oracle",
         "sample": f"{units} whole (batch row, value head) sequences of T={w.T}, Dk=Dv={w.Dk}, "
-                  f"{w.gate} gate, fp64 token recurrence; {dt:.1f} s",
+                  f"{w.gate} gate, fp64 token recurrence, run {reps} times; {dt:.1f} s",
         "seconds": dt,
     }
 
@@ -233,6 +263,101 @@ def workload_config(w, world):
             "l2": ("inputs exceed L2, no flush" if ab > L2_BYTES else "L2 flushed between steps")}
 
 
+# ----------------------------------------------------------------------------- decode
+def run_decode_bench(args, w, wr, rank, world, local, dev):
+    """One step = one gdr_decode_step over the whole batch: every (batch row, value head)
+    state is read and written once. Each step takes the next pre-generated token."""
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_68_b200 as gdr
+    from gated_delta_rule_68_b200.workloads import make_inputs
+
+    n_tok = args.warmup + args.steps
+    inp_cpu = make_inputs(wr.with_(T=n_tok), "cpu")
+    inp = {n: t.to(dev) for n, t in inp_cpu.items()}
+    state = inp["h0"].clone()
+    o = torch.empty((w.B, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(s):
+        gdr.gdr_decode_step(inp["q"][s], inp["k"][s], inp["v"][s], inp["g"][s], inp["beta"][s], state, o=o,
+                            stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = gdr.gdr_kernel_launches()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for s in range(args.warmup, n_tok):
+            step(s)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    launches = gdr.gdr_kernel_launches() - n0
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+
+    e2e = None
+    if not args.no_e2e:   # one token's inputs up, its outputs down, every step
+        host = {n: inp_cpu[n][0].pin_memory() for n in ("q", "k", "v", "g", "beta")}
+        dbuf = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in host.values())
+        d2h = o_h.numel() * o_h.element_size()
+
+        def e2e_step():
+            for n, x in host.items():
+                dbuf[n].copy_(x, non_blocking=True)
+            gdr.gdr_decode_step(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], state, o=o,
+                                stream=stream)
+            o_h.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+        e2e = {"value": job_tokens_per_s(w.B * w.Hv, world, te), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.steps,
+               "ms_per_step": te}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(w)
+    achieved = alg / (ms / 1e3) / 1e9
+    traffic, traffic_kernel = recorded_traffic(w.name)
+    line = {
+        "metric": "gated-delta decode tokens/s (B·Hv per sec per step) bf16 d=128; % of roofline",
+        "value": job_tokens_per_s(w.B * w.Hv, world, ms_max), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded CPU generator, one fresh token per step; state 0.02 N(0,1))",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
+                     "traffic": traffic, "traffic_kernel": traffic_kernel, "kernel": "gdr_decode_step"},
+        "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches,
+        "launches_per_step": launches / args.steps, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main(argv=None):
     args = parse_args(argv)
@@ -256,7 +381,9 @@ def main(argv=None):
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
-    wr = w.with_(seed=w.seed + rank)
+    wr = rank_workload(w, rank)
+    if w.decode:
+        return run_decode_bench(args, w, wr, rank, world, local, dev)
     inp_cpu = make_inputs(wr, "cpu")
     inp = {n: (None if t is None else t.to(dev)) for n, t in inp_cpu.items()}
     o = torch.empty((w.B, w.T, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)
@@ -296,10 +423,7 @@ def main(argv=None):
     launches = gdr.gdr_kernel_launches() - n0
     barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -331,12 +455,10 @@ def main(argv=None):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * w.head_tokens / (float(te.item()) / 1e3), "unit": "tokens/s",
+        te = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+        e2e = {"value": job_tokens_per_s(w.head_tokens, world, te), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-               "ms_per_step": float(te.item())}
+               "ms_per_step": te}
 
     if world > 1:
         dist.barrier()
@@ -353,7 +475,7 @@ def main(argv=None):
         cpu = cpu_oracle_sample(w)
     line = {
         "metric": METRIC,
-        "value": world * w.head_tokens / (ms_max / 1e3),
+        "value": job_tokens_per_s(w.head_tokens, world, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,

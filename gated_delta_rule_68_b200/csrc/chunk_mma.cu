@@ -229,8 +229,6 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
     const int bh = blockIdx.x;
     const int b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, NC = (T + C - 1) / C;
-    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q), *kg = reinterpret_cast<const uint4 *>(a.k);
-    const uint4 *vg = reinterpret_cast<const uint4 *>(a.v);
 
     // Row block (16 rows) and column half (64 columns) of this warp in the [64 x 128] products.
     const int rw0 = 16 * (w & 3), cw0 = 64 * (w >> 2);
