@@ -24,7 +24,7 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
-           "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc")
+           "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts")
 
 # Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
 GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -75,6 +75,13 @@ def gdr_last_error() -> str:
 
 def gdr_kernel_launches() -> int:
     return int(lib().gdr_kernel_launches())
+
+
+def gdr_fused_error_counts():
+    """(load_timeouts, range_errors) of the fused kernel on the current device; see include/gdr.h."""
+    t, r = ctypes.c_uint(0), ctypes.c_uint(0)
+    lib().gdr_fused_error_counts(ctypes.byref(t), ctypes.byref(r))
+    return int(t.value), int(r.value)
 
 
 def _check(status):

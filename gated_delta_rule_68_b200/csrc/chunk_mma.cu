@@ -1,25 +1,32 @@
-// Fused chunked forward of the gated delta rule with a scalar per-head gate
-// (Gated DeltaNet) on the warp-level tensor cores: mma.sync m16n8k16 with fp16
-// operands and fp32 accumulators, bf16 inputs, Dk = Dv = 128, chunks of C = 64
-// tokens. One CTA (8 warps) per (batch row, value head) walks the whole
-// sequence; the fp32 state lives in the warps' accumulator registers and never
-// leaves the SM until the final state is written.
+// Fused chunked forward of the gated delta rule on the warp-level tensor cores:
+// mma.sync m16n8k16 with fp16 operands and fp32 accumulators, bf16 inputs,
+// Dk = Dv = 128, chunks of C = 64 tokens, for a scalar decay per head (Gated
+// DeltaNet) or one per key channel (Kimi Delta Attention). One CTA (8 warps) per
+// (batch row, value head), or two splitting the value columns when that still
+// fills the SMs in one wave, walks the whole sequence; the fp32 state lives in
+// the warps' accumulator registers and never leaves the SM until the final state
+// is written.
 //
 // Method: the exact chunkwise form of
-//   S_t = (I - beta_t k_t k_t^T) exp(g_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
-// (NextTransformer, "Source notes", "Linear attention", row gdn; SinkProbe
-// (Attention-Sink) README: delta-rule layer in exact chunkwise form). With
-// G_r = sum_{j<=r} g_j inside the chunk, Gamma_r = exp(G_r), Gamma_C = Gamma_63:
-//   A_ri = beta_r exp(G_r - G_i) k_r.k_i  (i < r),   T = (I + A)^-1
-//   W = T diag(beta Gamma) K,   U = T diag(beta) V,   U' = U - W S
-//   O_r = Gamma_r (Q S)_r + (M U')_r,   M_ri = exp(G_r - G_i) q_r.k_i  (i <= r)
-//   S_next = Gamma_C S + K^T diag(e) U',   e_i = exp(G_C - G_i)
-// Every gate factor is folded where it is at most 1, so no operand grows past
-// the size of its inputs. The products run on tensor cores; A, the inverse T
-// and the gate factors are fp32 on CUDA cores. fp16 operands (bf16 inputs
-// convert exactly in fp16's normal range) keep the result within 2e-2 of the
-// fp64 recurrence by max |error| / rms; inputs and states must stay inside the
-// fp16 range (|x| < 6.5e4).
+//   S_t = (I - beta_t k_t k_t^T) diag(exp g_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
+// (NextTransformer, "Source notes", "Linear attention", rows gdn and kda;
+// SinkProbe (Attention-Sink) README: delta-rule layer in exact chunkwise form).
+// With G_r = sum_{j<=r} g_j inside the chunk (per channel for the channel gate),
+// Gamma_r = exp(G_r), Gamma_C = Gamma_63:
+//   A_ri = beta_r sum_c k_rc k_ic exp(G_rc - G_ic)  (i < r),   T = (I + A)^-1
+//   W = T diag(beta) (K o Gamma),   U = T diag(beta) V,   U' = U - W S
+//   O = (Q o Gamma) S + M U',   M_ri = sum_c q_rc k_ic exp(G_rc - G_ic)  (i <= r)
+//   S_next = diag(Gamma_C) S + (K o Gamma_C / Gamma)^T U'
+// Scalar gate: the exp factors are per row and fold into the Gram epilogue, into
+// T diag(beta Gamma) and into row scalings, all at most 1. Channel gate: the
+// Gram's operands carry them, rows of K and Q scaled by exp(G_r - G_31) and rows
+// of K by exp(G_31 - G_i), so each factor spans at most 32 tokens of decay (a
+// factor outside fp16's range is counted, see gdr_fused_error_counts); the other
+// operands carry factors at most 1. The products run on tensor cores; A, the
+// diagonal blocks of the inverse and the gate factors are fp32 on CUDA cores.
+// fp16 operands (bf16 inputs convert exactly in fp16's normal range) keep the
+// result within 2e-2 of the fp64 recurrence by max |error| / rms; inputs and
+// states must stay inside the fp16 range (|x| < 6.5e4).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -52,8 +59,8 @@ constexpr int OFF_TB = OFF_M + SZ_C;            // T diag(beta) [r][i]
 constexpr int OFF_TG = OFF_TB + SZ_C;           // T diag(beta Gamma) [r][i]
 constexpr int OFF_STG = OFF_TG + SZ_C;          // next chunk's K, Q, V as loaded (bf16 [3][64][128])
 constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32 [2][64])
-constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta: 64 fp32 each
-constexpr int SMEM_BYTES = OFF_VEC + 4 * 64 * 4;
+constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta (64 fp32 each); 2 x 128 fp32 sums
+constexpr int SMEM_BYTES = OFF_VEC + 512 * 4;
 // The scratch of the inverse reuses tiles that are dead while it is live: fp32
 // A sits in the U' tile, the fp16 inverse T in the diag(e) U' tile, and the
 // fp16 copy of A (an operand of the block-row products) after each warp's
@@ -194,14 +201,22 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u)
     return r;
 }
 
-// Chunk loads that never completed (each abandons its CTA's remaining chunks).
+// Chunk loads that never completed (each abandons its CTA's remaining chunks), and
+// per-channel gate factors that left the fp16 range (their chunk's results are not valid).
 __device__ unsigned int g_fused_load_timeouts;
+__device__ unsigned int g_fused_range_errors;
 
-template <typename TOut>
+// GATE 0: one decay per (token, head); GATE 1: one per (token, head, key channel).
+// NS: value columns are split over NS CTAs per (b, h), each owning D / NS of them
+// (its part of the state, U, U', O); the Gram, the inverse and W are computed by each.
+template <typename TOut, int GATE, int NS>
 __global__ void __launch_bounds__(NT, 1)
-fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                     const __grid_constant__ CUtensorMap map_v)
+fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                 const __grid_constant__ CUtensorMap map_v)
 {
+    constexpr int DVC = D / NS;      // value columns of this CTA
+    constexpr int NJ = DVC / 16;     // n8 tiles of a warp in the [64 x DVC] products (half the columns)
+    constexpr int NJS = DVC / 8;     // n8 tiles of a warp's state rows
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // 128-byte aligned base: the TMA destination tiles need it.
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -211,35 +226,41 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
     __half *sS = reinterpret_cast<__half *>(sm + OFF_S), *sM = reinterpret_cast<__half *>(sm + OFF_M);
     __half *sTB = reinterpret_cast<__half *>(sm + OFF_TB), *sTG = reinterpret_cast<__half *>(sm + OFF_TG);
     float *sA = reinterpret_cast<float *>(sm + OFF_A);
-    __half *sAh = reinterpret_cast<__half *>(sm + OFF_AH), *sTh = reinterpret_cast<__half *>(sm + OFF_TH);
-    float *sG = reinterpret_cast<float *>(sm + OFF_VEC);  // [64] G_r
-    float *sEg = sG + 64;                                  // [64] exp(G_r)
+    // The per-channel gate needs no T diag(beta Gamma) (Gamma rides on K), and its
+    // diag(e) U' tile holds K diag(Gamma_C / Gamma): T goes to the T diag(beta Gamma) tile.
+    __half *sAh = reinterpret_cast<__half *>(sm + OFF_AH);
+    __half *sTh = reinterpret_cast<__half *>(sm + (GATE ? OFF_TG : OFF_TH));
+    float *sG = reinterpret_cast<float *>(sm + OFF_VEC);  // [64] G_r           | GATE 1: [128] Gamma_C
+    float *sEg = sG + 64;                                  // [64] exp(G_r)      |
     float *sEt = sG + 128;                                 // [64] exp(G_C - G_r)
     float *sBeta = sG + 192;                               // [64]
+    float *sTot = sG + 256;                                // GATE 1: [2][128] per-channel sums of each half chunk
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
     const uint32_t aTB = smem_u32(sTB), aTG = smem_u32(sTG), aAh = smem_u32(sAh), aTh = smem_u32(sTh);
     const uint4 *sStg = reinterpret_cast<const uint4 *>(sm + OFF_STG);
+    const __nv_bfloat16 *sStgH = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_STG);
     const float *sGst = reinterpret_cast<const float *>(sm + OFF_GST);   // [64] g, then [64] beta
     const uint32_t aStg = smem_u32(sm + OFF_STG), aGst = smem_u32(sm + OFF_GST);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     __half *sXw = reinterpret_cast<__half *>(sm + OFF_X) + w * 16 * LDX;   // this warp's 16 x 16 tile
     const uint32_t aXw = smem_u32(sXw);
-    const int bh = blockIdx.x;
+    const int split = blockIdx.x % NS, bh = blockIdx.x / NS, dv0 = split * DVC;
     const int b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, NC = (T + C - 1) / C;
 
-    // Row block (16 rows) and column half (64 columns) of this warp in the [64 x 128] products.
-    const int rw0 = 16 * (w & 3), cw0 = 64 * (w >> 2);
+    // Row block (16 rows) and column half of this warp in the [64 x DVC] products.
+    const int rw0 = 16 * (w & 3), cw0 = (DVC / 2) * (w >> 2);
 
-    // State S [dk][dv] in registers: warp w holds dk rows 16w..16w+15; n8 tile j holds dv 8j..8j+7.
-    float accS[16][4];
+    // State S[:, dv0 .. dv0 + DVC) in registers: warp w holds dk rows 16w..16w+15;
+    // n8 tile j holds local columns 8j..8j+7.
+    float accS[NJS][4];
     {
-        const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D : nullptr;
+        const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + dv0 : nullptr;
         const int r0 = 16 * w + g;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < NJS; ++j) {
             const int c = 8 * j + 2 * t4;
             float2 x0 = make_float2(0.f, 0.f), x1 = x0;
             if (h0) {
@@ -252,11 +273,9 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
         }
     }
 
-    // Chunk c's K, Q, V rows, g and beta -> staging buffers, asynchronously (rows past
-    // the end of the sequence are zero-filled).
-    // Chunk c's K, Q, V tiles -> bf16 staging by three TMA box loads that
-    // complete on ld_bar (rows past the end of the sequence read as zero); g and
-    // beta by 4-byte asynchronous copies.
+    // Chunk c's K, Q tiles and this CTA's V columns -> bf16 staging by three TMA box
+    // loads that complete on ld_bar (tokens past T read as zero); beta, and the
+    // scalar gate, by 4-byte asynchronous copies.
     __shared__ uint64_t ld_bar;
     const uint32_t aBar = smem_u32(&ld_bar);
     if (tid == 0) mbar_init(aBar, 1);
@@ -264,12 +283,12 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
     auto issue_loads = [&](int c) {
         const int t0 = c * C, n = min(C, T - t0);
         if (tid == 0) {
-            mbar_expect_tx(aBar, 3u * C * D * 2);
+            mbar_expect_tx(aBar, (2u * C * D + C * DVC) * 2);
             tma_load_4d(aStg, &map_k, 0, hk, t0, b, aBar);
             tma_load_4d(aStg + C * D * 2, &map_q, 0, hk, t0, b, aBar);
-            tma_load_4d(aStg + 2 * C * D * 2, &map_v, 0, h, t0, b, aBar);
+            tma_load_4d(aStg + 2 * C * D * 2, &map_v, dv0, h, t0, b, aBar);
         }
-        if (tid < 2 * C) {
+        if (tid < 2 * C && (GATE == 0 || tid >= C)) {
             const int r = tid & (C - 1);
             const float *src = tid < C ? a.g : a.beta;
             if (r < n) src += ((long)b * T + t0 + r) * a.Hv + h;
@@ -288,43 +307,89 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
             return;
         }
 
-        // ---------------- gate prefix G, exp(G), exp(G_C - G) (warp 0); beta (warps 2, 3)
-        if (w == 0) {
-            const float x0 = sGst[2 * lane], x1 = sGst[2 * lane + 1];
-            float s = x0 + x1;
+        // ---------------- gates and fp16 operand tiles
+        // GATE 1 keeps each channel's prefix G for 32 rows in registers: thread
+        // (c, hf) owns key channel c = tid % 128 and rows 32 hf .. 32 hf + 31.
+        float Gv[GATE ? 32 : 1];
+        float gm = 0.f, gcs = 0.f;   // GATE 1: G at row 31 and at row 63 of channel c
+        const int ch_c = tid & (D - 1), ch_h = tid >> 7;
+        if (GATE == 0) {
+            if (w == 0) {   // G, exp(G), exp(G_C - G)
+                const float x0 = sGst[2 * lane], x1 = sGst[2 * lane + 1];
+                float s = x0 + x1;
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, s, off);
-                if (lane >= off) s += y;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, off);
+                    if (lane >= off) s += y;
+                }
+                const float e0 = s - x1, e1 = s;
+                const float gc = __shfl_sync(0xffffffffu, s, 31);
+                sG[2 * lane] = e0;
+                sG[2 * lane + 1] = e1;
+                sEg[2 * lane] = __expf(e0);
+                sEg[2 * lane + 1] = __expf(e1);
+                sEt[2 * lane] = __expf(gc - e0);
+                sEt[2 * lane + 1] = __expf(gc - e1);
+            } else if (w == 2 || w == 3) {
+                sBeta[tid - 64] = sGst[C + tid - 64];
             }
-            const float e0 = s - x1, e1 = s;
-            const float gc = __shfl_sync(0xffffffffu, s, 31);
-            sG[2 * lane] = e0;
-            sG[2 * lane + 1] = e1;
-            sEg[2 * lane] = __expf(e0);
-            sEg[2 * lane + 1] = __expf(e1);
-            sEt[2 * lane] = __expf(gc - e0);
-            sEt[2 * lane + 1] = __expf(gc - e1);
-        } else if (w == 2 || w == 3) {
-            sBeta[tid - 64] = sGst[C + tid - 64];
-        }
-
-        // ---------------- staged bf16 K, Q, V -> fp16 tiles
 #pragma unroll 4
-        for (int idx = tid; idx < 3 * C * 16; idx += NT) {
-            const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
-            __half *dst = which == 0 ? sK : (which == 1 ? sQ : sV);
-            *reinterpret_cast<uint4 *>(dst + r * LDD + c16 * 8) = bf16x8_to_f16x8(sStg[idx]);
+            for (int idx = tid; idx < 2 * C * 16; idx += NT) {   // K and Q as they are
+                const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
+                *reinterpret_cast<uint4 *>((which ? sQ : sK) + r * LDD + c16 * 8) = bf16x8_to_f16x8(sStg[idx]);
+            }
+        } else {
+            const float *gp = a.g + (((long)b * T + t0 + 32 * ch_h) * a.Hv + h) * D + ch_c;
+            const long gstride = (long)a.Hv * D;
+            float s = 0.f;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                s += (32 * ch_h + r < n) ? __ldg(gp + r * gstride) : 0.f;
+                Gv[r] = s;
+            }
+            sTot[ch_h * D + ch_c] = s;
+            if (w == 2 || w == 3) sBeta[tid - 64] = sGst[C + tid - 64];
+            __syncthreads();
+            gm = sTot[ch_c];
+            gcs = gm + sTot[D + ch_c];
+            if (ch_h) {
+#pragma unroll
+                for (int r = 0; r < 32; ++r) Gv[r] += gm;
+            } else {
+                sG[ch_c] = __expf(gcs);   // Gamma_C of channel c
+            }
+            // Gram operands about the reference row 31: rows of K and Q scaled by
+            // exp(G_r - G_31), columns of K by exp(G_31 - G_i). Each factor spans at
+            // most 32 tokens of decay; a product over a pair i <= r is exp(G_r - G_i).
+            bool bad = false;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const int row = 32 * ch_h + r;
+                const float f1 = __expf(Gv[r] - gm), f2 = __expf(gm - Gv[r]);
+                const float kv = __bfloat162float(sStgH[row * D + ch_c]);
+                const float qv = __bfloat162float(sStgH[C * D + row * D + ch_c]);
+                const float kr = kv * f1, qr = qv * f1, kc = kv * f2;
+                bad |= fabsf(kr) > 65504.f || fabsf(qr) > 65504.f || fabsf(kc) > 65504.f;
+                sK[row * LDD + ch_c] = __float2half_rn(kr);
+                sQ[row * LDD + ch_c] = __float2half_rn(qr);
+                sW[row * LDD + ch_c] = __float2half_rn(kc);
+            }
+            if (bad) atomicAdd(&g_fused_range_errors, 1u);
+        }
+        for (int idx = tid; idx < C * (DVC / 8); idx += NT) {   // this CTA's V columns
+            const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
+            *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) = bf16x8_to_f16x8(sStg[2 * C * 16 + idx]);
         }
         __syncthreads();
-        if (ch + 1 < NC) issue_loads(ch + 1);
+        if (GATE == 0 && ch + 1 < NC) issue_loads(ch + 1);
 
-        // ---------------- Gram [K ; Q] K^T: warps 0-3 rows of K, warps 4-7 rows of Q
+        // ---------------- Gram: warps 0-3 rows of K, warps 4-7 rows of Q, against the
+        // 64 key rows (GATE 1: the scaled row and column operands)
         {
             float acc[8][4];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-            const uint32_t abase = w < 4 ? aK : aQ;
+            const uint32_t abase = w < 4 ? aK : aQ, bbase = GATE ? aW : aK;
 #pragma unroll
             for (int k0 = 0; k0 < D; k0 += 16) {
                 uint32_t af[4];
@@ -332,40 +397,57 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
                     uint32_t bf[4];
-                    ldsm(bf, b_nk(aK, LDD, 16 * np, k0, lane));
+                    ldsm(bf, b_nk(bbase, LDD, 16 * np, k0, lane));
                     mma(acc[2 * np], af, bf[0], bf[1]);
                     mma(acc[2 * np + 1], af, bf[2], bf[3]);
                 }
             }
-            // A rows (fp32) from warps 0-3; M rows (fp16) from warps 4-7
+            if (GATE) __syncthreads();   // the scaled tiles are rewritten below
+            // A rows (fp32 and fp16) from warps 0-3; M rows (fp16) from warps 4-7
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int r = rw0 + g + 8 * hh;
-                const float gr = sG[r], br = sBeta[r];
+                const float gr = GATE ? 0.f : sG[r], br = sBeta[r];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int i = 8 * j + 2 * t4;
                     const float d0 = acc[j][2 * hh], d1 = acc[j][2 * hh + 1];
+                    const float f0 = GATE ? 1.f : __expf(gr - sG[i]), f1 = GATE ? 1.f : __expf(gr - sG[i + 1]);
                     if (w < 4) {
-                        const float x0 = i < r ? br * __expf(gr - sG[i]) * d0 : 0.f;
-                        const float x1 = i + 1 < r ? br * __expf(gr - sG[i + 1]) * d1 : 0.f;
+                        const float x0 = i < r ? br * f0 * d0 : 0.f;
+                        const float x1 = i + 1 < r ? br * f1 * d1 : 0.f;
                         sA[r * LDF + i] = x0;
                         sA[r * LDF + i + 1] = x1;
                         st_h2(sAh + r * LDC + i, x0, x1);
                     } else {
-                        st_h2(sM + r * LDC + i, i <= r ? __expf(gr - sG[i]) * d0 : 0.f,
-                              i + 1 <= r ? __expf(gr - sG[i + 1]) * d1 : 0.f);
+                        st_h2(sM + r * LDC + i, i <= r ? f0 * d0 : 0.f, i + 1 <= r ? f1 * d1 : 0.f);
                     }
                 }
             }
         }
+        if (GATE) {
+            // K diag(Gamma) (for W), Q diag(Gamma) (for O) and K diag(Gamma_C / Gamma)
+            // (for the state update); every factor is at most 1.
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const int row = 32 * ch_h + r;
+                const float e1 = __expf(Gv[r]), e2 = __expf(gcs - Gv[r]);
+                const float kv = __bfloat162float(sStgH[row * D + ch_c]);
+                const float qv = __bfloat162float(sStgH[C * D + row * D + ch_c]);
+                sK[row * LDD + ch_c] = __float2half_rn(kv * e1);
+                sQ[row * LDD + ch_c] = __float2half_rn(qv * e1);
+                sUE[row * LDD + ch_c] = __float2half_rn(kv * e2);
+            }
+        }
         __syncthreads();
+        if (GATE == 1 && ch + 1 < NC) issue_loads(ch + 1);
 
         // ---------------- T = (I + A)^-1 (entries above the diagonal are never
         // written and read as zero). The 16x16 diagonal blocks by forward
         // substitution in fp32; then block rows bi = 1..3 on tensor cores, one
         // warp per block (bi, bj):
         //   X = sum_{m=bj}^{bi-1} A_{bi,m} T_{m,bj},   T_{bi,bj} = -T_{bi,bi} X
+        // The producers also write T diag(beta) and (GATE 0) T diag(beta Gamma).
         if (tid < 64) {
             const int base = (tid >> 4) * 16, col = tid & 15;
             float tv[16];
@@ -379,21 +461,21 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
                 }
                 tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -(s0 + s1));
             }
-            const float bc = sBeta[base + col], bgc = bc * sEg[base + col];
+            const float bc = sBeta[base + col], bgc = GATE ? 0.f : bc * sEg[base + col];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 const int o = (base + r) * LDC + base + col;
                 sTh[o] = __float2half_rn(tv[r]);
                 sTB[o] = __float2half_rn(tv[r] * bc);
-                sTG[o] = __float2half_rn(tv[r] * bgc);
+                if (GATE == 0) sTG[o] = __float2half_rn(tv[r] * bgc);
             }
         } else {
-            // zeros in the six blocks above the diagonal of T diag(beta), T diag(beta Gamma)
+            // zeros in the six blocks above the diagonal of T diag(beta) (and T diag(beta Gamma))
             const int e = tid - 64, blk = e >> 5, row = (e >> 1) & 15, hf = e & 1;
             const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
             const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
             *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
+            if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
         }
         __syncthreads();
 #pragma unroll 1
@@ -422,67 +504,80 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
                     mma(y[0], af, bf[0], bf[1]);
                     mma(y[1], af, bf[2], bf[3]);
                 }
-                // T_{bi,bj} = -y, and its columns scaled by beta and by beta Gamma
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r0 = 16 * bi + g, c = 16 * bj + 8 * j + 2 * t4;
                     const float b0 = sBeta[c], b1 = sBeta[c + 1];
-                    const float e0 = b0 * sEg[c], e1 = b1 * sEg[c + 1];
                     st_h2(sTh + r0 * LDC + c, -y[j][0], -y[j][1]);
                     st_h2(sTh + (r0 + 8) * LDC + c, -y[j][2], -y[j][3]);
                     st_h2(sTB + r0 * LDC + c, -y[j][0] * b0, -y[j][1] * b1);
                     st_h2(sTB + (r0 + 8) * LDC + c, -y[j][2] * b0, -y[j][3] * b1);
-                    st_h2(sTG + r0 * LDC + c, -y[j][0] * e0, -y[j][1] * e1);
-                    st_h2(sTG + (r0 + 8) * LDC + c, -y[j][2] * e0, -y[j][3] * e1);
+                    if (GATE == 0) {
+                        const float e0 = b0 * sEg[c], e1 = b1 * sEg[c + 1];
+                        st_h2(sTG + r0 * LDC + c, -y[j][0] * e0, -y[j][1] * e1);
+                        st_h2(sTG + (r0 + 8) * LDC + c, -y[j][2] * e0, -y[j][3] * e1);
+                    }
                 }
             }
             __syncthreads();
         }
 
-        // ---------------- W = T diag(beta Gamma) K,  U = T diag(beta) V  (warp tile 16 x 64)
-        float accU[8][4];
+        // ---------------- W = T diag(beta Gamma) K (GATE 1: T diag(beta) (K diag Gamma)),
+        // all 128 key columns, warp tile 16 x 64
         {
             float accW[8][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                accW[j][0] = accW[j][1] = accW[j][2] = accW[j][3] = accU[j][0] = accU[j][1] = accU[j][2] =
-                    accU[j][3] = 0.f;
+            for (int j = 0; j < 8; ++j) accW[j][0] = accW[j][1] = accW[j][2] = accW[j][3] = 0.f;
+            const int kw0 = 64 * (w >> 2);
 #pragma unroll
             for (int k0 = 0; k0 < C; k0 += 16) {
-                uint32_t atg[4], atb[4];
-                ldsm(atg, a_rm(aTG, LDC, rw0, k0, lane));
-                ldsm(atb, a_rm(aTB, LDC, rw0, k0, lane));
+                uint32_t at[4];
+                ldsm(at, a_rm(GATE ? aTB : aTG, LDC, rw0, k0, lane));
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
-                    uint32_t bk[4], bv[4];
-                    ldsm_t(bk, b_kn(aK, LDD, cw0 + 16 * np, k0, lane));
-                    ldsm_t(bv, b_kn(aV, LDD, cw0 + 16 * np, k0, lane));
-                    mma(accW[2 * np], atg, bk[0], bk[1]);
-                    mma(accW[2 * np + 1], atg, bk[2], bk[3]);
-                    mma(accU[2 * np], atb, bv[0], bv[1]);
-                    mma(accU[2 * np + 1], atb, bv[2], bv[3]);
+                    uint32_t bk[4];
+                    ldsm_t(bk, b_kn(aK, LDD, kw0 + 16 * np, k0, lane));
+                    mma(accW[2 * np], at, bk[0], bk[1]);
+                    mma(accW[2 * np + 1], at, bk[2], bk[3]);
                 }
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const int c = cw0 + 8 * j + 2 * t4;
+                const int c = kw0 + 8 * j + 2 * t4;
                 st_h2(sW + (rw0 + g) * LDD + c, -accW[j][0], -accW[j][1]);
                 st_h2(sW + (rw0 + g + 8) * LDD + c, -accW[j][2], -accW[j][3]);
             }
         }
+        // ---------------- U = T diag(beta) V on this CTA's value columns (warp tile 16 x DVC/2)
+        float accU[NJ][4];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) accU[j][0] = accU[j][1] = accU[j][2] = accU[j][3] = 0.f;
+#pragma unroll
+        for (int k0 = 0; k0 < C; k0 += 16) {
+            uint32_t atb[4];
+            ldsm(atb, a_rm(aTB, LDC, rw0, k0, lane));
+#pragma unroll
+            for (int np = 0; np < NJ / 2; ++np) {
+                uint32_t bv[4];
+                ldsm_t(bv, b_kn(aV, LDD, cw0 + 16 * np, k0, lane));
+                mma(accU[2 * np], atb, bv[0], bv[1]);
+                mma(accU[2 * np + 1], atb, bv[2], bv[3]);
+            }
+        }
         __syncthreads();
 
-        // ---------------- U' = U - W S,  O1 = Q S  (K-dim dk)
-        float accO[8][4];
+        // ---------------- U' = U - W S,  O1 = Q S (GATE 0: then scaled by Gamma_r;
+        // GATE 1: Q already carries Gamma), K-dim dk
+        float accO[NJ][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) accO[j][0] = accO[j][1] = accO[j][2] = accO[j][3] = 0.f;
+        for (int j = 0; j < NJ; ++j) accO[j][0] = accO[j][1] = accO[j][2] = accO[j][3] = 0.f;
 #pragma unroll
         for (int k0 = 0; k0 < D; k0 += 16) {
             uint32_t aw[4], aq[4];
             ldsm(aw, a_rm(aW, LDD, rw0, k0, lane));
             ldsm(aq, a_rm(aQ, LDD, rw0, k0, lane));
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < NJ / 2; ++np) {
                 uint32_t bs[4];
                 ldsm_t(bs, b_kn(aS, LDD, cw0 + 16 * np, k0, lane));
                 mma(accU[2 * np], aw, bs[0], bs[1]);
@@ -492,16 +587,18 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
             }
         }
         {
-            const float eg0 = sEg[rw0 + g], eg1 = sEg[rw0 + g + 8];
-            const float et0 = sEt[rw0 + g], et1 = sEt[rw0 + g + 8];
+            const float eg0 = GATE ? 1.f : sEg[rw0 + g], eg1 = GATE ? 1.f : sEg[rw0 + g + 8];
+            const float et0 = GATE ? 1.f : sEt[rw0 + g], et1 = GATE ? 1.f : sEt[rw0 + g + 8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < NJ; ++j) {
                 accO[j][0] *= eg0; accO[j][1] *= eg0; accO[j][2] *= eg1; accO[j][3] *= eg1;
                 const int c = cw0 + 8 * j + 2 * t4;
                 st_h2(sU + (rw0 + g) * LDD + c, accU[j][0], accU[j][1]);
                 st_h2(sU + (rw0 + g + 8) * LDD + c, accU[j][2], accU[j][3]);
-                st_h2(sUE + (rw0 + g) * LDD + c, accU[j][0] * et0, accU[j][1] * et0);
-                st_h2(sUE + (rw0 + g + 8) * LDD + c, accU[j][2] * et1, accU[j][3] * et1);
+                if (GATE == 0) {
+                    st_h2(sUE + (rw0 + g) * LDD + c, accU[j][0] * et0, accU[j][1] * et0);
+                    st_h2(sUE + (rw0 + g + 8) * LDD + c, accU[j][2] * et1, accU[j][3] * et1);
+                }
             }
         }
         __syncthreads();
@@ -512,7 +609,7 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
             uint32_t am[4];
             ldsm(am, a_rm(aM, LDC, rw0, k0, lane));
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < NJ / 2; ++np) {
                 uint32_t bu[4];
                 ldsm_t(bu, b_kn(aU, LDD, cw0 + 16 * np, k0, lane));
                 mma(accO[2 * np], am, bu[0], bu[1]);
@@ -520,38 +617,40 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
             }
         }
         {
-            TOut *op = reinterpret_cast<TOut *>(a.o) + (((long)b * T + t0) * a.Hv + h) * D + cw0 + 2 * t4;
+            TOut *op = reinterpret_cast<TOut *>(a.o) + (((long)b * T + t0) * a.Hv + h) * D + dv0 + cw0 + 2 * t4;
             const long rs = (long)a.Hv * D;
             const int r0 = rw0 + g, r1 = rw0 + g + 8;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < NJ; ++j) {
                 if (r0 < n) store_out2(op + r0 * rs + 8 * j, accO[j][0], accO[j][1]);
                 if (r1 < n) store_out2(op + r1 * rs + 8 * j, accO[j][2], accO[j][3]);
             }
         }
 
-        // ---------------- S <- Gamma_C S + K^T diag(e) U'  (warp rows dk 16w.., all dv)
+        // ---------------- S <- Gamma_C S + K^T diag(e) U'  (GATE 1: diag(Gamma_C) S +
+        // (K diag(Gamma_C / Gamma))^T U'); warp rows dk 16w.., this CTA's columns
         {
-            const float gc = sEg[C - 1];
+            const int r0 = 16 * w + g;
+            const float gc0 = GATE ? sG[r0] : sEg[C - 1], gc1 = GATE ? sG[r0 + 8] : sEg[C - 1];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                accS[j][0] *= gc; accS[j][1] *= gc; accS[j][2] *= gc; accS[j][3] *= gc;
+            for (int j = 0; j < NJS; ++j) {
+                accS[j][0] *= gc0; accS[j][1] *= gc0; accS[j][2] *= gc1; accS[j][3] *= gc1;
             }
+            const uint32_t aKs = GATE ? aUE : aK, aUs = GATE ? aU : aUE;
 #pragma unroll
             for (int k0 = 0; k0 < C; k0 += 16) {
                 uint32_t ak[4];
-                ldsm_t(ak, a_tr(aK, LDD, 16 * w, k0, lane));
+                ldsm_t(ak, a_tr(aKs, LDD, 16 * w, k0, lane));
 #pragma unroll
-                for (int np = 0; np < 8; ++np) {
+                for (int np = 0; np < NJS / 2; ++np) {
                     uint32_t bu[4];
-                    ldsm_t(bu, b_kn(aUE, LDD, 16 * np, k0, lane));
+                    ldsm_t(bu, b_kn(aUs, LDD, 16 * np, k0, lane));
                     mma(accS[2 * np], ak, bu[0], bu[1]);
                     mma(accS[2 * np + 1], ak, bu[2], bu[3]);
                 }
             }
-            const int r0 = 16 * w + g;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < NJS; ++j) {
                 const int c = 8 * j + 2 * t4;
                 st_h2(sS + r0 * LDD + c, accS[j][0], accS[j][1]);
                 st_h2(sS + (r0 + 8) * LDD + c, accS[j][2], accS[j][3]);
@@ -561,10 +660,10 @@ fused_fwd_gdn_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const
     }
 
     if (a.hT) {
-        float *hp = a.hT + (size_t)bh * D * D;
+        float *hp = a.hT + (size_t)bh * D * D + dv0;
         const int r0 = 16 * w + g;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < NJS; ++j) {
             const int c = 8 * j + 2 * t4;
             *reinterpret_cast<float2 *>(hp + (size_t)r0 * D + c) = make_float2(accS[j][0], accS[j][1]);
             *reinterpret_cast<float2 *>(hp + (size_t)(r0 + 8) * D + c) = make_float2(accS[j][2], accS[j][3]);
@@ -590,14 +689,14 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// Tensor map of a [B][T][H][128] bf16 tensor for boxes of 64 consecutive
-// tokens of one head: dims (d, head, t, b), box (128, 1, 64, 1). Tokens past T
-// read as zero.
-bool make_map(CUtensorMap *map, const void *base, int B, int T, int H)
+// Tensor map of a [B][T][H][128] bf16 tensor for boxes of `cols` channels of 64
+// consecutive tokens of one head: dims (d, head, t, b), box (cols, 1, 64, 1).
+// Tokens past T read as zero.
+bool make_map(CUtensorMap *map, const void *base, int B, int T, int H, int cols)
 {
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)C, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)cols, 1, (cuuint32_t)C, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const EncodeTiledFn encode = encode_tiled();
     return encode && encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
@@ -605,30 +704,64 @@ bool make_map(CUtensorMap *map, const void *base, int B, int T, int H)
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TOut>
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+        return 0;
+    return n;
+}
+
+template <typename TOut, int GATE, int NS>
 cudaError_t launch_t(const FwdArgs &a, cudaStream_t st)
 {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, a.B, a.T, a.Hk) || !make_map(&mk, a.k, a.B, a.T, a.Hk) ||
-        !make_map(&mv, a.v, a.B, a.T, a.Hv))
+    if (!make_map(&mq, a.q, a.B, a.T, a.Hk, D) || !make_map(&mk, a.k, a.B, a.T, a.Hk, D) ||
+        !make_map(&mv, a.v, a.B, a.T, a.Hv, D / NS))
         return cudaErrorInvalidValue;
     const int smem = SMEM_BYTES + 128;
-    cudaError_t e = cudaFuncSetAttribute(fused_fwd_gdn_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kernel = fused_fwd_kernel<TOut, GATE, NS>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    fused_fwd_gdn_kernel<TOut><<<(unsigned)((long)a.B * a.Hv), NT, smem, st>>>(a, mq, mk, mv);
+    kernel<<<(unsigned)((long)a.B * a.Hv * NS), NT, smem, st>>>(a, mq, mk, mv);
     return cudaGetLastError();
+}
+
+template <typename TOut, int GATE>
+cudaError_t launch_g(const FwdArgs &a, cudaStream_t st)
+{
+    // Split the value columns over two CTAs when that still fits the SMs in one wave.
+    const long units = (long)a.B * a.Hv;
+    return 2 * units <= sm_count() ? launch_t<TOut, GATE, 2>(a, st) : launch_t<TOut, GATE, 1>(a, st);
+}
+
+template <typename TOut>
+cudaError_t launch_o(const FwdArgs &a, cudaStream_t st)
+{
+    return a.gate_mode == 0 ? launch_g<TOut, 0>(a, st) : launch_g<TOut, 1>(a, st);
 }
 
 }  // namespace
 
 bool fused_supported(const FwdArgs &a)
 {
-    return in_bf16(a.dtype) && a.gate_mode == 0 && a.Dk == D && a.Dv == D;
+    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D;
 }
 
 cudaError_t launch_fwd_fused(const FwdArgs &a, cudaStream_t st)
 {
-    return out_f32(a.dtype) ? launch_t<float>(a, st) : launch_t<__nv_bfloat16>(a, st);
+    return out_f32(a.dtype) ? launch_o<float>(a, st) : launch_o<__nv_bfloat16>(a, st);
+}
+
+unsigned int fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors)
+{
+    unsigned int t = 0, r = 0;
+    cudaMemcpyFromSymbol(&t, g_fused_load_timeouts, sizeof(t));
+    cudaMemcpyFromSymbol(&r, g_fused_range_errors, sizeof(r));
+    if (load_timeouts) *load_timeouts = t;
+    if (range_errors) *range_errors = r;
+    return t + r;
 }
 
 }  // namespace gdr

@@ -72,6 +72,11 @@ const char *gdr_last_error(void) { return g_err; }
 
 unsigned long long gdr_kernel_launches(void) { return g_launches.load(); }
 
+unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors)
+{
+    return gdr::fused_error_counts(load_timeouts, range_errors);
+}
+
 size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype)
 {
     if (check_common(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) != GDR_OK) return 0;

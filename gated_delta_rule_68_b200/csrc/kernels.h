@@ -27,10 +27,13 @@ struct FwdArgs {
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 
-// Fused chunked forward on the warp-level tensor cores (scalar gate, bf16 inputs,
-// Dk = Dv = 128): one kernel, no workspace.
+// Fused chunked forward on the warp-level tensor cores (bf16 inputs, Dk = Dv = 128,
+// either gate): one kernel, no workspace.
 bool fused_supported(const FwdArgs &a);
 cudaError_t launch_fwd_fused(const FwdArgs &a, cudaStream_t st);
+// Device-side failure counts of the fused kernel since the library was loaded on this
+// device: chunk loads that timed out, and per-channel gate factors outside the fp16 range.
+unsigned int fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors);
 
 // fp32 CUDA-core chunked forward (three kernels). Needs simt_workspace_size() bytes.
 size_t simt_workspace_size(const FwdArgs &a);

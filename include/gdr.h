@@ -87,6 +87,20 @@ GDR_API const char *gdr_last_error(void);
 GDR_API unsigned long long gdr_kernel_launches(void);
 
 /*
+ * Device-side failure counts of the fused chunked kernel (bf16 inputs,
+ * Dk = Dv = 128) on the current device, accumulated since the library was
+ * loaded there. Either pointer may be NULL; returns the sum of the two.
+ *   load_timeouts  chunk input loads that had not arrived after one second;
+ *                  the (batch row, value head) unit stops, so that call's o and
+ *                  hT are incomplete.
+ *   range_errors   chunks whose per-key-channel gate factors left the fp16
+ *                  range (a decay stronger than about exp(-11) within 32
+ *                  tokens); that chunk's results are not valid.
+ * Reads device memory, so it waits for prior work on the default stream.
+ */
+GDR_API unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors);
+
+/*
  * Bytes of device workspace gdr_fwd_chunked needs for these sizes (0 when it
  * needs none). Returns 0 for invalid arguments as well; gdr_fwd_chunked then
  * reports the actual error.

@@ -51,15 +51,15 @@ def test_noalloc_matches_fwd_chunked_on_two_calls(dtype, gate):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # Per-key-channel gate, B=2, T=16384, 32 heads: its workspace is far beyond the fixed scratch.
-    w = WORKLOADS["kda_bf16"]
-    need = gdr.gdr_fwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16)
+    # fp32 inputs (the CUDA-core path), B=2, T=16384, 32 heads: a workspace far beyond the scratch.
+    w = WORKLOADS["kda_bf16"].with_(dtype="fp32")
+    need = gdr.gdr_fwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, gdr.GDR_GATE_CHANNEL, gdr.GDR_FP32)
     assert need > gdr.GDR_NOALLOC_SCRATCH_BYTES
     inp = make_inputs(w.with_(T=64), DEV)   # real buffers; the call must not touch them
-    o = torch.empty((w.B, 64, w.Hv, w.Dv), dtype=torch.bfloat16, device=DEV)
+    o = torch.empty((w.B, 64, w.Hv, w.Dv), dtype=torch.float32, device=DEV)
     vp = lambda t: ctypes.c_void_p(t.data_ptr())
     st = gdr.lib().gdr_fwd_chunked_noalloc(vp(inp["q"]), vp(inp["k"]), vp(inp["v"]), vp(inp["g"]),
                                            vp(inp["beta"]), None, vp(o), None, w.B, w.T, w.Hk, w.Hv,
-                                           w.Dk, w.Dv, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16, None)
+                                           w.Dk, w.Dv, gdr.GDR_GATE_CHANNEL, gdr.GDR_FP32, None)
     assert st == gdr.GDR_ERR_WORKSPACE
     assert "scratch" in gdr.gdr_last_error()
