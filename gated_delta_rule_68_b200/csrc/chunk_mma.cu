@@ -74,7 +74,8 @@ static_assert(C * LDF * 4 <= SZ_D, "A must fit in the U' tile");
 static_assert(C * LDC * 2 <= SZ_D, "T must fit in the diag(e) U' tile");
 static_assert(8 * 16 * LDX * 2 + C * LDC * 2 <= SZ_D, "block-row products and A must fit in the W tile");
 static_assert(SMEM_BYTES + 128 <= 227 * 1024, "shared memory");
-static_assert(OFF_STG % 128 == 0, "TMA destination alignment");
+static_assert(OFF_STG % 128 == 0 && OFF_V % 128 == 0, "TMA shared-memory alignment");
+static_assert(C * D * 4 <= 2 * SZ_D, "an fp32 o tile must fit in the V and W tiles");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -146,6 +147,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
                  :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
                  : "memory");
 }
+// One 4-d box from shared memory to a tensor (TMA tiled store); coordinates past
+// the tensor's end are not written. Completion is tracked per issuing thread.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];"
+                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src) : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t done;
@@ -212,7 +225,7 @@ __device__ unsigned int g_fused_range_errors;
 template <typename TOut, int GATE, int NS>
 __global__ void __launch_bounds__(NT, 1)
 fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                 const __grid_constant__ CUtensorMap map_v)
+                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
 {
     constexpr int DVC = D / NS;      // value columns of this CTA
     constexpr int NJ = DVC / 16;     // n8 tiles of a warp in the [64 x DVC] products (half the columns)
@@ -235,6 +248,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     float *sEt = sG + 128;                                 // [64] exp(G_C - G_r)
     float *sBeta = sG + 192;                               // [64]
     float *sTot = sG + 256;                                // GATE 1: [2][128] per-channel sums of each half chunk
+    float *sColf = sG + 256;                               // GATE 0: [4][64] exp(G_16R - G_i)
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
     const uint32_t aTB = smem_u32(sTB), aTG = smem_u32(sTG), aAh = smem_u32(sAh), aTh = smem_u32(sTh);
@@ -302,6 +316,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     for (int ch = 0; ch < NC; ++ch) {
         const int t0 = ch * C, n = min(C, T - t0);
         cp_async_wait_all();
+        if (tid == 0) tma_store_wait_read();   // the previous chunk's o tile has been read out
         if (!__syncthreads_and(mbar_wait_bounded(aBar, ch & 1))) {
             if (tid == 0) atomicAdd(&g_fused_load_timeouts, 1u);
             return;
@@ -330,6 +345,13 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 sEg[2 * lane + 1] = __expf(e1);
                 sEt[2 * lane] = __expf(gc - e0);
                 sEt[2 * lane + 1] = __expf(gc - e1);
+                // column factors exp(G_16R - G_i) for the Gram rows of block R (i < 16R + 16)
+#pragma unroll
+                for (int R = 0; R < 4; ++R) {
+                    const float gR = __shfl_sync(0xffffffffu, e0, 8 * R);
+                    sColf[R * C + 2 * lane] = 2 * lane < 16 * R + 16 ? __expf(gR - e0) : 0.f;
+                    sColf[R * C + 2 * lane + 1] = 2 * lane + 1 < 16 * R + 16 ? __expf(gR - e1) : 0.f;
+                }
             } else if (w == 2 || w == 3) {
                 sBeta[tid - 64] = sGst[C + tid - 64];
             }
@@ -376,12 +398,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
             if (bad) atomicAdd(&g_fused_range_errors, 1u);
         }
-        for (int idx = tid; idx < C * (DVC / 8); idx += NT) {   // this CTA's V columns
-            const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
-            *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) = bf16x8_to_f16x8(sStg[2 * C * 16 + idx]);
-        }
         __syncthreads();
-        if (GATE == 0 && ch + 1 < NC) issue_loads(ch + 1);
 
         // ---------------- Gram: warps 0-3 rows of K, warps 4-7 rows of Q, against the
         // 64 key rows (GATE 1: the scaled row and column operands)
@@ -407,12 +424,13 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int r = rw0 + g + 8 * hh;
-                const float gr = GATE ? 0.f : sG[r], br = sBeta[r];
+                const float rf = GATE ? 1.f : __expf(sG[r] - sG[r & ~15]), br = sBeta[r];
+                const float *cf = sColf + (r >> 4) * C;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int i = 8 * j + 2 * t4;
                     const float d0 = acc[j][2 * hh], d1 = acc[j][2 * hh + 1];
-                    const float f0 = GATE ? 1.f : __expf(gr - sG[i]), f1 = GATE ? 1.f : __expf(gr - sG[i + 1]);
+                    const float f0 = GATE ? 1.f : rf * cf[i], f1 = GATE ? 1.f : rf * cf[i + 1];
                     if (w < 4) {
                         const float x0 = i < r ? br * f0 * d0 : 0.f;
                         const float x1 = i + 1 < r ? br * f1 * d1 : 0.f;
@@ -440,7 +458,6 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
         }
         __syncthreads();
-        if (GATE == 1 && ch + 1 < NC) issue_loads(ch + 1);
 
         // ---------------- T = (I + A)^-1 (entries above the diagonal are never
         // written and read as zero). The 16x16 diagonal blocks by forward
@@ -476,8 +493,13 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
             *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
             if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
+            for (int idx = tid - 64; idx < C * (DVC / 8); idx += NT - 64) {   // this CTA's V columns
+                const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
+                *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) = bf16x8_to_f16x8(sStg[2 * C * 16 + idx]);
+            }
         }
         __syncthreads();
+        if (ch + 1 < NC) issue_loads(ch + 1);   // the staging area has been consumed
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {
             if (w < bi) {
@@ -616,15 +638,15 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 mma(accO[2 * np + 1], am, bu[2], bu[3]);
             }
         }
-        {
-            TOut *op = reinterpret_cast<TOut *>(a.o) + (((long)b * T + t0) * a.Hv + h) * D + dv0 + cw0 + 2 * t4;
-            const long rs = (long)a.Hv * D;
+        {   // o rows -> a dense [64][DVC] tile over the dead V and W tiles -> one TMA store
+            TOut *so = reinterpret_cast<TOut *>(sm + OFF_V) + cw0 + 2 * t4;
             const int r0 = rw0 + g, r1 = rw0 + g + 8;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                if (r0 < n) store_out2(op + r0 * rs + 8 * j, accO[j][0], accO[j][1]);
-                if (r1 < n) store_out2(op + r1 * rs + 8 * j, accO[j][2], accO[j][3]);
+                store_out2(so + r0 * DVC + 8 * j, accO[j][0], accO[j][1]);
+                store_out2(so + r1 * DVC + 8 * j, accO[j][2], accO[j][3]);
             }
+            fence_proxy_async();
         }
 
         // ---------------- S <- Gamma_C S + K^T diag(e) U'  (GATE 1: diag(Gamma_C) S +
@@ -657,7 +679,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
         }
         __syncthreads();
+        if (tid == 0) tma_store_4d(&map_o, dv0, h, t0, b, smem_u32(sm + OFF_V));
     }
+    if (tid == 0) tma_store_wait_all();
 
     if (a.hT) {
         float *hp = a.hT + (size_t)bh * D * D + dv0;
@@ -689,17 +713,19 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// Tensor map of a [B][T][H][128] bf16 tensor for boxes of `cols` channels of 64
+// Tensor map of a [B][T][H][128] bf16 (or fp32) tensor for boxes of `cols` channels of 64
 // consecutive tokens of one head: dims (d, head, t, b), box (cols, 1, 64, 1).
 // Tokens past T read as zero.
-bool make_map(CUtensorMap *map, const void *base, int B, int T, int H, int cols)
+bool make_map(CUtensorMap *map, const void *base, int B, int T, int H, int cols, bool f32 = false)
 {
+    const cuuint64_t es = f32 ? 4 : 2;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es, (cuuint64_t)T * H * D * es};
     const cuuint32_t box[4] = {(cuuint32_t)cols, 1, (cuuint32_t)C, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const EncodeTiledFn encode = encode_tiled();
-    return encode && encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+    return encode && encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                            const_cast<void *>(base), dims, strides, box,
                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -716,15 +742,16 @@ int sm_count()
 template <typename TOut, int GATE, int NS>
 cudaError_t launch_t(const FwdArgs &a, cudaStream_t st)
 {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, a.q, a.B, a.T, a.Hk, D) || !make_map(&mk, a.k, a.B, a.T, a.Hk, D) ||
-        !make_map(&mv, a.v, a.B, a.T, a.Hv, D / NS))
+        !make_map(&mv, a.v, a.B, a.T, a.Hv, D / NS) ||
+        !make_map(&mo, a.o, a.B, a.T, a.Hv, D / NS, sizeof(TOut) == 4))
         return cudaErrorInvalidValue;
     const int smem = SMEM_BYTES + 128;
     auto kernel = fused_fwd_kernel<TOut, GATE, NS>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kernel<<<(unsigned)((long)a.B * a.Hv * NS), NT, smem, st>>>(a, mq, mk, mv);
+    kernel<<<(unsigned)((long)a.B * a.Hv * NS), NT, smem, st>>>(a, mq, mk, mv, mo);
     return cudaGetLastError();
 }
 
