@@ -39,7 +39,11 @@ namespace {
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int NT = 256;          // 8 warps
+constexpr int NW = 16;           // warps per CTA
+constexpr int NT = 32 * NW;
+constexpr int NCB = NW / 4;      // column blocks of the [64 x n] products (4 row blocks of 16)
+constexpr int NCS = NW / 8;      // column blocks of the [128 x n] products (8 row blocks of 16)
+constexpr int NQ = NT / 128;     // row groups of the per-channel gate pass (one thread per channel and group)
 constexpr int LDD = D + 8;       // fp16 row stride of 128-wide tiles (272 B: ldmatrix rows hit distinct banks)
 constexpr int LDC = C + 8;       // fp16 row stride of 64-wide tiles (144 B)
 constexpr int LDF = C + 1;       // fp32 row stride of the 64 x 64 scratch
@@ -59,8 +63,8 @@ constexpr int OFF_TB = OFF_M + SZ_C;            // T diag(beta) [r][i]
 constexpr int OFF_TG = OFF_TB + SZ_C;           // T diag(beta Gamma) [r][i]
 constexpr int OFF_STG = OFF_TG + SZ_C;          // next chunk's K, Q, V as loaded (bf16 [3][64][128])
 constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32 [2][64])
-constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta (64 fp32 each); 2 x 128 fp32 sums
-constexpr int SMEM_BYTES = OFF_VEC + 512 * 4;
+constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta (64 fp32 each); NQ x 128 fp32 sums
+constexpr int SMEM_BYTES = OFF_VEC + (256 + NQ * 128) * 4;
 // The scratch of the inverse reuses tiles that are dead while it is live: fp32
 // A sits in the U' tile, the fp16 inverse T in the diag(e) U' tile, and the
 // fp16 copy of A (an operand of the block-row products) after each warp's
@@ -228,8 +232,11 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
 {
     constexpr int DVC = D / NS;      // value columns of this CTA
-    constexpr int NJ = DVC / 16;     // n8 tiles of a warp in the [64 x DVC] products (half the columns)
-    constexpr int NJS = DVC / 8;     // n8 tiles of a warp's state rows
+    constexpr int NJ = DVC / NCB / 8;   // n8 tiles of a warp in the [64 x DVC] products
+    constexpr int NJS = DVC / NCS / 8;  // n8 tiles of a warp's state rows
+    constexpr int NJW = D / NCB / 8;    // n8 tiles of a warp in W [64 x 128]
+    constexpr int NJG = C / NCS / 8;    // n8 tiles of a warp in the Gram [128 x 64]
+    constexpr int RPT = C / NQ;         // GATE 1: rows per thread in the per-channel pass
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // 128-byte aligned base: the TMA destination tiles need it.
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -247,7 +254,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     float *sEg = sG + 64;                                  // [64] exp(G_r)      |
     float *sEt = sG + 128;                                 // [64] exp(G_C - G_r)
     float *sBeta = sG + 192;                               // [64]
-    float *sTot = sG + 256;                                // GATE 1: [2][128] per-channel sums of each half chunk
+    float *sTot = sG + 256;                                // GATE 1: [NQ][128] per-channel sums of each row group
     float *sColf = sG + 256;                               // GATE 0: [4][64] exp(G_16R - G_i)
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
@@ -264,18 +271,20 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     const int b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, NC = (T + C - 1) / C;
 
-    // Row block (16 rows) and column half of this warp in the [64 x DVC] products.
-    const int rw0 = 16 * (w & 3), cw0 = (DVC / 2) * (w >> 2);
+    // Row block (16 rows) and column block of this warp in the [64 x DVC] products,
+    // and in the [128 x DVC] state.
+    const int rw0 = 16 * (w & 3), cw0 = (DVC / NCB) * (w >> 2);
+    const int rs0 = 16 * (w & 7), cs0 = (DVC / NCS) * (w >> 3);
 
     // State S[:, dv0 .. dv0 + DVC) in registers: warp w holds dk rows 16w..16w+15;
     // n8 tile j holds local columns 8j..8j+7.
     float accS[NJS][4];
     {
         const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + dv0 : nullptr;
-        const int r0 = 16 * w + g;
+        const int r0 = rs0 + g;
 #pragma unroll
         for (int j = 0; j < NJS; ++j) {
-            const int c = 8 * j + 2 * t4;
+            const int c = cs0 + 8 * j + 2 * t4;
             float2 x0 = make_float2(0.f, 0.f), x1 = x0;
             if (h0) {
                 x0 = *reinterpret_cast<const float2 *>(h0 + (size_t)r0 * D + c);
@@ -323,9 +332,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         }
 
         // ---------------- gates and fp16 operand tiles
-        // GATE 1 keeps each channel's prefix G for 32 rows in registers: thread
-        // (c, hf) owns key channel c = tid % 128 and rows 32 hf .. 32 hf + 31.
-        float Gv[GATE ? 32 : 1];
+        // GATE 1 keeps each channel's prefix G for RPT rows in registers: thread
+        // (c, q) owns key channel c = tid % 128 and rows RPT q .. RPT q + RPT - 1.
+        float Gv[GATE ? RPT : 1];
         float gm = 0.f, gcs = 0.f;   // GATE 1: G at row 31 and at row 63 of channel c
         const int ch_c = tid & (D - 1), ch_h = tid >> 7;
         if (GATE == 0) {
@@ -361,32 +370,35 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 *reinterpret_cast<uint4 *>((which ? sQ : sK) + r * LDD + c16 * 8) = bf16x8_to_f16x8(sStg[idx]);
             }
         } else {
-            const float *gp = a.g + (((long)b * T + t0 + 32 * ch_h) * a.Hv + h) * D + ch_c;
+            const float *gp = a.g + (((long)b * T + t0 + RPT * ch_h) * a.Hv + h) * D + ch_c;
             const long gstride = (long)a.Hv * D;
             float s = 0.f;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                s += (32 * ch_h + r < n) ? __ldg(gp + r * gstride) : 0.f;
+            for (int r = 0; r < RPT; ++r) {
+                s += (RPT * ch_h + r < n) ? __ldg(gp + r * gstride) : 0.f;
                 Gv[r] = s;
             }
             sTot[ch_h * D + ch_c] = s;
             if (w == 2 || w == 3) sBeta[tid - 64] = sGst[C + tid - 64];
             __syncthreads();
-            gm = sTot[ch_c];
-            gcs = gm + sTot[D + ch_c];
-            if (ch_h) {
+            float off = 0.f;
 #pragma unroll
-                for (int r = 0; r < 32; ++r) Gv[r] += gm;
-            } else {
-                sG[ch_c] = __expf(gcs);   // Gamma_C of channel c
+            for (int q = 0; q < NQ; ++q) {
+                const float tq = sTot[q * D + ch_c];
+                off += q < ch_h ? tq : 0.f;
+                gm += q < NQ / 2 ? tq : 0.f;
+                gcs += tq;
             }
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) Gv[r] += off;
+            if (ch_h == 0) sG[ch_c] = __expf(gcs);   // Gamma_C of channel c
             // Gram operands about the reference row 31: rows of K and Q scaled by
             // exp(G_r - G_31), columns of K by exp(G_31 - G_i). Each factor spans at
             // most 32 tokens of decay; a product over a pair i <= r is exp(G_r - G_i).
             bool bad = false;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int row = 32 * ch_h + r;
+            for (int r = 0; r < RPT; ++r) {
+                const int row = RPT * ch_h + r;
                 const float f1 = __expf(Gv[r] - gm), f2 = __expf(gm - Gv[r]);
                 const float kv = __bfloat162float(sStgH[row * D + ch_c]);
                 const float qv = __bfloat162float(sStgH[C * D + row * D + ch_c]);
@@ -403,18 +415,21 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         // ---------------- Gram: warps 0-3 rows of K, warps 4-7 rows of Q, against the
         // 64 key rows (GATE 1: the scaled row and column operands)
         {
-            float acc[8][4];
+            // warp tile: rows 16 (w & 7) of [K ; Q], key rows cg0 .. cg0 + 64 / NCS - 1
+            float acc[NJG][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-            const uint32_t abase = w < 4 ? aK : aQ, bbase = GATE ? aW : aK;
+            for (int j = 0; j < NJG; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+            const bool krow = (w & 7) < 4;
+            const int cg0 = (C / NCS) * (w >> 3);
+            const uint32_t abase = krow ? aK : aQ, bbase = GATE ? aW : aK;
 #pragma unroll
             for (int k0 = 0; k0 < D; k0 += 16) {
                 uint32_t af[4];
                 ldsm(af, a_rm(abase, LDD, rw0, k0, lane));
 #pragma unroll
-                for (int np = 0; np < 4; ++np) {
+                for (int np = 0; np < NJG / 2; ++np) {
                     uint32_t bf[4];
-                    ldsm(bf, b_nk(bbase, LDD, 16 * np, k0, lane));
+                    ldsm(bf, b_nk(bbase, LDD, cg0 + 16 * np, k0, lane));
                     mma(acc[2 * np], af, bf[0], bf[1]);
                     mma(acc[2 * np + 1], af, bf[2], bf[3]);
                 }
@@ -427,11 +442,11 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 const float rf = GATE ? 1.f : __expf(sG[r] - sG[r & ~15]), br = sBeta[r];
                 const float *cf = sColf + (r >> 4) * C;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i = 8 * j + 2 * t4;
+                for (int j = 0; j < NJG; ++j) {
+                    const int i = cg0 + 8 * j + 2 * t4;
                     const float d0 = acc[j][2 * hh], d1 = acc[j][2 * hh + 1];
                     const float f0 = GATE ? 1.f : rf * cf[i], f1 = GATE ? 1.f : rf * cf[i + 1];
-                    if (w < 4) {
+                    if (krow) {
                         const float x0 = i < r ? br * f0 * d0 : 0.f;
                         const float x1 = i + 1 < r ? br * f1 * d1 : 0.f;
                         sA[r * LDF + i] = x0;
@@ -447,8 +462,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             // K diag(Gamma) (for W), Q diag(Gamma) (for O) and K diag(Gamma_C / Gamma)
             // (for the state update); every factor is at most 1.
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int row = 32 * ch_h + r;
+            for (int r = 0; r < RPT; ++r) {
+                const int row = RPT * ch_h + r;
                 const float e1 = __expf(Gv[r]), e2 = __expf(gcs - Gv[r]);
                 const float kv = __bfloat162float(sStgH[row * D + ch_c]);
                 const float qv = __bfloat162float(sStgH[C * D + row * D + ch_c]);
@@ -488,11 +503,14 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
         } else {
             // zeros in the six blocks above the diagonal of T diag(beta) (and T diag(beta Gamma))
-            const int e = tid - 64, blk = e >> 5, row = (e >> 1) & 15, hf = e & 1;
-            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
-            *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
-            if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
+            const int e = tid - 64;
+            if (e < 6 * 32) {
+                const int blk = e >> 5, row = (e >> 1) & 15, hf = e & 1;
+                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
+                *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
+                if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
+            }
             for (int idx = tid - 64; idx < C * (DVC / 8); idx += NT - 64) {   // this CTA's V columns
                 const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
                 *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) = bf16x8_to_f16x8(sStg[2 * C * 16 + idx]);
@@ -547,16 +565,16 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         // ---------------- W = T diag(beta Gamma) K (GATE 1: T diag(beta) (K diag Gamma)),
         // all 128 key columns, warp tile 16 x 64
         {
-            float accW[8][4];
+            float accW[NJW][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) accW[j][0] = accW[j][1] = accW[j][2] = accW[j][3] = 0.f;
-            const int kw0 = 64 * (w >> 2);
+            for (int j = 0; j < NJW; ++j) accW[j][0] = accW[j][1] = accW[j][2] = accW[j][3] = 0.f;
+            const int kw0 = (D / NCB) * (w >> 2);
 #pragma unroll
             for (int k0 = 0; k0 < C; k0 += 16) {
                 uint32_t at[4];
                 ldsm(at, a_rm(GATE ? aTB : aTG, LDC, rw0, k0, lane));
 #pragma unroll
-                for (int np = 0; np < 4; ++np) {
+                for (int np = 0; np < NJW / 2; ++np) {
                     uint32_t bk[4];
                     ldsm_t(bk, b_kn(aK, LDD, kw0 + 16 * np, k0, lane));
                     mma(accW[2 * np], at, bk[0], bk[1]);
@@ -564,7 +582,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 }
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < NJW; ++j) {
                 const int c = kw0 + 8 * j + 2 * t4;
                 st_h2(sW + (rw0 + g) * LDD + c, -accW[j][0], -accW[j][1]);
                 st_h2(sW + (rw0 + g + 8) * LDD + c, -accW[j][2], -accW[j][3]);
@@ -652,7 +670,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         // ---------------- S <- Gamma_C S + K^T diag(e) U'  (GATE 1: diag(Gamma_C) S +
         // (K diag(Gamma_C / Gamma))^T U'); warp rows dk 16w.., this CTA's columns
         {
-            const int r0 = 16 * w + g;
+            const int r0 = rs0 + g;
             const float gc0 = GATE ? sG[r0] : sEg[C - 1], gc1 = GATE ? sG[r0 + 8] : sEg[C - 1];
 #pragma unroll
             for (int j = 0; j < NJS; ++j) {
@@ -662,18 +680,18 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 #pragma unroll
             for (int k0 = 0; k0 < C; k0 += 16) {
                 uint32_t ak[4];
-                ldsm_t(ak, a_tr(aKs, LDD, 16 * w, k0, lane));
+                ldsm_t(ak, a_tr(aKs, LDD, rs0, k0, lane));
 #pragma unroll
                 for (int np = 0; np < NJS / 2; ++np) {
                     uint32_t bu[4];
-                    ldsm_t(bu, b_kn(aUs, LDD, 16 * np, k0, lane));
+                    ldsm_t(bu, b_kn(aUs, LDD, cs0 + 16 * np, k0, lane));
                     mma(accS[2 * np], ak, bu[0], bu[1]);
                     mma(accS[2 * np + 1], ak, bu[2], bu[3]);
                 }
             }
 #pragma unroll
             for (int j = 0; j < NJS; ++j) {
-                const int c = 8 * j + 2 * t4;
+                const int c = cs0 + 8 * j + 2 * t4;
                 st_h2(sS + r0 * LDD + c, accS[j][0], accS[j][1]);
                 st_h2(sS + (r0 + 8) * LDD + c, accS[j][2], accS[j][3]);
             }
@@ -685,10 +703,10 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 
     if (a.hT) {
         float *hp = a.hT + (size_t)bh * D * D + dv0;
-        const int r0 = 16 * w + g;
+        const int r0 = rs0 + g;
 #pragma unroll
         for (int j = 0; j < NJS; ++j) {
-            const int c = 8 * j + 2 * t4;
+            const int c = cs0 + 8 * j + 2 * t4;
             *reinterpret_cast<float2 *>(hp + (size_t)r0 * D + c) = make_float2(accS[j][0], accS[j][1]);
             *reinterpret_cast<float2 *>(hp + (size_t)(r0 + 8) * D + c) = make_float2(accS[j][2], accS[j][3]);
         }
