@@ -336,6 +336,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         // (c, q) owns key channel c = tid % 128 and rows RPT q .. RPT q + RPT - 1.
         float Gv[GATE ? RPT : 1];
         float gm = 0.f, gcs = 0.f;   // GATE 1: G at row 31 and at row 63 of channel c
+        bool bad = false;            // GATE 1: a factor left the fp16 range
         const int ch_c = tid & (D - 1), ch_h = tid >> 7;
         if (GATE == 0) {
             if (w == 0) {   // G, exp(G), exp(G_C - G)
@@ -395,7 +396,6 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             // Gram operands about the reference row 31: rows of K and Q scaled by
             // exp(G_r - G_31), columns of K by exp(G_31 - G_i). Each factor spans at
             // most 32 tokens of decay; a product over a pair i <= r is exp(G_r - G_i).
-            bool bad = false;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const int row = RPT * ch_h + r;
@@ -408,9 +408,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 sQ[row * LDD + ch_c] = __float2half_rn(qr);
                 sW[row * LDD + ch_c] = __float2half_rn(kc);
             }
-            if (bad) atomicAdd(&g_fused_range_errors, 1u);
         }
-        __syncthreads();
+        if (__syncthreads_or(bad) && tid == 0 && split == 0)   // once per (unit, chunk)
+            atomicAdd(&g_fused_range_errors, 1u);
 
         // ---------------- Gram: warps 0-3 rows of K, warps 4-7 rows of Q, against the
         // 64 key rows (GATE 1: the scaled row and column operands)

@@ -127,6 +127,28 @@ def test_bad_workspace_raises():
     assert ei.value.status == gdr.GDR_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_one_cta_per_unit_when_units_fill_the_sms(gate):
+    """80 (batch row, value head) units: too many to split the value columns over two CTAs
+    per unit in one wave, so each unit gets one CTA (the small cases above get two)."""
+    w = WORKLOADS["gdn_bf16"].with_(B=5, T=130, Hk=16, Hv=16, gate=gate,
+                                    g_mu=4.0 if gate == "channel" else 3.0, seed=21)
+    full_check(w)
+
+
+def test_strong_channel_decay_is_reported_not_hidden():
+    """A per-channel decay of exp(-1) per token spans exp(-32) over half a chunk: the fused
+    kernel's fp16 factors overflow, and it says so in gdr_fused_error_counts."""
+    w = WORKLOADS["kda_bf16"].with_(B=1, T=64, Hk=1, Hv=1, seed=22)
+    inp = make_inputs(w, DEV)
+    inp["g"] = torch.full_like(inp["g"], -1.0)
+    _, before = gdr.gdr_fused_error_counts()
+    run_fwd(inp)
+    torch.cuda.synchronize()
+    _, after = gdr.gdr_fused_error_counts()
+    assert after == before + 1
+
+
 # ------------------------------------------------------------------ full-size workloads
 @pytest.mark.parametrize("name,n_units", [("gdn_bf16", 6), ("gva_gdn_bf16", 6), ("kda_bf16", 3)])
 def test_full_workload_sampled(name, n_units):
@@ -206,3 +228,10 @@ def test_decode_equals_chunked_forward():
     torch.cuda.synchronize()
     assert rel_err(sw(o_d), o_c.double().cpu().numpy()) <= TOL["bf16"]
     assert rel_err(s_d, s_c.double().cpu().numpy()) <= TOL["bf16"]
+
+
+def test_zz_fused_kernel_reported_no_load_timeouts():
+    """Runs after the other tests in this file: no chunk load ever timed out."""
+    torch.cuda.synchronize()
+    timeouts, _ = gdr.gdr_fused_error_counts()
+    assert timeouts == 0
