@@ -8,7 +8,8 @@ there is no CPU fallback. If libgdr.so is missing the first call raises.
 
 Layouts (row-major, contiguous): q,k [B,T,Hk,Dk]; v,o [B,T,Hv,Dv]; g [B,T,Hv]
 (scalar gate) or [B,T,Hv,Dk] (per-channel gate) in fp32; beta [B,T,Hv] fp32;
-h0, hT, state [B,Hv,Dk,Dv] fp32. Decode drops the T axis.
+h0, hT, state [B,Hv,Dk,Dv] fp32. Decode drops the T axis; packed sequences
+(gdr_fwd_chunked_varlen) drop the B axis and add cu_seqlens.
 """
 import ctypes
 import os
@@ -24,7 +25,8 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
-           "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts")
+           "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts",
+           "gdr_fwd_chunked_varlen")
 
 # Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
 GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -61,6 +63,10 @@ def lib():
         L.gdr_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [i] * 7 + [vp]
         L.gdr_fwd_chunked_noalloc.restype = i
         L.gdr_fwd_chunked_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp] + [i] * 8 + [vp]
+        L.gdr_fwd_chunked_varlen.restype = i
+        L.gdr_fwd_chunked_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp] + [i] * 8 + [vp]
+        L.gdr_fused_error_counts.restype = ctypes.c_uint
+        L.gdr_fused_error_counts.argtypes = [vp, vp]
         _lib = L
     return _lib
 
@@ -156,6 +162,39 @@ def gdr_fwd_chunked(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True,
     _check(lib().gdr_fwd_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
                                  _ptr(hT), B, T, Hk, Hv, Dk, Dv, gate_mode, dt, _ptr(workspace),
                                  ws_bytes, _stream(stream)))
+    return o, hT
+
+
+def gdr_fwd_chunked_varlen(q, k, v, g, beta, cu_seqlens, h0=None, *, o=None, hT=None, want_hT=True,
+                           stream=None, out_dtype=None):
+    """Chunked forward over packed sequences: q, k [T_total, Hk, Dk], v [T_total, Hv, Dv],
+    g [T_total, Hv] or [T_total, Hv, Dk], beta [T_total, Hv], cu_seqlens int32 [N + 1] on the
+    device. Returns (o [T_total, Hv, Dv], hT [N, Hv, Dk, Dv] or None)."""
+    T_total, Hk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    N = cu_seqlens.numel() - 1
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt, odt = _dtype_code(q, out_dtype)
+    gate_mode = GDR_GATE_CHANNEL if g.dim() == 3 else GDR_GATE_SCALAR
+    _need(q, "q", q.dtype)
+    _need(k, "k", q.dtype, q.shape)
+    _need(v, "v", q.dtype, (T_total, Hv, Dv))
+    _need(g, "g", torch.float32, (T_total, Hv) if gate_mode == 0 else (T_total, Hv, Dk))
+    _need(beta, "beta", torch.float32, (T_total, Hv))
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (N, Hv, Dk, Dv))
+    if o is None:
+        o = torch.empty((T_total, Hv, Dv), dtype=odt, device=q.device)
+    _need(o, "o", odt, (T_total, Hv, Dv))
+    if hT is None and want_hT:
+        hT = torch.empty((N, Hv, Dk, Dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _need(hT, "hT", torch.float32, (N, Hv, Dk, Dv))
+    _check(lib().gdr_fwd_chunked_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+                                        _ptr(hT), _ptr(cu_seqlens), N, T_total, Hk, Hv, Dk, Dv, gate_mode, dt,
+                                        _stream(stream)))
     return o, hT
 
 

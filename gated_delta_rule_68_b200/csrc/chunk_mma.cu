@@ -269,7 +269,16 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     const uint32_t aXw = smem_u32(sXw);
     const int split = blockIdx.x % NS, bh = blockIdx.x / NS, dv0 = split * DVC;
     const int b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
-    const int T = a.T, NC = (T + C - 1) / C;
+    // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
+    // maps, batch index tb and token offset tt0. Packed input: sequence b of cu_seqlens
+    // (clamped into the token axis), with rows past its end masked below.
+    int T = a.T, tb = b, tt0 = 0;
+    long tok0 = (long)b * a.T;
+    if (a.cu_seqlens) {
+        const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
+        T = s1 - s0, tb = 0, tt0 = s0, tok0 = s0;
+    }
+    const int NC = (T + C - 1) / C;
 
     // Row block (16 rows) and column block of this warp in the [64 x DVC] products,
     // and in the [128 x DVC] state.
@@ -307,14 +316,14 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         const int t0 = c * C, n = min(C, T - t0);
         if (tid == 0) {
             mbar_expect_tx(aBar, (2u * C * D + C * DVC) * 2);
-            tma_load_4d(aStg, &map_k, 0, hk, t0, b, aBar);
-            tma_load_4d(aStg + C * D * 2, &map_q, 0, hk, t0, b, aBar);
-            tma_load_4d(aStg + 2 * C * D * 2, &map_v, dv0, h, t0, b, aBar);
+            tma_load_4d(aStg, &map_k, 0, hk, tt0 + t0, tb, aBar);
+            tma_load_4d(aStg + C * D * 2, &map_q, 0, hk, tt0 + t0, tb, aBar);
+            tma_load_4d(aStg + 2 * C * D * 2, &map_v, dv0, h, tt0 + t0, tb, aBar);
         }
         if (tid < 2 * C && (GATE == 0 || tid >= C)) {
             const int r = tid & (C - 1);
             const float *src = tid < C ? a.g : a.beta;
-            if (r < n) src += ((long)b * T + t0 + r) * a.Hv + h;
+            if (r < n) src += (tok0 + t0 + r) * a.Hv + h;
             cp_async4(aGst + tid * 4, src, r < n ? 4u : 0u);
         }
         cp_async_commit();
@@ -368,10 +377,11 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 #pragma unroll 4
             for (int idx = tid; idx < 2 * C * 16; idx += NT) {   // K and Q as they are
                 const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
-                *reinterpret_cast<uint4 *>((which ? sQ : sK) + r * LDD + c16 * 8) = bf16x8_to_f16x8(sStg[idx]);
+                *reinterpret_cast<uint4 *>((which ? sQ : sK) + r * LDD + c16 * 8) =
+                    r < n ? bf16x8_to_f16x8(sStg[idx]) : make_uint4(0, 0, 0, 0);
             }
         } else {
-            const float *gp = a.g + (((long)b * T + t0 + RPT * ch_h) * a.Hv + h) * D + ch_c;
+            const float *gp = a.g + ((tok0 + t0 + RPT * ch_h) * a.Hv + h) * D + ch_c;
             const long gstride = (long)a.Hv * D;
             float s = 0.f;
 #pragma unroll
@@ -400,8 +410,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             for (int r = 0; r < RPT; ++r) {
                 const int row = RPT * ch_h + r;
                 const float f1 = __expf(Gv[r] - gm), f2 = __expf(gm - Gv[r]);
-                const float kv = __bfloat162float(sStgH[row * D + ch_c]);
-                const float qv = __bfloat162float(sStgH[C * D + row * D + ch_c]);
+                const float kv = row < n ? __bfloat162float(sStgH[row * D + ch_c]) : 0.f;
+                const float qv = row < n ? __bfloat162float(sStgH[C * D + row * D + ch_c]) : 0.f;
                 const float kr = kv * f1, qr = qv * f1, kc = kv * f2;
                 bad |= fabsf(kr) > 65504.f || fabsf(qr) > 65504.f || fabsf(kc) > 65504.f;
                 sK[row * LDD + ch_c] = __float2half_rn(kr);
@@ -465,8 +475,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             for (int r = 0; r < RPT; ++r) {
                 const int row = RPT * ch_h + r;
                 const float e1 = __expf(Gv[r]), e2 = __expf(gcs - Gv[r]);
-                const float kv = __bfloat162float(sStgH[row * D + ch_c]);
-                const float qv = __bfloat162float(sStgH[C * D + row * D + ch_c]);
+                const float kv = row < n ? __bfloat162float(sStgH[row * D + ch_c]) : 0.f;
+                const float qv = row < n ? __bfloat162float(sStgH[C * D + row * D + ch_c]) : 0.f;
                 sK[row * LDD + ch_c] = __float2half_rn(kv * e1);
                 sQ[row * LDD + ch_c] = __float2half_rn(qv * e1);
                 sUE[row * LDD + ch_c] = __float2half_rn(kv * e2);
@@ -513,7 +523,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
             for (int idx = tid - 64; idx < C * (DVC / 8); idx += NT - 64) {   // this CTA's V columns
                 const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
-                *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) = bf16x8_to_f16x8(sStg[2 * C * 16 + idx]);
+                *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) =
+                    r < n ? bf16x8_to_f16x8(sStg[2 * C * 16 + idx]) : make_uint4(0, 0, 0, 0);
             }
         }
         __syncthreads();
@@ -697,7 +708,15 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
         }
         __syncthreads();
-        if (tid == 0) tma_store_4d(&map_o, dv0, h, t0, b, smem_u32(sm + OFF_V));
+        if (a.cu_seqlens == nullptr || n == C) {
+            if (tid == 0) tma_store_4d(&map_o, dv0, h, tt0 + t0, tb, smem_u32(sm + OFF_V));
+        } else {   // the rows after a packed sequence's end belong to the next sequence
+            const TOut *so = reinterpret_cast<const TOut *>(sm + OFF_V);
+            TOut *op = reinterpret_cast<TOut *>(a.o) + ((tok0 + t0) * a.Hv + h) * D + dv0;
+            for (int idx = tid; idx < n * DVC; idx += NT)
+                op[(long)(idx / DVC) * a.Hv * D + idx % DVC] = so[idx];
+            __syncthreads();
+        }
     }
     if (tid == 0) tma_store_wait_all();
 
@@ -761,9 +780,10 @@ template <typename TOut, int GATE, int NS>
 cudaError_t launch_t(const FwdArgs &a, cudaStream_t st)
 {
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, a.q, a.B, a.T, a.Hk, D) || !make_map(&mk, a.k, a.B, a.T, a.Hk, D) ||
-        !make_map(&mv, a.v, a.B, a.T, a.Hv, D / NS) ||
-        !make_map(&mo, a.o, a.B, a.T, a.Hv, D / NS, sizeof(TOut) == 4))
+    const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
+    if (!make_map(&mq, a.q, mb, a.T, a.Hk, D) || !make_map(&mk, a.k, mb, a.T, a.Hk, D) ||
+        !make_map(&mv, a.v, mb, a.T, a.Hv, D / NS) ||
+        !make_map(&mo, a.o, mb, a.T, a.Hv, D / NS, sizeof(TOut) == 4))
         return cudaErrorInvalidValue;
     const int smem = SMEM_BYTES + 128;
     auto kernel = fused_fwd_kernel<TOut, GATE, NS>;

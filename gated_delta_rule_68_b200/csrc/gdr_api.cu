@@ -134,6 +134,45 @@ int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
     return GDR_OK;
 }
 
+int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                           const float *h0, void *o, float *hT, const int *cu_seqlens, int N, int T_total, int Hk,
+                           int Hv, int Dk, int Dv, int gate_mode, int dtype, void *stream)
+{
+    int st = check_common(N, T_total, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (st != GDR_OK) return st;
+    if (N > 0 && !cu_seqlens) return fail(GDR_ERR_INVALID_ARG, "cu_seqlens must be non-NULL");
+    if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return fail(GDR_ERR_MISALIGNED, "cu_seqlens is not 4-byte aligned");
+    const bool work = N > 0 && T_total > 0;
+    if (work && (!q || !k || !v || !g || !beta || !o))
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta and o must be non-NULL");
+    const void *ptrs[] = {q, k, v, g, beta, h0, o, hT};
+    const char *names[] = {"q", "k", "v", "g", "beta", "h0", "o", "hT"};
+    for (int i = 0; i < 8; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if (o && (o == q || o == k || o == v))
+        return fail(GDR_ERR_INVALID_ARG, "o must not alias q, k or v");
+    gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, N, T_total, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    a.cu_seqlens = cu_seqlens;
+    if (!gdr::fused_supported(a))
+        return fail(GDR_ERR_UNSUPPORTED, "packed sequences need bf16 inputs and Dk = Dv = 128");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!work) {
+        if (hT && N > 0) {
+            const size_t bytes = (size_t)N * Hv * Dk * Dv * sizeof(float);
+            cudaError_t e = h0 ? (h0 == hT ? cudaSuccess
+                                           : cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, s))
+                               : cudaMemsetAsync(hT, 0, bytes, s);
+            if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA: %s", cudaGetErrorString(e));
+        }
+        return GDR_OK;
+    }
+    cudaError_t e = gdr::launch_fwd_fused(a, s);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += 1;
+    return GDR_OK;
+}
+
 int gdr_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
                     float *state, void *o, int B, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype,
                     void *stream)

@@ -23,6 +23,9 @@ struct FwdArgs {
     void *o;
     float *hT;
     int B, T, Hk, Hv, Dk, Dv, gate_mode, dtype;
+    // Packed variable-length input (fused kernel only): B sequences packed along one
+    // token axis of length T; sequence n is tokens [cu_seqlens[n], cu_seqlens[n + 1]).
+    const int *cu_seqlens = nullptr;
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);

@@ -121,8 +121,10 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  * U' = U - W S, S <- diag(Gamma_C) S + (K*Gamma_C/Gamma)^T U', and the output
  * O = (Q*Gamma) S + tril((Q*Gamma)(K/Gamma)^T) U'.
  *
- * bf16 inputs run on the tcgen05 tensor cores with fp32 accumulation and an
- * fp32 carried state; fp32 inputs run in fp32 throughout.
+ * bf16 inputs with Dk = Dv = 128 run one fused kernel on the warp-level
+ * tensor cores (fp16 operands, fp32 accumulation, fp32 carried state; q, k,
+ * v and the state must stay inside the fp16 range, |x| < 6.5e4). Other
+ * shapes and fp32 inputs run fp32 CUDA-core kernels.
  * B == 0 or T == 0 is a valid no-op that still writes hT = h0 (or zeros).
  *
  * workspace: device buffer of at least gdr_fwd_workspace_size(...) bytes,
@@ -135,6 +137,31 @@ GDR_API int gdr_fwd_chunked(const void *q, const void *k, const void *v, const f
                     int B, int T, int Hk, int Hv, int Dk, int Dv,
                     int gate_mode, int dtype,
                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Chunked forward over packed sequences of different lengths (no counterpart
+ * on the source pages beyond their remark that the recurrent state is reset at
+ * each packed row).
+ *
+ * N sequences are packed along one token axis of T_total tokens: sequence n
+ * is tokens [cu_seqlens[n], cu_seqlens[n+1]) and starts from h0[n] (or zeros),
+ * its final state goes to hT[n]. Layouts: q, k [T_total, Hk, Dk]; v, o
+ * [T_total, Hv, Dv]; g [T_total, Hv] or [T_total, Hv, Dk]; beta [T_total, Hv];
+ * h0, hT [N, Hv, Dk, Dv] fp32. cu_seqlens: device int32 [N + 1], non-decreasing,
+ * cu_seqlens[0] = 0, cu_seqlens[N] = T_total (values are clamped into
+ * [0, T_total], so a malformed array yields wrong results, never an
+ * out-of-bounds access). Each sequence equals a gdr_fwd_chunked call on it
+ * alone, bit for bit.
+ *
+ * Runs only on the fused kernel: bf16 inputs (dtype GDR_BF16 or
+ * GDR_BF16_OUT_F32) with Dk = Dv = 128; anything else returns
+ * GDR_ERR_UNSUPPORTED. Needs no workspace. Pointers 16-byte aligned (cu_seqlens
+ * 4-byte aligned); o must not alias q, k or v.
+ */
+GDR_API int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *h0, void *o, float *hT,
+                           const int *cu_seqlens, int N, int T_total, int Hk, int Hv, int Dk, int Dv,
+                           int gate_mode, int dtype, void *stream);
 
 /*
  * One decode step for B independent sequences (the recurrence with T = 1):
