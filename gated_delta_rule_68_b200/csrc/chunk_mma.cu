@@ -77,8 +77,8 @@ constexpr int OFF_AH = OFF_X + 8 * 16 * LDX * 2;// fp16 A [64][72]
 static_assert(C * LDF * 4 <= SZ_D, "A must fit in the U' tile");
 static_assert(C * LDC * 2 <= SZ_D, "T must fit in the diag(e) U' tile");
 static_assert(8 * 16 * LDX * 2 + C * LDC * 2 <= SZ_D, "block-row products and A must fit in the W tile");
-static_assert(SMEM_BYTES + 128 <= 227 * 1024, "shared memory");
-static_assert(OFF_STG % 128 == 0 && OFF_V % 128 == 0, "TMA shared-memory alignment");
+static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory");
+static_assert(OFF_STG % 128 == 0 && OFF_V % 1024 == 0, "TMA shared-memory alignment (1024 B for the swizzled o tile)");
 static_assert(C * D * 4 <= 2 * SZ_D, "an fp32 o tile must fit in the V and W tiles");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -203,6 +203,16 @@ __device__ __forceinline__ void store_out2(__nv_bfloat16 *p, float x, float y)
     *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(x, y);
 }
 
+// Byte offset of element (r, c) of an o tile held as 128-byte-wide boxes of 64
+// rows in the TMA 128-byte swizzle (16-byte chunk j of row r sits at j ^ (r % 8)).
+template <typename TOut>
+__device__ __forceinline__ int o_swz(int r, int c)
+{
+    constexpr int EPB = 128 / sizeof(TOut);
+    const int byte = (c % EPB) * (int)sizeof(TOut);
+    return (c / EPB) * C * 128 + r * 128 + ((((byte >> 4) ^ (r & 7))) << 4) + (byte & 15);
+}
+
 // 8 bf16 -> 8 fp16 in one 16-byte word.
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u)
 {
@@ -238,8 +248,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     constexpr int NJG = C / NCS / 8;    // n8 tiles of a warp in the Gram [128 x 64]
     constexpr int RPT = C / NQ;         // GATE 1: rows per thread in the per-channel pass
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    // 128-byte aligned base: the TMA destination tiles need it.
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    // 1024-byte aligned base: the TMA tiles need 128 B, the swizzled o tile 1024 B.
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __half *sK = reinterpret_cast<__half *>(sm + OFF_K), *sQ = reinterpret_cast<__half *>(sm + OFF_Q);
     __half *sV = reinterpret_cast<__half *>(sm + OFF_V), *sW = reinterpret_cast<__half *>(sm + OFF_W);
     __half *sU = reinterpret_cast<__half *>(sm + OFF_U), *sUE = reinterpret_cast<__half *>(sm + OFF_UE);
@@ -667,13 +677,14 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 mma(accO[2 * np + 1], am, bu[2], bu[3]);
             }
         }
-        {   // o rows -> a dense [64][DVC] tile over the dead V and W tiles -> one TMA store
-            TOut *so = reinterpret_cast<TOut *>(sm + OFF_V) + cw0 + 2 * t4;
+        {   // o rows -> [DVC / EPB][64 rows][128 B] boxes in the 128-byte swizzle the TMA
+            // store expects, over the dead V and W tiles
             const int r0 = rw0 + g, r1 = rw0 + g + 8;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                store_out2(so + r0 * DVC + 8 * j, accO[j][0], accO[j][1]);
-                store_out2(so + r1 * DVC + 8 * j, accO[j][2], accO[j][3]);
+                const int c = cw0 + 8 * j + 2 * t4;
+                store_out2(reinterpret_cast<TOut *>(sm + OFF_V + o_swz<TOut>(r0, c)), accO[j][0], accO[j][1]);
+                store_out2(reinterpret_cast<TOut *>(sm + OFF_V + o_swz<TOut>(r1, c)), accO[j][2], accO[j][3]);
             }
             fence_proxy_async();
         }
@@ -709,12 +720,18 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         }
         __syncthreads();
         if (a.cu_seqlens == nullptr || n == C) {
-            if (tid == 0) tma_store_4d(&map_o, dv0, h, tt0 + t0, tb, smem_u32(sm + OFF_V));
+            if (tid == 0) {
+                constexpr int EPB = 128 / sizeof(TOut);   // elements per 128-byte box row
+#pragma unroll
+                for (int bx = 0; bx < DVC / EPB; ++bx)
+                    tma_store_4d(&map_o, dv0 + bx * EPB, h, tt0 + t0, tb, smem_u32(sm + OFF_V + bx * C * 128));
+            }
         } else {   // the rows after a packed sequence's end belong to the next sequence
-            const TOut *so = reinterpret_cast<const TOut *>(sm + OFF_V);
             TOut *op = reinterpret_cast<TOut *>(a.o) + ((tok0 + t0) * a.Hv + h) * D + dv0;
-            for (int idx = tid; idx < n * DVC; idx += NT)
-                op[(long)(idx / DVC) * a.Hv * D + idx % DVC] = so[idx];
+            for (int idx = tid; idx < n * DVC; idx += NT) {
+                const int r = idx / DVC, c = idx % DVC;
+                op[(long)r * a.Hv * D + c] = *reinterpret_cast<const TOut *>(sm + OFF_V + o_swz<TOut>(r, c));
+            }
             __syncthreads();
         }
     }
@@ -753,7 +770,8 @@ EncodeTiledFn encode_tiled()
 // Tensor map of a [B][T][H][128] bf16 (or fp32) tensor for boxes of `cols` channels of 64
 // consecutive tokens of one head: dims (d, head, t, b), box (cols, 1, 64, 1).
 // Tokens past T read as zero.
-bool make_map(CUtensorMap *map, const void *base, int B, int T, int H, int cols, bool f32 = false)
+bool make_map(CUtensorMap *map, const void *base, int B, int T, int H, int cols, bool f32 = false,
+              bool swizzle128 = false)
 {
     const cuuint64_t es = f32 ? 4 : 2;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -763,7 +781,8 @@ bool make_map(CUtensorMap *map, const void *base, int B, int T, int H, int cols,
     const EncodeTiledFn encode = encode_tiled();
     return encode && encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                             const_cast<void *>(base), dims, strides, box,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -783,9 +802,9 @@ cudaError_t launch_t(const FwdArgs &a, cudaStream_t st)
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
     if (!make_map(&mq, a.q, mb, a.T, a.Hk, D) || !make_map(&mk, a.k, mb, a.T, a.Hk, D) ||
         !make_map(&mv, a.v, mb, a.T, a.Hv, D / NS) ||
-        !make_map(&mo, a.o, mb, a.T, a.Hv, D / NS, sizeof(TOut) == 4))
+        !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
         return cudaErrorInvalidValue;
-    const int smem = SMEM_BYTES + 128;
+    const int smem = SMEM_BYTES + 1024;
     auto kernel = fused_fwd_kernel<TOut, GATE, NS>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
