@@ -339,6 +339,19 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         cp_async_commit();
     };
     if (NC > 0) issue_loads(0);
+    // GATE 1: this thread's per-channel gates of the next chunk, loaded into registers
+    // a chunk ahead so their latency hides behind the current chunk's work.
+    float gnext[GATE ? RPT : 1];
+    auto load_gates = [&](int c) {
+        if (GATE) {
+            const int t0 = c * C, n = min(C, T - t0);
+            const float *gp = a.g + ((tok0 + t0 + RPT * (tid >> 7)) * a.Hv + h) * D + (tid & (D - 1));
+            const long gstride = (long)a.Hv * D;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) gnext[r] = (RPT * (tid >> 7) + r < n) ? __ldg(gp + r * gstride) : 0.f;
+        }
+    };
+    if (NC > 0) load_gates(0);
 
 #pragma unroll 1
     for (int ch = 0; ch < NC; ++ch) {
@@ -391,12 +404,10 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     r < n ? bf16x8_to_f16x8(sStg[idx]) : make_uint4(0, 0, 0, 0);
             }
         } else {
-            const float *gp = a.g + ((tok0 + t0 + RPT * ch_h) * a.Hv + h) * D + ch_c;
-            const long gstride = (long)a.Hv * D;
             float s = 0.f;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                s += (RPT * ch_h + r < n) ? __ldg(gp + r * gstride) : 0.f;
+                s += gnext[r];
                 Gv[r] = s;
             }
             sTot[ch_h * D + ch_c] = s;
@@ -538,7 +549,10 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
         }
         __syncthreads();
-        if (ch + 1 < NC) issue_loads(ch + 1);   // the staging area has been consumed
+        if (ch + 1 < NC) {
+            issue_loads(ch + 1);   // the staging area has been consumed
+            load_gates(ch + 1);
+        }
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {
             if (w < bi) {
