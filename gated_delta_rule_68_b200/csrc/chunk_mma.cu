@@ -488,6 +488,52 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     }
                 }
             }
+            if (krow) {
+                // T = (I + A)^-1, its 16x16 diagonal block: the warp that holds that block of
+                // A solves it by forward substitution in fp32 (lane = column of the block)
+                const int rb = rw0 >> 4;
+                if (rb >= (cg0 >> 4) && rb < (cg0 >> 4) + NJG / 2) {
+                    __syncwarp();
+                    if (lane < 16) {
+                        const int base = 16 * rb, col = lane;
+                        float tv[16];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) {
+                            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                            for (int i = 0; i < r; i += 2) {
+                                s0 += sA[(base + r) * LDF + base + i] * tv[i];
+                                if (i + 1 < r) s1 += sA[(base + r) * LDF + base + i + 1] * tv[i + 1];
+                            }
+                            tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -(s0 + s1));
+                        }
+                        const float bc = sBeta[base + col], bgc = GATE ? 0.f : bc * sEg[base + col];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) {
+                            const int o = (base + r) * LDC + base + col;
+                            sTh[o] = __float2half_rn(tv[r]);
+                            sTB[o] = __float2half_rn(tv[r] * bc);
+                            if (GATE == 0) sTG[o] = __float2half_rn(tv[r] * bgc);
+                        }
+                    }
+                }
+            } else {
+                // the Q-row warps: zeros in the six blocks above the diagonal of T diag(beta)
+                // (and T diag(beta Gamma)), and this CTA's V columns to fp16
+                const int li = ((w >> 3) * 4 + (w & 7) - 4) * 32 + lane, nli = NT / 2;
+                if (li < 6 * 32) {
+                    const int blk = li >> 5, row = (li >> 1) & 15, hf = li & 1;
+                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                    const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
+                    *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
+                    if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
+                }
+                for (int idx = li; idx < C * (DVC / 8); idx += nli) {
+                    const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
+                    *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) =
+                        r < n ? bf16x8_to_f16x8(sStg[2 * C * 16 + idx]) : make_uint4(0, 0, 0, 0);
+                }
+            }
         }
         if (GATE) {
             // K diag(Gamma) (for W), Q diag(Gamma) (for O) and K diag(Gamma_C / Gamma)
@@ -506,49 +552,10 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         __syncthreads();
 
         // ---------------- T = (I + A)^-1 (entries above the diagonal are never
-        // written and read as zero). The 16x16 diagonal blocks by forward
-        // substitution in fp32; then block rows bi = 1..3 on tensor cores, one
-        // warp per block (bi, bj):
+        // written and read as zero): the diagonal blocks came with the Gram
+        // epilogue; block rows bi = 1..3 on tensor cores, one warp per block (bi, bj):
         //   X = sum_{m=bj}^{bi-1} A_{bi,m} T_{m,bj},   T_{bi,bj} = -T_{bi,bi} X
         // The producers also write T diag(beta) and (GATE 0) T diag(beta Gamma).
-        if (tid < 64) {
-            const int base = (tid >> 4) * 16, col = tid & 15;
-            float tv[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                for (int i = 0; i < r; i += 2) {
-                    s0 += sA[(base + r) * LDF + base + i] * tv[i];
-                    if (i + 1 < r) s1 += sA[(base + r) * LDF + base + i + 1] * tv[i + 1];
-                }
-                tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -(s0 + s1));
-            }
-            const float bc = sBeta[base + col], bgc = GATE ? 0.f : bc * sEg[base + col];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int o = (base + r) * LDC + base + col;
-                sTh[o] = __float2half_rn(tv[r]);
-                sTB[o] = __float2half_rn(tv[r] * bc);
-                if (GATE == 0) sTG[o] = __float2half_rn(tv[r] * bgc);
-            }
-        } else {
-            // zeros in the six blocks above the diagonal of T diag(beta) (and T diag(beta Gamma))
-            const int e = tid - 64;
-            if (e < 6 * 32) {
-                const int blk = e >> 5, row = (e >> 1) & 15, hf = e & 1;
-                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
-                *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
-                if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
-            }
-            for (int idx = tid - 64; idx < C * (DVC / 8); idx += NT - 64) {   // this CTA's V columns
-                const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
-                *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) =
-                    r < n ? bf16x8_to_f16x8(sStg[2 * C * 16 + idx]) : make_uint4(0, 0, 0, 0);
-            }
-        }
-        __syncthreads();
         if (ch + 1 < NC) {
             issue_loads(ch + 1);   // the staging area has been consumed
             load_gates(ch + 1);
