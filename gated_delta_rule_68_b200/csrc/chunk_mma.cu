@@ -33,23 +33,20 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mma_util.cuh"
 
 namespace gdr {
 namespace {
 
-constexpr int C = 64;
-constexpr int D = 128;
+using namespace mmau;
+
 constexpr int NW = 16;           // warps per CTA
 constexpr int NT = 32 * NW;
 constexpr int NCB = NW / 4;      // column blocks of the [64 x n] products (4 row blocks of 16)
 constexpr int NCS = NW / 8;      // column blocks of the [128 x n] products (8 row blocks of 16)
 constexpr int NQ = NT / 128;     // row groups of the per-channel gate pass (one thread per channel and group)
-constexpr int LDD = D + 8;       // fp16 row stride of 128-wide tiles (272 B: ldmatrix rows hit distinct banks)
-constexpr int LDC = C + 8;       // fp16 row stride of 64-wide tiles (144 B)
-constexpr int LDF = C + 1;       // fp32 row stride of the 64 x 64 scratch
 
 // Shared-memory layout (bytes).
-constexpr int SZ_D = C * LDD * 2;               // one [64][128] fp16 tile
 constexpr int OFF_K = 0;                        // K [i][dk]
 constexpr int OFF_Q = OFF_K + SZ_D;             // Q [r][dk]
 constexpr int OFF_V = OFF_Q + SZ_D;             // V [i][dv]
@@ -57,7 +54,6 @@ constexpr int OFF_W = OFF_V + SZ_D;             // -W [r][dk]
 constexpr int OFF_U = OFF_W + SZ_D;             // U' [i][dv]
 constexpr int OFF_UE = OFF_U + SZ_D;            // diag(e) U' [i][dv]
 constexpr int OFF_S = OFF_UE + SZ_D;            // S [dk][dv] fp16 copy of the state
-constexpr int SZ_C = C * LDC * 2;               // one [64][64] fp16 tile
 constexpr int OFF_M = OFF_S + D * LDD * 2;      // M [r][i]
 constexpr int OFF_TB = OFF_M + SZ_C;            // T diag(beta) [r][i]
 constexpr int OFF_TG = OFF_TB + SZ_C;           // T diag(beta Gamma) [r][i]
@@ -71,7 +67,6 @@ constexpr int SMEM_BYTES = OFF_VEC + (256 + NQ * 128) * 4;
 // 16 x 16 block-row product in the -W tile.
 constexpr int OFF_A = OFF_U;                    // fp32 A [64][65]
 constexpr int OFF_TH = OFF_UE;                  // fp16 T [64][72]
-constexpr int LDX = 24;                         // fp16 row stride of a warp's 16 x 16 product
 constexpr int OFF_X = OFF_W;                    // fp16 [8 warps][16][24]
 constexpr int OFF_AH = OFF_X + 8 * 16 * LDX * 2;// fp16 A [64][72]
 static_assert(C * LDF * 4 <= SZ_D, "A must fit in the U' tile");
@@ -80,153 +75,6 @@ static_assert(8 * 16 * LDX * 2 + C * LDC * 2 <= SZ_D, "block-row products and A 
 static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory");
 static_assert(OFF_STG % 128 == 0 && OFF_V % 1024 == 0, "TMA shared-memory alignment (1024 B for the swizzled o tile)");
 static_assert(C * D * 4 <= 2 * SZ_D, "an fp32 o tile must fit in the V and W tiles");
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void ldsm(uint32_t r[4], uint32_t addr)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
-}
-__device__ __forceinline__ void ldsm_t(uint32_t r[4], uint32_t addr)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
-}
-// c (16x8, fp32) += a (16x16, fp16, row) * b (16x8, fp16, col)
-__device__ __forceinline__ void mma(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Fragment addresses for ldmatrix.x4 (lane supplies one row address).
-// A tile (16 x 16) at rows r0.., cols k0.. of a row-major tile.
-__device__ __forceinline__ uint32_t a_rm(uint32_t base, int ld, int r0, int k0, int lane)
-{
-    return base + ((r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * ld + k0 + (lane >> 4) * 8) * 2;
-}
-// A tile (16 x 16) whose element (m, k) is St[k0 + k][m0 + m] of a row-major St (load with .trans).
-__device__ __forceinline__ uint32_t a_tr(uint32_t base, int ld, int m0, int k0, int lane)
-{
-    return base + ((k0 + (lane & 7) + (lane >> 4) * 8) * ld + m0 + ((lane >> 3) & 1) * 8) * 2;
-}
-// B tiles for n0..n0+15 (two n8 tiles) and k0..k0+15 of a tile stored [n][k] (plain load).
-__device__ __forceinline__ uint32_t b_nk(uint32_t base, int ld, int n0, int k0, int lane)
-{
-    return base + ((n0 + (lane & 7) + (lane >> 4) * 8) * ld + k0 + ((lane >> 3) & 1) * 8) * 2;
-}
-// B tiles for n0..n0+15 and k0..k0+15 of a tile stored [k][n] (load with .trans).
-__device__ __forceinline__ uint32_t b_kn(uint32_t base, int ld, int n0, int k0, int lane)
-{
-    return base + ((k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * ld + n0 + (lane >> 4) * 8) * 2;
-}
-
-// Asynchronous 4-byte global -> shared copy; bytes past src_bytes are filled with zeros.
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-// mbarrier-tracked bulk copies (whole rows, global -> shared) and a bounded wait.
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
-}
-// One 4-d box of a tensor map (TMA tiled load) into shared memory, completing on `bar`.
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
-                                            uint32_t bar)
-{
-    asm volatile("cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-                 "[%0], [%1, {%2, %3, %4, %5}], [%6];"
-                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-                 : "memory");
-}
-// One 4-d box from shared memory to a tensor (TMA tiled store); coordinates past
-// the tensor's end are not written. Completion is tracked per issuing thread.
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3, uint32_t src)
-{
-    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];"
-                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src) : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t done;
-    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}\n" : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-    return done != 0;
-}
-__device__ __forceinline__ uint64_t globaltimer_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-// Waits for phase `parity` of `bar` for at most one second; false if it gave up.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > 1000000000ull) return false;
-    return true;
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ void st_h2(__half *p, float x, float y)
-{
-    *reinterpret_cast<__half2 *>(p) = __floats2half2_rn(x, y);
-}
-
-__device__ __forceinline__ void store_out2(float *p, float x, float y)
-{
-    *reinterpret_cast<float2 *>(p) = make_float2(x, y);
-}
-__device__ __forceinline__ void store_out2(__nv_bfloat16 *p, float x, float y)
-{
-    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(x, y);
-}
-
-// Byte offset of element (r, c) of an o tile held as 128-byte-wide boxes of 64
-// rows in the TMA 128-byte swizzle (16-byte chunk j of row r sits at j ^ (r % 8)).
-template <typename TOut>
-__device__ __forceinline__ int o_swz(int r, int c)
-{
-    constexpr int EPB = 128 / sizeof(TOut);
-    const int byte = (c % EPB) * (int)sizeof(TOut);
-    return (c / EPB) * C * 128 + r * 128 + ((((byte >> 4) ^ (r & 7))) << 4) + (byte & 15);
-}
-
-// 8 bf16 -> 8 fp16 in one 16-byte word.
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u)
-{
-    const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&u);
-    uint4 r;
-    uint32_t *q = reinterpret_cast<uint32_t *>(&r);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(p[e]);
-        const __half2 hh = __floats2half2_rn(f.x, f.y);
-        q[e] = *reinterpret_cast<const uint32_t *>(&hh);
-    }
-    return r;
-}
 
 // Chunk loads that never completed (each abandons its CTA's remaining chunks), and
 // per-channel gate factors that left the fp16 range (their chunk's results are not valid).
