@@ -486,7 +486,7 @@ def main(argv=None):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded CPU generator; q,k L2-normalised N(0,1); v N(0,1); "
-                "g logsigmoid(N(3,1)); beta sigmoid(N(0,1)); h0 0.02 N(0,1))",
+                f"g logsigmoid(N({w.g_mu:g},1)); beta sigmoid(N(0,1)); h0 0.02 N(0,1))",
         "config": workload_config(w, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,

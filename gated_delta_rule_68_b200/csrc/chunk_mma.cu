@@ -91,7 +91,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 {
     constexpr int DVC = D / NS;      // value columns of this CTA
     constexpr int NJ = DVC / NCB / 8;   // n8 tiles of a warp in the [64 x DVC] products
-    constexpr int NJS = DVC / NCS / 8;  // n8 tiles of a warp's state rows
+    constexpr int NJS = DVC / 4 / 8;    // n8 tiles of a warp's state block (32 rows x DVC / 4)
     constexpr int NJW = D / NCB / 8;    // n8 tiles of a warp in W [64 x 128]
     constexpr int NJG = C / NCS / 8;    // n8 tiles of a warp in the Gram [128 x 64]
     constexpr int RPT = C / NQ;         // GATE 1: rows per thread in the per-channel pass
@@ -139,27 +139,31 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     const int NC = (T + C - 1) / C;
 
     // Row block (16 rows) and column block of this warp in the [64 x DVC] products,
-    // and in the [128 x DVC] state.
+    // and its 32 x DVC / 4 block of the [128 x DVC] state.
     const int rw0 = 16 * (w & 3), cw0 = (DVC / NCB) * (w >> 2);
-    const int rs0 = 16 * (w & 7), cs0 = (DVC / NCS) * (w >> 3);
+    const int rs0 = 32 * (w & 3), cs0 = (DVC / 4) * (w >> 2);
 
-    // State S[:, dv0 .. dv0 + DVC) in registers: warp w holds dk rows 16w..16w+15;
-    // n8 tile j holds local columns 8j..8j+7.
-    float accS[NJS][4];
+    // State S[:, dv0 .. dv0 + DVC) in registers: warp w holds dk rows rs0 .. rs0 + 31
+    // as two m16 tiles; n8 tile j holds local columns cs0 + 8j .. cs0 + 8j + 7.
+    float accS[2][NJS][4];
     {
         const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + dv0 : nullptr;
-        const int r0 = rs0 + g;
 #pragma unroll
-        for (int j = 0; j < NJS; ++j) {
-            const int c = cs0 + 8 * j + 2 * t4;
-            float2 x0 = make_float2(0.f, 0.f), x1 = x0;
-            if (h0) {
-                x0 = *reinterpret_cast<const float2 *>(h0 + (size_t)r0 * D + c);
-                x1 = *reinterpret_cast<const float2 *>(h0 + (size_t)(r0 + 8) * D + c);
+        for (int mt = 0; mt < 2; ++mt) {
+            const int r0 = rs0 + 16 * mt + g;
+#pragma unroll
+            for (int j = 0; j < NJS; ++j) {
+                const int c = cs0 + 8 * j + 2 * t4;
+                float2 x0 = make_float2(0.f, 0.f), x1 = x0;
+                if (h0) {
+                    x0 = *reinterpret_cast<const float2 *>(h0 + (size_t)r0 * D + c);
+                    x1 = *reinterpret_cast<const float2 *>(h0 + (size_t)(r0 + 8) * D + c);
+                }
+                float *x = accS[mt][j];
+                x[0] = x0.x; x[1] = x0.y; x[2] = x1.x; x[3] = x1.y;
+                st_h2(sS + r0 * LDD + c, x0.x, x0.y);
+                st_h2(sS + (r0 + 8) * LDD + c, x1.x, x1.y);
             }
-            accS[j][0] = x0.x; accS[j][1] = x0.y; accS[j][2] = x1.x; accS[j][3] = x1.y;
-            st_h2(sS + r0 * LDD + c, x0.x, x0.y);
-            st_h2(sS + (r0 + 8) * LDD + c, x1.x, x1.y);
         }
     }
 
@@ -301,16 +305,21 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             const bool krow = (w & 7) < 4;
             const int cg0 = (C / NCS) * (w >> 3);
             const uint32_t abase = krow ? aK : aQ, bbase = GATE ? aW : aK;
+            // Only key blocks at or left of the diagonal block are ever used (i <= r).
+            if (cg0 <= rw0) {
 #pragma unroll
-            for (int k0 = 0; k0 < D; k0 += 16) {
-                uint32_t af[4];
-                ldsm(af, a_rm(abase, LDD, rw0, k0, lane));
+                for (int k0 = 0; k0 < D; k0 += 16) {
+                    uint32_t af[4];
+                    ldsm(af, a_rm(abase, LDD, rw0, k0, lane));
 #pragma unroll
-                for (int np = 0; np < NJG / 2; ++np) {
-                    uint32_t bf[4];
-                    ldsm(bf, b_nk(bbase, LDD, cg0 + 16 * np, k0, lane));
-                    mma(acc[2 * np], af, bf[0], bf[1]);
-                    mma(acc[2 * np + 1], af, bf[2], bf[3]);
+                    for (int np = 0; np < NJG / 2; ++np) {
+                        if (cg0 + 16 * np <= rw0) {
+                            uint32_t bf[4];
+                            ldsm(bf, b_nk(bbase, LDD, cg0 + 16 * np, k0, lane));
+                            mma(acc[2 * np], af, bf[0], bf[1]);
+                            mma(acc[2 * np + 1], af, bf[2], bf[3]);
+                        }
+                    }
                 }
             }
             if (GATE) __syncthreads();   // the scaled tiles are rewritten below
@@ -366,16 +375,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     }
                 }
             } else {
-                // the Q-row warps: zeros in the six blocks above the diagonal of T diag(beta)
-                // (and T diag(beta Gamma)), and this CTA's V columns to fp16
+                // the Q-row warps: this CTA's V columns to fp16 (the blocks of T above
+                // its diagonal are never written: every product skips them)
                 const int li = ((w >> 3) * 4 + (w & 7) - 4) * 32 + lane, nli = NT / 2;
-                if (li < 6 * 32) {
-                    const int blk = li >> 5, row = (li >> 1) & 15, hf = li & 1;
-                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                    const int o = (16 * bi + row) * LDC + 16 * bj + 8 * hf;
-                    *reinterpret_cast<uint4 *>(sTB + o) = make_uint4(0, 0, 0, 0);
-                    if (GATE == 0) *reinterpret_cast<uint4 *>(sTG + o) = make_uint4(0, 0, 0, 0);
-                }
                 for (int idx = li; idx < C * (DVC / 8); idx += nli) {
                     const int r = idx / (DVC / 8), c8 = idx % (DVC / 8);
                     *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) =
@@ -399,8 +401,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         }
         __syncthreads();
 
-        // ---------------- T = (I + A)^-1 (entries above the diagonal are never
-        // written and read as zero): the diagonal blocks came with the Gram
+        // ---------------- T = (I + A)^-1 (blocks above the diagonal are neither
+        // written nor read): the diagonal blocks came with the Gram
         // epilogue; block rows bi = 1..3 on tensor cores, one warp per block (bi, bj):
         //   X = sum_{m=bj}^{bi-1} A_{bi,m} T_{m,bj},   T_{bi,bj} = -T_{bi,bi} X
         // The producers also write T diag(beta) and (GATE 0) T diag(beta Gamma).
@@ -461,6 +463,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             const int kw0 = (D / NCB) * (w >> 2);
 #pragma unroll
             for (int k0 = 0; k0 < C; k0 += 16) {
+                if (k0 > rw0) break;   // T is lower triangular
                 uint32_t at[4];
                 ldsm(at, a_rm(GATE ? aTB : aTG, LDC, rw0, k0, lane));
 #pragma unroll
@@ -484,6 +487,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         for (int j = 0; j < NJ; ++j) accU[j][0] = accU[j][1] = accU[j][2] = accU[j][3] = 0.f;
 #pragma unroll
         for (int k0 = 0; k0 < C; k0 += 16) {
+            if (k0 > rw0) break;
             uint32_t atb[4];
             ldsm(atb, a_rm(aTB, LDC, rw0, k0, lane));
 #pragma unroll
@@ -536,6 +540,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         // ---------------- O += M U'  and the output rows
 #pragma unroll
         for (int k0 = 0; k0 < C; k0 += 16) {
+            if (k0 > rw0) break;   // M is lower triangular
             uint32_t am[4];
             ldsm(am, a_rm(aM, LDC, rw0, k0, lane));
 #pragma unroll
@@ -559,32 +564,44 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         }
 
         // ---------------- S <- Gamma_C S + K^T diag(e) U'  (GATE 1: diag(Gamma_C) S +
-        // (K diag(Gamma_C / Gamma))^T U'); warp rows dk 16w.., this CTA's columns
+        // (K diag(Gamma_C / Gamma))^T U'); the warp's 32 x DVC / 4 block of the state
         {
-            const int r0 = rs0 + g;
-            const float gc0 = GATE ? sG[r0] : sEg[C - 1], gc1 = GATE ? sG[r0 + 8] : sEg[C - 1];
 #pragma unroll
-            for (int j = 0; j < NJS; ++j) {
-                accS[j][0] *= gc0; accS[j][1] *= gc0; accS[j][2] *= gc1; accS[j][3] *= gc1;
+            for (int mt = 0; mt < 2; ++mt) {
+                const int r0 = rs0 + 16 * mt + g;
+                const float gc0 = GATE ? sG[r0] : sEg[C - 1], gc1 = GATE ? sG[r0 + 8] : sEg[C - 1];
+#pragma unroll
+                for (int j = 0; j < NJS; ++j) {
+                    float *x = accS[mt][j];
+                    x[0] *= gc0; x[1] *= gc0; x[2] *= gc1; x[3] *= gc1;
+                }
             }
             const uint32_t aKs = GATE ? aUE : aK, aUs = GATE ? aU : aUE;
 #pragma unroll
             for (int k0 = 0; k0 < C; k0 += 16) {
-                uint32_t ak[4];
-                ldsm_t(ak, a_tr(aKs, LDD, rs0, k0, lane));
+                uint32_t ak[2][4];
+                ldsm_t(ak[0], a_tr(aKs, LDD, rs0, k0, lane));
+                ldsm_t(ak[1], a_tr(aKs, LDD, rs0 + 16, k0, lane));
 #pragma unroll
                 for (int np = 0; np < NJS / 2; ++np) {
                     uint32_t bu[4];
                     ldsm_t(bu, b_kn(aUs, LDD, cs0 + 16 * np, k0, lane));
-                    mma(accS[2 * np], ak, bu[0], bu[1]);
-                    mma(accS[2 * np + 1], ak, bu[2], bu[3]);
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        mma(accS[mt][2 * np], ak[mt], bu[0], bu[1]);
+                        mma(accS[mt][2 * np + 1], ak[mt], bu[2], bu[3]);
+                    }
                 }
             }
 #pragma unroll
-            for (int j = 0; j < NJS; ++j) {
-                const int c = cs0 + 8 * j + 2 * t4;
-                st_h2(sS + r0 * LDD + c, accS[j][0], accS[j][1]);
-                st_h2(sS + (r0 + 8) * LDD + c, accS[j][2], accS[j][3]);
+            for (int mt = 0; mt < 2; ++mt) {
+                const int r0 = rs0 + 16 * mt + g;
+#pragma unroll
+                for (int j = 0; j < NJS; ++j) {
+                    const int c = cs0 + 8 * j + 2 * t4;
+                    st_h2(sS + r0 * LDD + c, accS[mt][j][0], accS[mt][j][1]);
+                    st_h2(sS + (r0 + 8) * LDD + c, accS[mt][j][2], accS[mt][j][3]);
+                }
             }
         }
         __syncthreads();
@@ -608,12 +625,16 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 
     if (a.hT) {
         float *hp = a.hT + (size_t)bh * D * D + dv0;
-        const int r0 = rs0 + g;
 #pragma unroll
-        for (int j = 0; j < NJS; ++j) {
-            const int c = cs0 + 8 * j + 2 * t4;
-            *reinterpret_cast<float2 *>(hp + (size_t)r0 * D + c) = make_float2(accS[j][0], accS[j][1]);
-            *reinterpret_cast<float2 *>(hp + (size_t)(r0 + 8) * D + c) = make_float2(accS[j][2], accS[j][3]);
+        for (int mt = 0; mt < 2; ++mt) {
+            const int r0 = rs0 + 16 * mt + g;
+#pragma unroll
+            for (int j = 0; j < NJS; ++j) {
+                const int c = cs0 + 8 * j + 2 * t4;
+                const float *x = accS[mt][j];
+                *reinterpret_cast<float2 *>(hp + (size_t)r0 * D + c) = make_float2(x[0], x[1]);
+                *reinterpret_cast<float2 *>(hp + (size_t)(r0 + 8) * D + c) = make_float2(x[2], x[3]);
+            }
         }
     }
 }
