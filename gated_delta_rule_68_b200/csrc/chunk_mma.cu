@@ -60,16 +60,17 @@ constexpr int OFF_TG = OFF_TB + SZ_C;           // T diag(beta Gamma) [r][i]
 constexpr int OFF_STG = OFF_TG + SZ_C;          // next chunk's K, Q, V as loaded (bf16 [3][64][128])
 constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32 [2][64])
 constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta (64 fp32 each); NQ x 128 fp32 sums
-constexpr int SMEM_BYTES = OFF_VEC + (256 + NQ * 128) * 4;
-// The scratch of the inverse reuses tiles that are dead while it is live: fp32
-// A sits in the U' tile, the fp16 inverse T in the diag(e) U' tile, and the
-// fp16 copy of A (an operand of the block-row products) after each warp's
-// 16 x 16 block-row product in the -W tile.
-constexpr int OFF_A = OFF_U;                    // fp32 A [64][65]
+constexpr int SMEM_BYTES = OFF_VEC + (256 + NQ * 128 + 128) * 4;
+// The scratch of the inverse reuses tiles that are dead while it is live: the
+// fp32 diagonal blocks of A sit in the U' tile, the fp16 inverse T in the diag(e)
+// U' tile, and the fp16 copy of A (an operand of the block-row products) after
+// each warp's 16 x 16 block-row product in the -W tile.
+constexpr int LDT = 20;                         // fp32 stride of a transposed 16 x 16 block (conflict-free stores)
+constexpr int OFF_A = OFF_U;                    // fp32 [4 blocks][16][LDT], block b holds A_bb transposed
 constexpr int OFF_TH = OFF_UE;                  // fp16 T [64][72]
 constexpr int OFF_X = OFF_W;                    // fp16 [8 warps][16][24]
 constexpr int OFF_AH = OFF_X + 8 * 16 * LDX * 2;// fp16 A [64][72]
-static_assert(C * LDF * 4 <= SZ_D, "A must fit in the U' tile");
+static_assert(4 * 16 * LDT * 4 <= SZ_D, "the diagonal blocks of A must fit in the U' tile");
 static_assert(C * LDC * 2 <= SZ_D, "T must fit in the diag(e) U' tile");
 static_assert(8 * 16 * LDX * 2 + C * LDC * 2 <= SZ_D, "block-row products and A must fit in the W tile");
 static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory");
@@ -108,11 +109,12 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     // diag(e) U' tile holds K diag(Gamma_C / Gamma): T goes to the T diag(beta Gamma) tile.
     __half *sAh = reinterpret_cast<__half *>(sm + OFF_AH);
     __half *sTh = reinterpret_cast<__half *>(sm + (GATE ? OFF_TG : OFF_TH));
-    float *sG = reinterpret_cast<float *>(sm + OFF_VEC);  // [64] G_r           | GATE 1: [128] Gamma_C
+    float *sG = reinterpret_cast<float *>(sm + OFF_VEC);  // [64] G_r           | GATE 1: [128] exp(G_31)
     float *sEg = sG + 64;                                  // [64] exp(G_r)      |
     float *sEt = sG + 128;                                 // [64] exp(G_C - G_r)
     float *sBeta = sG + 192;                               // [64]
     float *sTot = sG + 256;                                // GATE 1: [NQ][128] per-channel sums of each row group
+    float *sP2 = sG + 256 + NQ * 128;                      // GATE 1: [128] exp(G_C - G_31)
     float *sColf = sG + 256;                               // GATE 0: [4][64] exp(G_16R - G_i)
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
@@ -161,8 +163,10 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 }
                 float *x = accS[mt][j];
                 x[0] = x0.x; x[1] = x0.y; x[2] = x1.x; x[3] = x1.y;
-                st_h2(sS + r0 * LDD + c, x0.x, x0.y);
-                st_h2(sS + (r0 + 8) * LDD + c, x1.x, x1.y);
+                if (GATE == 0) {   // GATE 1 writes its scaled copy in each chunk's gate pass
+                    st_h2(sS + r0 * LDD + c, x0.x, x0.y);
+                    st_h2(sS + (r0 + 8) * LDD + c, x1.x, x1.y);
+                }
             }
         }
     }
@@ -200,7 +204,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             const float *gp = a.g + ((tok0 + t0 + RPT * (tid >> 7)) * a.Hv + h) * D + (tid & (D - 1));
             const long gstride = (long)a.Hv * D;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) gnext[r] = (RPT * (tid >> 7) + r < n) ? __ldg(gp + r * gstride) : 0.f;
+            for (int r = 0; r < RPT; ++r)   // rows past the end re-read the last row; the
+                gnext[r] = __ldg(gp + min(r, n - 1 - RPT * (tid >> 7)) * gstride);   // consumer masks them
         }
     };
     if (NC > 0) load_gates(0);
@@ -209,7 +214,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     for (int ch = 0; ch < NC; ++ch) {
         const int t0 = ch * C, n = min(C, T - t0);
         cp_async_wait_all();
-        if (tid == 0) tma_store_wait_read();   // the previous chunk's o tile has been read out
+        // The previous chunk's o tile (in the V tile, and for fp32 o also in W) must have
+        // been read out before those tiles are rewritten, which first happens in the Gram
+        // epilogue: the wait comes just before the barrier that ends the gate pass.
         if (!__syncthreads_and(mbar_wait_bounded(aBar, ch & 1))) {
             if (tid == 0) atomicAdd(&g_fused_load_timeouts, 1u);
             return;
@@ -259,7 +266,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             float s = 0.f;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                s += gnext[r];
+                s += RPT * ch_h + r < n ? gnext[r] : 0.f;
                 Gv[r] = s;
             }
             sTot[ch_h * D + ch_c] = s;
@@ -275,10 +282,18 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
 #pragma unroll
             for (int r = 0; r < RPT; ++r) Gv[r] += off;
-            if (ch_h == 0) sG[ch_c] = __expf(gcs);   // Gamma_C of channel c
-            // Gram operands about the reference row 31: rows of K and Q scaled by
-            // exp(G_r - G_31), columns of K by exp(G_31 - G_i). Each factor spans at
-            // most 32 tokens of decay; a product over a pair i <= r is exp(G_r - G_i).
+            if (ch_h == 0) {   // the state's row factors of channel c (their product is Gamma_C)
+                sG[ch_c] = __expf(gm);
+                sP2[ch_c] = __expf(gcs - gm);
+            }
+            // Operands about the reference row 31: rows of K and Q scaled by
+            // f1 = exp(G_r - G_31), K by f2 = exp(G_31 - G_r). Each factor spans at most
+            // 32 tokens of decay; a product over a pair i <= r is exp(G_r - G_i). The same
+            // tiles serve every product of the chunk, with the channel constants moved onto
+            // the state: K diag(Gamma) = (K diag f1) diag(exp G_31), Q likewise, and
+            // K diag(Gamma_C / Gamma) = (K diag f2) diag(exp(G_C - G_31)). So W is formed
+            // from K diag f1, O1 and W S use S' = diag(exp G_31) S, and the state update
+            // is S <- diag(exp(G_C - G_31)) (S' + (K diag f2)^T U').
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const int row = RPT * ch_h + r;
@@ -289,11 +304,24 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 bad |= fabsf(kr) > 65504.f || fabsf(qr) > 65504.f || fabsf(kc) > 65504.f;
                 sK[row * LDD + ch_c] = __float2half_rn(kr);
                 sQ[row * LDD + ch_c] = __float2half_rn(qr);
-                sW[row * LDD + ch_c] = __float2half_rn(kc);
+                sUE[row * LDD + ch_c] = __float2half_rn(kc);
             }
         }
-        if (__syncthreads_or(bad) && tid == 0 && split == 0)   // once per (unit, chunk)
-            atomicAdd(&g_fused_range_errors, 1u);
+        if (tid == 0) tma_store_wait_read();
+        __syncthreads();
+        if (GATE) {   // S' = diag(exp G_31) S, this warp's block, as the fp16 operand
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const int r0 = rs0 + 16 * mt + g;
+                const float p0 = sG[r0], p1 = sG[r0 + 8];
+#pragma unroll
+                for (int j = 0; j < NJS; ++j) {
+                    const int c = cs0 + 8 * j + 2 * t4;
+                    st_h2(sS + r0 * LDD + c, accS[mt][j][0] * p0, accS[mt][j][1] * p0);
+                    st_h2(sS + (r0 + 8) * LDD + c, accS[mt][j][2] * p1, accS[mt][j][3] * p1);
+                }
+            }
+        }
 
         // ---------------- Gram: warps 0-3 rows of K, warps 4-7 rows of Q, against the
         // 64 key rows (GATE 1: the scaled row and column operands)
@@ -304,7 +332,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             for (int j = 0; j < NJG; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
             const bool krow = (w & 7) < 4;
             const int cg0 = (C / NCS) * (w >> 3);
-            const uint32_t abase = krow ? aK : aQ, bbase = GATE ? aW : aK;
+            const uint32_t abase = krow ? aK : aQ, bbase = GATE ? aUE : aK;
             // Only key blocks at or left of the diagonal block are ever used (i <= r).
             if (cg0 <= rw0) {
 #pragma unroll
@@ -322,7 +350,6 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     }
                 }
             }
-            if (GATE) __syncthreads();   // the scaled tiles are rewritten below
             // A rows (fp32 and fp16) from warps 0-3; M rows (fp16) from warps 4-7
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -337,8 +364,11 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     if (krow) {
                         const float x0 = i < r ? br * f0 * d0 : 0.f;
                         const float x1 = i + 1 < r ? br * f1 * d1 : 0.f;
-                        sA[r * LDF + i] = x0;
-                        sA[r * LDF + i + 1] = x1;
+                        if ((i >> 4) == (rw0 >> 4)) {   // diagonal block: fp32, transposed
+                            float *at = sA + (rw0 >> 4) * 16 * LDT + (i & 15) * LDT + (r & 15);
+                            at[0] = x0;
+                            at[LDT] = x1;
+                        }
                         st_h2(sAh + r * LDC + i, x0, x1);
                     } else {
                         st_h2(sM + r * LDC + i, i <= r ? f0 * d0 : 0.f, i + 1 <= r ? f1 * d1 : 0.f);
@@ -347,22 +377,27 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             }
             if (krow) {
                 // T = (I + A)^-1, its 16x16 diagonal block: the warp that holds that block of
-                // A solves it by forward substitution in fp32 (lane = column of the block)
+                // A solves (I + A_bb) t = e_col by forward substitution in fp32 (lane = column
+                // col of the block), column-oriented: once t_i is final, every later t_r
+                // takes its A_ri t_i, so the dependent chain is one FMA per pivot.
                 const int rb = rw0 >> 4;
                 if (rb >= (cg0 >> 4) && rb < (cg0 >> 4) + NJG / 2) {
                     __syncwarp();
                     if (lane < 16) {
                         const int base = 16 * rb, col = lane;
+                        const float *at = sA + rb * 16 * LDT;   // at[i * LDT + r] = A[base + r][base + i]
                         float tv[16];
 #pragma unroll
-                        for (int r = 0; r < 16; ++r) {
-                            float s0 = 0.f, s1 = 0.f;
+                        for (int r = 0; r < 16; ++r) tv[r] = r == col ? 1.f : 0.f;
 #pragma unroll
-                            for (int i = 0; i < r; i += 2) {
-                                s0 += sA[(base + r) * LDF + base + i] * tv[i];
-                                if (i + 1 < r) s1 += sA[(base + r) * LDF + base + i + 1] * tv[i + 1];
-                            }
-                            tv[r] = (r < col) ? 0.f : (r == col ? 1.f : -(s0 + s1));
+                        for (int i = 0; i < 15; ++i) {
+                            float ac[16];
+#pragma unroll
+                            for (int q4 = i / 4; q4 < 4; ++q4)
+                                *reinterpret_cast<float4 *>(ac + 4 * q4) =
+                                    *reinterpret_cast<const float4 *>(at + i * LDT + 4 * q4);
+#pragma unroll
+                            for (int r = i + 1; r < 16; ++r) tv[r] = fmaf(-ac[r], tv[i], tv[r]);
                         }
                         const float bc = sBeta[base + col], bgc = GATE ? 0.f : bc * sEg[base + col];
 #pragma unroll
@@ -383,20 +418,6 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     *reinterpret_cast<uint4 *>(sV + r * LDD + c8 * 8) =
                         r < n ? bf16x8_to_f16x8(sStg[2 * C * 16 + idx]) : make_uint4(0, 0, 0, 0);
                 }
-            }
-        }
-        if (GATE) {
-            // K diag(Gamma) (for W), Q diag(Gamma) (for O) and K diag(Gamma_C / Gamma)
-            // (for the state update); every factor is at most 1.
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const int row = RPT * ch_h + r;
-                const float e1 = __expf(Gv[r]), e2 = __expf(gcs - Gv[r]);
-                const float kv = row < n ? __bfloat162float(sStgH[row * D + ch_c]) : 0.f;
-                const float qv = row < n ? __bfloat162float(sStgH[C * D + row * D + ch_c]) : 0.f;
-                sK[row * LDD + ch_c] = __float2half_rn(kv * e1);
-                sQ[row * LDD + ch_c] = __float2half_rn(qv * e1);
-                sUE[row * LDD + ch_c] = __float2half_rn(kv * e2);
             }
         }
         __syncthreads();
@@ -477,6 +498,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 #pragma unroll
             for (int j = 0; j < NJW; ++j) {
                 const int c = kw0 + 8 * j + 2 * t4;
+                if (GATE)   // W carries f1, which can exceed 1
+                    bad |= fmaxf(fmaxf(fabsf(accW[j][0]), fabsf(accW[j][1])),
+                                 fmaxf(fabsf(accW[j][2]), fabsf(accW[j][3]))) > 65504.f;
                 st_h2(sW + (rw0 + g) * LDD + c, -accW[j][0], -accW[j][1]);
                 st_h2(sW + (rw0 + g + 8) * LDD + c, -accW[j][2], -accW[j][3]);
             }
@@ -498,26 +522,37 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 mma(accU[2 * np + 1], atb, bv[2], bv[3]);
             }
         }
-        __syncthreads();
+        // GATE 1: an fp16 operand of this chunk left the fp16 range (its results are not valid)
+        if (__syncthreads_or(bad) && tid == 0 && split == 0)   // once per (unit, chunk)
+            atomicAdd(&g_fused_range_errors, 1u);
 
         // ---------------- U' = U - W S,  O1 = Q S (GATE 0: then scaled by Gamma_r;
-        // GATE 1: Q already carries Gamma), K-dim dk
+        // GATE 1: Q already carries Gamma), K-dim dk. The fragments of step ks + 1
+        // are loaded before the products of step ks.
         float accO[NJ][4];
 #pragma unroll
         for (int j = 0; j < NJ; ++j) accO[j][0] = accO[j][1] = accO[j][2] = accO[j][3] = 0.f;
+        {
+            uint32_t fa[2][2][4], fb[2][NJ / 2][4];   // [buffer][W, Q], [buffer][n16 block]
+            auto load = [&](int buf, int k0) {
+                ldsm(fa[buf][0], a_rm(aW, LDD, rw0, k0, lane));
+                ldsm(fa[buf][1], a_rm(aQ, LDD, rw0, k0, lane));
 #pragma unroll
-        for (int k0 = 0; k0 < D; k0 += 16) {
-            uint32_t aw[4], aq[4];
-            ldsm(aw, a_rm(aW, LDD, rw0, k0, lane));
-            ldsm(aq, a_rm(aQ, LDD, rw0, k0, lane));
+                for (int np = 0; np < NJ / 2; ++np) ldsm_t(fb[buf][np], b_kn(aS, LDD, cw0 + 16 * np, k0, lane));
+            };
+            load(0, 0);
 #pragma unroll
-            for (int np = 0; np < NJ / 2; ++np) {
-                uint32_t bs[4];
-                ldsm_t(bs, b_kn(aS, LDD, cw0 + 16 * np, k0, lane));
-                mma(accU[2 * np], aw, bs[0], bs[1]);
-                mma(accU[2 * np + 1], aw, bs[2], bs[3]);
-                mma(accO[2 * np], aq, bs[0], bs[1]);
-                mma(accO[2 * np + 1], aq, bs[2], bs[3]);
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int cur = ks & 1;
+                if (ks + 1 < D / 16) load(cur ^ 1, 16 * (ks + 1));
+#pragma unroll
+                for (int np = 0; np < NJ / 2; ++np) {
+                    const uint32_t *b = fb[cur][np];
+                    mma(accU[2 * np], fa[cur][0], b[0], b[1]);
+                    mma(accU[2 * np + 1], fa[cur][0], b[2], b[3]);
+                    mma(accO[2 * np], fa[cur][1], b[0], b[1]);
+                    mma(accO[2 * np + 1], fa[cur][1], b[2], b[3]);
+                }
             }
         }
         {
@@ -563,8 +598,8 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
             fence_proxy_async();
         }
 
-        // ---------------- S <- Gamma_C S + K^T diag(e) U'  (GATE 1: diag(Gamma_C) S +
-        // (K diag(Gamma_C / Gamma))^T U'); the warp's 32 x DVC / 4 block of the state
+        // ---------------- S <- Gamma_C S + K^T diag(e) U'  (GATE 1: S <- diag(exp(G_C -
+        // G_31)) (diag(exp G_31) S + (K diag f2)^T U')); the warp's 32 x DVC / 4 block
         {
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
@@ -577,30 +612,42 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 }
             }
             const uint32_t aKs = GATE ? aUE : aK, aUs = GATE ? aU : aUE;
+            uint32_t fk[2][2][4], fu[2][NJS / 2][4];   // step ks + 1 loads before step ks products
+            auto load = [&](int buf, int k0) {
+                ldsm_t(fk[buf][0], a_tr(aKs, LDD, rs0, k0, lane));
+                ldsm_t(fk[buf][1], a_tr(aKs, LDD, rs0 + 16, k0, lane));
 #pragma unroll
-            for (int k0 = 0; k0 < C; k0 += 16) {
-                uint32_t ak[2][4];
-                ldsm_t(ak[0], a_tr(aKs, LDD, rs0, k0, lane));
-                ldsm_t(ak[1], a_tr(aKs, LDD, rs0 + 16, k0, lane));
+                for (int np = 0; np < NJS / 2; ++np) ldsm_t(fu[buf][np], b_kn(aUs, LDD, cs0 + 16 * np, k0, lane));
+            };
+            load(0, 0);
+#pragma unroll
+            for (int ks = 0; ks < C / 16; ++ks) {
+                const int cur = ks & 1;
+                if (ks + 1 < C / 16) load(cur ^ 1, 16 * (ks + 1));
 #pragma unroll
                 for (int np = 0; np < NJS / 2; ++np) {
-                    uint32_t bu[4];
-                    ldsm_t(bu, b_kn(aUs, LDD, cs0 + 16 * np, k0, lane));
+                    const uint32_t *b = fu[cur][np];
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt) {
-                        mma(accS[mt][2 * np], ak[mt], bu[0], bu[1]);
-                        mma(accS[mt][2 * np + 1], ak[mt], bu[2], bu[3]);
+                        mma(accS[mt][2 * np], fk[cur][mt], b[0], b[1]);
+                        mma(accS[mt][2 * np + 1], fk[cur][mt], b[2], b[3]);
                     }
                 }
             }
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 const int r0 = rs0 + 16 * mt + g;
+                const float p0 = GATE ? sP2[r0] : 1.f, p1 = GATE ? sP2[r0 + 8] : 1.f;
 #pragma unroll
                 for (int j = 0; j < NJS; ++j) {
-                    const int c = cs0 + 8 * j + 2 * t4;
-                    st_h2(sS + r0 * LDD + c, accS[mt][j][0], accS[mt][j][1]);
-                    st_h2(sS + (r0 + 8) * LDD + c, accS[mt][j][2], accS[mt][j][3]);
+                    float *x = accS[mt][j];
+                    if (GATE) {   // its fp16 copy is written with the next chunk's exp(G_31)
+                        x[0] *= p0; x[1] *= p0; x[2] *= p1; x[3] *= p1;
+                    } else {
+                        const int c = cs0 + 8 * j + 2 * t4;
+                        st_h2(sS + r0 * LDD + c, x[0], x[1]);
+                        st_h2(sS + (r0 + 8) * LDD + c, x[2], x[3]);
+                    }
                 }
             }
         }

@@ -15,7 +15,6 @@ constexpr int C = 64;            // tokens per chunk
 constexpr int D = 128;           // key and value width
 constexpr int LDD = D + 8;       // fp16 row stride of 128-wide tiles (272 B: ldmatrix rows hit distinct banks)
 constexpr int LDC = C + 8;       // fp16 row stride of 64-wide tiles (144 B)
-constexpr int LDF = C + 1;       // fp32 row stride of the 64 x 64 scratch
 constexpr int LDX = 24;          // fp16 row stride of a warp's 16 x 16 product
 constexpr int SZ_D = C * LDD * 2;  // one [64][128] fp16 tile
 constexpr int SZ_C = C * LDC * 2;  // one [64][64] fp16 tile
@@ -123,6 +122,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     while (!mbar_try_wait(bar, parity))
         if (globaltimer_ns() - t0 > 1000000000ull) return false;
     return true;
+}
+
+// Barrier `id` over the first `nthreads` threads that reach it (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
