@@ -44,7 +44,7 @@ constexpr int NW = 16;           // warps per CTA
 constexpr int NT = 32 * NW;
 constexpr int NCB = NW / 4;      // column blocks of the [64 x n] products (4 row blocks of 16)
 constexpr int NCS = NW / 8;      // column blocks of the [128 x n] products (8 row blocks of 16)
-constexpr int NQ = NT / 128;     // row groups of the per-channel gate pass (one thread per channel and group)
+constexpr int NQ = NT / 64;      // row groups of the per-channel gate pass (one thread per channel pair and group)
 
 // Shared-memory layout (bytes).
 constexpr int OFF_K = 0;                        // K [i][dk]
@@ -197,15 +197,15 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     if (NC > 0) issue_loads(0);
     // GATE 1: this thread's per-channel gates of the next chunk, loaded into registers
     // a chunk ahead so their latency hides behind the current chunk's work.
-    float gnext[GATE ? RPT : 1];
+    float2 gnext[GATE ? RPT : 1];
     auto load_gates = [&](int c) {
         if (GATE) {
-            const int t0 = c * C, n = min(C, T - t0);
-            const float *gp = a.g + ((tok0 + t0 + RPT * (tid >> 7)) * a.Hv + h) * D + (tid & (D - 1));
+            const int t0 = c * C, n = min(C, T - t0), q = tid >> 6;
+            const float *gp = a.g + ((tok0 + t0 + RPT * q) * a.Hv + h) * D + 2 * (tid & 63);
             const long gstride = (long)a.Hv * D;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r)   // rows past the end re-read the last row; the
-                gnext[r] = __ldg(gp + min(r, n - 1 - RPT * (tid >> 7)) * gstride);   // consumer masks them
+            for (int r = 0; r < RPT; ++r)   // rows past the end re-read the last row; the consumer masks them
+                gnext[r] = __ldg(reinterpret_cast<const float2 *>(gp + min(r, n - 1 - RPT * q) * gstride));
         }
     };
     if (NC > 0) load_gates(0);
@@ -223,12 +223,12 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         }
 
         // ---------------- gates and fp16 operand tiles
-        // GATE 1 keeps each channel's prefix G for RPT rows in registers: thread
-        // (c, q) owns key channel c = tid % 128 and rows RPT q .. RPT q + RPT - 1.
-        float Gv[GATE ? RPT : 1];
-        float gm = 0.f, gcs = 0.f;   // GATE 1: G at row 31 and at row 63 of channel c
-        bool bad = false;            // GATE 1: a factor left the fp16 range
-        const int ch_c = tid & (D - 1), ch_h = tid >> 7;
+        // GATE 1 keeps the prefix G of two channels over RPT rows in registers: thread
+        // (p, q) owns key channels 2p, 2p + 1 (p = tid % 64) and rows RPT q .. RPT q + RPT - 1.
+        float2 Gv[GATE ? RPT : 1];
+        float2 gm = make_float2(0.f, 0.f), gcs = gm;   // GATE 1: G at row 31 and at row 63
+        bool bad = false;                              // GATE 1: an operand left the fp16 range
+        const int ch_p = tid & 63, ch_h = tid >> 6;
         if (GATE == 0) {
             if (w == 0) {   // G, exp(G), exp(G_C - G)
                 const float x0 = sGst[2 * lane], x1 = sGst[2 * lane + 1];
@@ -263,28 +263,28 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                     r < n ? bf16x8_to_f16x8(sStg[idx]) : make_uint4(0, 0, 0, 0);
             }
         } else {
-            float s = 0.f;
+            float2 s = make_float2(0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                s += RPT * ch_h + r < n ? gnext[r] : 0.f;
+                if (RPT * ch_h + r < n) { s.x += gnext[r].x; s.y += gnext[r].y; }
                 Gv[r] = s;
             }
-            sTot[ch_h * D + ch_c] = s;
+            *reinterpret_cast<float2 *>(sTot + ch_h * D + 2 * ch_p) = s;
             if (w == 2 || w == 3) sBeta[tid - 64] = sGst[C + tid - 64];
             __syncthreads();
-            float off = 0.f;
+            float2 off = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
-                const float tq = sTot[q * D + ch_c];
-                off += q < ch_h ? tq : 0.f;
-                gm += q < NQ / 2 ? tq : 0.f;
-                gcs += tq;
+                const float2 tq = *reinterpret_cast<const float2 *>(sTot + q * D + 2 * ch_p);
+                if (q < ch_h) { off.x += tq.x; off.y += tq.y; }
+                if (q < NQ / 2) { gm.x += tq.x; gm.y += tq.y; }
+                gcs.x += tq.x; gcs.y += tq.y;
             }
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) Gv[r] += off;
-            if (ch_h == 0) {   // the state's row factors of channel c (their product is Gamma_C)
-                sG[ch_c] = __expf(gm);
-                sP2[ch_c] = __expf(gcs - gm);
+            for (int r = 0; r < RPT; ++r) { Gv[r].x += off.x; Gv[r].y += off.y; }
+            if (ch_h == 0) {   // the state's row factors of these channels (their product is Gamma_C)
+                *reinterpret_cast<float2 *>(sG + 2 * ch_p) = make_float2(__expf(gm.x), __expf(gm.y));
+                *reinterpret_cast<float2 *>(sP2 + 2 * ch_p) = make_float2(__expf(gcs.x - gm.x), __expf(gcs.y - gm.y));
             }
             // Operands about the reference row 31: rows of K and Q scaled by
             // f1 = exp(G_r - G_31), K by f2 = exp(G_31 - G_r). Each factor spans at most
@@ -297,14 +297,20 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const int row = RPT * ch_h + r;
-                const float f1 = __expf(Gv[r] - gm), f2 = __expf(gm - Gv[r]);
-                const float kv = row < n ? __bfloat162float(sStgH[row * D + ch_c]) : 0.f;
-                const float qv = row < n ? __bfloat162float(sStgH[C * D + row * D + ch_c]) : 0.f;
-                const float kr = kv * f1, qr = qv * f1, kc = kv * f2;
-                bad |= fabsf(kr) > 65504.f || fabsf(qr) > 65504.f || fabsf(kc) > 65504.f;
-                sK[row * LDD + ch_c] = __float2half_rn(kr);
-                sQ[row * LDD + ch_c] = __float2half_rn(qr);
-                sUE[row * LDD + ch_c] = __float2half_rn(kc);
+                const float2 f1 = make_float2(__expf(Gv[r].x - gm.x), __expf(Gv[r].y - gm.y));
+                const float2 f2 = make_float2(__expf(gm.x - Gv[r].x), __expf(gm.y - Gv[r].y));
+                float2 kv = make_float2(0.f, 0.f), qv = kv;
+                if (row < n) {
+                    kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sStgH + row * D + 2 * ch_p));
+                    qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sStgH + C * D + row * D + 2 * ch_p));
+                }
+                const float2 kr = make_float2(kv.x * f1.x, kv.y * f1.y), qr = make_float2(qv.x * f1.x, qv.y * f1.y);
+                const float2 kc = make_float2(kv.x * f2.x, kv.y * f2.y);
+                bad |= fmaxf(fmaxf(fabsf(kr.x), fabsf(kr.y)), fmaxf(fmaxf(fabsf(qr.x), fabsf(qr.y)),
+                                                                   fmaxf(fabsf(kc.x), fabsf(kc.y)))) > 65504.f;
+                *reinterpret_cast<__half2 *>(sK + row * LDD + 2 * ch_p) = __floats2half2_rn(kr.x, kr.y);
+                *reinterpret_cast<__half2 *>(sQ + row * LDD + 2 * ch_p) = __floats2half2_rn(qr.x, qr.y);
+                *reinterpret_cast<__half2 *>(sUE + row * LDD + 2 * ch_p) = __floats2half2_rn(kc.x, kc.y);
             }
         }
         if (tid == 0) tma_store_wait_read();
