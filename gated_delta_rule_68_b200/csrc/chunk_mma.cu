@@ -180,17 +180,19 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     __syncthreads();
     auto issue_loads = [&](int c) {
         const int t0 = c * C, n = min(C, T - t0);
-        if (tid == 0) {
+        // issued by the last warps: warps 0-2 run the inverse right after this
+        if (tid == NT - 32) {
             mbar_expect_tx(aBar, (2u * C * D + C * DVC) * 2);
             tma_load_4d(aStg, &map_k, 0, hk, tt0 + t0, tb, aBar);
             tma_load_4d(aStg + C * D * 2, &map_q, 0, hk, tt0 + t0, tb, aBar);
             tma_load_4d(aStg + 2 * C * D * 2, &map_v, dv0, h, tt0 + t0, tb, aBar);
         }
-        if (tid < 2 * C && (GATE == 0 || tid >= C)) {
-            const int r = tid & (C - 1);
-            const float *src = tid < C ? a.g : a.beta;
+        const int u = tid - (NT - 2 * C);   // [0, C): g of row u, [C, 2C): beta of row u - C
+        if (u >= 0 && (GATE == 0 || u >= C)) {
+            const int r = u & (C - 1);
+            const float *src = u < C ? a.g : a.beta;
             if (r < n) src += (tok0 + t0 + r) * a.Hv + h;
-            cp_async4(aGst + tid * 4, src, r < n ? 4u : 0u);
+            cp_async4(aGst + u * 4, src, r < n ? 4u : 0u);
         }
         cp_async_commit();
     };
