@@ -82,13 +82,13 @@ static_assert(C * D * 4 <= 2 * SZ_D, "an fp32 o tile must fit in the V and W til
 __device__ unsigned int g_fused_load_timeouts;
 __device__ unsigned int g_fused_range_errors;
 
-// GATE 0: one decay per (token, head); GATE 1: one per (token, head, key channel).
-// NS: value columns are split over NS CTAs per (b, h), each owning D / NS of them
-// (its part of the state, U, U', O); the Gram, the inverse and W are computed by each.
+// One CTA's part of unit bh = (b, h). GATE 0: one decay per (token, head); GATE 1: one
+// per (token, head, key channel). NS: the unit's value columns are split over NS CTAs,
+// CTA `split` owning D / NS of them (its part of the state, U, U', O); the Gram, the
+// inverse and W are computed by each.
 template <typename TOut, int GATE, int NS>
-__global__ void __launch_bounds__(NT, 1)
-fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
+__device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *map_q, const CUtensorMap *map_k,
+                                           const CUtensorMap *map_v, const CUtensorMap *map_o, int bh, int split)
 {
     constexpr int DVC = D / NS;      // value columns of this CTA
     constexpr int NJ = DVC / NCB / 8;   // n8 tiles of a warp in the [64 x DVC] products
@@ -127,7 +127,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     __half *sXw = reinterpret_cast<__half *>(sm + OFF_X) + w * 16 * LDX;   // this warp's 16 x 16 tile
     const uint32_t aXw = smem_u32(sXw);
-    const int split = blockIdx.x % NS, bh = blockIdx.x / NS, dv0 = split * DVC;
+    const int dv0 = split * DVC;
     const int b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
     // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
     // maps, batch index tb and token offset tt0. Packed input: sequence b of cu_seqlens
@@ -183,9 +183,9 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
         // issued by the last warps: warps 0-2 run the inverse right after this
         if (tid == NT - 32) {
             mbar_expect_tx(aBar, (2u * C * D + C * DVC) * 2);
-            tma_load_4d(aStg, &map_k, 0, hk, tt0 + t0, tb, aBar);
-            tma_load_4d(aStg + C * D * 2, &map_q, 0, hk, tt0 + t0, tb, aBar);
-            tma_load_4d(aStg + 2 * C * D * 2, &map_v, dv0, h, tt0 + t0, tb, aBar);
+            tma_load_4d(aStg, map_k, 0, hk, tt0 + t0, tb, aBar);
+            tma_load_4d(aStg + C * D * 2, map_q, 0, hk, tt0 + t0, tb, aBar);
+            tma_load_4d(aStg + 2 * C * D * 2, map_v, dv0, h, tt0 + t0, tb, aBar);
         }
         const int u = tid - (NT - 2 * C);   // [0, C): g of row u, [C, 2C): beta of row u - C
         if (u >= 0 && (GATE == 0 || u >= C)) {
@@ -665,7 +665,7 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 constexpr int EPB = 128 / sizeof(TOut);   // elements per 128-byte box row
 #pragma unroll
                 for (int bx = 0; bx < DVC / EPB; ++bx)
-                    tma_store_4d(&map_o, dv0 + bx * EPB, h, tt0 + t0, tb, smem_u32(sm + OFF_V + bx * C * 128));
+                    tma_store_4d(map_o, dv0 + bx * EPB, h, tt0 + t0, tb, smem_u32(sm + OFF_V + bx * C * 128));
             }
         } else {   // the rows after a packed sequence's end belong to the next sequence
             TOut *op = reinterpret_cast<TOut *>(a.o) + ((tok0 + t0) * a.Hv + h) * D + dv0;
@@ -691,6 +691,25 @@ fused_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __g
                 *reinterpret_cast<float2 *>(hp + (size_t)(r0 + 8) * D + c) = make_float2(x[2], x[3]);
             }
         }
+    }
+}
+
+
+// Blocks [0, n_whole) each run a whole unit; each later pair of blocks splits one of
+// the remaining units by value columns. Whole units are dispatched first, and the
+// halves fill the SMs as those free up.
+template <typename TOut, int GATE>
+__global__ void __launch_bounds__(NT, 1)
+fused_fwd_kernel(FwdArgs a, int n_whole, const __grid_constant__ CUtensorMap map_q,
+                 const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v1,
+                 const __grid_constant__ CUtensorMap map_v2, const __grid_constant__ CUtensorMap map_o)
+{
+    const int blk = blockIdx.x;
+    if (blk < n_whole) {
+        fused_unit<TOut, GATE, 1>(a, &map_q, &map_k, &map_v1, &map_o, blk, 0);
+    } else {
+        const int i = blk - n_whole;
+        fused_unit<TOut, GATE, 2>(a, &map_q, &map_k, &map_v2, &map_o, n_whole + i / 2, i % 2);
     }
 }
 
@@ -740,29 +759,28 @@ int sm_count()
     return n;
 }
 
-template <typename TOut, int GATE, int NS>
-cudaError_t launch_t(const FwdArgs &a, cudaStream_t st)
-{
-    CUtensorMap mq, mk, mv, mo;
-    const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
-    if (!make_map(&mq, a.q, mb, a.T, a.Hk, D) || !make_map(&mk, a.k, mb, a.T, a.Hk, D) ||
-        !make_map(&mv, a.v, mb, a.T, a.Hv, D / NS) ||
-        !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
-        return cudaErrorInvalidValue;
-    const int smem = SMEM_BYTES + 1024;
-    auto kernel = fused_fwd_kernel<TOut, GATE, NS>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    kernel<<<(unsigned)((long)a.B * a.Hv * NS), NT, smem, st>>>(a, mq, mk, mv, mo);
-    return cudaGetLastError();
-}
-
 template <typename TOut, int GATE>
 cudaError_t launch_g(const FwdArgs &a, cudaStream_t st)
 {
-    // Split the value columns over two CTAs when that still fits the SMs in one wave.
-    const long units = (long)a.B * a.Hv;
-    return 2 * units <= sm_count() ? launch_t<TOut, GATE, 2>(a, st) : launch_t<TOut, GATE, 1>(a, st);
+    // Whole units while they fit one wave of SMs; when all units fit as halves, every
+    // unit is split; when the units past one wave fit as halves in a second, those are.
+    const long units = (long)a.B * a.Hv, sms = sm_count();
+    long n_whole = units;
+    if (2 * units <= sms) n_whole = 0;
+    else if (units > sms && 2 * (units - sms) <= sms) n_whole = sms;
+    CUtensorMap mq, mk, mv1, mv2, mo;
+    const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
+    if (!make_map(&mq, a.q, mb, a.T, a.Hk, D) || !make_map(&mk, a.k, mb, a.T, a.Hk, D) ||
+        !make_map(&mv1, a.v, mb, a.T, a.Hv, D) || !make_map(&mv2, a.v, mb, a.T, a.Hv, D / 2) ||
+        !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
+        return cudaErrorInvalidValue;
+    const int smem = SMEM_BYTES + 1024;
+    auto kernel = fused_fwd_kernel<TOut, GATE>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const long grid = n_whole + 2 * (units - n_whole);
+    kernel<<<(unsigned)grid, NT, smem, st>>>(a, (int)n_whole, mq, mk, mv1, mv2, mo);
+    return cudaGetLastError();
 }
 
 template <typename TOut>

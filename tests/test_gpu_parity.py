@@ -136,6 +136,15 @@ def test_one_cta_per_unit_when_units_fill_the_sms(gate):
     full_check(w)
 
 
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_units_past_one_wave_are_split_in_halves(gate):
+    """160 units on a 148-SM B200: the first 148 run whole, each of the last 12 is split
+    over two CTAs by value columns (one launch, both kinds of CTA). Every unit is checked."""
+    w = WORKLOADS["gdn_bf16"].with_(B=10, T=130, Hk=16, Hv=16, gate=gate,
+                                    g_mu=4.0 if gate == "channel" else 3.0, seed=23)
+    full_check(w)
+
+
 def test_strong_channel_decay_is_reported_not_hidden():
     """A per-channel decay of exp(-1) per token spans exp(-32) over half a chunk: the fused
     kernel's fp16 factors overflow, and it says so in gdr_fused_error_counts."""
