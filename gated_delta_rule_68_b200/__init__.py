@@ -26,7 +26,7 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
            "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts",
-           "gdr_fwd_chunked_varlen")
+           "gdr_fwd_chunked_varlen", "gdr_causal_conv_silu", "gdr_rmsnorm_gated")
 
 # Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
 GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -67,6 +67,10 @@ def lib():
         L.gdr_fwd_chunked_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp] + [i] * 8 + [vp]
         L.gdr_fused_error_counts.restype = ctypes.c_uint
         L.gdr_fused_error_counts.argtypes = [vp, vp]
+        L.gdr_causal_conv_silu.restype = i
+        L.gdr_causal_conv_silu.argtypes = [vp, fp, fp, vp, vp, vp, vp] + [i] * 5 + [vp]
+        L.gdr_rmsnorm_gated.restype = i
+        L.gdr_rmsnorm_gated.argtypes = [vp, vp, fp, vp, ctypes.c_long, i, ctypes.c_float, i, vp]
         _lib = L
     return _lib
 
@@ -249,3 +253,60 @@ def gdr_fwd_chunked_noalloc(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_
                                          _ptr(o), _ptr(hT), B, T, Hk, Hv, Dk, Dv, gate_mode, dt,
                                          _stream(stream)))
     return o, hT
+
+
+def gdr_causal_conv_silu(x, w, bias=None, state_in=None, cu_seqlens=None, *, y=None, state_out=None,
+                         want_state=False, stream=None):
+    """Short causal convolution (4 taps) + SiLU; see include/gdr.h. x: [B, T, Ch] (or [T, Ch]
+    with cu_seqlens int32 [N + 1]); w: [Ch, 4] fp32; bias: [Ch] fp32; state_in: [B or N, Ch, 3]
+    in x's dtype. Returns (y, state_out or None)."""
+    if x.dtype == torch.bfloat16:
+        dt = GDR_BF16
+    elif x.dtype == torch.float32:
+        dt = GDR_FP32
+    else:
+        raise TypeError(f"unsupported x dtype {x.dtype}")
+    if cu_seqlens is None:
+        B, T, Ch = x.shape
+    else:
+        T, Ch = x.shape
+        B = cu_seqlens.numel() - 1
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,))
+    _need(x, "x", x.dtype)
+    _need(w, "w", torch.float32, (Ch, w.shape[1]))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (Ch,))
+    if state_in is not None:
+        _need(state_in, "state_in", x.dtype, (B, Ch, 3))
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", x.dtype, tuple(x.shape))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, Ch, 3), dtype=x.dtype, device=x.device)
+    if state_out is not None:
+        _need(state_out, "state_out", x.dtype, (B, Ch, 3))
+    _check(lib().gdr_causal_conv_silu(_ptr(x), _ptr(w), _ptr(bias), _ptr(state_in), _ptr(state_out), _ptr(y),
+                                      _ptr(cu_seqlens), B, T, Ch, w.shape[1], dt, _stream(stream)))
+    return y, state_out
+
+
+def gdr_rmsnorm_gated(o, z, weight, eps=1e-5, *, y=None, stream=None):
+    """y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z) over the last axis (64 or 128);
+    o, z, y in one dtype (bf16 or fp32); y may be o (in place)."""
+    if o.dtype == torch.bfloat16:
+        dt = GDR_BF16
+    elif o.dtype == torch.float32:
+        dt = GDR_FP32
+    else:
+        raise TypeError(f"unsupported o dtype {o.dtype}")
+    D = o.shape[-1]
+    _need(o, "o", o.dtype)
+    _need(z, "z", o.dtype, tuple(o.shape))
+    _need(weight, "weight", torch.float32, (D,))
+    if y is None:
+        y = torch.empty_like(o)
+    _need(y, "y", o.dtype, tuple(o.shape))
+    rows = o.numel() // D if D else 0
+    _check(lib().gdr_rmsnorm_gated(_ptr(o), _ptr(z), _ptr(weight), _ptr(y), rows, D, float(eps), dt,
+                                   _stream(stream)))
+    return y

@@ -201,4 +201,56 @@ int gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
     return GDR_OK;
 }
 
+int gdr_causal_conv_silu(const void *x, const float *w, const float *bias, const void *state_in, void *state_out,
+                         void *y, const int *cu_seqlens, int B, int T, int Ch, int width, int dtype, void *stream)
+{
+    if (B < 0 || T < 0 || Ch <= 0) return fail(GDR_ERR_INVALID_ARG, "sizes must be non-negative, Ch positive");
+    if (dtype != GDR_BF16 && dtype != GDR_FP32)
+        return fail(GDR_ERR_INVALID_ARG, "dtype must be GDR_BF16 or GDR_FP32 (got %d)", dtype);
+    if (width != 4) return fail(GDR_ERR_UNSUPPORTED, "the convolution has 4 taps (got width %d)", width);
+    if (Ch % 8) return fail(GDR_ERR_UNSUPPORTED, "Ch must be a multiple of 8 (got %d)", Ch);
+    const long rows = cu_seqlens ? (long)T : (long)B * T;
+    if (rows > 0 && (!x || !w || !y)) return fail(GDR_ERR_INVALID_ARG, "x, w and y must be non-NULL");
+    if (rows > 0 && B == 0) return fail(GDR_ERR_INVALID_ARG, "packed tokens need at least one sequence");
+    if (B > 0 && cu_seqlens && ((uintptr_t)cu_seqlens & 3u))
+        return fail(GDR_ERR_MISALIGNED, "cu_seqlens is not 4-byte aligned");
+    const void *ptrs[] = {x, w, y};
+    const char *names[] = {"x", "w", "y"};
+    for (int i = 0; i < 3; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    const uintptr_t es = dtype == GDR_FP32 ? 4 : 2;
+    if (((uintptr_t)state_in % es) || ((uintptr_t)state_out % es) || ((uintptr_t)bias & 3u))
+        return fail(GDR_ERR_MISALIGNED, "a state or bias pointer is not aligned to its element size");
+    if (x && x == y) return fail(GDR_ERR_INVALID_ARG, "y must not alias x");
+    if (rows == 0 && (!state_out || B == 0)) return GDR_OK;   // nothing to compute or pass through
+    gdr::ConvArgs a;
+    a.x = x; a.w = w; a.bias = bias; a.state_in = state_in; a.state_out = state_out; a.y = y;
+    a.cu_seqlens = cu_seqlens; a.nseq = B; a.T = T; a.rows = rows; a.Ch = Ch; a.fp32 = dtype == GDR_FP32;
+    cudaError_t e = gdr::launch_conv_silu(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += gdr::conv_launches(a);
+    return GDR_OK;
+}
+
+int gdr_rmsnorm_gated(const void *o, const void *z, const float *weight, void *y, long rows, int D, float eps,
+                      int dtype, void *stream)
+{
+    if (rows < 0) return fail(GDR_ERR_INVALID_ARG, "rows must be non-negative");
+    if (dtype != GDR_BF16 && dtype != GDR_FP32)
+        return fail(GDR_ERR_INVALID_ARG, "dtype must be GDR_BF16 or GDR_FP32 (got %d)", dtype);
+    if (D != 64 && D != 128) return fail(GDR_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+    if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be non-negative");
+    if (rows == 0) return GDR_OK;
+    if (!o || !z || !weight || !y) return fail(GDR_ERR_INVALID_ARG, "o, z, weight and y must be non-NULL");
+    const uintptr_t es = dtype == GDR_FP32 ? 4 : 2;
+    if (((uintptr_t)o % es) || ((uintptr_t)z % es) || ((uintptr_t)y % es) || ((uintptr_t)weight & 3u))
+        return fail(GDR_ERR_MISALIGNED, "a pointer is not aligned to its element size");
+    gdr::NormArgs a;
+    a.o = o; a.z = z; a.w = weight; a.y = y; a.rows = rows; a.D = D; a.eps = eps; a.fp32 = dtype == GDR_FP32;
+    cudaError_t e = gdr::launch_rmsnorm_gated(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += 1;
+    return GDR_OK;
+}
+
 }  // extern "C"

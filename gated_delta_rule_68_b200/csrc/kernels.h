@@ -42,4 +42,33 @@ unsigned int fused_error_counts(unsigned int *load_timeouts, unsigned int *range
 size_t simt_workspace_size(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a, void *ws, cudaStream_t st);
 
+// Short causal convolution (4 taps) + SiLU over [rows, Ch] (prologue.cu). Sequence n
+// is tokens [cu_seqlens[n], cu_seqlens[n + 1]) when cu_seqlens is given, else
+// [n T, n T + T); states are [nseq, Ch, 3] in the dtype of x (oldest input first).
+struct ConvArgs {
+    const void *x;
+    const float *w, *bias;
+    const void *state_in;
+    void *state_out, *y;
+    const int *cu_seqlens;
+    int nseq, T;
+    long rows;
+    int Ch;
+    bool fp32;
+};
+int conv_launches(const ConvArgs &a);
+cudaError_t launch_conv_silu(const ConvArgs &a, cudaStream_t st);
+
+// y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) per row of D (64 or 128) elements.
+struct NormArgs {
+    const void *o, *z;
+    const float *w;
+    void *y;
+    long rows;
+    int D;
+    float eps;
+    bool fp32;
+};
+cudaError_t launch_rmsnorm_gated(const NormArgs &a, cudaStream_t st);
+
 }  // namespace gdr

@@ -1,0 +1,246 @@
+// The layer's elementwise stages around the recurrence: the short causal
+// convolution with SiLU on the q/k/v projections, and the gated RMSNorm on the
+// output (NextTransformer "Source notes", section "Linear attention", rows
+// deltanet, kda and gdn; "Backend and numerical limits"; Atlas entry 03, a
+// four-token causal convolution). Both are HBM-bound streams: every input
+// element is read once and every output element written once.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+
+namespace gdr {
+namespace {
+
+constexpr int CONV_W = 4;     // taps; tap CONV_W - 1 sits on the current token
+constexpr int CONV_RUN = 16;  // consecutive tokens per thread
+constexpr int CONV_TPB = 256;
+
+struct Vec8 { float v[8]; };
+
+__device__ __forceinline__ Vec8 load8(const __nv_bfloat16 *p)
+{
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    Vec8 r;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        r.v[2 * i] = f.x;
+        r.v[2 * i + 1] = f.y;
+    }
+    return r;
+}
+__device__ __forceinline__ Vec8 load8(const float *p)
+{
+    const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+    Vec8 r = {{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
+    return r;
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const Vec8 &x)
+{
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x.v[2 * i], x.v[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = u;
+}
+__device__ __forceinline__ void store8(float *p, const Vec8 &x)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(x.v[0], x.v[1], x.v[2], x.v[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(x.v[4], x.v[5], x.v[6], x.v[7]);
+}
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ void from_f(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void from_f(float *p, float x) { *p = x; }
+
+__device__ __forceinline__ float silu(float y) { return y / (1.f + __expf(-y)); }
+
+// Sequence n of the token axis: [s0, s1). Without cu_seqlens, sequence n is
+// tokens n*T .. n*T + T - 1.
+struct Seqs {
+    const int *cu;
+    int n, T;
+    __device__ int start(int i) const { return cu ? cu[i] : i * T; }
+};
+
+// Thread (run, group): channels 8 group .. 8 group + 7 of tokens run*RUN ..
+// run*RUN + RUN - 1 of the flattened token axis. The last CONV_W - 1 inputs
+// of the current sequence ride along in registers; at a sequence's first token
+// they come from state_in (or are zero).
+template <typename T_>
+__global__ void __launch_bounds__(CONV_TPB)
+conv_silu_kernel(const T_ *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
+                 const T_ *__restrict__ state_in, T_ *__restrict__ state_out, T_ *__restrict__ y, Seqs sq,
+                 long rows, int Ch)
+{
+    const int ngroups = Ch / 8;
+    const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int grp = (int)(gid % ngroups);
+    const long t0 = (gid / ngroups) * CONV_RUN;
+    if (t0 >= rows) return;
+    const long t1 = min(t0 + (long)CONV_RUN, rows);
+    const int c0 = 8 * grp;
+
+    float wt[8][CONV_W], bs[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 q = *reinterpret_cast<const float4 *>(w + (size_t)(c0 + i) * CONV_W);
+        wt[i][0] = q.x; wt[i][1] = q.y; wt[i][2] = q.z; wt[i][3] = q.w;
+        bs[i] = bias ? bias[c0 + i] : 0.f;
+    }
+    // the sequence holding t0: the last n with start(n) <= t0 (empty sequences skipped)
+    int lo = 0, hi = sq.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sq.start(mid) <= t0) lo = mid; else hi = mid - 1;
+    }
+    int n = lo;
+    long s0 = sq.start(n), s1 = sq.start(n + 1);
+    // history: the CONV_W - 1 inputs before t0 in the sequence's virtual axis
+    // [state_in (oldest first) ; x[s0] ; x[s0 + 1] ; ...]
+    float h[CONV_W - 1][8];
+    auto fill_history = [&](long t) {
+#pragma unroll
+        for (int j = 0; j < CONV_W - 1; ++j) {
+            const long vt = t - s0 + j;   // virtual index of the input CONV_W - 1 - j tokens back
+            if (vt >= CONV_W - 1) {
+                const Vec8 a = load8(x + (size_t)(s0 + vt - (CONV_W - 1)) * Ch + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) h[j][i] = a.v[i];
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    h[j][i] = state_in ? to_f(state_in[((size_t)n * Ch + c0 + i) * (CONV_W - 1) + vt]) : 0.f;
+            }
+        }
+    };
+    fill_history(t0);
+    for (long t = t0; t < t1; ++t) {
+        while (t >= s1) {   // next sequence (skipping empty ones)
+            ++n;
+            s0 = s1;
+            s1 = sq.start(n + 1);
+            if (t < s1) fill_history(t);
+        }
+        const Vec8 xt = load8(x + (size_t)t * Ch + c0);
+        Vec8 o;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float acc = bs[i];
+#pragma unroll
+            for (int j = 0; j < CONV_W - 1; ++j) acc = fmaf(wt[i][j], h[j][i], acc);
+            acc = fmaf(wt[i][CONV_W - 1], xt.v[i], acc);
+            o.v[i] = silu(acc);
+        }
+        store8(y + (size_t)t * Ch + c0, o);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+#pragma unroll
+            for (int j = 0; j < CONV_W - 2; ++j) h[j][i] = h[j + 1][i];
+            h[CONV_W - 2][i] = xt.v[i];
+        }
+        if (state_out && t == s1 - 1) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < CONV_W - 1; ++j)
+                    from_f(&state_out[((size_t)n * Ch + c0 + i) * (CONV_W - 1) + j], h[j][i]);
+        }
+    }
+}
+
+// Sequences with no tokens pass their state through (zero without state_in).
+template <typename T_>
+__global__ void conv_state_empty_kernel(const T_ *__restrict__ state_in, T_ *__restrict__ state_out, Seqs sq,
+                                        int Ch)
+{
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long per = (long)Ch * (CONV_W - 1);
+    if (i >= (long)sq.n * per) return;
+    const int n = (int)(i / per);
+    if (sq.start(n + 1) != sq.start(n)) return;
+    state_out[i] = state_in ? state_in[i] : T_(0.f);
+}
+
+// One warp per row of D = 32 * PER elements.
+template <typename T_, int PER>
+__global__ void __launch_bounds__(256)
+rmsnorm_gated_kernel(const T_ *__restrict__ o, const T_ *__restrict__ z, const float *__restrict__ wt,
+                     T_ *__restrict__ y, long rows, float eps)
+{
+    const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    constexpr int D = 32 * PER;
+    const size_t base = (size_t)row * D + lane * PER;
+    float ov[PER], zv[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        ov[i] = to_f(o[base + i]);
+        zv[i] = to_f(z[base + i]);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) ss = fmaf(ov[i], ov[i], ss);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float rstd = rsqrtf(ss / D + eps);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) from_f(&y[base + i], ov[i] * rstd * wt[lane * PER + i] * silu(zv[i]));
+}
+
+template <typename T_>
+cudaError_t conv_t(const ConvArgs &a, cudaStream_t st)
+{
+    const Seqs sq{a.cu_seqlens, a.nseq, a.T};
+    const long rows = a.rows;
+    if (rows > 0) {
+        const long threads = ((rows + CONV_RUN - 1) / CONV_RUN) * (a.Ch / 8);
+        conv_silu_kernel<T_><<<(unsigned)((threads + CONV_TPB - 1) / CONV_TPB), CONV_TPB, 0, st>>>(
+            static_cast<const T_ *>(a.x), a.w, a.bias, static_cast<const T_ *>(a.state_in),
+            static_cast<T_ *>(a.state_out), static_cast<T_ *>(a.y), sq, rows, a.Ch);
+    }
+    if (a.state_out && (a.cu_seqlens || rows == 0)) {
+        const long n = (long)a.nseq * a.Ch * (CONV_W - 1);
+        if (n > 0)
+            conv_state_empty_kernel<T_><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+                static_cast<const T_ *>(a.state_in), static_cast<T_ *>(a.state_out), sq, a.Ch);
+    }
+    return cudaGetLastError();
+}
+
+template <typename T_>
+cudaError_t norm_t(const NormArgs &a, cudaStream_t st)
+{
+    const unsigned grid = (unsigned)((a.rows + 7) / 8);
+    if (a.D == 128)
+        rmsnorm_gated_kernel<T_, 4><<<grid, 256, 0, st>>>(static_cast<const T_ *>(a.o), static_cast<const T_ *>(a.z),
+                                                          a.w, static_cast<T_ *>(a.y), a.rows, a.eps);
+    else
+        rmsnorm_gated_kernel<T_, 2><<<grid, 256, 0, st>>>(static_cast<const T_ *>(a.o), static_cast<const T_ *>(a.z),
+                                                          a.w, static_cast<T_ *>(a.y), a.rows, a.eps);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int conv_launches(const ConvArgs &a)
+{
+    return (a.rows > 0 ? 1 : 0) + ((a.state_out && (a.cu_seqlens || a.rows == 0) && a.nseq > 0) ? 1 : 0);
+}
+
+cudaError_t launch_conv_silu(const ConvArgs &a, cudaStream_t st)
+{
+    return a.fp32 ? conv_t<float>(a, st) : conv_t<__nv_bfloat16>(a, st);
+}
+
+cudaError_t launch_rmsnorm_gated(const NormArgs &a, cudaStream_t st)
+{
+    if (a.rows <= 0) return cudaSuccess;
+    return a.fp32 ? norm_t<float>(a, st) : norm_t<__nv_bfloat16>(a, st);
+}
+
+}  // namespace gdr

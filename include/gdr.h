@@ -205,6 +205,42 @@ GDR_API int gdr_fwd_chunked_noalloc(const void *q, const void *k, const void *v,
                                     int B, int T, int Hk, int Hv, int Dk, int Dv,
                                     int gate_mode, int dtype, void *stream);
 
+/*
+ * The layer's short causal convolution with SiLU, applied to the q/k/v
+ * projections before the recurrence (NextTransformer "Source notes", section
+ * "Linear attention", rows deltanet and kda: causal conv + SiLU; "Backend and
+ * numerical limits": a causal convolution with SiLU activation; Atlas entry 03,
+ * a four-token causal convolution). Depthwise over channels:
+ *   y[t, c] = SiLU(bias[c] + sum_{j=0..3} w[c, j] x[t - 3 + j, c]),
+ *   SiLU(a) = a / (1 + e^-a),
+ * with the inputs before a sequence's first token taken from state_in (else 0).
+ *
+ * x, y: [B, T, Ch] (or, with cu_seqlens, [T, Ch]: B sequences packed along T
+ * tokens, sequence n is tokens [cu_seqlens[n], cu_seqlens[n+1]), cu_seqlens a
+ * device int32 [B + 1], non-decreasing, from 0 to T). w: [Ch, 4] fp32 (tap 3 on
+ * the current token), bias: [Ch] fp32 or NULL. state_in, state_out: [B, Ch, 3]
+ * in the dtype of x, the three inputs before each sequence / its last three
+ * (oldest first), each may be NULL (state_out of an empty sequence is state_in,
+ * or zeros). dtype: GDR_BF16 or GDR_FP32 for x, y and the states; arithmetic in
+ * fp32. width must be 4 and Ch a multiple of 8 (else GDR_ERR_UNSUPPORTED).
+ * x, w, y 16-byte aligned; y must not alias x. The caller owns every buffer.
+ */
+GDR_API int gdr_causal_conv_silu(const void *x, const float *w, const float *bias, const void *state_in,
+                                 void *state_out, void *y, const int *cu_seqlens, int B, int T, int Ch,
+                                 int width, int dtype, void *stream);
+
+/*
+ * The gated RMSNorm on the recurrence's output (NextTransformer "Source notes",
+ * row gdn: output RMSNorm x gain x SiLU gate; "Backend and numerical limits"):
+ *   y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z)
+ * per row of D elements (one head of one token). o, z, y: [rows, D] in `dtype`
+ * (GDR_BF16 or GDR_FP32; arithmetic in fp32); weight: [D] fp32. D must be 64
+ * or 128 (else GDR_ERR_UNSUPPORTED). y may alias o (in place). Pointers aligned
+ * to their element size.
+ */
+GDR_API int gdr_rmsnorm_gated(const void *o, const void *z, const float *weight, void *y, long rows, int D,
+                              float eps, int dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -118,3 +118,54 @@ def test_workspace_size_rules(L):
 ])
 def test_decode_rejects(L, kw, status):
     assert dec(L, **kw) == status
+
+
+def conv(L, x=A, w=A, bias=0, sin=0, sout=0, y=A + (1 << 16), cu=0, B=1, T=16, Ch=64, width=4, dtype=0):
+    vp = ctypes.c_void_p
+    return L.gdr_causal_conv_silu(vp(x), vp(w), vp(bias or None), vp(sin or None), vp(sout or None), vp(y),
+                                  vp(cu or None), B, T, Ch, width, dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(width=3), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(Ch=12), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dtype=2), gdr.GDR_ERR_INVALID_ARG),
+    (dict(B=-1), gdr.GDR_ERR_INVALID_ARG),
+    (dict(x=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(y=A), gdr.GDR_ERR_INVALID_ARG),          # y aliases x
+    (dict(x=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(w=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(cu=A + 2), gdr.GDR_ERR_MISALIGNED),
+    (dict(cu=A, B=0), gdr.GDR_ERR_INVALID_ARG),    # packed tokens with no sequence
+])
+def test_conv_rejects_bad_arguments(L, kw, status):
+    before = L.gdr_kernel_launches()
+    assert conv(L, **kw) == status
+    assert L.gdr_kernel_launches() == before
+
+
+def norm(L, o=A, z=A, w=A, y=A, rows=4, D=128, eps=1e-5, dtype=0):
+    vp = ctypes.c_void_p
+    return L.gdr_rmsnorm_gated(vp(o), vp(z), vp(w), vp(y), rows, D, ctypes.c_float(eps), dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dtype=2), gdr.GDR_ERR_INVALID_ARG),
+    (dict(rows=-1), gdr.GDR_ERR_INVALID_ARG),
+    (dict(eps=-1.0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(z=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(o=A + 1), gdr.GDR_ERR_MISALIGNED),
+    (dict(w=A + 2), gdr.GDR_ERR_MISALIGNED),
+])
+def test_rmsnorm_gated_rejects_bad_arguments(L, kw, status):
+    before = L.gdr_kernel_launches()
+    assert norm(L, **kw) == status
+    assert L.gdr_kernel_launches() == before
+
+
+def test_empty_calls_launch_nothing(L):
+    before = L.gdr_kernel_launches()
+    assert norm(L, rows=0) == gdr.GDR_OK
+    assert conv(L, T=0) == gdr.GDR_OK    # no tokens, no state_out: nothing to do
+    assert L.gdr_kernel_launches() == before
