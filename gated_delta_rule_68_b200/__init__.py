@@ -26,7 +26,8 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
            "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts",
-           "gdr_fwd_chunked_varlen", "gdr_causal_conv_silu", "gdr_rmsnorm_gated")
+           "gdr_fwd_chunked_varlen", "gdr_causal_conv_silu", "gdr_rmsnorm_gated",
+           "gdr_fwd_chunked_norm")
 
 # Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
 GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -69,6 +70,8 @@ def lib():
         L.gdr_fused_error_counts.argtypes = [vp, vp]
         L.gdr_causal_conv_silu.restype = i
         L.gdr_causal_conv_silu.argtypes = [vp, fp, fp, vp, vp, vp, vp] + [i] * 5 + [vp]
+        L.gdr_fwd_chunked_norm.restype = i
+        L.gdr_fwd_chunked_norm.argtypes = ([vp, vp, vp, fp, fp, fp, vp, fp, vp] + [i] * 9 + [vp, fp, ctypes.c_float, vp])
         L.gdr_rmsnorm_gated.restype = i
         L.gdr_rmsnorm_gated.argtypes = [vp, vp, fp, vp, ctypes.c_long, i, ctypes.c_float, i, vp]
         _lib = L
@@ -310,3 +313,48 @@ def gdr_rmsnorm_gated(o, z, weight, eps=1e-5, *, y=None, stream=None):
     _check(lib().gdr_rmsnorm_gated(_ptr(o), _ptr(z), _ptr(weight), _ptr(y), rows, D, float(eps), dt,
                                    _stream(stream)))
     return y
+
+
+def gdr_fwd_chunked_norm(q, k, v, g, beta, h0=None, *, cu_seqlens=None, qk_l2norm=False, z=None,
+                         norm_weight=None, norm_eps=1e-5, o=None, hT=None, want_hT=True, stream=None,
+                         out_dtype=None):
+    """Chunked forward with in-kernel q/k L2 normalisation and/or the gated output RMSNorm
+    (see include/gdr.h). Shapes as gdr_fwd_chunked, or as gdr_fwd_chunked_varlen when
+    cu_seqlens is given; z like o (bf16), norm_weight [Dv] fp32. Returns (o, hT)."""
+    packed = cu_seqlens is not None
+    if packed:
+        T, Hk, Dk = q.shape
+        Hv, Dv = v.shape[1], v.shape[2]
+        B = cu_seqlens.numel() - 1
+        tok = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,))
+    else:
+        B, T, Hk, Dk = q.shape
+        Hv, Dv = v.shape[2], v.shape[3]
+        tok = (B, T)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt, odt = _dtype_code(q, out_dtype)
+    gate_mode = GDR_GATE_CHANNEL if g.dim() == len(tok) + 2 else GDR_GATE_SCALAR
+    _need(q, "q", q.dtype)
+    _need(k, "k", q.dtype, q.shape)
+    _need(v, "v", q.dtype, tok + (Hv, Dv))
+    _need(g, "g", torch.float32, tok + ((Hv,) if gate_mode == 0 else (Hv, Dk)))
+    _need(beta, "beta", torch.float32, tok + (Hv,))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (B, Hv, Dk, Dv))
+    if z is not None:
+        _need(z, "z", torch.bfloat16, tok + (Hv, Dv))
+        _need(norm_weight, "norm_weight", torch.float32, (Dv,))
+    if o is None:
+        o = torch.empty(tok + (Hv, Dv), dtype=odt, device=q.device)
+    _need(o, "o", odt, tok + (Hv, Dv))
+    if hT is None and want_hT:
+        hT = torch.empty((B, Hv, Dk, Dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _need(hT, "hT", torch.float32, (B, Hv, Dk, Dv))
+    _check(lib().gdr_fwd_chunked_norm(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+                                      _ptr(hT), _ptr(cu_seqlens), B, T, Hk, Hv, Dk, Dv, gate_mode, dt,
+                                      int(bool(qk_l2norm)), _ptr(z), _ptr(norm_weight), float(norm_eps),
+                                      _stream(stream)))
+    return o, hT

@@ -60,7 +60,7 @@ constexpr int OFF_TG = OFF_TB + SZ_C;           // T diag(beta Gamma) [r][i]
 constexpr int OFF_STG = OFF_TG + SZ_C;          // next chunk's K, Q, V as loaded (bf16 [3][64][128])
 constexpr int OFF_GST = OFF_STG + 3 * C * D * 2;// next chunk's g and beta (fp32 [2][64])
 constexpr int OFF_VEC = OFF_GST + 2 * C * 4;    // G, exp(G), exp(G_C - G), beta (64 fp32 each); NQ x 128 fp32 sums
-constexpr int SMEM_BYTES = OFF_VEC + (256 + NQ * 128 + 128) * 4;
+constexpr int SMEM_BYTES = OFF_VEC + (256 + NQ * 128 + 128 + 256) * 4;
 // The scratch of the inverse reuses tiles that are dead while it is live: the
 // fp32 diagonal blocks of A sit in the U' tile, the fp16 inverse T in the diag(e)
 // U' tile, and the fp16 copy of A (an operand of the block-row products) after
@@ -115,6 +115,9 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
     float *sBeta = sG + 192;                               // [64]
     float *sTot = sG + 256;                                // GATE 1: [NQ][128] per-channel sums of each row group
     float *sP2 = sG + 256 + NQ * 128;                      // GATE 1: [128] exp(G_C - G_31)
+    float *sRstd = sP2 + 128;                              // GATE 1, q/k L2 norm: [K rows; Q rows] 1 / |row|
+    float *sNW = sRstd + 128;                              // gated output norm: [128] weight
+    float *sRowSS = sTot;                                  // gated output norm: [64 rows][4] sums of squares
     float *sColf = sG + 256;                               // GATE 0: [4][64] exp(G_16R - G_i)
     const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t aU = smem_u32(sU), aUE = smem_u32(sUE), aS = smem_u32(sS), aM = smem_u32(sM);
@@ -177,6 +180,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
     __shared__ uint64_t ld_bar;
     const uint32_t aBar = smem_u32(&ld_bar);
     if (tid == 0) mbar_init(aBar, 1);
+    if (a.z && tid < D) sNW[tid] = a.norm_w[tid];
     __syncthreads();
     auto issue_loads = [&](int c) {
         const int t0 = c * C, n = min(C, T - t0);
@@ -259,10 +263,17 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 sBeta[tid - 64] = sGst[C + tid - 64];
             }
 #pragma unroll 4
-            for (int idx = tid; idx < 2 * C * 16; idx += NT) {   // K and Q as they are
+            for (int idx = tid; idx < 2 * C * 16; idx += NT) {   // K and Q (a half warp per row)
                 const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
-                *reinterpret_cast<uint4 *>((which ? sQ : sK) + r * LDD + c16 * 8) =
-                    r < n ? bf16x8_to_f16x8(sStg[idx]) : make_uint4(0, 0, 0, 0);
+                const uint4 u = sStg[idx];
+                uint4 h;
+                if (a.qk_l2norm) {
+                    const float ss = halfwarp_sum(bf16x8_sumsq(u));
+                    h = bf16x8_scaled_f16x8(u, rsqrtf(ss + 1e-6f));
+                } else {
+                    h = bf16x8_to_f16x8(u);
+                }
+                *reinterpret_cast<uint4 *>((which ? sQ : sK) + r * LDD + c16 * 8) = r < n ? h : make_uint4(0, 0, 0, 0);
             }
         } else {
             float2 s = make_float2(0.f, 0.f);
@@ -273,6 +284,14 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
             }
             *reinterpret_cast<float2 *>(sTot + ch_h * D + 2 * ch_p) = s;
             if (w == 2 || w == 3) sBeta[tid - 64] = sGst[C + tid - 64];
+            if (a.qk_l2norm) {   // 1 / |row| of the 64 K rows and 64 Q rows, a half warp per row
+#pragma unroll
+                for (int rr = 0; rr < 2 * C / (NT / 16); ++rr) {
+                    const int R = (tid >> 4) + rr * (NT / 16);
+                    const float ss = halfwarp_sum(bf16x8_sumsq(sStg[R * 16 + (tid & 15)]));
+                    if ((tid & 15) == 0) sRstd[R] = rsqrtf(ss + 1e-6f);
+                }
+            }
             __syncthreads();
             float2 off = make_float2(0.f, 0.f);
 #pragma unroll
@@ -305,6 +324,10 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 if (row < n) {
                     kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sStgH + row * D + 2 * ch_p));
                     qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sStgH + C * D + row * D + 2 * ch_p));
+                    if (a.qk_l2norm) {
+                        const float rk = sRstd[row], rq = sRstd[C + row];
+                        kv.x *= rk; kv.y *= rk; qv.x *= rq; qv.y *= rq;
+                    }
                 }
                 const float2 kr = make_float2(kv.x * f1.x, kv.y * f1.y), qr = make_float2(qv.x * f1.x, qv.y * f1.y);
                 const float2 kc = make_float2(kv.x * f2.x, kv.y * f2.y);
@@ -581,6 +604,17 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
         __syncthreads();
 
         // ---------------- O += M U'  and the output rows
+        uint32_t zr[2][NJ];   // gated output norm: this thread's z pairs (rows past n re-read row n - 1)
+        if (a.z) {
+            const __nv_bfloat16 *zp = static_cast<const __nv_bfloat16 *>(a.z) + ((tok0 + t0) * a.Hv + h) * D + dv0;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const long r = min(rw0 + g + 8 * hh, n - 1);
+#pragma unroll
+                for (int j = 0; j < NJ; ++j)
+                    zr[hh][j] = __ldg(reinterpret_cast<const unsigned int *>(zp + r * a.Hv * D + cw0 + 8 * j + 2 * t4));
+            }
+        }
 #pragma unroll
         for (int k0 = 0; k0 < C; k0 += 16) {
             if (k0 > rw0) break;   // M is lower triangular
@@ -593,6 +627,38 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 mma(accO[2 * np], am, bu[0], bu[1]);
                 mma(accO[2 * np + 1], am, bu[2], bu[3]);
             }
+        }
+        if (a.z) {   // o <- o / sqrt(mean(o^2) + eps) * weight * SiLU(z) per row (the CTA has every column)
+            const int r0 = rw0 + g, r1 = rw0 + g + 8;
+            float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                ss0 = fmaf(accO[j][0], accO[j][0], fmaf(accO[j][1], accO[j][1], ss0));
+                ss1 = fmaf(accO[j][2], accO[j][2], fmaf(accO[j][3], accO[j][3], ss1));
+            }
+#pragma unroll
+            for (int off = 1; off < 4; off <<= 1) {
+                ss0 += __shfl_xor_sync(0xffffffffu, ss0, off);
+                ss1 += __shfl_xor_sync(0xffffffffu, ss1, off);
+            }
+            if (t4 == 0) {
+                sRowSS[r0 * NCB + (w >> 2)] = ss0;
+                sRowSS[r1 * NCB + (w >> 2)] = ss1;
+            }
+            __syncthreads();
+            const float4 p0 = *reinterpret_cast<const float4 *>(sRowSS + r0 * NCB);
+            const float4 p1 = *reinterpret_cast<const float4 *>(sRowSS + r1 * NCB);
+            const float rs[2] = {rsqrtf((p0.x + p0.y + p0.z + p0.w) * (1.f / D) + a.norm_eps),
+                                 rsqrtf((p1.x + p1.y + p1.z + p1.w) * (1.f / D) + a.norm_eps)};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    const int c = cw0 + 8 * j + 2 * t4;
+                    const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[hh][j]));
+                    accO[j][2 * hh] *= rs[hh] * sNW[c] * (zf.x / (1.f + __expf(-zf.x)));
+                    accO[j][2 * hh + 1] *= rs[hh] * sNW[c + 1] * (zf.y / (1.f + __expf(-zf.y)));
+                }
         }
         {   // o rows -> [DVC / EPB][64 rows][128 B] boxes in the 128-byte swizzle the TMA
             // store expects, over the dead V and W tiles
@@ -766,7 +832,8 @@ cudaError_t launch_g(const FwdArgs &a, cudaStream_t st)
     // unit is split; when the units past one wave fit as halves in a second, those are.
     const long units = (long)a.B * a.Hv, sms = sm_count();
     long n_whole = units;
-    if (2 * units <= sms) n_whole = 0;
+    if (a.z) n_whole = units;   // the gated output norm needs every column of a row in one CTA
+    else if (2 * units <= sms) n_whole = 0;
     else if (units > sms && 2 * (units - sms) <= sms) n_whole = sms;
     CUtensorMap mq, mk, mv1, mv2, mo;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens

@@ -173,6 +173,50 @@ int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, const fl
     return GDR_OK;
 }
 
+int gdr_fwd_chunked_norm(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                         const float *h0, void *o, float *hT, const int *cu_seqlens, int B, int T, int Hk, int Hv,
+                         int Dk, int Dv, int gate_mode, int dtype, int qk_l2norm, const void *z,
+                         const float *norm_weight, float norm_eps, void *stream)
+{
+    int st = check_common(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (st != GDR_OK) return st;
+    if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return fail(GDR_ERR_MISALIGNED, "cu_seqlens is not 4-byte aligned");
+    const bool work = B > 0 && T > 0;
+    if (work && (!q || !k || !v || !g || !beta || !o))
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta and o must be non-NULL");
+    if (z && !norm_weight) return fail(GDR_ERR_INVALID_ARG, "norm_weight must be non-NULL when z is given");
+    if (!(norm_eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "norm_eps must be non-negative");
+    const void *ptrs[] = {q, k, v, g, beta, h0, o, hT, z};
+    const char *names[] = {"q", "k", "v", "g", "beta", "h0", "o", "hT", "z"};
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if ((uintptr_t)norm_weight & 3u) return fail(GDR_ERR_MISALIGNED, "norm_weight is not 4-byte aligned");
+    if (o && (o == q || o == k || o == v || o == z)) return fail(GDR_ERR_INVALID_ARG, "o must not alias q, k, v or z");
+    gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    a.cu_seqlens = cu_seqlens;
+    a.qk_l2norm = qk_l2norm != 0;
+    a.z = z;
+    a.norm_w = norm_weight;
+    a.norm_eps = norm_eps;
+    if (!gdr::fused_supported(a))
+        return fail(GDR_ERR_UNSUPPORTED, "the fused options need bf16 inputs and Dk = Dv = 128");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!work) {
+        if (hT && B > 0) {
+            const size_t bytes = (size_t)B * Hv * Dk * Dv * sizeof(float);
+            cudaError_t e = h0 ? (h0 == hT ? cudaSuccess
+                                           : cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, s))
+                               : cudaMemsetAsync(hT, 0, bytes, s);
+            if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA: %s", cudaGetErrorString(e));
+        }
+        return GDR_OK;
+    }
+    cudaError_t e = gdr::launch_fwd_fused(a, s);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += 1;
+    return GDR_OK;
+}
+
 int gdr_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
                     float *state, void *o, int B, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype,
                     void *stream)

@@ -26,6 +26,13 @@ struct FwdArgs {
     // Packed variable-length input (fused kernel only): B sequences packed along one
     // token axis of length T; sequence n is tokens [cu_seqlens[n], cu_seqlens[n + 1]).
     const int *cu_seqlens = nullptr;
+    // Fused kernel only. qk_l2norm: q and k rows are divided by sqrt(sum of squares + 1e-6)
+    // as they are loaded. z: when set ([B, T, Hv, Dv] bf16, like o), o receives
+    // o / sqrt(mean(o^2) + norm_eps) * norm_w * SiLU(z) per row of Dv (norm_w [Dv] fp32).
+    int qk_l2norm = 0;
+    const void *z = nullptr;
+    const float *norm_w = nullptr;
+    float norm_eps = 0.f;
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);

@@ -172,6 +172,42 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u)
     return r;
 }
 
+// Sum of squares of 8 bf16 values.
+__device__ __forceinline__ float bf16x8_sumsq(uint4 u)
+{
+    const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p[e]);
+        s = fmaf(f.x, f.x, fmaf(f.y, f.y, s));
+    }
+    return s;
+}
+
+// 8 bf16 values times `scale`, rounded to fp16.
+__device__ __forceinline__ uint4 bf16x8_scaled_f16x8(uint4 u, float scale)
+{
+    const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    uint4 r;
+    uint32_t *q = reinterpret_cast<uint32_t *>(&r);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p[e]);
+        const __half2 hh = __floats2half2_rn(f.x * scale, f.y * scale);
+        q[e] = *reinterpret_cast<const uint32_t *>(&hh);
+    }
+    return r;
+}
+
+// Sum over the 16 lanes of a half warp (all 32 lanes take part).
+__device__ __forceinline__ float halfwarp_sum(float s)
+{
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return s;
+}
+
 // The driver's tensor-map encoder, looked up through the runtime once, so the
 // library needs no link-time dependency on the driver library.
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,

@@ -164,6 +164,32 @@ GDR_API int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, 
                            int gate_mode, int dtype, void *stream);
 
 /*
+ * Chunked forward with the layer's normalisations fused into the kernel
+ * (NextTransformer "Source notes", section "Linear attention": L2-normalized
+ * Q/K in rows deltanet and kda; the GDN output RMSNorm x gain x SiLU gate in
+ * row gdn; "Backend and numerical limits": a gated RMSNorm on the output).
+ *
+ * Arguments as gdr_fwd_chunked, plus:
+ * - cu_seqlens: NULL, or packed sequences exactly as gdr_fwd_chunked_varlen (B
+ *   is then N and T is T_total; q, k [T, Hk, Dk] and so on).
+ * - qk_l2norm: non-zero to divide every q and k row (one head of one token) by
+ *   sqrt(sum of squares + 1e-6) as it is loaded.
+ * - z: NULL, or the output gate [B, T, Hv, Dv] bf16 (the layout of o). Then o
+ *   receives o / sqrt(mean(o^2) + norm_eps) * norm_weight * SiLU(z) per row of
+ *   Dv, where o is the recurrence's output; norm_weight [Dv] fp32 is required.
+ *
+ * Runs only on the fused kernel: bf16 inputs (GDR_BF16 or GDR_BF16_OUT_F32)
+ * with Dk = Dv = 128, else GDR_ERR_UNSUPPORTED. No workspace. A call with z
+ * keeps each (b, h) in one CTA. Pointers 16-byte aligned (norm_weight 4-byte,
+ * cu_seqlens 4-byte); o must not alias q, k, v or z.
+ */
+GDR_API int gdr_fwd_chunked_norm(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *h0, void *o, float *hT,
+                                 const int *cu_seqlens, int B, int T, int Hk, int Hv, int Dk, int Dv,
+                                 int gate_mode, int dtype, int qk_l2norm, const void *z,
+                                 const float *norm_weight, float norm_eps, void *stream);
+
+/*
  * One decode step for B independent sequences (the recurrence with T = 1):
  *   S' = diag(exp(g)) S;  u = beta (v - S'^T k);  S <- S' + k u^T;  o = S^T q.
  * state [B, Hv, Dk, Dv] fp32 is read and overwritten in place; q, k [B, Hk, Dk],
