@@ -58,6 +58,8 @@ def algorithmic_bytes(w):
     decode workload, per step: the state read and written once, and one token's inputs
     and output for every (batch row, value head)."""
     es = 2 if w.dtype == "bf16" else 4
+    if w.layer:
+        return layer_conv_bytes(w) + algorithmic_bytes(w.with_(layer=False)) + w.B * w.T * w.Hv * w.Dv * es
     if w.decode:
         tok = w.B * (2 * w.Hk * w.Dk * es + 2 * w.Hv * w.Dv * es
                      + w.Hv * (w.Dk if w.gate == "channel" else 1) * 4 + w.Hv * 4)
@@ -68,6 +70,12 @@ def algorithmic_bytes(w):
     beta = w.B * w.T * w.Hv * 4
     states = (2 if w.h0_std > 0 else 1) * w.B * w.Hv * w.Dk * w.Dv * 4
     return qk + vo + g + beta + states
+
+
+def layer_conv_bytes(w):
+    """The short convolution reads the q/k/v projections once and writes them once."""
+    es = 2 if w.dtype == "bf16" else 4
+    return 2 * w.B * w.T * (2 * w.Hk * w.Dk + w.Hv * w.Dv) * es
 
 
 def measured_peaks():
@@ -218,12 +226,159 @@ def cpu_oracle_sample(w, target_s=12.0, seed_rank=0):
     }
 
 
+def layer_oracle_unit(inp, b, h):
+    """The oracle composition for one (b, h) unit of the layer: the short convolution of the
+    unit's q, k and v channels, L2 norms of q and k, the fp64 recurrence, the gated RMSNorm."""
+    import oracle
+    from oracle import prologue
+    D = inp["z"].shape[-1]
+    Hk, Hv = inp["xq"].shape[-1] // D, inp["z"].shape[2]
+    hk = h // (Hv // Hk)
+    sl = lambda n, hh: inp[n][b:b + 1, :, hh * D:(hh + 1) * D]
+    wsl = lambda n, hh: inp[n][hh * D:(hh + 1) * D]
+    q, _ = prologue.causal_conv_silu(sl("xq", hk), wsl("wq", hk))
+    k, _ = prologue.causal_conv_silu(sl("xk", hk), wsl("wk", hk))
+    v, _ = prologue.causal_conv_silu(sl("xv", h), wsl("wv", h))
+    q, k = prologue.l2norm(q), prologue.l2norm(k)
+    h0 = None if inp["h0"] is None else inp["h0"][b:b + 1, h:h + 1]
+    o, hT = oracle.recurrent(q[:, :, None], k[:, :, None], v[:, :, None], inp["g"][b:b + 1, :, h:h + 1],
+                             inp["beta"][b:b + 1, :, h:h + 1], h0, nthreads=1)
+    return prologue.rmsnorm_gated(o[0, :, 0], inp["z"][b, :, h], inp["nw"]), hT
+
+
+def layer_cpu_sample(w, target_s=12.0, seed_rank=0):
+    """Time the oracle composition on whole sequences of (b, h) units for about target_s."""
+    from gated_delta_rule_68_b200.workloads import make_layer_inputs
+    inp = make_layer_inputs(w.with_(seed=w.seed + seed_rank), "cpu")
+    units, dt = 0, 0.0
+    while units == 0 or (dt < target_s and units < w.B * w.Hv):
+        b, h = divmod(units, w.Hv)
+        t0 = time.perf_counter()
+        layer_oracle_unit(inp, b, h)
+        dt += time.perf_counter() - t0
+        units += 1
+    return {"value": units * w.T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{units} whole (batch row, value head) sequences of T={w.T}: conv + SiLU, L2 norms, "
+                      f"fp64 token recurrence, gated RMSNorm, one thread; {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_layer_bench(args, w, wr, rank, world, local, dev):
+    """One step = the layer's recurrence block: three short convolutions (+ SiLU) of the q/k/v
+    projections, then the fused chunked forward with in-kernel q/k L2 norms and the gated
+    output RMSNorm."""
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_68_b200 as gdr
+    from gated_delta_rule_68_b200.workloads import make_layer_inputs
+
+    inp_cpu = make_layer_inputs(wr, "cpu")
+    inp = {n: (None if t is None else t.to(dev)) for n, t in inp_cpu.items()}
+    yq, yk, yv = (torch.empty_like(inp[n]) for n in ("xq", "xk", "xv"))
+    o = torch.empty((w.B, w.T, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)
+    hT = torch.empty((w.B, w.Hv, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    shp_k, shp_v = (w.B, w.T, w.Hk, w.Dk), (w.B, w.T, w.Hv, w.Dv)
+
+    def convs(x):
+        gdr.gdr_causal_conv_silu(x["xq"], x["wq"], y=yq, stream=stream)
+        gdr.gdr_causal_conv_silu(x["xk"], x["wk"], y=yk, stream=stream)
+        gdr.gdr_causal_conv_silu(x["xv"], x["wv"], y=yv, stream=stream)
+
+    def layer(x):
+        convs(x)
+        gdr.gdr_fwd_chunked_norm(yq.view(shp_k), yk.view(shp_k), yv.view(shp_v), x["g"], x["beta"], x["h0"],
+                                 qk_l2norm=True, z=x["z"], norm_weight=x["nw"], o=o, hT=hT, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, steps):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    for _ in range(args.warmup):
+        layer(inp)
+    torch.cuda.synchronize()
+    n0 = gdr.gdr_kernel_launches()
+    with ClockSampler(local) as clk:
+        ms = timed(lambda: layer(inp), args.steps)
+    launches = gdr.gdr_kernel_launches() - n0
+    ms_max = max_over_ranks(ms, dev)
+    conv_ms = timed(lambda: convs(inp), args.steps)
+    fwd_ms = ms - conv_ms
+
+    e2e = None
+    if not args.no_e2e:
+        host = {n: (None if x is None else x.pin_memory()) for n, x in inp_cpu.items()}
+        dbuf = {n: (None if x is None else torch.empty_like(x, device=dev)) for n, x in inp_cpu.items()}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hT_h = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
+        d2h = o_h.numel() * o_h.element_size() + hT_h.numel() * hT_h.element_size()
+
+        def e2e_step():
+            for n, x in host.items():
+                if x is not None:
+                    dbuf[n].copy_(x, non_blocking=True)
+            layer(dbuf)
+            o_h.copy_(o, non_blocking=True)
+            hT_h.copy_(hT, non_blocking=True)
+
+        e2e_step()
+        e2e_steps = max(3, min(args.steps, 10))
+        te = max_over_ranks(timed(e2e_step, e2e_steps), dev)
+        e2e = {"value": job_tokens_per_s(w.head_tokens, world, te), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": te}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peaks()
+    alg, conv_alg = algorithmic_bytes(w), layer_conv_bytes(w)
+    fwd_alg = alg - conv_alg
+    cpu = layer_cpu_sample(w) if world == 1 and not args.no_cpu_baseline else None
+    line = {
+        "metric": METRIC, "value": job_tokens_per_s(w.head_tokens, world, ms_max), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded CPU generator; q/k/v projections N(0,1), conv taps 0.5 N(0,1); "
+                f"g logsigmoid(N({w.g_mu:g},1)); beta sigmoid(N(0,1)); h0 0.02 N(0,1); z N(0,1))",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "hbm", "achieved": fwd_alg / (fwd_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": fwd_alg / (fwd_ms / 1e3) / 1e9 / peak, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": fwd_alg, "traffic": None,
+                     "kernel": "gdr_fwd_chunked_norm (q/k L2 norm and gated output norm fused)"},
+        "step_roofline": {"achieved": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peak,
+                          "algorithmic_bytes": alg},
+        "conv": {"ms_per_step": conv_ms, "launches_per_step": 3, "algorithmic_bytes": conv_alg,
+                 "achieved_gbs": conv_alg / (conv_ms / 1e3) / 1e9,
+                 "frac": conv_alg / (conv_ms / 1e3) / 1e9 / peak},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "launches_per_step": launches / args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
     import oracle
     from gated_delta_rule_68_b200.workloads import make_inputs
 
+    if w.layer:
+        return run_layer_reference(args, w, world)
     cores = oracle.threads_used(0, 1 << 30)
     units = max(cores, 8)
     sample = w.with_(B=units, Hk=1, Hv=1)
@@ -249,6 +404,35 @@ def run_reference(args, w, rank, world):
                          "kind": "oracle",
                          "sample": f"each step: {units} whole (batch row, value head) sequences of "
                                    f"T={w.T} of the workload, fp64 token recurrence"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_layer_reference(args, w, world):
+    """The reference arm on the layer workload: each step is the oracle composition on two whole
+    (b, h) sequences, on one host core."""
+    from gated_delta_rule_68_b200.workloads import make_layer_inputs
+    inp = make_layer_inputs(w, "cpu")
+    units = 2
+    times = []
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        for u in range(units):
+            layer_oracle_unit(inp, *divmod(u, w.Hv))
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    value = units * w.T / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same recipe as the GPU arm)", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {units} whole (batch row, value head) sequences of T={w.T}: "
+                                   "conv + SiLU, L2 norms, fp64 token recurrence, gated RMSNorm"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -384,6 +568,8 @@ def main(argv=None):
     wr = rank_workload(w, rank)
     if w.decode:
         return run_decode_bench(args, w, wr, rank, world, local, dev)
+    if w.layer:
+        return run_layer_bench(args, w, wr, rank, world, local, dev)
     inp_cpu = make_inputs(wr, "cpu")
     inp = {n: (None if t is None else t.to(dev)) for n, t in inp_cpu.items()}
     o = torch.empty((w.B, w.T, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)

@@ -88,7 +88,8 @@ __device__ unsigned int g_fused_range_errors;
 // inverse and W are computed by each.
 template <typename TOut, int GATE, int NS>
 __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *map_q, const CUtensorMap *map_k,
-                                           const CUtensorMap *map_v, const CUtensorMap *map_o, int bh, int split)
+                                           const CUtensorMap *map_v, const CUtensorMap *map_o,
+                                           const CUtensorMap *map_z, int bh, int split)
 {
     constexpr int DVC = D / NS;      // value columns of this CTA
     constexpr int NJ = DVC / NCB / 8;   // n8 tiles of a warp in the [64 x DVC] products
@@ -177,9 +178,12 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
     // Chunk c's K, Q tiles and this CTA's V columns -> bf16 staging by three TMA box
     // loads that complete on ld_bar (tokens past T read as zero); beta, and the
     // scalar gate, by 4-byte asynchronous copies.
-    __shared__ uint64_t ld_bar;
-    const uint32_t aBar = smem_u32(&ld_bar);
-    if (tid == 0) mbar_init(aBar, 1);
+    __shared__ uint64_t ld_bar, z_bar;
+    const uint32_t aBar = smem_u32(&ld_bar), aZBar = smem_u32(&z_bar);
+    if (tid == 0) {
+        mbar_init(aBar, 1);
+        mbar_init(aZBar, 1);
+    }
     if (a.z && tid < D) sNW[tid] = a.norm_w[tid];
     __syncthreads();
     auto issue_loads = [&](int c) {
@@ -556,6 +560,15 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
         // GATE 1: an fp16 operand of this chunk left the fp16 range (its results are not valid)
         if (__syncthreads_or(bad) && tid == 0 && split == 0)   // once per (unit, chunk)
             atomicAdd(&g_fused_range_errors, 1u);
+        // Gated output norm: the chunk's z tile into the V tile (dead from here on), in the
+        // 128-byte swizzle of a bf16 o tile, so that each thread later finds its z values
+        // where it writes its outputs.
+        if (a.z && tid == NT - 32) {
+            mbar_expect_tx(aZBar, C * D * 2);
+#pragma unroll
+            for (int bx = 0; bx < D / 64; ++bx)
+                tma_load_4d(smem_u32(sm + OFF_V + bx * C * 128), map_z, 64 * bx, h, tt0 + t0, tb, aZBar);
+        }
 
         // ---------------- U' = U - W S,  O1 = Q S (GATE 0: then scaled by Gamma_r;
         // GATE 1: Q already carries Gamma), K-dim dk. The fragments of step ks + 1
@@ -601,20 +614,16 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 }
             }
         }
-        __syncthreads();
+        if (a.z) {   // the barrier also waits for the z tile (issued after W/U)
+            if (!__syncthreads_and(mbar_wait_bounded(aZBar, ch & 1))) {
+                if (tid == 0) atomicAdd(&g_fused_load_timeouts, 1u);
+                return;
+            }
+        } else {
+            __syncthreads();
+        }
 
         // ---------------- O += M U'  and the output rows
-        uint32_t zr[2][NJ];   // gated output norm: this thread's z pairs (rows past n re-read row n - 1)
-        if (a.z) {
-            const __nv_bfloat16 *zp = static_cast<const __nv_bfloat16 *>(a.z) + ((tok0 + t0) * a.Hv + h) * D + dv0;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const long r = min(rw0 + g + 8 * hh, n - 1);
-#pragma unroll
-                for (int j = 0; j < NJ; ++j)
-                    zr[hh][j] = __ldg(reinterpret_cast<const unsigned int *>(zp + r * a.Hv * D + cw0 + 8 * j + 2 * t4));
-            }
-        }
 #pragma unroll
         for (int k0 = 0; k0 < C; k0 += 16) {
             if (k0 > rw0) break;   // M is lower triangular
@@ -630,6 +639,13 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
         }
         if (a.z) {   // o <- o / sqrt(mean(o^2) + eps) * weight * SiLU(z) per row (the CTA has every column)
             const int r0 = rw0 + g, r1 = rw0 + g + 8;
+            uint32_t zr[2][NJ];   // read before the barrier below: an fp32 o tile overwrites other rows' z
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int j = 0; j < NJ; ++j)
+                    zr[hh][j] = *reinterpret_cast<const uint32_t *>(
+                        sm + OFF_V + o_swz<__nv_bfloat16>(rw0 + g + 8 * hh, cw0 + 8 * j + 2 * t4));
             float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
@@ -656,8 +672,8 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 for (int j = 0; j < NJ; ++j) {
                     const int c = cw0 + 8 * j + 2 * t4;
                     const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zr[hh][j]));
-                    accO[j][2 * hh] *= rs[hh] * sNW[c] * (zf.x / (1.f + __expf(-zf.x)));
-                    accO[j][2 * hh + 1] *= rs[hh] * sNW[c + 1] * (zf.y / (1.f + __expf(-zf.y)));
+                    accO[j][2 * hh] *= rs[hh] * sNW[c] * __fdividef(zf.x, 1.f + __expf(-zf.x));
+                    accO[j][2 * hh + 1] *= rs[hh] * sNW[c + 1] * __fdividef(zf.y, 1.f + __expf(-zf.y));
                 }
         }
         {   // o rows -> [DVC / EPB][64 rows][128 B] boxes in the 128-byte swizzle the TMA
@@ -768,14 +784,15 @@ template <typename TOut, int GATE>
 __global__ void __launch_bounds__(NT, 1)
 fused_fwd_kernel(FwdArgs a, int n_whole, const __grid_constant__ CUtensorMap map_q,
                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v1,
-                 const __grid_constant__ CUtensorMap map_v2, const __grid_constant__ CUtensorMap map_o)
+                 const __grid_constant__ CUtensorMap map_v2, const __grid_constant__ CUtensorMap map_o,
+                 const __grid_constant__ CUtensorMap map_z)
 {
     const int blk = blockIdx.x;
     if (blk < n_whole) {
-        fused_unit<TOut, GATE, 1>(a, &map_q, &map_k, &map_v1, &map_o, blk, 0);
+        fused_unit<TOut, GATE, 1>(a, &map_q, &map_k, &map_v1, &map_o, &map_z, blk, 0);
     } else {
         const int i = blk - n_whole;
-        fused_unit<TOut, GATE, 2>(a, &map_q, &map_k, &map_v2, &map_o, n_whole + i / 2, i % 2);
+        fused_unit<TOut, GATE, 2>(a, &map_q, &map_k, &map_v2, &map_o, &map_z, n_whole + i / 2, i % 2);
     }
 }
 
@@ -835,18 +852,20 @@ cudaError_t launch_g(const FwdArgs &a, cudaStream_t st)
     if (a.z) n_whole = units;   // the gated output norm needs every column of a row in one CTA
     else if (2 * units <= sms) n_whole = 0;
     else if (units > sms && 2 * (units - sms) <= sms) n_whole = sms;
-    CUtensorMap mq, mk, mv1, mv2, mo;
+    CUtensorMap mq, mk, mv1, mv2, mo, mz;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
     if (!make_map(&mq, a.q, mb, a.T, a.Hk, D) || !make_map(&mk, a.k, mb, a.T, a.Hk, D) ||
         !make_map(&mv1, a.v, mb, a.T, a.Hv, D) || !make_map(&mv2, a.v, mb, a.T, a.Hv, D / 2) ||
         !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
+        return cudaErrorInvalidValue;
+    if (a.z ? !make_map(&mz, a.z, mb, a.T, a.Hv, 64, false, true) : (mz = mo, false))   // z: the bf16 o box
         return cudaErrorInvalidValue;
     const int smem = SMEM_BYTES + 1024;
     auto kernel = fused_fwd_kernel<TOut, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const long grid = n_whole + 2 * (units - n_whole);
-    kernel<<<(unsigned)grid, NT, smem, st>>>(a, (int)n_whole, mq, mk, mv1, mv2, mo);
+    kernel<<<(unsigned)grid, NT, smem, st>>>(a, (int)n_whole, mq, mk, mv1, mv2, mo, mz);
     return cudaGetLastError();
 }
 

@@ -286,9 +286,8 @@ int gdr_rmsnorm_gated(const void *o, const void *z, const float *weight, void *y
     if (!(eps >= 0.f)) return fail(GDR_ERR_INVALID_ARG, "eps must be non-negative");
     if (rows == 0) return GDR_OK;
     if (!o || !z || !weight || !y) return fail(GDR_ERR_INVALID_ARG, "o, z, weight and y must be non-NULL");
-    const uintptr_t es = dtype == GDR_FP32 ? 4 : 2;
-    if (((uintptr_t)o % es) || ((uintptr_t)z % es) || ((uintptr_t)y % es) || ((uintptr_t)weight & 3u))
-        return fail(GDR_ERR_MISALIGNED, "a pointer is not aligned to its element size");
+    if (!aligned16(o) || !aligned16(z) || !aligned16(y) || ((uintptr_t)weight & 3u))
+        return fail(GDR_ERR_MISALIGNED, "o, z and y must be 16-byte aligned, weight 4-byte aligned");
     gdr::NormArgs a;
     a.o = o; a.z = z; a.w = weight; a.y = y; a.rows = rows; a.D = D; a.eps = eps; a.fp32 = dtype == GDR_FP32;
     cudaError_t e = gdr::launch_rmsnorm_gated(a, (cudaStream_t)stream);

@@ -14,7 +14,7 @@ namespace gdr {
 namespace {
 
 constexpr int CONV_W = 4;     // taps; tap CONV_W - 1 sits on the current token
-constexpr int CONV_RUN = 16;  // consecutive tokens per thread
+constexpr int CONV_RUN = 8;   // consecutive tokens per thread
 constexpr int CONV_TPB = 256;
 
 struct Vec8 { float v[8]; };
@@ -56,7 +56,7 @@ __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ void from_f(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void from_f(float *p, float x) { *p = x; }
 
-__device__ __forceinline__ float silu(float y) { return y / (1.f + __expf(-y)); }
+__device__ __forceinline__ float silu(float y) { return __fdividef(y, 1.f + __expf(-y)); }
 
 // Sequence n of the token axis: [s0, s1). Without cu_seqlens, sequence n is
 // tokens n*T .. n*T + T - 1.
@@ -66,24 +66,58 @@ struct Seqs {
     __device__ int start(int i) const { return cu ? cu[i] : i * T; }
 };
 
+// 8 channels of one token as loaded (bf16: one 16-byte word; fp32: two), unpacked on use.
+template <typename T_> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+    __device__ float get(int i) const
+    {
+        const __nv_bfloat162 h = reinterpret_cast<const __nv_bfloat162 *>(&u)[i >> 1];
+        return (i & 1) ? __high2float(h) : __low2float(h);
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ void load(const float *p)
+    {
+        a = *reinterpret_cast<const float4 *>(p);
+        b = *reinterpret_cast<const float4 *>(p + 4);
+    }
+    __device__ float get(int i) const
+    {
+        const float4 &q = i < 4 ? a : b;
+        const int j = i & 3;
+        return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
+    }
+};
+
 // Thread (run, group): channels 8 group .. 8 group + 7 of tokens run*RUN ..
-// run*RUN + RUN - 1 of the flattened token axis. The last CONV_W - 1 inputs
-// of the current sequence ride along in registers; at a sequence's first token
-// they come from state_in (or are zero).
+// run*RUN + RUN - 1 of the flattened token axis. The run's inputs and the
+// CONV_W - 1 before it are loaded first (all loads in flight together); the
+// taps then walk the run in registers. At a sequence's first token the history
+// comes from state_in (or is zero).
 template <typename T_>
 __global__ void __launch_bounds__(CONV_TPB)
 conv_silu_kernel(const T_ *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
                  const T_ *__restrict__ state_in, T_ *__restrict__ state_out, T_ *__restrict__ y, Seqs sq,
                  long rows, int Ch)
 {
+    constexpr int H = CONV_W - 1;
     const int ngroups = Ch / 8;
     const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
     const int grp = (int)(gid % ngroups);
     const long t0 = (gid / ngroups) * CONV_RUN;
     if (t0 >= rows) return;
-    const long t1 = min(t0 + (long)CONV_RUN, rows);
+    const int nt = (int)min((long)CONV_RUN, rows - t0);
     const int c0 = 8 * grp;
 
+    Raw8<T_> xr[H + CONV_RUN];   // tokens t0 - H .. t0 + RUN - 1 (addresses clamped into the axis)
+#pragma unroll
+    for (int i = 0; i < H + CONV_RUN; ++i) {
+        const long t = min(max(t0 - H + i, 0L), rows - 1);
+        xr[i].load(x + (size_t)t * Ch + c0);
+    }
     float wt[8][CONV_W], bs[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -99,55 +133,55 @@ conv_silu_kernel(const T_ *__restrict__ x, const float *__restrict__ w, const fl
     }
     int n = lo;
     long s0 = sq.start(n), s1 = sq.start(n + 1);
-    // history: the CONV_W - 1 inputs before t0 in the sequence's virtual axis
+    // history of token t: the H inputs before it in the sequence's virtual axis
     // [state_in (oldest first) ; x[s0] ; x[s0 + 1] ; ...]
-    float h[CONV_W - 1][8];
-    auto fill_history = [&](long t) {
+    float h[H][8];
+    auto fill_history = [&](int u) {   // token t0 + u (u a compile-time index)
 #pragma unroll
-        for (int j = 0; j < CONV_W - 1; ++j) {
-            const long vt = t - s0 + j;   // virtual index of the input CONV_W - 1 - j tokens back
-            if (vt >= CONV_W - 1) {
-                const Vec8 a = load8(x + (size_t)(s0 + vt - (CONV_W - 1)) * Ch + c0);
+        for (int j = 0; j < H; ++j) {
+            const long vt = t0 + u - s0 + j;   // virtual index of the input H - j tokens back
 #pragma unroll
-                for (int i = 0; i < 8; ++i) h[j][i] = a.v[i];
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    h[j][i] = state_in ? to_f(state_in[((size_t)n * Ch + c0 + i) * (CONV_W - 1) + vt]) : 0.f;
+            for (int i = 0; i < 8; ++i) {
+                float v = 0.f;
+                if (vt >= H) {
+                    v = xr[u + j].get(i);   // token t0 + u - H + j, preloaded
+                } else if (state_in) {
+                    v = to_f(state_in[((size_t)n * Ch + c0 + i) * H + vt]);
+                }
+                h[j][i] = v;
             }
         }
     };
-    fill_history(t0);
-    for (long t = t0; t < t1; ++t) {
+    fill_history(0);
+#pragma unroll
+    for (int u = 0; u < CONV_RUN; ++u) {
+        if (u >= nt) break;
+        const long t = t0 + u;
         while (t >= s1) {   // next sequence (skipping empty ones)
             ++n;
             s0 = s1;
             s1 = sq.start(n + 1);
-            if (t < s1) fill_history(t);
+            if (t < s1) fill_history(u);
         }
-        const Vec8 xt = load8(x + (size_t)t * Ch + c0);
         Vec8 o;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
+            const float xi = xr[H + u].get(i);
             float acc = bs[i];
 #pragma unroll
-            for (int j = 0; j < CONV_W - 1; ++j) acc = fmaf(wt[i][j], h[j][i], acc);
-            acc = fmaf(wt[i][CONV_W - 1], xt.v[i], acc);
+            for (int j = 0; j < H; ++j) acc = fmaf(wt[i][j], h[j][i], acc);
+            acc = fmaf(wt[i][H], xi, acc);
             o.v[i] = silu(acc);
+#pragma unroll
+            for (int j = 0; j < H - 1; ++j) h[j][i] = h[j + 1][i];
+            h[H - 1][i] = xi;
         }
         store8(y + (size_t)t * Ch + c0, o);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-#pragma unroll
-            for (int j = 0; j < CONV_W - 2; ++j) h[j][i] = h[j + 1][i];
-            h[CONV_W - 2][i] = xt.v[i];
-        }
         if (state_out && t == s1 - 1) {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < CONV_W - 1; ++j)
-                    from_f(&state_out[((size_t)n * Ch + c0 + i) * (CONV_W - 1) + j], h[j][i]);
+                for (int j = 0; j < H; ++j) from_f(&state_out[((size_t)n * Ch + c0 + i) * H + j], h[j][i]);
         }
     }
 }
@@ -165,7 +199,56 @@ __global__ void conv_state_empty_kernel(const T_ *__restrict__ state_in, T_ *__r
     state_out[i] = state_in ? state_in[i] : T_(0.f);
 }
 
-// One warp per row of D = 32 * PER elements.
+// One warp per row of D = 32 * PER elements; lane l owns elements PER l .. PER l + PER - 1.
+template <typename T_, int PER> struct RowVec;
+template <> struct RowVec<__nv_bfloat16, 4> {
+    static __device__ void load(const __nv_bfloat16 *p, float *v)
+    {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+    }
+    static __device__ void store(__nv_bfloat16 *p, const float *v)
+    {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t *>(&a);
+        u.y = *reinterpret_cast<const uint32_t *>(&b);
+        *reinterpret_cast<uint2 *>(p) = u;
+    }
+};
+template <> struct RowVec<__nv_bfloat16, 2> {
+    static __device__ void load(const __nv_bfloat16 *p, float *v)
+    {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+        v[0] = a.x; v[1] = a.y;
+    }
+    static __device__ void store(__nv_bfloat16 *p, const float *v)
+    {
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v[0], v[1]);
+    }
+};
+template <> struct RowVec<float, 4> {
+    static __device__ void load(const float *p, float *v)
+    {
+        const float4 a = *reinterpret_cast<const float4 *>(p);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    }
+    static __device__ void store(float *p, const float *v)
+    {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+template <> struct RowVec<float, 2> {
+    static __device__ void load(const float *p, float *v)
+    {
+        const float2 a = *reinterpret_cast<const float2 *>(p);
+        v[0] = a.x; v[1] = a.y;
+    }
+    static __device__ void store(float *p, const float *v) { *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]); }
+};
+
 template <typename T_, int PER>
 __global__ void __launch_bounds__(256)
 rmsnorm_gated_kernel(const T_ *__restrict__ o, const T_ *__restrict__ z, const float *__restrict__ wt,
@@ -177,11 +260,8 @@ rmsnorm_gated_kernel(const T_ *__restrict__ o, const T_ *__restrict__ z, const f
     constexpr int D = 32 * PER;
     const size_t base = (size_t)row * D + lane * PER;
     float ov[PER], zv[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        ov[i] = to_f(o[base + i]);
-        zv[i] = to_f(z[base + i]);
-    }
+    RowVec<T_, PER>::load(o + base, ov);
+    RowVec<T_, PER>::load(z + base, zv);
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) ss = fmaf(ov[i], ov[i], ss);
@@ -189,7 +269,8 @@ rmsnorm_gated_kernel(const T_ *__restrict__ o, const T_ *__restrict__ z, const f
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     const float rstd = rsqrtf(ss / D + eps);
 #pragma unroll
-    for (int i = 0; i < PER; ++i) from_f(&y[base + i], ov[i] * rstd * wt[lane * PER + i] * silu(zv[i]));
+    for (int i = 0; i < PER; ++i) ov[i] = ov[i] * rstd * wt[lane * PER + i] * silu(zv[i]);
+    RowVec<T_, PER>::store(y + base, ov);
 }
 
 template <typename T_>

@@ -41,6 +41,7 @@ class Workload:
     h0_std: float       # 0.0 means h0 absent (zeros)
     seed: int
     decode: bool = False
+    layer: bool = False   # inputs are the raw q/k/v projections of the layer (make_layer_inputs)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -70,6 +71,9 @@ WORKLOADS = {
     "decode_bf16": Workload("decode_bf16", B=256, T=512, Hk=16, Hv=48, Dk=128, Dv=128,
                             gate="scalar", dtype="bf16", g_mu=3.0, h0_std=0.02, seed=4,
                             decode=True),
+    "gdn_layer_bf16": Workload("gdn_layer_bf16", B=8, T=2048, Hk=16, Hv=16, Dk=128, Dv=128,
+                               gate="scalar", dtype="bf16", g_mu=3.0, h0_std=0.02, seed=5,
+                               layer=True),
 }
 
 
@@ -100,6 +104,36 @@ def make_inputs(w: Workload, device="cpu"):
     beta = torch.sigmoid(randn(*lead, w.Hv))
     h0 = (randn(w.B, w.Hv, w.Dk, w.Dv) * w.h0_std) if w.h0_std > 0 else None
     out = dict(q=q, k=k, v=v, g=g, beta=beta, h0=h0)
+    if device != "cpu":
+        out = {n: (None if t is None else t.to(device)) for n, t in out.items()}
+    return out
+
+
+def make_layer_inputs(w: Workload, device="cpu"):
+    """The layer around the recurrence, drawn in this order from one generator:
+
+      xq, xk ~ N(0, 1) [B, T, Hk*Dk], xv ~ N(0, 1) [B, T, Hv*Dv] (bf16): the q/k/v
+             projections before the short convolution
+      wq, wk [Hk*Dk, 4], wv [Hv*Dv, 4] = 0.5 N(0, 1) (fp32): the convolution taps
+      g, beta, h0 as in make_inputs
+      z ~ N(0, 1) [B, T, Hv, Dv] (bf16): the output gate
+      nw = 1 + 0.1 N(0, 1) [Dv] (fp32): the output norm's weight
+    """
+    gen = torch.Generator(device="cpu").manual_seed(w.seed)
+    dt = w.torch_dtype
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    out = dict(xq=randn(w.B, w.T, w.Hk * w.Dk).to(dt), xk=randn(w.B, w.T, w.Hk * w.Dk).to(dt),
+               xv=randn(w.B, w.T, w.Hv * w.Dv).to(dt))
+    out.update(wq=0.5 * randn(w.Hk * w.Dk, 4), wk=0.5 * randn(w.Hk * w.Dk, 4), wv=0.5 * randn(w.Hv * w.Dv, 4))
+    gshape = (w.B, w.T, w.Hv) if w.gate == "scalar" else (w.B, w.T, w.Hv, w.Dk)
+    out["g"] = torch.nn.functional.logsigmoid(randn(*gshape) + w.g_mu)
+    out["beta"] = torch.sigmoid(randn(w.B, w.T, w.Hv))
+    out["h0"] = (randn(w.B, w.Hv, w.Dk, w.Dv) * w.h0_std) if w.h0_std > 0 else None
+    out["z"] = randn(w.B, w.T, w.Hv, w.Dv).to(dt)
+    out["nw"] = 1.0 + 0.1 * randn(w.Dv)
     if device != "cpu":
         out = {n: (None if t is None else t.to(device)) for n, t in out.items()}
     return out

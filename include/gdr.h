@@ -261,8 +261,8 @@ GDR_API int gdr_causal_conv_silu(const void *x, const float *w, const float *bia
  *   y = o / sqrt(mean(o^2) + eps) * weight * SiLU(z)
  * per row of D elements (one head of one token). o, z, y: [rows, D] in `dtype`
  * (GDR_BF16 or GDR_FP32; arithmetic in fp32); weight: [D] fp32. D must be 64
- * or 128 (else GDR_ERR_UNSUPPORTED). y may alias o (in place). Pointers aligned
- * to their element size.
+ * or 128 (else GDR_ERR_UNSUPPORTED). y may alias o (in place). o, z and y
+ * 16-byte aligned, weight 4-byte aligned.
  */
 GDR_API int gdr_rmsnorm_gated(const void *o, const void *z, const float *weight, void *y, long rows, int D,
                               float eps, int dtype, void *stream);
