@@ -14,7 +14,9 @@ namespace gdr {
 namespace {
 
 constexpr int CONV_W = 4;     // taps; tap CONV_W - 1 sits on the current token
-constexpr int CONV_RUN = 8;   // consecutive tokens per thread
+constexpr int CONV_RUN = 8;   // tokens loaded together
+constexpr int CONV_TOK = 8;   // consecutive tokens per thread
+constexpr int CONV_WS = 44;   // shared floats per 8-channel group: 32 taps, 8 biases, 4 pad (conflict-free)
 constexpr int CONV_TPB = 256;
 
 struct Vec8 { float v[8]; };
@@ -71,6 +73,13 @@ template <typename T_> struct Raw8;
 template <> struct Raw8<__nv_bfloat16> {
     uint4 u;
     __device__ void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+    __device__ void gather(const __nv_bfloat16 *p, int stride)   // p[0], p[stride], ..., or zeros
+    {
+        __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = p ? p[i * stride] : __float2bfloat16_rn(0.f);
+    }
+    __device__ __nv_bfloat16 raw(int i) const { return reinterpret_cast<const __nv_bfloat16 *>(&u)[i]; }
     __device__ float get(int i) const
     {
         const __nv_bfloat162 h = reinterpret_cast<const __nv_bfloat162 *>(&u)[i >> 1];
@@ -84,6 +93,12 @@ template <> struct Raw8<float> {
         a = *reinterpret_cast<const float4 *>(p);
         b = *reinterpret_cast<const float4 *>(p + 4);
     }
+    __device__ void gather(const float *p, int stride)
+    {
+        a = p ? make_float4(p[0], p[stride], p[2 * stride], p[3 * stride]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        b = p ? make_float4(p[4 * stride], p[5 * stride], p[6 * stride], p[7 * stride]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __device__ float raw(int i) const { return get(i); }
     __device__ float get(int i) const
     {
         const float4 &q = i < 4 ? a : b;
@@ -92,11 +107,12 @@ template <> struct Raw8<float> {
     }
 };
 
-// Thread (run, group): channels 8 group .. 8 group + 7 of tokens run*RUN ..
-// run*RUN + RUN - 1 of the flattened token axis. The run's inputs and the
-// CONV_W - 1 before it are loaded first (all loads in flight together); the
-// taps then walk the run in registers. At a sequence's first token the history
-// comes from state_in (or is zero).
+// Thread (span, group): channels 8 group .. 8 group + 7 of CONV_TOK consecutive
+// tokens of the flattened token axis, in runs of CONV_RUN. A run's inputs are
+// loaded first (all loads in flight together), together with the CONV_W - 1
+// before it (for later runs, the previous run's tail, already in registers);
+// the taps then walk the run in registers. At a sequence's first token the
+// history comes from state_in (or is zero).
 template <typename T_>
 __global__ void __launch_bounds__(CONV_TPB)
 conv_silu_kernel(const T_ *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias,
@@ -104,85 +120,97 @@ conv_silu_kernel(const T_ *__restrict__ x, const float *__restrict__ w, const fl
                  long rows, int Ch)
 {
     constexpr int H = CONV_W - 1;
-    const int ngroups = Ch / 8;
-    const long gid = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    const int grp = (int)(gid % ngroups);
-    const long t0 = (gid / ngroups) * CONV_RUN;
-    if (t0 >= rows) return;
-    const int nt = (int)min((long)CONV_RUN, rows - t0);
+    // Block: 32 channel groups (one per lane) x CONV_TPB / 32 runs of CONV_TOK tokens
+    // (one per warp); the 32 groups' taps and biases are staged once, coalesced.
+    __shared__ __align__(16) float sw[32 * CONV_WS];
+    const int ngroups = Ch / 8, gblocks = (ngroups + 31) / 32;
+    const int gb = (int)(blockIdx.x % gblocks), lane = threadIdx.x & 31;
+    const long rb = blockIdx.x / gblocks;
+    const int grp = gb * 32 + lane;
+    const long tb = (rb * (CONV_TPB / 32) + (threadIdx.x >> 5)) * CONV_TOK;
     const int c0 = 8 * grp;
-
-    Raw8<T_> xr[H + CONV_RUN];   // tokens t0 - H .. t0 + RUN - 1 (addresses clamped into the axis)
+    const bool active = grp < ngroups && tb < rows;
+    Raw8<T_> xr[H + CONV_RUN];   // tokens t0 - H .. t0 + RUN - 1 of the current run (addresses clamped)
+    if (active) {   // the first run's loads go out before the taps are staged
 #pragma unroll
-    for (int i = 0; i < H + CONV_RUN; ++i) {
-        const long t = min(max(t0 - H + i, 0L), rows - 1);
-        xr[i].load(x + (size_t)t * Ch + c0);
+        for (int i = 0; i < H; ++i) xr[i].load(x + (size_t)max(tb - H + i, 0L) * Ch + c0);
+#pragma unroll
+        for (int i = 0; i < CONV_RUN; ++i) xr[H + i].load(x + (size_t)min(tb + i, rows - 1) * Ch + c0);
     }
+    {
+        const int slot = threadIdx.x >> 3, ch = threadIdx.x & 7, gg = gb * 32 + slot;   // 256 threads: 32 x 8
+        if (gg < ngroups) {
+            *reinterpret_cast<float4 *>(sw + slot * CONV_WS + ch * 4) =
+                *reinterpret_cast<const float4 *>(w + ((size_t)gg * 8 + ch) * CONV_W);
+            sw[slot * CONV_WS + 32 + ch] = bias ? bias[(size_t)gg * 8 + ch] : 0.f;
+        }
+    }
+    __syncthreads();
+    if (!active) return;
     float wt[8][CONV_W], bs[8];
+    {
+        const float *ws = sw + lane * CONV_WS;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float4 q = *reinterpret_cast<const float4 *>(w + (size_t)(c0 + i) * CONV_W);
-        wt[i][0] = q.x; wt[i][1] = q.y; wt[i][2] = q.z; wt[i][3] = q.w;
-        bs[i] = bias ? bias[c0 + i] : 0.f;
+        for (int i = 0; i < 8; ++i) {
+            const float4 q = *reinterpret_cast<const float4 *>(ws + i * 4);
+            wt[i][0] = q.x; wt[i][1] = q.y; wt[i][2] = q.z; wt[i][3] = q.w;
+            bs[i] = ws[32 + i];
+        }
     }
-    // the sequence holding t0: the last n with start(n) <= t0 (empty sequences skipped)
+    // the sequence holding tb: the last n with start(n) <= tb (empty sequences skipped)
     int lo = 0, hi = sq.n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (sq.start(mid) <= t0) lo = mid; else hi = mid - 1;
+        if (sq.start(mid) <= tb) lo = mid; else hi = mid - 1;
     }
     int n = lo;
     long s0 = sq.start(n), s1 = sq.start(n + 1);
-    // history of token t: the H inputs before it in the sequence's virtual axis
-    // [state_in (oldest first) ; x[s0] ; x[s0 + 1] ; ...]
-    float h[H][8];
-    auto fill_history = [&](int u) {   // token t0 + u (u a compile-time index)
+#pragma unroll 1
+    for (long t0 = tb; t0 < min(tb + CONV_TOK, rows); t0 += CONV_RUN) {
+        const int nt = (int)min((long)CONV_RUN, rows - t0);
+        if (t0 != tb) {
 #pragma unroll
-        for (int j = 0; j < H; ++j) {
-            const long vt = t0 + u - s0 + j;   // virtual index of the input H - j tokens back
+            for (int i = 0; i < CONV_RUN; ++i) xr[H + i].load(x + (size_t)min(t0 + i, rows - 1) * Ch + c0);
+        }
+        // The taps of token t0 + u read xr[u .. u + H]. Where those history slots precede
+        // the sequence's first token they take state_in (or zero) instead: the sequence's
+        // virtual axis is [state_in (oldest first) ; x[s0] ; x[s0 + 1] ; ...].
+        auto fix_history = [&](int u) {   // u a compile-time index
+#pragma unroll
+            for (int j = 0; j < H; ++j) {
+                const long vt = t0 + u - s0 + j;
+                if (vt < H) xr[u + j].gather(state_in ? state_in + ((size_t)n * Ch + c0) * H + vt : nullptr, H);
+            }
+        };
+        if (t0 == tb) fix_history(0);
+#pragma unroll
+        for (int u = 0; u < CONV_RUN; ++u) {
+            if (u >= nt) break;
+            const long t = t0 + u;
+            while (t >= s1) {   // next sequence (skipping empty ones)
+                ++n;
+                s0 = s1;
+                s1 = sq.start(n + 1);
+                if (t < s1) fix_history(u);
+            }
+            Vec8 o;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float v = 0.f;
-                if (vt >= H) {
-                    v = xr[u + j].get(i);   // token t0 + u - H + j, preloaded
-                } else if (state_in) {
-                    v = to_f(state_in[((size_t)n * Ch + c0 + i) * H + vt]);
-                }
-                h[j][i] = v;
+                float acc = bs[i];
+#pragma unroll
+                for (int j = 0; j <= H; ++j) acc = fmaf(wt[i][j], xr[u + j].get(i), acc);
+                o.v[i] = silu(acc);
+            }
+            store8(y + (size_t)t * Ch + c0, o);
+            if (state_out && t == s1 - 1) {   // the sequence's last H inputs, as given
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < H; ++j) state_out[((size_t)n * Ch + c0 + i) * H + j] = xr[u + 1 + j].raw(i);
             }
         }
-    };
-    fill_history(0);
 #pragma unroll
-    for (int u = 0; u < CONV_RUN; ++u) {
-        if (u >= nt) break;
-        const long t = t0 + u;
-        while (t >= s1) {   // next sequence (skipping empty ones)
-            ++n;
-            s0 = s1;
-            s1 = sq.start(n + 1);
-            if (t < s1) fill_history(u);
-        }
-        Vec8 o;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float xi = xr[H + u].get(i);
-            float acc = bs[i];
-#pragma unroll
-            for (int j = 0; j < H; ++j) acc = fmaf(wt[i][j], h[j][i], acc);
-            acc = fmaf(wt[i][H], xi, acc);
-            o.v[i] = silu(acc);
-#pragma unroll
-            for (int j = 0; j < H - 1; ++j) h[j][i] = h[j + 1][i];
-            h[H - 1][i] = xi;
-        }
-        store8(y + (size_t)t * Ch + c0, o);
-        if (state_out && t == s1 - 1) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int j = 0; j < H; ++j) from_f(&state_out[((size_t)n * Ch + c0 + i) * H + j], h[j][i]);
-        }
+        for (int i = 0; i < H; ++i) xr[i] = xr[CONV_RUN + i];   // the next run's halo
     }
 }
 
@@ -279,8 +307,9 @@ cudaError_t conv_t(const ConvArgs &a, cudaStream_t st)
     const Seqs sq{a.cu_seqlens, a.nseq, a.T};
     const long rows = a.rows;
     if (rows > 0) {
-        const long threads = ((rows + CONV_RUN - 1) / CONV_RUN) * (a.Ch / 8);
-        conv_silu_kernel<T_><<<(unsigned)((threads + CONV_TPB - 1) / CONV_TPB), CONV_TPB, 0, st>>>(
+        const long runs = (rows + CONV_TOK - 1) / CONV_TOK, per_block = CONV_TPB / 32;
+        const long blocks = ((a.Ch / 8 + 31) / 32) * ((runs + per_block - 1) / per_block);
+        conv_silu_kernel<T_><<<(unsigned)blocks, CONV_TPB, 0, st>>>(
             static_cast<const T_ *>(a.x), a.w, a.bias, static_cast<const T_ *>(a.state_in),
             static_cast<T_ *>(a.state_out), static_cast<T_ *>(a.y), sq, rows, a.Ch);
     }
