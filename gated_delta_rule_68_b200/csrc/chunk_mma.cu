@@ -86,7 +86,7 @@ __device__ unsigned int g_fused_range_errors;
 // per (token, head, key channel). NS: the unit's value columns are split over NS CTAs,
 // CTA `split` owning D / NS of them (its part of the state, U, U', O); the Gram, the
 // inverse and W are computed by each.
-template <typename TOut, int GATE, int NS>
+template <typename TOut, int GATE, int NS, bool NORM>
 __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *map_q, const CUtensorMap *map_k,
                                            const CUtensorMap *map_v, const CUtensorMap *map_o,
                                            const CUtensorMap *map_z, int bh, int split)
@@ -184,7 +184,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
         mbar_init(aBar, 1);
         mbar_init(aZBar, 1);
     }
-    if (a.z && tid < D) sNW[tid] = a.norm_w[tid];
+    if (NORM && a.z && tid < D) sNW[tid] = a.norm_w[tid];
     __syncthreads();
     auto issue_loads = [&](int c) {
         const int t0 = c * C, n = min(C, T - t0);
@@ -271,7 +271,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 const int which = idx / (C * 16), rem = idx % (C * 16), r = rem >> 4, c16 = rem & 15;
                 const uint4 u = sStg[idx];
                 uint4 h;
-                if (a.qk_l2norm) {
+                if (NORM && a.qk_l2norm) {
                     const float ss = halfwarp_sum(bf16x8_sumsq(u));
                     h = bf16x8_scaled_f16x8(u, rsqrtf(ss + 1e-6f));
                 } else {
@@ -288,7 +288,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
             }
             *reinterpret_cast<float2 *>(sTot + ch_h * D + 2 * ch_p) = s;
             if (w == 2 || w == 3) sBeta[tid - 64] = sGst[C + tid - 64];
-            if (a.qk_l2norm) {   // 1 / |row| of the 64 K rows and 64 Q rows, a half warp per row
+            if (NORM && a.qk_l2norm) {   // 1 / |row| of the 64 K rows and 64 Q rows, a half warp per row
 #pragma unroll
                 for (int rr = 0; rr < 2 * C / (NT / 16); ++rr) {
                     const int R = (tid >> 4) + rr * (NT / 16);
@@ -328,7 +328,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 if (row < n) {
                     kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sStgH + row * D + 2 * ch_p));
                     qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sStgH + C * D + row * D + 2 * ch_p));
-                    if (a.qk_l2norm) {
+                    if (NORM && a.qk_l2norm) {
                         const float rk = sRstd[row], rq = sRstd[C + row];
                         kv.x *= rk; kv.y *= rk; qv.x *= rq; qv.y *= rq;
                     }
@@ -563,7 +563,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
         // Gated output norm: the chunk's z tile into the V tile (dead from here on), in the
         // 128-byte swizzle of a bf16 o tile, so that each thread later finds its z values
         // where it writes its outputs.
-        if (a.z && tid == NT - 32) {
+        if (NORM && a.z && tid == NT - 32) {
             mbar_expect_tx(aZBar, C * D * 2);
 #pragma unroll
             for (int bx = 0; bx < D / 64; ++bx)
@@ -614,7 +614,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 }
             }
         }
-        if (a.z) {   // the barrier also waits for the z tile (issued after W/U)
+        if (NORM && a.z) {   // the barrier also waits for the z tile (issued after W/U)
             if (!__syncthreads_and(mbar_wait_bounded(aZBar, ch & 1))) {
                 if (tid == 0) atomicAdd(&g_fused_load_timeouts, 1u);
                 return;
@@ -637,7 +637,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
                 mma(accO[2 * np + 1], am, bu[2], bu[3]);
             }
         }
-        if (a.z) {   // o <- o / sqrt(mean(o^2) + eps) * weight * SiLU(z) per row (the CTA has every column)
+        if (NORM && a.z) {   // o <- o / sqrt(mean(o^2) + eps) * weight * SiLU(z) per row (the CTA has every column)
             const int r0 = rw0 + g, r1 = rw0 + g + 8;
             uint32_t zr[2][NJ];   // read before the barrier below: an fp32 o tile overwrites other rows' z
 #pragma unroll
@@ -780,7 +780,7 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
 // Blocks [0, n_whole) each run a whole unit; each later pair of blocks splits one of
 // the remaining units by value columns. Whole units are dispatched first, and the
 // halves fill the SMs as those free up.
-template <typename TOut, int GATE>
+template <typename TOut, int GATE, bool NORM>
 __global__ void __launch_bounds__(NT, 1)
 fused_fwd_kernel(FwdArgs a, int n_whole, const __grid_constant__ CUtensorMap map_q,
                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v1,
@@ -789,10 +789,10 @@ fused_fwd_kernel(FwdArgs a, int n_whole, const __grid_constant__ CUtensorMap map
 {
     const int blk = blockIdx.x;
     if (blk < n_whole) {
-        fused_unit<TOut, GATE, 1>(a, &map_q, &map_k, &map_v1, &map_o, &map_z, blk, 0);
+        fused_unit<TOut, GATE, 1, NORM>(a, &map_q, &map_k, &map_v1, &map_o, &map_z, blk, 0);
     } else {
         const int i = blk - n_whole;
-        fused_unit<TOut, GATE, 2>(a, &map_q, &map_k, &map_v2, &map_o, &map_z, n_whole + i / 2, i % 2);
+        fused_unit<TOut, GATE, 2, NORM>(a, &map_q, &map_k, &map_v2, &map_o, &map_z, n_whole + i / 2, i % 2);
     }
 }
 
@@ -861,7 +861,9 @@ cudaError_t launch_g(const FwdArgs &a, cudaStream_t st)
     if (a.z ? !make_map(&mz, a.z, mb, a.T, a.Hv, 64, false, true) : (mz = mo, false))   // z: the bf16 o box
         return cudaErrorInvalidValue;
     const int smem = SMEM_BYTES + 1024;
-    auto kernel = fused_fwd_kernel<TOut, GATE>;
+    // The layer's normalisations are compiled into a separate instance, so a call without
+    // them runs the same code as before they existed.
+    auto kernel = (a.qk_l2norm || a.z) ? fused_fwd_kernel<TOut, GATE, true> : fused_fwd_kernel<TOut, GATE, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const long grid = n_whole + 2 * (units - n_whole);
