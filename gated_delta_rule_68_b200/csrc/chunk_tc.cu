@@ -1,0 +1,701 @@
+// Chunked forward of the gated delta rule with a scalar decay per head (Gated
+// DeltaNet) on the fifth-generation tensor cores: tcgen05.mma with operands in
+// shared memory and fp32 accumulators in tensor memory, bf16 inputs,
+// Dk = Dv = 128, chunks of C = 64 tokens. One CTA per (batch row, value head).
+//
+// Method: the exact chunkwise form of
+//   S_t = (I - beta_t k_t k_t^T) exp(g_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
+// (NextTransformer, "Source notes", "Linear attention", row gdn; SinkProbe
+// (Attention-Sink) README: delta-rule layer in exact chunkwise form). Inside a
+// chunk, with G_r = sum_{j<=r} g_j, Gamma_r = exp(G_r), Gamma_C = Gamma_63:
+//   A_ri = beta_r exp(G_r - G_i) k_r.k_i (i < r),   T = (I + A)^-1
+//   W = T diag(beta Gamma) K,   U = T diag(beta) V,   U' = U - W S
+//   O = diag(Gamma) Q S + M U',   M_ri = exp(G_r - G_i) q_r.k_i (i <= r)
+//   S_next = Gamma_C S + Kt^T U',   Kt = diag(Gamma_C / Gamma) K.
+// Substituting U' makes both outputs affine in the entering state S:
+//   S_next = Gamma_C S + P S + R,   P = -Kt^T W,  R = Kt^T U
+//   O      = Qh S + Uh,             Qh = diag(Gamma) Q - M W,  Uh = M U
+// and P, R, Qh, Uh depend on the chunk's inputs alone. So the kernel runs two
+// warpgroups:
+//   - the chunk group (warps 4-7) builds P, R, Qh, Uh for one chunk after the
+//     other: the Gram [K; Q] K^T, the gate factors, the inverse (fp32 16 x 16
+//     diagonal blocks, off-diagonal blocks by warp-level MMA), then W, U and the
+//     four products, all large products on tcgen05;
+//   - the state group (warps 0-3) keeps S (fp32, one value column per thread, in
+//     registers) and per chunk issues one batch of MMAs that adds P S to R and
+//     Qh S to Uh in tensor memory, then forms S_next = Gamma_C S + (P S + R),
+//     writes its fp16 copy (the next batch's operand) and stores o.
+// The chunk group runs one chunk ahead of the state group, so the inverse and
+// the other chunk-local work overlap the state chain, and the state chain of a
+// chunk is one MMA batch and two short epilogues.
+//
+// Precision: products take fp16 operands (bf16 inputs convert exactly inside
+// fp16's normal range) with fp32 accumulation; the state carry Gamma_C S is fp32
+// and only its product with P uses the fp16 copy of S. q, k, v and the state
+// must stay inside the fp16 range (|x| < 6.5e4).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "mma_util.cuh"
+#include "tc_util.cuh"
+
+namespace gdr {
+namespace {
+
+using namespace mmau;
+using namespace tcu;
+
+constexpr int NTH = 256;   // warps 0-3: state group, warps 4-7: chunk group
+
+// Shared memory (byte offsets from a 1024-byte aligned base). Operand tiles are
+// 128-byte swizzled rows (tc_util.cuh).
+constexpr uint32_t STG_BYTES = 49152;           // one chunk's inputs: [K; Q] (2 atoms of 128 rows) and V (2 atoms of 64 rows)
+constexpr uint32_t STG_Q = 8192;                //   Q rows start at row 64 of each [K; Q] atom
+constexpr uint32_t STG_V = 32768;
+constexpr uint32_t OFF_P16 = 2 * STG_BYTES;     // P [dk_out][dk_in] fp16, 2 atoms of 16 KB
+constexpr uint32_t OFF_QH16 = OFF_P16 + 32768;  // Qh^T [dk][r] fp16
+constexpr uint32_t OFF_ST16 = OFF_QH16 + 16384; // S^T [dv][dk] fp16, 2 atoms of 16 KB
+constexpr uint32_t OFF_R1 = OFF_ST16 + 32768;   // T' and T'' (8 KB each) and the inverse's scratch; then W^T, U^T
+constexpr uint32_t OFF_TP = OFF_R1;             // T diag(beta Gamma) [r][i] fp16
+constexpr uint32_t OFF_TPP = OFF_R1 + 8192;     // T diag(beta) [r][i] fp16
+constexpr uint32_t OFF_W16 = OFF_R1;            // W^T [dk][r] fp16 (written once T', T'' are dead)
+constexpr uint32_t OFF_U16 = OFF_R1 + 16384;    // U^T [dv][r] fp16
+constexpr uint32_t OFF_INV = OFF_R1 + 16384;    // inverse scratch (dead before U^T is written)
+constexpr uint32_t OFF_M16 = OFF_R1 + 32768;    // M [r][i] fp16
+constexpr uint32_t OFF_VEC = OFF_M16 + 8192;    // per-chunk vectors (fp32)
+// Inverse scratch: fp32 diagonal blocks of A (transposed, [4][16][20]), reused by the
+// 16 x 16 products' intermediates; fp16 off-diagonal rows 16..63 of A ([48][56]);
+// fp16 diagonal inverses D_b ([4][16][24]) and the first off-diagonal blocks T_10, T_32.
+constexpr int LDAD = 20, LDA16 = 56, LDT16 = 24;
+constexpr uint32_t INV_AD = OFF_INV, INV_XY = OFF_INV;
+constexpr uint32_t INV_A16 = OFF_INV + 4 * 16 * LDAD * 4;
+constexpr uint32_t INV_D = INV_A16 + 48 * LDA16 * 2;
+constexpr uint32_t INV_T1 = INV_D + 4 * 16 * LDT16 * 2;
+constexpr uint32_t INV_END = INV_T1 + 2 * 16 * LDT16 * 2;
+static_assert(INV_END <= OFF_U16 + 16384, "inverse scratch must fit beside T' and T''");
+// vectors
+// Per-chunk vectors, two sets (chunk parity): G, Gamma, f = Gamma_C / Gamma, beta,
+// beta Gamma, row and column factors of exp(G_r - G_i), Gamma_C.
+constexpr int V_G = 0, V_GAM = 64, V_F = 128, V_BETA = 192, V_BG = 256, V_EROW = 320, V_ECOL = 384,
+              V_GC = 640, V_SET = 644, V_N = 2 * V_SET;
+constexpr uint32_t SMEM_USED = OFF_VEC + V_N * 4;
+constexpr uint32_t SMEM_TC = SMEM_USED + 1024;
+static_assert(SMEM_TC <= 227 * 1024, "shared memory");
+
+// Tensor memory columns (512 allocated): the state product (R, then P S + R), the
+// o accumulator (Uh, then Qh S + Uh), the Gram, Qh^T, and W^T / U^T, then P.
+constexpr uint32_t TM_S = 0, TM_O = 128, TM_G = 192, TM_X = 256, TM_Y = 320;
+
+// mbarriers
+enum {
+    B_LD0, B_LD1,   // chunk inputs landed in staging buffer 0 / 1 (TMA)
+    B_G0, B_G1,     // Gram of the chunk in staging buffer 0 / 1 done
+    B_CV0, B_CV1,   // fp16 tiles and gate vectors of the chunk in buffer 0 / 1 written (128 arrivals)
+    B_W,            // W^T, U^T done
+    B_P,            // P, R, Qh, Uh of a chunk done (waited on by both groups)
+    B_ST,           // state batch done
+    B_GE,           // the chunk group has read the Gram out of tensor memory (128 arrivals)
+    B_YE,           // the state group has read P and Qh out of Y and X (128 arrivals)
+    B_SE,           // the state group has read the state product (128 arrivals)
+    B_OE,           // the state group has read the o accumulator (128 arrivals)
+    B_DR0, B_DR1,   // end-of-kernel drain of each issuing thread's MMAs
+    NBAR
+};
+
+constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false, false);
+constexpr uint32_t ID_WU = idesc_f16(128, 64, false, true, false);
+constexpr uint32_t ID_P = idesc_f16(128, 128, false, true, false, true);
+constexpr uint32_t ID_R = idesc_f16(128, 128, false, false, true);
+constexpr uint32_t ID_X = idesc_f16(128, 64, false, false, false, true);
+constexpr uint32_t ID_QG = idesc_f16(128, 64, false, true, false);
+constexpr uint32_t ID_UH = idesc_f16(128, 64, false, false, false);
+constexpr uint32_t ID_S = idesc_f16(128, 128, false, false, false);
+constexpr uint32_t ID_O = idesc_f16(128, 64, false, false, true);
+
+// Waits that timed out (each abandons its CTA's remaining work).
+__device__ unsigned int g_tc_timeouts;
+
+__device__ __forceinline__ uint32_t pack_h2(float x, float y)
+{
+    const __half2 h = __floats2half2_rn(x, y);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+// 8 fp32 -> one 16-byte chunk of fp16 at shared address `addr`.
+__device__ __forceinline__ void st_chunk8(uint32_t addr, const float *x)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pack_h2(x[0], x[1])),
+                 "r"(pack_h2(x[2], x[3])), "r"(pack_h2(x[4], x[5])), "r"(pack_h2(x[6], x[7]))
+                 : "memory");
+}
+__device__ __forceinline__ void st_h1(uint8_t *sm, uint32_t off, float x)
+{
+    *reinterpret_cast<__half *>(sm + off) = __float2half_rn(x);
+}
+
+__device__ __forceinline__ void out_store2(float *p, float x, float y) { *reinterpret_cast<float2 *>(p) = make_float2(x, y); }
+__device__ __forceinline__ void out_store2(__nv_bfloat16 *p, float x, float y)
+{
+    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(x, y);
+}
+
+// c (16 x 16, fp32, two n8 tiles) += A (16 x 16 row-major at aA, stride lda) B (16 x 16 stored [k][n] at aB, stride ldb).
+__device__ __forceinline__ void mma16(float c0[4], float c1[4], uint32_t aA, int lda, uint32_t aB, int ldb, int lane)
+{
+    uint32_t af[4], bf[4];
+    ldsm(af, a_rm(aA, lda, 0, 0, lane));
+    ldsm_t(bf, b_kn(aB, ldb, 0, 0, lane));
+    mma(c0, af, bf[0], bf[1]);
+    mma(c1, af, bf[2], bf[3]);
+}
+// Stores a 16 x 16 fp32 product (two n8 tiles), times `s`, as fp16 row-major at p (stride ld).
+__device__ __forceinline__ void st_tile16(__half *p, int ld, const float c0[4], const float c1[4], float s, int lane)
+{
+    const int g = lane >> 2, t4 = lane & 3;
+    st_h2(p + g * ld + 2 * t4, s * c0[0], s * c0[1]);
+    st_h2(p + (g + 8) * ld + 2 * t4, s * c0[2], s * c0[3]);
+    st_h2(p + g * ld + 8 + 2 * t4, s * c1[0], s * c1[1]);
+    st_h2(p + (g + 8) * ld + 8 + 2 * t4, s * c1[2], s * c1[3]);
+}
+// Writes block (R0.., I0..) of T, given as two n8 tiles times `s`, into T diag(beta Gamma)
+// and T diag(beta) (swizzled [r][i] tiles).
+__device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const float c0[4], const float c1[4], float s,
+                                          const float *vec, int lane)
+{
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const float *c = nt ? c1 : c0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int r = R0 + g + 8 * (e >> 1), i = I0 + 8 * nt + 2 * t4 + (e & 1);
+            const float t = s * c[e];
+            st_h1(sm, OFF_TP + swz_off(r, i, 0), t * vec[V_BG + i]);
+            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t * vec[V_BETA + i]);
+        }
+    }
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(NTH, 1)
+tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+              const __grid_constant__ CUtensorMap map_v)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb0 = smem_u32(sm);
+    float *vec = reinterpret_cast<float *>(sm + OFF_VEC);
+    __shared__ uint64_t bars[NBAR];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
+    const int p = tid & 127;          // row of the 128-row products owned by this thread
+    const int bh = blockIdx.x, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
+    const int T = a.T, NC = (T + C - 1) / C;
+    const long tok0 = (long)b * T;
+
+    if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), 512);
+    if (tid == 0) {
+        const uint32_t counts[NBAR] = {1, 1, 1, 1, 128, 128, 1, 1, 1, 128, 128, 128, 128, 1, 1};
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
+        abort_sh = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = tmem_base_sh;
+
+    // Bounded wait; after any timeout every later wait of the CTA returns at once, so
+    // the two groups still meet at all their barriers and the kernel ends.
+    auto wait = [&](int i, uint32_t parity) {
+        if (*reinterpret_cast<volatile int *>(&abort_sh)) return;
+        if (!mbar_wait_bounded(bar(i), parity)) {
+            *reinterpret_cast<volatile int *>(&abort_sh) = 1;
+            atomicAdd(&g_tc_timeouts, 1u);
+        }
+    };
+
+    if (warp >= 4) {
+        // ============================ chunk group ============================
+        // Per chunk: the gated Gram's epilogue (A, M), the inverse (T diag(beta Gamma),
+        // T diag(beta)), W^T and U^T, then P, R, Qh, Uh.
+        const int wq = warp - 4;
+        const bool issuer = tid == 128;
+        for (int c = 0; c < NC; ++c) {
+            const int sb = c & 1;
+            const uint32_t stg = sb0 + sb * STG_BYTES;
+            uint8_t *stgp = sm + sb * STG_BYTES;
+            const float *vc = vec + sb * V_SET;
+            // The previous chunk's last products are done with M, W^T, U^T and the inverse's tiles.
+            if (c >= 1) wait(B_P, (c - 1) & 1);
+            wait(B_CV0 + sb, (c >> 1) & 1);
+            // Gram epilogue: A (rows < 64) and M (rows 64..127)
+            wait(B_G0 + sb, (c >> 1) & 1);
+            tc_fence_after();
+            {
+                float v[64];
+                tmem_ld32(tmem_addr(tb, q4, TM_G), v);
+                tmem_ld32(tmem_addr(tb, q4, TM_G + 32), v + 32);
+                tc_fence_before();
+                mbar_arrive(bar(B_GE));
+                // exp(G_r - G_i) = exp(G_r - G_16R) exp(G_16R - G_i), R = r / 16
+                const int r = p & 63, rb = r >> 4;
+                const float4 *ec4 = reinterpret_cast<const float4 *>(vc + V_ECOL + rb * 64);
+                const float rowf = p < 64 ? vc[V_BETA + r] * vc[V_EROW + r] : vc[V_EROW + r];
+                const int lim = p < 64 ? r : r + 1;   // A: i < r;  M: i <= r
+#pragma unroll
+                for (int i4 = 0; i4 < 16; ++i4) {
+                    const float4 e = ec4[i4];
+                    const int i = 4 * i4;
+                    v[i] = i < lim ? rowf * e.x * v[i] : 0.f;
+                    v[i + 1] = i + 1 < lim ? rowf * e.y * v[i + 1] : 0.f;
+                    v[i + 2] = i + 2 < lim ? rowf * e.z * v[i + 2] : 0.f;
+                    v[i + 3] = i + 3 < lim ? rowf * e.w * v[i + 3] : 0.f;
+                }
+                if (p >= 64) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(r, j, OFF_M16), v + 8 * j);
+                } else {
+                    // fp16 blocks left of the diagonal block (rows 16..63 of A), fp32 diagonal block transposed
+                    const uint32_t a16 = sb0 + INV_A16 + (uint32_t)((r - 16) * LDA16) * 2u;
+#pragma unroll
+                    for (int j = 0; j < 6; ++j)
+                        if (j < 2 * rb) st_chunk8(a16 + 16 * j, v + 8 * j);
+                    float *ad = reinterpret_cast<float *>(sm + INV_AD) + rb * 16 * LDAD + (r - 16 * rb);
+                    switch (rb) {
+#define GDR_AD_CASE(K)                                                         \
+    case K:                                                                    \
+        _Pragma("unroll") for (int ii = 0; ii < 16; ++ii) ad[ii * LDAD] = v[16 * K + ii]; \
+        break;
+                        GDR_AD_CASE(0) GDR_AD_CASE(1) GDR_AD_CASE(2) GDR_AD_CASE(3)
+#undef GDR_AD_CASE
+                    }
+                }
+            }
+            fence_proxy_async();
+            named_bar_sync(1, 128);
+
+            // Inverse, level 0: warp wq inverts the unit lower 16 x 16 block I + A_bb (b = wq)
+            // by forward substitution (lane j < 16 holds column j); lanes 16..31 zero the
+            // blocks of T above the diagonal.
+            if (lane < 16) {
+                const int j = lane;
+                float t[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) t[rr] = rr == j ? 1.f : 0.f;
+                const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;
+#pragma unroll
+                for (int i = 0; i < 15; ++i) {
+                    float col[16];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 x = *reinterpret_cast<const float4 *>(ad + i * LDAD + 4 * k4);
+                        col[4 * k4] = x.x, col[4 * k4 + 1] = x.y, col[4 * k4 + 2] = x.z, col[4 * k4 + 3] = x.w;
+                    }
+                    const float ti = t[i];
+#pragma unroll
+                    for (int rr = i + 1; rr < 16; ++rr) t[rr] = fmaf(-col[rr], ti, t[rr]);
+                }
+                __half *dd = reinterpret_cast<__half *>(sm + INV_D) + wq * 16 * LDT16;
+                const int I = 16 * wq + j;
+                const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    dd[rr * LDT16 + j] = __float2half_rn(t[rr]);
+                    st_h1(sm, OFF_TP + swz_off(16 * wq + rr, I, 0), t[rr] * sbg);
+                    st_h1(sm, OFF_TPP + swz_off(16 * wq + rr, I, 0), t[rr] * sbt);
+                }
+            } else {
+                // zero chunks: rows of block R, 16-byte chunks 2(R+1) .. 7
+                const int u = wq * 16 + (lane - 16);   // 0..63: one row each
+                const int R = u >> 4;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                for (int j = 2 * (R + 1); j < 8; ++j) {
+                    *reinterpret_cast<uint4 *>(sm + swz_chunk(u, j, OFF_TP)) = z;
+                    *reinterpret_cast<uint4 *>(sm + swz_chunk(u, j, OFF_TPP)) = z;
+                }
+            }
+            named_bar_sync(1, 128);
+
+            const uint32_t aD = sb0 + INV_D, aA16 = sb0 + INV_A16, aXY = sb0 + INV_XY, aT1 = sb0 + INV_T1;
+            constexpr uint32_t T16B = 16 * LDT16 * 2;   // bytes of one [16][24] fp16 tile
+            // Level 1: T_10 = -D_1 A_10 D_0 (warp 1), T_32 = -D_3 A_32 D_2 (warp 3).
+            if (wq & 1) {
+                const int m = wq - 1;
+                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+                mma16(c0, c1, aA16 + ((16 * (wq - 1)) * LDA16 + 16 * m) * 2, LDA16, aD + m * T16B, LDT16, lane);
+                __half *xw = reinterpret_cast<__half *>(sm + INV_XY) + wq * 16 * LDT16;
+                st_tile16(xw, LDT16, c0, c1, 1.f, lane);
+                __syncwarp();
+                float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+                mma16(d0, d1, aD + wq * T16B, LDT16, aXY + wq * T16B, LDT16, lane);
+                st_tile16(reinterpret_cast<__half *>(sm + INV_T1) + (wq >> 1) * 16 * LDT16, LDT16, d0, d1, -1.f,
+                          lane);
+                st_tblock(sm, 16 * wq, 16 * m, d0, d1, -1.f, vc, lane);
+            }
+            named_bar_sync(1, 128);
+            // Level 2 (warp wq -> block (a, bc) of the lower-left 32 x 32 block, a = 2 + wq / 2, bc = wq % 2):
+            //   Y_a,bc = A_a,0:2 T_0:2,bc;   T_a,bc = -(T_a,2:4 Y_2:4,bc)
+            {
+                const int ar = 2 + (wq >> 1), bc = wq & 1;
+                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t arow = aA16 + ((16 * (ar - 1)) * LDA16) * 2;
+                if (bc == 0) {
+                    mma16(c0, c1, arow, LDA16, aD, LDT16, lane);                    // A_a0 D_0
+                    mma16(c0, c1, arow + 16 * 2, LDA16, aT1, LDT16, lane);          // A_a1 T_10
+                } else {
+                    mma16(c0, c1, arow + 16 * 2, LDA16, aD + T16B, LDT16, lane);    // A_a1 D_1
+                }
+                __half *yw = reinterpret_cast<__half *>(sm + INV_XY) + wq * 16 * LDT16;
+                st_tile16(yw, LDT16, c0, c1, 1.f, lane);
+            }
+            named_bar_sync(1, 128);
+            {
+                const int ar = 2 + (wq >> 1), bc = wq & 1;
+                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+                if (ar == 2) {
+                    mma16(c0, c1, aD + 2 * T16B, LDT16, aXY + bc * T16B, LDT16, lane);           // D_2 Y_2,bc
+                } else {
+                    mma16(c0, c1, aT1 + T16B, LDT16, aXY + bc * T16B, LDT16, lane);              // T_32 Y_2,bc
+                    mma16(c0, c1, aD + 3 * T16B, LDT16, aXY + (2 + bc) * T16B, LDT16, lane);     // D_3 Y_3,bc
+                }
+                st_tblock(sm, 16 * ar, 16 * bc, c0, c1, -1.f, vc, lane);
+            }
+            fence_proxy_async();
+            named_bar_sync(1, 128);
+
+            // W^T = K^T T'^T -> Y[0:64),  U^T = V^T T''^T -> Y[64:128), once the state
+            // group has read the previous chunk's P and Qh out of Y and X.
+            if (issuer) {
+                if (c >= 1) wait(B_YE, (c - 1) & 1);
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint64_t bt = sdesc(sb0 + OFF_TP + s * 32, 16, 1024);
+                    mma_ss(tb + TM_Y, sdesc(stg + s * 2048, 16384, 1024), bt, ID_WU, s > 0);
+                }
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint64_t bt = sdesc(sb0 + OFF_TPP + s * 32, 16, 1024);
+                    mma_ss(tb + TM_Y + 64, sdesc(stg + STG_V + s * 2048, 8192, 1024), bt, ID_WU, s > 0);
+                }
+                mma_commit(bar(B_W));
+            }
+            wait(B_W, c & 1);
+            tc_fence_after();
+            {
+                float v[32];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 32 * half), v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * half + j, OFF_W16), v + 8 * j);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 64 + 32 * half), v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * half + j, OFF_U16), v + 8 * j);
+                }
+            }
+            // K -> Kt = diag(Gamma_C / Gamma) K in place (the W product is done with K)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const int e = p + 128 * jj, tok = (e >> 3) & 63;
+                uint4 *pch = reinterpret_cast<uint4 *>(stgp + (e >> 9) * 16384) + (e & 511);
+                const float f = vc[V_F + tok];
+                uint4 u = *pch;
+                __half2 *hh = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 x = __half22float2(hh[k]);
+                    hh[k] = __floats2half2_rn(x.x * f, x.y * f);
+                }
+                *pch = u;
+            }
+            // diag(Gamma) [r][j] into the dead V tile: 4 of its 16-byte chunks per thread
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int e = p + 128 * jj, r = e >> 3, j = e & 7;
+                float x[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? vc[V_GAM + r] : 0.f;
+                st_chunk8(stg + STG_V + swz_chunk(r, j, 0), x);
+            }
+            tc_fence_before();
+            fence_proxy_async();
+            named_bar_sync(1, 128);
+
+            // P = -Kt^T W -> Y,  R^T = U^T Kt -> state product,  X = Q^T diag(Gamma) - W^T M^T -> X,
+            // Uh^T = U^T M^T -> o accumulator.
+            if (issuer) {
+                if (c >= 1) wait(B_SE, (c - 1) & 1);
+                if (c >= 1) wait(B_OE, (c - 1) & 1);
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tb + TM_Y, sdesc(stg + s * 2048, 16384, 1024), sdesc(sb0 + OFF_W16 + s * 32, 16, 1024),
+                           ID_P, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tb + TM_S, sdesc(sb0 + OFF_U16 + s * 32, 16, 1024), sdesc(stg + s * 2048, 16384, 1024),
+                           ID_R, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tb + TM_X, sdesc(stg + STG_Q + s * 2048, 16384, 1024),
+                           sdesc(stg + STG_V + s * 32, 16, 1024), ID_QG, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tb + TM_X, sdesc(sb0 + OFF_W16 + s * 32, 16, 1024), sdesc(sb0 + OFF_M16 + s * 32, 16, 1024),
+                           ID_X, true);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tb + TM_O, sdesc(sb0 + OFF_U16 + s * 32, 16, 1024), sdesc(sb0 + OFF_M16 + s * 32, 16, 1024),
+                           ID_UH, s > 0);
+                mma_commit(bar(B_P));
+            }
+        }
+        if (issuer) {
+            mma_commit(bar(B_DR1));
+            mbar_wait_bounded(bar(B_DR1), 0);
+        }
+    } else {
+        // ============================ state group ============================
+        // Thread p owns value column p: S[:, p] in fp32 registers. Besides the state step
+        // of chunk c, the group readies chunk c + 2: its TMA loads, the bf16 -> fp16
+        // conversion of K, Q and V in place, the gate vectors and the Gram.
+        const bool issuer = tid == 0;
+        auto issue_loads = [&](int c) {
+            const int sb = c & 1;
+            const uint32_t stg = sb0 + sb * STG_BYTES, bl = bar(B_LD0 + sb);
+            const int t0 = c * C;
+            mbar_expect_tx(bl, STG_BYTES);
+            tma_load_4d(stg, &map_k, 0, hk, t0, b, bl);
+            tma_load_4d(stg + 16384, &map_k, 64, hk, t0, b, bl);
+            tma_load_4d(stg + STG_Q, &map_q, 0, hk, t0, b, bl);
+            tma_load_4d(stg + 16384 + STG_Q, &map_q, 64, hk, t0, b, bl);
+            tma_load_4d(stg + STG_V, &map_v, 0, h, t0, b, bl);
+            tma_load_4d(stg + STG_V + 8192, &map_v, 64, h, t0, b, bl);
+        };
+        // g and beta of chunk c (zero past T), read by warp 0: lane l has rows l and l + 32.
+        auto load_gb = [&](int c, float gb[4]) {
+            const int t0 = c * C;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int t = t0 + lane + 32 * e;
+                const bool ok = t < T;
+                const size_t ix = (size_t)(tok0 + t) * a.Hv + h;
+                gb[e] = ok ? a.g[ix] : 0.f;
+                gb[2 + e] = ok ? a.beta[ix] : 0.f;
+            }
+        };
+        // Chunk c's tiles to fp16 in place and its gate vectors (warp 0), then its Gram.
+        auto ready_chunk = [&](int c, const float gb[4]) {
+            const int sb = c & 1;
+            uint8_t *stgp = sm + sb * STG_BYTES;
+            float *vs = vec + sb * V_SET;
+            wait(B_LD0 + sb, (c >> 1) & 1);
+#pragma unroll 8
+            for (int j = 0; j < 24; ++j) {
+                uint4 *pch = reinterpret_cast<uint4 *>(stgp) + p + 128 * j;   // all 3072 chunks of [K; Q] and V
+                *pch = bf16x8_to_f16x8(*pch);
+            }
+            if (warp == 0) {
+                float s0 = gb[0], s1 = gb[1];
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y0 = __shfl_up_sync(0xffffffffu, s0, off), y1 = __shfl_up_sync(0xffffffffu, s1, off);
+                    if (lane >= off) s0 += y0, s1 += y1;
+                }
+                s1 += __shfl_sync(0xffffffffu, s0, 31);
+                const float GC = __shfl_sync(0xffffffffu, s1, 31);
+                const float G[2] = {s0, s1};
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = lane + 32 * e;
+                    const float be = gb[2 + e];
+                    const float gam = __expf(G[e]);
+                    vs[V_G + r] = G[e];
+                    vs[V_GAM + r] = gam;
+                    vs[V_F + r] = __expf(GC - G[e]);
+                    vs[V_BETA + r] = be;
+                    vs[V_BG + r] = be * gam;
+                }
+                if (lane == 0) vs[V_GC] = __expf(GC);
+                __syncwarp();
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = lane + 32 * e;
+                    vs[V_EROW + r] = __expf(vs[V_G + r] - vs[V_G + (r & ~15)]);
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) vs[V_ECOL + rb * 64 + r] = __expf(vs[V_G + 16 * rb] - vs[V_G + r]);
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(bar(B_CV0 + sb));
+            named_bar_sync(2, 128);
+            if (issuer) {
+                const uint32_t stg = sb0 + sb * STG_BYTES;
+                if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t ad = stg + (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_ss(tb + TM_G, sdesc(ad, 16, 1024), sdesc(ad, 16, 1024), ID_GRAM, s > 0);
+                }
+                mma_commit(bar(B_G0 + sb));
+            }
+        };
+
+        float S[128];
+        {
+            const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + p : nullptr;
+#pragma unroll
+            for (int dk = 0; dk < 128; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) st_chunk8(sb0 + swz_chunk(p, j & 7, OFF_ST16 + (j >> 3) * 16384), S + 8 * j);
+        }
+        float gbn[4] = {0.f, 0.f, 0.f, 0.f};
+        if (issuer) {
+            issue_loads(0);
+            if (NC > 1) issue_loads(1);
+        }
+        if (warp == 0) load_gb(0, gbn);
+        ready_chunk(0, gbn);
+        if (NC > 1) {
+            if (warp == 0) load_gb(1, gbn);
+            ready_chunk(1, gbn);
+        }
+        TOut *ob = reinterpret_cast<TOut *>(a.o) + ((size_t)tok0 * a.Hv + h) * D + p;
+        for (int c = 0; c < NC; ++c) {
+            // P and Qh of this chunk, out of tensor memory into the operand tiles
+            wait(B_P, c & 1);
+            if (issuer && c + 2 < NC) issue_loads(c + 2);   // chunk c's staging buffer is free
+            if (warp == 0 && c + 2 < NC) load_gb(c + 2, gbn);
+            tc_fence_after();
+            {
+                float v[32];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 32 * qq), v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        st_chunk8(sb0 + swz_chunk(p, (4 * qq + j) & 7, OFF_P16 + (qq >> 1) * 16384), v + 8 * j);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * half), v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * half + j, OFF_QH16), v + 8 * j);
+                }
+            }
+            const float gC = vec[(c & 1) * V_SET + V_GC];
+            tc_fence_before();
+            mbar_arrive(bar(B_YE));
+            fence_proxy_async();
+            named_bar_sync(2, 128);
+            if (issuer) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_ss(tb + TM_S, sdesc(sb0 + OFF_ST16 + koff, 16, 1024), sdesc(sb0 + OFF_P16 + koff, 16, 1024),
+                           ID_S, true);
+                }
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_ss(tb + TM_O, sdesc(sb0 + OFF_ST16 + koff, 16, 1024), sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024),
+                           ID_O, true);
+                }
+                mma_commit(bar(B_ST));
+            }
+            wait(B_ST, c & 1);
+            tc_fence_after();
+            // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                float v[32];
+                tmem_ld32(tmem_addr(tb, q4, TM_S + 32 * qq), v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) S[32 * qq + i] = fmaf(gC, S[32 * qq + i], v[i]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    st_chunk8(sb0 + swz_chunk(p, (4 * qq + j) & 7, OFF_ST16 + (qq >> 1) * 16384), S + 32 * qq + 8 * j);
+            }
+            // o rows of this chunk: column p of Qh S + Uh
+            // (even lane: row r, columns p and p + 1; odd lane: row r + 1, columns p - 1 and p)
+            {
+                float o[64];
+                tmem_ld32(tmem_addr(tb, q4, TM_O), o);
+                tmem_ld32(tmem_addr(tb, q4, TM_O + 32), o + 32);
+                tc_fence_before();
+                mbar_arrive(bar(B_SE));
+                mbar_arrive(bar(B_OE));
+                const int nvalid = min(C, T - c * C), odd = p & 1;
+                const size_t rs = (size_t)a.Hv * D;
+                TOut *orow = ob + (size_t)(c * C + odd) * rs - odd;
+#pragma unroll
+                for (int i = 0; i < 64; i += 2) {
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + 1], 1);
+                    if (i + odd < nvalid) out_store2(orow + (size_t)i * rs, odd ? other : o[i], odd ? o[i + 1] : other);
+                }
+            }
+            if (c + 2 < NC) ready_chunk(c + 2, gbn);
+        }
+        if (a.hT) {
+            float *hp = a.hT + (size_t)bh * D * D + p;
+#pragma unroll
+            for (int dk = 0; dk < 128; ++dk) hp[(size_t)dk * D] = S[dk];
+        }
+        if (issuer) {
+            mma_commit(bar(B_DR0));
+            mbar_wait_bounded(bar(B_DR0), 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tb, 512);
+    }
+}
+
+template <typename TOut>
+cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
+{
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, a.q, a.B, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, a.B, a.T, a.Hk, 64, false, true) ||
+        !make_map(&mv, a.v, a.B, a.T, a.Hv, 64, false, true))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
+    if (e != cudaSuccess) return e;
+    tc_fwd_kernel<TOut><<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const FwdArgs &a)
+{
+    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && a.gate_mode == 0 && !a.cu_seqlens && !a.qk_l2norm && !a.z;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st)
+{
+    return out_f32(a.dtype) ? launch_tc_t<float>(a, st) : launch_tc_t<__nv_bfloat16>(a, st);
+}
+
+unsigned int tc_error_count()
+{
+    unsigned int t = 0;
+    cudaMemcpyFromSymbol(&t, g_tc_timeouts, sizeof(t));
+    return t;
+}
+
+}  // namespace gdr

@@ -74,7 +74,12 @@ unsigned long long gdr_kernel_launches(void) { return g_launches.load(); }
 
 unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors)
 {
-    return gdr::fused_error_counts(load_timeouts, range_errors);
+    unsigned int t = 0, r = 0;
+    gdr::fused_error_counts(&t, &r);
+    t += gdr::tc_error_count();
+    if (load_timeouts) *load_timeouts = t;
+    if (range_errors) *range_errors = r;
+    return t + r;
 }
 
 size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype)
@@ -118,6 +123,12 @@ int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
     }
 
     const gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (gdr::tc_supported(a)) {
+        cudaError_t e = gdr::launch_fwd_tc(a, s);
+        if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+        g_launches += 1;
+        return GDR_OK;
+    }
     if (gdr::fused_supported(a)) {
         cudaError_t e = gdr::launch_fwd_fused(a, s);
         if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));

@@ -45,6 +45,13 @@ cudaError_t launch_fwd_fused(const FwdArgs &a, cudaStream_t st);
 // device: chunk loads that timed out, and per-channel gate factors outside the fp16 range.
 unsigned int fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors);
 
+// Chunked forward on the tcgen05 tensor cores (scalar gate, bf16 inputs, Dk = Dv = 128,
+// fixed-length sequences, no layer options): one kernel, no workspace.
+bool tc_supported(const FwdArgs &a);
+cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st);
+// Waits of the tcgen05 kernel that timed out since the library was loaded on this device.
+unsigned int tc_error_count();
+
 // fp32 CUDA-core chunked forward (three kernels). Needs simt_workspace_size() bytes.
 size_t simt_workspace_size(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a, void *ws, cudaStream_t st);

@@ -1,0 +1,119 @@
+// Building blocks of the fifth-generation tensor-core (tcgen05) kernels: tensor
+// memory allocation, shared-memory matrix descriptors for the 128-byte swizzled
+// layout, the instruction descriptor of kind::f16, MMA issue and completion,
+// tensor-memory loads, and the byte offsets of the swizzled tiles that threads
+// write.
+//
+// Every operand tile here is "row-major with 128-byte rows": a row holds 64
+// 16-bit elements, rows sit 128 bytes apart, groups of 8 rows 1024 bytes apart,
+// and the 16-byte chunk j of row r is stored at chunk j ^ (r % 8) (the TMA
+// 128-byte swizzle, so the tiles must start on 1024-byte boundaries). A wider
+// matrix is a sequence of such 64-column atoms, `atom_stride` bytes apart.
+// Read with the rows as the M (or N) index, a tile is a K-major operand; read
+// with the rows as the K index, it is an MN-major operand.
+#pragma once
+#include <stdint.h>
+
+namespace gdr {
+namespace tcu {
+
+// Byte offset of element (row, col) in a tile of 128-byte swizzled rows whose
+// 64-column atoms are `atom_stride` bytes apart.
+__host__ __device__ __forceinline__ uint32_t swz_off(int row, int col, uint32_t atom_stride)
+{
+    const uint32_t byte = (uint32_t)(col & 63) * 2u;
+    return (uint32_t)(col >> 6) * atom_stride + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+           ((((byte >> 4) ^ (uint32_t)(row & 7))) << 4) + (byte & 15u);
+}
+// Byte offset of 16-byte chunk j (columns 8j .. 8j + 7 of the atom) of row `row`.
+__host__ __device__ __forceinline__ uint32_t swz_chunk(int row, int j, uint32_t atom_base)
+{
+    return atom_base + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+           (((uint32_t)j ^ (uint32_t)(row & 7)) << 4);
+}
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and stride
+// byte offsets (16-byte units), descriptor version 1, 128-byte swizzle.
+//   K-major:  SBO = stride between 8-row groups (1024); LBO unused.
+//   MN-major: LBO = stride between 64-element atoms along M/N; SBO = stride
+//             between 8-row groups along K (1024).
+__host__ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16 with fp32 accumulation.
+//   bf16: both operands bf16 (else fp16); a_mn / b_mn: MN-major operand; neg_a: D += (-A) B.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool a_mn, bool b_mn, bool neg_a = false)
+{
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((neg_a ? 1u : 0u) << 13) |
+           ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+#if defined(__CUDACC__)
+// Tensor memory: allocation by one whole warp; the column base is written to shared memory.
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] B[smem] for one K = 16 step, issued by one thread.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+                 ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)acc)
+                 : "memory");
+}
+// Arrive once on the mbarrier when every MMA this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's lane (32x32b shape), waited on in
+// the same statement so no register is read before the load has landed.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Plain arrival of this thread on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Tensor-memory address of lane quarter q (lanes 32q .. 32q + 31), column col.
+__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, int q, int col)
+{
+    return base + ((uint32_t)(32 * q) << 16) + (uint32_t)col;
+}
+#endif
+
+}  // namespace tcu
+}  // namespace gdr
