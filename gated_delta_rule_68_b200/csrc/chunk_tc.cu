@@ -48,7 +48,9 @@ namespace {
 using namespace mmau;
 using namespace tcu;
 
-constexpr int NTH = 256;   // warps 0-3: state group, warps 4-7: chunk group
+constexpr int GW = 8;            // warps per group
+constexpr int GT = 32 * GW;      // threads per group
+constexpr int NTH = 2 * GT;      // warps 0-7: state group, warps 8-15: chunk group
 
 // Shared memory (byte offsets from a 1024-byte aligned base). Operand tiles are
 // 128-byte swizzled rows (tc_util.cuh).
@@ -66,15 +68,13 @@ constexpr uint32_t OFF_U16 = OFF_R1 + 16384;    // U^T [dv][r] fp16
 constexpr uint32_t OFF_INV = OFF_R1 + 16384;    // inverse scratch (dead before U^T is written)
 constexpr uint32_t OFF_M16 = OFF_R1 + 32768;    // M [r][i] fp16
 constexpr uint32_t OFF_VEC = OFF_M16 + 8192;    // per-chunk vectors (fp32)
-// Inverse scratch: fp32 diagonal blocks of A (transposed, [4][16][20]), reused by the
-// 16 x 16 products' intermediates; fp16 off-diagonal rows 16..63 of A ([48][56]);
-// fp16 diagonal inverses D_b ([4][16][24]) and the first off-diagonal blocks T_10, T_32.
+// Inverse scratch: fp32 diagonal blocks of A (transposed, [4][16][20]), fp16
+// off-diagonal rows 16..63 of A ([48][56]) and fp16 diagonal inverses D_b ([4][16][24]).
 constexpr int LDAD = 20, LDA16 = 56, LDT16 = 24;
-constexpr uint32_t INV_AD = OFF_INV, INV_XY = OFF_INV;
+constexpr uint32_t INV_AD = OFF_INV;
 constexpr uint32_t INV_A16 = OFF_INV + 4 * 16 * LDAD * 4;
 constexpr uint32_t INV_D = INV_A16 + 48 * LDA16 * 2;
-constexpr uint32_t INV_T1 = INV_D + 4 * 16 * LDT16 * 2;
-constexpr uint32_t INV_END = INV_T1 + 2 * 16 * LDT16 * 2;
+constexpr uint32_t INV_END = INV_D + 4 * 16 * LDT16 * 2;
 static_assert(INV_END <= OFF_U16 + 16384, "inverse scratch must fit beside T' and T''");
 // vectors
 // Per-chunk vectors, two sets (chunk parity): G, Gamma, f = Gamma_C / Gamma, beta,
@@ -95,7 +95,8 @@ enum {
     B_G0, B_G1,     // Gram of the chunk in staging buffer 0 / 1 done
     B_CV0, B_CV1,   // fp16 tiles and gate vectors of the chunk in buffer 0 / 1 written (128 arrivals)
     B_W,            // W^T, U^T done
-    B_P,            // P, R, Qh, Uh of a chunk done (waited on by both groups)
+    B_P1,           // R, Qh, Uh of a chunk done (M and U^T free)
+    B_P,            // P too: all four products of a chunk done (waited on by both groups)
     B_ST,           // state batch done
     B_GE,           // the chunk group has read the Gram out of tensor memory (128 arrivals)
     B_YE,           // the state group has read P and Qh out of Y and X (128 arrivals)
@@ -150,15 +151,40 @@ __device__ __forceinline__ void mma16(float c0[4], float c1[4], uint32_t aA, int
     mma(c0, af, bf[0], bf[1]);
     mma(c1, af, bf[2], bf[3]);
 }
-// Stores a 16 x 16 fp32 product (two n8 tiles), times `s`, as fp16 row-major at p (stride ld).
-__device__ __forceinline__ void st_tile16(__half *p, int ld, const float c0[4], const float c1[4], float s, int lane)
+// The fp32 accumulator of a 16 x 16 product (two n8 tiles) is laid out as the A
+// fragment of the next m16n8k16 product: c0 holds columns 0..7, c1 columns 8..15.
+__device__ __forceinline__ void acc_to_a(uint32_t a[4], const float c0[4], const float c1[4])
 {
-    const int g = lane >> 2, t4 = lane & 3;
-    st_h2(p + g * ld + 2 * t4, s * c0[0], s * c0[1]);
-    st_h2(p + (g + 8) * ld + 2 * t4, s * c0[2], s * c0[3]);
-    st_h2(p + g * ld + 8 + 2 * t4, s * c1[0], s * c1[1]);
-    st_h2(p + (g + 8) * ld + 8 + 2 * t4, s * c1[2], s * c1[3]);
+    a[0] = pack_h2(c0[0], c0[1]);
+    a[1] = pack_h2(c0[2], c0[3]);
+    a[2] = pack_h2(c1[0], c1[1]);
+    a[3] = pack_h2(c1[2], c1[3]);
 }
+// c (fresh) = A (fragment in registers) B (16 x 16 stored [k][n] at aB, stride ldb).
+__device__ __forceinline__ void mma16r(float c0[4], float c1[4], const uint32_t af[4], uint32_t aB, int ldb, int lane)
+{
+    uint32_t bf[4];
+    ldsm_t(bf, b_kn(aB, ldb, 0, 0, lane));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c0[e] = c1[e] = 0.f;
+    mma(c0, af, bf[0], bf[1]);
+    mma(c1, af, bf[2], bf[3]);
+}
+// c = (A0 B0) B1 ... : a left-to-right chain; the first factor A0 from shared memory.
+__device__ __forceinline__ void chain_start(float c0[4], float c1[4], uint32_t aA, int lda, uint32_t aB, int ldb,
+                                            int lane)
+{
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c0[e] = c1[e] = 0.f;
+    mma16(c0, c1, aA, lda, aB, ldb, lane);
+}
+__device__ __forceinline__ void chain_next(float c0[4], float c1[4], uint32_t aB, int ldb, int lane)
+{
+    uint32_t af[4];
+    acc_to_a(af, c0, c1);
+    mma16r(c0, c1, af, aB, ldb, lane);
+}
+
 // Writes block (R0.., I0..) of T, given as two n8 tiles times `s`, into T diag(beta Gamma)
 // and T diag(beta) (swizzled [r][i] tiles).
 __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const float c0[4], const float c1[4], float s,
@@ -194,14 +220,15 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
-    const int p = tid & 127;          // row of the 128-row products owned by this thread
+    const int p = 32 * q4 + lane;     // row of the 128-row products owned by this thread
+    const int hf = (warp >> 2) & 1;   // which half of that row's columns this thread takes
     const int bh = blockIdx.x, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, NC = (T + C - 1) / C;
     const long tok0 = (long)b * T;
 
     if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), 512);
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 1, 1, 128, 128, 1, 1, 1, 128, 128, 128, 128, 1, 1};
+        const uint32_t counts[NBAR] = {1, 1, 1, 1, GT, GT, 1, 1, 1, 1, GT, GT, GT, GT, 1, 1};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
         abort_sh = 0;
     }
@@ -220,36 +247,36 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         }
     };
 
-    if (warp >= 4) {
+    if (warp >= GW) {
         // ============================ chunk group ============================
         // Per chunk: the gated Gram's epilogue (A, M), the inverse (T diag(beta Gamma),
         // T diag(beta)), W^T and U^T, then P, R, Qh, Uh.
-        const int wq = warp - 4;
-        const bool issuer = tid == 128;
+        const int gt = tid - GT;          // 0 .. GT-1
+        const int wq = q4;                // warp within a half of the group
+        const bool issuer = gt == 0;
         for (int c = 0; c < NC; ++c) {
             const int sb = c & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES;
             uint8_t *stgp = sm + sb * STG_BYTES;
             const float *vc = vec + sb * V_SET;
-            // The previous chunk's last products are done with M, W^T, U^T and the inverse's tiles.
-            if (c >= 1) wait(B_P, (c - 1) & 1);
+            // The previous chunk's last products are done with M and U^T (the inverse's scratch).
+            if (c >= 1) wait(B_P1, (c - 1) & 1);
             wait(B_CV0 + sb, (c >> 1) & 1);
-            // Gram epilogue: A (rows < 64) and M (rows 64..127)
+            // Gram epilogue: A (rows < 64) and M (rows 64..127), columns 32 hf .. 32 hf + 31
             wait(B_G0 + sb, (c >> 1) & 1);
             tc_fence_after();
             {
-                float v[64];
-                tmem_ld32(tmem_addr(tb, q4, TM_G), v);
-                tmem_ld32(tmem_addr(tb, q4, TM_G + 32), v + 32);
+                float v[32];
+                tmem_ld32(tmem_addr(tb, q4, TM_G + 32 * hf), v);
                 tc_fence_before();
                 mbar_arrive(bar(B_GE));
                 // exp(G_r - G_i) = exp(G_r - G_16R) exp(G_16R - G_i), R = r / 16
                 const int r = p & 63, rb = r >> 4;
-                const float4 *ec4 = reinterpret_cast<const float4 *>(vc + V_ECOL + rb * 64);
+                const float4 *ec4 = reinterpret_cast<const float4 *>(vc + V_ECOL + rb * 64 + 32 * hf);
                 const float rowf = p < 64 ? vc[V_BETA + r] * vc[V_EROW + r] : vc[V_EROW + r];
-                const int lim = p < 64 ? r : r + 1;   // A: i < r;  M: i <= r
+                const int lim = (p < 64 ? r : r + 1) - 32 * hf;   // A: i < r;  M: i <= r
 #pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) {
+                for (int i4 = 0; i4 < 8; ++i4) {
                     const float4 e = ec4[i4];
                     const int i = 4 * i4;
                     v[i] = i < lim ? rowf * e.x * v[i] : 0.f;
@@ -259,115 +286,136 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 }
                 if (p >= 64) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(r, j, OFF_M16), v + 8 * j);
+                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(r, 4 * hf + j, OFF_M16), v + 8 * j);
                 } else {
                     // fp16 blocks left of the diagonal block (rows 16..63 of A), fp32 diagonal block transposed
                     const uint32_t a16 = sb0 + INV_A16 + (uint32_t)((r - 16) * LDA16) * 2u;
 #pragma unroll
-                    for (int j = 0; j < 6; ++j)
-                        if (j < 2 * rb) st_chunk8(a16 + 16 * j, v + 8 * j);
-                    float *ad = reinterpret_cast<float *>(sm + INV_AD) + rb * 16 * LDAD + (r - 16 * rb);
-                    switch (rb) {
-#define GDR_AD_CASE(K)                                                         \
-    case K:                                                                    \
-        _Pragma("unroll") for (int ii = 0; ii < 16; ++ii) ad[ii * LDAD] = v[16 * K + ii]; \
-        break;
-                        GDR_AD_CASE(0) GDR_AD_CASE(1) GDR_AD_CASE(2) GDR_AD_CASE(3)
-#undef GDR_AD_CASE
+                    for (int j = 0; j < 4; ++j)
+                        if (4 * hf + j < 2 * rb) st_chunk8(a16 + 16 * (4 * hf + j), v + 8 * j);
+                    if ((rb >> 1) == hf) {
+                        float *ad = reinterpret_cast<float *>(sm + INV_AD) + rb * 16 * LDAD + (r - 16 * rb);
+                        if (rb & 1) {
+#pragma unroll
+                            for (int ii = 0; ii < 16; ++ii) ad[ii * LDAD] = v[16 + ii];
+                        } else {
+#pragma unroll
+                            for (int ii = 0; ii < 16; ++ii) ad[ii * LDAD] = v[ii];
+                        }
                     }
                 }
             }
             fence_proxy_async();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, GT);
 
-            // Inverse, level 0: warp wq inverts the unit lower 16 x 16 block I + A_bb (b = wq)
-            // by forward substitution (lane j < 16 holds column j); lanes 16..31 zero the
-            // blocks of T above the diagonal.
-            if (lane < 16) {
-                const int j = lane;
-                float t[16];
+            // ... and with W^T (the tiles of T) before they are rewritten.
+            if (c >= 1) wait(B_P, (c - 1) & 1);
+            // Inverse, level 0: warp wq of the first half inverts the unit lower 16 x 16 block
+            // I + A_bb (b = wq) by forward substitution (lane j < 16 holds column j); the
+            // second half zeroes the blocks of T above the diagonal.
+            if (hf == 0) {
+                if (lane < 16) {
+                    const int j = lane;
+                    float t[16];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) t[rr] = rr == j ? 1.f : 0.f;
-                const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;
+                    for (int rr = 0; rr < 16; ++rr) t[rr] = rr == j ? 1.f : 0.f;
+                    const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;
 #pragma unroll
-                for (int i = 0; i < 15; ++i) {
-                    float col[16];
+                    for (int i = 0; i < 15; ++i) {
+                        float col[16];
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const float4 x = *reinterpret_cast<const float4 *>(ad + i * LDAD + 4 * k4);
-                        col[4 * k4] = x.x, col[4 * k4 + 1] = x.y, col[4 * k4 + 2] = x.z, col[4 * k4 + 3] = x.w;
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const float4 x = *reinterpret_cast<const float4 *>(ad + i * LDAD + 4 * k4);
+                            col[4 * k4] = x.x, col[4 * k4 + 1] = x.y, col[4 * k4 + 2] = x.z, col[4 * k4 + 3] = x.w;
+                        }
+                        const float ti = t[i];
+#pragma unroll
+                        for (int rr = i + 1; rr < 16; ++rr) t[rr] = fmaf(-col[rr], ti, t[rr]);
                     }
-                    const float ti = t[i];
+                    __half *dd = reinterpret_cast<__half *>(sm + INV_D) + wq * 16 * LDT16;
+                    const int I = 16 * wq + j;
+                    const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
 #pragma unroll
-                    for (int rr = i + 1; rr < 16; ++rr) t[rr] = fmaf(-col[rr], ti, t[rr]);
-                }
-                __half *dd = reinterpret_cast<__half *>(sm + INV_D) + wq * 16 * LDT16;
-                const int I = 16 * wq + j;
-                const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    dd[rr * LDT16 + j] = __float2half_rn(t[rr]);
-                    st_h1(sm, OFF_TP + swz_off(16 * wq + rr, I, 0), t[rr] * sbg);
-                    st_h1(sm, OFF_TPP + swz_off(16 * wq + rr, I, 0), t[rr] * sbt);
+                    for (int rr = 0; rr < 16; ++rr) {
+                        dd[rr * LDT16 + j] = __float2half_rn(t[rr]);
+                        st_h1(sm, OFF_TP + swz_off(16 * wq + rr, I, 0), t[rr] * sbg);
+                        st_h1(sm, OFF_TPP + swz_off(16 * wq + rr, I, 0), t[rr] * sbt);
+                    }
                 }
             } else {
-                // zero chunks: rows of block R, 16-byte chunks 2(R+1) .. 7
-                const int u = wq * 16 + (lane - 16);   // 0..63: one row each
-                const int R = u >> 4;
+                // zero chunks: row u of block R = u / 16, 16-byte chunks 2(R+1) .. 7, of one of the two tiles
+                const int u = (gt - GT / 2) & 63, R = u >> 4;
+                const uint32_t tile = (gt - GT / 2) < 64 ? OFF_TP : OFF_TPP;
                 const uint4 z = make_uint4(0, 0, 0, 0);
-                for (int j = 2 * (R + 1); j < 8; ++j) {
-                    *reinterpret_cast<uint4 *>(sm + swz_chunk(u, j, OFF_TP)) = z;
-                    *reinterpret_cast<uint4 *>(sm + swz_chunk(u, j, OFF_TPP)) = z;
-                }
+                for (int j = 2 * (R + 1); j < 8; ++j) *reinterpret_cast<uint4 *>(sm + swz_chunk(u, j, tile)) = z;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, GT);
 
-            const uint32_t aD = sb0 + INV_D, aA16 = sb0 + INV_A16, aXY = sb0 + INV_XY, aT1 = sb0 + INV_T1;
-            constexpr uint32_t T16B = 16 * LDT16 * 2;   // bytes of one [16][24] fp16 tile
-            // Level 1: T_10 = -D_1 A_10 D_0 (warp 1), T_32 = -D_3 A_32 D_2 (warp 3).
-            if (wq & 1) {
-                const int m = wq - 1;
-                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-                mma16(c0, c1, aA16 + ((16 * (wq - 1)) * LDA16 + 16 * m) * 2, LDA16, aD + m * T16B, LDT16, lane);
-                __half *xw = reinterpret_cast<__half *>(sm + INV_XY) + wq * 16 * LDT16;
-                st_tile16(xw, LDT16, c0, c1, 1.f, lane);
-                __syncwarp();
-                float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-                mma16(d0, d1, aD + wq * T16B, LDT16, aXY + wq * T16B, LDT16, lane);
-                st_tile16(reinterpret_cast<__half *>(sm + INV_T1) + (wq >> 1) * 16 * LDT16, LDT16, d0, d1, -1.f,
-                          lane);
-                st_tblock(sm, 16 * wq, 16 * m, d0, d1, -1.f, vc, lane);
-            }
-            named_bar_sync(1, 128);
-            // Level 2 (warp wq -> block (a, bc) of the lower-left 32 x 32 block, a = 2 + wq / 2, bc = wq % 2):
-            //   Y_a,bc = A_a,0:2 T_0:2,bc;   T_a,bc = -(T_a,2:4 Y_2:4,bc)
-            {
-                const int ar = 2 + (wq >> 1), bc = wq & 1;
-                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t arow = aA16 + ((16 * (ar - 1)) * LDA16) * 2;
-                if (bc == 0) {
-                    mma16(c0, c1, arow, LDA16, aD, LDT16, lane);                    // A_a0 D_0
-                    mma16(c0, c1, arow + 16 * 2, LDA16, aT1, LDT16, lane);          // A_a1 T_10
+            // Off-diagonal blocks of T = (I + A)^-1 (D_b the diagonal inverses): expanding
+            //   T_ij = -D_i sum_{j <= m < i} A_im T_mj
+            // gives sums of alternating chains D A D A ... D, each evaluated left to right so
+            // that every right factor is a D or A tile in shared memory and every partial
+            // product stays in registers (the accumulator is the next A fragment).
+            //   warp 0: T_10 = -D1 A10 D0,  T_21 = -D2 A21 D1
+            //   warp 1: T_32 = -D3 A32 D2,  T_20 = (D2 A21 D1 A10 - D2 A20) D0
+            //   warp 2: T_31 = (D3 A32 D2 A21 - D3 A31) D1
+            //   warp 3: T_30 = ((D3 A31 - D3 A32 D2 A21) D1 A10 + D3 A32 D2 A20 - D3 A30) D0
+            if (hf == 0) {
+                const uint32_t aD = sb0 + INV_D, aA16 = sb0 + INV_A16;
+                constexpr uint32_t T16B = 16 * LDT16 * 2;   // bytes of one [16][24] fp16 tile
+                auto Dt = [&](int i) { return aD + i * T16B; };
+                auto At = [&](int i, int j) { return aA16 + ((16 * (i - 1)) * LDA16 + 16 * j) * 2; };
+                float c0[4], c1[4], u0[4], u1[4];
+                if (wq == 0) {
+                    chain_start(c0, c1, Dt(1), LDT16, At(1, 0), LDA16, lane);
+                    chain_next(c0, c1, Dt(0), LDT16, lane);
+                    st_tblock(sm, 16, 0, c0, c1, -1.f, vc, lane);
+                    chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
+                    chain_next(c0, c1, Dt(1), LDT16, lane);
+                    st_tblock(sm, 32, 16, c0, c1, -1.f, vc, lane);
+                } else if (wq == 1) {
+                    chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
+                    chain_next(c0, c1, Dt(2), LDT16, lane);
+                    st_tblock(sm, 48, 32, c0, c1, -1.f, vc, lane);
+                    chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
+                    chain_next(c0, c1, Dt(1), LDT16, lane);
+                    chain_next(c0, c1, At(1, 0), LDA16, lane);
+                    chain_start(u0, u1, Dt(2), LDT16, At(2, 0), LDA16, lane);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
+                    chain_next(c0, c1, Dt(0), LDT16, lane);
+                    st_tblock(sm, 32, 0, c0, c1, 1.f, vc, lane);
+                } else if (wq == 2) {
+                    chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
+                    chain_next(c0, c1, Dt(2), LDT16, lane);
+                    chain_next(c0, c1, At(2, 1), LDA16, lane);
+                    chain_start(u0, u1, Dt(3), LDT16, At(3, 1), LDA16, lane);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
+                    chain_next(c0, c1, Dt(1), LDT16, lane);
+                    st_tblock(sm, 48, 16, c0, c1, 1.f, vc, lane);
                 } else {
-                    mma16(c0, c1, arow + 16 * 2, LDA16, aD + T16B, LDT16, lane);    // A_a1 D_1
+                    float q0[4], q1[4], h0[4], h1[4];
+                    chain_start(q0, q1, Dt(3), LDT16, At(3, 2), LDA16, lane);   // Q = D3 A32 D2
+                    chain_next(q0, q1, Dt(2), LDT16, lane);
+                    uint32_t qf[4];
+                    acc_to_a(qf, q0, q1);
+                    mma16r(h0, h1, qf, At(2, 1), LDA16, lane);                  // Q A21
+                    chain_start(u0, u1, Dt(3), LDT16, At(3, 1), LDA16, lane);   // D3 A31
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) u0[e] -= h0[e], u1[e] -= h1[e];
+                    chain_next(u0, u1, Dt(1), LDT16, lane);                     // (D3 A31 - Q A21) D1 A10
+                    chain_next(u0, u1, At(1, 0), LDA16, lane);
+                    mma16r(h0, h1, qf, At(2, 0), LDA16, lane);                  // Q A20
+                    chain_start(c0, c1, Dt(3), LDT16, At(3, 0), LDA16, lane);   // D3 A30
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) c0[e] = u0[e] + h0[e] - c0[e], c1[e] = u1[e] + h1[e] - c1[e];
+                    chain_next(c0, c1, Dt(0), LDT16, lane);
+                    st_tblock(sm, 48, 0, c0, c1, 1.f, vc, lane);
                 }
-                __half *yw = reinterpret_cast<__half *>(sm + INV_XY) + wq * 16 * LDT16;
-                st_tile16(yw, LDT16, c0, c1, 1.f, lane);
-            }
-            named_bar_sync(1, 128);
-            {
-                const int ar = 2 + (wq >> 1), bc = wq & 1;
-                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-                if (ar == 2) {
-                    mma16(c0, c1, aD + 2 * T16B, LDT16, aXY + bc * T16B, LDT16, lane);           // D_2 Y_2,bc
-                } else {
-                    mma16(c0, c1, aT1 + T16B, LDT16, aXY + bc * T16B, LDT16, lane);              // T_32 Y_2,bc
-                    mma16(c0, c1, aD + 3 * T16B, LDT16, aXY + (2 + bc) * T16B, LDT16, lane);     // D_3 Y_3,bc
-                }
-                st_tblock(sm, 16 * ar, 16 * bc, c0, c1, -1.f, vc, lane);
             }
             fence_proxy_async();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, GT);
 
             // W^T = K^T T'^T -> Y[0:64),  U^T = V^T T''^T -> Y[64:128), once the state
             // group has read the previous chunk's P and Qh out of Y and X.
@@ -390,23 +438,17 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             tc_fence_after();
             {
                 float v[32];
+                tmem_ld32(tmem_addr(tb, q4, TM_Y + 32 * hf), v);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 32 * half), v);
+                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_W16), v + 8 * j);
+                tmem_ld32(tmem_addr(tb, q4, TM_Y + 64 + 32 * hf), v);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * half + j, OFF_W16), v + 8 * j);
-                }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 64 + 32 * half), v);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * half + j, OFF_U16), v + 8 * j);
-                }
+                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_U16), v + 8 * j);
             }
             // K -> Kt = diag(Gamma_C / Gamma) K in place (the W product is done with K)
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const int e = p + 128 * jj, tok = (e >> 3) & 63;
+            for (int jj = 0; jj < 1024 / GT; ++jj) {
+                const int e = gt + GT * jj, tok = (e >> 3) & 63;
                 uint4 *pch = reinterpret_cast<uint4 *>(stgp + (e >> 9) * 16384) + (e & 511);
                 const float f = vc[V_F + tok];
                 uint4 u = *pch;
@@ -418,10 +460,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 }
                 *pch = u;
             }
-            // diag(Gamma) [r][j] into the dead V tile: 4 of its 16-byte chunks per thread
+            // diag(Gamma) [r][j] into the dead V tile
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int e = p + 128 * jj, r = e >> 3, j = e & 7;
+            for (int jj = 0; jj < 512 / GT; ++jj) {
+                const int e = gt + GT * jj, r = e >> 3, j = e & 7;
                 float x[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? vc[V_GAM + r] : 0.f;
@@ -429,18 +471,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             }
             tc_fence_before();
             fence_proxy_async();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, GT);
 
-            // P = -Kt^T W -> Y,  R^T = U^T Kt -> state product,  X = Q^T diag(Gamma) - W^T M^T -> X,
-            // Uh^T = U^T M^T -> o accumulator.
+            // R^T = U^T Kt -> state product,  X = Q^T diag(Gamma) - W^T M^T -> X,
+            // Uh^T = U^T M^T -> o accumulator (these free M and U^T), then P = -Kt^T W -> Y.
             if (issuer) {
                 if (c >= 1) wait(B_SE, (c - 1) & 1);
                 if (c >= 1) wait(B_OE, (c - 1) & 1);
                 tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_ss(tb + TM_Y, sdesc(stg + s * 2048, 16384, 1024), sdesc(sb0 + OFF_W16 + s * 32, 16, 1024),
-                           ID_P, s > 0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_ss(tb + TM_S, sdesc(sb0 + OFF_U16 + s * 32, 16, 1024), sdesc(stg + s * 2048, 16384, 1024),
@@ -457,6 +495,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 for (int s = 0; s < 4; ++s)
                     mma_ss(tb + TM_O, sdesc(sb0 + OFF_U16 + s * 32, 16, 1024), sdesc(sb0 + OFF_M16 + s * 32, 16, 1024),
                            ID_UH, s > 0);
+                mma_commit(bar(B_P1));
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tb + TM_Y, sdesc(stg + s * 2048, 16384, 1024), sdesc(sb0 + OFF_W16 + s * 32, 16, 1024),
+                           ID_P, s > 0);
                 mma_commit(bar(B_P));
             }
         }
@@ -466,9 +509,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         }
     } else {
         // ============================ state group ============================
-        // Thread p owns value column p: S[:, p] in fp32 registers. Besides the state step
-        // of chunk c, the group readies chunk c + 2: its TMA loads, the bf16 -> fp16
-        // conversion of K, Q and V in place, the gate vectors and the Gram.
+        // Thread (p, hf) owns rows dk = 64 hf .. 64 hf + 63 of value column p of S, in fp32
+        // registers. Besides the state step of chunk c, the group readies chunk c + 2: its
+        // TMA loads, the bf16 -> fp16 conversion of K, Q and V in place, the gate vectors
+        // and the Gram.
         const bool issuer = tid == 0;
         auto issue_loads = [&](int c) {
             const int sb = c & 1;
@@ -500,12 +544,13 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             uint8_t *stgp = sm + sb * STG_BYTES;
             float *vs = vec + sb * V_SET;
             wait(B_LD0 + sb, (c >> 1) & 1);
-#pragma unroll 8
-            for (int j = 0; j < 24; ++j) {
-                uint4 *pch = reinterpret_cast<uint4 *>(stgp) + p + 128 * j;   // all 3072 chunks of [K; Q] and V
+#pragma unroll
+            for (int j = 0; j < 3072 / GT; ++j) {
+                uint4 *pch = reinterpret_cast<uint4 *>(stgp) + tid + GT * j;   // all chunks of [K; Q] and V
                 *pch = bf16x8_to_f16x8(*pch);
             }
-            if (warp == 0) {
+            // Gate vectors: every warp scans G (lane l: rows l, l + 32), then writes its share.
+            if (warp < 6) {
                 float s0 = gb[0], s1 = gb[1];
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -515,30 +560,33 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 s1 += __shfl_sync(0xffffffffu, s0, 31);
                 const float GC = __shfl_sync(0xffffffffu, s1, 31);
                 const float G[2] = {s0, s1};
+                if (warp == 0) {
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int r = lane + 32 * e;
-                    const float be = gb[2 + e];
-                    const float gam = __expf(G[e]);
-                    vs[V_G + r] = G[e];
-                    vs[V_GAM + r] = gam;
-                    vs[V_F + r] = __expf(GC - G[e]);
-                    vs[V_BETA + r] = be;
-                    vs[V_BG + r] = be * gam;
-                }
-                if (lane == 0) vs[V_GC] = __expf(GC);
-                __syncwarp();
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int r = lane + 32 * e;
-                    vs[V_EROW + r] = __expf(vs[V_G + r] - vs[V_G + (r & ~15)]);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) vs[V_ECOL + rb * 64 + r] = __expf(vs[V_G + 16 * rb] - vs[V_G + r]);
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = lane + 32 * e;
+                        const float be = gb[2 + e];
+                        const float gam = __expf(G[e]);
+                        vs[V_G + r] = G[e];
+                        vs[V_GAM + r] = gam;
+                        vs[V_F + r] = __expf(GC - G[e]);
+                        vs[V_BETA + r] = be;
+                        vs[V_BG + r] = be * gam;
+                    }
+                    if (lane == 0) vs[V_GC] = __expf(GC);
+                } else if (warp == 1) {   // exp(G_r - G_16R), R = r / 16
+                    const float b0 = __shfl_sync(0xffffffffu, s0, lane & ~15), b1 = __shfl_sync(0xffffffffu, s1, lane & ~15);
+                    vs[V_EROW + lane] = __expf(s0 - b0);
+                    vs[V_EROW + 32 + lane] = __expf(s1 - b1);
+                } else {                  // exp(G_16R - G_i) for R = warp - 2
+                    const int rb = warp - 2;
+                    const float ref = rb < 2 ? __shfl_sync(0xffffffffu, s0, 16 * rb) : __shfl_sync(0xffffffffu, s1, 16 * (rb - 2));
+                    vs[V_ECOL + rb * 64 + lane] = __expf(ref - s0);
+                    vs[V_ECOL + rb * 64 + 32 + lane] = __expf(ref - s1);
                 }
             }
             fence_proxy_async();
             mbar_arrive(bar(B_CV0 + sb));
-            named_bar_sync(2, 128);
+            named_bar_sync(2, GT);
             if (issuer) {
                 const uint32_t stg = sb0 + sb * STG_BYTES;
                 if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
@@ -552,53 +600,48 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             }
         };
 
-        float S[128];
+        float S[64];
         {
-            const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + p : nullptr;
+            const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + (size_t)(64 * hf) * D + p : nullptr;
 #pragma unroll
-            for (int dk = 0; dk < 128; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
+            for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) st_chunk8(sb0 + swz_chunk(p, j & 7, OFF_ST16 + (j >> 3) * 16384), S + 8 * j);
+            for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
         }
         float gbn[4] = {0.f, 0.f, 0.f, 0.f};
         if (issuer) {
             issue_loads(0);
             if (NC > 1) issue_loads(1);
         }
-        if (warp == 0) load_gb(0, gbn);
+        load_gb(0, gbn);
         ready_chunk(0, gbn);
         if (NC > 1) {
-            if (warp == 0) load_gb(1, gbn);
+            load_gb(1, gbn);
             ready_chunk(1, gbn);
         }
-        TOut *ob = reinterpret_cast<TOut *>(a.o) + ((size_t)tok0 * a.Hv + h) * D + p;
         for (int c = 0; c < NC; ++c) {
             // P and Qh of this chunk, out of tensor memory into the operand tiles
             wait(B_P, c & 1);
             if (issuer && c + 2 < NC) issue_loads(c + 2);   // chunk c's staging buffer is free
-            if (warp == 0 && c + 2 < NC) load_gb(c + 2, gbn);
+            if (c + 2 < NC) load_gb(c + 2, gbn);
             tc_fence_after();
             {
                 float v[32];
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 32 * qq), v);
+                for (int qq = 0; qq < 2; ++qq) {
+                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 64 * hf + 32 * qq), v);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        st_chunk8(sb0 + swz_chunk(p, (4 * qq + j) & 7, OFF_P16 + (qq >> 1) * 16384), v + 8 * j);
+                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * qq + j, OFF_P16 + hf * 16384), v + 8 * j);
                 }
+                tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * half), v);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * half + j, OFF_QH16), v + 8 * j);
-                }
+                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
             }
             const float gC = vec[(c & 1) * V_SET + V_GC];
             tc_fence_before();
             mbar_arrive(bar(B_YE));
             fence_proxy_async();
-            named_bar_sync(2, 128);
+            named_bar_sync(2, GT);
             if (issuer) {
                 tc_fence_after();
 #pragma unroll
@@ -619,29 +662,28 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             tc_fence_after();
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
+            for (int qq = 0; qq < 2; ++qq) {
                 float v[32];
-                tmem_ld32(tmem_addr(tb, q4, TM_S + 32 * qq), v);
+                tmem_ld32(tmem_addr(tb, q4, TM_S + 64 * hf + 32 * qq), v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) S[32 * qq + i] = fmaf(gC, S[32 * qq + i], v[i]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    st_chunk8(sb0 + swz_chunk(p, (4 * qq + j) & 7, OFF_ST16 + (qq >> 1) * 16384), S + 32 * qq + 8 * j);
+                    st_chunk8(sb0 + swz_chunk(p, 4 * qq + j, OFF_ST16 + hf * 16384), S + 32 * qq + 8 * j);
             }
-            // o rows of this chunk: column p of Qh S + Uh
+            // o rows 32 hf .. 32 hf + 31 of this chunk: column p of Qh S + Uh
             // (even lane: row r, columns p and p + 1; odd lane: row r + 1, columns p - 1 and p)
             {
-                float o[64];
-                tmem_ld32(tmem_addr(tb, q4, TM_O), o);
-                tmem_ld32(tmem_addr(tb, q4, TM_O + 32), o + 32);
+                float o[32];
+                tmem_ld32(tmem_addr(tb, q4, TM_O + 32 * hf), o);
                 tc_fence_before();
                 mbar_arrive(bar(B_SE));
                 mbar_arrive(bar(B_OE));
-                const int nvalid = min(C, T - c * C), odd = p & 1;
+                const int nvalid = min(C, T - c * C) - 32 * hf, odd = p & 1;
                 const size_t rs = (size_t)a.Hv * D;
-                TOut *orow = ob + (size_t)(c * C + odd) * rs - odd;
+                TOut *orow = reinterpret_cast<TOut *>(a.o) + ((size_t)tok0 * a.Hv + h) * D + p + (size_t)(c * C + 32 * hf + odd) * rs - odd;
 #pragma unroll
-                for (int i = 0; i < 64; i += 2) {
+                for (int i = 0; i < 32; i += 2) {
                     const float other = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + 1], 1);
                     if (i + odd < nvalid) out_store2(orow + (size_t)i * rs, odd ? other : o[i], odd ? o[i + 1] : other);
                 }
@@ -649,9 +691,9 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             if (c + 2 < NC) ready_chunk(c + 2, gbn);
         }
         if (a.hT) {
-            float *hp = a.hT + (size_t)bh * D * D + p;
+            float *hp = a.hT + (size_t)bh * D * D + (size_t)(64 * hf) * D + p;
 #pragma unroll
-            for (int dk = 0; dk < 128; ++dk) hp[(size_t)dk * D] = S[dk];
+            for (int dk = 0; dk < 64; ++dk) hp[(size_t)dk * D] = S[dk];
         }
         if (issuer) {
             mma_commit(bar(B_DR0));
