@@ -98,8 +98,10 @@ __device__ __forceinline__ void fused_unit(const FwdArgs &a, const CUtensorMap *
     constexpr int NJG = C / NCS / 8;    // n8 tiles of a warp in the Gram [128 x 64]
     constexpr int RPT = C / NQ;         // GATE 1: rows per thread in the per-channel pass
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    // 1024-byte aligned base: the TMA tiles need 128 B, the swizzled o tile 1024 B.
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base: the TMA tiles need 128 B, the swizzled o tile 1024 B. An offset
+    // into the __shared__ array (not an integer round trip), so that accesses through it stay
+    // shared-memory instructions.
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __half *sK = reinterpret_cast<__half *>(sm + OFF_K), *sQ = reinterpret_cast<__half *>(sm + OFF_Q);
     __half *sV = reinterpret_cast<__half *>(sm + OFF_V), *sW = reinterpret_cast<__half *>(sm + OFF_W);
     __half *sU = reinterpret_cast<__half *>(sm + OFF_U), *sUE = reinterpret_cast<__half *>(sm + OFF_UE);

@@ -210,7 +210,9 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
               const __grid_constant__ CUtensorMap map_v)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Offset into the __shared__ array (not an integer round trip), so that accesses
+    // through it stay shared-memory instructions.
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb0 = smem_u32(sm);
     float *vec = reinterpret_cast<float *>(sm + OFF_VEC);
     __shared__ uint64_t bars[NBAR];
@@ -223,8 +225,17 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     const int p = 32 * q4 + lane;     // row of the 128-row products owned by this thread
     const int hf = (warp >> 2) & 1;   // which half of that row's columns this thread takes
     const int bh = blockIdx.x, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
-    const int T = a.T, NC = (T + C - 1) / C;
-    const long tok0 = (long)b * T;
+    // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
+    // maps, batch index tbb and token offset tt0. Packed input: sequence b of cu_seqlens
+    // (clamped into the token axis); the rows of its last chunk past its end are zeroed
+    // when the chunk is converted, since the loaded tile holds the next sequence there.
+    int T = a.T, tbb = b, tt0 = 0;
+    long tok0 = (long)b * a.T;
+    if (a.cu_seqlens) {
+        const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
+        T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
+    }
+    const int NC = (T + C - 1) / C;
 
     if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), 512);
     if (tid == 0) {
@@ -517,14 +528,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         auto issue_loads = [&](int c) {
             const int sb = c & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES, bl = bar(B_LD0 + sb);
-            const int t0 = c * C;
+            const int t0 = tt0 + c * C;
             mbar_expect_tx(bl, STG_BYTES);
-            tma_load_4d(stg, &map_k, 0, hk, t0, b, bl);
-            tma_load_4d(stg + 16384, &map_k, 64, hk, t0, b, bl);
-            tma_load_4d(stg + STG_Q, &map_q, 0, hk, t0, b, bl);
-            tma_load_4d(stg + 16384 + STG_Q, &map_q, 64, hk, t0, b, bl);
-            tma_load_4d(stg + STG_V, &map_v, 0, h, t0, b, bl);
-            tma_load_4d(stg + STG_V + 8192, &map_v, 64, h, t0, b, bl);
+            tma_load_4d(stg, &map_k, 0, hk, t0, tbb, bl);
+            tma_load_4d(stg + 16384, &map_k, 64, hk, t0, tbb, bl);
+            tma_load_4d(stg + STG_Q, &map_q, 0, hk, t0, tbb, bl);
+            tma_load_4d(stg + 16384 + STG_Q, &map_q, 64, hk, t0, tbb, bl);
+            tma_load_4d(stg + STG_V, &map_v, 0, h, t0, tbb, bl);
+            tma_load_4d(stg + STG_V + 8192, &map_v, 64, h, t0, tbb, bl);
         };
         // g and beta of chunk c (zero past T), read by warp 0: lane l has rows l and l + 32.
         auto load_gb = [&](int c, float gb[4]) {
@@ -544,10 +555,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             uint8_t *stgp = sm + sb * STG_BYTES;
             float *vs = vec + sb * V_SET;
             wait(B_LD0 + sb, (c >> 1) & 1);
+            const int nvalid = min(C, T - c * C);
 #pragma unroll
             for (int j = 0; j < 3072 / GT; ++j) {
-                uint4 *pch = reinterpret_cast<uint4 *>(stgp) + tid + GT * j;   // all chunks of [K; Q] and V
-                *pch = bf16x8_to_f16x8(*pch);
+                // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64 rows)
+                const int e = tid + GT * j;
+                const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
+                uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
+                *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
             }
             // Gate vectors: every warp scans G (lane l: rows l, l + 32), then writes its share.
             if (warp < 6) {
@@ -609,12 +624,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
         }
         float gbn[4] = {0.f, 0.f, 0.f, 0.f};
-        if (issuer) {
+        if (issuer && NC > 0) {
             issue_loads(0);
             if (NC > 1) issue_loads(1);
         }
-        load_gb(0, gbn);
-        ready_chunk(0, gbn);
+        if (NC > 0) {
+            load_gb(0, gbn);
+            ready_chunk(0, gbn);
+        }
         if (NC > 1) {
             load_gb(1, gbn);
             ready_chunk(1, gbn);
@@ -712,8 +729,9 @@ template <typename TOut>
 cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
 {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, a.B, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, a.B, a.T, a.Hk, 64, false, true) ||
-        !make_map(&mv, a.v, a.B, a.T, a.Hv, 64, false, true))
+    const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
+    if (!make_map(&mq, a.q, mb, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, mb, a.T, a.Hk, 64, false, true) ||
+        !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
@@ -725,7 +743,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
 
 bool tc_supported(const FwdArgs &a)
 {
-    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && a.gate_mode == 0 && !a.cu_seqlens && !a.qk_l2norm && !a.z;
+    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && a.gate_mode == 0 && !a.qk_l2norm && !a.z;
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st)

@@ -178,7 +178,7 @@ int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, const fl
         }
         return GDR_OK;
     }
-    cudaError_t e = gdr::launch_fwd_fused(a, s);
+    cudaError_t e = gdr::tc_supported(a) ? gdr::launch_fwd_tc(a, s) : gdr::launch_fwd_fused(a, s);
     if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
     g_launches += 1;
     return GDR_OK;
@@ -222,7 +222,7 @@ int gdr_fwd_chunked_norm(const void *q, const void *k, const void *v, const floa
         }
         return GDR_OK;
     }
-    cudaError_t e = gdr::launch_fwd_fused(a, s);
+    cudaError_t e = gdr::tc_supported(a) ? gdr::launch_fwd_tc(a, s) : gdr::launch_fwd_fused(a, s);
     if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
     g_launches += 1;
     return GDR_OK;
