@@ -270,8 +270,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             const uint32_t stg = sb0 + sb * STG_BYTES;
             uint8_t *stgp = sm + sb * STG_BYTES;
             const float *vc = vec + sb * V_SET;
-            // The previous chunk's last products are done with M and U^T (the inverse's scratch).
-            if (c >= 1) wait(B_P1, (c - 1) & 1);
             wait(B_CV0 + sb, (c >> 1) & 1);
             // Gram epilogue: A (rows < 64) and M (rows 64..127), columns 32 hf .. 32 hf + 31
             wait(B_G0 + sb, (c >> 1) & 1);
@@ -295,6 +293,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     v[i + 2] = i + 2 < lim ? rowf * e.z * v[i + 2] : 0.f;
                     v[i + 3] = i + 3 < lim ? rowf * e.w * v[i + 3] : 0.f;
                 }
+                // The previous chunk's first products are done with M and U^T (the inverse's scratch).
+                if (c >= 1) wait(B_P1, (c - 1) & 1);
                 if (p >= 64) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(r, 4 * hf + j, OFF_M16), v + 8 * j);
@@ -448,13 +448,12 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             wait(B_W, c & 1);
             tc_fence_after();
             {
-                float v[32];
-                tmem_ld32(tmem_addr(tb, q4, TM_Y + 32 * hf), v);
+                float v[64];
+                tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 32 * hf), tmem_addr(tb, q4, TM_Y + 64 + 32 * hf), v);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_W16), v + 8 * j);
-                tmem_ld32(tmem_addr(tb, q4, TM_Y + 64 + 32 * hf), v);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_U16), v + 8 * j);
+                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_U16), v + 32 + 8 * j);
             }
             // K -> Kt = diag(Gamma_C / Gamma) K in place (the W product is done with K)
 #pragma unroll
@@ -638,21 +637,23 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         }
         for (int c = 0; c < NC; ++c) {
             // P and Qh of this chunk, out of tensor memory into the operand tiles
+            wait(B_P1, c & 1);
+            tc_fence_after();
+            {
+                float v[32];
+                tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
+            }
             wait(B_P, c & 1);
             if (issuer && c + 2 < NC) issue_loads(c + 2);   // chunk c's staging buffer is free
             if (c + 2 < NC) load_gb(c + 2, gbn);
             tc_fence_after();
             {
-                float v[32];
+                float v[64];
+                tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 64 * hf), tmem_addr(tb, q4, TM_Y + 64 * hf + 32), v);
 #pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
-                    tmem_ld32(tmem_addr(tb, q4, TM_Y + 64 * hf + 32 * qq), v);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * qq + j, OFF_P16 + hf * 16384), v + 8 * j);
-                }
-                tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
+                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
             }
             const float gC = vec[(c & 1) * V_SET + V_GC];
             tc_fence_before();
@@ -678,15 +679,13 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             wait(B_ST, c & 1);
             tc_fence_after();
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
+            {
+                float v[64];
+                tmem_ld32x2(tmem_addr(tb, q4, TM_S + 64 * hf), tmem_addr(tb, q4, TM_S + 64 * hf + 32), v);
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                float v[32];
-                tmem_ld32(tmem_addr(tb, q4, TM_S + 64 * hf + 32 * qq), v);
+                for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) S[32 * qq + i] = fmaf(gC, S[32 * qq + i], v[i]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    st_chunk8(sb0 + swz_chunk(p, 4 * qq + j, OFF_ST16 + hf * 16384), S + 32 * qq + 8 * j);
+                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
             }
             // o rows 32 hf .. 32 hf + 31 of this chunk: column p of Qh S + Uh
             // (even lane: row r, columns p and p + 1; odd lane: row r + 1, columns p - 1 and p)
