@@ -87,12 +87,13 @@ GDR_API const char *gdr_last_error(void);
 GDR_API unsigned long long gdr_kernel_launches(void);
 
 /*
- * Device-side failure counts of the fused chunked kernel (bf16 inputs,
+ * Device-side failure counts of the tensor-core chunked kernels (bf16 inputs,
  * Dk = Dv = 128) on the current device, accumulated since the library was
  * loaded there. Either pointer may be NULL; returns the sum of the two.
- *   load_timeouts  chunk input loads that had not arrived after one second;
- *                  the (batch row, value head) unit stops, so that call's o and
- *                  hT are incomplete.
+ *   load_timeouts  waits inside the kernel (chunk input loads, or a hand-off
+ *                  between its warp groups) that gave up after one second; the
+ *                  (batch row, value head) unit stops, so that call's o and hT
+ *                  are incomplete.
  *   range_errors   chunks whose per-key-channel gate factors left the fp16
  *                  range (a decay stronger than about exp(-11) within 32
  *                  tokens); that chunk's results are not valid.
@@ -121,10 +122,14 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  * U' = U - W S, S <- diag(Gamma_C) S + (K*Gamma_C/Gamma)^T U', and the output
  * O = (Q*Gamma) S + tril((Q*Gamma)(K/Gamma)^T) U'.
  *
- * bf16 inputs with Dk = Dv = 128 run one fused kernel on the warp-level
- * tensor cores (fp16 operands, fp32 accumulation, fp32 carried state; q, k,
- * v and the state must stay inside the fp16 range, |x| < 6.5e4). Other
- * shapes and fp32 inputs run fp32 CUDA-core kernels.
+ * bf16 inputs with Dk = Dv = 128 run one tensor-core kernel: for the scalar
+ * gate on tcgen05 (where the chunk's state map is used in the equivalent
+ * affine form S <- Gamma_C S + P S + R, O = Qh S + Uh, with P = -(K*Gamma_C/
+ * Gamma)^T W, R = (K*Gamma_C/Gamma)^T U, Qh = (Q*Gamma) - M W, Uh = M U and M
+ * the masked (Q*Gamma)(K/Gamma)^T above), for the per-channel gate on the
+ * warp-level tensor cores. Both use fp16 operands, fp32 accumulation and an
+ * fp32 carried state; q, k, v and the state must stay inside the fp16 range,
+ * |x| < 6.5e4. Other shapes and fp32 inputs run fp32 CUDA-core kernels.
  * B == 0 or T == 0 is a valid no-op that still writes hT = h0 (or zeros).
  *
  * workspace: device buffer of at least gdr_fwd_workspace_size(...) bytes,
