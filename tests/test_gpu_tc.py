@@ -1,0 +1,99 @@
+"""Edge cases of the scalar-gate tensor-core path (bf16 inputs, Dk = Dv = 128) against the
+fp64 oracle, through the C ABI (needs a B200).
+
+This path keeps the state map of each 64-token chunk in affine form and hands each
+chunk from one warp group to another, so the cases here aim at chunk boundaries,
+partial chunks, grouped value heads, more CTAs than one wave of SMs, in-place states,
+decays strong enough to underflow the in-chunk gate products, and the two output dtypes.
+Tolerances as in test_gpu_parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_68_b200 as gdr
+import oracle
+from gated_delta_rule_68_b200.workloads import WORKLOADS, make_inputs
+from tests.gpu_util import TOL, oracle_units, rel_err, rel_err_excess, sample_units
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def run_fwd(inp, **kw):
+    return gdr.gdr_fwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], **kw)
+
+
+def check_all(w, out_dtype=None):
+    inp = make_inputs(w, DEV)
+    o, hT = run_fwd(inp, **({} if out_dtype is None else {"out_dtype": out_dtype}))
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
+    eo = rel_err(o, o_ref) if out_dtype == torch.float32 else rel_err_excess(o, o_ref, "bf16")
+    es = rel_err(hT, s_ref)
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"], (w, eo, es)
+    return inp, o, hT
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 191])
+def test_chunk_boundaries_grouped_heads(T):
+    check_all(WORKLOADS["gva_gdn_bf16"].with_(B=2, T=T, Hk=2, Hv=6, seed=100 + T))
+
+
+@pytest.mark.parametrize("Hk,Hv", [(1, 4), (4, 4), (2, 8)])
+def test_head_groupings(Hk, Hv):
+    check_all(WORKLOADS["gdn_bf16"].with_(B=2, T=150, Hk=Hk, Hv=Hv, seed=200 + Hk * 10 + Hv))
+
+
+def test_fp32_output_and_bf16_output_agree():
+    """The bf16-o launch is round-to-nearest bf16 of the fp32-o launch, bit for bit (both
+    run the same arithmetic and round only at the store)."""
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=200, Hk=2, Hv=4, seed=300)
+    inp, o32, h32 = check_all(w, out_dtype=torch.float32)
+    o16, h16 = run_fwd(inp)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(h16, h32)
+
+
+def test_more_ctas_than_two_waves_of_sms():
+    """B * Hv = 320 units, one CTA each: more than two waves of 148 SMs."""
+    w = WORKLOADS["gdn_bf16"].with_(B=20, T=130, Hk=4, Hv=16, seed=400)
+    inp = make_inputs(w, DEV)
+    o, hT = run_fwd(inp, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    units = sample_units(w.B, w.Hv, 8, seed=1)
+    o_ref, s_ref = oracle_units(inp, units)
+    for n, (b, h) in enumerate(units):
+        assert rel_err(o[b, :, h], o_ref[n]) <= TOL["bf16"], (b, h)
+        assert rel_err(hT[b, h], s_ref[n]) <= TOL["bf16"], (b, h)
+
+
+def test_in_place_state():
+    """hT may alias h0: the state is read at the start and written at the end."""
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=100, Hk=2, Hv=2, seed=500)
+    inp = make_inputs(w, DEV)
+    o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
+    state = inp["h0"].clone()
+    o, hT = gdr.gdr_fwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], state, hT=state,
+                                out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert hT.data_ptr() == state.data_ptr()
+    assert rel_err(o, o_ref) <= TOL["bf16"] and rel_err(state, s_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("g_mu", [-1.0, 8.0])
+def test_strong_and_weak_decay(g_mu):
+    """g = logsigmoid(N(mu, 1)): mu = -1 decays by about e^-80 over a chunk, so the
+    in-chunk Gamma underflows; mu = 8 keeps the state nearly undamped over the sequence."""
+    check_all(WORKLOADS["gdn_bf16"].with_(B=2, T=260, Hk=2, Hv=4, g_mu=g_mu, seed=600 + int(g_mu)),
+              out_dtype=torch.float32)
+
+
+def test_repeated_calls_are_bitwise_identical():
+    w = WORKLOADS["gdn_bf16"].with_(B=3, T=333, Hk=2, Hv=6, seed=700)
+    inp = make_inputs(w, DEV)
+    o1, h1 = run_fwd(inp)
+    o2, h2 = run_fwd(inp)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
