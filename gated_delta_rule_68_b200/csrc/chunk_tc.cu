@@ -136,6 +136,8 @@ __device__ __forceinline__ void st_h1(uint8_t *sm, uint32_t off, float x)
     *reinterpret_cast<__half *>(sm + off) = __float2half_rn(x);
 }
 
+__device__ __forceinline__ void out_store1(float *p, float x) { *p = x; }
+__device__ __forceinline__ void out_store1(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void out_store2(float *p, float x, float y) { *reinterpret_cast<float2 *>(p) = make_float2(x, y); }
 __device__ __forceinline__ void out_store2(__nv_bfloat16 *p, float x, float y)
 {
@@ -207,7 +209,7 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
 template <typename TOut>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-              const __grid_constant__ CUtensorMap map_v)
+              const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // Offset into the __shared__ array (not an integer round trip), so that accesses
@@ -687,25 +689,54 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
             }
-            // o rows 32 hf .. 32 hf + 31 of this chunk: column p of Qh S + Uh
-            // (even lane: row r, columns p and p + 1; odd lane: row r + 1, columns p - 1 and p)
+            // o rows 32 hf .. 32 hf + 31 of this chunk (column p of Qh S + Uh) into the o tile
+            // (the P tile, dead until the next chunk) in the TMA 128-byte swizzle, then out by
+            // TMA stores, which clip tokens past T. The partial last chunk of a packed
+            // sequence is stored with plain stores instead, so it never touches the next
+            // sequence's rows (even lane: row r, columns p and p + 1; odd lane: row r + 1,
+            // columns p - 1 and p).
+            const int nvalid = min(C, T - c * C);
+            const bool tile = !(a.cu_seqlens && nvalid < C);
             {
                 float o[32];
                 tmem_ld32(tmem_addr(tb, q4, TM_O + 32 * hf), o);
                 tc_fence_before();
                 mbar_arrive(bar(B_SE));
                 mbar_arrive(bar(B_OE));
-                const int nvalid = min(C, T - c * C) - 32 * hf, odd = p & 1;
-                const size_t rs = (size_t)a.Hv * D;
-                TOut *orow = reinterpret_cast<TOut *>(a.o) + ((size_t)tok0 * a.Hv + h) * D + p + (size_t)(c * C + 32 * hf + odd) * rs - odd;
+                if (tile) {
+                    constexpr int EPB = 128 / sizeof(TOut);
+                    const uint32_t byte = (uint32_t)(p % EPB) * sizeof(TOut);
+                    uint8_t *base = sm + OFF_P16 + (p / EPB) * C * 128 + (32 * hf) * 128 + (byte & 15);
+                    uint32_t xo[8];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float other = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + 1], 1);
-                    if (i + odd < nvalid) out_store2(orow + (size_t)i * rs, odd ? other : o[i], odd ? o[i + 1] : other);
+                    for (int s8 = 0; s8 < 8; ++s8) xo[s8] = ((byte >> 4) ^ s8) << 4;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) out_store1(reinterpret_cast<TOut *>(base + i * 128 + xo[i & 7]), o[i]);
+                    fence_proxy_async();
+                } else {
+                    const int nv = nvalid - 32 * hf, odd = p & 1;
+                    const size_t rs = (size_t)a.Hv * D;
+                    TOut *orow = reinterpret_cast<TOut *>(a.o) + ((size_t)tok0 * a.Hv + h) * D + p +
+                                 (size_t)(c * C + 32 * hf + odd) * rs - odd;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + 1], 1);
+                        if (i + odd < nv) out_store2(orow + (size_t)i * rs, odd ? other : o[i], odd ? o[i + 1] : other);
+                    }
                 }
             }
+            named_bar_sync(2, GT);
+            if (issuer && tile) {
+                constexpr int EPB = 128 / sizeof(TOut);
+#pragma unroll
+                for (int k = 0; k < D / EPB; ++k)
+                    tma_store_4d(&map_o, k * EPB, h, tt0 + c * C, tbb, sb0 + OFF_P16 + k * C * 128);
+            }
             if (c + 2 < NC) ready_chunk(c + 2, gbn);
+            if (issuer) tma_store_wait_read();   // the o tile is read before the next P tile is written
+            named_bar_sync(2, GT);
         }
+        if (issuer) tma_store_wait_all();
         if (a.hT) {
             float *hp = a.hT + (size_t)bh * D * D + (size_t)(64 * hf) * D + p;
 #pragma unroll
@@ -727,14 +758,15 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 template <typename TOut>
 cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
 {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
     if (!make_map(&mq, a.q, mb, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, mb, a.T, a.Hk, 64, false, true) ||
-        !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true))
+        !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true) ||
+        !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
-    tc_fwd_kernel<TOut><<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv);
+    tc_fwd_kernel<TOut><<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv, mo);
     return cudaGetLastError();
 }
 
