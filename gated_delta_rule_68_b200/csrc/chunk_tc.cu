@@ -81,7 +81,8 @@ static_assert(INV_END <= OFF_U16 + 16384, "inverse scratch must fit beside T' an
 // beta Gamma, row and column factors of exp(G_r - G_i), Gamma_C.
 constexpr int V_G = 0, V_GAM = 64, V_F = 128, V_BETA = 192, V_BG = 256, V_EROW = 320, V_ECOL = 384,
               V_GC = 640, V_SET = 644, V_N = 2 * V_SET;
-constexpr uint32_t SMEM_USED = OFF_VEC + V_N * 4;
+constexpr uint32_t OFF_NW = OFF_VEC + V_N * 4;    // gated output norm: [128] weight
+constexpr uint32_t SMEM_USED = OFF_NW + 128 * 4;
 constexpr uint32_t SMEM_TC = SMEM_USED + 1024;
 static_assert(SMEM_TC <= 227 * 1024, "shared memory");
 
@@ -137,6 +138,15 @@ __device__ __forceinline__ void st_h1(uint8_t *sm, uint32_t off, float x)
 }
 
 __device__ __forceinline__ void out_store1(float *p, float x) { *p = x; }
+__device__ __forceinline__ uint32_t pack_bf2(float x, float y)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ void prefetch_l1(const void *p)
+{
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void out_store1(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void out_store2(float *p, float x, float y) { *reinterpret_cast<float2 *>(p) = make_float2(x, y); }
 __device__ __forceinline__ void out_store2(__nv_bfloat16 *p, float x, float y)
@@ -206,7 +216,10 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
     }
 }
 
-template <typename TOut>
+// NORM: the layer's options (compiled as a separate instance, so the plain forward runs
+// exactly its own code): q and k rows divided by sqrt(sum of squares + 1e-6) as they are
+// converted, and o rows replaced by o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
+template <typename TOut, bool NORM>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
@@ -240,6 +253,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     const int NC = (T + C - 1) / C;
 
     if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), 512);
+    if (NORM && a.z && tid < D) reinterpret_cast<float *>(sm + OFF_NW)[tid] = a.norm_w[tid];
     if (tid == 0) {
         const uint32_t counts[NBAR] = {1, 1, 1, 1, GT, GT, 1, 1, 1, 1, GT, GT, GT, GT, 1, 1};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
@@ -557,13 +571,37 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             float *vs = vec + sb * V_SET;
             wait(B_LD0 + sb, (c >> 1) & 1);
             const int nvalid = min(C, T - c * C);
+            if (NORM && a.qk_l2norm) {
+                // [K; Q] rows: chunks e and e + 1024 are the two halves of one row, and a row's 8
+                // chunks of a half sit in 8 adjacent threads
 #pragma unroll
-            for (int j = 0; j < 3072 / GT; ++j) {
-                // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64 rows)
-                const int e = tid + GT * j;
-                const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
-                uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
-                *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                for (int j = 0; j < 4; ++j) {
+                    const int e = tid + GT * j, row = (e >> 3) & 63;
+                    uint4 *p0 = reinterpret_cast<uint4 *>(stgp) + e, *p1 = p0 + 1024;
+                    const uint4 u0 = *p0, u1 = *p1;
+                    float ss = bf16x8_sumsq(u0) + bf16x8_sumsq(u1);
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+                    const float sc = rsqrtf(ss + 1e-6f);
+                    *p0 = row < nvalid ? bf16x8_scaled_f16x8(u0, sc) : make_uint4(0, 0, 0, 0);
+                    *p1 = row < nvalid ? bf16x8_scaled_f16x8(u1, sc) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int j = 8; j < 3072 / GT; ++j) {
+                    const int e = tid + GT * j, row = ((e - 2048) >> 3) & 63;
+                    uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
+                    *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 3072 / GT; ++j) {
+                    // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64 rows)
+                    const int e = tid + GT * j;
+                    const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
+                    uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
+                    *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                }
             }
             // Gate vectors: every warp scans G (lane l: rows l, l + 32), then writes its share.
             if (warp < 6) {
@@ -638,6 +676,12 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             ready_chunk(1, gbn);
         }
         for (int c = 0; c < NC; ++c) {
+            if (NORM && a.z) {   // this chunk's z row segment (pass B's) into L1
+                const int r = 8 * warp + (lane & 7), k = lane >> 3;
+                if (c * C + r < T)
+                    prefetch_l1(reinterpret_cast<const __nv_bfloat16 *>(a.z) +
+                                ((size_t)(tok0 + c * C + r) * a.Hv + h) * D + 32 * k);
+            }
             // P and Qh of this chunk, out of tensor memory into the operand tiles
             wait(B_P1, c & 1);
             tc_fence_after();
@@ -697,7 +741,79 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             // columns p - 1 and p).
             const int nvalid = min(C, T - c * C);
             const bool tile = !(a.cu_seqlens && nvalid < C);
-            {
+            if (NORM && a.z) {
+                // Pass A: fp32 o into the P tile (dead until the next chunk), in the TMA swizzle of
+                // an fp32 o tile. Pass B, a row per 4 threads (row r = 8 warp + lane % 8, columns
+                // 32 k .. 32 k + 31, k = lane / 8): the row's mean square, then
+                // o / sqrt(mean + eps) * weight * SiLU(z) into the o tile (bf16: the Qh tile;
+                // fp32: in place), or, for a packed sequence's partial last chunk, to global memory.
+                {
+                    float o[32];
+                    tmem_ld32(tmem_addr(tb, q4, TM_O + 32 * hf), o);
+                    tc_fence_before();
+                    mbar_arrive(bar(B_SE));
+                    mbar_arrive(bar(B_OE));
+                    const uint32_t byte = (uint32_t)(p & 31) * 4u;
+                    uint8_t *base = sm + OFF_P16 + (p >> 5) * C * 128 + (32 * hf) * 128 + (byte & 15);
+                    uint32_t xo[8];
+#pragma unroll
+                    for (int s8 = 0; s8 < 8; ++s8) xo[s8] = ((byte >> 4) ^ s8) << 4;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) *reinterpret_cast<float *>(base + i * 128 + xo[i & 7]) = o[i];
+                }
+                named_bar_sync(2, GT);
+                const int r = 8 * warp + (lane & 7), k = lane >> 3;
+                float x[32];
+                const uint8_t *rowp = sm + OFF_P16 + k * C * 128 + r * 128;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(rowp + ((jj ^ (r & 7)) << 4));
+                    x[4 * jj] = v4.x, x[4 * jj + 1] = v4.y, x[4 * jj + 2] = v4.z, x[4 * jj + 3] = v4.w;
+                }
+                float ss = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ss = fmaf(x[i], x[i], ss);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+                const float rsd = rsqrtf(ss * (1.f / D) + a.norm_eps);
+                const bool rv = r < nvalid;
+                const __nv_bfloat16 *zrow =
+                    reinterpret_cast<const __nv_bfloat16 *>(a.z) + ((size_t)(tok0 + c * C + r) * a.Hv + h) * D + 32 * k;
+                const float *nw = reinterpret_cast<const float *>(sm + OFF_NW) + 32 * k;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const uint4 zz = rv ? *reinterpret_cast<const uint4 *>(zrow + 8 * q8) : make_uint4(0, 0, 0, 0);
+                    const __nv_bfloat162 *z2 = reinterpret_cast<const __nv_bfloat162 *>(&zz);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 zf = __bfloat1622float2(z2[e]);
+                        const int i = 8 * q8 + 2 * e;
+                        x[i] *= rsd * nw[i] * __fdividef(zf.x, 1.f + __expf(-zf.x));
+                        x[i + 1] *= rsd * nw[i + 1] * __fdividef(zf.y, 1.f + __expf(-zf.y));
+                    }
+                }
+                if (tile) {
+                    if (sizeof(TOut) == 4) {
+                        uint8_t *wp = sm + OFF_P16 + k * C * 128 + r * 128;
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj)
+                            *reinterpret_cast<float4 *>(wp + ((jj ^ (r & 7)) << 4)) =
+                                make_float4(x[4 * jj], x[4 * jj + 1], x[4 * jj + 2], x[4 * jj + 3]);
+                    } else {
+                        uint8_t *wp = sm + OFF_QH16 + (k >> 1) * C * 128 + r * 128;
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            *reinterpret_cast<uint4 *>(wp + (((4 * (k & 1) + jj) ^ (r & 7)) << 4)) = make_uint4(
+                                pack_bf2(x[8 * jj], x[8 * jj + 1]), pack_bf2(x[8 * jj + 2], x[8 * jj + 3]),
+                                pack_bf2(x[8 * jj + 4], x[8 * jj + 5]), pack_bf2(x[8 * jj + 6], x[8 * jj + 7]));
+                    }
+                    fence_proxy_async();
+                } else if (rv) {
+                    TOut *orow = reinterpret_cast<TOut *>(a.o) + ((size_t)(tok0 + c * C + r) * a.Hv + h) * D + 32 * k;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) out_store2(orow + i, x[i], x[i + 1]);
+                }
+            } else {
                 float o[32];
                 tmem_ld32(tmem_addr(tb, q4, TM_O + 32 * hf), o);
                 tc_fence_before();
@@ -728,9 +844,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             named_bar_sync(2, GT);
             if (issuer && tile) {
                 constexpr int EPB = 128 / sizeof(TOut);
+                // the normalised bf16 o tile is in the Qh tile
+                const uint32_t src = (NORM && a.z && sizeof(TOut) == 2) ? OFF_QH16 : OFF_P16;
 #pragma unroll
                 for (int k = 0; k < D / EPB; ++k)
-                    tma_store_4d(&map_o, k * EPB, h, tt0 + c * C, tbb, sb0 + OFF_P16 + k * C * 128);
+                    tma_store_4d(&map_o, k * EPB, h, tt0 + c * C, tbb, sb0 + src + k * C * 128);
             }
             if (c + 2 < NC) ready_chunk(c + 2, gbn);
             if (issuer) tma_store_wait_read();   // the o tile is read before the next P tile is written
@@ -764,9 +882,12 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
         !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true) ||
         !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
+    // The layer's options are compiled into a separate instance, so a call without them runs
+    // the same code as before they existed.
+    auto kernel = (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true> : tc_fwd_kernel<TOut, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
-    tc_fwd_kernel<TOut><<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv, mo);
+    kernel<<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv, mo);
     return cudaGetLastError();
 }
 
@@ -774,7 +895,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
 
 bool tc_supported(const FwdArgs &a)
 {
-    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && a.gate_mode == 0 && !a.qk_l2norm && !a.z;
+    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && a.gate_mode == 0;
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st)
