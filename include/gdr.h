@@ -158,9 +158,10 @@ GDR_API int gdr_fwd_chunked(const void *q, const void *k, const void *v, const f
  * out-of-bounds access). Each sequence equals a gdr_fwd_chunked call on it
  * alone, bit for bit.
  *
- * Runs only on the fused kernel: bf16 inputs (dtype GDR_BF16 or
+ * Runs only on the tensor-core kernels: bf16 inputs (dtype GDR_BF16 or
  * GDR_BF16_OUT_F32) with Dk = Dv = 128; anything else returns
- * GDR_ERR_UNSUPPORTED. Needs no workspace. Pointers 16-byte aligned (cu_seqlens
+ * GDR_ERR_UNSUPPORTED. The scalar gate runs the same kernel as
+ * gdr_fwd_chunked, so each packed sequence equals a separate call bit for bit. Needs no workspace. Pointers 16-byte aligned (cu_seqlens
  * 4-byte aligned); o must not alias q, k or v.
  */
 GDR_API int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, const float *g,
@@ -183,9 +184,10 @@ GDR_API int gdr_fwd_chunked_varlen(const void *q, const void *k, const void *v, 
  *   receives o / sqrt(mean(o^2) + norm_eps) * norm_weight * SiLU(z) per row of
  *   Dv, where o is the recurrence's output; norm_weight [Dv] fp32 is required.
  *
- * Runs only on the fused kernel: bf16 inputs (GDR_BF16 or GDR_BF16_OUT_F32)
- * with Dk = Dv = 128, else GDR_ERR_UNSUPPORTED. No workspace. A call with z
- * keeps each (b, h) in one CTA. Pointers 16-byte aligned (norm_weight 4-byte,
+ * Runs only on the tensor-core kernels: bf16 inputs (GDR_BF16 or
+ * GDR_BF16_OUT_F32) with Dk = Dv = 128, else GDR_ERR_UNSUPPORTED. No workspace.
+ * Without options it equals gdr_fwd_chunked bit for bit. A call with z keeps
+ * each (b, h) in one CTA. Pointers 16-byte aligned (norm_weight 4-byte,
  * cu_seqlens 4-byte); o must not alias q, k, v or z.
  */
 GDR_API int gdr_fwd_chunked_norm(const void *q, const void *k, const void *v, const float *g,
