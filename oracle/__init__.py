@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package. The CUDA library
 (``gated_delta_rule_68_b200``) never imports it and shares no code with it.
 
-Two functions:
+Functions:
 
 ``recurrent``  the plain definition: the token-by-token recurrence in fp64
                (C, ``gdr_oracle.c``), following NextTransformer "Source notes",
@@ -14,6 +14,8 @@ Two functions:
                (``chunked.py``), the algebra the CUDA kernels implement, pinned
                against ``recurrent`` as the SinkProbe README describes for its
                delta-rule layer (chunk sizes 1, 8, 16, 64; agreement 1e-10).
+``backward``   the gradients of the recurrence: the adjoint of each step of the
+               token loop, in reverse order, in fp64 (C, ``gdr_oracle.c``).
 
 Pins (tests/test_oracle_pins.py) tie ``recurrent`` to closed forms, brute
 force and invariants that do not use this code. The GQA/GVA head-mapping
@@ -41,6 +43,8 @@ def _load():
         lib.gdr_oracle_recurrent.restype = ctypes.c_int
         lib.gdr_oracle_threads.argtypes = [ctypes.c_int, ctypes.c_long]
         lib.gdr_oracle_threads.restype = ctypes.c_int
+        lib.gdr_oracle_backward.argtypes = [dp] * 14 + [ctypes.c_int] * 8
+        lib.gdr_oracle_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -107,3 +111,26 @@ def decode_steps(q, k, v, g, beta, h0, nthreads=0):
                          beta[s][:, None], S, nthreads=nthreads)
         outs.append(o[:, 0])
     return np.stack(outs, 0), S
+
+
+def backward(q, k, v, g, beta, h0, do, dhT=None, gate_mode=None, nthreads=0):
+    """Gradients of L = sum(do * o) + sum(dhT * hT) through the token recurrence, fp64.
+
+    Shapes as in ``recurrent``; do [B,T,Hv,Dv]; dhT [B,Hv,Dk,Dv] or None (zero).
+    Returns a dict with dq, dk [B,T,Hk,Dk], dv [B,T,Hv,Dv], dg (g's shape),
+    dbeta [B,T,Hv] and dh0 [B,Hv,Dk,Dv] as fp64 numpy arrays.
+    """
+    q, k, v, g, beta, h0, do, dhT = (_f64(x) for x in (q, k, v, g, beta, h0, do, dhT))
+    B, T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    if gate_mode is None:
+        gate_mode = 1 if g.ndim == 4 else 0
+    assert do.shape == v.shape and beta.shape == (B, T, Hv)
+    out = {"dq": np.zeros(q.shape), "dk": np.zeros(k.shape), "dv": np.zeros(v.shape),
+           "dg": np.zeros(g.shape), "dbeta": np.zeros(beta.shape), "dh0": np.zeros((B, Hv, Dk, Dv))}
+    rc = _load().gdr_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(do),
+                                     _ptr(dhT), *(_ptr(out[n]) for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0")),
+                                     B, T, Hk, Hv, Dk, Dv, gate_mode, int(nthreads))
+    if rc != 0:
+        raise ValueError("gdr_oracle_backward rejected its arguments")
+    return out
