@@ -74,6 +74,10 @@ def lib():
         L.gdr_fwd_chunked_norm.argtypes = ([vp, vp, vp, fp, fp, fp, vp, fp, vp] + [i] * 9 + [vp, fp, ctypes.c_float, vp])
         L.gdr_rmsnorm_gated.restype = i
         L.gdr_rmsnorm_gated.argtypes = [vp, vp, fp, vp, ctypes.c_long, i, ctypes.c_float, i, vp]
+        L.gdr_bwd_workspace_size.restype = sz
+        L.gdr_bwd_workspace_size.argtypes = [i] * 8
+        L.gdr_bwd.restype = i
+        L.gdr_bwd.argtypes = [vp] * 14 + [i] * 8 + [vp, sz, vp]
         _lib = L
     return _lib
 
@@ -136,6 +140,40 @@ def _need(t, name, dtype=None, shape=None):
 
 def gdr_fwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
     return int(lib().gdr_fwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype))
+
+
+def gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
+    return int(lib().gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype))
+
+
+def gdr_bwd(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None):
+    """Backward of the recurrence: fp32 gradients of sum(dout * o) + sum(dhT * hT) with respect
+    to q, k, v, g, beta and h0, as a dict (dq, dk, dv, dg, dbeta, dh0). dout has q's dtype."""
+    B, T, Hk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    dt, _ = _dtype_code(q, None)
+    gate_mode = GDR_GATE_CHANNEL if g.dim() == 4 else GDR_GATE_SCALAR
+    _need(q, "q", q.dtype)
+    _need(k, "k", q.dtype, q.shape)
+    _need(v, "v", q.dtype, (B, T, Hv, Dv))
+    _need(dout, "dout", q.dtype, (B, T, Hv, Dv))
+    _need(g, "g", torch.float32, (B, T, Hv) if gate_mode == 0 else (B, T, Hv, Dk))
+    _need(beta, "beta", torch.float32, (B, T, Hv))
+    for t, n in ((h0, "h0"), (dhT, "dhT")):
+        if t is not None:
+            _need(t, n, torch.float32, (B, Hv, Dk, Dv))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = {"dq": torch.empty((B, T, Hk, Dk), **f32), "dk": torch.empty((B, T, Hk, Dk), **f32),
+           "dv": torch.empty((B, T, Hv, Dv), **f32), "dg": torch.empty(tuple(g.shape), **f32),
+           "dbeta": torch.empty((B, T, Hv), **f32), "dh0": torch.empty((B, Hv, Dk, Dv), **f32)}
+    need = gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dt)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().gdr_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(dout), _ptr(dhT),
+                         *(_ptr(out[n]) for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0")),
+                         B, T, Hk, Hv, Dk, Dv, gate_mode, dt, _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
 
 
 def gdr_fwd_chunked(q, k, v, g, beta, h0=None, *, o=None, hT=None, want_hT=True,

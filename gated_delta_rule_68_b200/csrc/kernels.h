@@ -52,6 +52,21 @@ cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st);
 // Waits of the tcgen05 kernel that timed out since the library was loaded on this device.
 unsigned int tc_error_count();
 
+// Backward of the recurrence (bwd.cu): gradients of L = sum(dout * o) + sum(dhT * hT), all
+// fp32 [q, k: B,T,Hk,Dk; v: B,T,Hv,Dv; g: g's layout; beta: B,T,Hv; h0: B,Hv,Dk,Dv].
+// dq, dk, dg and dbeta are accumulated with atomics and must be zero on entry.
+struct BwdArgs {
+    const void *q, *k, *v;
+    const float *g, *beta, *h0;
+    const void *dout;
+    const float *dhT;
+    float *dq, *dk, *dv, *dg, *dbeta, *dh0;
+    int B, T, Hk, Hv, Dk, Dv, gate_mode, dtype;
+};
+bool bwd_supported(const BwdArgs &a);
+size_t bwd_workspace_size(const BwdArgs &a);
+cudaError_t launch_bwd(const BwdArgs &a, void *ws, cudaStream_t st);
+
 // fp32 CUDA-core chunked forward (three kernels). Needs simt_workspace_size() bytes.
 size_t simt_workspace_size(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a, void *ws, cudaStream_t st);

@@ -87,6 +87,37 @@ GDR_API const char *gdr_last_error(void);
 GDR_API unsigned long long gdr_kernel_launches(void);
 
 /*
+ * Backward of the recurrence (NextTransformer, "Source notes", "Linear attention":
+ * the gdn and kda updates; their adjoint, step by step in reverse).
+ *
+ * Gradients of L = sum(dout * o) + sum(dhT * hT), where (o, hT) is what
+ * gdr_fwd_chunked computes from the same q, k, v, g, beta, h0 (h0 == NULL: zero
+ * state; dhT == NULL: zero):
+ *   dq, dk  [B, T, Hk, Dk] fp32 (summed over the value heads sharing a key head)
+ *   dv      [B, T, Hv, Dv] fp32
+ *   dg      [B, T, Hv] or [B, T, Hv, Dk] fp32 (g's layout)
+ *   dbeta   [B, T, Hv] fp32
+ *   dh0     [B, Hv, Dk, Dv] fp32
+ * Inputs as for gdr_fwd_chunked; dout [B, T, Hv, Dv] in the input dtype (GDR_BF16
+ * or GDR_BF16_OUT_F32: bf16; GDR_FP32: fp32), dhT fp32. The arithmetic is fp32:
+ * a forward pass stores the state before every 8th token in the workspace, then a
+ * reverse pass recomputes each block of 8 tokens and reverses its steps.
+ * Needs Dk of 64 or 128 and Dv of 64 or 128 (else GDR_ERR_UNSUPPORTED); the other
+ * argument errors are those of gdr_fwd_chunked. All pointers 16-byte aligned;
+ * the outputs must not alias the inputs or each other. T == 0 writes dh0 = dhT
+ * (or zeros) and nothing else.
+ *
+ * workspace: device buffer of at least gdr_bwd_workspace_size(...) bytes
+ * (B * Hv * ceil(T / 8) * Dk * Dv * 4), owned by the caller; two calls that
+ * overlap in time must not share one. Asynchronous on `stream`.
+ */
+GDR_API size_t gdr_bwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype);
+GDR_API int gdr_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    const float *h0, const void *dout, const float *dhT, float *dq, float *dk, float *dv,
+                    float *dg, float *dbeta, float *dh0, int B, int T, int Hk, int Hv, int Dk, int Dv,
+                    int gate_mode, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Device-side failure counts of the tensor-core chunked kernels (bf16 inputs,
  * Dk = Dv = 128) on the current device, accumulated since the library was
  * loaded there. Either pointer may be NULL; returns the sum of the two.
