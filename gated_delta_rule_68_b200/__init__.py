@@ -27,7 +27,7 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
            "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts",
            "gdr_fwd_chunked_varlen", "gdr_causal_conv_silu", "gdr_rmsnorm_gated",
-           "gdr_fwd_chunked_norm")
+           "gdr_fwd_chunked_norm", "gdr_bwd_workspace_size", "gdr_bwd")
 
 # Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
 GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
