@@ -47,6 +47,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="gdn_bf16")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--T", type=int, default=None,
+                   help="override the workload's sequence length (small cases for profiling)")
     a = p.parse_args(argv)
     a.warmup = max(a.warmup, 3)
     return a
@@ -88,14 +90,25 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha():
+# The sources each captured kernel is built from: a recorded DRAM figure stands only while
+# these files are unchanged.
+KERNEL_SOURCES = {
+    "tc_fwd_kernel": ("chunk_tc.cu", "tc_util.cuh", "common.cuh", "kernels.h"),
+    "fused_fwd_kernel": ("chunk_mma.cu", "common.cuh", "kernels.h"),
+    "bwd_kernel": ("bwd.cu", "common.cuh", "kernels.h"),
+}
+
+
+def kernel_sources_sha(kernel=None):
     csrc = os.path.join(ROOT, "gated_delta_rule_68_b200", "csrc")
+    names = sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh", ".h")))
+    if kernel is not None:
+        names = sorted(KERNEL_SOURCES[kernel.split("<")[0]])
     h = hashlib.sha256()
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh", ".h")):
-            h.update(n.encode())
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(f.read())
+    for n in names:
+        h.update(n.encode())
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 
@@ -107,7 +120,7 @@ def recorded_traffic(workload):
             d = json.load(f)[workload]
     except Exception:
         return None, None
-    if d.get("kernel_sources_sha256") != kernel_sources_sha():
+    if d.get("kernel_sources_sha256") != kernel_sources_sha(d.get("kernel")):
         return None, d.get("kernel")
     return float(d["dram_bytes_per_launch"]), d.get("kernel")
 
@@ -379,6 +392,8 @@ def run_reference(args, w, rank, world):
 
     if w.layer:
         return run_layer_reference(args, w, world)
+    if w.bwd:
+        return run_bwd_reference(args, w, world)
     cores = oracle.threads_used(0, 1 << 30)
     units = max(cores, 8)
     sample = w.with_(B=units, Hk=1, Hv=1)
@@ -439,8 +454,203 @@ def run_layer_reference(args, w, world):
     return 0
 
 
+# ----------------------------------------------------------------------------- backward
+BWD_METRIC = "gated-delta bwd tokens/s (B·T·Hv per sec) bf16 d=128; % of roofline"
+
+
+def bwd_bytes(w):
+    """HBM bytes the backward must move per call: q, k, v, do, g, beta, h0 and dhT read once;
+    dq, dk, dv, dg, dbeta and dh0 (fp32) written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    gw = w.Dk if w.gate == "channel" else 1
+    ins = 2 * w.B * w.T * w.Hk * w.Dk * es + 2 * w.B * w.T * w.Hv * w.Dv * es + w.B * w.T * w.Hv * (gw + 1) * 4
+    outs = 2 * w.B * w.T * w.Hk * w.Dk * 4 + w.B * w.T * w.Hv * (w.Dv + gw + 1) * 4
+    states = 3 * w.B * w.Hv * w.Dk * w.Dv * 4
+    return ins + outs + states
+
+
+def bwd_flops(w):
+    """fp32 flops per call of the token-level backward: per (batch row, value head, token) and
+    state element, 5 to rebuild the decayed state and the delta step (decay, k-projection,
+    rank-one update) and 15 for the adjoint (the q do^T and k dp^T rank-one terms, the
+    k-projection of dS, dq, the two dk terms, the gate's row sums and the decay of dS)."""
+    return 20 * w.B * w.T * w.Hv * w.Dk * w.Dv
+
+
+def alu_peak_tflops(sm_mhz):
+    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops per clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def bwd_cpu_sample(w, target_s=12.0):
+    """Time the fp64 oracle backward on whole (b, h) sequences of the workload (Hk = Hv = 1 units)."""
+    import oracle
+    from gated_delta_rule_68_b200.workloads import make_inputs, make_upstream
+    cores = oracle.threads_used(0, 1 << 30)
+    one = w.with_(B=1, Hk=1, Hv=1)
+    inp, up = make_inputs(one, "cpu"), make_upstream(one, "cpu")
+    t0 = time.perf_counter()
+    oracle.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], up["do"], up["dhT"],
+                    nthreads=1)
+    t_unit = time.perf_counter() - t0
+    units = max(1, min(w.B * w.Hv, int(target_s * cores / max(t_unit, 1e-6))))
+    sample = w.with_(B=units, Hk=1, Hv=1)
+    inp, up = make_inputs(sample, "cpu"), make_upstream(sample, "cpu")
+    t0 = time.perf_counter()
+    oracle.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], up["do"], up["dhT"],
+                    nthreads=0)
+    dt = time.perf_counter() - t0
+    return {"value": units * w.T / dt, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+            "kind": "oracle",
+            "sample": f"{units} whole (batch row, value head) sequences of T={w.T}, Dk=Dv={w.Dk}: fp64 token "
+                      f"recurrence forward and its adjoint; {dt:.1f} s", "seconds": dt}
+
+
+def run_bwd_bench(args, w, wr, rank, world, local, dev):
+    """One step = one gdr_bwd call over the whole workload: the checkpointing forward pass and
+    the reverse sweep, every gradient written."""
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_68_b200 as gdr
+    from gated_delta_rule_68_b200.workloads import make_inputs, make_upstream
+
+    inp_cpu = make_inputs(wr, "cpu")
+    inp_cpu.update(make_upstream(wr, "cpu"))
+    inp = {n: (None if t is None else t.to(dev)) for n, t in inp_cpu.items()}
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dq": torch.empty(inp["q"].shape, **f32), "dk": torch.empty(inp["k"].shape, **f32),
+           "dv": torch.empty(inp["v"].shape, **f32), "dg": torch.empty(inp["g"].shape, **f32),
+           "dbeta": torch.empty(inp["beta"].shape, **f32), "dh0": torch.empty((w.B, w.Hv, w.Dk, w.Dv), **f32)}
+    need = gdr.gdr_bwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, w.gate_mode,
+                                      gdr.GDR_BF16 if w.dtype == "bf16" else gdr.GDR_FP32)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x):
+        gdr.gdr_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], x["do"], x["dhT"], workspace=ws,
+                    stream=stream, out=out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(inp)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = gdr.gdr_kernel_launches()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(inp)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    launches = gdr.gdr_kernel_launches() - n0
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms, dev)
+
+    e2e = None
+    if not args.no_e2e:
+        host = {n: (None if x is None else x.pin_memory()) for n, x in inp_cpu.items()}
+        dbuf = {n: (None if x is None else torch.empty_like(x, device=dev)) for n, x in inp_cpu.items()}
+        out_h = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in out.items()}
+        h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
+        d2h = sum(x.numel() * x.element_size() for x in out_h.values())
+        e2e_steps = max(3, min(args.steps, 5))
+
+        def e2e_step():
+            for n, x in host.items():
+                if x is not None:
+                    dbuf[n].copy_(x, non_blocking=True)
+            step(dbuf)
+            for n, x in out_h.items():
+                x.copy_(out[n], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+        e2e = {"value": job_tokens_per_s(w.head_tokens, world, te), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": te}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    clocks = clk.summary()
+    peak_mhz = clocks.get("sm_max_mhz") or 1965
+    peak = alu_peak_tflops(peak_mhz)
+    flops = bwd_flops(w)
+    achieved = flops / (ms / 1e3) / 1e12
+    hbm, hbm_kind = measured_peaks()
+    alg = bwd_bytes(w)
+    traffic, traffic_kernel = recorded_traffic(w.name)
+    cpu = bwd_cpu_sample(w) if world == 1 and not args.no_cpu_baseline else None
+    line = {
+        "metric": BWD_METRIC, "value": job_tokens_per_s(w.head_tokens, world, ms_max), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded CPU generator; inputs as the gdn_bf16 recipe; do N(0,1) bf16, "
+                "dhT 0.1 N(0,1) fp32)",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 x {peak_mhz} MHz",
+                     "algorithmic_flops_per_launch": flops, "traffic": traffic, "traffic_kernel": traffic_kernel,
+                     "kernel": "gdr_bwd step (bwd_ckpt_kernel + bwd_kernel)"},
+        "hbm_roofline": {"algorithmic_bytes": alg, "achieved": alg / (ms / 1e3) / 1e9, "peak": hbm,
+                         "frac": alg / (ms / 1e3) / 1e9 / hbm, "peak_source": hbm_kind},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "launches_per_step": launches / args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_bwd_reference(args, w, world):
+    """The reference arm on the backward workload: each step is the fp64 oracle backward on
+    whole (b, h) sequences, on the host cores."""
+    import oracle
+    from gated_delta_rule_68_b200.workloads import make_inputs, make_upstream
+    units = max(oracle.threads_used(0, 1 << 30), 4)
+    sample = w.with_(B=units, Hk=1, Hv=1)
+    inp, up = make_inputs(sample, "cpu"), make_upstream(sample, "cpu")
+    times = []
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], up["do"], up["dhT"],
+                        nthreads=0)
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    value = units * w.T / per_step
+    line = {
+        "impl": "reference", "metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same recipe as the GPU arm)", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+                         "kind": "oracle",
+                         "sample": f"each step: {units} whole (batch row, value head) sequences of T={w.T}, "
+                                   "fp64 forward and adjoint"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def workload_config(w, world):
-    ab = algorithmic_bytes(w)
+    ab = bwd_bytes(w) if w.bwd else algorithmic_bytes(w)
     return {"workload": w.name, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "Dk": w.Dk, "Dv": w.Dv,
             "gate": w.gate, "chunk": 64, "global_batch": w.B * world,
             "parallelism": f"dp{world} (independent batch shards, no collective)",
@@ -551,6 +761,8 @@ def main(argv=None):
 
     from gated_delta_rule_68_b200.workloads import WORKLOADS, make_inputs
     w = WORKLOADS[args.workload]
+    if args.T is not None:
+        w = w.with_(name=f"{w.name}_T{args.T}", T=args.T)
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
 
@@ -570,6 +782,8 @@ def main(argv=None):
         return run_decode_bench(args, w, wr, rank, world, local, dev)
     if w.layer:
         return run_layer_bench(args, w, wr, rank, world, local, dev)
+    if w.bwd:
+        return run_bwd_bench(args, w, wr, rank, world, local, dev)
     inp_cpu = make_inputs(wr, "cpu")
     inp = {n: (None if t is None else t.to(dev)) for n, t in inp_cpu.items()}
     o = torch.empty((w.B, w.T, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)

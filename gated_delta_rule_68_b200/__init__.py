@@ -146,9 +146,10 @@ def gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
     return int(lib().gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype))
 
 
-def gdr_bwd(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None):
+def gdr_bwd(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None, out=None):
     """Backward of the recurrence: fp32 gradients of sum(dout * o) + sum(dhT * hT) with respect
-    to q, k, v, g, beta and h0, as a dict (dq, dk, dv, dg, dbeta, dh0). dout has q's dtype."""
+    to q, k, v, g, beta and h0, as a dict (dq, dk, dv, dg, dbeta, dh0). dout has q's dtype.
+    out, if given, is such a dict of preallocated fp32 tensors to write into."""
     B, T, Hk, Dk = q.shape
     Hv, Dv = v.shape[2], v.shape[3]
     dt, _ = _dtype_code(q, None)
@@ -163,9 +164,12 @@ def gdr_bwd(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None
         if t is not None:
             _need(t, n, torch.float32, (B, Hv, Dk, Dv))
     f32 = dict(dtype=torch.float32, device=q.device)
-    out = {"dq": torch.empty((B, T, Hk, Dk), **f32), "dk": torch.empty((B, T, Hk, Dk), **f32),
-           "dv": torch.empty((B, T, Hv, Dv), **f32), "dg": torch.empty(tuple(g.shape), **f32),
-           "dbeta": torch.empty((B, T, Hv), **f32), "dh0": torch.empty((B, Hv, Dk, Dv), **f32)}
+    shapes = {"dq": (B, T, Hk, Dk), "dk": (B, T, Hk, Dk), "dv": (B, T, Hv, Dv), "dg": tuple(g.shape),
+              "dbeta": (B, T, Hv), "dh0": (B, Hv, Dk, Dv)}
+    if out is None:
+        out = {n: torch.empty(s, **f32) for n, s in shapes.items()}
+    for n, s in shapes.items():
+        _need(out[n], n, torch.float32, s)
     need = gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dt)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

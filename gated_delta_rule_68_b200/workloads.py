@@ -19,7 +19,8 @@ The shapes and distributions are the five workloads of the gated delta-rule
 study: a tiny fp32 GDN case, a nanochat-scale GDN layer, a grouped-value GDN
 layer (16 key heads shared by 48 value heads, as in the Qwen GDN blocks of the
 Frontier-model atlas, item 08), a KDA layer with a per-channel gate, and a
-batch-256 decode loop.
+batch-256 decode loop; plus the layer around the recurrence (make_layer_inputs)
+and the backward of the nanochat-scale layer (make_upstream).
 """
 from dataclasses import dataclass, replace
 
@@ -42,6 +43,7 @@ class Workload:
     seed: int
     decode: bool = False
     layer: bool = False   # inputs are the raw q/k/v projections of the layer (make_layer_inputs)
+    bwd: bool = False     # one step is the backward (gdr_bwd) with upstream gradients (make_upstream)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -74,6 +76,8 @@ WORKLOADS = {
     "gdn_layer_bf16": Workload("gdn_layer_bf16", B=8, T=2048, Hk=16, Hv=16, Dk=128, Dv=128,
                                gate="scalar", dtype="bf16", g_mu=3.0, h0_std=0.02, seed=5,
                                layer=True),
+    "gdn_bwd_bf16": Workload("gdn_bwd_bf16", B=8, T=2048, Hk=16, Hv=16, Dk=128, Dv=128,
+                             gate="scalar", dtype="bf16", g_mu=3.0, h0_std=0.02, seed=6, bwd=True),
 }
 
 
@@ -107,6 +111,15 @@ def make_inputs(w: Workload, device="cpu"):
     if device != "cpu":
         out = {n: (None if t is None else t.to(device)) for n, t in out.items()}
     return out
+
+
+def make_upstream(w: Workload, device="cpu"):
+    """Upstream gradients of a backward step, from a second generator seeded w.seed + 1000003:
+    do ~ N(0, 1) [B, T, Hv, Dv] in the workload dtype, then dhT = 0.1 N(0, 1) [B, Hv, Dk, Dv] fp32."""
+    gen = torch.Generator(device="cpu").manual_seed(w.seed + 1000003)
+    do = torch.randn((w.B, w.T, w.Hv, w.Dv), generator=gen).to(w.torch_dtype)
+    dhT = 0.1 * torch.randn((w.B, w.Hv, w.Dk, w.Dv), generator=gen)
+    return {"do": do.to(device), "dhT": dhT.to(device)}
 
 
 def make_layer_inputs(w: Workload, device="cpu"):
