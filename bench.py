@@ -93,8 +93,8 @@ def measured_peaks():
 # The sources each captured kernel is built from: a recorded DRAM figure stands only while
 # these files are unchanged.
 KERNEL_SOURCES = {
-    "tc_fwd_kernel": ("chunk_tc.cu", "tc_util.cuh", "common.cuh", "kernels.h"),
-    "fused_fwd_kernel": ("chunk_mma.cu", "common.cuh", "kernels.h"),
+    "tc_fwd_kernel": ("chunk_tc.cu", "tc_util.cuh", "mma_util.cuh", "common.cuh", "kernels.h"),
+    "fused_fwd_kernel": ("chunk_mma.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
     "bwd_kernel": ("bwd.cu", "common.cuh", "kernels.h"),
 }
 
@@ -360,6 +360,7 @@ def run_layer_bench(args, w, wr, rank, world, local, dev):
     peak, peak_kind = measured_peaks()
     alg, conv_alg = algorithmic_bytes(w), layer_conv_bytes(w)
     fwd_alg = alg - conv_alg
+    traffic, traffic_kernel = recorded_traffic(w.name)
     cpu = layer_cpu_sample(w) if world == 1 and not args.no_cpu_baseline else None
     line = {
         "metric": METRIC, "value": job_tokens_per_s(w.head_tokens, world, ms_max), "unit": "tokens/s",
@@ -370,7 +371,7 @@ def run_layer_bench(args, w, wr, rank, world, local, dev):
         "config": workload_config(w, world),
         "roofline": {"bound": "hbm", "achieved": fwd_alg / (fwd_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": fwd_alg / (fwd_ms / 1e3) / 1e9 / peak, "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": fwd_alg, "traffic": None,
+                     "algorithmic_bytes_per_launch": fwd_alg, "traffic": traffic, "traffic_kernel": traffic_kernel,
                      "kernel": "gdr_fwd_chunked_norm (q/k L2 norm and gated output norm fused)"},
         "step_roofline": {"achieved": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peak,
                           "algorithmic_bytes": alg},

@@ -1,5 +1,5 @@
-// Backward of the gated delta rule: gradients of L = sum(do * o) + sum(dhT * hT)
-// with respect to q, k, v, g, beta and h0, in fp32 on the CUDA cores.
+// Backward of the gated delta rule: gradients of L = sum(do * o) + sum(dhT * hT) with respect
+// to q, k, v, g, beta and h0, in fp32 on the CUDA cores.
 //
 // Per token t (NextTransformer, "Source notes", "Linear attention", rows gdn and
 // kda: decay before the delta update, readout after it):
@@ -11,7 +11,7 @@
 //             dS <- diag(a_t) dSb;  and dh0 = dS after the first token.
 //
 // The columns of S (value channels) evolve independently, so one CTA takes a
-// (batch row, value head, 32-column slice) and each of its Dk threads a row of
+// (batch row, value head, 16-column slice) and each of its Dk threads a row of
 // that slice. Two kernels:
 //   1. a forward pass that stores the state before every 8th token (workspace);
 //   2. a reverse pass that, per block of 8 tokens, recomputes the decayed states
@@ -19,10 +19,14 @@
 //      steps. dv and dh0 belong to one slice and are stored; dq and dk (summed
 //      over slices and over the value heads that share a key head), dbeta and dg
 //      are accumulated with atomics into zeroed outputs.
-// Column sums over the Dk rows (p and du) use a shuffle transpose-reduce per warp
-// and shared memory across warps.
+// Both kernels stage a block's inputs (k, q, the slice's v and do columns, g, beta)
+// in shared memory with asynchronous copies one block ahead, so no token waits on a
+// global load. Column sums over the Dk rows (p and du) use a shuffle transpose-reduce
+// per warp and shared memory across warps. The reverse kernel's shared memory (about
+// 92 KB for bf16 inputs and the scalar gate, 110 KB at most) lets two CTAs share an SM.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -30,19 +34,106 @@
 namespace gdr {
 namespace {
 
-constexpr int BW = 32;      // value columns per CTA
+constexpr int BW = 16;      // value columns per CTA
 constexpr int BLK = 8;      // tokens between checkpoints
-constexpr int SBLD = 36;    // fp32 row stride of a recomputed state slice (conflict-free 16-byte stores)
+constexpr int SBLD = 20;    // fp32 row stride of a recomputed state slice (conflict-free 16-byte stores)
 
-// Sum over the block's rows of x[j] for the 32 columns: a transpose-reduce inside each
-// warp (lane j ends with the warp's sum of column j), then across warps through shared
-// memory. Every thread returns with all 32 totals in tot (shared, read after the call).
+__device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void cp16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(saddr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// One block's inputs in shared memory: k and q rows of the key head, the slice's
+// columns of v and do, the gate (one value, or Dk for the per-channel gate) and beta.
+template <typename TIn, int GATE, int DK>
+struct alignas(16) Stage {
+    TIn k[BLK][DK];
+    TIn q[BLK][DK];
+    TIn v[BLK][BW];
+    TIn d[BLK][BW];
+    float g[BLK][GATE ? DK : 4];
+    float beta[BLK];
+};
+
+// Issue the asynchronous copies of tokens t0 .. t0 + n - 1 (q and do only for the reverse
+// pass) as one commit group. Every source row starts on a 16-byte boundary: the API checks
+// the base pointers, and row strides and slice offsets are multiples of 16 bytes.
+template <typename TIn, int GATE, int DK, bool REV>
+__device__ __forceinline__ void stage_issue(Stage<TIn, GATE, DK> &s, const BwdArgs &a, int b, int h, int hk,
+                                            int j0, int t0, int n)
+{
+    constexpr int E = 16 / sizeof(TIn);            // elements per 16-byte copy
+    constexpr int CR = DK / E, CV = BW / E;        // copies per k row and per v slice row
+    const int tid = threadIdx.x;
+    const TIn *k = reinterpret_cast<const TIn *>(a.k), *q = reinterpret_cast<const TIn *>(a.q);
+    const TIn *v = reinterpret_cast<const TIn *>(a.v), *d = reinterpret_cast<const TIn *>(a.dout);
+    for (int c = tid; c < n * CR; c += DK) {
+        const int tt = c / CR, x = (c % CR) * E;
+        const size_t off = (((size_t)b * a.T + t0 + tt) * a.Hk + hk) * DK + x;
+        cp16(&s.k[tt][x], k + off);
+        if (REV) cp16(&s.q[tt][x], q + off);
+    }
+    for (int c = tid; c < n * CV; c += DK) {
+        const int tt = c / CV, x = (c % CV) * E;
+        const size_t off = (((size_t)b * a.T + t0 + tt) * a.Hv + h) * a.Dv + j0 + x;
+        cp16(&s.v[tt][x], v + off);
+        if (REV) cp16(&s.d[tt][x], d + off);
+    }
+    if (GATE) {
+        for (int c = tid; c < n * (DK / 4); c += DK) {
+            const int tt = c / (DK / 4), x = (c % (DK / 4)) * 4;
+            cp16(&s.g[tt][x], a.g + (((size_t)b * a.T + t0 + tt) * a.Hv + h) * DK + x);
+        }
+    } else if (tid < n) {
+        cp4(&s.g[tid][0], a.g + ((size_t)b * a.T + t0 + tid) * a.Hv + h);
+    }
+    if (tid >= 32 && tid < 32 + n)
+        cp4(&s.beta[tid - 32], a.beta + ((size_t)b * a.T + t0 + tid - 32) * a.Hv + h);
+    cp_commit();
+}
+
+template <typename TIn>
+__device__ __forceinline__ float ld(const TIn *p) { return In<TIn>::load(p); }
+
+// The BW values of a staged slice row (broadcast reads).
+__device__ __forceinline__ void load_row(const float *p, float x[BW])
+{
+#pragma unroll
+    for (int j = 0; j < BW / 4; ++j) {
+        const float4 f = reinterpret_cast<const float4 *>(p)[j];
+        x[4 * j] = f.x, x[4 * j + 1] = f.y, x[4 * j + 2] = f.z, x[4 * j + 3] = f.w;
+    }
+}
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float x[BW])
+{
+#pragma unroll
+    for (int j = 0; j < BW / 8; ++j) {
+        const uint4 u = reinterpret_cast<const uint4 *>(p)[j];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {   // a bf16 is the high half of its fp32 value
+            x[8 * j + 2 * m] = __uint_as_float(w[m] << 16);
+            x[8 * j + 2 * m + 1] = __uint_as_float(w[m] & 0xffff0000u);
+        }
+    }
+}
+
+// Sum over the block's rows of x[j] for the BW columns: a transpose-reduce inside each
+// warp (lanes j and j + 16 end with the warp's sum of column j), then across warps
+// through shared memory. Every thread returns with all BW totals in tot (shared).
 template <int NWARP>
 __device__ __forceinline__ void column_sums(float x[BW], float *red, float *tot)
 {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
+    for (int s = BW / 2; s >= 1; s >>= 1) {
         const bool upper = (lane & s) != 0;
 #pragma unroll
         for (int i = 0; i < s; ++i) {
@@ -51,7 +142,8 @@ __device__ __forceinline__ void column_sums(float x[BW], float *red, float *tot)
             x[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
         }
     }
-    red[w * BW + lane] = x[0];
+    x[0] += __shfl_xor_sync(0xffffffffu, x[0], 16);
+    if (lane < BW) red[w * BW + lane] = x[0];
     __syncthreads();
     if (threadIdx.x < BW) {
         float s = 0.f;
@@ -62,43 +154,44 @@ __device__ __forceinline__ void column_sums(float x[BW], float *red, float *tot)
     __syncthreads();
 }
 
-template <typename TIn>
-__device__ __forceinline__ float ld(const TIn *p) { return In<TIn>::load(p); }
-
 template <typename TIn, int GATE, int DK>
 __global__ void __launch_bounds__(DK)
 bwd_ckpt_kernel(BwdArgs a, float *ck)
 {
     constexpr int NWARP = DK / 32;
-    __shared__ float red[NWARP * BW], tot[BW], vrows[2 * BW];   // v rows of even and odd tokens
+    __shared__ Stage<TIn, GATE, DK> st[2];
+    __shared__ __align__(16) float red[NWARP * BW], tot[BW];
     const int i = threadIdx.x, j0 = blockIdx.x * BW, unit = blockIdx.y;
     const int b = unit / a.Hv, h = unit % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, M = (T + BLK - 1) / BLK, Dv = a.Dv;
+    if (M > 0) stage_issue<TIn, GATE, DK, false>(st[0], a, b, h, hk, j0, 0, min(BLK, T));
     float S[BW];
     const float *h0 = a.h0 ? a.h0 + ((size_t)unit * DK + i) * Dv + j0 : nullptr;
 #pragma unroll
     for (int j = 0; j < BW; ++j) S[j] = h0 ? h0[j] : 0.f;
     float *cku = ck + (size_t)unit * M * DK * Dv;
-    auto store = [&](int m) {
+    for (int m = 0; m < M; ++m) {
+        const int t0 = m * BLK, n = min(BLK, T - t0);
         float4 *dst = reinterpret_cast<float4 *>(cku + ((size_t)m * DK + i) * Dv + j0);
 #pragma unroll
         for (int j = 0; j < BW / 4; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-    };
-    store(0);
-    for (int t = 0; t < T; ++t) {
-        const size_t tv = (size_t)b * T + t;
-        const float ai = __expf(GATE ? a.g[(tv * a.Hv + h) * DK + i] : a.g[tv * a.Hv + h]);
-        const float ki = ld(reinterpret_cast<const TIn *>(a.k) + (tv * a.Hk + hk) * DK + i);
-        const float bt = a.beta[tv * a.Hv + h];
-        float *vrow = vrows + (t & 1) * BW;
-        if (i < BW) vrow[i] = ld(reinterpret_cast<const TIn *>(a.v) + (tv * a.Hv + h) * Dv + j0 + i);
-        float x[BW];
+        cp_wait_all();
+        __syncthreads();   // block m staged; every thread is done with block m - 1's buffer
+        if (m + 1 < M)
+            stage_issue<TIn, GATE, DK, false>(st[(m + 1) & 1], a, b, h, hk, j0, t0 + BLK, min(BLK, T - t0 - BLK));
+        const Stage<TIn, GATE, DK> &s = st[m & 1];
+        for (int tt = 0; tt < n; ++tt) {
+            const float ai = __expf(s.g[tt][GATE ? i : 0]);
+            const float ki = ld(&s.k[tt][i]);
+            const float bt = s.beta[tt];
+            float x[BW], vr[BW];
 #pragma unroll
-        for (int j = 0; j < BW; ++j) S[j] *= ai, x[j] = S[j] * ki;
-        column_sums<NWARP>(x, red, tot);
+            for (int j = 0; j < BW; ++j) S[j] *= ai, x[j] = S[j] * ki;
+            column_sums<NWARP>(x, red, tot);
+            load_row(&s.v[tt][0], vr);
 #pragma unroll
-        for (int j = 0; j < BW; ++j) S[j] = fmaf(ki, bt * (vrow[j] - tot[j]), S[j]);
-        if ((t + 1) % BLK == 0 && t + 1 < T) store((t + 1) / BLK);
+            for (int j = 0; j < BW; ++j) S[j] = fmaf(ki, bt * (vr[j] - tot[j]), S[j]);
+        }
     }
 }
 
@@ -107,15 +200,15 @@ __global__ void __launch_bounds__(DK)
 bwd_kernel(BwdArgs a, const float *ck)
 {
     constexpr int NWARP = DK / 32;
-    extern __shared__ __align__(16) float smf[];
-    float *Sbs = smf;                                   // [BLK][DK][SBLD] recomputed Sb of the block's tokens
-    float *es = Sbs + BLK * DK * SBLD;                  // [BLK][32] e of the block's tokens
-    float *red = es + BLK * BW, *tot = red + NWARP * BW, *vrows = tot + BW, *drow = vrows + 2 * BW;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    Stage<TIn, GATE, DK> *st = reinterpret_cast<Stage<TIn, GATE, DK> *>(smraw);
+    float *Sbs = reinterpret_cast<float *>(smraw + 2 * sizeof(Stage<TIn, GATE, DK>));  // [BLK][DK][SBLD]
+    float *es = Sbs + BLK * DK * SBLD;                  // [BLK][BW] e of the block's tokens
+    float *red = es + BLK * BW, *tot = red + NWARP * BW;
     const int i = threadIdx.x, lane = i & 31, j0 = blockIdx.x * BW, unit = blockIdx.y;
     const int b = unit / a.Hv, h = unit % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, M = (T + BLK - 1) / BLK, Dv = a.Dv;
-    const TIn *q = reinterpret_cast<const TIn *>(a.q), *k = reinterpret_cast<const TIn *>(a.k);
-    const TIn *v = reinterpret_cast<const TIn *>(a.v), *dout = reinterpret_cast<const TIn *>(a.dout);
+    if (M > 0) stage_issue<TIn, GATE, DK, true>(st[(M - 1) & 1], a, b, h, hk, j0, (M - 1) * BLK, T - (M - 1) * BLK);
     float dS[BW];
     const float *dhT = a.dhT ? a.dhT + ((size_t)unit * DK + i) * Dv + j0 : nullptr;
 #pragma unroll
@@ -123,7 +216,6 @@ bwd_kernel(BwdArgs a, const float *ck)
     const float *cku = ck + (size_t)unit * M * DK * Dv;
     for (int m = M - 1; m >= 0; --m) {
         const int t0 = m * BLK, n = min(BLK, T - t0);
-        // recompute the block's decayed states Sb and e from its checkpoint
         float S[BW];
         {
             const float4 *src = reinterpret_cast<const float4 *>(cku + ((size_t)m * DK + i) * Dv + j0);
@@ -133,34 +225,35 @@ bwd_kernel(BwdArgs a, const float *ck)
                 S[4 * j] = x.x, S[4 * j + 1] = x.y, S[4 * j + 2] = x.z, S[4 * j + 3] = x.w;
             }
         }
+        cp_wait_all();
+        __syncthreads();   // block m staged; every thread is done with block m + 1 (its buffer, Sbs, es)
+        if (m > 0) stage_issue<TIn, GATE, DK, true>(st[(m - 1) & 1], a, b, h, hk, j0, t0 - BLK, BLK);
+        const Stage<TIn, GATE, DK> &s = st[m & 1];
+        // recompute the block's decayed states Sb and e from its checkpoint
         for (int tt = 0; tt < n; ++tt) {
-            const size_t tv = (size_t)b * T + t0 + tt;
-            const float ai = __expf(GATE ? a.g[(tv * a.Hv + h) * DK + i] : a.g[tv * a.Hv + h]);
-            const float ki = ld(k + (tv * a.Hk + hk) * DK + i);
-            const float bt = a.beta[tv * a.Hv + h];
-            float *vrow = vrows + (tt & 1) * BW;   // even and odd tokens alternate
-            if (i < BW) vrow[i] = ld(v + (tv * a.Hv + h) * Dv + j0 + i);
-            float x[BW];
+            const float ai = __expf(s.g[tt][GATE ? i : 0]);
+            const float ki = ld(&s.k[tt][i]);
+            const float bt = s.beta[tt];
+            float x[BW], vr[BW];
             float4 *sb = reinterpret_cast<float4 *>(Sbs + ((size_t)tt * DK + i) * SBLD);
 #pragma unroll
             for (int j = 0; j < BW; ++j) S[j] *= ai, x[j] = S[j] * ki;
 #pragma unroll
             for (int j = 0; j < BW / 4; ++j) sb[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
             column_sums<NWARP>(x, red, tot);
-            if (i < BW) es[tt * BW + i] = vrow[i] - tot[i];
+            load_row(&s.v[tt][0], vr);
+            if (i < BW) es[tt * BW + i] = ld(&s.v[tt][i]) - tot[i];
 #pragma unroll
-            for (int j = 0; j < BW; ++j) S[j] = fmaf(ki, bt * (vrow[j] - tot[j]), S[j]);
+            for (int j = 0; j < BW; ++j) S[j] = fmaf(ki, bt * (vr[j] - tot[j]), S[j]);
         }
-        __syncthreads();
+        __syncthreads();   // es of the block visible to every thread
         // reverse the block's steps
         for (int tt = n - 1; tt >= 0; --tt) {
             const size_t tv = (size_t)b * T + t0 + tt;
-            const float ai = __expf(GATE ? a.g[(tv * a.Hv + h) * DK + i] : a.g[tv * a.Hv + h]);
+            const float ai = __expf(s.g[tt][GATE ? i : 0]);
+            const float ki = ld(&s.k[tt][i]), qi = ld(&s.q[tt][i]);
+            const float bt = s.beta[tt];
             const size_t kq = (tv * a.Hk + hk) * DK + i;
-            const float ki = ld(k + kq), qi = ld(q + kq);
-            const float bt = a.beta[tv * a.Hv + h];
-            if (i < BW) drow[i] = ld(dout + (tv * a.Hv + h) * Dv + j0 + i);
-            __syncthreads();
             float Sb[BW], e[BW], dd[BW];
             {
                 const float4 *sb = reinterpret_cast<const float4 *>(Sbs + ((size_t)tt * DK + i) * SBLD);
@@ -170,35 +263,43 @@ bwd_kernel(BwdArgs a, const float *ck)
                     Sb[4 * j] = x.x, Sb[4 * j + 1] = x.y, Sb[4 * j + 2] = x.z, Sb[4 * j + 3] = x.w;
                 }
             }
+            load_row(es + tt * BW, e);
+            load_row(&s.d[tt][0], dd);
+            // o = S'^T q: dS += q do^T, dq = S' do (two partial sums shorten the chain)
+            float dq0 = 0.f, dq1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < BW; ++j) e[j] = es[tt * BW + j], dd[j] = drow[j];
-            // o = S'^T q
-            float dq = 0.f;
-#pragma unroll
-            for (int j = 0; j < BW; ++j) {
+            for (int j = 0; j < BW; j += 2) {
                 dS[j] = fmaf(qi, dd[j], dS[j]);
-                dq = fmaf(fmaf(ki, bt * e[j], Sb[j]), dd[j], dq);
+                dS[j + 1] = fmaf(qi, dd[j + 1], dS[j + 1]);
+                dq0 = fmaf(fmaf(ki, bt * e[j], Sb[j]), dd[j], dq0);
+                dq1 = fmaf(fmaf(ki, bt * e[j + 1], Sb[j + 1]), dd[j + 1], dq1);
             }
-            atomicAdd(a.dq + kq, dq);
+            atomicAdd(a.dq + kq, dq0 + dq1);
             // S' = Sb + k u^T
             float x[BW];
 #pragma unroll
             for (int j = 0; j < BW; ++j) x[j] = dS[j] * ki;
             column_sums<NWARP>(x, red, tot);
-            float dk = 0.f, db = 0.f, rg = 0.f;
+            float dk0 = 0.f, dk1 = 0.f, db0 = 0.f, db1 = 0.f, rg0 = 0.f, rg1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < BW; ++j) {
-                const float du = tot[j], dp = -bt * du;
-                dk = fmaf(dS[j], bt * e[j], dk);       // dS u
-                db = fmaf(du, e[j], db);
-                dk = fmaf(Sb[j], dp, dk);              // Sb dp
-                const float dSb = fmaf(ki, dp, dS[j]);
-                rg = fmaf(dSb, Sb[j], rg);
-                dS[j] = ai * dSb;
+            for (int j = 0; j < BW; j += 2) {
+                const float du0 = tot[j], dp0 = -bt * du0, du1 = tot[j + 1], dp1 = -bt * du1;
+                dk0 = fmaf(dS[j], bt * e[j], dk0);           // dS u
+                dk1 = fmaf(dS[j + 1], bt * e[j + 1], dk1);
+                dk0 = fmaf(Sb[j], dp0, dk0);                 // Sb dp
+                dk1 = fmaf(Sb[j + 1], dp1, dk1);
+                db0 = fmaf(du0, e[j], db0);
+                db1 = fmaf(du1, e[j + 1], db1);
+                const float dSb0 = fmaf(ki, dp0, dS[j]), dSb1 = fmaf(ki, dp1, dS[j + 1]);
+                rg0 = fmaf(dSb0, Sb[j], rg0);
+                rg1 = fmaf(dSb1, Sb[j + 1], rg1);
+                dS[j] = ai * dSb0;
+                dS[j + 1] = ai * dSb1;
             }
-            atomicAdd(a.dk + kq, dk);
-            if (i == 0) atomicAdd(a.dbeta + tv * a.Hv + h, db);
+            atomicAdd(a.dk + kq, dk0 + dk1);
+            if (i == 0) atomicAdd(a.dbeta + tv * a.Hv + h, db0 + db1);
             if (i < BW) a.dv[(tv * a.Hv + h) * Dv + j0 + i] = bt * tot[i];
+            float rg = rg0 + rg1;
             if (GATE) {
                 atomicAdd(a.dg + (tv * a.Hv + h) * DK + i, rg);
             } else {
@@ -214,8 +315,12 @@ bwd_kernel(BwdArgs a, const float *ck)
         reinterpret_cast<float4 *>(dh0)[j] = make_float4(dS[4 * j], dS[4 * j + 1], dS[4 * j + 2], dS[4 * j + 3]);
 }
 
-template <int DK>
-constexpr size_t bwd_smem() { return ((size_t)BLK * DK * SBLD + BLK * BW + (DK / 32) * BW + 4 * BW) * sizeof(float); }
+template <typename TIn, int GATE, int DK>
+constexpr size_t bwd_smem()
+{
+    return 2 * sizeof(Stage<TIn, GATE, DK>) +
+           ((size_t)BLK * DK * SBLD + BLK * BW + (DK / 32) * BW + BW) * sizeof(float);
+}
 
 template <typename TIn, int GATE, int DK>
 cudaError_t launch_t(const BwdArgs &a, void *ws, cudaStream_t st)
@@ -225,10 +330,10 @@ cudaError_t launch_t(const BwdArgs &a, void *ws, cudaStream_t st)
     bwd_ckpt_kernel<TIn, GATE, DK><<<grid, DK, 0, st>>>(a, ck);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_kernel<TIn, GATE, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)bwd_smem<DK>());
+    constexpr size_t smem = bwd_smem<TIn, GATE, DK>();
+    e = cudaFuncSetAttribute(bwd_kernel<TIn, GATE, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_kernel<TIn, GATE, DK><<<grid, DK, bwd_smem<DK>(), st>>>(a, ck);
+    bwd_kernel<TIn, GATE, DK><<<grid, DK, smem, st>>>(a, ck);
     return cudaGetLastError();
 }
 
