@@ -10,20 +10,22 @@
 //             dg = row sums of dSb * Sb (summed over rows for a scalar gate);
 //             dS <- diag(a_t) dSb;  and dh0 = dS after the first token.
 //
-// The columns of S (value channels) evolve independently, so one CTA takes a
-// (batch row, value head, 16-column slice) and each of its Dk threads a row of
-// that slice. Two kernels:
-//   1. a forward pass that stores the state before every 8th token (workspace);
-//   2. a reverse pass that, per block of 8 tokens, recomputes the decayed states
-//      Sb from the block's checkpoint into shared memory, then runs the 8 reverse
+// The columns of S (value channels) evolve independently, so one CTA of four warps
+// takes a (batch row, value head, 16-column slice): each warp owns 4 columns over all
+// Dk rows, each lane Dk / 32 consecutive rows of them. The sums over rows (p, du) are
+// then sums within a warp (9 shuffles for the 4 columns), and only the sums over
+// columns (dq, dk, a per-channel dg) cross warps, once per reverse step through
+// shared memory. Two kernels:
+//   1. a forward pass that stores the state before every 6th token (workspace, in
+//      the kernels' own per-thread order);
+//   2. a reverse pass that, per block of 6 tokens, recomputes the decayed states
+//      Sb from the block's checkpoint into shared memory, then runs the 6 reverse
 //      steps. dv and dh0 belong to one slice and are stored; dq and dk (summed
 //      over slices and over the value heads that share a key head), dbeta and dg
 //      are accumulated with atomics into zeroed outputs.
 // Both kernels stage a block's inputs (k, q, the slice's v and do columns, g, beta)
 // in shared memory with asynchronous copies one block ahead, so no token waits on a
-// global load. Column sums over the Dk rows (p and du) use a shuffle transpose-reduce
-// per warp and shared memory across warps. The reverse kernel's shared memory (about
-// 92 KB for bf16 inputs and the scalar gate, 110 KB at most) lets two CTAs share an SM.
+// global load.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -34,9 +36,11 @@
 namespace gdr {
 namespace {
 
+constexpr int NT = 128;     // threads per CTA: four warps
+constexpr int CW = 4;       // value columns per warp
 constexpr int BW = 16;      // value columns per CTA
-constexpr int BLK = 8;      // tokens between checkpoints
-constexpr int SBLD = 20;    // fp32 row stride of a recomputed state slice (conflict-free 16-byte stores)
+constexpr int BLK = 6;      // tokens between checkpoints (69 KB of shared memory: three CTAs per SM)
+constexpr unsigned FULL = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void cp16(void *dst, const void *src)
@@ -74,20 +78,20 @@ __device__ __forceinline__ void stage_issue(Stage<TIn, GATE, DK> &s, const BwdAr
     const int tid = threadIdx.x;
     const TIn *k = reinterpret_cast<const TIn *>(a.k), *q = reinterpret_cast<const TIn *>(a.q);
     const TIn *v = reinterpret_cast<const TIn *>(a.v), *d = reinterpret_cast<const TIn *>(a.dout);
-    for (int c = tid; c < n * CR; c += DK) {
+    for (int c = tid; c < n * CR; c += NT) {
         const int tt = c / CR, x = (c % CR) * E;
         const size_t off = (((size_t)b * a.T + t0 + tt) * a.Hk + hk) * DK + x;
         cp16(&s.k[tt][x], k + off);
         if (REV) cp16(&s.q[tt][x], q + off);
     }
-    for (int c = tid; c < n * CV; c += DK) {
+    for (int c = tid; c < n * CV; c += NT) {
         const int tt = c / CV, x = (c % CV) * E;
         const size_t off = (((size_t)b * a.T + t0 + tt) * a.Hv + h) * a.Dv + j0 + x;
         cp16(&s.v[tt][x], v + off);
         if (REV) cp16(&s.d[tt][x], d + off);
     }
     if (GATE) {
-        for (int c = tid; c < n * (DK / 4); c += DK) {
+        for (int c = tid; c < n * (DK / 4); c += NT) {
             const int tt = c / (DK / 4), x = (c % (DK / 4)) * 4;
             cp16(&s.g[tt][x], a.g + (((size_t)b * a.T + t0 + tt) * a.Hv + h) * DK + x);
         }
@@ -99,227 +103,301 @@ __device__ __forceinline__ void stage_issue(Stage<TIn, GATE, DK> &s, const BwdAr
     cp_commit();
 }
 
-template <typename TIn>
-__device__ __forceinline__ float ld(const TIn *p) { return In<TIn>::load(p); }
-
-// The BW values of a staged slice row (broadcast reads).
-__device__ __forceinline__ void load_row(const float *p, float x[BW])
+// N consecutive values as fp32 (N = 2 or 4; a bf16 is the high half of its fp32 value).
+template <int N>
+__device__ __forceinline__ void load_n(const float *p, float x[N])
 {
-#pragma unroll
-    for (int j = 0; j < BW / 4; ++j) {
-        const float4 f = reinterpret_cast<const float4 *>(p)[j];
-        x[4 * j] = f.x, x[4 * j + 1] = f.y, x[4 * j + 2] = f.z, x[4 * j + 3] = f.w;
+    if (N == 4) {
+        const float4 f = *reinterpret_cast<const float4 *>(p);
+        x[0] = f.x, x[1] = f.y, x[2] = f.z, x[3] = f.w;
+    } else {
+        const float2 f = *reinterpret_cast<const float2 *>(p);
+        x[0] = f.x, x[1] = f.y;
     }
 }
-__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float x[BW])
+template <int N>
+__device__ __forceinline__ void load_n(const __nv_bfloat16 *p, float x[N])
 {
+    if (N == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        x[0] = __uint_as_float(u.x << 16), x[1] = __uint_as_float(u.x & 0xffff0000u);
+        x[2] = __uint_as_float(u.y << 16), x[3] = __uint_as_float(u.y & 0xffff0000u);
+    } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+        x[0] = __uint_as_float(u << 16), x[1] = __uint_as_float(u & 0xffff0000u);
+    }
+}
+template <int N>
+__device__ __forceinline__ void store_n(float *p, const float x[N])
+{
+    if (N == 4) *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    else *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+}
+
+// Totals over the warp's Dk rows of x[r][c] for its 4 columns, returned to every lane:
+// the lane's rows first, then a reduce-scatter across lanes (after the xor-1 and xor-2
+// exchanges lane l holds column 2 (l & 1) + (l >> 1 & 1)), a sum over the other lanes,
+// and an all-gather back to 4 columns.
+template <int R>
+__device__ __forceinline__ void col_sums(const float x[R][CW], float t[CW])
+{
+    float v[CW];
 #pragma unroll
-    for (int j = 0; j < BW / 8; ++j) {
-        const uint4 u = reinterpret_cast<const uint4 *>(p)[j];
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int c = 0; c < CW; ++c) {
+        v[c] = x[0][c];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {   // a bf16 is the high half of its fp32 value
-            x[8 * j + 2 * m] = __uint_as_float(w[m] << 16);
-            x[8 * j + 2 * m + 1] = __uint_as_float(w[m] & 0xffff0000u);
-        }
+        for (int r = 1; r < R; ++r) v[c] += x[r][c];
+    }
+    const int lane = threadIdx.x & 31;
+    const bool b0 = lane & 1, b1 = lane & 2;
+    const float a0 = (b0 ? v[2] : v[0]) + __shfl_xor_sync(FULL, b0 ? v[0] : v[2], 1);
+    const float a1 = (b0 ? v[3] : v[1]) + __shfl_xor_sync(FULL, b0 ? v[1] : v[3], 1);
+    float s = (b1 ? a1 : a0) + __shfl_xor_sync(FULL, b1 ? a0 : a1, 2);
+    s += __shfl_xor_sync(FULL, s, 4);
+    s += __shfl_xor_sync(FULL, s, 8);
+    s += __shfl_xor_sync(FULL, s, 16);
+    const float o = __shfl_xor_sync(FULL, s, 2);
+    const float u0 = b1 ? o : s, u1 = b1 ? s : o;               // columns 2 b0, 2 b0 + 1
+    const float p0 = __shfl_xor_sync(FULL, u0, 1), p1 = __shfl_xor_sync(FULL, u1, 1);
+    t[0] = b0 ? p0 : u0;
+    t[1] = b0 ? p1 : u1;
+    t[2] = b0 ? u0 : p0;
+    t[3] = b0 ? u1 : p1;
+}
+
+// The gate factors a_t of the lane's rows.
+template <typename TIn, int GATE, int DK>
+__device__ __forceinline__ void gate_rows(const Stage<TIn, GATE, DK> &s, int tt, int row0, float ar[DK / 32])
+{
+    constexpr int R = DK / 32;
+    if (GATE) {
+        load_n<R>(&s.g[tt][row0], ar);
+#pragma unroll
+        for (int r = 0; r < R; ++r) ar[r] = __expf(ar[r]);
+    } else {
+        const float a0 = __expf(s.g[tt][0]);
+#pragma unroll
+        for (int r = 0; r < R; ++r) ar[r] = a0;
     }
 }
 
-// Sum over the block's rows of x[j] for the BW columns: a transpose-reduce inside each
-// warp (lanes j and j + 16 end with the warp's sum of column j), then across warps
-// through shared memory. Every thread returns with all BW totals in tot (shared).
-template <int NWARP>
-__device__ __forceinline__ void column_sums(float x[BW], float *red, float *tot)
+// Offset (floats) of a thread's checkpoint: [unit][block][slice][thread][R rows x 4 columns].
+template <int DK>
+__device__ __forceinline__ size_t ck_off(int unit, int m, int M, int slice, int nslice)
 {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-    for (int s = BW / 2; s >= 1; s >>= 1) {
-        const bool upper = (lane & s) != 0;
-#pragma unroll
-        for (int i = 0; i < s; ++i) {
-            const float send = upper ? x[i] : x[i + s];
-            const float keep = upper ? x[i + s] : x[i];
-            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-        }
-    }
-    x[0] += __shfl_xor_sync(0xffffffffu, x[0], 16);
-    if (lane < BW) red[w * BW + lane] = x[0];
-    __syncthreads();
-    if (threadIdx.x < BW) {
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k < NWARP; ++k) s += red[k * BW + threadIdx.x];
-        tot[threadIdx.x] = s;
-    }
-    __syncthreads();
+    return (((size_t)unit * M + m) * nslice + slice) * ((size_t)DK * BW) + (size_t)threadIdx.x * (DK / 32) * CW;
 }
 
 template <typename TIn, int GATE, int DK>
-__global__ void __launch_bounds__(DK)
+__global__ void __launch_bounds__(NT)
 bwd_ckpt_kernel(BwdArgs a, float *ck)
 {
-    constexpr int NWARP = DK / 32;
+    constexpr int R = DK / 32;
     __shared__ Stage<TIn, GATE, DK> st[2];
-    __shared__ __align__(16) float red[NWARP * BW], tot[BW];
-    const int i = threadIdx.x, j0 = blockIdx.x * BW, unit = blockIdx.y;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int slice = blockIdx.x, j0 = slice * BW, unit = blockIdx.y;
     const int b = unit / a.Hv, h = unit % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, M = (T + BLK - 1) / BLK, Dv = a.Dv;
+    const int row0 = R * lane, col0 = j0 + CW * w;
     if (M > 0) stage_issue<TIn, GATE, DK, false>(st[0], a, b, h, hk, j0, 0, min(BLK, T));
-    float S[BW];
-    const float *h0 = a.h0 ? a.h0 + ((size_t)unit * DK + i) * Dv + j0 : nullptr;
+    float S[R][CW];
 #pragma unroll
-    for (int j = 0; j < BW; ++j) S[j] = h0 ? h0[j] : 0.f;
-    float *cku = ck + (size_t)unit * M * DK * Dv;
+    for (int r = 0; r < R; ++r) {
+        if (a.h0) load_n<CW>(a.h0 + ((size_t)unit * DK + row0 + r) * Dv + col0, S[r]);
+        else S[r][0] = S[r][1] = S[r][2] = S[r][3] = 0.f;
+    }
     for (int m = 0; m < M; ++m) {
         const int t0 = m * BLK, n = min(BLK, T - t0);
-        float4 *dst = reinterpret_cast<float4 *>(cku + ((size_t)m * DK + i) * Dv + j0);
+        float *dst = ck + ck_off<DK>(unit, m, M, slice, gridDim.x);
 #pragma unroll
-        for (int j = 0; j < BW / 4; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+        for (int r = 0; r < R; ++r) store_n<CW>(dst + r * CW, S[r]);
         cp_wait_all();
         __syncthreads();   // block m staged; every thread is done with block m - 1's buffer
         if (m + 1 < M)
             stage_issue<TIn, GATE, DK, false>(st[(m + 1) & 1], a, b, h, hk, j0, t0 + BLK, min(BLK, T - t0 - BLK));
         const Stage<TIn, GATE, DK> &s = st[m & 1];
         for (int tt = 0; tt < n; ++tt) {
-            const float ai = __expf(s.g[tt][GATE ? i : 0]);
-            const float ki = ld(&s.k[tt][i]);
+            float kr[R], ar[R], vc[CW], x[R][CW], p[CW];
+            load_n<R>(&s.k[tt][row0], kr);
+            gate_rows(s, tt, row0, ar);
             const float bt = s.beta[tt];
-            float x[BW], vr[BW];
+            load_n<CW>(&s.v[tt][CW * w], vc);
 #pragma unroll
-            for (int j = 0; j < BW; ++j) S[j] *= ai, x[j] = S[j] * ki;
-            column_sums<NWARP>(x, red, tot);
-            load_row(&s.v[tt][0], vr);
+            for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int j = 0; j < BW; ++j) S[j] = fmaf(ki, bt * (vr[j] - tot[j]), S[j]);
+                for (int c = 0; c < CW; ++c) S[r][c] *= ar[r], x[r][c] = S[r][c] * kr[r];
+            col_sums<R>(x, p);
+#pragma unroll
+            for (int c = 0; c < CW; ++c) p[c] = bt * (vc[c] - p[c]);
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) S[r][c] = fmaf(kr[r], p[c], S[r][c]);
         }
     }
 }
 
+// Shared memory of the reverse kernel (byte offsets; every region 16-byte aligned).
 template <typename TIn, int GATE, int DK>
-__global__ void __launch_bounds__(DK)
+struct RevSmem {
+    static constexpr int NV = (DK / 32) * CW;                             // state values per thread
+    static constexpr size_t sbs = 2 * sizeof(Stage<TIn, GATE, DK>);       // [BLK][NT][NV] Sb, per thread
+    static constexpr size_t es = sbs + (size_t)BLK * NT * NV * 4;         // [BLK][BW] e of the block's tokens
+    static constexpr size_t rp = es + (size_t)BLK * BW * 4;               // [2][3][4][DK] row partials
+    static constexpr size_t rs = rp + (size_t)2 * 3 * 4 * DK * 4;         // [2][2][4] warp totals
+    static constexpr size_t bytes = rs + 2 * 2 * 4 * 4;
+};
+
+template <typename TIn, int GATE, int DK>
+__global__ void __launch_bounds__(NT)
 bwd_kernel(BwdArgs a, const float *ck)
 {
-    constexpr int NWARP = DK / 32;
+    constexpr int R = DK / 32, NV = R * CW;
+    using L = RevSmem<TIn, GATE, DK>;
     extern __shared__ __align__(16) unsigned char smraw[];
     Stage<TIn, GATE, DK> *st = reinterpret_cast<Stage<TIn, GATE, DK> *>(smraw);
-    float *Sbs = reinterpret_cast<float *>(smraw + 2 * sizeof(Stage<TIn, GATE, DK>));  // [BLK][DK][SBLD]
-    float *es = Sbs + BLK * DK * SBLD;                  // [BLK][BW] e of the block's tokens
-    float *red = es + BLK * BW, *tot = red + NWARP * BW;
-    const int i = threadIdx.x, lane = i & 31, j0 = blockIdx.x * BW, unit = blockIdx.y;
+    float *Sbs = reinterpret_cast<float *>(smraw + L::sbs);
+    float *es = reinterpret_cast<float *>(smraw + L::es);
+    float *rp = reinterpret_cast<float *>(smraw + L::rp);
+    float *rs = reinterpret_cast<float *>(smraw + L::rs);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int slice = blockIdx.x, j0 = slice * BW, unit = blockIdx.y;
     const int b = unit / a.Hv, h = unit % a.Hv, hk = h / (a.Hv / a.Hk);
     const int T = a.T, M = (T + BLK - 1) / BLK, Dv = a.Dv;
+    const int row0 = R * lane, col0 = j0 + CW * w;
+    // a thread's Sb rows sit in 16-byte slots r ^ swz, so that the eight lanes of each
+    // 128-byte phase of a warp's access hit distinct banks
+    const int swz = (lane / (8 / R)) & (R - 1);
     if (M > 0) stage_issue<TIn, GATE, DK, true>(st[(M - 1) & 1], a, b, h, hk, j0, (M - 1) * BLK, T - (M - 1) * BLK);
-    float dS[BW];
-    const float *dhT = a.dhT ? a.dhT + ((size_t)unit * DK + i) * Dv + j0 : nullptr;
+    float dS[R][CW];
 #pragma unroll
-    for (int j = 0; j < BW; ++j) dS[j] = dhT ? dhT[j] : 0.f;
-    const float *cku = ck + (size_t)unit * M * DK * Dv;
+    for (int r = 0; r < R; ++r) {
+        if (a.dhT) load_n<CW>(a.dhT + ((size_t)unit * DK + row0 + r) * Dv + col0, dS[r]);
+        else dS[r][0] = dS[r][1] = dS[r][2] = dS[r][3] = 0.f;
+    }
     for (int m = M - 1; m >= 0; --m) {
         const int t0 = m * BLK, n = min(BLK, T - t0);
-        float S[BW];
+        float S[R][CW];
         {
-            const float4 *src = reinterpret_cast<const float4 *>(cku + ((size_t)m * DK + i) * Dv + j0);
+            const float *src = ck + ck_off<DK>(unit, m, M, slice, gridDim.x);
 #pragma unroll
-            for (int j = 0; j < BW / 4; ++j) {
-                const float4 x = src[j];
-                S[4 * j] = x.x, S[4 * j + 1] = x.y, S[4 * j + 2] = x.z, S[4 * j + 3] = x.w;
-            }
+            for (int r = 0; r < R; ++r) load_n<CW>(src + r * CW, S[r]);
         }
         cp_wait_all();
-        __syncthreads();   // block m staged; every thread is done with block m + 1 (its buffer, Sbs, es)
+        __syncthreads();   // block m staged; every thread is done with block m + 1 (buffer, es)
         if (m > 0) stage_issue<TIn, GATE, DK, true>(st[(m - 1) & 1], a, b, h, hk, j0, t0 - BLK, BLK);
         const Stage<TIn, GATE, DK> &s = st[m & 1];
         // recompute the block's decayed states Sb and e from its checkpoint
         for (int tt = 0; tt < n; ++tt) {
-            const float ai = __expf(s.g[tt][GATE ? i : 0]);
-            const float ki = ld(&s.k[tt][i]);
+            float kr[R], ar[R], vc[CW], x[R][CW], p[CW];
+            load_n<R>(&s.k[tt][row0], kr);
+            gate_rows(s, tt, row0, ar);
             const float bt = s.beta[tt];
-            float x[BW], vr[BW];
-            float4 *sb = reinterpret_cast<float4 *>(Sbs + ((size_t)tt * DK + i) * SBLD);
+            load_n<CW>(&s.v[tt][CW * w], vc);
+            float *sb = Sbs + ((size_t)tt * NT + tid) * NV;
 #pragma unroll
-            for (int j = 0; j < BW; ++j) S[j] *= ai, x[j] = S[j] * ki;
+            for (int r = 0; r < R; ++r) {
 #pragma unroll
-            for (int j = 0; j < BW / 4; ++j) sb[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-            column_sums<NWARP>(x, red, tot);
-            load_row(&s.v[tt][0], vr);
-            if (i < BW) es[tt * BW + i] = ld(&s.v[tt][i]) - tot[i];
+                for (int c = 0; c < CW; ++c) S[r][c] *= ar[r], x[r][c] = S[r][c] * kr[r];
+                store_n<CW>(sb + (r ^ swz) * CW, S[r]);
+            }
+            col_sums<R>(x, p);
 #pragma unroll
-            for (int j = 0; j < BW; ++j) S[j] = fmaf(ki, bt * (vr[j] - tot[j]), S[j]);
+            for (int c = 0; c < CW; ++c) p[c] = vc[c] - p[c];        // e
+            if (lane == 0) store_n<CW>(es + tt * BW + CW * w, p);
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) S[r][c] = fmaf(kr[r] * bt, p[c], S[r][c]);
         }
-        __syncthreads();   // es of the block visible to every thread
+        __syncwarp();      // e of the warp's columns visible to its lanes
         // reverse the block's steps
         for (int tt = n - 1; tt >= 0; --tt) {
-            const size_t tv = (size_t)b * T + t0 + tt;
-            const float ai = __expf(s.g[tt][GATE ? i : 0]);
-            const float ki = ld(&s.k[tt][i]), qi = ld(&s.q[tt][i]);
+            const int t = t0 + tt, par = t & 1;
+            const size_t tv = (size_t)b * T + t;
+            float kr[R], qr[R], ar[R], dd[CW], e[CW], Sb[R][CW];
+            load_n<R>(&s.k[tt][row0], kr);
+            load_n<R>(&s.q[tt][row0], qr);
+            gate_rows(s, tt, row0, ar);
             const float bt = s.beta[tt];
-            const size_t kq = (tv * a.Hk + hk) * DK + i;
-            float Sb[BW], e[BW], dd[BW];
+            load_n<CW>(&s.d[tt][CW * w], dd);
+            load_n<CW>(es + tt * BW + CW * w, e);
             {
-                const float4 *sb = reinterpret_cast<const float4 *>(Sbs + ((size_t)tt * DK + i) * SBLD);
+                const float *sb = Sbs + ((size_t)tt * NT + tid) * NV;
 #pragma unroll
-                for (int j = 0; j < BW / 4; ++j) {
-                    const float4 x = sb[j];
-                    Sb[4 * j] = x.x, Sb[4 * j + 1] = x.y, Sb[4 * j + 2] = x.z, Sb[4 * j + 3] = x.w;
+                for (int r = 0; r < R; ++r) load_n<CW>(sb + (r ^ swz) * CW, Sb[r]);
+            }
+            // o = S'^T q with S' = Sb + k (beta e)^T: dS += q do^T, dq = S' do
+            float dq[R], x[R][CW], du[CW];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float kb = kr[r] * bt;
+                float acc = 0.f;
+#pragma unroll
+                for (int c = 0; c < CW; ++c) {
+                    dS[r][c] = fmaf(qr[r], dd[c], dS[r][c]);
+                    acc = fmaf(fmaf(kb, e[c], Sb[r][c]), dd[c], acc);
+                    x[r][c] = dS[r][c] * kr[r];
+                }
+                dq[r] = acc;
+            }
+            col_sums<R>(x, du);
+            float dk[R], rg[R], dp[CW], db = 0.f;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) dp[c] = -bt * du[c], db = fmaf(du[c], e[c], db);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float k0 = 0.f, g0 = 0.f;
+#pragma unroll
+                for (int c = 0; c < CW; ++c) {
+                    k0 = fmaf(dS[r][c], bt * e[c], k0);      // dS u
+                    k0 = fmaf(Sb[r][c], dp[c], k0);          // Sb dp
+                    const float dSb = fmaf(kr[r], dp[c], dS[r][c]);
+                    g0 = fmaf(dSb, Sb[r][c], g0);
+                    dS[r][c] = ar[r] * dSb;
+                }
+                dk[r] = k0, rg[r] = g0;
+            }
+            if (lane == 0) {
+                const float dv4[CW] = {bt * du[0], bt * du[1], bt * du[2], bt * du[3]};
+                store_n<CW>(a.dv + (tv * a.Hv + h) * Dv + col0, dv4);
+            }
+            // row partials of this warp's columns; buffers alternate with the token parity
+            float *rpp = rp + (size_t)par * 3 * 4 * DK;
+            store_n<R>(rpp + (0 * 4 + w) * DK + row0, dq);
+            store_n<R>(rpp + (1 * 4 + w) * DK + row0, dk);
+            if (GATE) {
+                store_n<R>(rpp + (2 * 4 + w) * DK + row0, rg);
+            } else {
+                float gs = rg[0];
+#pragma unroll
+                for (int r = 1; r < R; ++r) gs += rg[r];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) gs += __shfl_xor_sync(FULL, gs, off);
+                if (lane == 0) rs[(par * 2 + 1) * 4 + w] = gs;
+            }
+            if (lane == 0) rs[(par * 2 + 0) * 4 + w] = db;
+            __syncthreads();   // every warp's partials written; the other parity's buffers were read
+            if (tid < DK) {
+                const size_t kq = (tv * a.Hk + hk) * DK + tid;
+                const float *q0 = rpp, *q1 = rpp + 4 * DK;
+                atomicAdd(a.dq + kq, (q0[tid] + q0[DK + tid]) + (q0[2 * DK + tid] + q0[3 * DK + tid]));
+                atomicAdd(a.dk + kq, (q1[tid] + q1[DK + tid]) + (q1[2 * DK + tid] + q1[3 * DK + tid]));
+                if (GATE) {
+                    const float *q2 = rpp + 8 * DK;
+                    atomicAdd(a.dg + (tv * a.Hv + h) * DK + tid,
+                              (q2[tid] + q2[DK + tid]) + (q2[2 * DK + tid] + q2[3 * DK + tid]));
                 }
             }
-            load_row(es + tt * BW, e);
-            load_row(&s.d[tt][0], dd);
-            // o = S'^T q: dS += q do^T, dq = S' do (two partial sums shorten the chain)
-            float dq0 = 0.f, dq1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < BW; j += 2) {
-                dS[j] = fmaf(qi, dd[j], dS[j]);
-                dS[j + 1] = fmaf(qi, dd[j + 1], dS[j + 1]);
-                dq0 = fmaf(fmaf(ki, bt * e[j], Sb[j]), dd[j], dq0);
-                dq1 = fmaf(fmaf(ki, bt * e[j + 1], Sb[j + 1]), dd[j + 1], dq1);
-            }
-            atomicAdd(a.dq + kq, dq0 + dq1);
-            // S' = Sb + k u^T
-            float x[BW];
-#pragma unroll
-            for (int j = 0; j < BW; ++j) x[j] = dS[j] * ki;
-            column_sums<NWARP>(x, red, tot);
-            float dk0 = 0.f, dk1 = 0.f, db0 = 0.f, db1 = 0.f, rg0 = 0.f, rg1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < BW; j += 2) {
-                const float du0 = tot[j], dp0 = -bt * du0, du1 = tot[j + 1], dp1 = -bt * du1;
-                dk0 = fmaf(dS[j], bt * e[j], dk0);           // dS u
-                dk1 = fmaf(dS[j + 1], bt * e[j + 1], dk1);
-                dk0 = fmaf(Sb[j], dp0, dk0);                 // Sb dp
-                dk1 = fmaf(Sb[j + 1], dp1, dk1);
-                db0 = fmaf(du0, e[j], db0);
-                db1 = fmaf(du1, e[j + 1], db1);
-                const float dSb0 = fmaf(ki, dp0, dS[j]), dSb1 = fmaf(ki, dp1, dS[j + 1]);
-                rg0 = fmaf(dSb0, Sb[j], rg0);
-                rg1 = fmaf(dSb1, Sb[j + 1], rg1);
-                dS[j] = ai * dSb0;
-                dS[j + 1] = ai * dSb1;
-            }
-            atomicAdd(a.dk + kq, dk0 + dk1);
-            if (i == 0) atomicAdd(a.dbeta + tv * a.Hv + h, db0 + db1);
-            if (i < BW) a.dv[(tv * a.Hv + h) * Dv + j0 + i] = bt * tot[i];
-            float rg = rg0 + rg1;
-            if (GATE) {
-                atomicAdd(a.dg + (tv * a.Hv + h) * DK + i, rg);
-            } else {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) rg += __shfl_xor_sync(0xffffffffu, rg, off);
-                if (lane == 0) atomicAdd(a.dg + tv * a.Hv + h, rg);
+            if (tid == 0) {
+                const float *r0 = rs + par * 2 * 4;
+                atomicAdd(a.dbeta + tv * a.Hv + h, (r0[0] + r0[1]) + (r0[2] + r0[3]));
+                if (!GATE) atomicAdd(a.dg + tv * a.Hv + h, (r0[4] + r0[5]) + (r0[6] + r0[7]));
             }
         }
     }
-    float *dh0 = a.dh0 + ((size_t)unit * DK + i) * Dv + j0;
 #pragma unroll
-    for (int j = 0; j < BW / 4; ++j)
-        reinterpret_cast<float4 *>(dh0)[j] = make_float4(dS[4 * j], dS[4 * j + 1], dS[4 * j + 2], dS[4 * j + 3]);
-}
-
-template <typename TIn, int GATE, int DK>
-constexpr size_t bwd_smem()
-{
-    return 2 * sizeof(Stage<TIn, GATE, DK>) +
-           ((size_t)BLK * DK * SBLD + BLK * BW + (DK / 32) * BW + BW) * sizeof(float);
+    for (int r = 0; r < R; ++r) store_n<CW>(a.dh0 + ((size_t)unit * DK + row0 + r) * Dv + col0, dS[r]);
 }
 
 template <typename TIn, int GATE, int DK>
@@ -327,13 +405,13 @@ cudaError_t launch_t(const BwdArgs &a, void *ws, cudaStream_t st)
 {
     const dim3 grid(a.Dv / BW, a.B * a.Hv);
     float *ck = reinterpret_cast<float *>(ws);
-    bwd_ckpt_kernel<TIn, GATE, DK><<<grid, DK, 0, st>>>(a, ck);
+    bwd_ckpt_kernel<TIn, GATE, DK><<<grid, NT, 0, st>>>(a, ck);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    constexpr size_t smem = bwd_smem<TIn, GATE, DK>();
+    constexpr size_t smem = RevSmem<TIn, GATE, DK>::bytes;
     e = cudaFuncSetAttribute(bwd_kernel<TIn, GATE, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_kernel<TIn, GATE, DK><<<grid, DK, smem, st>>>(a, ck);
+    bwd_kernel<TIn, GATE, DK><<<grid, NT, smem, st>>>(a, ck);
     return cudaGetLastError();
 }
 
