@@ -16,10 +16,10 @@
 // then sums within a warp (9 shuffles for the 4 columns), and only the sums over
 // columns (dq, dk, a per-channel dg) cross warps, once per reverse step through
 // shared memory. Two kernels:
-//   1. a forward pass that stores the state before every 6th token (workspace, in
+//   1. a forward pass that stores the state before every 4th token (workspace, in
 //      the kernels' own per-thread order);
-//   2. a reverse pass that, per block of 6 tokens, recomputes the decayed states
-//      Sb from the block's checkpoint into shared memory, then runs the 6 reverse
+//   2. a reverse pass that, per block of 4 tokens, recomputes the decayed states
+//      Sb from the block's checkpoint into shared memory, then runs the 4 reverse
 //      steps. dv and dh0 belong to one slice and are stored; dq and dk (summed
 //      over slices and over the value heads that share a key head), dbeta and dg
 //      are accumulated with atomics into zeroed outputs.
@@ -39,7 +39,7 @@ namespace {
 constexpr int NT = 128;     // threads per CTA: four warps
 constexpr int CW = 4;       // value columns per warp
 constexpr int BW = 16;      // value columns per CTA
-constexpr int BLK = 6;      // tokens between checkpoints (69 KB of shared memory: three CTAs per SM)
+constexpr int BLK = 4;      // tokens between checkpoints (50 KB of shared memory: four CTAs per SM)
 constexpr unsigned FULL = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }

@@ -100,15 +100,15 @@ GDR_API unsigned long long gdr_kernel_launches(void);
  *   dh0     [B, Hv, Dk, Dv] fp32
  * Inputs as for gdr_fwd_chunked; dout [B, T, Hv, Dv] in the input dtype (GDR_BF16
  * or GDR_BF16_OUT_F32: bf16; GDR_FP32: fp32), dhT fp32. The arithmetic is fp32:
- * a forward pass stores the state before every 6th token in the workspace, then a
- * reverse pass recomputes each block of 6 tokens and reverses its steps.
+ * a forward pass stores the state before every 4th token in the workspace, then a
+ * reverse pass recomputes each block of 4 tokens and reverses its steps.
  * Needs Dk of 64 or 128 and Dv of 64 or 128 (else GDR_ERR_UNSUPPORTED); the other
  * argument errors are those of gdr_fwd_chunked. All pointers 16-byte aligned;
  * the outputs must not alias the inputs or each other. T == 0 writes dh0 = dhT
  * (or zeros) and nothing else.
  *
  * workspace: device buffer of at least gdr_bwd_workspace_size(...) bytes
- * (B * Hv * ceil(T / 6) * Dk * Dv * 4), owned by the caller; two calls that
+ * (B * Hv * ceil(T / 4) * Dk * Dv * 4), owned by the caller; two calls that
  * overlap in time must not share one. Asynchronous on `stream`.
  */
 GDR_API size_t gdr_bwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype);
