@@ -89,3 +89,55 @@ def test_rejects_unsupported_and_small_workspace():
         gdr.gdr_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do, dhT,
                     workspace=torch.empty(16, dtype=torch.uint8, device=DEV))
     assert ei.value.status == gdr.GDR_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("T", [3, 7, 11])
+def test_lengths_that_leave_a_partial_checkpoint_block(T):
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=T, Hk=1, Hv=2, gate="channel", g_mu=2.0, seed=820 + T)
+    check(w, seed=20 + T)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 128), (128, 64)])
+def test_rectangular_states(Dk, Dv):
+    w = WORKLOADS["gdn_bf16"].with_(B=1, T=50, Hk=2, Hv=4, Dk=Dk, Dv=Dv, dtype="fp32", seed=830 + Dk)
+    check(w, seed=7)
+
+
+def test_strong_decay():
+    """g = logsigmoid(N(-1, 1)): the state forgets within a few tokens, and a = exp(g)
+    spans several orders of magnitude inside one checkpoint block."""
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=70, Hk=2, Hv=2, g_mu=-1.0, seed=840)
+    check(w, seed=8)
+
+
+def sampled_unit_check(w, units, seed):
+    """Gradients of the full-size workload against the oracle run on the sampled (b, key head)
+    groups: each group carries every value head that shares its key head, so dq and dk
+    (summed over those heads) are complete."""
+    inp = make_inputs(w, DEV)
+    do, dhT = upstream(w, seed)
+    got = gdr.gdr_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do, dhT)
+    torch.cuda.synchronize()
+    grp = w.Hv // w.Hk
+    for b, hk in units:
+        hv = slice(hk * grp, (hk + 1) * grp)
+        sk = lambda x: x[b:b + 1, :, hk:hk + 1].cpu()
+        sv = lambda x: x[b:b + 1, :, hv].cpu()
+        ref = oracle.backward(sk(inp["q"]), sk(inp["k"]), sv(inp["v"]), sv(inp["g"]), sv(inp["beta"]),
+                              inp["h0"][b:b + 1, hv].cpu(), sv(do), dhT[b:b + 1, hv].cpu())
+        sel = {"dq": got["dq"][b:b + 1, :, hk:hk + 1], "dk": got["dk"][b:b + 1, :, hk:hk + 1],
+               "dv": got["dv"][b:b + 1, :, hv], "dg": got["dg"][b:b + 1, :, hv],
+               "dbeta": got["dbeta"][b:b + 1, :, hv], "dh0": got["dh0"][b:b + 1, hv]}
+        for n in NAMES:
+            err = rel_err(sel[n], ref[n])
+            assert err <= TOL, (w.name, b, hk, n, err)
+
+
+def test_grouped_value_shape_sampled_units():
+    """B=4, T=4096, Hk=16, Hv=48: three value heads per key head."""
+    sampled_unit_check(WORKLOADS["gva_gdn_bf16"], [(0, 0), (3, 15)], seed=9)
+
+
+def test_kda_shape_sampled_units():
+    """B=2, T=16384, H=32, per-channel gate (a 17 GB checkpoint workspace)."""
+    sampled_unit_check(WORKLOADS["kda_bf16"], [(0, 0), (1, 31)], seed=10)
