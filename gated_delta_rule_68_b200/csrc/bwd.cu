@@ -134,19 +134,19 @@ __device__ __forceinline__ void store_n(float *p, const float x[N])
     else *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
 }
 
-// Totals over the warp's Dk rows of x[r][c] for its 4 columns, returned to every lane:
-// the lane's rows first, then a reduce-scatter across lanes (after the xor-1 and xor-2
+// Totals over the warp's Dk rows of x[r][c] * y[r] for its 4 columns, returned to every
+// lane: the lane's rows first, then a reduce-scatter across lanes (after the xor-1 and xor-2
 // exchanges lane l holds column 2 (l & 1) + (l >> 1 & 1)), a sum over the other lanes,
 // and an all-gather back to 4 columns.
 template <int R>
-__device__ __forceinline__ void col_sums(const float x[R][CW], float t[CW])
+__device__ __forceinline__ void col_sums(const float x[R][CW], const float y[R], float t[CW])
 {
     float v[CW];
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
-        v[c] = x[0][c];
+        v[c] = x[0][c] * y[0];
 #pragma unroll
-        for (int r = 1; r < R; ++r) v[c] += x[r][c];
+        for (int r = 1; r < R; ++r) v[c] = fmaf(x[r][c], y[r], v[c]);
     }
     const int lane = threadIdx.x & 31;
     const bool b0 = lane & 1, b1 = lane & 2;
@@ -217,7 +217,7 @@ bwd_ckpt_kernel(BwdArgs a, float *ck)
             stage_issue<TIn, GATE, DK, false>(st[(m + 1) & 1], a, b, h, hk, j0, t0 + BLK, min(BLK, T - t0 - BLK));
         const Stage<TIn, GATE, DK> &s = st[m & 1];
         for (int tt = 0; tt < n; ++tt) {
-            float kr[R], ar[R], vc[CW], x[R][CW], p[CW];
+            float kr[R], ar[R], vc[CW], p[CW];
             load_n<R>(&s.k[tt][row0], kr);
             gate_rows(s, tt, row0, ar);
             const float bt = s.beta[tt];
@@ -225,8 +225,8 @@ bwd_ckpt_kernel(BwdArgs a, float *ck)
 #pragma unroll
             for (int r = 0; r < R; ++r)
 #pragma unroll
-                for (int c = 0; c < CW; ++c) S[r][c] *= ar[r], x[r][c] = S[r][c] * kr[r];
-            col_sums<R>(x, p);
+                for (int c = 0; c < CW; ++c) S[r][c] *= ar[r];
+            col_sums<R>(S, kr, p);
 #pragma unroll
             for (int c = 0; c < CW; ++c) p[c] = bt * (vc[c] - p[c]);
 #pragma unroll
@@ -289,7 +289,7 @@ bwd_kernel(BwdArgs a, const float *ck)
         const Stage<TIn, GATE, DK> &s = st[m & 1];
         // recompute the block's decayed states Sb and e from its checkpoint
         for (int tt = 0; tt < n; ++tt) {
-            float kr[R], ar[R], vc[CW], x[R][CW], p[CW];
+            float kr[R], ar[R], vc[CW], p[CW];
             load_n<R>(&s.k[tt][row0], kr);
             gate_rows(s, tt, row0, ar);
             const float bt = s.beta[tt];
@@ -298,10 +298,10 @@ bwd_kernel(BwdArgs a, const float *ck)
 #pragma unroll
             for (int r = 0; r < R; ++r) {
 #pragma unroll
-                for (int c = 0; c < CW; ++c) S[r][c] *= ar[r], x[r][c] = S[r][c] * kr[r];
+                for (int c = 0; c < CW; ++c) S[r][c] *= ar[r];
                 store_n<CW>(sb + (r ^ swz) * CW, S[r]);
             }
-            col_sums<R>(x, p);
+            col_sums<R>(S, kr, p);
 #pragma unroll
             for (int c = 0; c < CW; ++c) p[c] = vc[c] - p[c];        // e
             if (lane == 0) store_n<CW>(es + tt * BW + CW * w, p);
@@ -327,21 +327,23 @@ bwd_kernel(BwdArgs a, const float *ck)
 #pragma unroll
                 for (int r = 0; r < R; ++r) load_n<CW>(sb + (r ^ swz) * CW, Sb[r]);
             }
-            // o = S'^T q with S' = Sb + k (beta e)^T: dS += q do^T, dq = S' do
-            float dq[R], x[R][CW], du[CW];
+            // o = S'^T q with S' = Sb + k (beta e)^T: dS += q do^T, and
+            // dq = S' do = Sb do + k beta (e . do)
+            float dq[R], du[CW], ed = 0.f;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) ed = fmaf(e[c], dd[c], ed);
+            ed *= bt;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float kb = kr[r] * bt;
-                float acc = 0.f;
+                float acc = kr[r] * ed;
 #pragma unroll
                 for (int c = 0; c < CW; ++c) {
                     dS[r][c] = fmaf(qr[r], dd[c], dS[r][c]);
-                    acc = fmaf(fmaf(kb, e[c], Sb[r][c]), dd[c], acc);
-                    x[r][c] = dS[r][c] * kr[r];
+                    acc = fmaf(Sb[r][c], dd[c], acc);
                 }
                 dq[r] = acc;
             }
-            col_sums<R>(x, du);
+            col_sums<R>(dS, kr, du);
             float dk[R], rg[R], dp[CW], db = 0.f;
 #pragma unroll
             for (int c = 0; c < CW; ++c) dp[c] = -bt * du[c], db = fmaf(du[c], e[c], db);
