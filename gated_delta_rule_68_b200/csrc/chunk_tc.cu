@@ -103,7 +103,7 @@ enum {
     B_YE,           // the state group has read P and Qh out of Y and X (128 arrivals)
     B_SE,           // the state group has read the state product (128 arrivals)
     B_OE,           // the state group has read the o accumulator (128 arrivals)
-    B_DR0, B_DR1,   // end-of-kernel drain of each issuing thread's MMAs
+    B_DR0, B_DR1, B_DR2,   // end-of-kernel drain of each issuing thread's MMAs
     NBAR
 };
 
@@ -255,7 +255,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), 512);
     if (NORM && a.z && tid < D) reinterpret_cast<float *>(sm + OFF_NW)[tid] = a.norm_w[tid];
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 1, 1, GT, GT, 1, 1, 1, 1, GT, GT, GT, GT, 1, 1};
+        const uint32_t counts[NBAR] = {1, 1, 1, 1, GT, GT, 1, 1, 1, 1, GT, GT, GT, GT, 1, 1, 1};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
         abort_sh = 0;
     }
@@ -540,6 +540,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // TMA loads, the bf16 -> fp16 conversion of K, Q and V in place, the gate vectors
         // and the Gram.
         const bool issuer = tid == 0;
+        const bool gissuer = tid == 7 * 32;   // the Gram's issuer: warp 7 has no gate-vector work
         auto issue_loads = [&](int c) {
             const int sb = c & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES, bl = bar(B_LD0 + sb);
@@ -564,7 +565,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 gb[2 + e] = ok ? a.beta[ix] : 0.f;
             }
         };
-        // Chunk c's tiles to fp16 in place and its gate vectors (warp 0), then its Gram.
+        // Chunk c's tiles to fp16 in place, then its Gram (warp 7) while warps 0 .. 6 write its
+        // gate vectors.
         auto ready_chunk = [&](int c, const float gb[4]) {
             const int sb = c & 1;
             uint8_t *stgp = sm + sb * STG_BYTES;
@@ -594,17 +596,36 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
                 }
             } else {
+                // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64
+                // rows), four loads in flight before their conversions
 #pragma unroll
-                for (int j = 0; j < 3072 / GT; ++j) {
-                    // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64 rows)
-                    const int e = tid + GT * j;
-                    const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
-                    uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
-                    *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                for (int j0 = 0; j0 < 3072 / GT; j0 += 4) {
+                    uint4 u[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) u[j] = reinterpret_cast<const uint4 *>(stgp)[tid + GT * (j0 + j)];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int e = tid + GT * (j0 + j);
+                        const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
+                        reinterpret_cast<uint4 *>(stgp)[e] = row < nvalid ? bf16x8_to_f16x8(u[j]) : make_uint4(0, 0, 0, 0);
+                    }
                 }
             }
-            // Gate vectors: every warp scans G (lane l: rows l, l + 32), then writes its share.
-            if (warp < 6) {
+            fence_proxy_async();
+            named_bar_sync(2, GT);   // every tile of the chunk converted
+            if (gissuer) {
+                const uint32_t stg = sb0 + sb * STG_BYTES;
+                if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t ad = stg + (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_ss(tb + TM_G, sdesc(ad, 16, 1024), sdesc(ad, 16, 1024), ID_GRAM, s > 0);
+                }
+                mma_commit(bar(B_G0 + sb));
+            }
+            // Gate vectors: warps 0 .. 6 scan G (lane l: rows l, l + 32), then write their shares.
+            if (warp < 7) {
                 float s0 = gb[0], s1 = gb[1];
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -618,15 +639,19 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int r = lane + 32 * e;
-                        const float be = gb[2 + e];
-                        const float gam = __expf(G[e]);
                         vs[V_G + r] = G[e];
-                        vs[V_GAM + r] = gam;
-                        vs[V_F + r] = __expf(GC - G[e]);
-                        vs[V_BETA + r] = be;
-                        vs[V_BG + r] = be * gam;
+                        vs[V_GAM + r] = __expf(G[e]);
                     }
                     if (lane == 0) vs[V_GC] = __expf(GC);
+                } else if (warp == 6) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = lane + 32 * e;
+                        const float be = gb[2 + e];
+                        vs[V_F + r] = __expf(GC - G[e]);
+                        vs[V_BETA + r] = be;
+                        vs[V_BG + r] = be * __expf(G[e]);
+                    }
                 } else if (warp == 1) {   // exp(G_r - G_16R), R = r / 16
                     const float b0 = __shfl_sync(0xffffffffu, s0, lane & ~15), b1 = __shfl_sync(0xffffffffu, s1, lane & ~15);
                     vs[V_EROW + lane] = __expf(s0 - b0);
@@ -638,20 +663,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     vs[V_ECOL + rb * 64 + 32 + lane] = __expf(ref - s1);
                 }
             }
-            fence_proxy_async();
             mbar_arrive(bar(B_CV0 + sb));
-            named_bar_sync(2, GT);
-            if (issuer) {
-                const uint32_t stg = sb0 + sb * STG_BYTES;
-                if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t ad = stg + (s >> 2) * 16384 + (s & 3) * 32;
-                    mma_ss(tb + TM_G, sdesc(ad, 16, 1024), sdesc(ad, 16, 1024), ID_GRAM, s > 0);
-                }
-                mma_commit(bar(B_G0 + sb));
-            }
         };
 
         float S[64];
@@ -863,6 +875,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         if (issuer) {
             mma_commit(bar(B_DR0));
             mbar_wait_bounded(bar(B_DR0), 0);
+        }
+        if (gissuer) {
+            mma_commit(bar(B_DR2));
+            mbar_wait_bounded(bar(B_DR2), 0);
         }
     }
     tc_fence_before();
