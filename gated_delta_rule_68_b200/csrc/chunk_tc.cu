@@ -338,37 +338,39 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             // ... and with W^T (the tiles of T) before they are rewritten.
             if (c >= 1) wait(B_P, (c - 1) & 1);
             // Inverse, level 0: warp wq of the first half inverts the unit lower 16 x 16 block
-            // I + A_bb (b = wq) by forward substitution (lane j < 16 holds column j); the
-            // second half zeroes the blocks of T above the diagonal.
+            // I + A_bb (b = wq) by forward substitution (lanes j and j + 16 both hold column j,
+            // so that the 48 stores per column split evenly: lanes 0-15 write D_b and rows 0-7
+            // of T', lanes 16-31 write T'' and rows 8-15 of T'); the second half zeroes the
+            // blocks of T above the diagonal.
             if (hf == 0) {
-                if (lane < 16) {
-                    const int j = lane;
-                    float t[16];
+                const int j = lane & 15;
+                const bool lo = lane < 16;
+                float t[16];
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) t[rr] = rr == j ? 1.f : 0.f;
-                    const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;
+                for (int rr = 0; rr < 16; ++rr) t[rr] = rr == j ? 1.f : 0.f;
+                const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;
 #pragma unroll
-                    for (int i = 0; i < 15; ++i) {
-                        float col[16];
+                for (int i = 0; i < 15; ++i) {
+                    float col[16];
 #pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const float4 x = *reinterpret_cast<const float4 *>(ad + i * LDAD + 4 * k4);
-                            col[4 * k4] = x.x, col[4 * k4 + 1] = x.y, col[4 * k4 + 2] = x.z, col[4 * k4 + 3] = x.w;
-                        }
-                        const float ti = t[i];
-#pragma unroll
-                        for (int rr = i + 1; rr < 16; ++rr) t[rr] = fmaf(-col[rr], ti, t[rr]);
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 x = *reinterpret_cast<const float4 *>(ad + i * LDAD + 4 * k4);
+                        col[4 * k4] = x.x, col[4 * k4 + 1] = x.y, col[4 * k4 + 2] = x.z, col[4 * k4 + 3] = x.w;
                     }
-                    __half *dd = reinterpret_cast<__half *>(sm + INV_D) + wq * 16 * LDT16;
-                    const int I = 16 * wq + j;
-                    const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
+                    const float ti = t[i];
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) {
-                        dd[rr * LDT16 + j] = __float2half_rn(t[rr]);
-                        st_h1(sm, OFF_TP + swz_off(16 * wq + rr, I, 0), t[rr] * sbg);
-                        st_h1(sm, OFF_TPP + swz_off(16 * wq + rr, I, 0), t[rr] * sbt);
-                    }
+                    for (int rr = i + 1; rr < 16; ++rr) t[rr] = fmaf(-col[rr], ti, t[rr]);
                 }
+                const int I = 16 * wq + j;
+                const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
+                const uint32_t dd0 = INV_D + (uint32_t)(wq * 16 * LDT16 + j) * 2u;
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr)   // D_b row rr (lanes 0-15), T'' row rr (lanes 16-31)
+                    st_h1(sm, lo ? dd0 + (uint32_t)(rr * LDT16) * 2u : OFF_TPP + swz_off(16 * wq + rr, I, 0),
+                          lo ? t[rr] : t[rr] * sbt);
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr)    // T' row rr (lanes 0-15), row rr + 8 (lanes 16-31)
+                    st_h1(sm, OFF_TP + swz_off(16 * wq + (lo ? rr : rr + 8), I, 0), (lo ? t[rr] : t[rr + 8]) * sbg);
             } else {
                 // zero chunks: row u of block R = u / 16, 16-byte chunks 2(R+1) .. 7, of one of the two tiles
                 const int u = (gt - GT / 2) & 63, R = u >> 4;
