@@ -16,15 +16,18 @@
 //   S_next = Gamma_C S + P S + R,   P = -Kt^T W,  R = Kt^T U
 //   O      = Qh S + Uh,             Qh = diag(Gamma) Q - M W,  Uh = M U
 // and P, R, Qh, Uh depend on the chunk's inputs alone. So the kernel runs two
-// warpgroups:
-//   - the chunk group (warps 4-7) builds P, R, Qh, Uh for one chunk after the
-//     other: the Gram [K; Q] K^T, the gate factors, the inverse (fp32 16 x 16
-//     diagonal blocks, off-diagonal blocks by warp-level MMA), then W, U and the
-//     four products, all large products on tcgen05;
-//   - the state group (warps 0-3) keeps S (fp32, one value column per thread, in
-//     registers) and per chunk issues one batch of MMAs that adds P S to R and
+// groups of eight warps:
+//   - the chunk group (warps 8-15) builds P, R, Qh, Uh for one chunk after the
+//     other: the gated Gram epilogue (A and M), the inverse (fp32 16 x 16
+//     diagonal blocks, off-diagonal blocks as register-chained warp-level MMAs),
+//     then W, U and the four products, all large products on tcgen05;
+//   - the state group (warps 0-7) keeps S (fp32 in registers, half a value column
+//     per thread) and per chunk issues one batch of MMAs that adds P S to R and
 //     Qh S to Uh in tensor memory, then forms S_next = Gamma_C S + (P S + R),
-//     writes its fp16 copy (the next batch's operand) and stores o.
+//     writes its fp16 copy (the next batch's operand) and stores o through a
+//     swizzled shared-memory tile and TMA. In the rest of its time it readies
+//     chunk c + 2: TMA loads, bf16 -> fp16 conversion in place, the gate vectors
+//     and the Gram [K; Q] K^T (issued by warp 7).
 // The chunk group runs one chunk ahead of the state group, so the inverse and
 // the other chunk-local work overlap the state chain, and the state chain of a
 // chunk is one MMA batch and two short epilogues.
