@@ -132,7 +132,7 @@ def rank_workload(w, rank):
 
 
 def max_over_ranks(x, device=None):
-    """The largest of every rank's value (the step time the job is judged by)."""
+    """The largest of every rank's value (the step time of the whole job)."""
     import torch
     import torch.distributed as dist
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
