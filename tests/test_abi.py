@@ -169,3 +169,39 @@ def test_empty_calls_launch_nothing(L):
     assert norm(L, rows=0) == gdr.GDR_OK
     assert conv(L, T=0) == gdr.GDR_OK    # no tokens, no state_out: nothing to do
     assert L.gdr_kernel_launches() == before
+
+
+def bwd(L, q=A, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, h0=0, do=A + 20480, dhT=0,
+        dq=A + 24576, dk=A + 28672, dv=A + 32768, dg=A + 36864, dbeta=A + 40960, dh0=A + 45056,
+        B=1, T=16, Hk=1, Hv=1, Dk=128, Dv=128, gate=0, dtype=0, ws=0, ws_bytes=0):
+    vp = ctypes.c_void_p
+    ptrs = [q, k, v, g, beta, h0, do, dhT, dq, dk, dv, dg, dbeta, dh0]
+    return L.gdr_bwd(*(vp(p or None) for p in ptrs), B, T, Hk, Hv, Dk, Dv, gate, dtype, vp(ws or None),
+                     ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hk=2, Hv=3), gdr.GDR_ERR_INVALID_ARG),
+    (dict(Dk=96), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(Dv=32), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(gate=3), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dtype=9), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dh0=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(do=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dq=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dbeta=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(dhT=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(), gdr.GDR_ERR_WORKSPACE),                          # no workspace given
+    (dict(ws=A + (1 << 24), ws_bytes=16), gdr.GDR_ERR_WORKSPACE),
+])
+def test_bwd_rejects(L, kw, status):
+    assert bwd(L, **kw) == status
+    assert len(gdr.gdr_last_error()) > 0
+
+
+def test_bwd_workspace_size_rules(L):
+    # the state before every 4th token, fp32, per (batch row, value head)
+    assert L.gdr_bwd_workspace_size(2, 10, 1, 3, 128, 64, 0, 0) == 2 * 3 * 3 * 128 * 64 * 4
+    assert L.gdr_bwd_workspace_size(1, 8, 1, 1, 64, 64, 1, 1) == 2 * 64 * 64 * 4
+    assert L.gdr_bwd_workspace_size(0, 8, 1, 1, 64, 64, 0, 0) == 0
+    assert L.gdr_bwd_workspace_size(1, 0, 1, 1, 64, 64, 0, 0) == 0
