@@ -18,6 +18,13 @@ region. ``roofline`` compares algorithmic HBM bytes per launch with the
 measured HBM copy bandwidth. ``cpu_baseline`` times the fp64 CPU oracle on a
 bounded sample of the same workload on this host's cores.
 
+Other workloads (``--workload``): ``gva_gdn_bf16`` and ``kda_bf16`` (the same
+step on the grouped-value and per-channel-gate shapes), ``decode_bf16`` (one
+``gdr_decode_step`` over the batch per step), ``gdn_layer_bf16`` (three short
+convolutions plus the forward with its q/k and output norms) and ``gdn_bwd_bf16``
+(one ``gdr_bwd`` call per step, against the fp32 ALU roofline). ``--T`` shortens
+a workload's sequences for profiling small cases.
+
 ``--impl reference`` times that oracle alone (the reference arm): each step is
 a bounded sample of the workload on the host cores.
 """

@@ -66,7 +66,7 @@ int set_failure(int status, const char *msg) { return fail(status, "%s", msg); }
 
 extern "C" {
 
-int gdr_version(void) { return 100; }
+int gdr_version(void) { return 200; }
 
 const char *gdr_last_error(void) { return g_err; }
 

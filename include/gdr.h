@@ -64,7 +64,7 @@ typedef enum {
     GDR_ERR_INVALID_ARG = 1,   /* bad size, Hv % Hk != 0, NULL required pointer, bad enum */
     GDR_ERR_UNSUPPORTED = 2,   /* Dk or Dv not 64 or 128 */
     GDR_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
-    GDR_ERR_WORKSPACE = 4,     /* workspace missing or smaller than gdr_fwd_workspace_size() */
+    GDR_ERR_WORKSPACE = 4,     /* workspace missing or smaller than gdr_fwd_workspace_size() (gdr_bwd_workspace_size() for gdr_bwd) */
     GDR_ERR_CUDA = 5           /* a CUDA launch or runtime call failed */
 } gdr_status;
 
