@@ -837,36 +837,77 @@ def main(argv=None):
     e2e = None
     if not args.no_e2e:
         host = {n: (None if x is None else x.pin_memory()) for n, x in inp_cpu.items()}
-        dbuf = {n: (None if x is None else torch.empty_like(x, device=dev)) for n, x in inp_cpu.items()}
-        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        hT_h = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for x in host.values() if x is not None)
-        d2h = o_h.numel() * o_h.element_size() + hT_h.numel() * hT_h.element_size()
+        names = [n for n, x in host.items() if x is not None]
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+        d2h = o.numel() * o.element_size() + hT.numel() * hT.element_size()
         e2e_steps = max(3, min(args.steps, 10))
+        # Two sets of device and pinned result buffers: step i's inputs go in on s_in and its
+        # results out on s_out while step i - 1 computes, as a pipelined caller would run it.
+        dbufs = [{n: torch.empty_like(host[n], device=dev) for n in names} for _ in range(2)]
+        obufs = [(torch.empty_like(o), torch.empty_like(hT)) for _ in range(2)]
+        hbufs = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(hT.shape, dtype=hT.dtype).pin_memory())
+                 for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_ready, comp_done, out_done = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+        used = [False, False]
 
-        def e2e_step():
-            for n, x in host.items():
-                if x is not None:
-                    dbuf[n].copy_(x, non_blocking=True)
-            gdr.gdr_fwd_chunked(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["h0"], o=o,
-                                hT=hT, workspace=ws, stream=stream)
-            o_h.copy_(o, non_blocking=True)
-            hT_h.copy_(hT, non_blocking=True)
+        def e2e_step(i):
+            j = i % 2
+            d, (od, hd), (oh, hh) = dbufs[j], obufs[j], hbufs[j]
+            if used[j]:
+                s_in.wait_event(comp_done[j])     # step i - 2 has read this input set
+            with torch.cuda.stream(s_in):
+                for n in names:
+                    d[n].copy_(host[n], non_blocking=True)
+                in_ready[j].record(s_in)
+            stream.wait_event(in_ready[j])
+            if used[j]:
+                stream.wait_event(out_done[j])    # step i - 2's results have left this output set
+            gdr.gdr_fwd_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("h0"), o=od, hT=hd,
+                                workspace=ws, stream=stream)
+            comp_done[j].record(stream)
+            s_out.wait_event(comp_done[j])
+            with torch.cuda.stream(s_out):
+                oh.copy_(od, non_blocking=True)
+                hh.copy_(hd, non_blocking=True)
+                out_done[j].record(s_out)
+            used[j] = True
 
-        for _ in range(2):
-            e2e_step()
+        def serial_step():
+            d = dbufs[0]
+            for n in names:
+                d[n].copy_(host[n], non_blocking=True)
+            gdr.gdr_fwd_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("h0"), o=o, hT=hT,
+                                workspace=ws, stream=stream)
+            hbufs[0][0].copy_(o, non_blocking=True)
+            hbufs[0][1].copy_(hT, non_blocking=True)
+
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)                      # before the first copy in
+        for i in range(2, 2 + e2e_steps):
+            e2e_step(i)
+        e1.record(s_out)                     # after the last copy out
         torch.cuda.synchronize()
         te = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+        # the same steps one after another on one stream, for reference
+        serial_step()
+        torch.cuda.synchronize()
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        for _ in range(e2e_steps):
+            serial_step()
+        e3.record(stream)
+        torch.cuda.synchronize()
+        ts = max_over_ranks(e2.elapsed_time(e3) / e2e_steps, dev)
         e2e = {"value": job_tokens_per_s(w.head_tokens, world, te), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-               "ms_per_step": te}
+               "ms_per_step": te, "pipelined": "inputs of step i+1 and results of step i-1 cross the "
+               "host link while step i computes (two copy streams, two buffer sets)",
+               "serial_ms_per_step": ts}
 
     if world > 1:
         dist.barrier()
