@@ -402,6 +402,8 @@ def run_reference(args, w, rank, world):
         return run_layer_reference(args, w, world)
     if w.bwd:
         return run_bwd_reference(args, w, world)
+    if w.decode:
+        return run_decode_reference(args, w, world)
     cores = oracle.threads_used(0, 1 << 30)
     units = max(cores, 8)
     sample = w.with_(B=units, Hk=1, Hv=1)
@@ -666,6 +668,61 @@ def workload_config(w, world):
 
 
 # ----------------------------------------------------------------------------- decode
+def decode_oracle_sample(w, target_s=12.0):
+    """Time the fp64 oracle's decode steps on a bounded sample: `units` (batch row, value
+    head) states stepped through `steps` tokens, chosen to take about target_s seconds."""
+    import oracle
+    from gated_delta_rule_68_b200.workloads import make_inputs
+    cores = oracle.threads_used(0, 1 << 30)
+    units, steps = max(cores, 8), 8
+    sample = w.with_(B=units, Hk=1, Hv=1, T=steps)
+    inp = make_inputs(sample, "cpu")
+    arrs = [inp[n].double().numpy() for n in ("q", "k", "v", "g", "beta", "h0")]
+    reps, dt = 0, 0.0
+    while reps == 0 or (dt < target_s and reps < 1000):
+        t0 = time.perf_counter()
+        oracle.decode_steps(*arrs)
+        dt += time.perf_counter() - t0
+        reps += 1
+    return {"value": reps * units * steps / dt, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{units} (batch row, value head) states of Dk=Dv={w.Dk} through {steps} decode steps, "
+                      f"fp64, run {reps} times; {dt:.1f} s"}
+
+
+def run_decode_reference(args, w, world):
+    """The reference arm on the decode workload: each step is one fp64 decode step of a sample
+    of (batch row, value head) states on the host cores."""
+    import oracle
+    from gated_delta_rule_68_b200.workloads import make_inputs
+    units = max(oracle.threads_used(0, 1 << 30), 8)
+    sample = w.with_(B=units, Hk=1, Hv=1, T=args.warmup + args.steps)
+    inp = make_inputs(sample, "cpu")
+    q, k, v, g, beta = (inp[n].double().numpy() for n in ("q", "k", "v", "g", "beta"))
+    S = inp["h0"].double().numpy()
+    times = []
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        _, S = oracle.decode_steps(q[it:it + 1], k[it:it + 1], v[it:it + 1], g[it:it + 1], beta[it:it + 1], S)
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    value = units / per_step
+    metric = "gated-delta decode tokens/s (B·Hv per sec per step) bf16 d=128; % of roofline"
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same recipe as the GPU arm)", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads_used(0, units),
+                         "kind": "oracle",
+                         "sample": f"each step: one fp64 decode step of {units} (batch row, value head) states"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_decode_bench(args, w, wr, rank, world, local, dev):
     """One step = one gdr_decode_step over the whole batch: every (batch row, value head)
     state is read and written once. Each step takes the next pre-generated token."""
@@ -753,7 +810,8 @@ def run_decode_bench(args, w, wr, rank, world, local, dev):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg,
                      "traffic": traffic, "traffic_kernel": traffic_kernel, "kernel": "gdr_decode_step"},
-        "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches,
+        "cpu_baseline": decode_oracle_sample(w) if world == 1 and not args.no_cpu_baseline else None,
+        "e2e": e2e, "gpu_launches": launches,
         "launches_per_step": launches / args.steps, "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -36,3 +36,19 @@ def test_backward_reference_arm_prints_one_line(capsys):
     line = json.loads(capsys.readouterr().out.strip())
     assert line["impl"] == "reference" and line["metric"] == bench.BWD_METRIC and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_decode_reference_arm_prints_one_line(capsys):
+    w = WORKLOADS["decode_bf16"].with_(Dk=16, Dv=16)
+
+    class Args:
+        warmup, steps = 1, 2
+    assert bench.run_decode_reference(Args, w, 1) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["value"] > 0 and "decode" in line["metric"]
+
+
+def test_decode_oracle_sample_is_bounded():
+    w = WORKLOADS["decode_bf16"].with_(Dk=16, Dv=16)
+    cpu = bench.decode_oracle_sample(w, target_s=0.5)
+    assert cpu["kind"] == "oracle" and cpu["value"] > 0 and cpu["seconds"] < 5.0
