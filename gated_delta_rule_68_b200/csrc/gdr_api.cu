@@ -135,6 +135,9 @@ int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
         g_launches += 1;
         return GDR_OK;
     }
+    if (B > 65535)   // its kernels put the batch row on the grid's z axis
+        return fail(GDR_ERR_UNSUPPORTED, "the CUDA-core path (fp32 inputs, d = 64, rectangular states) takes at "
+                                         "most 65535 batch rows; got %d", B);
     const size_t need = gdr::simt_workspace_size(a);
     if (need > 0 && (!workspace || workspace_bytes < need))
         return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, workspace_bytes,
@@ -267,6 +270,9 @@ int gdr_bwd(const void *q, const void *k, const void *v, const float *g, const f
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.dh0 = dh0;
     a.B = B; a.T = T; a.Hk = Hk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.gate_mode = gate_mode; a.dtype = dtype;
     if (!gdr::bwd_supported(a)) return fail(GDR_ERR_UNSUPPORTED, "the backward needs Dk of 64 or 128");
+    if ((long)B * Hv > 65535)   // (batch row, value head) is the grid's y axis
+        return fail(GDR_ERR_UNSUPPORTED, "the backward takes at most 65535 (batch row, value head) pairs; got %ld",
+                    (long)B * Hv);
     const size_t need = gdr::bwd_workspace_size(a);
     if (!workspace || workspace_bytes < need)
         return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, workspace_bytes,

@@ -102,7 +102,8 @@ GDR_API unsigned long long gdr_kernel_launches(void);
  * or GDR_BF16_OUT_F32: bf16; GDR_FP32: fp32), dhT fp32. The arithmetic is fp32:
  * a forward pass stores the state before every 4th token in the workspace, then a
  * reverse pass recomputes each block of 4 tokens and reverses its steps.
- * Needs Dk of 64 or 128 and Dv of 64 or 128 (else GDR_ERR_UNSUPPORTED); the other
+ * Needs Dk of 64 or 128, Dv of 64 or 128 and B * Hv <= 65535 (else
+ * GDR_ERR_UNSUPPORTED); the other
  * argument errors are those of gdr_fwd_chunked. All pointers 16-byte aligned;
  * the outputs must not alias the inputs or each other. T == 0 writes dh0 = dhT
  * (or zeros) and nothing else.
@@ -160,7 +161,8 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  * the masked (Q*Gamma)(K/Gamma)^T above), for the per-channel gate on the
  * warp-level tensor cores. Both use fp16 operands, fp32 accumulation and an
  * fp32 carried state; q, k, v and the state must stay inside the fp16 range,
- * |x| < 6.5e4. Other shapes and fp32 inputs run fp32 CUDA-core kernels.
+ * |x| < 6.5e4. Other shapes and fp32 inputs run fp32 CUDA-core kernels, which
+ * take at most 65535 batch rows (else GDR_ERR_UNSUPPORTED).
  * B == 0 or T == 0 is a valid no-op that still writes hT = h0 (or zeros).
  *
  * workspace: device buffer of at least gdr_fwd_workspace_size(...) bytes,

@@ -205,3 +205,12 @@ def test_bwd_workspace_size_rules(L):
     assert L.gdr_bwd_workspace_size(1, 8, 1, 1, 64, 64, 1, 1) == 2 * 64 * 64 * 4
     assert L.gdr_bwd_workspace_size(0, 8, 1, 1, 64, 64, 0, 0) == 0
     assert L.gdr_bwd_workspace_size(1, 0, 1, 1, 64, 64, 0, 0) == 0
+
+
+def test_grid_limits_are_reported_before_launch(L):
+    # the backward's (batch row, value head) axis and the CUDA-core path's batch axis
+    assert bwd(L, B=70000, Hv=1, ws=A + (1 << 24), ws_bytes=1 << 62) == gdr.GDR_ERR_UNSUPPORTED
+    assert "65535" in gdr.gdr_last_error()
+    st = fwd(L, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, o=A + 20480, B=70000, dtype=gdr.GDR_FP32,
+             ws=A + (1 << 24), ws_bytes=1 << 62)
+    assert st == gdr.GDR_ERR_UNSUPPORTED and "65535" in gdr.gdr_last_error()
