@@ -56,6 +56,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--T", type=int, default=None,
                    help="override the workload's sequence length (small cases for profiling)")
+    p.add_argument("--B", type=int, default=None,
+                   help="override the workload's batch size (small cases for profiling)")
     a = p.parse_args(argv)
     a.warmup = max(a.warmup, 3)
     return a
@@ -829,6 +831,8 @@ def main(argv=None):
     w = WORKLOADS[args.workload]
     if args.T is not None:
         w = w.with_(name=f"{w.name}_T{args.T}", T=args.T)
+    if args.B is not None:
+        w = w.with_(name=f"{w.name}_B{args.B}", B=args.B)
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
 

@@ -10,7 +10,7 @@
 // Method: the exact chunkwise form of
 //   S_t = (I - beta_t k_t k_t^T) diag(exp g_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
 // (NextTransformer, "Source notes", "Linear attention", rows gdn and kda;
-// SinkProbe (Attention-Sink) README: delta-rule layer in exact chunkwise form).
+// SinkProbe (Attention-Sink) README: its delta-rule layer, evaluated chunk by chunk).
 // With G_r = sum_{j<=r} g_j inside the chunk (per channel for the channel gate),
 // Gamma_r = exp(G_r), Gamma_C = Gamma_63:
 //   A_ri = beta_r sum_c k_rc k_ic exp(G_rc - G_ic)  (i < r),   T = (I + A)^-1

@@ -2,9 +2,9 @@
 //
 // This path serves fp32 inputs, where the 1e-4 accuracy asked of fp32 rules
 // out bf16 or tf32 tensor-core operands, and any shape the tensor-core path
-// does not take. It follows the exact chunkwise form (SinkProbe
-// (Attention-Sink) README: the delta-rule layer "computed in exact chunkwise
-// form"), with chunks of C = 64 tokens. For one (b, h) and one chunk with
+// does not take. It evaluates the recurrence chunk by chunk with no
+// approximation (SinkProbe (Attention-Sink) README, description of its
+// delta-rule layer), with chunks of C = 64 tokens. For one (b, h) and one chunk with
 // cumulative log-gate G_r = sum_{j<=r} g_j and Gamma = exp(G):
 //
 //   prep  (chunk-parallel)  A = tril(diag(beta)(K*Gamma)(K/Gamma)^T, -1)

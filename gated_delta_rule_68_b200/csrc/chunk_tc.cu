@@ -6,7 +6,7 @@
 // Method: the exact chunkwise form of
 //   S_t = (I - beta_t k_t k_t^T) exp(g_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
 // (NextTransformer, "Source notes", "Linear attention", row gdn; SinkProbe
-// (Attention-Sink) README: delta-rule layer in exact chunkwise form). Inside a
+// (Attention-Sink) README: its delta-rule layer, evaluated chunk by chunk). Inside a
 // chunk, with G_r = sum_{j<=r} g_j, Gamma_r = exp(G_r), Gamma_C = Gamma_63:
 //   A_ri = beta_r exp(G_r - G_i) k_r.k_i (i < r),   T = (I + A)^-1
 //   W = T diag(beta Gamma) K,   U = T diag(beta) V,   U' = U - W S
@@ -120,8 +120,33 @@ constexpr uint32_t ID_UH = idesc_f16(128, 64, false, false, false);
 constexpr uint32_t ID_S = idesc_f16(128, 128, false, false, false);
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false, true);
 
-// Waits that timed out (each abandons its CTA's remaining work).
+// Waits that timed out (each abandons its CTA's remaining work), and units in which a
+// value rounded to an fp16 operand left fp16's range (inf or NaN: that unit's o and hT
+// are not valid).
 __device__ unsigned int g_tc_timeouts;
+__device__ unsigned int g_tc_range_errors;
+
+// Values of magnitude 65520 and above round to inf in fp16. Each stage that rounds values
+// to fp16 operands takes their largest |x| and raises the CTA's flag if it is out of range
+// (a NaN can only follow an earlier overflow or a non-finite input, and inputs are checked
+// on their fp16 bits).
+__device__ __forceinline__ float amax_n(const float *x, int n)
+{
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < n; ++i) m = fmaxf(m, fabsf(x[i]));
+    return m;
+}
+__device__ __forceinline__ void flag_range(int *flag, float m)
+{
+    if (!(m < 65520.f)) *reinterpret_cast<volatile int *>(flag) = 1;
+}
+// Bit 15 (31) of the result is set when the low (high) half of a packed fp16 pair is inf or NaN.
+__device__ __forceinline__ uint32_t f16x8_bad(uint4 u)
+{
+    constexpr uint32_t E = 0x7c007c00u, C1 = 0x04000400u;
+    return ((u.x & E) + C1) | ((u.y & E) + C1) | ((u.z & E) + C1) | ((u.w & E) + C1);
+}
 
 __device__ __forceinline__ uint32_t pack_h2(float x, float y)
 {
@@ -203,8 +228,9 @@ __device__ __forceinline__ void chain_next(float c0[4], float c1[4], uint32_t aB
 // Writes block (R0.., I0..) of T, given as two n8 tiles times `s`, into T diag(beta Gamma)
 // and T diag(beta) (swizzled [r][i] tiles).
 __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const float c0[4], const float c1[4], float s,
-                                          const float *vec, int lane)
+                                          const float *vec, int lane, int *range_flag)
 {
+    float m = 0.f;
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -212,11 +238,13 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = R0 + g + 8 * (e >> 1), i = I0 + 8 * nt + 2 * t4 + (e & 1);
-            const float t = s * c[e];
-            st_h1(sm, OFF_TP + swz_off(r, i, 0), t * vec[V_BG + i]);
-            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t * vec[V_BETA + i]);
+            const float t = s * c[e], t1 = t * vec[V_BG + i], t2 = t * vec[V_BETA + i];
+            m = fmaxf(m, fmaxf(fabsf(t1), fabsf(t2)));
+            st_h1(sm, OFF_TP + swz_off(r, i, 0), t1);
+            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t2);
         }
     }
+    flag_range(range_flag, m);
 }
 
 // NORM: the layer's options (compiled as a separate instance, so the plain forward runs
@@ -236,6 +264,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     __shared__ uint64_t bars[NBAR];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    __shared__ int range_sh;   // set when a value rounded to an fp16 operand is out of range
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -261,6 +290,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         const uint32_t counts[NBAR] = {1, 1, 1, 1, GT, GT, 1, 1, 1, 1, GT, GT, GT, GT, 1, 1, 1};
         for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), counts[i]);
         abort_sh = 0;
+        range_sh = 0;
     }
     tc_fence_before();
     __syncthreads();
@@ -312,6 +342,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     v[i + 2] = i + 2 < lim ? rowf * e.z * v[i + 2] : 0.f;
                     v[i + 3] = i + 3 < lim ? rowf * e.w * v[i + 3] : 0.f;
                 }
+                flag_range(&range_sh, amax_n(v, 32));
                 // The previous chunk's first products are done with M and U^T (the inverse's scratch).
                 if (c >= 1) wait(B_P1, (c - 1) & 1);
                 if (p >= 64) {
@@ -366,6 +397,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 }
                 const int I = 16 * wq + j;
                 const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
+                flag_range(&range_sh, amax_n(t, 16) * fmaxf(1.f, fmaxf(fabsf(sbg), fabsf(sbt))));
                 const uint32_t dd0 = INV_D + (uint32_t)(wq * 16 * LDT16 + j) * 2u;
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr)   // D_b row rr (lanes 0-15), T'' row rr (lanes 16-31)
@@ -401,14 +433,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 if (wq == 0) {
                     chain_start(c0, c1, Dt(1), LDT16, At(1, 0), LDA16, lane);
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 16, 0, c0, c1, -1.f, vc, lane);
+                    st_tblock(sm, 16, 0, c0, c1, -1.f, vc, lane, &range_sh);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
-                    st_tblock(sm, 32, 16, c0, c1, -1.f, vc, lane);
+                    st_tblock(sm, 32, 16, c0, c1, -1.f, vc, lane, &range_sh);
                 } else if (wq == 1) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
-                    st_tblock(sm, 48, 32, c0, c1, -1.f, vc, lane);
+                    st_tblock(sm, 48, 32, c0, c1, -1.f, vc, lane, &range_sh);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
                     chain_next(c0, c1, At(1, 0), LDA16, lane);
@@ -416,7 +448,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 32, 0, c0, c1, 1.f, vc, lane);
+                    st_tblock(sm, 32, 0, c0, c1, 1.f, vc, lane, &range_sh);
                 } else if (wq == 2) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
@@ -425,7 +457,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(1), LDT16, lane);
-                    st_tblock(sm, 48, 16, c0, c1, 1.f, vc, lane);
+                    st_tblock(sm, 48, 16, c0, c1, 1.f, vc, lane, &range_sh);
                 } else {
                     float q0[4], q1[4], h0[4], h1[4];
                     chain_start(q0, q1, Dt(3), LDT16, At(3, 2), LDA16, lane);   // Q = D3 A32 D2
@@ -443,7 +475,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] = u0[e] + h0[e] - c0[e], c1[e] = u1[e] + h1[e] - c1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 48, 0, c0, c1, 1.f, vc, lane);
+                    st_tblock(sm, 48, 0, c0, c1, 1.f, vc, lane, &range_sh);
                 }
             }
             fence_proxy_async();
@@ -471,6 +503,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 32 * hf), tmem_addr(tb, q4, TM_Y + 64 + 32 * hf), v);
+                flag_range(&range_sh, amax_n(v, 64));
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_W16), v + 8 * j);
 #pragma unroll
@@ -578,6 +611,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             float *vs = vec + sb * V_SET;
             wait(B_LD0 + sb, (c >> 1) & 1);
             const int nvalid = min(C, T - c * C);
+            uint32_t rin = 0;   // fp16 inf/NaN bits of the converted inputs
             if (NORM && a.qk_l2norm) {
                 // [K; Q] rows: chunks e and e + 1024 are the two halves of one row, and a row's 8
                 // chunks of a half sit in 8 adjacent threads
@@ -591,14 +625,19 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
                     ss += __shfl_xor_sync(0xffffffffu, ss, 4);
                     const float sc = rsqrtf(ss + 1e-6f);
-                    *p0 = row < nvalid ? bf16x8_scaled_f16x8(u0, sc) : make_uint4(0, 0, 0, 0);
-                    *p1 = row < nvalid ? bf16x8_scaled_f16x8(u1, sc) : make_uint4(0, 0, 0, 0);
+                    const uint4 h0v = row < nvalid ? bf16x8_scaled_f16x8(u0, sc) : make_uint4(0, 0, 0, 0);
+                    const uint4 h1v = row < nvalid ? bf16x8_scaled_f16x8(u1, sc) : make_uint4(0, 0, 0, 0);
+                    rin |= f16x8_bad(h0v) | f16x8_bad(h1v);
+                    *p0 = h0v;
+                    *p1 = h1v;
                 }
 #pragma unroll
                 for (int j = 8; j < 3072 / GT; ++j) {
                     const int e = tid + GT * j, row = ((e - 2048) >> 3) & 63;
                     uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
-                    *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                    const uint4 hv = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                    rin |= f16x8_bad(hv);
+                    *pch = hv;
                 }
             } else {
                 // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64
@@ -612,10 +651,13 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int j = 0; j < 4; ++j) {
                         const int e = tid + GT * (j0 + j);
                         const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
-                        reinterpret_cast<uint4 *>(stgp)[e] = row < nvalid ? bf16x8_to_f16x8(u[j]) : make_uint4(0, 0, 0, 0);
+                        const uint4 hv = row < nvalid ? bf16x8_to_f16x8(u[j]) : make_uint4(0, 0, 0, 0);
+                        rin |= f16x8_bad(hv);
+                        reinterpret_cast<uint4 *>(stgp)[e] = hv;
                     }
                 }
             }
+            if (rin & 0x80008000u) *reinterpret_cast<volatile int *>(&range_sh) = 1;
             fence_proxy_async();
             named_bar_sync(2, GT);   // every tile of the chunk converted
             if (gissuer) {
@@ -676,6 +718,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + (size_t)(64 * hf) * D + p : nullptr;
 #pragma unroll
             for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
+            flag_range(&range_sh, amax_n(S, 64));
 #pragma unroll
             for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
         }
@@ -705,6 +748,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[32];
                 tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
+                flag_range(&range_sh, amax_n(v, 32));
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
             }
@@ -715,6 +759,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 64 * hf), tmem_addr(tb, q4, TM_Y + 64 * hf + 32), v);
+                flag_range(&range_sh, amax_n(v, 64));
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
             }
@@ -747,6 +792,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tmem_ld32x2(tmem_addr(tb, q4, TM_S + 64 * hf), tmem_addr(tb, q4, TM_S + 64 * hf + 32), v);
 #pragma unroll
                 for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
+                flag_range(&range_sh, amax_n(S, 64));
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
             }
@@ -888,6 +934,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     }
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && range_sh) atomicAdd(&g_tc_range_errors, 1u);
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tb, 512);
@@ -929,6 +976,13 @@ unsigned int tc_error_count()
     unsigned int t = 0;
     cudaMemcpyFromSymbol(&t, g_tc_timeouts, sizeof(t));
     return t;
+}
+
+unsigned int tc_range_error_count()
+{
+    unsigned int r = 0;
+    cudaMemcpyFromSymbol(&r, g_tc_range_errors, sizeof(r));
+    return r;
 }
 
 }  // namespace gdr

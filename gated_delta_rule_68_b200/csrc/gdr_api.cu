@@ -77,6 +77,7 @@ unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *r
     unsigned int t = 0, r = 0;
     gdr::fused_error_counts(&t, &r);
     t += gdr::tc_error_count();
+    r += gdr::tc_range_error_count();
     if (load_timeouts) *load_timeouts = t;
     if (range_errors) *range_errors = r;
     return t + r;

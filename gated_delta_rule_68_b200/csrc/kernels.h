@@ -49,8 +49,10 @@ unsigned int fused_error_counts(unsigned int *load_timeouts, unsigned int *range
 // fixed-length sequences, no layer options): one kernel, no workspace.
 bool tc_supported(const FwdArgs &a);
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st);
-// Waits of the tcgen05 kernel that timed out since the library was loaded on this device.
+// Waits of the tcgen05 kernel that timed out since the library was loaded on this device,
+// and its units in which a value rounded to an fp16 operand was inf or NaN.
 unsigned int tc_error_count();
+unsigned int tc_range_error_count();
 
 // Backward of the recurrence (bwd.cu): gradients of L = sum(dout * o) + sum(dhT * hT), all
 // fp32 [q, k: B,T,Hk,Dk; v: B,T,Hv,Dv; g: g's layout; beta: B,T,Hv; h0: B,Hv,Dk,Dv].

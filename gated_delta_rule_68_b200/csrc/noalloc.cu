@@ -14,11 +14,16 @@
 // loaded on a GPU and stays reserved on every GPU that loaded it until the
 // process exits. Its address is looked up once per device, with that device
 // current, on the first call made on that device; make that first call before
-// any stream capture. All calls share the one array and its contents carry
+// any stream capture. The address belongs to the context it was looked up in:
+// after a device reset (cudaDeviceReset) the next context may place the array
+// elsewhere, so the address is kept with the id of its context and looked up
+// again, on the first call after the reset, when the calling thread's current
+// context has another id. All calls share the one array and its contents carry
 // over from the previous call: every region a call reads is written earlier
 // in the same call, so nothing needs clearing, but calls that overlap in time
 // on one GPU (other streams, other threads) race on it and must be serialised
 // by the caller.
+#include <cuda.h>
 #include <stdio.h>
 
 #include <mutex>
@@ -36,7 +41,35 @@ static __device__ __align__(256) unsigned char g_scratch[GDR_NOALLOC_SCRATCH_BYT
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
+struct ScratchAddr {
+    unsigned long long ctx_id;  // id of the context the address belongs to
+    void *addr;                 // device address of g_scratch in that context
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
+
+// Id of the calling thread's current context (unique for the life of the process);
+// false when no context is current or the driver lacks the calls. The two driver calls
+// are resolved through the runtime, so the library links no driver library.
+bool current_context_id(unsigned long long *id)
+{
+    using GetCurrent = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *p1 = nullptr, *p2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess)
+            return false;
+        get_current = reinterpret_cast<GetCurrent>(p1);
+        get_id = reinterpret_cast<GetId>(p2);
+    }
+    CUcontext ctx = nullptr;
+    return get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -62,13 +95,21 @@ extern "C" int gdr_fwd_chunked_noalloc(const void *q, const void *k, const void 
         if (dev < 0 || dev >= kMaxDevices)
             return gdr::set_failure(GDR_ERR_UNSUPPORTED, "device ordinal beyond 63");
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!g_scratch_addr[dev]) {
+        ScratchAddr &sa = g_scratch_addr[dev];
+        unsigned long long id = 0;
+        if (!sa.addr || !current_context_id(&id) || id != sa.ctx_id) {
+            // First call on this device, or on a context other than the one the cached
+            // address was looked up in. The lookup makes the device's primary context
+            // current if none is.
             void *p = nullptr;
             e = cudaGetSymbolAddress(&p, g_scratch);
             if (e != cudaSuccess) return gdr::set_failure(GDR_ERR_CUDA, cudaGetErrorString(e));
-            g_scratch_addr[dev] = p;
+            if (!current_context_id(&id))
+                return gdr::set_failure(GDR_ERR_CUDA, "no current CUDA context after the scratch lookup");
+            sa.ctx_id = id;
+            sa.addr = p;
         }
-        scratch = g_scratch_addr[dev];
+        scratch = sa.addr;
     }
     return gdr_fwd_chunked(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype, scratch,
                            scratch ? (size_t)GDR_NOALLOC_SCRATCH_BYTES : 0, stream);

@@ -126,9 +126,14 @@ GDR_API int gdr_bwd(const void *q, const void *k, const void *v, const float *g,
  *                  between its warp groups) that gave up after one second; the
  *                  (batch row, value head) unit stops, so that call's o and hT
  *                  are incomplete.
- *   range_errors   chunks whose per-key-channel gate factors left the fp16
- *                  range (a decay stronger than about exp(-11) within 32
- *                  tokens); that chunk's results are not valid.
+ *   range_errors   per-channel gate (warp-level kernel): chunks whose
+ *                  per-key-channel gate factors left the fp16 range (a decay
+ *                  stronger than about exp(-11) within 32 tokens); that
+ *                  chunk's results are not valid. Scalar gate (tcgen05
+ *                  kernel): (batch row, value head) units in which a value
+ *                  rounded to an fp16 operand was inf or NaN (an input, the
+ *                  copy of the state, A, M, the inverse, W, U, P or Qh);
+ *                  that unit's o and hT are not valid.
  * Reads device memory, so it waits for prior work on the default stream.
  */
 GDR_API unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors);
@@ -147,7 +152,7 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  *
  * Computes o_t for every t in [0, T) and, if hT != NULL, the state after the
  * last token. h0 == NULL means a zero initial state. The result equals the
- * token recurrence above (exact chunkwise form; SinkProbe (Attention-Sink)
+ * token recurrence above (chunk by chunk, no approximation; SinkProbe (Attention-Sink)
  * README, description of its delta-rule layer): per 64-token chunk a UT/WY
  * transform A = tril(diag(beta)(K*Gamma)(K/Gamma)^T, -1), T = (I + A)^-1,
  * W = T diag(beta)(K*Gamma), U = T diag(beta) V, then the state scan
@@ -161,7 +166,8 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  * the masked (Q*Gamma)(K/Gamma)^T above), for the per-channel gate on the
  * warp-level tensor cores. Both use fp16 operands, fp32 accumulation and an
  * fp32 carried state; q, k, v and the state must stay inside the fp16 range,
- * |x| < 6.5e4. Other shapes and fp32 inputs run fp32 CUDA-core kernels, which
+ * |x| < 6.5e4 (both kernels count violations, see gdr_fused_error_counts;
+ * the call still returns GDR_OK). Other shapes and fp32 inputs run fp32 CUDA-core kernels, which
  * take at most 65535 batch rows (else GDR_ERR_UNSUPPORTED).
  * B == 0 or T == 0 is a valid no-op that still writes hT = h0 (or zeros).
  *
@@ -260,7 +266,9 @@ GDR_API int gdr_decode_step(const void *q, const void *k, const void *v, const f
  * on every GPU where the library's no-allocation code is loaded and stays
  * reserved until the process exits. The first call on a device looks up the
  * array's address on that device: make that first call before any stream
- * capture. Every call shares the one array and it keeps the previous call's
+ * capture. That address belongs to the device's context at the time; after a
+ * device reset (cudaDeviceReset) the first call in the new context looks it up
+ * again, so make that call before any capture too. Every call shares the one array and it keeps the previous call's
  * contents (each call writes every part it reads before reading it), so
  * calls that overlap in time on one GPU race and must be serialised by the
  * caller. Nothing here calls cudaMalloc, cudaFree or any allocating routine.

@@ -25,15 +25,22 @@ def run_fwd(inp, **kw):
 
 def full_check(w, tol=None, plain=False):
     """Every element of o and hT against the oracle. The five workloads use the plain
-    metric; smaller cases allow the bf16 rounding of o on top (rel_err_excess)."""
+    metric; smaller cases allow the bf16 rounding of o on top (rel_err_excess). bf16
+    cases are also run with an fp32 o, held to the plain metric. No call may report an
+    fp16 range error."""
     inp = make_inputs(w, DEV)
+    _, r0 = gdr.gdr_fused_error_counts()
     o, hT = run_fwd(inp)
+    o32 = run_fwd(inp, out_dtype=torch.float32)[0] if w.dtype == "bf16" else o
     torch.cuda.synchronize()
+    _, r1 = gdr.gdr_fused_error_counts()
+    assert r1 == r0, (w, r1 - r0)
     o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
     tol = tol or TOL[w.dtype]
     eo = rel_err(o, o_ref) if plain else rel_err_excess(o, o_ref, w.dtype)
+    eo32 = rel_err(o32, o_ref)
     es = rel_err(hT, s_ref)
-    assert eo <= tol and es <= tol, (w, eo, es)
+    assert eo <= tol and eo32 <= tol and es <= tol, (w, eo, eo32, es)
     return eo, es
 
 
@@ -168,9 +175,13 @@ def test_full_workload_sampled(name, n_units):
     w = WORKLOADS[name]
     inp_cpu = make_inputs(w, "cpu")
     inp = {n: (None if t is None else t.to(DEV)) for n, t in inp_cpu.items()}
+    torch.cuda.synchronize()
+    _, r0 = gdr.gdr_fused_error_counts()
     o16, hT16 = run_fwd(inp)
     o32, hT = run_fwd(inp, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    _, r1 = gdr.gdr_fused_error_counts()
+    assert r1 == r0, (name, r1 - r0)   # no unit or chunk left the fp16 range
     assert o16.dtype == torch.bfloat16 and torch.equal(o16, o32.to(torch.bfloat16))
     assert torch.equal(hT16, hT)
     units = sample_units(w.B, w.Hv, n_units, seed=w.seed)
@@ -240,7 +251,9 @@ def test_decode_equals_chunked_forward():
 
 
 def test_zz_fused_kernel_reported_no_load_timeouts():
-    """Runs after the other tests in this file: no chunk load ever timed out."""
+    """Runs after the other tests in this file: no chunk load ever timed out, and the only
+    range errors are the one that test_strong_channel_decay_is_reported_not_hidden plants."""
     torch.cuda.synchronize()
-    timeouts, _ = gdr.gdr_fused_error_counts()
+    timeouts, ranges = gdr.gdr_fused_error_counts()
     assert timeouts == 0
+    assert ranges <= 1

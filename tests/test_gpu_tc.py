@@ -25,13 +25,23 @@ def run_fwd(inp, **kw):
 
 
 def check_all(w, out_dtype=None):
+    """Every element against the oracle. A bf16-o call is also repeated with an fp32 o,
+    which must meet the plain bound (no allowance for rounding o to bf16) and round to
+    the bf16 o bit for bit; neither call may report an fp16 range error."""
     inp = make_inputs(w, DEV)
+    _, r0 = gdr.gdr_fused_error_counts()
     o, hT = run_fwd(inp, **({} if out_dtype is None else {"out_dtype": out_dtype}))
+    o32, hT32 = (o, hT) if out_dtype == torch.float32 else run_fwd(inp, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    _, r1 = gdr.gdr_fused_error_counts()
+    assert r1 == r0
     o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
     eo = rel_err(o, o_ref) if out_dtype == torch.float32 else rel_err_excess(o, o_ref, "bf16")
+    eo32 = rel_err(o32, o_ref)
     es = rel_err(hT, s_ref)
-    assert eo <= TOL["bf16"] and es <= TOL["bf16"], (w, eo, es)
+    assert eo <= TOL["bf16"] and eo32 <= TOL["bf16"] and es <= TOL["bf16"], (w, eo, eo32, es)
+    if out_dtype != torch.float32:
+        assert torch.equal(o, o32.to(torch.bfloat16)) and torch.equal(hT, hT32)
     return inp, o, hT
 
 
@@ -97,3 +107,48 @@ def test_repeated_calls_are_bitwise_identical():
     o2, h2 = run_fwd(inp)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def _growing_state_inputs(v_scale, T=320, seed=800):
+    """g = 0 and beta = 1 with v scaled up (kept inside fp16's range): the state grows
+    with the sequence, to about 7.5e4 by token 192 at v_scale = 2e4."""
+    w = WORKLOADS["gdn_bf16"].with_(B=1, T=T, Hk=1, Hv=1, seed=seed)
+    inp = make_inputs(w, DEV)
+    inp["g"] = torch.zeros_like(inp["g"])
+    inp["beta"] = torch.ones_like(inp["beta"])
+    inp["v"] = (inp["v"].float() * v_scale).clamp(-6e4, 6e4).to(torch.bfloat16)
+    return inp
+
+
+def test_state_past_fp16_range_is_counted():
+    """A state that outgrows fp16 (its copy is an operand of the next chunk's products)
+    makes the call count one range error for its unit; the call itself still succeeds."""
+    inp = _growing_state_inputs(2e4)
+    _, before = gdr.gdr_fused_error_counts()
+    run_fwd(inp)
+    torch.cuda.synchronize()
+    _, after = gdr.gdr_fused_error_counts()
+    assert after == before + 1
+
+
+def test_initial_state_past_fp16_range_is_counted():
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=70, Hk=1, Hv=2, seed=801)
+    inp = make_inputs(w, DEV)
+    inp["h0"][1, 0, 3, 5] = 1e5   # one unit: batch row 1, value head 0
+    _, before = gdr.gdr_fused_error_counts()
+    run_fwd(inp)
+    torch.cuda.synchronize()
+    _, after = gdr.gdr_fused_error_counts()
+    assert after == before + 1
+
+
+def test_large_values_inside_fp16_range_are_not_counted():
+    """The same growth with v 20 times smaller stays inside fp16 and meets the tolerance."""
+    inp = _growing_state_inputs(1e3)
+    _, before = gdr.gdr_fused_error_counts()
+    o, hT = run_fwd(inp, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _, after = gdr.gdr_fused_error_counts()
+    assert after == before
+    o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
+    assert rel_err(o, o_ref) <= TOL["bf16"] and rel_err(hT, s_ref) <= TOL["bf16"]
