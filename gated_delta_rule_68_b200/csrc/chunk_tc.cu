@@ -126,26 +126,22 @@ constexpr uint32_t ID_O = idesc_f16(128, 64, false, false, true);
 __device__ unsigned int g_tc_timeouts;
 __device__ unsigned int g_tc_range_errors;
 
-// Values of magnitude 65520 and above round to inf in fp16. Each stage that rounds values
-// to fp16 operands takes their largest |x| and raises the CTA's flag if it is out of range
-// (a NaN can only follow an earlier overflow or a non-finite input, and inputs are checked
-// on their fp16 bits).
-__device__ __forceinline__ float amax_n(const float *x, int n)
+// Range: an fp16 operand that overflowed (or an inf/NaN input) cannot come out of a tensor-core
+// product as a finite value (inf * 0 is NaN, inf + x is inf), and every product feeds either
+// the state or o. So a unit whose fp16 operands left the range ends with a non-finite o or
+// final state: those are checked (x * 0 is 0 for finite x and NaN otherwise), cheaply and off
+// the chunk group's path, and the CTA's flag is raised.
+__device__ __forceinline__ bool any_nonfinite32(const float *x)
 {
-    float m = 0.f;
+    float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
 #pragma unroll
-    for (int i = 0; i < n; ++i) m = fmaxf(m, fabsf(x[i]));
-    return m;
-}
-__device__ __forceinline__ void flag_range(int *flag, float m)
-{
-    if (!(m < 65520.f)) *reinterpret_cast<volatile int *>(flag) = 1;
-}
-// Bit 15 (31) of the result is set when the low (high) half of a packed fp16 pair is inf or NaN.
-__device__ __forceinline__ uint32_t f16x8_bad(uint4 u)
-{
-    constexpr uint32_t E = 0x7c007c00u, C1 = 0x04000400u;
-    return ((u.x & E) + C1) | ((u.y & E) + C1) | ((u.z & E) + C1) | ((u.w & E) + C1);
+    for (int i = 0; i < 32; i += 4) {
+        z0 = fmaf(x[i], 0.f, z0);
+        z1 = fmaf(x[i + 1], 0.f, z1);
+        z2 = fmaf(x[i + 2], 0.f, z2);
+        z3 = fmaf(x[i + 3], 0.f, z3);
+    }
+    return (z0 + z1) + (z2 + z3) != 0.f;
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float x, float y)
@@ -225,12 +221,24 @@ __device__ __forceinline__ void chain_next(float c0[4], float c1[4], uint32_t aB
     mma16r(c0, c1, af, aB, ldb, lane);
 }
 
+// c (16 x 16, two n8 accumulator tiles) (+)= A B, A given by its A fragment and B by the A
+// fragment of B^T: the B fragment of columns 8 nt .. 8 nt + 7 of B is registers nt and nt + 2
+// of that fragment.
+__device__ __forceinline__ void mma16_ff(float c[2][4], const uint32_t a[4], const uint32_t bt[4], bool acc)
+{
+    if (!acc) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[0][e] = c[1][e] = 0.f;
+    }
+    mma(c[0], a, bt[0], bt[2]);
+    mma(c[1], a, bt[1], bt[3]);
+}
+
 // Writes block (R0.., I0..) of T, given as two n8 tiles times `s`, into T diag(beta Gamma)
 // and T diag(beta) (swizzled [r][i] tiles).
 __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const float c0[4], const float c1[4], float s,
-                                          const float *vec, int lane, int *range_flag)
+                                          const float *vec, int lane)
 {
-    float m = 0.f;
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -238,13 +246,11 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = R0 + g + 8 * (e >> 1), i = I0 + 8 * nt + 2 * t4 + (e & 1);
-            const float t = s * c[e], t1 = t * vec[V_BG + i], t2 = t * vec[V_BETA + i];
-            m = fmaxf(m, fmaxf(fabsf(t1), fabsf(t2)));
-            st_h1(sm, OFF_TP + swz_off(r, i, 0), t1);
-            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t2);
+            const float t = s * c[e];
+            st_h1(sm, OFF_TP + swz_off(r, i, 0), t * vec[V_BG + i]);
+            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t * vec[V_BETA + i]);
         }
     }
-    flag_range(range_flag, m);
 }
 
 // NORM: the layer's options (compiled as a separate instance, so the plain forward runs
@@ -264,7 +270,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     __shared__ uint64_t bars[NBAR];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
-    __shared__ int range_sh;   // set when a value rounded to an fp16 operand is out of range
+    __shared__ int range_sh;   // set when this unit's o or final state came out non-finite
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -342,7 +348,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     v[i + 2] = i + 2 < lim ? rowf * e.z * v[i + 2] : 0.f;
                     v[i + 3] = i + 3 < lim ? rowf * e.w * v[i + 3] : 0.f;
                 }
-                flag_range(&range_sh, amax_n(v, 32));
                 // The previous chunk's first products are done with M and U^T (the inverse's scratch).
                 if (c >= 1) wait(B_P1, (c - 1) & 1);
                 if (p >= 64) {
@@ -372,40 +377,67 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             // ... and with W^T (the tiles of T) before they are rewritten.
             if (c >= 1) wait(B_P, (c - 1) & 1);
             // Inverse, level 0: warp wq of the first half inverts the unit lower 16 x 16 block
-            // I + A_bb (b = wq) by forward substitution (lanes j and j + 16 both hold column j,
-            // so that the 48 stores per column split evenly: lanes 0-15 write D_b and rows 0-7
-            // of T', lanes 16-31 write T'' and rows 8-15 of T'); the second half zeroes the
-            // blocks of T above the diagonal.
+            // I + N (N = A_bb, b = wq) in the product form
+            //   (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8)      (N^16 = 0)
+            // on the warp-level tensor cores, with the running product carried in fp32. Each
+            // power is kept with its transpose: the accumulator of X is the A fragment of X, and
+            // the B fragment of X regroups the A fragment of X^T, so no product needs a
+            // shared-memory round trip. D_b, the b-th diagonal blocks of T diag(beta Gamma) and
+            // T diag(beta) go out as fp16 pairs. The second half zeroes the blocks of T above
+            // the diagonal.
             if (hf == 0) {
-                const int j = lane & 15;
-                const bool lo = lane < 16;
-                float t[16];
+                const int g8 = lane >> 2, t4 = lane & 3;
+                const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;   // ad[i][r] = N[r][i]
+                float n[2][4], nt[2][4];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) t[rr] = rr == j ? 1.f : 0.f;
-                const float *ad = reinterpret_cast<const float *>(sm + INV_AD) + wq * 16 * LDAD;
+                for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                for (int i = 0; i < 15; ++i) {
-                    float col[16];
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const float4 x = *reinterpret_cast<const float4 *>(ad + i * LDAD + 4 * k4);
-                        col[4 * k4] = x.x, col[4 * k4 + 1] = x.y, col[4 * k4 + 2] = x.z, col[4 * k4 + 3] = x.w;
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = g8 + 8 * (e >> 1), col = 8 * tt + 2 * t4 + (e & 1);
+                        n[tt][e] = ad[col * LDAD + r];    // N[r][col]
+                        nt[tt][e] = ad[r * LDAD + col];   // N^T[r][col]
                     }
-                    const float ti = t[i];
+                uint32_t aN[4], aNT[4], aP2[4], aP2T[4], aP4[4], aP4T[4], aP8T[4], ax[4];
+                acc_to_a(aN, n[0], n[1]);
+                acc_to_a(aNT, nt[0], nt[1]);
+                float p[2][4], pt[2][4];
+                mma16_ff(p, aN, aNT, false);       // N^2
+                mma16_ff(pt, aNT, aN, false);      // (N^2)^T
+                acc_to_a(aP2, p[0], p[1]);
+                acc_to_a(aP2T, pt[0], pt[1]);
+                mma16_ff(p, aP2, aP2T, false);     // N^4
+                mma16_ff(pt, aP2T, aP2, false);    // (N^4)^T
+                acc_to_a(aP4, p[0], p[1]);
+                acc_to_a(aP4T, pt[0], pt[1]);
+                mma16_ff(pt, aP4T, aP4, false);    // (N^8)^T
+                acc_to_a(aP8T, pt[0], pt[1]);
+                float x[2][4];                     // X = I - N, then X <- X + X N^(2^j)
 #pragma unroll
-                    for (int rr = i + 1; rr < 16; ++rr) t[rr] = fmaf(-col[rr], ti, t[rr]);
-                }
-                const int I = 16 * wq + j;
-                const float sbg = vc[V_BG + I], sbt = vc[V_BETA + I];
-                flag_range(&range_sh, amax_n(t, 16) * fmaxf(1.f, fmaxf(fabsf(sbg), fabsf(sbt))));
-                const uint32_t dd0 = INV_D + (uint32_t)(wq * 16 * LDT16 + j) * 2u;
+                for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr)   // D_b row rr (lanes 0-15), T'' row rr (lanes 16-31)
-                    st_h1(sm, lo ? dd0 + (uint32_t)(rr * LDT16) * 2u : OFF_TPP + swz_off(16 * wq + rr, I, 0),
-                          lo ? t[rr] : t[rr] * sbt);
+                    for (int e = 0; e < 4; ++e)
+                        x[tt][e] = ((g8 + 8 * (e >> 1)) == (8 * tt + 2 * t4 + (e & 1)) ? 1.f : 0.f) - n[tt][e];
+                acc_to_a(ax, x[0], x[1]);
+                mma16_ff(x, ax, aP2T, true);
+                acc_to_a(ax, x[0], x[1]);
+                mma16_ff(x, ax, aP4T, true);
+                acc_to_a(ax, x[0], x[1]);
+                mma16_ff(x, ax, aP8T, true);
+                // x[tt][2h], x[tt][2h + 1] = D_b[r][col], D_b[r][col + 1]: r = g8 + 8h, col = 8tt + 2t4
+                const int I0 = 16 * wq;
 #pragma unroll
-                for (int rr = 0; rr < 8; ++rr)    // T' row rr (lanes 0-15), row rr + 8 (lanes 16-31)
-                    st_h1(sm, OFF_TP + swz_off(16 * wq + (lo ? rr : rr + 8), I, 0), (lo ? t[rr] : t[rr + 8]) * sbg);
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = g8 + 8 * hh, col = 8 * tt + 2 * t4, i = I0 + col;
+                        const float x0 = x[tt][2 * hh], x1 = x[tt][2 * hh + 1];
+                        const float u0 = x0 * vc[V_BG + i], u1 = x1 * vc[V_BG + i + 1];
+                        const float w0 = x0 * vc[V_BETA + i], w1 = x1 * vc[V_BETA + i + 1];
+                        *reinterpret_cast<uint32_t *>(sm + INV_D + (uint32_t)((wq * 16 + r) * LDT16 + col) * 2u) =
+                            pack_h2(x0, x1);
+                        *reinterpret_cast<uint32_t *>(sm + OFF_TP + swz_off(I0 + r, i, 0)) = pack_h2(u0, u1);
+                        *reinterpret_cast<uint32_t *>(sm + OFF_TPP + swz_off(I0 + r, i, 0)) = pack_h2(w0, w1);
+                    }
             } else {
                 // zero chunks: row u of block R = u / 16, 16-byte chunks 2(R+1) .. 7, of one of the two tiles
                 const int u = (gt - GT / 2) & 63, R = u >> 4;
@@ -433,14 +465,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 if (wq == 0) {
                     chain_start(c0, c1, Dt(1), LDT16, At(1, 0), LDA16, lane);
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 16, 0, c0, c1, -1.f, vc, lane, &range_sh);
+                    st_tblock(sm, 16, 0, c0, c1, -1.f, vc, lane);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
-                    st_tblock(sm, 32, 16, c0, c1, -1.f, vc, lane, &range_sh);
+                    st_tblock(sm, 32, 16, c0, c1, -1.f, vc, lane);
                 } else if (wq == 1) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
-                    st_tblock(sm, 48, 32, c0, c1, -1.f, vc, lane, &range_sh);
+                    st_tblock(sm, 48, 32, c0, c1, -1.f, vc, lane);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
                     chain_next(c0, c1, At(1, 0), LDA16, lane);
@@ -448,7 +480,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 32, 0, c0, c1, 1.f, vc, lane, &range_sh);
+                    st_tblock(sm, 32, 0, c0, c1, 1.f, vc, lane);
                 } else if (wq == 2) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
@@ -457,7 +489,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(1), LDT16, lane);
-                    st_tblock(sm, 48, 16, c0, c1, 1.f, vc, lane, &range_sh);
+                    st_tblock(sm, 48, 16, c0, c1, 1.f, vc, lane);
                 } else {
                     float q0[4], q1[4], h0[4], h1[4];
                     chain_start(q0, q1, Dt(3), LDT16, At(3, 2), LDA16, lane);   // Q = D3 A32 D2
@@ -475,7 +507,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] = u0[e] + h0[e] - c0[e], c1[e] = u1[e] + h1[e] - c1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 48, 0, c0, c1, 1.f, vc, lane, &range_sh);
+                    st_tblock(sm, 48, 0, c0, c1, 1.f, vc, lane);
                 }
             }
             fence_proxy_async();
@@ -503,7 +535,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 32 * hf), tmem_addr(tb, q4, TM_Y + 64 + 32 * hf), v);
-                flag_range(&range_sh, amax_n(v, 64));
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_W16), v + 8 * j);
 #pragma unroll
@@ -611,7 +642,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             float *vs = vec + sb * V_SET;
             wait(B_LD0 + sb, (c >> 1) & 1);
             const int nvalid = min(C, T - c * C);
-            uint32_t rin = 0;   // fp16 inf/NaN bits of the converted inputs
             if (NORM && a.qk_l2norm) {
                 // [K; Q] rows: chunks e and e + 1024 are the two halves of one row, and a row's 8
                 // chunks of a half sit in 8 adjacent threads
@@ -625,19 +655,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
                     ss += __shfl_xor_sync(0xffffffffu, ss, 4);
                     const float sc = rsqrtf(ss + 1e-6f);
-                    const uint4 h0v = row < nvalid ? bf16x8_scaled_f16x8(u0, sc) : make_uint4(0, 0, 0, 0);
-                    const uint4 h1v = row < nvalid ? bf16x8_scaled_f16x8(u1, sc) : make_uint4(0, 0, 0, 0);
-                    rin |= f16x8_bad(h0v) | f16x8_bad(h1v);
-                    *p0 = h0v;
-                    *p1 = h1v;
+                    *p0 = row < nvalid ? bf16x8_scaled_f16x8(u0, sc) : make_uint4(0, 0, 0, 0);
+                    *p1 = row < nvalid ? bf16x8_scaled_f16x8(u1, sc) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
                 for (int j = 8; j < 3072 / GT; ++j) {
                     const int e = tid + GT * j, row = ((e - 2048) >> 3) & 63;
                     uint4 *pch = reinterpret_cast<uint4 *>(stgp) + e;
-                    const uint4 hv = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
-                    rin |= f16x8_bad(hv);
-                    *pch = hv;
+                    *pch = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
                 }
             } else {
                 // all chunks of [K; Q] (2 atoms of 128 rows, Q from row 64) and V (2 atoms of 64
@@ -651,13 +676,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int j = 0; j < 4; ++j) {
                         const int e = tid + GT * (j0 + j);
                         const int row = e < 2048 ? ((e >> 3) & 127) & 63 : ((e - 2048) >> 3) & 63;
-                        const uint4 hv = row < nvalid ? bf16x8_to_f16x8(u[j]) : make_uint4(0, 0, 0, 0);
-                        rin |= f16x8_bad(hv);
-                        reinterpret_cast<uint4 *>(stgp)[e] = hv;
+                        reinterpret_cast<uint4 *>(stgp)[e] = row < nvalid ? bf16x8_to_f16x8(u[j]) : make_uint4(0, 0, 0, 0);
                     }
                 }
             }
-            if (rin & 0x80008000u) *reinterpret_cast<volatile int *>(&range_sh) = 1;
             fence_proxy_async();
             named_bar_sync(2, GT);   // every tile of the chunk converted
             if (gissuer) {
@@ -718,7 +740,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + (size_t)(64 * hf) * D + p : nullptr;
 #pragma unroll
             for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
-            flag_range(&range_sh, amax_n(S, 64));
 #pragma unroll
             for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
         }
@@ -748,7 +769,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[32];
                 tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
-                flag_range(&range_sh, amax_n(v, 32));
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
             }
@@ -759,7 +779,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 64 * hf), tmem_addr(tb, q4, TM_Y + 64 * hf + 32), v);
-                flag_range(&range_sh, amax_n(v, 64));
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
             }
@@ -792,7 +811,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tmem_ld32x2(tmem_addr(tb, q4, TM_S + 64 * hf), tmem_addr(tb, q4, TM_S + 64 * hf + 32), v);
 #pragma unroll
                 for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
-                flag_range(&range_sh, amax_n(S, 64));
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
             }
@@ -816,6 +834,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     tc_fence_before();
                     mbar_arrive(bar(B_SE));
                     mbar_arrive(bar(B_OE));
+                    if (any_nonfinite32(o)) *reinterpret_cast<volatile int *>(&range_sh) = 1;
                     const uint32_t byte = (uint32_t)(p & 31) * 4u;
                     uint8_t *base = sm + OFF_P16 + (p >> 5) * C * 128 + (32 * hf) * 128 + (byte & 15);
                     uint32_t xo[8];
@@ -882,6 +901,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tc_fence_before();
                 mbar_arrive(bar(B_SE));
                 mbar_arrive(bar(B_OE));
+                float z = 0.f;   // x * 0 is 0 for finite x, NaN otherwise
                 if (tile) {
                     constexpr int EPB = 128 / sizeof(TOut);
                     const uint32_t byte = (uint32_t)(p % EPB) * sizeof(TOut);
@@ -890,7 +910,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int s8 = 0; s8 < 8; ++s8) xo[s8] = ((byte >> 4) ^ s8) << 4;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) out_store1(reinterpret_cast<TOut *>(base + i * 128 + xo[i & 7]), o[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        out_store1(reinterpret_cast<TOut *>(base + i * 128 + xo[i & 7]), o[i]);
+                        z = fmaf(o[i], 0.f, z);
+                    }
                     fence_proxy_async();
                 } else {
                     const int nv = nvalid - 32 * hf, odd = p & 1;
@@ -901,8 +924,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int i = 0; i < 32; i += 2) {
                         const float other = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + 1], 1);
                         if (i + odd < nv) out_store2(orow + (size_t)i * rs, odd ? other : o[i], odd ? o[i + 1] : other);
+                        z = fmaf(o[i], 0.f, fmaf(o[i + 1], 0.f, z));
                     }
                 }
+                if (z != 0.f) *reinterpret_cast<volatile int *>(&range_sh) = 1;
             }
             named_bar_sync(2, GT);
             if (issuer && tile) {
@@ -918,6 +943,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             named_bar_sync(2, GT);
         }
         if (issuer) tma_store_wait_all();
+        if (any_nonfinite32(S) || any_nonfinite32(S + 32)) *reinterpret_cast<volatile int *>(&range_sh) = 1;
         if (a.hT) {
             float *hp = a.hT + (size_t)bh * D * D + (size_t)(64 * hf) * D + p;
 #pragma unroll

@@ -75,6 +75,16 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, 
                  ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)acc)
                  : "memory");
 }
+// D[tmem] (+)= A[tmem] B[smem] for one K = 16 step: A is 128 lanes (its rows) of 16-bit
+// elements packed two per 32-bit column, element k in the low half of column k / 2 when
+// k is even; one step reads 8 columns from a_tmem.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, bool acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"((uint32_t)acc)
+                 : "memory");
+}
 // Arrive once on the mbarrier when every MMA this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
@@ -119,6 +129,21 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t a0, uint32_t a1, float v[64
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// 32 consecutive 32-bit columns of this thread's lane (32x32b shape), from registers;
+// tmem_wait_st() waits until this thread's stores have landed.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t v[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+                   "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+                   "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+                   "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Plain arrival of this thread on an mbarrier.
 __device__ __forceinline__ void mbar_arrive(uint32_t bar)

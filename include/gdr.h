@@ -130,10 +130,12 @@ GDR_API int gdr_bwd(const void *q, const void *k, const void *v, const float *g,
  *                  per-key-channel gate factors left the fp16 range (a decay
  *                  stronger than about exp(-11) within 32 tokens); that
  *                  chunk's results are not valid. Scalar gate (tcgen05
- *                  kernel): (batch row, value head) units in which a value
- *                  rounded to an fp16 operand was inf or NaN (an input, the
- *                  copy of the state, A, M, the inverse, W, U, P or Qh);
- *                  that unit's o and hT are not valid.
+ *                  kernel): (batch row, value head) units whose o or final
+ *                  state came out inf or NaN. That happens when a value
+ *                  rounded to an fp16 operand overflowed (the copy of the
+ *                  state, A, M, the inverse, W, U, P, Qh), since a product
+ *                  of an inf operand is never finite, or when an input was
+ *                  inf or NaN; that unit's o and hT are not valid.
  * Reads device memory, so it waits for prior work on the default stream.
  */
 GDR_API unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors);

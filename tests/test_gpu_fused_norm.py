@@ -124,3 +124,16 @@ def test_fused_norms_full_workload_sampled(name):
         og = prologue.rmsnorm_gated(o_ref[i], inp["z"][b, :, h], inp["nw"])
         assert rel_err(o[b, :, h].float(), og) <= TOL["bf16"] + 2.0 ** -8 * np.max(np.abs(og)) / np.sqrt(np.mean(og ** 2))
         assert rel_err(hT[b, h], s_ref[i]) <= TOL["bf16"]
+
+
+def test_warp_level_kernel_mixed_launch_with_channel_gate():
+    """The per-channel gate with the layer's options runs the warp-level kernel. With 160
+    (batch row, value head) units on a 148-SM B200 its launch mixes whole units and units
+    split over two CTAs by value columns; every unit is checked."""
+    w = WORKLOADS["gdn_bf16"].with_(B=10, T=130, Hk=16, Hv=16, gate="channel", g_mu=4.0, seed=77)
+    inp = layer_inputs(w, DEV, scale_qk=True)
+    o, hT = run(inp, True, False)
+    torch.cuda.synchronize()
+    o_ref, s_ref = reference(inp, True, False)
+    eo, es = rel_err(o, o_ref), rel_err(hT, s_ref)
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"], (eo, es)

@@ -136,8 +136,7 @@ def test_bad_workspace_raises():
 
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
 def test_one_cta_per_unit_when_units_fill_the_sms(gate):
-    """80 (batch row, value head) units: too many to split the value columns over two CTAs
-    per unit in one wave, so each unit gets one CTA (the small cases above get two)."""
+    """80 (batch row, value head) units, one CTA each on the tcgen05 kernel (either gate)."""
     w = WORKLOADS["gdn_bf16"].with_(B=5, T=130, Hk=16, Hv=16, gate=gate,
                                     g_mu=4.0 if gate == "channel" else 3.0, seed=21)
     full_check(w)
@@ -145,8 +144,9 @@ def test_one_cta_per_unit_when_units_fill_the_sms(gate):
 
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
 def test_units_past_one_wave_are_split_in_halves(gate):
-    """160 units on a 148-SM B200: the first 148 run whole, each of the last 12 is split
-    over two CTAs by value columns (one launch, both kinds of CTA). Every unit is checked."""
+    """160 units on a 148-SM B200: more CTAs than SMs, so a second wave of CTAs. Every unit
+    is checked. (The warp-level kernel's mixed whole/split launch is covered in
+    test_gpu_fused_norm.py.)"""
     w = WORKLOADS["gdn_bf16"].with_(B=10, T=130, Hk=16, Hv=16, gate=gate,
                                     g_mu=4.0 if gate == "channel" else 3.0, seed=23)
     full_check(w)
@@ -251,9 +251,8 @@ def test_decode_equals_chunked_forward():
 
 
 def test_zz_fused_kernel_reported_no_load_timeouts():
-    """Runs after the other tests in this file: no chunk load ever timed out, and the only
-    range errors are the one that test_strong_channel_decay_is_reported_not_hidden plants."""
+    """Runs after the other tests in this file: no chunk load ever timed out. (Range errors
+    are checked call by call: tests elsewhere plant some on purpose.)"""
     torch.cuda.synchronize()
-    timeouts, ranges = gdr.gdr_fused_error_counts()
+    timeouts, _ = gdr.gdr_fused_error_counts()
     assert timeouts == 0
-    assert ranges <= 1

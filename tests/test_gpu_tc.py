@@ -152,3 +152,28 @@ def test_large_values_inside_fp16_range_are_not_counted():
     assert after == before
     o_ref, s_ref = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
     assert rel_err(o, o_ref) <= TOL["bf16"] and rel_err(hT, s_ref) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ per-channel gate (KDA)
+@pytest.mark.parametrize("T", [1, 31, 32, 63, 64, 65, 191])
+def test_channel_gate_chunk_boundaries_grouped_heads(T):
+    """The per-channel gate on the tcgen05 kernel: partial chunks on both sides of the
+    in-chunk reference row 31, three value heads per key head."""
+    check_all(WORKLOADS["kda_bf16"].with_(B=2, T=T, Hk=2, Hv=6, seed=900 + T))
+
+
+@pytest.mark.parametrize("g_mu", [2.0, 8.0])
+def test_channel_gate_strong_and_weak_decay(g_mu):
+    """g = logsigmoid(N(mu, 1)) per key channel: mu = 2 decays by about e^-4 per 32 tokens
+    (the factors exp(+-(G - G_31)) stay inside fp16), mu = 8 barely decays at all."""
+    check_all(WORKLOADS["kda_bf16"].with_(B=2, T=300, Hk=2, Hv=4, g_mu=g_mu, seed=950 + int(g_mu)),
+              out_dtype=torch.float32)
+
+
+def test_channel_gate_repeated_calls_are_bitwise_identical():
+    w = WORKLOADS["kda_bf16"].with_(B=2, T=333, Hk=2, Hv=4, seed=990)
+    inp = make_inputs(w, DEV)
+    o1, h1 = run_fwd(inp)
+    o2, h2 = run_fwd(inp)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
