@@ -32,10 +32,25 @@
 // the other chunk-local work overlap the state chain, and the state chain of a
 // chunk is one MMA batch and two short epilogues.
 //
+// Per-channel gate (Kimi Delta Attention, "Linear attention", row kda; GATE = 1): G
+// and Gamma are per key channel, so the decays no longer factor out of the Gram into
+// row and column scalings. Instead the Gram's operands carry them, relative to the
+// chunk's row 31 so that each factor spans at most 32 tokens of decay:
+//   Ks = K * exp(G - G_31), Qs = Q * exp(G - G_31), Kb = K * exp(G_31 - G),
+//   A = tril(diag(beta) Ks Kb^T, -1),  M = tril(Qs Kb^T, 0),  T'' = T diag(beta),
+//   W' = T'' Ks (W = W' diag(exp G_31)),  U = T'' V,  Kt = Kb diag(exp(G_C - G_31)),
+//   P = -Kt^T W' diag(exp G_31),  R = Kt^T U,  Qh = diag(exp G_31) (Qs - M W')^T ... ^T,
+//   S_next = diag(Gamma_C) S + P S + R.
+// The column factor of P and the row factor of Qh^T are applied as the state group
+// copies them out of tensor memory, and diag(Gamma_C) in its fp32 update. The fp16
+// copy of S then lives in tensor memory (the state products read it as their A
+// operand there), which frees the shared memory for two Kb tiles.
+//
 // Precision: products take fp16 operands (bf16 inputs convert exactly inside
 // fp16's normal range) with fp32 accumulation; the state carry Gamma_C S is fp32
 // and only its product with P uses the fp16 copy of S. q, k, v and the state
-// must stay inside the fp16 range (|x| < 6.5e4).
+// must stay inside the fp16 range (|x| < 6.5e4), and with the per-channel gate
+// each factor exp(+-(G - G_31)) too; a unit whose results come out non-finite is counted.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -90,8 +105,17 @@ constexpr uint32_t SMEM_TC = SMEM_USED + 1024;
 static_assert(SMEM_TC <= 227 * 1024, "shared memory");
 
 // Tensor memory columns (512 allocated): the state product (R, then P S + R), the
-// o accumulator (Uh, then Qh S + Uh), the Gram, Qh^T, and W^T / U^T, then P.
-constexpr uint32_t TM_S = 0, TM_O = 128, TM_G = 192, TM_X = 256, TM_Y = 320;
+// o accumulator (Uh, then Qh S + Uh), the Gram, Qh^T, and W^T / U^T, then P;
+// per-channel gate: the fp16 copy of S^T (128 lanes x 128 fp16, two per column).
+constexpr uint32_t TM_S = 0, TM_O = 128, TM_G = 192, TM_X = 256, TM_Y = 320, TM_S16 = 448;
+
+// Per-channel gate: the S^T region holds the Kb tiles of the two staging buffers
+// ([64][128] fp16, two 64-column atoms of 8 KB each), and the vector region per chunk
+// parity: beta [64], exp(G_31) [128], Gamma_C [128], exp(G_C - G_31) [128]; then the
+// gate pass's per-row-group channel sums [4][128].
+constexpr uint32_t OFF_KB = OFF_ST16;
+constexpr int KV_BETA = 0, KV_E31 = 64, KV_GC = 192, KV_ECM = 320, KV_SET = 448, KV_TOT = 2 * KV_SET;
+static_assert(OFF_VEC + (KV_TOT + 4 * 128) * 4 <= SMEM_USED, "per-channel vectors must fit the vector region");
 
 // mbarriers
 enum {
@@ -171,6 +195,10 @@ __device__ __forceinline__ void prefetch_l1(const void *p)
 {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void out_store1(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void out_store2(float *p, float x, float y) { *reinterpret_cast<float2 *>(p) = make_float2(x, y); }
 __device__ __forceinline__ void out_store2(__nv_bfloat16 *p, float x, float y)
@@ -235,7 +263,8 @@ __device__ __forceinline__ void mma16_ff(float c[2][4], const uint32_t a[4], con
 }
 
 // Writes block (R0.., I0..) of T, given as two n8 tiles times `s`, into T diag(beta Gamma)
-// and T diag(beta) (swizzled [r][i] tiles).
+// and T diag(beta) (swizzled [r][i] tiles); per-channel gate: T diag(beta) only.
+template <int GATE>
 __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const float c0[4], const float c1[4], float s,
                                           const float *vec, int lane)
 {
@@ -247,8 +276,8 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
         for (int e = 0; e < 4; ++e) {
             const int r = R0 + g + 8 * (e >> 1), i = I0 + 8 * nt + 2 * t4 + (e & 1);
             const float t = s * c[e];
-            st_h1(sm, OFF_TP + swz_off(r, i, 0), t * vec[V_BG + i]);
-            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t * vec[V_BETA + i]);
+            if (GATE == 0) st_h1(sm, OFF_TP + swz_off(r, i, 0), t * vec[V_BG + i]);
+            st_h1(sm, OFF_TPP + swz_off(r, i, 0), t * vec[GATE ? KV_BETA + i : V_BETA + i]);
         }
     }
 }
@@ -256,7 +285,7 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
 // NORM: the layer's options (compiled as a separate instance, so the plain forward runs
 // exactly its own code): q and k rows divided by sqrt(sum of squares + 1e-6) as they are
 // converted, and o rows replaced by o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
-template <typename TOut, bool NORM>
+template <typename TOut, bool NORM, int GATE>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
@@ -289,6 +318,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
     }
     const int NC = (T + C - 1) / C;
+    constexpr int VSET = GATE ? KV_SET : V_SET;   // floats per chunk-parity set of vectors
+    static_assert(!(GATE && NORM), "the layer options run on the warp-level kernel with the per-channel gate");
 
     if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), 512);
     if (NORM && a.z && tid < D) reinterpret_cast<float *>(sm + OFF_NW)[tid] = a.norm_w[tid];
@@ -324,7 +355,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             const int sb = c & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES;
             uint8_t *stgp = sm + sb * STG_BYTES;
-            const float *vc = vec + sb * V_SET;
+            const float *vc = vec + sb * VSET;
             wait(B_CV0 + sb, (c >> 1) & 1);
             // Gram epilogue: A (rows < 64) and M (rows 64..127), columns 32 hf .. 32 hf + 31
             wait(B_G0 + sb, (c >> 1) & 1);
@@ -334,19 +365,25 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tmem_ld32(tmem_addr(tb, q4, TM_G + 32 * hf), v);
                 tc_fence_before();
                 mbar_arrive(bar(B_GE));
-                // exp(G_r - G_i) = exp(G_r - G_16R) exp(G_16R - G_i), R = r / 16
                 const int r = p & 63, rb = r >> 4;
-                const float4 *ec4 = reinterpret_cast<const float4 *>(vc + V_ECOL + rb * 64 + 32 * hf);
-                const float rowf = p < 64 ? vc[V_BETA + r] * vc[V_EROW + r] : vc[V_EROW + r];
                 const int lim = (p < 64 ? r : r + 1) - 32 * hf;   // A: i < r;  M: i <= r
+                if (GATE == 0) {
+                    // exp(G_r - G_i) = exp(G_r - G_16R) exp(G_16R - G_i), R = r / 16
+                    const float4 *ec4 = reinterpret_cast<const float4 *>(vc + V_ECOL + rb * 64 + 32 * hf);
+                    const float rowf = p < 64 ? vc[V_BETA + r] * vc[V_EROW + r] : vc[V_EROW + r];
 #pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 e = ec4[i4];
-                    const int i = 4 * i4;
-                    v[i] = i < lim ? rowf * e.x * v[i] : 0.f;
-                    v[i + 1] = i + 1 < lim ? rowf * e.y * v[i + 1] : 0.f;
-                    v[i + 2] = i + 2 < lim ? rowf * e.z * v[i + 2] : 0.f;
-                    v[i + 3] = i + 3 < lim ? rowf * e.w * v[i + 3] : 0.f;
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 e = ec4[i4];
+                        const int i = 4 * i4;
+                        v[i] = i < lim ? rowf * e.x * v[i] : 0.f;
+                        v[i + 1] = i + 1 < lim ? rowf * e.y * v[i + 1] : 0.f;
+                        v[i + 2] = i + 2 < lim ? rowf * e.z * v[i + 2] : 0.f;
+                        v[i + 3] = i + 3 < lim ? rowf * e.w * v[i + 3] : 0.f;
+                    }
+                } else {   // the decays ride on the operands: A = beta_r (Ks Kb^T)_ri, M = (Qs Kb^T)_ri
+                    const float rowf = p < 64 ? vc[KV_BETA + r] : 1.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = i < lim ? rowf * v[i] : 0.f;
                 }
                 // The previous chunk's first products are done with M and U^T (the inverse's scratch).
                 if (c >= 1) wait(B_P1, (c - 1) & 1);
@@ -431,12 +468,15 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int hh = 0; hh < 2; ++hh) {
                         const int r = g8 + 8 * hh, col = 8 * tt + 2 * t4, i = I0 + col;
                         const float x0 = x[tt][2 * hh], x1 = x[tt][2 * hh + 1];
-                        const float u0 = x0 * vc[V_BG + i], u1 = x1 * vc[V_BG + i + 1];
-                        const float w0 = x0 * vc[V_BETA + i], w1 = x1 * vc[V_BETA + i + 1];
+                        constexpr int VB = GATE ? KV_BETA : V_BETA;
+                        const float w0 = x0 * vc[VB + i], w1 = x1 * vc[VB + i + 1];
                         *reinterpret_cast<uint32_t *>(sm + INV_D + (uint32_t)((wq * 16 + r) * LDT16 + col) * 2u) =
                             pack_h2(x0, x1);
-                        *reinterpret_cast<uint32_t *>(sm + OFF_TP + swz_off(I0 + r, i, 0)) = pack_h2(u0, u1);
                         *reinterpret_cast<uint32_t *>(sm + OFF_TPP + swz_off(I0 + r, i, 0)) = pack_h2(w0, w1);
+                        if (GATE == 0) {
+                            const float u0 = x0 * vc[V_BG + i], u1 = x1 * vc[V_BG + i + 1];
+                            *reinterpret_cast<uint32_t *>(sm + OFF_TP + swz_off(I0 + r, i, 0)) = pack_h2(u0, u1);
+                        }
                     }
             } else {
                 // zero chunks: row u of block R = u / 16, 16-byte chunks 2(R+1) .. 7, of one of the two tiles
@@ -465,14 +505,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 if (wq == 0) {
                     chain_start(c0, c1, Dt(1), LDT16, At(1, 0), LDA16, lane);
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 16, 0, c0, c1, -1.f, vc, lane);
+                    st_tblock<GATE>(sm, 16, 0, c0, c1, -1.f, vc, lane);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
-                    st_tblock(sm, 32, 16, c0, c1, -1.f, vc, lane);
+                    st_tblock<GATE>(sm, 32, 16, c0, c1, -1.f, vc, lane);
                 } else if (wq == 1) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
-                    st_tblock(sm, 48, 32, c0, c1, -1.f, vc, lane);
+                    st_tblock<GATE>(sm, 48, 32, c0, c1, -1.f, vc, lane);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
                     chain_next(c0, c1, At(1, 0), LDA16, lane);
@@ -480,7 +520,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 32, 0, c0, c1, 1.f, vc, lane);
+                    st_tblock<GATE>(sm, 32, 0, c0, c1, 1.f, vc, lane);
                 } else if (wq == 2) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
@@ -489,7 +529,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(1), LDT16, lane);
-                    st_tblock(sm, 48, 16, c0, c1, 1.f, vc, lane);
+                    st_tblock<GATE>(sm, 48, 16, c0, c1, 1.f, vc, lane);
                 } else {
                     float q0[4], q1[4], h0[4], h1[4];
                     chain_start(q0, q1, Dt(3), LDT16, At(3, 2), LDA16, lane);   // Q = D3 A32 D2
@@ -507,7 +547,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                     for (int e = 0; e < 4; ++e) c0[e] = u0[e] + h0[e] - c0[e], c1[e] = u1[e] + h1[e] - c1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
-                    st_tblock(sm, 48, 0, c0, c1, 1.f, vc, lane);
+                    st_tblock<GATE>(sm, 48, 0, c0, c1, 1.f, vc, lane);
                 }
             }
             fence_proxy_async();
@@ -520,7 +560,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
-                    const uint64_t bt = sdesc(sb0 + OFF_TP + s * 32, 16, 1024);
+                    const uint64_t bt = sdesc(sb0 + (GATE ? OFF_TPP : OFF_TP) + s * 32, 16, 1024);
                     mma_ss(tb + TM_Y, sdesc(stg + s * 2048, 16384, 1024), bt, ID_WU, s > 0);
                 }
 #pragma unroll
@@ -540,28 +580,45 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_U16), v + 32 + 8 * j);
             }
-            // K -> Kt = diag(Gamma_C / Gamma) K in place (the W product is done with K)
+            // K -> Kt = diag(Gamma_C / Gamma) K in place (the W product is done with K); per-channel
+            // gate: Kt = Kb diag(exp(G_C - G_31)) into the K slot (Ks is done with too)
 #pragma unroll
             for (int jj = 0; jj < 1024 / GT; ++jj) {
                 const int e = gt + GT * jj, tok = (e >> 3) & 63;
                 uint4 *pch = reinterpret_cast<uint4 *>(stgp + (e >> 9) * 16384) + (e & 511);
-                const float f = vc[V_F + tok];
-                uint4 u = *pch;
-                __half2 *hh = reinterpret_cast<__half2 *>(&u);
+                if (GATE == 0) {
+                    const float f = vc[V_F + tok];
+                    uint4 u = *pch;
+                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 x = __half22float2(hh[k]);
-                    hh[k] = __floats2half2_rn(x.x * f, x.y * f);
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 x = __half22float2(hh[k]);
+                        hh[k] = __floats2half2_rn(x.x * f, x.y * f);
+                    }
+                    *pch = u;
+                } else {
+                    // physical 16-byte chunk e % 8 of row tok holds key channels 8 ((e % 8) ^ (tok % 8)) ..
+                    const int ch0 = 64 * (e >> 9) + 8 * ((e & 7) ^ (tok & 7));
+                    uint4 u = *(reinterpret_cast<const uint4 *>(sm + OFF_KB + sb * 16384 + (e >> 9) * 8192) + (e & 511));
+                    const float4 f0 = *reinterpret_cast<const float4 *>(vc + KV_ECM + ch0);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(vc + KV_ECM + ch0 + 4);
+                    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 x = __half22float2(hh[k]);
+                        hh[k] = __floats2half2_rn(x.x * f[2 * k], x.y * f[2 * k + 1]);
+                    }
+                    *pch = u;
                 }
-                *pch = u;
             }
-            // diag(Gamma) [r][j] into the dead V tile
+            // diag(Gamma) [r][j] (per-channel gate: the identity) into the dead V tile
 #pragma unroll
             for (int jj = 0; jj < 512 / GT; ++jj) {
                 const int e = gt + GT * jj, r = e >> 3, j = e & 7;
                 float x[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? vc[V_GAM + r] : 0.f;
+                for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? (GATE ? 1.f : vc[V_GAM + r]) : 0.f;
                 st_chunk8(stg + STG_V + swz_chunk(r, j, 0), x);
             }
             tc_fence_before();
@@ -630,7 +687,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 const int t = t0 + lane + 32 * e;
                 const bool ok = t < T;
                 const size_t ix = (size_t)(tok0 + t) * a.Hv + h;
-                gb[e] = ok ? a.g[ix] : 0.f;
+                gb[e] = (GATE == 0 && ok) ? a.g[ix] : 0.f;
                 gb[2 + e] = ok ? a.beta[ix] : 0.f;
             }
         };
@@ -735,13 +792,124 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             mbar_arrive(bar(B_CV0 + sb));
         };
 
+        // Per-channel gate: chunk c's gate pass. Thread (cp, rg) = (tid % 64, tid / 64) owns key
+        // channels 2 cp, 2 cp + 1 and rows 16 rg .. 16 rg + 15. G is the in-chunk prefix of g per
+        // channel (rows past the sequence's end add 0, so G_31 and G_C stop at its last token);
+        // K and Q become Ks = K exp(G - G_31) and Qs = Q exp(G - G_31) in place, Kb = K exp(G_31 - G)
+        // goes to the buffer's Kb tile, and V is converted to fp16. Then the Gram [Ks; Qs] Kb^T.
+        auto ready_chunk_kda = [&](int c, const float gb[4]) {
+            const int sb = c & 1;
+            uint8_t *stgp = sm + sb * STG_BYTES;
+            float *vk = vec + sb * KV_SET;
+            float *tot = vec + KV_TOT;
+            const int nvalid = min(C, T - c * C);
+            const int cp = tid & 63, rg = tid >> 6, r0 = 16 * rg;
+            float2 gq[16];
+            {
+                const float *gp = a.g + ((size_t)(tok0 + (long)c * C + r0) * a.Hv + h) * D + 2 * cp;
+                const size_t gs = (size_t)a.Hv * D;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    gq[i] = r0 + i < nvalid ? __ldg(reinterpret_cast<const float2 *>(gp + (size_t)i * gs))
+                                            : make_float2(0.f, 0.f);
+            }
+            wait(B_LD0 + sb, (c >> 1) & 1);
+#pragma unroll
+            for (int j = 0; j < 1024 / GT; ++j) {   // V (2 atoms of 64 rows) to fp16, rows past the end zeroed
+                const int e = tid + GT * j, row = (e >> 3) & 63;
+                uint4 *pch = reinterpret_cast<uint4 *>(stgp + STG_V) + e;
+                const uint4 hv = row < nvalid ? bf16x8_to_f16x8(*pch) : make_uint4(0, 0, 0, 0);
+                *pch = hv;
+            }
+            float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                run.x += gq[i].x;
+                run.y += gq[i].y;
+                gq[i] = run;
+            }
+            reinterpret_cast<float2 *>(tot + rg * D)[cp] = run;
+            named_bar_sync(2, GT);   // the row groups' sums
+            const float2 t0 = reinterpret_cast<const float2 *>(tot)[cp], t1 = reinterpret_cast<const float2 *>(tot + D)[cp],
+                         t2 = reinterpret_cast<const float2 *>(tot + 2 * D)[cp];
+            const float2 g31 = make_float2(t0.x + t1.x, t0.y + t1.y);
+            const float2 off = rg == 0 ? make_float2(0.f, 0.f)
+                               : rg == 1 ? t0 : rg == 2 ? g31 : make_float2(g31.x + t2.x, g31.y + t2.y);
+            if (rg == 0) {
+                const float2 t3 = reinterpret_cast<const float2 *>(tot + 3 * D)[cp];
+                const float2 gc = make_float2(g31.x + t2.x + t3.x, g31.y + t2.y + t3.y);
+                reinterpret_cast<float2 *>(vk + KV_E31)[cp] = make_float2(__expf(g31.x), __expf(g31.y));
+                reinterpret_cast<float2 *>(vk + KV_GC)[cp] = make_float2(__expf(gc.x), __expf(gc.y));
+                reinterpret_cast<float2 *>(vk + KV_ECM)[cp] = make_float2(__expf(gc.x - g31.x), __expf(gc.y - g31.y));
+            }
+            if (warp == 0) {
+                vk[KV_BETA + lane] = gb[2];
+                vk[KV_BETA + 32 + lane] = gb[3];
+            }
+            uint8_t *kbp = sm + OFF_KB + sb * 16384;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = r0 + i;
+                const float gx = off.x + gq[i].x, gy = off.y + gq[i].y;
+                const float e1x = __expf(gx - g31.x), e1y = __expf(gy - g31.y);
+                const float e2x = __expf(g31.x - gx), e2y = __expf(g31.y - gy);
+                const uint32_t ok = swz_off(r, 2 * cp, 16384), oq = swz_off(64 + r, 2 * cp, 16384);
+                const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(stgp + ok));
+                const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(stgp + oq));
+                const bool live = r < nvalid;
+                const uint32_t ks = live ? pack_h2(kf.x * e1x, kf.y * e1y) : 0u;
+                const uint32_t qs = live ? pack_h2(qf.x * e1x, qf.y * e1y) : 0u;
+                const uint32_t kb = live ? pack_h2(kf.x * e2x, kf.y * e2y) : 0u;
+                *reinterpret_cast<uint32_t *>(stgp + ok) = ks;
+                *reinterpret_cast<uint32_t *>(stgp + oq) = qs;
+                *reinterpret_cast<uint32_t *>(kbp + swz_off(r, 2 * cp, 8192)) = kb;
+            }
+            fence_proxy_async();
+            named_bar_sync(2, GT);   // every tile of the chunk written
+            if (gissuer) {
+                const uint32_t stg = sb0 + sb * STG_BYTES, kbs = sb0 + OFF_KB + sb * 16384;
+                if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ss(tb + TM_G, sdesc(stg + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                           sdesc(kbs + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_GRAM, s > 0);
+                mma_commit(bar(B_G0 + sb));
+            }
+            mbar_arrive(bar(B_CV0 + sb));
+        };
+        auto ready = [&](int c, const float gb[4]) {
+            if (GATE) ready_chunk_kda(c, gb);
+            else ready_chunk(c, gb);
+        };
         float S[64];
+        // The fp16 copy of the state S^T [dv][dk]: a shared-memory operand tile, or for the
+        // per-channel gate tensor-memory columns TM_S16 + 32 hf .. of lane p (two dk per column).
+        // Per-channel gate: the copy read by chunk cn is S~ = diag(exp G_31) S with chunk cn's G_31:
+        // then P S = P' S~ and Qh S = X' S~ with P' = -Kt^T W' and X' = (Qs - M W')^T ^T as the chunk
+        // group leaves them in tensor memory, so neither needs a scaling on its way out.
+        auto store_s16 = [&](int cn) {
+            if (GATE == 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
+            } else {
+                const float4 *e4 = reinterpret_cast<const float4 *>(vec + (cn & 1) * KV_SET + KV_E31 + 64 * hf);
+                uint32_t w[32];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float4 e = e4[j];
+                    w[2 * j] = pack_h2(S[4 * j] * e.x, S[4 * j + 1] * e.y);
+                    w[2 * j + 1] = pack_h2(S[4 * j + 2] * e.z, S[4 * j + 3] * e.w);
+                }
+                tmem_st32(tmem_addr(tb, q4, TM_S16 + 32 * hf), w);
+                tmem_wait_st();
+            }
+        };
         {
             const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + (size_t)(64 * hf) * D + p : nullptr;
 #pragma unroll
             for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
+            if (GATE == 0) store_s16(0);
         }
         float gbn[4] = {0.f, 0.f, 0.f, 0.f};
         if (issuer && NC > 0) {
@@ -750,12 +918,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         }
         if (NC > 0) {
             load_gb(0, gbn);
-            ready_chunk(0, gbn);
+            ready(0, gbn);
         }
         if (NC > 1) {
             load_gb(1, gbn);
-            ready_chunk(1, gbn);
+            ready(1, gbn);
         }
+        if (GATE && NC > 0) store_s16(0);   // needs chunk 0's exp(G_31)
+        tc_fence_before();
         for (int c = 0; c < NC; ++c) {
             if (NORM && a.z) {   // this chunk's z row segment (pass B's) into L1
                 const int r = 8 * warp + (lane & 7), k = lane >> 3;
@@ -775,6 +945,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             wait(B_P, c & 1);
             if (issuer && c + 2 < NC) issue_loads(c + 2);   // chunk c's staging buffer is free
             if (c + 2 < NC) load_gb(c + 2, gbn);
+            if (GATE && c + 2 < NC && (c + 2) * C + (tid >> 2) < T)
+                prefetch_l2(a.g + ((size_t)(tok0 + (long)(c + 2) * C + (tid >> 2)) * a.Hv + h) * D + 32 * (tid & 3));
             tc_fence_after();
             {
                 float v[64];
@@ -782,7 +954,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
             }
-            const float gC = vec[(c & 1) * V_SET + V_GC];
+            const float gC = GATE ? 0.f : vec[(c & 1) * V_SET + V_GC];
             tc_fence_before();
             mbar_arrive(bar(B_YE));
             fence_proxy_async();
@@ -792,28 +964,49 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
-                    mma_ss(tb + TM_S, sdesc(sb0 + OFF_ST16 + koff, 16, 1024), sdesc(sb0 + OFF_P16 + koff, 16, 1024),
-                           ID_S, true);
+                    if (GATE == 0)
+                        mma_ss(tb + TM_S, sdesc(sb0 + OFF_ST16 + koff, 16, 1024), sdesc(sb0 + OFF_P16 + koff, 16, 1024),
+                               ID_S, true);
+                    else
+                        mma_ts(tb + TM_S, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_P16 + koff, 16, 1024), ID_S, true);
                 }
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
-                    mma_ss(tb + TM_O, sdesc(sb0 + OFF_ST16 + koff, 16, 1024), sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024),
-                           ID_O, true);
+                    if (GATE == 0)
+                        mma_ss(tb + TM_O, sdesc(sb0 + OFF_ST16 + koff, 16, 1024),
+                               sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024), ID_O, true);
+                    else
+                        mma_ts(tb + TM_O, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024), ID_O, true);
                 }
                 mma_commit(bar(B_ST));
             }
             wait(B_ST, c & 1);
             tc_fence_after();
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
-            {
+            if (GATE == 0) {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_S + 64 * hf), tmem_addr(tb, q4, TM_S + 64 * hf + 32), v);
 #pragma unroll
                 for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
+            } else {   // S <- diag(Gamma_C) S + (P S + R), row dk = 64 hf + i, in two halves of 32
+                const float4 *g4 = reinterpret_cast<const float4 *>(vec + (c & 1) * KV_SET + KV_GC + 64 * hf);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    float v[32];
+                    tmem_ld32(tmem_addr(tb, q4, TM_S + 64 * hf + 32 * h2), v);
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 gg = g4[8 * h2 + i4];
+                        float *sp = S + 32 * h2 + 4 * i4;
+                        sp[0] = fmaf(gg.x, sp[0], v[4 * i4]);
+                        sp[1] = fmaf(gg.y, sp[1], v[4 * i4 + 1]);
+                        sp[2] = fmaf(gg.z, sp[2], v[4 * i4 + 2]);
+                        sp[3] = fmaf(gg.w, sp[3], v[4 * i4 + 3]);
+                    }
+                }
             }
+            store_s16(c + 1);
             // o rows 32 hf .. 32 hf + 31 of this chunk (column p of Qh S + Uh) into the o tile
             // (the P tile, dead until the next chunk) in the TMA 128-byte swizzle, then out by
             // TMA stores, which clip tokens past T. The partial last chunk of a packed
@@ -938,7 +1131,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 for (int k = 0; k < D / EPB; ++k)
                     tma_store_4d(&map_o, k * EPB, h, tt0 + c * C, tbb, sb0 + src + k * C * 128);
             }
-            if (c + 2 < NC) ready_chunk(c + 2, gbn);
+            if (c + 2 < NC) ready(c + 2, gbn);
             if (issuer) tma_store_wait_read();   // the o tile is read before the next P tile is written
             named_bar_sync(2, GT);
         }
@@ -978,7 +1171,8 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
         return cudaErrorInvalidValue;
     // The layer's options are compiled into a separate instance, so a call without them runs
     // the same code as before they existed.
-    auto kernel = (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true> : tc_fwd_kernel<TOut, false>;
+    auto kernel = a.gate_mode ? tc_fwd_kernel<TOut, false, 1>
+                              : (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true, 0> : tc_fwd_kernel<TOut, false, 0>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
     kernel<<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv, mo);
@@ -989,7 +1183,8 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
 
 bool tc_supported(const FwdArgs &a)
 {
-    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && a.gate_mode == 0;
+    // The per-channel gate with the layer's options stays on the warp-level kernel.
+    return in_bf16(a.dtype) && a.Dk == D && a.Dv == D && (a.gate_mode == 0 || (!a.qk_l2norm && !a.z));
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st)
