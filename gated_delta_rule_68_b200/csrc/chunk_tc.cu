@@ -55,6 +55,9 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
+#include <chrono>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_util.cuh"
@@ -191,6 +194,16 @@ __device__ __forceinline__ uint32_t pack_bf2(float x, float y)
     const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     return *reinterpret_cast<const uint32_t *>(&h);
 }
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 __device__ __forceinline__ void prefetch_l1(const void *p)
 {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
@@ -285,7 +298,7 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
 // NORM: the layer's options (compiled as a separate instance, so the plain forward runs
 // exactly its own code): q and k rows divided by sqrt(sum of squares + 1e-6) as they are
 // converted, and o rows replaced by o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
-template <typename TOut, bool NORM, int GATE>
+template <typename TOut, bool NORM, int GATE, bool SCHED>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
@@ -306,18 +319,39 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
     const int p = 32 * q4 + lane;     // row of the 128-row products owned by this thread
     const int hf = (warp >> 2) & 1;   // which half of that row's columns this thread takes
-    const int bh = blockIdx.x, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
-    // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
-    // maps, batch index tbb and token offset tt0. Packed input: sequence b of cu_seqlens
-    // (clamped into the token axis); the rows of its last chunk past its end are zeroed
-    // when the chunk is converted, since the loaded tile holds the next sequence there.
-    int T = a.T, tbb = b, tt0 = 0;
-    long tok0 = (long)b * a.T;
-    if (a.cu_seqlens) {
-        const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
-        T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
-    }
-    const int NC = (T + C - 1) / C;
+    // The CTA's work, as pieces (unit, chunks [c0, c1)). Without a schedule (a.sched_len == 0)
+    // one piece: the whole unit blockIdx.x. With one (fixed-length sequences, more units than
+    // SMs), the units' chunks are laid end to end and cut into runs of a.sched_len
+    // chunk-steps, run i for CTA i, wrapped as in McNaughton's rule: the unit cut by the end
+    // of run i does its first chunks at the start of run i + 1 and its last chunks at the end
+    // of run i. The first part leaves its state in the workspace and raises its flag; the
+    // last part waits for the flag and starts from that state. A unit has at most sched_len
+    // chunks, so its first part always ends before its last part begins. Mbarrier phases and
+    // staging buffers follow the CTA's running step count, not the chunk index.
+    enum { WHOLE = 0, FIRST = 1, LAST = 2 };
+    const int nc_unit = (a.T + C - 1) / C;                 // chunks per unit without cu_seqlens
+    const long w_all = (long)a.B * a.Hv * nc_unit;
+    // The piece that starts at position pos of this CTA's run (pos < run end): unit, first and
+    // end chunk (end -1: the unit's chunk count), kind, and the position after it.
+    struct Piece { int u, c0, c1, kind; long next; };
+    auto piece_at = [&](long pos) -> Piece {
+        Piece pc;
+        if (!SCHED) {
+            pc.u = blockIdx.x, pc.c0 = 0, pc.c1 = -1, pc.kind = WHOLE, pc.next = 1;
+            return pc;
+        }
+        const long r1 = min((long)(blockIdx.x + 1) * a.sched_len, w_all);
+        pc.u = (int)(pos / nc_unit);
+        const int cu = (int)(pos % nc_unit);
+        pc.next = min(r1, (long)(pc.u + 1) * nc_unit);
+        const int len = (int)(pc.next - pos);
+        if (cu != 0) pc.c0 = 0, pc.c1 = len, pc.kind = FIRST;
+        else if (len < nc_unit) pc.c0 = nc_unit - len, pc.c1 = nc_unit, pc.kind = LAST;
+        else pc.c0 = 0, pc.c1 = nc_unit, pc.kind = WHOLE;
+        return pc;
+    };
+    const long run0 = SCHED ? (long)blockIdx.x * a.sched_len : 0;
+    const long run1 = SCHED ? min(run0 + a.sched_len, w_all) : 1;
     constexpr int VSET = GATE ? KV_SET : V_SET;   // floats per chunk-parity set of vectors
     static_assert(!(GATE && NORM), "the layer options run on the warp-level kernel with the per-channel gate");
 
@@ -351,14 +385,32 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         const int gt = tid - GT;          // 0 .. GT-1
         const int wq = q4;                // warp within a half of the group
         const bool issuer = gt == 0;
-        for (int c = 0; c < NC; ++c) {
-            const int sb = c & 1;
+        // One piece: unit pu, chunks [pc0, pc1) (pc1 < 0: all of them), the CTA's step count
+        // at its first chunk gsb.
+        auto chunk_piece = [&](const int pu, const int pc0, const int pc1, const int gsb) {
+            const int bh = pu, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
+            // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
+            // maps, batch index tbb and token offset tt0. Packed input: sequence b of cu_seqlens
+            // (clamped into the token axis); the rows of its last chunk past its end are zeroed
+            // when the chunk is converted, since the loaded tile holds the next sequence there.
+            int T = a.T, tbb = b, tt0 = 0;
+            long tok0 = (long)b * a.T;
+            if (a.cu_seqlens) {
+                const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
+                T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
+            }
+            const int NC = (T + C - 1) / C;
+            const int c0 = pc0, c1 = pc1 < 0 ? NC : pc1;
+            (void)hk, (void)tbb, (void)tt0;
+        for (int c = c0; c < c1; ++c) {
+            const int gs = gsb + (c - c0);
+            const int sb = gs & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES;
             uint8_t *stgp = sm + sb * STG_BYTES;
             const float *vc = vec + sb * VSET;
-            wait(B_CV0 + sb, (c >> 1) & 1);
+            wait(B_CV0 + sb, (gs >> 1) & 1);
             // Gram epilogue: A (rows < 64) and M (rows 64..127), columns 32 hf .. 32 hf + 31
-            wait(B_G0 + sb, (c >> 1) & 1);
+            wait(B_G0 + sb, (gs >> 1) & 1);
             tc_fence_after();
             {
                 float v[32];
@@ -386,7 +438,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int i = 0; i < 32; ++i) v[i] = i < lim ? rowf * v[i] : 0.f;
                 }
                 // The previous chunk's first products are done with M and U^T (the inverse's scratch).
-                if (c >= 1) wait(B_P1, (c - 1) & 1);
+                if (gs >= 1) wait(B_P1, (gs - 1) & 1);
                 if (p >= 64) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(r, 4 * hf + j, OFF_M16), v + 8 * j);
@@ -412,7 +464,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             named_bar_sync(1, GT);
 
             // ... and with W^T (the tiles of T) before they are rewritten.
-            if (c >= 1) wait(B_P, (c - 1) & 1);
+            if (gs >= 1) wait(B_P, (gs - 1) & 1);
             // Inverse, level 0: warp wq of the first half inverts the unit lower 16 x 16 block
             // I + N (N = A_bb, b = wq) in the product form
             //   (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8)      (N^16 = 0)
@@ -556,7 +608,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             // W^T = K^T T'^T -> Y[0:64),  U^T = V^T T''^T -> Y[64:128), once the state
             // group has read the previous chunk's P and Qh out of Y and X.
             if (issuer) {
-                if (c >= 1) wait(B_YE, (c - 1) & 1);
+                if (gs >= 1) wait(B_YE, (gs - 1) & 1);
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
@@ -570,7 +622,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 }
                 mma_commit(bar(B_W));
             }
-            wait(B_W, c & 1);
+            wait(B_W, gs & 1);
             tc_fence_after();
             {
                 float v[64];
@@ -628,8 +680,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             // R^T = U^T Kt -> state product,  X = Q^T diag(Gamma) - W^T M^T -> X,
             // Uh^T = U^T M^T -> o accumulator (these free M and U^T), then P = -Kt^T W -> Y.
             if (issuer) {
-                if (c >= 1) wait(B_SE, (c - 1) & 1);
-                if (c >= 1) wait(B_OE, (c - 1) & 1);
+                if (gs >= 1) wait(B_SE, (gs - 1) & 1);
+                if (gs >= 1) wait(B_OE, (gs - 1) & 1);
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
@@ -655,6 +707,18 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 mma_commit(bar(B_P));
             }
         }
+        };
+        if constexpr (SCHED) {
+            int gsb = 0;
+            for (long ppos = run0; ppos < run1;) {
+                const Piece pcs = piece_at(ppos);
+                ppos = pcs.next;
+                chunk_piece(pcs.u, pcs.c0, pcs.c1, gsb);
+                gsb += pcs.c1 - pcs.c0;
+            }
+        } else {
+            chunk_piece(blockIdx.x, 0, -1, 0);
+        }
         if (issuer) {
             mma_commit(bar(B_DR1));
             mbar_wait_bounded(bar(B_DR1), 0);
@@ -667,8 +731,25 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // and the Gram.
         const bool issuer = tid == 0;
         const bool gissuer = tid == 7 * 32;   // the Gram's issuer: warp 7 has no gate-vector work
-        auto issue_loads = [&](int c) {
-            const int sb = c & 1;
+        // One piece: unit pu, chunks [pc0, pc1) (pc1 < 0: all of them), its kind, and the CTA's
+        // step count at its first chunk gsb.
+        auto state_piece = [&](const int pu, const int pc0, const int pc1, const int pkind, const int gsb) {
+            const int bh = pu, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
+            // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
+            // maps, batch index tbb and token offset tt0. Packed input: sequence b of cu_seqlens
+            // (clamped into the token axis); the rows of its last chunk past its end are zeroed
+            // when the chunk is converted, since the loaded tile holds the next sequence there.
+            int T = a.T, tbb = b, tt0 = 0;
+            long tok0 = (long)b * a.T;
+            if (a.cu_seqlens) {
+                const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
+                T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
+            }
+            const int NC = (T + C - 1) / C;
+            const int c0 = pc0, c1 = pc1 < 0 ? NC : pc1;
+            (void)hk, (void)tbb, (void)tt0;
+        auto issue_loads = [&](int c, int gs) {
+            const int sb = gs & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES, bl = bar(B_LD0 + sb);
             const int t0 = tt0 + c * C;
             mbar_expect_tx(bl, STG_BYTES);
@@ -693,11 +774,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         };
         // Chunk c's tiles to fp16 in place, then its Gram (warp 7) while warps 0 .. 6 write its
         // gate vectors.
-        auto ready_chunk = [&](int c, const float gb[4]) {
-            const int sb = c & 1;
+        auto ready_chunk = [&](int c, int gs, const float gb[4]) {
+            const int sb = gs & 1;
             uint8_t *stgp = sm + sb * STG_BYTES;
             float *vs = vec + sb * V_SET;
-            wait(B_LD0 + sb, (c >> 1) & 1);
+            wait(B_LD0 + sb, (gs >> 1) & 1);
             const int nvalid = min(C, T - c * C);
             if (NORM && a.qk_l2norm) {
                 // [K; Q] rows: chunks e and e + 1024 are the two halves of one row, and a row's 8
@@ -741,7 +822,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             named_bar_sync(2, GT);   // every tile of the chunk converted
             if (gissuer) {
                 const uint32_t stg = sb0 + sb * STG_BYTES;
-                if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
+                if (gs >= 1) wait(B_GE, (gs - 1) & 1);   // the chunk group has read the previous Gram
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
@@ -797,8 +878,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // channel (rows past the sequence's end add 0, so G_31 and G_C stop at its last token);
         // K and Q become Ks = K exp(G - G_31) and Qs = Q exp(G - G_31) in place, Kb = K exp(G_31 - G)
         // goes to the buffer's Kb tile, and V is converted to fp16. Then the Gram [Ks; Qs] Kb^T.
-        auto ready_chunk_kda = [&](int c, const float gb[4]) {
-            const int sb = c & 1;
+        auto ready_chunk_kda = [&](int c, int gs, const float gb[4]) {
+            const int sb = gs & 1;
             uint8_t *stgp = sm + sb * STG_BYTES;
             float *vk = vec + sb * KV_SET;
             float *tot = vec + KV_TOT;
@@ -813,7 +894,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     gq[i] = r0 + i < nvalid ? __ldg(reinterpret_cast<const float2 *>(gp + (size_t)i * gs))
                                             : make_float2(0.f, 0.f);
             }
-            wait(B_LD0 + sb, (c >> 1) & 1);
+            wait(B_LD0 + sb, (gs >> 1) & 1);
 #pragma unroll
             for (int j = 0; j < 1024 / GT; ++j) {   // V (2 atoms of 64 rows) to fp16, rows past the end zeroed
                 const int e = tid + GT * j, row = (e >> 3) & 63;
@@ -868,7 +949,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             named_bar_sync(2, GT);   // every tile of the chunk written
             if (gissuer) {
                 const uint32_t stg = sb0 + sb * STG_BYTES, kbs = sb0 + OFF_KB + sb * 16384;
-                if (c >= 1) wait(B_GE, (c - 1) & 1);   // the chunk group has read the previous Gram
+                if (gs >= 1) wait(B_GE, (gs - 1) & 1);   // the chunk group has read the previous Gram
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
@@ -878,9 +959,9 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             }
             mbar_arrive(bar(B_CV0 + sb));
         };
-        auto ready = [&](int c, const float gb[4]) {
-            if (GATE) ready_chunk_kda(c, gb);
-            else ready_chunk(c, gb);
+        auto ready = [&](int c, int gs, const float gb[4]) {
+            if (GATE) ready_chunk_kda(c, gs, gb);
+            else ready_chunk(c, gs, gb);
         };
         float S[64];
         // The fp16 copy of the state S^T [dv][dk]: a shared-memory operand tile, or for the
@@ -888,12 +969,12 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // Per-channel gate: the copy read by chunk cn is S~ = diag(exp G_31) S with chunk cn's G_31:
         // then P S = P' S~ and Qh S = X' S~ with P' = -Kt^T W' and X' = (Qs - M W')^T ^T as the chunk
         // group leaves them in tensor memory, so neither needs a scaling on its way out.
-        auto store_s16 = [&](int cn) {
+        auto store_s16 = [&](int gsn) {
             if (GATE == 0) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
             } else {
-                const float4 *e4 = reinterpret_cast<const float4 *>(vec + (cn & 1) * KV_SET + KV_E31 + 64 * hf);
+                const float4 *e4 = reinterpret_cast<const float4 *>(vec + (gsn & 1) * KV_SET + KV_E31 + 64 * hf);
                 uint32_t w[32];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -906,27 +987,45 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             }
         };
         {
-            const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D + (size_t)(64 * hf) * D + p : nullptr;
+            // The entering state: h0, or for the last part of a cut unit the state its first part
+            // left (flag and state of boundary blockIdx.x + 1, written by the next CTA).
+            const float *h0 = a.h0 ? a.h0 + (size_t)bh * D * D : nullptr;
+            if (SCHED && pkind == LAST) {
+                const int bd = blockIdx.x + 1;
+                if (tid == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_u64(a.sched_flags + bd) != a.sched_tag)
+                        if (globaltimer_ns() - t0 > 1000000000ull) {
+                            *reinterpret_cast<volatile int *>(&abort_sh) = 1;
+                            atomicAdd(&g_tc_timeouts, 1u);
+                            break;
+                        }
+                }
+                named_bar_sync(2, GT);
+                h0 = a.sched_states + (size_t)bd * D * D;
+            }
+            if (h0) h0 += (size_t)(64 * hf) * D + p;
 #pragma unroll
-            for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? h0[(size_t)dk * D] : 0.f;
-            if (GATE == 0) store_s16(0);
+            for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? __ldcg(h0 + (size_t)dk * D) : 0.f;
+            if (GATE == 0) store_s16(gsb);
         }
         float gbn[4] = {0.f, 0.f, 0.f, 0.f};
-        if (issuer && NC > 0) {
-            issue_loads(0);
-            if (NC > 1) issue_loads(1);
+        if (issuer && c1 > c0) {
+            issue_loads(c0, gsb);
+            if (c1 > c0 + 1) issue_loads(c0 + 1, gsb + 1);
         }
-        if (NC > 0) {
-            load_gb(0, gbn);
-            ready(0, gbn);
+        if (c1 > c0) {
+            load_gb(c0, gbn);
+            ready(c0, gsb, gbn);
         }
-        if (NC > 1) {
-            load_gb(1, gbn);
-            ready(1, gbn);
+        if (c1 > c0 + 1) {
+            load_gb(c0 + 1, gbn);
+            ready(c0 + 1, gsb + 1, gbn);
         }
-        if (GATE && NC > 0) store_s16(0);   // needs chunk 0's exp(G_31)
+        if (GATE && c1 > c0) store_s16(gsb);   // needs the first chunk's exp(G_31)
         tc_fence_before();
-        for (int c = 0; c < NC; ++c) {
+        for (int c = c0; c < c1; ++c) {
+            const int gs = gsb + (c - c0);
             if (NORM && a.z) {   // this chunk's z row segment (pass B's) into L1
                 const int r = 8 * warp + (lane & 7), k = lane >> 3;
                 if (c * C + r < T)
@@ -934,7 +1033,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                                 ((size_t)(tok0 + c * C + r) * a.Hv + h) * D + 32 * k);
             }
             // P and Qh of this chunk, out of tensor memory into the operand tiles
-            wait(B_P1, c & 1);
+            wait(B_P1, gs & 1);
             tc_fence_after();
             {
                 float v[32];
@@ -942,10 +1041,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
             }
-            wait(B_P, c & 1);
-            if (issuer && c + 2 < NC) issue_loads(c + 2);   // chunk c's staging buffer is free
-            if (c + 2 < NC) load_gb(c + 2, gbn);
-            if (GATE && c + 2 < NC && (c + 2) * C + (tid >> 2) < T)
+            wait(B_P, gs & 1);
+            if (issuer && c + 2 < c1) issue_loads(c + 2, gs + 2);   // chunk c's staging buffer is free
+            if (c + 2 < c1) load_gb(c + 2, gbn);
+            if (GATE && c + 2 < c1 && (c + 2) * C + (tid >> 2) < T)
                 prefetch_l2(a.g + ((size_t)(tok0 + (long)(c + 2) * C + (tid >> 2)) * a.Hv + h) * D + 32 * (tid & 3));
             tc_fence_after();
             {
@@ -954,7 +1053,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
             }
-            const float gC = GATE ? 0.f : vec[(c & 1) * V_SET + V_GC];
+            const float gC = GATE ? 0.f : vec[(gs & 1) * V_SET + V_GC];
             tc_fence_before();
             mbar_arrive(bar(B_YE));
             fence_proxy_async();
@@ -981,7 +1080,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 }
                 mma_commit(bar(B_ST));
             }
-            wait(B_ST, c & 1);
+            wait(B_ST, gs & 1);
             tc_fence_after();
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
             if (GATE == 0) {
@@ -990,7 +1089,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
             } else {   // S <- diag(Gamma_C) S + (P S + R), row dk = 64 hf + i, in two halves of 32
-                const float4 *g4 = reinterpret_cast<const float4 *>(vec + (c & 1) * KV_SET + KV_GC + 64 * hf);
+                const float4 *g4 = reinterpret_cast<const float4 *>(vec + (gs & 1) * KV_SET + KV_GC + 64 * hf);
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     float v[32];
@@ -1006,7 +1105,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     }
                 }
             }
-            store_s16(c + 1);
+            store_s16(gs + 1);
             // o rows 32 hf .. 32 hf + 31 of this chunk (column p of Qh S + Uh) into the o tile
             // (the P tile, dead until the next chunk) in the TMA 128-byte swizzle, then out by
             // TMA stores, which clip tokens past T. The partial last chunk of a packed
@@ -1131,16 +1230,43 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 for (int k = 0; k < D / EPB; ++k)
                     tma_store_4d(&map_o, k * EPB, h, tt0 + c * C, tbb, sb0 + src + k * C * 128);
             }
-            if (c + 2 < NC) ready(c + 2, gbn);
+            if (c + 2 < c1) ready(c + 2, gs + 2, gbn);
             if (issuer) tma_store_wait_read();   // the o tile is read before the next P tile is written
             named_bar_sync(2, GT);
         }
         if (issuer) tma_store_wait_all();
         if (any_nonfinite32(S) || any_nonfinite32(S + 32)) *reinterpret_cast<volatile int *>(&range_sh) = 1;
-        if (a.hT) {
-            float *hp = a.hT + (size_t)bh * D * D + (size_t)(64 * hf) * D + p;
+        // The state after the piece: the final state to hT, or, after a first part, to this
+        // CTA's boundary (blockIdx.x) in the workspace, then the boundary's flag.
+        float *hout = SCHED && pkind == FIRST ? a.sched_states + (size_t)blockIdx.x * D * D : a.hT ? a.hT + (size_t)bh * D * D
+                                                                                          : nullptr;
+        if (hout) {
+            float *hp = hout + (size_t)(64 * hf) * D + p;
 #pragma unroll
             for (int dk = 0; dk < 64; ++dk) hp[(size_t)dk * D] = S[dk];
+        }
+        named_bar_sync(2, GT);
+        if (tid == 0) {
+            if (SCHED && pkind == FIRST) {
+                __threadfence();
+                st_release_u64(a.sched_flags + blockIdx.x, a.sched_tag);
+            }
+            if (range_sh) {
+                atomicAdd(&g_tc_range_errors, 1u);
+                range_sh = 0;
+            }
+        }
+        };
+        if constexpr (SCHED) {
+            int gsb = 0;
+            for (long ppos = run0; ppos < run1;) {
+                const Piece pcs = piece_at(ppos);
+                ppos = pcs.next;
+                state_piece(pcs.u, pcs.c0, pcs.c1, pcs.kind, gsb);
+                gsb += pcs.c1 - pcs.c0;
+            }
+        } else {
+            state_piece(blockIdx.x, 0, -1, WHOLE, 0);
         }
         if (issuer) {
             mma_commit(bar(B_DR0));
@@ -1153,7 +1279,6 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && range_sh) atomicAdd(&g_tc_range_errors, 1u);
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tb, 512);
@@ -1169,17 +1294,52 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
         !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true) ||
         !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
         return cudaErrorInvalidValue;
-    // The layer's options are compiled into a separate instance, so a call without them runs
-    // the same code as before they existed.
-    auto kernel = a.gate_mode ? tc_fwd_kernel<TOut, false, 1>
-                              : (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true, 0> : tc_fwd_kernel<TOut, false, 0>;
+    // The layer's options and the per-channel gate are separate instances, and so is the
+    // wrap-around schedule, so that a call without them runs the same code as before they existed.
+    auto kernel = a.sched_len ? (a.gate_mode ? tc_fwd_kernel<TOut, false, 1, true> : tc_fwd_kernel<TOut, false, 0, true>)
+                  : a.gate_mode ? tc_fwd_kernel<TOut, false, 1, false>
+                  : (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true, 0, false> : tc_fwd_kernel<TOut, false, 0, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
-    kernel<<<(unsigned)((long)a.B * a.Hv), NTH, SMEM_TC, st>>>(a, mq, mk, mv, mo);
+    const long units = (long)a.B * a.Hv, steps = units * ((a.T + C - 1) / C);
+    const long grid = a.sched_len ? (steps + a.sched_len - 1) / a.sched_len : units;
+    kernel<<<(unsigned)grid, NTH, SMEM_TC, st>>>(a, mq, mk, mv, mo);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+// The wrap-around schedule: with U units of n chunks on S SMs (U > S, fixed length) each
+// CTA takes ceil(U n / S) chunk-steps; the cuts between CTAs need a 64-bit flag and a
+// [Dk][Dv] fp32 state each.
+static bool sched_shape(const FwdArgs &a, long *len, long *grid)
+{
+    const long units = (long)a.B * a.Hv, nc = (a.T + C - 1) / C, sms = sm_count();
+    if (a.cu_seqlens || nc == 0 || sms <= 0 || units <= sms) return false;
+    *len = (units * nc + sms - 1) / sms;
+    *grid = (units * nc + *len - 1) / *len;
+    return true;
+}
+size_t tc_sched_bytes(const FwdArgs &a)
+{
+    long len, grid;
+    if (a.qk_l2norm || a.z || !sched_shape(a, &len, &grid)) return 0;
+    return (size_t)((grid * 8 + 255) / 256 * 256) + (size_t)grid * D * D * sizeof(float);
+}
+void tc_set_sched(FwdArgs &a, void *workspace)
+{
+    long len, grid;
+    if (!workspace || a.qk_l2norm || a.z || !sched_shape(a, &len, &grid)) return;
+    // A tag per launch, unlike any earlier one in this process and not 0: whatever a flag holds
+    // from before never reads as this launch's.
+    static std::atomic<unsigned long long> counter{0};
+    static const unsigned long long base =
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() << 20;
+    a.sched_len = (int)len;
+    a.sched_tag = (base + ++counter) | 1ull;
+    a.sched_flags = reinterpret_cast<unsigned long long *>(workspace);
+    a.sched_states = reinterpret_cast<float *>(reinterpret_cast<char *>(workspace) + (grid * 8 + 255) / 256 * 256);
+}
 
 bool tc_supported(const FwdArgs &a)
 {

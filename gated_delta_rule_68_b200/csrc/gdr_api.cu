@@ -89,6 +89,7 @@ size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int 
     if (B == 0 || T == 0) return 0;
     const gdr::FwdArgs a = make_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                                     nullptr, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (gdr::tc_supported(a)) return gdr::tc_sched_bytes(a);
     return gdr::fused_supported(a) ? 0 : gdr::simt_workspace_size(a);
 }
 
@@ -123,8 +124,12 @@ int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
         return GDR_OK;
     }
 
-    const gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    gdr::FwdArgs a = make_fwd(q, k, v, g, beta, h0, o, hT, B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
     if (gdr::tc_supported(a)) {
+        // More units than SMs: a workspace of gdr_fwd_workspace_size() bytes lets the kernel
+        // spread the units' chunks evenly over the SMs; without it, one CTA per unit.
+        const size_t need = gdr::tc_sched_bytes(a);
+        if (need > 0 && workspace && workspace_bytes >= need) gdr::tc_set_sched(a, workspace);
         cudaError_t e = gdr::launch_fwd_tc(a, s);
         if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
         g_launches += 1;

@@ -33,6 +33,13 @@ struct FwdArgs {
     const void *z = nullptr;
     const float *norm_w = nullptr;
     float norm_eps = 0.f;
+    // tcgen05 kernel, fixed-length sequences with more (batch row, value head) units than
+    // SMs: sched_len chunk-steps per CTA (0: one CTA per unit); the per-launch tag, flags and
+    // states of the units cut between two CTAs live in the caller's workspace.
+    int sched_len = 0;
+    unsigned long long sched_tag = 0;
+    unsigned long long *sched_flags = nullptr;
+    float *sched_states = nullptr;
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
@@ -49,6 +56,11 @@ unsigned int fused_error_counts(unsigned int *load_timeouts, unsigned int *range
 // fixed-length sequences, no layer options): one kernel, no workspace.
 bool tc_supported(const FwdArgs &a);
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t st);
+// Workspace bytes that let the tcgen05 kernel balance units over the SMs (0 when it runs one
+// CTA per unit anyway), and the schedule it then takes: fills a.sched_len, a.sched_tag and
+// the workspace pointers.
+size_t tc_sched_bytes(const FwdArgs &a);
+void tc_set_sched(FwdArgs &a, void *workspace);
 // Waits of the tcgen05 kernel that timed out since the library was loaded on this device,
 // and its units in which a value rounded to an fp16 operand was inf or NaN.
 unsigned int tc_error_count();

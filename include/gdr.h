@@ -143,7 +143,10 @@ GDR_API unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigne
 /*
  * Bytes of device workspace gdr_fwd_chunked needs for these sizes (0 when it
  * needs none). Returns 0 for invalid arguments as well; gdr_fwd_chunked then
- * reports the actual error.
+ * reports the actual error. For the tcgen05 kernel with more (batch row, value
+ * head) units than the current device has SMs, this is the workspace that lets
+ * it spread the units' chunks evenly over the SMs (it depends on the device's
+ * SM count); that kernel also runs with less, one CTA per unit.
  */
 GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv,
                               int gate_mode, int dtype);
@@ -165,9 +168,12 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  * gate on tcgen05 (where the chunk's state map is used in the equivalent
  * affine form S <- Gamma_C S + P S + R, O = Qh S + Uh, with P = -(K*Gamma_C/
  * Gamma)^T W, R = (K*Gamma_C/Gamma)^T U, Qh = (Q*Gamma) - M W, Uh = M U and M
- * the masked (Q*Gamma)(K/Gamma)^T above), for the per-channel gate on the
- * warp-level tensor cores. Both use fp16 operands, fp32 accumulation and an
- * fp32 carried state; q, k, v and the state must stay inside the fp16 range,
+ * the masked (Q*Gamma)(K/Gamma)^T above), for the per-channel gate too, with
+ * the decays carried by the Gram's operands (K exp(G - G_31), Q exp(G - G_31),
+ * K exp(G_31 - G), G the in-chunk prefix per key channel and G_31 its value at
+ * the chunk's row 31); with the layer options (gdr_fwd_chunked_norm) the
+ * per-channel gate runs on the warp-level tensor cores. All use fp16 operands,
+ * fp32 accumulation and an fp32 carried state; q, k, v and the state must stay inside the fp16 range,
  * |x| < 6.5e4 (both kernels count violations, see gdr_fused_error_counts;
  * the call still returns GDR_OK). Other shapes and fp32 inputs run fp32 CUDA-core kernels, which
  * take at most 65535 batch rows (else GDR_ERR_UNSUPPORTED).
@@ -176,7 +182,12 @@ GDR_API size_t gdr_fwd_workspace_size(int B, int T, int Hk, int Hv, int Dk, int 
  * workspace: device buffer of at least gdr_fwd_workspace_size(...) bytes,
  * 256-byte aligned, owned by the caller; may be NULL when that size is 0.
  * Its contents on entry are ignored. Two calls that overlap in time on the
- * GPU must not share one workspace.
+ * GPU must not share one workspace. With the tcgen05 kernel and more units
+ * than SMs it holds, per CTA boundary, a flag and the state of the unit cut
+ * there: the first CTA runs the unit's first chunks and hands its state over,
+ * the other runs the rest; each launch tags its flags, so stale contents are
+ * harmless. A NULL or smaller workspace is not an error there: the kernel
+ * then runs one CTA per unit (in more than one wave of SMs).
  */
 GDR_API int gdr_fwd_chunked(const void *q, const void *k, const void *v, const float *g,
                     const float *beta, const float *h0, void *o, float *hT,

@@ -177,3 +177,29 @@ def test_channel_gate_repeated_calls_are_bitwise_identical():
     o2, h2 = run_fwd(inp)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+# ------------------------------------------------------------------ more units than SMs
+@pytest.mark.parametrize("gate,T", [("scalar", 200), ("channel", 200), ("scalar", 130), ("scalar", 64)])
+def test_units_spread_over_the_sms_equal_one_cta_per_unit(gate, T):
+    """More (batch row, value head) units than SMs: with the workspace gdr_fwd_workspace_size
+    asks for, the kernel spreads the units' chunks evenly over the SMs, cutting some units
+    between two CTAs (the first part hands its state to the second through the workspace);
+    with none it runs one CTA per unit. Both do each chunk's arithmetic the same way and the
+    hand-off is an exact fp32 copy, so the results are equal bit for bit; sampled units also
+    meet the oracle."""
+    w = WORKLOADS["gdn_bf16"].with_(B=11, T=T, Hk=4, Hv=16, gate=gate,
+                                    g_mu=4.0 if gate == "channel" else 3.0, seed=1100 + T)
+    need = gdr.gdr_fwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, w.gate_mode, gdr.GDR_BF16)
+    assert need > 0   # 176 units on 148 SMs
+    inp = make_inputs(w, DEV)
+    o1, h1 = run_fwd(inp, out_dtype=torch.float32)   # the binding passes the workspace
+    none = torch.empty(0, dtype=torch.uint8, device=DEV)
+    o2, h2 = run_fwd(inp, out_dtype=torch.float32, workspace=none)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    units = sample_units(w.B, w.Hv, 6, seed=3)
+    o_ref, s_ref = oracle_units(inp, units)
+    for n, (b, h) in enumerate(units):
+        assert rel_err(o1[b, :, h], o_ref[n]) <= TOL["bf16"], (b, h)
+        assert rel_err(h1[b, h], s_ref[n]) <= TOL["bf16"], (b, h)
