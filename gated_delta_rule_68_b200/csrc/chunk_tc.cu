@@ -319,6 +319,19 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
     const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
     const int p = 32 * q4 + lane;     // row of the 128-row products owned by this thread
     const int hf = (warp >> 2) & 1;   // which half of that row's columns this thread takes
+    // Without a schedule the CTA's one unit is blockIdx.x: its batch row, heads, and sequence
+    // (tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor maps, batch index tbb
+    // and token offset tt0). Packed input: sequence b of cu_seqlens (clamped into the token
+    // axis); the rows of its last chunk past its end are zeroed when the chunk is converted,
+    // since the loaded tile holds the next sequence there.
+    const int u_bh = blockIdx.x, u_b = u_bh / a.Hv, u_h = u_bh % a.Hv, u_hk = u_h / (a.Hv / a.Hk);
+    int u_T = a.T, u_tbb = u_b, u_tt0 = 0;
+    long u_tok0 = (long)u_b * a.T;
+    if (a.cu_seqlens) {
+        const int s0 = min(max(a.cu_seqlens[u_b], 0), a.T), s1 = min(max(a.cu_seqlens[u_b + 1], s0), a.T);
+        u_T = s1 - s0, u_tbb = 0, u_tt0 = s0, u_tok0 = s0;
+    }
+    const int u_NC = (u_T + C - 1) / C;
     // The CTA's work, as pieces (unit, chunks [c0, c1)). Without a schedule (a.sched_len == 0)
     // one piece: the whole unit blockIdx.x. With one (fixed-length sequences, more units than
     // SMs), the units' chunks are laid end to end and cut into runs of a.sched_len
@@ -388,20 +401,17 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // One piece: unit pu, chunks [pc0, pc1) (pc1 < 0: all of them), the CTA's step count
         // at its first chunk gsb.
         auto chunk_piece = [&](const int pu, const int pc0, const int pc1, const int gsb) {
-            const int bh = pu, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
-            // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
-            // maps, batch index tbb and token offset tt0. Packed input: sequence b of cu_seqlens
-            // (clamped into the token axis); the rows of its last chunk past its end are zeroed
-            // when the chunk is converted, since the loaded tile holds the next sequence there.
-            int T = a.T, tbb = b, tt0 = 0;
-            long tok0 = (long)b * a.T;
-            if (a.cu_seqlens) {
-                const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
-                T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
-            }
-            const int NC = (T + C - 1) / C;
+            // The piece's unit: without a schedule the kernel-level values (computed before the
+            // groups split, which keeps the state group's registers within budget); with one,
+            // fixed-length sequences.
+            const int bh = SCHED ? pu : u_bh;
+            const int b = SCHED ? bh / a.Hv : u_b, h = SCHED ? bh % a.Hv : u_h;
+            const int hk = SCHED ? h / (a.Hv / a.Hk) : u_hk;
+            const int T = SCHED ? a.T : u_T, tbb = SCHED ? b : u_tbb, tt0 = SCHED ? 0 : u_tt0;
+            const long tok0 = SCHED ? (long)b * a.T : u_tok0;
+            const int NC = SCHED ? nc_unit : u_NC;
             const int c0 = pc0, c1 = pc1 < 0 ? NC : pc1;
-            (void)hk, (void)tbb, (void)tt0;
+            (void)hk, (void)tbb, (void)tt0, (void)tok0, (void)T;
         for (int c = c0; c < c1; ++c) {
             const int gs = gsb + (c - c0);
             const int sb = gs & 1;
@@ -734,20 +744,17 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // One piece: unit pu, chunks [pc0, pc1) (pc1 < 0: all of them), its kind, and the CTA's
         // step count at its first chunk gsb.
         auto state_piece = [&](const int pu, const int pc0, const int pc1, const int pkind, const int gsb) {
-            const int bh = pu, b = bh / a.Hv, h = bh % a.Hv, hk = h / (a.Hv / a.Hk);
-            // This unit's sequence: tokens tok0 .. tok0 + T - 1 of the token axis; in the tensor
-            // maps, batch index tbb and token offset tt0. Packed input: sequence b of cu_seqlens
-            // (clamped into the token axis); the rows of its last chunk past its end are zeroed
-            // when the chunk is converted, since the loaded tile holds the next sequence there.
-            int T = a.T, tbb = b, tt0 = 0;
-            long tok0 = (long)b * a.T;
-            if (a.cu_seqlens) {
-                const int s0 = min(max(a.cu_seqlens[b], 0), a.T), s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
-                T = s1 - s0, tbb = 0, tt0 = s0, tok0 = s0;
-            }
-            const int NC = (T + C - 1) / C;
+            // The piece's unit: without a schedule the kernel-level values (computed before the
+            // groups split, which keeps the state group's registers within budget); with one,
+            // fixed-length sequences.
+            const int bh = SCHED ? pu : u_bh;
+            const int b = SCHED ? bh / a.Hv : u_b, h = SCHED ? bh % a.Hv : u_h;
+            const int hk = SCHED ? h / (a.Hv / a.Hk) : u_hk;
+            const int T = SCHED ? a.T : u_T, tbb = SCHED ? b : u_tbb, tt0 = SCHED ? 0 : u_tt0;
+            const long tok0 = SCHED ? (long)b * a.T : u_tok0;
+            const int NC = SCHED ? nc_unit : u_NC;
             const int c0 = pc0, c1 = pc1 < 0 ? NC : pc1;
-            (void)hk, (void)tbb, (void)tt0;
+            (void)hk, (void)tbb, (void)tt0, (void)tok0, (void)T;
         auto issue_loads = [&](int c, int gs) {
             const int sb = gs & 1;
             const uint32_t stg = sb0 + sb * STG_BYTES, bl = bar(B_LD0 + sb);
