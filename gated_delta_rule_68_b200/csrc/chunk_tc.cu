@@ -117,6 +117,9 @@ constexpr uint32_t TM_S = 0, TM_O = 128, TM_G = 192, TM_X = 256, TM_Y = 320, TM_
 // parity: beta [64], exp(G_31) [128], Gamma_C [128], exp(G_C - G_31) [128]; then the
 // gate pass's per-row-group channel sums [4][128].
 constexpr uint32_t OFF_KB = OFF_ST16;
+// Scalar gate: the same region holds Kt = diag(Gamma_C / Gamma) K ([64][128] fp16, two 64-column
+// atoms of 8 KB) and diag(Gamma) ([64][64] fp16), written while the inverse's chains run.
+constexpr uint32_t OFF_KT = OFF_ST16, OFF_DG = OFF_ST16 + 16384;
 constexpr int KV_BETA = 0, KV_E31 = 64, KV_GC = 192, KV_ECM = 320, KV_SET = 448, KV_TOT = 2 * KV_SET;
 static_assert(OFF_VEC + (KV_TOT + 4 * 128) * 4 <= SMEM_USED, "per-channel vectors must fit the vector region");
 
@@ -611,6 +614,32 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     chain_next(c0, c1, Dt(0), LDT16, lane);
                     st_tblock<GATE>(sm, 48, 0, c0, c1, 1.f, vc, lane);
                 }
+            } else if (GATE == 0) {
+                // Meanwhile the other half (CUDA cores only, so the chains keep the tensor pipe):
+                // Kt = diag(Gamma_C / Gamma) K into its own tile, and diag(Gamma). The previous
+                // chunk's products that read both are done (waited before level 0).
+                const int ht = gt - GT / 2;   // 0 .. 127
+#pragma unroll
+                for (int jj = 0; jj < 1024 / (GT / 2); ++jj) {
+                    const int e = ht + (GT / 2) * jj, tok = (e >> 3) & 63;
+                    const float f = vc[V_F + tok];
+                    uint4 u = *(reinterpret_cast<const uint4 *>(stgp + (e >> 9) * 16384) + (e & 511));
+                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 x = __half22float2(hh[k]);
+                        hh[k] = __floats2half2_rn(x.x * f, x.y * f);
+                    }
+                    *(reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192) + (e & 511)) = u;
+                }
+#pragma unroll
+                for (int jj = 0; jj < 512 / (GT / 2); ++jj) {
+                    const int e = ht + (GT / 2) * jj, r = e >> 3, j = e & 7;
+                    float x[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? vc[V_GAM + r] : 0.f;
+                    st_chunk8(sb0 + swz_chunk(r, j, OFF_DG), x);
+                }
             }
             fence_proxy_async();
             named_bar_sync(1, GT);
@@ -642,23 +671,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_U16), v + 32 + 8 * j);
             }
-            // K -> Kt = diag(Gamma_C / Gamma) K in place (the W product is done with K); per-channel
-            // gate: Kt = Kb diag(exp(G_C - G_31)) into the K slot (Ks is done with too)
+            // Per-channel gate: Kt = Kb diag(exp(G_C - G_31)) into the K slot (the W product is done
+            // with Ks), and the identity in diag(Gamma)'s place into the dead V tile. (The scalar
+            // gate built Kt and diag(Gamma) during the chains.)
+            if (GATE == 1) {
 #pragma unroll
-            for (int jj = 0; jj < 1024 / GT; ++jj) {
-                const int e = gt + GT * jj, tok = (e >> 3) & 63;
-                uint4 *pch = reinterpret_cast<uint4 *>(stgp + (e >> 9) * 16384) + (e & 511);
-                if (GATE == 0) {
-                    const float f = vc[V_F + tok];
-                    uint4 u = *pch;
-                    __half2 *hh = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 x = __half22float2(hh[k]);
-                        hh[k] = __floats2half2_rn(x.x * f, x.y * f);
-                    }
-                    *pch = u;
-                } else {
+                for (int jj = 0; jj < 1024 / GT; ++jj) {
+                    const int e = gt + GT * jj, tok = (e >> 3) & 63;
+                    uint4 *pch = reinterpret_cast<uint4 *>(stgp + (e >> 9) * 16384) + (e & 511);
                     // physical 16-byte chunk e % 8 of row tok holds key channels 8 ((e % 8) ^ (tok % 8)) ..
                     const int ch0 = 64 * (e >> 9) + 8 * ((e & 7) ^ (tok & 7));
                     uint4 u = *(reinterpret_cast<const uint4 *>(sm + OFF_KB + sb * 16384 + (e >> 9) * 8192) + (e & 511));
@@ -673,15 +693,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     }
                     *pch = u;
                 }
-            }
-            // diag(Gamma) [r][j] (per-channel gate: the identity) into the dead V tile
 #pragma unroll
-            for (int jj = 0; jj < 512 / GT; ++jj) {
-                const int e = gt + GT * jj, r = e >> 3, j = e & 7;
-                float x[8];
+                for (int jj = 0; jj < 512 / GT; ++jj) {
+                    const int e = gt + GT * jj, r = e >> 3, j = e & 7;
+                    float x[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? (GATE ? 1.f : vc[V_GAM + r]) : 0.f;
-                st_chunk8(stg + STG_V + swz_chunk(r, j, 0), x);
+                    for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? 1.f : 0.f;
+                    st_chunk8(stg + STG_V + swz_chunk(r, j, 0), x);
+                }
             }
             tc_fence_before();
             fence_proxy_async();
@@ -695,12 +714,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_ss(tb + TM_S, sdesc(sb0 + OFF_U16 + s * 32, 16, 1024), sdesc(stg + s * 2048, 16384, 1024),
-                           ID_R, s > 0);
+                    mma_ss(tb + TM_S, sdesc(sb0 + OFF_U16 + s * 32, 16, 1024),
+                           GATE ? sdesc(stg + s * 2048, 16384, 1024) : sdesc(sb0 + OFF_KT + s * 2048, 8192, 1024), ID_R,
+                           s > 0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_ss(tb + TM_X, sdesc(stg + STG_Q + s * 2048, 16384, 1024),
-                           sdesc(stg + STG_V + s * 32, 16, 1024), ID_QG, s > 0);
+                           GATE ? sdesc(stg + STG_V + s * 32, 16, 1024) : sdesc(sb0 + OFF_DG + s * 32, 16, 1024), ID_QG,
+                           s > 0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_ss(tb + TM_X, sdesc(sb0 + OFF_W16 + s * 32, 16, 1024), sdesc(sb0 + OFF_M16 + s * 32, 16, 1024),
@@ -712,8 +733,9 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 mma_commit(bar(B_P1));
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_ss(tb + TM_Y, sdesc(stg + s * 2048, 16384, 1024), sdesc(sb0 + OFF_W16 + s * 32, 16, 1024),
-                           ID_P, s > 0);
+                    mma_ss(tb + TM_Y,
+                           GATE ? sdesc(stg + s * 2048, 16384, 1024) : sdesc(sb0 + OFF_KT + s * 2048, 8192, 1024),
+                           sdesc(sb0 + OFF_W16 + s * 32, 16, 1024), ID_P, s > 0);
                 mma_commit(bar(B_P));
             }
         }
@@ -978,8 +1000,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
         // group leaves them in tensor memory, so neither needs a scaling on its way out.
         auto store_s16 = [&](int gsn) {
             if (GATE == 0) {
+                uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_ST16 + hf * 16384), S + 8 * j);
+                for (int j = 0; j < 32; ++j) w[j] = pack_h2(S[2 * j], S[2 * j + 1]);
+                tmem_st32(tmem_addr(tb, q4, TM_S16 + 32 * hf), w);
+                tmem_wait_st();
             } else {
                 const float4 *e4 = reinterpret_cast<const float4 *>(vec + (gsn & 1) * KV_SET + KV_E31 + 64 * hf);
                 uint32_t w[32];
@@ -1070,20 +1095,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
-                    if (GATE == 0)
-                        mma_ss(tb + TM_S, sdesc(sb0 + OFF_ST16 + koff, 16, 1024), sdesc(sb0 + OFF_P16 + koff, 16, 1024),
-                               ID_S, true);
-                    else
-                        mma_ts(tb + TM_S, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_P16 + koff, 16, 1024), ID_S, true);
+                    mma_ts(tb + TM_S, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_P16 + koff, 16, 1024), ID_S, true);
                 }
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
-                    const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
-                    if (GATE == 0)
-                        mma_ss(tb + TM_O, sdesc(sb0 + OFF_ST16 + koff, 16, 1024),
-                               sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024), ID_O, true);
-                    else
-                        mma_ts(tb + TM_O, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024), ID_O, true);
+                    mma_ts(tb + TM_O, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024), ID_O, true);
                 }
                 mma_commit(bar(B_ST));
             }
