@@ -549,6 +549,17 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 const uint32_t tile = (gt - GT / 2) < 64 ? OFF_TP : OFF_TPP;
                 const uint4 z = make_uint4(0, 0, 0, 0);
                 for (int j = 2 * (R + 1); j < 8; ++j) *reinterpret_cast<uint4 *>(sm + swz_chunk(u, j, tile)) = z;
+                if (GATE == 0) {   // and diag(Gamma) [r][j] for the Qh product (its previous reader is done)
+                    const int ht = gt - GT / 2;
+#pragma unroll
+                    for (int jj = 0; jj < 512 / (GT / 2); ++jj) {
+                        const int e = ht + (GT / 2) * jj, r = e >> 3, j = e & 7;
+                        float x[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? vc[V_GAM + r] : 0.f;
+                        st_chunk8(sb0 + swz_chunk(r, j, OFF_DG), x);
+                    }
+                }
             }
             named_bar_sync(1, GT);
 
@@ -616,29 +627,18 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 }
             } else if (GATE == 0) {
                 // Meanwhile the other half (CUDA cores only, so the chains keep the tensor pipe):
-                // Kt = diag(Gamma_C / Gamma) K into its own tile, and diag(Gamma). The previous
-                // chunk's products that read both are done (waited before level 0).
+                // Kt = diag(Gamma_C / Gamma) K into its own tile. The previous chunk's products
+                // that read it are done (waited before level 0).
                 const int ht = gt - GT / 2;   // 0 .. 127
 #pragma unroll
                 for (int jj = 0; jj < 1024 / (GT / 2); ++jj) {
                     const int e = ht + (GT / 2) * jj, tok = (e >> 3) & 63;
-                    const float f = vc[V_F + tok];
+                    const __half2 f = __float2half2_rn(vc[V_F + tok]);   // the fp16 product of fp16 values is exact
                     uint4 u = *(reinterpret_cast<const uint4 *>(stgp + (e >> 9) * 16384) + (e & 511));
                     __half2 *hh = reinterpret_cast<__half2 *>(&u);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 x = __half22float2(hh[k]);
-                        hh[k] = __floats2half2_rn(x.x * f, x.y * f);
-                    }
+                    for (int k = 0; k < 4; ++k) hh[k] = __hmul2(hh[k], f);
                     *(reinterpret_cast<uint4 *>(sm + OFF_KT + (e >> 9) * 8192) + (e & 511)) = u;
-                }
-#pragma unroll
-                for (int jj = 0; jj < 512 / (GT / 2); ++jj) {
-                    const int e = ht + (GT / 2) * jj, r = e >> 3, j = e & 7;
-                    float x[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) x[k] = (8 * j + k == r) ? vc[V_GAM + r] : 0.f;
-                    st_chunk8(sb0 + swz_chunk(r, j, OFF_DG), x);
                 }
             }
             fence_proxy_async();
@@ -1107,10 +1107,22 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             tc_fence_after();
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
             if (GATE == 0) {
-                float v[64];
-                tmem_ld32x2(tmem_addr(tb, q4, TM_S + 64 * hf), tmem_addr(tb, q4, TM_S + 64 * hf + 32), v);
+                // In two halves of 32 rows, each written to its 16 columns of the copy as soon as
+                // it is done (so the packed copy never sits beside the whole state in registers).
 #pragma unroll
-                for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    float v[32];
+                    tmem_ld32(tmem_addr(tb, q4, TM_S + 64 * hf + 32 * h2), v);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        S[32 * h2 + 2 * j] = fmaf(gC, S[32 * h2 + 2 * j], v[2 * j]);
+                        S[32 * h2 + 2 * j + 1] = fmaf(gC, S[32 * h2 + 2 * j + 1], v[2 * j + 1]);
+                        w[j] = pack_h2(S[32 * h2 + 2 * j], S[32 * h2 + 2 * j + 1]);
+                    }
+                    tmem_st16(tmem_addr(tb, q4, TM_S16 + 32 * hf + 16 * h2), w);
+                }
+                tmem_wait_st();
             } else {   // S <- diag(Gamma_C) S + (P S + R), row dk = 64 hf + i, in two halves of 32
                 const float4 *g4 = reinterpret_cast<const float4 *>(vec + (gs & 1) * KV_SET + KV_GC + 64 * hf);
 #pragma unroll
@@ -1128,7 +1140,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     }
                 }
             }
-            store_s16(gs + 1);
+            if (GATE) store_s16(gs + 1);
             // o rows 32 hf .. 32 hf + 31 of this chunk (column p of Qh S + Uh) into the o tile
             // (the P tile, dead until the next chunk) in the TMA 128-byte swizzle, then out by
             // TMA stores, which clip tokens past T. The partial last chunk of a packed
