@@ -105,6 +105,7 @@ KERNEL_SOURCES = {
     "tc_fwd_kernel": ("chunk_tc.cu", "tc_util.cuh", "mma_util.cuh", "common.cuh", "kernels.h"),
     "fused_fwd_kernel": ("chunk_mma.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
     "bwd_kernel": ("bwd.cu", "common.cuh", "kernels.h"),
+    "decode_kernel": ("decode.cu", "common.cuh", "kernels.h"),
 }
 
 

@@ -80,7 +80,7 @@ constexpr uint32_t STG_Q = 8192;                //   Q rows start at row 64 of e
 constexpr uint32_t STG_V = 32768;
 constexpr uint32_t OFF_P16 = 2 * STG_BYTES;     // P [dk_out][dk_in] fp16, 2 atoms of 16 KB
 constexpr uint32_t OFF_QH16 = OFF_P16 + 32768;  // Qh^T [dk][r] fp16
-constexpr uint32_t OFF_ST16 = OFF_QH16 + 16384; // S^T [dv][dk] fp16, 2 atoms of 16 KB
+constexpr uint32_t OFF_ST16 = OFF_QH16 + 16384; // 32 KB: Kt and diag(Gamma), or the per-channel gate's Kb tiles
 constexpr uint32_t OFF_R1 = OFF_ST16 + 32768;   // T' and T'' (8 KB each) and the inverse's scratch; then W^T, U^T
 constexpr uint32_t OFF_TP = OFF_R1;             // T diag(beta Gamma) [r][i] fp16
 constexpr uint32_t OFF_TPP = OFF_R1 + 8192;     // T diag(beta) [r][i] fp16
@@ -108,8 +108,9 @@ constexpr uint32_t SMEM_TC = SMEM_USED + 1024;
 static_assert(SMEM_TC <= 227 * 1024, "shared memory");
 
 // Tensor memory columns (512 allocated): the state product (R, then P S + R), the
-// o accumulator (Uh, then Qh S + Uh), the Gram, Qh^T, and W^T / U^T, then P;
-// per-channel gate: the fp16 copy of S^T (128 lanes x 128 fp16, two per column).
+// o accumulator (Uh, then Qh S + Uh), the Gram, Qh^T, and W^T / U^T, then P, and
+// the fp16 copy of S^T that the state batch reads as its A operand (128 lanes x
+// 128 fp16, two per column).
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_G = 192, TM_X = 256, TM_Y = 320, TM_S16 = 448;
 
 // Per-channel gate: the S^T region holds the Kb tiles of the two staging buffers
@@ -1106,7 +1107,15 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             wait(B_ST, gs & 1);
             tc_fence_after();
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
-            if (GATE == 0) {
+            if (GATE == 0 && NORM) {
+                // The layer instance's state group is its longer chain: one TMEM wait for all
+                // 64 columns (it has the registers for it).
+                float v[64];
+                tmem_ld32x2(tmem_addr(tb, q4, TM_S + 64 * hf), tmem_addr(tb, q4, TM_S + 64 * hf + 32), v);
+#pragma unroll
+                for (int i = 0; i < 64; ++i) S[i] = fmaf(gC, S[i], v[i]);
+                store_s16(gs + 1);
+            } else if (GATE == 0) {
                 // In two halves of 32 rows, each written to its 16 columns of the copy as soon as
                 // it is done (so the packed copy never sits beside the whole state in registers).
 #pragma unroll
