@@ -22,8 +22,9 @@ Other workloads (``--workload``): ``gva_gdn_bf16`` and ``kda_bf16`` (the same
 step on the grouped-value and per-channel-gate shapes), ``decode_bf16`` (one
 ``gdr_decode_step`` over the batch per step), ``gdn_layer_bf16`` (three short
 convolutions plus the forward with its q/k and output norms) and ``gdn_bwd_bf16``
-(one ``gdr_bwd`` call per step, against the fp32 ALU roofline). ``--T`` shortens
-a workload's sequences for profiling small cases.
+(one ``gdr_bwd_chunked`` call per step, the tensor-core chunked backward, against
+the measured tensor-core peak; the fp32 ``gdr_bwd`` is timed beside it). ``--T``
+shortens a workload's sequences for profiling small cases.
 
 ``--impl reference`` times that oracle alone (the reference arm): each step is
 a bounded sample of the workload on the host cores.
@@ -42,6 +43,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "gated-delta fwd tokens/s (B·T·Hv per sec) bf16 d=128; % of roofline"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -99,6 +101,18 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s) measured by a cuBLAS GEMM burst on this pool's B200s;
+    fp16 runs at the same nominal rate."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (bf16 cuBLAS burst; fp16 at the same nominal rate)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 # The sources each captured kernel is built from: a recorded DRAM figure stands only while
 # these files are unchanged.
 KERNEL_SOURCES = {
@@ -106,6 +120,7 @@ KERNEL_SOURCES = {
     "fused_fwd_kernel": ("chunk_mma.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
     "bwd_kernel": ("bwd.cu", "common.cuh", "kernels.h"),
     "decode_kernel": ("decode.cu", "common.cuh", "kernels.h"),
+    "bwdc_chunk_kernel": ("bwd_chunk.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
 }
 
 
@@ -490,6 +505,17 @@ def bwd_flops(w):
     return 20 * w.B * w.T * w.Hv * w.Dk * w.Dv
 
 
+def bwdc_flops(w):
+    """Tensor-core flops per call of the chunked backward, per (unit, 64-token chunk): the
+    forward pass's products (Gram [K; Q] K^T, W and U, R, Qh, Uh, P and the state batch),
+    the reverse scan's dS^T P and dO^T Qh, and the chunk kernel's 6400 m16n8k16 products
+    (Grams, W, U, U', dU', dM, dQ, dK3, dW, T^T dU', T^T dW, dT, T^T dT T^T, the dK terms)."""
+    fwd = 5 * 2 * 128 * 64 * 128 + 2 * 128 * 64 * 64 + 2 * 128 * 128 * 128 + 2 * 128 * 64 * 128
+    scan = 2 * 128 * 128 * 128 + 2 * 128 * 128 * 64
+    chunk = 6400 * 2 * 16 * 8 * 16
+    return w.B * w.Hv * ((w.T + 63) // 64) * (fwd + scan + chunk)
+
+
 def alu_peak_tflops(sm_mhz):
     """fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops per clock."""
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -520,8 +546,11 @@ def bwd_cpu_sample(w, target_s=12.0):
 
 
 def run_bwd_bench(args, w, wr, rank, world, local, dev):
-    """One step = one gdr_bwd call over the whole workload: the checkpointing forward pass and
-    the reverse sweep, every gradient written."""
+    """One step = one backward call over the whole workload, every gradient written: the
+    tensor-core chunked backward (gdr_bwd_chunked: forward pass storing the chunk maps, reverse
+    scan of the state gradient, per-chunk gradients) for the scalar gate with bf16 inputs and
+    d = 128, else the fp32 token-level gdr_bwd (checkpointing forward pass and reverse sweep).
+    The chunked line also times the fp32 path on the same inputs, outside the timed region."""
     import torch
     import torch.distributed as dist
     import gated_delta_rule_68_b200 as gdr
@@ -534,14 +563,17 @@ def run_bwd_bench(args, w, wr, rank, world, local, dev):
     out = {"dq": torch.empty(inp["q"].shape, **f32), "dk": torch.empty(inp["k"].shape, **f32),
            "dv": torch.empty(inp["v"].shape, **f32), "dg": torch.empty(inp["g"].shape, **f32),
            "dbeta": torch.empty(inp["beta"].shape, **f32), "dh0": torch.empty((w.B, w.Hv, w.Dk, w.Dv), **f32)}
-    need = gdr.gdr_bwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, w.gate_mode,
-                                      gdr.GDR_BF16 if w.dtype == "bf16" else gdr.GDR_FP32)
+    dt = gdr.GDR_BF16 if w.dtype == "bf16" else gdr.GDR_FP32
+    chunked = w.dtype == "bf16" and w.gate == "scalar" and w.Dk == 128 and w.Dv == 128
+    ws_size = gdr.gdr_bwd_chunked_workspace_size if chunked else gdr.gdr_bwd_workspace_size
+    need = ws_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, w.gate_mode, dt)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    bwd_fn = gdr.gdr_bwd_chunked if chunked else gdr.gdr_bwd
 
     def step(x):
-        gdr.gdr_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], x["do"], x["dhT"], workspace=ws,
-                    stream=stream, out=out)
+        bwd_fn(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], x["do"], x["dhT"], workspace=ws,
+               stream=stream, out=out)
 
     def barrier():
         if world > 1:
@@ -564,6 +596,29 @@ def run_bwd_bench(args, w, wr, rank, world, local, dev):
     barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, dev)
+
+    fp32_path = None
+    if chunked:   # the fp32 token-level path on the same inputs, for comparison (not the timed region)
+        need32 = gdr.gdr_bwd_workspace_size(w.B, w.T, w.Hk, w.Hv, w.Dk, w.Dv, w.gate_mode, dt)
+        ws32 = torch.empty(max(need32, 1), dtype=torch.uint8, device=dev)
+        out32 = {n: torch.empty_like(t) for n, t in out.items()}
+
+        def step32():
+            gdr.gdr_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], inp["do"], inp["dhT"],
+                        workspace=ws32, stream=stream, out=out32)
+
+        step32()
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(3):
+            step32()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        fp32_path = {"ms_per_step": max_over_ranks(f0.elapsed_time(f1) / 3, dev), "steps": 3,
+                     "kernel": "gdr_bwd (bwd_ckpt_kernel + bwd_kernel, fp32)"}
+        del ws32, out32
 
     e2e = None
     if not args.no_e2e:
@@ -602,25 +657,38 @@ def run_bwd_bench(args, w, wr, rank, world, local, dev):
         return 0
     clocks = clk.summary()
     peak_mhz = clocks.get("sm_max_mhz") or 1965
-    peak = alu_peak_tflops(peak_mhz)
-    flops = bwd_flops(w)
-    achieved = flops / (ms / 1e3) / 1e12
     hbm, hbm_kind = measured_peaks()
     alg = bwd_bytes(w)
     traffic, traffic_kernel = recorded_traffic(w.name)
     cpu = bwd_cpu_sample(w) if world == 1 and not args.no_cpu_baseline else None
+    if chunked:
+        # tensor-bound at the measured dense bf16 peak (fp16 runs at the same rate): the products'
+        # time there is above the HBM time of the backward's algorithmic bytes
+        flops = bwdc_flops(w)
+        tpk, tkind = measured_tensor_peak()
+        achieved = flops / (ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tpk, "unit": "TFLOP/s",
+                    "frac": achieved / tpk, "peak_source": tkind, "algorithmic_flops_per_launch": flops,
+                    "traffic": traffic, "traffic_kernel": traffic_kernel,
+                    "kernel": "gdr_bwd_chunked step (tc_fwd_kernel storing the chunk maps + bwdc_scan_kernel "
+                              "+ bwdc_chunk_kernel)"}
+    else:
+        peak = alu_peak_tflops(peak_mhz)
+        flops = bwd_flops(w)
+        achieved = flops / (ms / 1e3) / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak,
+                    "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 x {peak_mhz} MHz",
+                    "algorithmic_flops_per_launch": flops, "traffic": traffic, "traffic_kernel": traffic_kernel,
+                    "kernel": "gdr_bwd step (bwd_ckpt_kernel + bwd_kernel)"}
     line = {
         "metric": BWD_METRIC, "value": job_tokens_per_s(w.head_tokens, world, ms_max), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16" if chunked else "f32",
         "data": "synthetic (seeded CPU generator; inputs as the gdn_bf16 recipe; do N(0,1) bf16, "
                 "dhT 0.1 N(0,1) fp32)",
         "config": workload_config(w, world),
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak,
-                     "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 x {peak_mhz} MHz",
-                     "algorithmic_flops_per_launch": flops, "traffic": traffic, "traffic_kernel": traffic_kernel,
-                     "kernel": "gdr_bwd step (bwd_ckpt_kernel + bwd_kernel)"},
+        "roofline": roofline, "fp32_token_path": fp32_path,
         "hbm_roofline": {"algorithmic_bytes": alg, "achieved": alg / (ms / 1e3) / 1e9, "peak": hbm,
                          "frac": alg / (ms / 1e3) / 1e9 / hbm, "peak_source": hbm_kind},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "launches_per_step": launches / args.steps,

@@ -27,7 +27,8 @@ GDR_BF16, GDR_FP32, GDR_BF16_OUT_F32 = 0, 1, 2
 EXPORTS = ("gdr_version", "gdr_last_error", "gdr_kernel_launches", "gdr_fwd_workspace_size",
            "gdr_fwd_chunked", "gdr_decode_step", "gdr_fwd_chunked_noalloc", "gdr_fused_error_counts",
            "gdr_fwd_chunked_varlen", "gdr_causal_conv_silu", "gdr_rmsnorm_gated",
-           "gdr_fwd_chunked_norm", "gdr_bwd_workspace_size", "gdr_bwd")
+           "gdr_fwd_chunked_norm", "gdr_bwd_workspace_size", "gdr_bwd",
+           "gdr_bwd_chunked_workspace_size", "gdr_bwd_chunked")
 
 # Scratch held by gdr_fwd_chunked_noalloc (GDR_NOALLOC_SCRATCH_BYTES in include/gdr.h).
 GDR_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -78,6 +79,10 @@ def lib():
         L.gdr_bwd_workspace_size.argtypes = [i] * 8
         L.gdr_bwd.restype = i
         L.gdr_bwd.argtypes = [vp] * 14 + [i] * 8 + [vp, sz, vp]
+        L.gdr_bwd_chunked_workspace_size.restype = sz
+        L.gdr_bwd_chunked_workspace_size.argtypes = [i] * 8
+        L.gdr_bwd_chunked.restype = i
+        L.gdr_bwd_chunked.argtypes = [vp] * 14 + [i] * 8 + [vp, sz, vp]
         _lib = L
     return _lib
 
@@ -146,10 +151,25 @@ def gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
     return int(lib().gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype))
 
 
+def gdr_bwd_chunked_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) -> int:
+    return int(lib().gdr_bwd_chunked_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype))
+
+
 def gdr_bwd(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None, out=None):
     """Backward of the recurrence: fp32 gradients of sum(dout * o) + sum(dhT * hT) with respect
     to q, k, v, g, beta and h0, as a dict (dq, dk, dv, dg, dbeta, dh0). dout has q's dtype.
     out, if given, is such a dict of preallocated fp32 tensors to write into."""
+    return _bwd_call("gdr_bwd", gdr_bwd_workspace_size, q, k, v, g, beta, h0, dout, dhT, workspace, stream, out)
+
+
+def gdr_bwd_chunked(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None, out=None):
+    """The same gradients by the tensor-core chunked backward (scalar gate, bf16 inputs,
+    Dk = Dv = 128; fp16 operands, so of the forward's accuracy rather than fp32)."""
+    return _bwd_call("gdr_bwd_chunked", gdr_bwd_chunked_workspace_size, q, k, v, g, beta, h0, dout, dhT,
+                     workspace, stream, out)
+
+
+def _bwd_call(fn, ws_size, q, k, v, g, beta, h0, dout, dhT, workspace, stream, out):
     B, T, Hk, Dk = q.shape
     Hv, Dv = v.shape[2], v.shape[3]
     dt, _ = _dtype_code(q, None)
@@ -170,11 +190,11 @@ def gdr_bwd(q, k, v, g, beta, h0, dout, dhT=None, *, workspace=None, stream=None
         out = {n: torch.empty(s, **f32) for n, s in shapes.items()}
     for n, s in shapes.items():
         _need(out[n], n, torch.float32, s)
-    need = gdr_bwd_workspace_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dt)
+    need = ws_size(B, T, Hk, Hv, Dk, Dv, gate_mode, dt)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().gdr_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(dout), _ptr(dhT),
+    _check(getattr(lib(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(dout), _ptr(dhT),
                          *(_ptr(out[n]) for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0")),
                          B, T, Hk, Hv, Dk, Dv, gate_mode, dt, _ptr(workspace), ws_bytes, _stream(stream)))
     return out

@@ -299,10 +299,39 @@ __device__ __forceinline__ void st_tblock(uint8_t *sm, int R0, int I0, const flo
     }
 }
 
+// The backward's forward pass: 8 fp32 values as 8 fp16 at a 16-byte aligned global address.
+__device__ __forceinline__ void st_global_h8(void *gp, const float *v)
+{
+    uint4 u;
+    u.x = pack_h2(v[0], v[1]);
+    u.y = pack_h2(v[2], v[3]);
+    u.z = pack_h2(v[4], v[5]);
+    u.w = pack_h2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(gp) = u;
+}
+// Block (R0.., I0..) of T (two n8 tiles times s) into the unit's [64][64] fp16 T in global memory.
+__device__ __forceinline__ void st_tglobal(__half *tg, int R0, int I0, const float c0[4], const float c1[4], float s,
+                                           int lane)
+{
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const float *c = nt ? c1 : c0;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = R0 + g + 8 * hh, i = I0 + 8 * nt + 2 * t4;
+            *reinterpret_cast<uint32_t *>(tg + r * 64 + i) = pack_h2(s * c[2 * hh], s * c[2 * hh + 1]);
+        }
+    }
+}
+
 // NORM: the layer's options (compiled as a separate instance, so the plain forward runs
 // exactly its own code): q and k rows divided by sqrt(sum of squares + 1e-6) as they are
 // converted, and o rows replaced by o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
-template <typename TOut, bool NORM, int GATE, bool SCHED>
+// SAVE (scalar gate, one CTA per unit): the first pass of the chunked backward. Per chunk it
+// also writes the entering state S^T, P, Qh^T and T (unscaled, lower triangle and diagonal
+// blocks) to the caller's buffers as fp16, and stores no o.
+template <typename TOut, bool NORM, int GATE, bool SCHED, bool SAVE = false>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o)
@@ -422,6 +451,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             const uint32_t stg = sb0 + sb * STG_BYTES;
             uint8_t *stgp = sm + sb * STG_BYTES;
             const float *vc = vec + sb * VSET;
+            __half *tg = SAVE ? reinterpret_cast<__half *>(a.save_t) + ((size_t)bh * NC + c) * (C * C) : nullptr;
+            (void)tg;
             wait(B_CV0 + sb, (gs >> 1) & 1);
             // Gram epilogue: A (rows < 64) and M (rows 64..127), columns 32 hf .. 32 hf + 31
             wait(B_G0 + sb, (gs >> 1) & 1);
@@ -539,6 +570,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                         *reinterpret_cast<uint32_t *>(sm + INV_D + (uint32_t)((wq * 16 + r) * LDT16 + col) * 2u) =
                             pack_h2(x0, x1);
                         *reinterpret_cast<uint32_t *>(sm + OFF_TPP + swz_off(I0 + r, i, 0)) = pack_h2(w0, w1);
+                        if (SAVE) *reinterpret_cast<uint32_t *>(tg + (I0 + r) * C + i) = pack_h2(x0, x1);
                         if (GATE == 0) {
                             const float u0 = x0 * vc[V_BG + i], u1 = x1 * vc[V_BG + i + 1];
                             *reinterpret_cast<uint32_t *>(sm + OFF_TP + swz_off(I0 + r, i, 0)) = pack_h2(u0, u1);
@@ -583,13 +615,16 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     chain_start(c0, c1, Dt(1), LDT16, At(1, 0), LDA16, lane);
                     chain_next(c0, c1, Dt(0), LDT16, lane);
                     st_tblock<GATE>(sm, 16, 0, c0, c1, -1.f, vc, lane);
+                    if (SAVE) st_tglobal(tg, 16, 0, c0, c1, -1.f, lane);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
                     st_tblock<GATE>(sm, 32, 16, c0, c1, -1.f, vc, lane);
+                    if (SAVE) st_tglobal(tg, 32, 16, c0, c1, -1.f, lane);
                 } else if (wq == 1) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
                     st_tblock<GATE>(sm, 48, 32, c0, c1, -1.f, vc, lane);
+                    if (SAVE) st_tglobal(tg, 48, 32, c0, c1, -1.f, lane);
                     chain_start(c0, c1, Dt(2), LDT16, At(2, 1), LDA16, lane);
                     chain_next(c0, c1, Dt(1), LDT16, lane);
                     chain_next(c0, c1, At(1, 0), LDA16, lane);
@@ -598,6 +633,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
                     st_tblock<GATE>(sm, 32, 0, c0, c1, 1.f, vc, lane);
+                    if (SAVE) st_tglobal(tg, 32, 0, c0, c1, 1.f, lane);
                 } else if (wq == 2) {
                     chain_start(c0, c1, Dt(3), LDT16, At(3, 2), LDA16, lane);
                     chain_next(c0, c1, Dt(2), LDT16, lane);
@@ -607,6 +643,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int e = 0; e < 4; ++e) c0[e] -= u0[e], c1[e] -= u1[e];
                     chain_next(c0, c1, Dt(1), LDT16, lane);
                     st_tblock<GATE>(sm, 48, 16, c0, c1, 1.f, vc, lane);
+                    if (SAVE) st_tglobal(tg, 48, 16, c0, c1, 1.f, lane);
                 } else {
                     float q0[4], q1[4], h0[4], h1[4];
                     chain_start(q0, q1, Dt(3), LDT16, At(3, 2), LDA16, lane);   // Q = D3 A32 D2
@@ -625,6 +662,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     for (int e = 0; e < 4; ++e) c0[e] = u0[e] + h0[e] - c0[e], c1[e] = u1[e] + h1[e] - c1[e];
                     chain_next(c0, c1, Dt(0), LDT16, lane);
                     st_tblock<GATE>(sm, 48, 0, c0, c1, 1.f, vc, lane);
+                    if (SAVE) st_tglobal(tg, 48, 0, c0, c1, 1.f, lane);
                 }
             } else if (GATE == 0) {
                 // Meanwhile the other half (CUDA cores only, so the chains keep the tensor pipe):
@@ -1065,6 +1103,12 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     prefetch_l1(reinterpret_cast<const __nv_bfloat16 *>(a.z) +
                                 ((size_t)(tok0 + c * C + r) * a.Hv + h) * D + 32 * k);
             }
+            const size_t save_at = SAVE ? ((size_t)bh * NC + c) * D + p : 0;
+            if (SAVE) {   // the state entering chunk c: row p of S^T, columns 64 hf ..
+                __half *sg = reinterpret_cast<__half *>(a.save_s) + save_at * D + 64 * hf;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) st_global_h8(sg + 8 * j, S + 8 * j);
+            }
             // P and Qh of this chunk, out of tensor memory into the operand tiles
             wait(B_P1, gs & 1);
             tc_fence_after();
@@ -1073,6 +1117,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
+                if (SAVE) {   // row p of Qh^T, tokens 32 hf ..
+                    __half *qg = reinterpret_cast<__half *>(a.save_qh) + save_at * C + 32 * hf;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_global_h8(qg + 8 * j, v + 8 * j);
+                }
             }
             wait(B_P, gs & 1);
             if (issuer && c + 2 < c1) issue_loads(c + 2, gs + 2);   // chunk c's staging buffer is free
@@ -1085,6 +1134,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 64 * hf), tmem_addr(tb, q4, TM_Y + 64 * hf + 32), v);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
+                if (SAVE) {   // row p of P, columns 64 hf ..
+                    __half *pg = reinterpret_cast<__half *>(a.save_p) + save_at * D + 64 * hf;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) st_global_h8(pg + 8 * j, v + 8 * j);
+                }
             }
             const float gC = GATE ? 0.f : vec[(gs & 1) * V_SET + V_GC];
             tc_fence_before();
@@ -1266,7 +1320,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                 if (z != 0.f) *reinterpret_cast<volatile int *>(&range_sh) = 1;
             }
             named_bar_sync(2, GT);
-            if (issuer && tile) {
+            if (!SAVE && issuer && tile) {
                 constexpr int EPB = 128 / sizeof(TOut);
                 // the normalised bf16 o tile is in the Qh tile
                 const uint32_t src = (NORM && a.z && sizeof(TOut) == 2) ? OFF_QH16 : OFF_P16;
@@ -1275,7 +1329,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     tma_store_4d(&map_o, k * EPB, h, tt0 + c * C, tbb, sb0 + src + k * C * 128);
             }
             if (c + 2 < c1) ready(c + 2, gs + 2, gbn);
-            if (issuer) tma_store_wait_read();   // the o tile is read before the next P tile is written
+            if (!SAVE && issuer) tma_store_wait_read();   // the o tile is read before the next P tile is written
             named_bar_sync(2, GT);
         }
         if (issuer) tma_store_wait_all();
@@ -1335,14 +1389,18 @@ cudaError_t launch_tc_t(const FwdArgs &a, cudaStream_t st)
     CUtensorMap mq, mk, mv, mo;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed input: one batch row of T tokens
     if (!make_map(&mq, a.q, mb, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, mb, a.T, a.Hk, 64, false, true) ||
-        !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true) ||
-        !make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
+        !make_map(&mv, a.v, mb, a.T, a.Hv, 64, false, true))
+        return cudaErrorInvalidValue;
+    if (a.save_s) mo = mq;   // the backward's forward pass stores no o (the map is never used)
+    else if (!make_map(&mo, a.o, mb, a.T, a.Hv, 128 / sizeof(TOut), sizeof(TOut) == 4, true))
         return cudaErrorInvalidValue;
     // The layer's options and the per-channel gate are separate instances, and so is the
     // wrap-around schedule, so that a call without them runs the same code as before they existed.
     auto kernel = a.sched_len ? (a.gate_mode ? tc_fwd_kernel<TOut, false, 1, true> : tc_fwd_kernel<TOut, false, 0, true>)
                   : a.gate_mode ? tc_fwd_kernel<TOut, false, 1, false>
-                  : (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true, 0, false> : tc_fwd_kernel<TOut, false, 0, false>;
+                  : (a.qk_l2norm || a.z) ? tc_fwd_kernel<TOut, true, 0, false>
+                  : a.save_s             ? tc_fwd_kernel<TOut, false, 0, false, true>
+                                         : tc_fwd_kernel<TOut, false, 0, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
     const long units = (long)a.B * a.Hv, steps = units * ((a.T + C - 1) / C);

@@ -66,7 +66,7 @@ int set_failure(int status, const char *msg) { return fail(status, "%s", msg); }
 
 extern "C" {
 
-int gdr_version(void) { return 200; }
+int gdr_version(void) { return 300; }
 
 const char *gdr_last_error(void) { return g_err; }
 
@@ -293,6 +293,62 @@ int gdr_bwd(const void *q, const void *k, const void *v, const float *g, const f
     if (e == cudaSuccess) e = gdr::launch_bwd(a, workspace, s);
     if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
     g_launches += 2;
+    return GDR_OK;
+}
+
+size_t gdr_bwd_chunked_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype)
+{
+    if (check_common(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype) != GDR_OK) return 0;
+    gdr::BwdArgs a{};
+    a.B = B; a.T = T; a.Hk = Hk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.gate_mode = gate_mode; a.dtype = dtype;
+    return (B == 0 || T == 0 || !gdr::bwdc_supported(a)) ? 0 : gdr::bwdc_workspace_size(a);
+}
+
+int gdr_bwd_chunked(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    const float *h0, const void *dout, const float *dhT, float *dq, float *dk, float *dv, float *dg,
+                    float *dbeta, float *dh0, int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode, int dtype,
+                    void *workspace, size_t workspace_bytes, void *stream)
+{
+    int st = check_common(B, T, Hk, Hv, Dk, Dv, gate_mode, dtype);
+    if (st != GDR_OK) return st;
+    gdr::BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0; a.dout = dout; a.dhT = dhT;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.dh0 = dh0;
+    a.B = B; a.T = T; a.Hk = Hk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.gate_mode = gate_mode; a.dtype = dtype;
+    if (!gdr::bwdc_supported(a))
+        return fail(GDR_ERR_UNSUPPORTED, "the chunked backward needs the scalar gate, bf16 inputs and Dk = Dv = 128");
+    const bool work = B > 0 && T > 0;
+    if (B > 0 && !dh0) return fail(GDR_ERR_INVALID_ARG, "dh0 must be non-NULL");
+    if (work && (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta))
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, dout and the gradient outputs must be non-NULL");
+    const void *ptrs[] = {q, k, v, g, beta, h0, dout, dhT, dq, dk, dv, dg, dbeta, dh0, workspace};
+    const char *names[] = {"q", "k", "v", "g", "beta", "h0", "dout", "dhT", "dq", "dk", "dv", "dg", "dbeta", "dh0",
+                           "workspace"};
+    for (int i = 0; i < 15; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(GDR_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!work) {   // dh0 = dhT (or zeros); no token, no other gradient
+        if (B > 0) {
+            const size_t bytes = (size_t)B * Hv * Dk * Dv * sizeof(float);
+            cudaError_t e = dhT ? cudaMemcpyAsync(dh0, dhT, bytes, cudaMemcpyDeviceToDevice, s)
+                                : cudaMemsetAsync(dh0, 0, bytes, s);
+            if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA: %s", cudaGetErrorString(e));
+        }
+        return GDR_OK;
+    }
+    const long cus = (long)B * Hv * ((T + 63) / 64);
+    if (cus > 2147483647L)
+        return fail(GDR_ERR_UNSUPPORTED, "the chunked backward takes at most 2^31 - 1 (unit, chunk) pairs");
+    const size_t need = gdr::bwdc_workspace_size(a);
+    if (!workspace || workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, workspace_bytes,
+                    workspace ? "" : " (NULL)");
+    const size_t nqk = (size_t)B * T * Hk * Dk * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(dq, 0, nqk, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nqk, s);
+    if (e == cudaSuccess) e = gdr::launch_bwdc(a, workspace, s);
+    if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
+    g_launches += 3;
     return GDR_OK;
 }
 

@@ -40,6 +40,10 @@ struct FwdArgs {
     unsigned long long sched_tag = 0;
     unsigned long long *sched_flags = nullptr;
     float *sched_states = nullptr;
+    // tcgen05 kernel, scalar gate: the chunked backward's forward pass. Per (unit, chunk),
+    // fp16: the entering state S^T [Dv][Dk], P [Dk][Dk], Qh^T [Dk][64] and T [64][64] (the
+    // lower triangle; entries above the diagonal blocks are not written). No o is stored.
+    void *save_s = nullptr, *save_p = nullptr, *save_qh = nullptr, *save_t = nullptr;
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
@@ -80,6 +84,12 @@ struct BwdArgs {
 bool bwd_supported(const BwdArgs &a);
 size_t bwd_workspace_size(const BwdArgs &a);
 cudaError_t launch_bwd(const BwdArgs &a, void *ws, cudaStream_t st);
+// Chunked backward on tensor cores (bwd_chunk.cu): scalar gate, bf16 inputs, Dk = Dv = 128.
+// dq and dk are accumulated with atomics and must be zero on entry; dv, dg, dbeta and dh0
+// are written once.
+bool bwdc_supported(const BwdArgs &a);
+size_t bwdc_workspace_size(const BwdArgs &a);
+cudaError_t launch_bwdc(const BwdArgs &a, void *ws, cudaStream_t st);
 
 // fp32 CUDA-core chunked forward (three kernels). Needs simt_workspace_size() bytes.
 size_t simt_workspace_size(const FwdArgs &a);

@@ -119,6 +119,36 @@ GDR_API int gdr_bwd(const void *q, const void *k, const void *v, const float *g,
                     int gate_mode, int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Chunked backward on tensor cores (NextTransformer, "Source notes", "Linear
+ * attention": the gdn update's first-order backward). Same gradients, arguments,
+ * layouts and outputs as gdr_bwd, for the scalar gate with bf16 inputs
+ * (GDR_BF16 or GDR_BF16_OUT_F32: q, k, v and dout bf16) and Dk = Dv = 128; other
+ * sizes or modes return GDR_ERR_UNSUPPORTED (gdr_bwd takes them).
+ *
+ * Three passes, chunks of 64 tokens: the tcgen05 forward stores each chunk's
+ * entering state, its P, Qh and T = (I + A)^-1 (the chunk map of gdr_fwd_chunked)
+ * in the workspace; a reverse scan over the chunks carries the state gradient
+ * dS <- Gamma_C dS + P^T dS + Qh^T dout, the transposed chunk map, and stores it per
+ * chunk; then every chunk forms its own gradients from its entering state, the
+ * gradient of the state it leaves, dout and its inputs, all chunks at once. The
+ * products take fp16 operands with fp32 accumulation (the forward's precision), so
+ * results are of the forward's accuracy class (about 1e-3 relative), not fp32:
+ * gdr_bwd is the fp32 path. q, k, v, dout and the states must stay inside the fp16
+ * range. dq and dk are sums over CTAs (atomics), so they are repeatable to
+ * rounding only.
+ *
+ * workspace: device buffer of at least gdr_bwd_chunked_workspace_size(...) bytes
+ * (B * Hv * ceil(T / 64) * 120 KiB), owned by the caller; two calls that overlap
+ * in time must not share one. Asynchronous on `stream`.
+ */
+GDR_API size_t gdr_bwd_chunked_workspace_size(int B, int T, int Hk, int Hv, int Dk, int Dv, int gate_mode,
+                                              int dtype);
+GDR_API int gdr_bwd_chunked(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                            const float *h0, const void *dout, const float *dhT, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *dh0, int B, int T, int Hk, int Hv, int Dk, int Dv,
+                            int gate_mode, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Device-side failure counts of the tensor-core chunked kernels (bf16 inputs,
  * Dk = Dv = 128) on the current device, accumulated since the library was
  * loaded there. Either pointer may be NULL; returns the sum of the two.

@@ -173,11 +173,11 @@ def test_empty_calls_launch_nothing(L):
 
 def bwd(L, q=A, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, h0=0, do=A + 20480, dhT=0,
         dq=A + 24576, dk=A + 28672, dv=A + 32768, dg=A + 36864, dbeta=A + 40960, dh0=A + 45056,
-        B=1, T=16, Hk=1, Hv=1, Dk=128, Dv=128, gate=0, dtype=0, ws=0, ws_bytes=0):
+        B=1, T=16, Hk=1, Hv=1, Dk=128, Dv=128, gate=0, dtype=0, ws=0, ws_bytes=0, fn="gdr_bwd"):
     vp = ctypes.c_void_p
     ptrs = [q, k, v, g, beta, h0, do, dhT, dq, dk, dv, dg, dbeta, dh0]
-    return L.gdr_bwd(*(vp(p or None) for p in ptrs), B, T, Hk, Hv, Dk, Dv, gate, dtype, vp(ws or None),
-                     ws_bytes, None)
+    return getattr(L, fn)(*(vp(p or None) for p in ptrs), B, T, Hk, Hv, Dk, Dv, gate, dtype, vp(ws or None),
+                          ws_bytes, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -197,6 +197,35 @@ def bwd(L, q=A, k=A + 4096, v=A + 8192, g=A + 12288, beta=A + 16384, h0=0, do=A 
 def test_bwd_rejects(L, kw, status):
     assert bwd(L, **kw) == status
     assert len(gdr.gdr_last_error()) > 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(gate=1), gdr.GDR_ERR_UNSUPPORTED),                 # the per-channel gate: gdr_bwd
+    (dict(dtype=gdr.GDR_FP32), gdr.GDR_ERR_UNSUPPORTED),     # fp32 inputs: gdr_bwd
+    (dict(Dk=64, Dv=64), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(Hk=2, Hv=3), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dh0=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(do=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dk=0), gdr.GDR_ERR_INVALID_ARG),
+    (dict(dg=MIS), gdr.GDR_ERR_MISALIGNED),
+    (dict(), gdr.GDR_ERR_WORKSPACE),
+    (dict(ws=A + (1 << 24), ws_bytes=16), gdr.GDR_ERR_WORKSPACE),
+])
+def test_bwd_chunked_rejects(L, kw, status):
+    before = L.gdr_kernel_launches()
+    assert bwd(L, fn="gdr_bwd_chunked", **kw) == status
+    assert len(gdr.gdr_last_error()) > 0
+    assert L.gdr_kernel_launches() == before
+
+
+def test_bwd_chunked_workspace_size_rules(L):
+    # S^T, P and the state gradient [128][128], Qh^T [128][64] and T [64][64], fp16, per chunk
+    per_chunk = (3 * 128 * 128 + 128 * 64 + 64 * 64) * 2
+    assert L.gdr_bwd_chunked_workspace_size(2, 130, 1, 3, 128, 128, 0, 0) == 2 * 3 * 3 * per_chunk
+    assert L.gdr_bwd_chunked_workspace_size(1, 64, 2, 2, 128, 128, 0, 2) == 2 * per_chunk
+    assert L.gdr_bwd_chunked_workspace_size(1, 64, 1, 1, 128, 128, 1, 0) == 0   # unsupported
+    assert L.gdr_bwd_chunked_workspace_size(0, 64, 1, 1, 128, 128, 0, 0) == 0
+    assert L.gdr_bwd_chunked_workspace_size(1, 0, 1, 1, 128, 128, 0, 0) == 0
 
 
 def test_bwd_workspace_size_rules(L):
