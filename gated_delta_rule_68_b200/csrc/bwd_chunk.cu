@@ -36,6 +36,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_util.cuh"
+#include "tc_util.cuh"
 
 namespace gdr {
 namespace {
@@ -120,127 +121,170 @@ __device__ __forceinline__ void zero_acc(float (*acc)[4])
 }
 
 // ------------------------------------------------------------------ pass 2: the reverse scan
-constexpr uint32_t SB_P = 0;                                 // P [128][LDD] fp16
-constexpr uint32_t SB_QH = D * LDD * 2;                      // Qh^T [128][LDC] fp16
-constexpr uint32_t SB_DO = SB_QH + D * LDC * 2;              // dO [64][LDD] fp16
-constexpr uint32_t SB_BUF = SB_DO + C * LDD * 2;
-constexpr uint32_t SMEM_SCAN = 2 * SB_BUF;
+// One CTA of 8 warps per (batch row, value head), on tcgen05. Per chunk, in reverse order:
+//     D = dO^T Qh + dS^T P          (128 x 128 fp32 accumulator in tensor memory)
+//     dS^T <- Gamma_C dS^T + D      (fp32, in registers: thread (p, hf) holds row p of dS^T,
+//                                    columns 64 hf .. 64 hf + 63)
+// A of the second product is the fp16 copy of dS^T in tensor memory (as the forward's state
+// batch reads S^T); P and Qh^T are the forward's 128-byte swizzled operand tiles, bulk-copied
+// from the workspace; dO comes by TMA and is converted to fp16 in place.
+constexpr uint32_t SC_P = 0;                  // P [dk_out][dk_in], 2 atoms of 16 KB
+constexpr uint32_t SC_QH = 32768;             // Qh^T [dk][token], 16 KB
+constexpr uint32_t SC_DO = SC_QH + 16384;     // dO [token][dv], 2 atoms of 8 KB
+constexpr uint32_t SC_BUF = SC_DO + 16384;    // one chunk's operands (64 KB)
+constexpr uint32_t SC_BAR = 2 * SC_BUF;       // mbarriers: loads (2), products, drain; TMEM base
+constexpr uint32_t SMEM_SCAN = SC_BAR + 64 + 1024;
+constexpr uint32_t TS_D = 0, TS_A = 128;      // tensor-memory columns: accumulator, fp16 copy of dS^T
+constexpr uint32_t ID_SQ = tcu::idesc_f16(128, 128, false, true, false);   // dO^T Qh
+constexpr uint32_t ID_SP = tcu::idesc_f16(128, 128, false, false, true);   // dS^T P
 
-// Warp w carries rows 16 w .. 16 w + 15 of dS^T ([Dv][Dk]) in acc[16][4]: tile nt holds
-// columns 8 nt .. 8 nt + 7 (the m16n8 accumulator layout), so the fp16 A fragment of
-// dS^T for k-step j is tiles 2 j and 2 j + 1 repacked.
-__global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws)
+__device__ unsigned int g_bwdc_timeouts;
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
-    extern __shared__ __align__(128) uint8_t sm[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, const __grid_constant__ CUtensorMap map_do)
+{
+    using namespace tcu;
+    extern __shared__ __align__(1024) uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, hf = warp >> 2, p = 32 * q4 + lane;
     const int unit = blockIdx.x, b = unit / a.Hv, h = unit % a.Hv;
     const int NC = (a.T + C - 1) / C;
-    const uint32_t sb = smem_u32(sm);
-    float acc[16][4];
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int dv = 16 * warp + g8 + 8 * (e >> 1), dk = 8 * nt + 2 * t4 + (e & 1);
-            acc[nt][e] = a.dhT ? a.dhT[((size_t)unit * D + dk) * D + dv] : 0.f;
+    auto bar = [&](int i) { return sb + SC_BAR + 8 * i; };   // 0, 1: loads; 2: products; 3: drain
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + SC_BAR + 32);
+    __shared__ int abort_sh;
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(bar(i), 1);
+        abort_sh = 0;
+    }
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tmem_slot;
+    auto wait = [&](int i, uint32_t parity) {
+        if (*reinterpret_cast<volatile int *>(&abort_sh)) return;
+        if (!mbar_wait_bounded(bar(i), parity)) {
+            *reinterpret_cast<volatile int *>(&abort_sh) = 1;
+            atomicAdd(&g_bwdc_timeouts, 1u);
         }
-    auto load = [&](int c, int buf) {
-        const uint32_t base = sb + buf * SB_BUF;
-        const __half *P = ws.p + ((size_t)unit * NC + c) * D * D;
-        for (int i = tid; i < D * 16; i += NT) {
-            const int r = i >> 4, j = i & 15;
-            cp_async16(base + SB_P + (r * LDD + 8 * j) * 2, P + r * D + 8 * j, 16);
-        }
-        const __half *Qh = ws.qh + ((size_t)unit * NC + c) * D * C;
-        for (int i = tid; i < D * 8; i += NT) {
-            const int r = i >> 3, j = i & 7;
-            cp_async16(base + SB_QH + (r * LDC + 8 * j) * 2, Qh + r * C + 8 * j, 16);
-        }
-        const __nv_bfloat16 *dO = reinterpret_cast<const __nv_bfloat16 *>(a.dout);
-        for (int i = tid; i < C * 16; i += NT) {
-            const int r = i >> 4, j = i & 15, t = c * C + r;
-            const bool ok = t < a.T;
-            cp_async16(base + SB_DO + (r * LDD + 8 * j) * 2,
-                       dO + (((size_t)b * a.T + (ok ? t : 0)) * a.Hv + h) * D + 8 * j, ok ? 16 : 0);
-        }
-        cp_async_commit();
     };
-    load(NC - 1, 0);
-    for (int c = NC - 1; c >= 0; --c) {
-        const int buf = (NC - 1 - c) & 1;
-        if (c > 0) {
-            load(c - 1, buf ^ 1);
-            cp_async_wait1();
-        } else {
-            cp_async_wait_all();
-        }
-        for (int i = tid; i < C * 16; i += NT) {   // this thread's dO copies, to fp16
-            const int r = i >> 4, j = i & 15;
-            bf16_to_fp16_16B(sm + buf * SB_BUF + SB_DO + (r * LDD + 8 * j) * 2);
-        }
-        float gsum = 0.f;   // Gamma_C of chunk c: exp of the sum of its g
-        for (int r = lane; r < C; r += 32) {
-            const int t = c * C + r;
+    auto issue_loads = [&](int c, int buf) {   // chunk c's operands into buffer buf
+        const uint32_t base = sb + buf * SC_BUF, bl = bar(buf);
+        const size_t cu = (size_t)unit * NC + c;
+        mbar_expect_tx(bl, SC_BUF);
+        bulk_g2s(base + SC_P, ws.p + cu * D * D, 32768, bl);
+        bulk_g2s(base + SC_QH, ws.qh + cu * D * C, 16384, bl);
+        tma_load_4d(base + SC_DO, &map_do, 0, h, c * C, b, bl);
+        tma_load_4d(base + SC_DO + 8192, &map_do, 64, h, c * C, b, bl);
+    };
+
+    // dS^T entering the reverse scan: dhT^T
+    float dS[64];
+    {
+        const float *src = a.dhT ? a.dhT + (size_t)unit * D * D + (size_t)(64 * hf) * D + p : nullptr;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) dS[i] = src ? __ldg(src + (size_t)i * D) : 0.f;
+    }
+    auto store_copy = [&]() {   // the fp16 copy of dS^T in tensor memory, the next products' A
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = pack_h2f(dS[2 * j], dS[2 * j + 1]);
+        tmem_st32(tmem_addr(tb, q4, TS_A + 32 * hf), w);
+        tmem_wait_st();
+    };
+    store_copy();
+    if (tid == 0) {
+        issue_loads(NC - 1, 0);
+        if (NC > 1) issue_loads(NC - 2, 1);
+    }
+    for (int s = 0; s < NC; ++s) {
+        const int c = NC - 1 - s, buf = s & 1;
+        // Gamma_C of chunk c: exp of the sum of its g (loads in flight during the wait below)
+        float gsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int t = c * C + lane + 32 * k;
             if (t < a.T) gsum += a.g[((size_t)b * a.T + t) * a.Hv + h];
         }
+        wait(buf, (s >> 1) & 1);
+        {   // this thread's 64 bytes of dO to fp16 (rows past T arrive as zeros)
+            uint8_t *d = sm + buf * SC_BUF + SC_DO + tid * 64;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) bf16_to_fp16_16B(d + 16 * k);
+        }
+        {   // dS_next of chunk c: row p of dS^T, columns 64 hf .., fp16
+            uint4 *dst = reinterpret_cast<uint4 *>(ws.ds + ((size_t)unit * NC + c) * D * D + (size_t)p * D + 64 * hf);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                dst[j] = make_uint4(pack_h2f(dS[8 * j], dS[8 * j + 1]), pack_h2f(dS[8 * j + 2], dS[8 * j + 3]),
+                                    pack_h2f(dS[8 * j + 4], dS[8 * j + 5]), pack_h2f(dS[8 * j + 6], dS[8 * j + 7]));
+        }
         const float gC = __expf(warp_sum(gsum));
+        fence_proxy_async();
+        tc_fence_before();
         __syncthreads();
-        // dS_next of chunk c, as fp16 [Dv][Dk]
-        __half *dsg = ws.ds + ((size_t)unit * NC + c) * D * D;
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t base = sb + buf * SC_BUF;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int r0 = 16 * warp + g8, col = 8 * nt + 2 * t4;
-            *reinterpret_cast<uint32_t *>(dsg + (size_t)r0 * D + col) = pack_h2f(acc[nt][0], acc[nt][1]);
-            *reinterpret_cast<uint32_t *>(dsg + (size_t)(r0 + 8) * D + col) = pack_h2f(acc[nt][2], acc[nt][3]);
+            for (int k = 0; k < 4; ++k)
+                mma_ss(tb + TS_D, sdesc(base + SC_DO + k * 2048, 8192, 1024), sdesc(base + SC_QH + k * 32, 16, 1024),
+                       ID_SQ, k > 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                mma_ts(tb + TS_D, tb + TS_A + 8 * k, sdesc(base + SC_P + k * 2048, 16384, 1024), ID_SP, true);
+            mma_commit(bar(2));
         }
-        uint32_t af[8][4];
+        wait(2, s & 1);
+        tc_fence_after();
+        if (tid == 0 && s + 2 < NC) issue_loads(c - 2, buf);   // the products are done with buf
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            af[j][0] = pack_h2f(acc[2 * j][0], acc[2 * j][1]);
-            af[j][1] = pack_h2f(acc[2 * j][2], acc[2 * j][3]);
-            af[j][2] = pack_h2f(acc[2 * j + 1][0], acc[2 * j + 1][1]);
-            af[j][3] = pack_h2f(acc[2 * j + 1][2], acc[2 * j + 1][3]);
-        }
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float v[32];
+            tmem_ld32(tmem_addr(tb, q4, TS_D + 64 * hf + 32 * h2), v);
+            uint32_t w[16];
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] *= gC;
-        const uint32_t base = sb + buf * SB_BUF;
-        // dS^T P: B = P stored [dk_out = k][dk_in = n]
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t bf[4];
-                ldsm_t(bf, b_kn(base + SB_P, LDD, 16 * np, 16 * j, lane));
-                mma(acc[2 * np], af[j], bf[0], bf[1]);
-                mma(acc[2 * np + 1], af[j], bf[2], bf[3]);
+            for (int j = 0; j < 16; ++j) {
+                dS[32 * h2 + 2 * j] = fmaf(gC, dS[32 * h2 + 2 * j], v[2 * j]);
+                dS[32 * h2 + 2 * j + 1] = fmaf(gC, dS[32 * h2 + 2 * j + 1], v[2 * j + 1]);
+                w[j] = pack_h2f(dS[32 * h2 + 2 * j], dS[32 * h2 + 2 * j + 1]);
             }
-        // dO^T Qh: A = dO^T (dO stored [token][dv]), B = Qh stored as Qh^T [dk = n][token = k]
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t a4[4];
-            ldsm_t(a4, a_tr(base + SB_DO, LDD, 16 * warp, 16 * j, lane));
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t bf[4];
-                ldsm(bf, b_nk(base + SB_QH, LDC, 16 * np, 16 * j, lane));
-                mma(acc[2 * np], a4, bf[0], bf[1]);
-                mma(acc[2 * np + 1], a4, bf[2], bf[3]);
-            }
+            tmem_st16(tmem_addr(tb, q4, TS_A + 32 * hf + 16 * h2), w);
         }
-        __syncthreads();   // the buffer is read before the next iteration's loads refill it
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
     }
+    {   // dh0 = dS entering chunk 0
+        float *dst = a.dh0 + (size_t)unit * D * D + (size_t)(64 * hf) * D + p;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int dv = 16 * warp + g8 + 8 * (e >> 1), dk = 8 * nt + 2 * t4 + (e & 1);
-            a.dh0[((size_t)unit * D + dk) * D + dv] = acc[nt][e];
-        }
+        for (int i = 0; i < 64; ++i) dst[(size_t)i * D] = dS[i];
+    }
+    if (tid == 0) {   // every product this thread issued has completed before the memory is freed
+        tc_fence_after();
+        mma_commit(bar(3));
+        mbar_wait_bounded(bar(3), 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tb, 256);
+    }
 }
 
 // ------------------------------------------------------------------ pass 3: per-chunk gradients
+// 8 warps; warp (rw, cw) = (warp & 1, warp >> 1) computes rows 32 rw .. 32 rw + 31 of every
+// product (two m16 blocks, mi = 0, 1) and columns 32 cw .. of the 128-wide ones, 16 cw .. of
+// the 64-wide ones: each fragment loaded from shared memory feeds two to four MMAs.
+constexpr int NTC = 256;
 constexpr uint32_t SZ_DT = C * LDD * 2;     // [64][136] fp16
 constexpr uint32_t SZ_ST = D * LDD * 2;     // [128][136] fp16
 constexpr uint32_t SZ_CT = C * LDC * 2;     // [64][72] fp16
@@ -251,19 +295,59 @@ constexpr uint32_t OC_T = OC_DS + SZ_ST;      // T [64][LDC]
 constexpr uint32_t OC_M = OC_T + SZ_CT;       // M, then dM * D [64][LDC]
 constexpr uint32_t OC_W = OC_M + SZ_CT;       // W, then dU' [64][LDD]
 constexpr uint32_t OC_U = OC_W + SZ_DT;       // U', then dT, then dB * D [64][LDC]
-constexpr uint32_t OC_VEC = OC_U + SZ_DT;     // vectors: G, Gamma, beta, f, dG, dbeta [64] each; scalars
-// vectors: G, Gamma, beta, f [64]; per column half of the warps, the row sums of dG and dbeta
-// [2][64] each; per warp, sum(dK3 * K) and sum(dS_next * S) [8] each (summed in a fixed order,
+constexpr uint32_t OC_VEC = OC_U + SZ_DT;
+// vectors: G, Gamma, beta, f [64]; per column quarter of the warps, the row sums of dG and dbeta
+// [4][64] each; per warp, sum(dK3 * K) and sum(dS_next * S) [8] each (summed in a fixed order,
 // so that dg and dbeta repeat bit for bit)
-constexpr int VG = 0, VGAM = 64, VBETA = 128, VF = 192, VDG = 256, VDB = 384, VT3 = 512, VSS = 520;
+constexpr int VG = 0, VGAM = 64, VBETA = 128, VF = 192, VDG = 256, VDB = 512, VT3 = 768, VSS = 776;
 constexpr uint32_t SMEM_CHUNK = OC_VEC + (VSS + 8) * 4;
 static_assert(SMEM_CHUNK <= 227 * 1024, "shared memory");
 
-__global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
+// acc[2][2 NP][4] += A (rows r0 .. r0 + 31, K = 16 KS) B (columns n0 .. n0 + 16 NP), as wgemm.
+// ascale(af, j, mi) may rescale the A fragment of k-step j, row block mi.
+template <int KS, int NP, bool AT, bool BT, typename AS>
+__device__ __forceinline__ void wgemm2(float (*acc)[2 * NP][4], uint32_t aB, int lda, int r0, uint32_t bB, int ldb,
+                                       int n0, int lane, AS ascale)
+{
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+        uint32_t af[2][4];
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+            if (AT) ldsm_t(af[mi], a_tr(aB, lda, r0 + 16 * mi, 16 * j, lane));
+            else ldsm(af[mi], a_rm(aB, lda, r0 + 16 * mi, 16 * j, lane));
+            ascale(af[mi], j, mi);
+        }
+#pragma unroll
+        for (int np = 0; np < NP; ++np) {
+            uint32_t bf[4];
+            if (BT) ldsm_t(bf, b_kn(bB, ldb, n0 + 16 * np, 16 * j, lane));
+            else ldsm(bf, b_nk(bB, ldb, n0 + 16 * np, 16 * j, lane));
+#pragma unroll
+            for (int mi = 0; mi < 2; ++mi) {
+                mma(acc[mi][2 * np], af[mi], bf[0], bf[1]);
+                mma(acc[mi][2 * np + 1], af[mi], bf[2], bf[3]);
+            }
+        }
+    }
+}
+struct NoScale2 {
+    __device__ __forceinline__ void operator()(uint32_t *, int, int) const {}
+};
+template <int N>
+__device__ __forceinline__ void zero2(float (*acc)[N][4])
+{
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int i = 0; i < N; ++i) acc[mi][i][0] = acc[mi][i][1] = acc[mi][i][2] = acc[mi][i][3] = 0.f;
+}
+
+__global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
 {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
-    const int rw = warp & 3, cw = warp >> 2, r0 = 16 * rw;
+    const int rw = warp & 1, cw = warp >> 1, r0 = 32 * rw;
     const int NC = (a.T + C - 1) / C;
     const int unit = blockIdx.x / NC, c = blockIdx.x % NC;
     const int b = unit / a.Hv, h = unit % a.Hv, hk = h / (a.Hv / a.Hk);
@@ -271,29 +355,31 @@ __global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
     float *vec = reinterpret_cast<float *>(sm + OC_VEC);
     const size_t cu = (size_t)unit * NC + c;
 
-    // ---- loads: q, k (key head), v, dO (value head) as bf16, rows past T zero; S^T, dS_next^T, T
+    // ---- loads, in two groups: q, k (key head), v, dO (value head) as bf16 with rows past T
+    // zero, and T; then S^T and dS_next^T, which arrive while the Grams, W and U are formed
     {
         const __nv_bfloat16 *src[4] = {reinterpret_cast<const __nv_bfloat16 *>(a.q),
                                        reinterpret_cast<const __nv_bfloat16 *>(a.k),
                                        reinterpret_cast<const __nv_bfloat16 *>(a.v),
                                        reinterpret_cast<const __nv_bfloat16 *>(a.dout)};
-        for (int i = tid; i < 4 * C * 16; i += NT) {
+        for (int i = tid; i < 4 * C * 16; i += NTC) {
             const int m = i >> 10, r = (i >> 4) & 63, j = i & 15, t = c * C + r;
             const bool ok = t < a.T;
             const int H = m < 2 ? a.Hk : a.Hv, hh = m < 2 ? hk : h;
             cp_async16(sb + m * SZ_DT + (r * LDD + 8 * j) * 2,
                        src[m] + (((size_t)b * a.T + (ok ? t : 0)) * H + hh) * D + 8 * j, ok ? 16 : 0);
         }
+        const __half *Tg = ws.t + cu * C * C;
+        for (int i = tid; i < C * 8; i += NTC) {
+            const int r = i >> 3, j = i & 7;
+            cp_async16(sb + OC_T + (r * LDC + 8 * j) * 2, Tg + r * C + 8 * j, 16);
+        }
+        cp_async_commit();
         const __half *S = ws.s + cu * D * D, *dS = ws.ds + cu * D * D;
-        for (int i = tid; i < D * 16; i += NT) {
+        for (int i = tid; i < D * 16; i += NTC) {
             const int r = i >> 4, j = i & 15;
             cp_async16(sb + OC_S + (r * LDD + 8 * j) * 2, S + r * D + 8 * j, 16);
             cp_async16(sb + OC_DS + (r * LDD + 8 * j) * 2, dS + r * D + 8 * j, 16);
-        }
-        const __half *Tg = ws.t + cu * C * C;
-        for (int i = tid; i < C * 8; i += NT) {
-            const int r = i >> 3, j = i & 7;
-            cp_async16(sb + OC_T + (r * LDC + 8 * j) * 2, Tg + r * C + 8 * j, 16);
         }
         cp_async_commit();
         if (tid < C) {
@@ -302,13 +388,13 @@ __global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
             vec[VG + tid] = ok ? a.g[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
             vec[VBETA + tid] = ok ? a.beta[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
         }
-        cp_async_wait_all();
-        for (int i = tid; i < 4 * C * 16; i += NT) {
+        cp_async_wait1();
+        for (int i = tid; i < 4 * C * 16; i += NTC) {
             const int m = i >> 10, r = (i >> 4) & 63, j = i & 15;
             bf16_to_fp16_16B(sm + m * SZ_DT + (r * LDD + 8 * j) * 2);
         }
         // T is lower triangular: clear what the forward left unwritten above the diagonal blocks
-        for (int i = tid; i < C * 8; i += NT) {
+        for (int i = tid; i < C * 8; i += NTC) {
             const int r = i >> 3, j = i & 7;
             __half *row = reinterpret_cast<__half *>(sm + OC_T) + r * LDC + 8 * j;
 #pragma unroll
@@ -333,76 +419,77 @@ __global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
         vec[VF + lane] = __expf(GL - x0);
         vec[VF + 32 + lane] = __expf(GL - x1);
     }
-    {   // sum(dS_next * S) over the whole state
-        float s = 0.f;
-        for (int i = tid; i < D * 16; i += NT) {
-            const int r = i >> 4, j = i & 15;
-            const __half2 *x = reinterpret_cast<const __half2 *>(sm + OC_S + (r * LDD + 8 * j) * 2);
-            const __half2 *y = reinterpret_cast<const __half2 *>(sm + OC_DS + (r * LDD + 8 * j) * 2);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 fx = __half22float2(x[e]), fy = __half22float2(y[e]);
-                s = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, s));
-            }
-        }
-        s = warp_sum(s);
-        if (lane == 0) vec[VSS + warp] = s;
-    }
     __syncthreads();
 
     const float *G = vec + VG, *Gam = vec + VGAM, *beta = vec + VBETA, *fv = vec + VF;
-    const int ra = r0 + g8, rb = ra + 8;   // this thread's two rows in every row block
+    // this thread's rows: row(mi, hi) = r0 + 16 mi + 8 hi + g8 (accumulator elements 2 hi, 2 hi + 1)
+    auto row = [&](int mi, int e) { return r0 + 16 * mi + g8 + 8 * (e >> 1); };
     auto dec = [&](int r, int i) { return r >= i ? __expf(G[r] - G[i]) : 0.f; };
-    // per-row partial sums of this thread (rows ra, rb), added to dG / dbeta at the end
-    float pg0 = 0.f, pg1 = 0.f, pb0 = 0.f, pb1 = 0.f, tot3 = 0.f;
-    auto rowdot = [&](const float (*acc)[4], uint32_t tile, int n0, float &s0, float &s1) {
-        // sum over this thread's columns of acc * tile (fp16 [64][LDD]) on rows ra and rb
+    // per-row partial sums of this thread, [mi][hi], added to dG / dbeta at the end
+    float pg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, tot3 = 0.f;
+    auto rowdot = [&](const float (*acc)[4][4], uint32_t tile, int n0, float (*s)[2]) {
+        // sum over this thread's columns of acc * tile (fp16 [64][LDD]) on its rows
         const __half *tp = reinterpret_cast<const __half *>(sm + tile);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int col = n0 + 8 * nt + 2 * t4;
-            const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(tp + ra * LDD + col));
-            const float2 y = __half22float2(*reinterpret_cast<const __half2 *>(tp + rb * LDD + col));
-            s0 = fmaf(acc[nt][0], x.x, fmaf(acc[nt][1], x.y, s0));
-            s1 = fmaf(acc[nt][2], y.x, fmaf(acc[nt][3], y.y, s1));
-        }
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int col = n0 + 8 * nt + 2 * t4;
+                const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(tp + row(mi, 0) * LDD + col));
+                const float2 y = __half22float2(*reinterpret_cast<const __half2 *>(tp + row(mi, 2) * LDD + col));
+                s[mi][0] = fmaf(acc[mi][nt][0], x.x, fmaf(acc[mi][nt][1], x.y, s[mi][0]));
+                s[mi][1] = fmaf(acc[mi][nt][2], y.x, fmaf(acc[mi][nt][3], y.y, s[mi][1]));
+            }
     };
-    auto store_h = [&](const float (*acc)[4], int ntn, uint32_t tile, int ld, int n0, float s) {
+    auto store_h = [&](const float (*acc)[4], int mi, int ntn, uint32_t tile, int ld, int n0, float sc) {
         __half *tp = reinterpret_cast<__half *>(sm + tile);
         for (int nt = 0; nt < ntn; ++nt) {
             const int col = n0 + 8 * nt + 2 * t4;
-            *reinterpret_cast<uint32_t *>(tp + ra * ld + col) = pack_h2f(s * acc[nt][0], s * acc[nt][1]);
-            *reinterpret_cast<uint32_t *>(tp + rb * ld + col) = pack_h2f(s * acc[nt][2], s * acc[nt][3]);
+            *reinterpret_cast<uint32_t *>(tp + row(mi, 0) * ld + col) = pack_h2f(sc * acc[nt][0], sc * acc[nt][1]);
+            *reinterpret_cast<uint32_t *>(tp + row(mi, 2) * ld + col) = pack_h2f(sc * acc[nt][2], sc * acc[nt][3]);
         }
     };
-    const int n128 = 64 * cw, n64 = 32 * cw;   // this warp's columns of 128- and 64-wide outputs
+    const int n128 = 32 * cw, n64 = 16 * cw;   // this warp's columns of 128- and 64-wide outputs
+    // per-row scalings of A fragments (rows g8 and g8 + 8 of block mi)
+    auto rowscale = [&](const float *v) {
+        return [=](uint32_t *af, int, int mi) {
+            const __half2 sa = __float2half2_rn(v[r0 + 16 * mi + g8]), sb2 = __float2half2_rn(v[r0 + 16 * mi + g8 + 8]);
+            hmul_frag(af[0], sa);
+            hmul_frag(af[1], sb2);
+            hmul_frag(af[2], sa);
+            hmul_frag(af[3], sb2);
+        };
+    };
 
     // ---- a: the Grams, M = tril(Q K^T * D) and Bm = tril(K K^T * D, -1)
-    float bm[4][4];
+    float bm[2][2][4];
     {
-        float qk[4][4], kk[4][4];
-        zero_acc<4>(qk);
-        zero_acc<4>(kk);
-        wgemm<8, 2, false, false>(qk, sb + OC_Q, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale());
-        wgemm<8, 2, false, false>(kk, sb + OC_K, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale());
+        float qk[2][2][4], kk[2][2][4];
+        zero2<2>(qk);
+        zero2<2>(kk);
+        wgemm2<8, 1, false, false>(qk, sb + OC_Q, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(kk, sb + OC_K, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale2());
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = e < 2 ? ra : rb, i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                const float d = dec(r, i);
-                qk[nt][e] *= d;
-                bm[nt][e] = r > i ? kk[nt][e] * d : 0.f;
-            }
-        store_h(qk, 4, OC_M, LDC, n64, 1.f);
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = row(mi, e), i = n64 + 8 * nt + 2 * t4 + (e & 1);
+                    const float d = dec(r, i);
+                    qk[mi][nt][e] *= d;
+                    bm[mi][nt][e] = r > i ? kk[mi][nt][e] * d : 0.f;
+                }
+            store_h(qk[mi], mi, 2, OC_M, LDC, n64, 1.f);
+        }
     }
     // ---- b: W = T diag(beta Gamma) K, U = T diag(beta) V, then U' = U - W S
     {
-        float w[8][4], u[8][4];
-        zero_acc<8>(w);
-        zero_acc<8>(u);
+        float w[2][4][4], u[2][4][4];
+        zero2<4>(w);
+        zero2<4>(u);
         auto colscale = [&](const float *s1, const float *s2) {
-            return [=](uint32_t *af, int j) {
+            return [=](uint32_t *af, int j, int) {
                 const int k0 = 16 * j + 2 * t4;
                 const __half2 lo = __floats2half2_rn(s1[k0] * (s2 ? s2[k0] : 1.f), s1[k0 + 1] * (s2 ? s2[k0 + 1] : 1.f));
                 const __half2 hi =
@@ -413,199 +500,250 @@ __global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
                 hmul_frag(af[3], hi);
             };
         };
-        wgemm<4, 4, false, true>(w, sb + OC_T, LDC, r0, sb + OC_K, LDD, n128, lane, colscale(beta, Gam));
-        wgemm<4, 4, false, true>(u, sb + OC_T, LDC, r0, sb + OC_V, LDD, n128, lane, colscale(beta, nullptr));
-        store_h(w, 8, OC_W, LDD, n128, 1.f);
+        wgemm2<4, 2, false, true>(w, sb + OC_T, LDC, r0, sb + OC_K, LDD, n128, lane, colscale(beta, Gam));
+        wgemm2<4, 2, false, true>(u, sb + OC_T, LDC, r0, sb + OC_V, LDD, n128, lane, colscale(beta, nullptr));
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) store_h(w[mi], mi, 4, OC_W, LDD, n128, 1.f);
+        cp_async_wait_all();   // S^T and dS_next^T
         __syncthreads();
+        {   // sum(dS_next * S) over the whole state
+            float s = 0.f;
+            for (int i = tid; i < D * 16; i += NTC) {
+                const int r = i >> 4, j = i & 15;
+                const __half2 *x = reinterpret_cast<const __half2 *>(sm + OC_S + (r * LDD + 8 * j) * 2);
+                const __half2 *y = reinterpret_cast<const __half2 *>(sm + OC_DS + (r * LDD + 8 * j) * 2);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 fx = __half22float2(x[e]), fy = __half22float2(y[e]);
+                    s = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, s));
+                }
+            }
+            s = warp_sum(s);
+            if (lane == 0) vec[VSS + warp] = s;
+        }
         const __half2 neg = __floats2half2_rn(-1.f, -1.f);
-        wgemm<8, 4, false, false>(u, sb + OC_W, LDD, r0, sb + OC_S, LDD, n128, lane, [=](uint32_t *af, int) {
+        wgemm2<8, 2, false, false>(u, sb + OC_W, LDD, r0, sb + OC_S, LDD, n128, lane, [=](uint32_t *af, int, int) {
             hmul_frag(af[0], neg);
             hmul_frag(af[1], neg);
             hmul_frag(af[2], neg);
             hmul_frag(af[3], neg);
         });
-        store_h(u, 8, OC_U, LDD, n128, 1.f);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) store_h(u[mi], mi, 4, OC_U, LDD, n128, 1.f);
     }
     __syncthreads();
     // ---- c: dU' = M^T dO + diag(f) K dS_next
     {
-        float du[8][4];
-        zero_acc<8>(du);
-        wgemm<4, 4, true, true>(du, sb + OC_M, LDC, r0, sb + OC_DO, LDD, n128, lane, NoScale());
-        const __half2 fa = __float2half2_rn(fv[ra]), fb = __float2half2_rn(fv[rb]);
-        wgemm<8, 4, false, false>(du, sb + OC_K, LDD, r0, sb + OC_DS, LDD, n128, lane, [=](uint32_t *af, int) {
-            hmul_frag(af[0], fa);
-            hmul_frag(af[1], fb);
-            hmul_frag(af[2], fa);
-            hmul_frag(af[3], fb);
-        });
-        store_h(du, 8, OC_W, LDD, n128, 1.f);   // W is dead
+        float du[2][4][4];
+        zero2<4>(du);
+        wgemm2<4, 2, true, true>(du, sb + OC_M, LDC, r0, sb + OC_DO, LDD, n128, lane, NoScale2());
+        wgemm2<8, 2, false, false>(du, sb + OC_K, LDD, r0, sb + OC_DS, LDD, n128, lane, rowscale(fv));
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) store_h(du[mi], mi, 4, OC_W, LDD, n128, 1.f);   // W is dead
     }
     __syncthreads();
     // ---- d: dM = tril(dO U'^T), stored as dM * D
     {
-        float dm[4][4];
-        zero_acc<4>(dm);
-        wgemm<8, 2, false, false>(dm, sb + OC_DO, LDD, r0, sb + OC_U, LDD, n64, lane, NoScale());
+        float dm[2][2][4];
+        zero2<2>(dm);
+        wgemm2<8, 1, false, false>(dm, sb + OC_DO, LDD, r0, sb + OC_U, LDD, n64, lane, NoScale2());
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = e < 2 ? ra : rb, i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                dm[nt][e] *= dec(r, i);
-            }
-        store_h(dm, 4, OC_M, LDC, n64, 1.f);   // M is dead
-    }
-    __syncthreads();
-    const bool va = c * C + ra < a.T, vb = c * C + rb < a.T;
-    const size_t rowq_a = (((size_t)b * a.T + c * C + ra) * a.Hk + hk) * D, rowq_b = rowq_a + (size_t)8 * a.Hk * D;
-    // ---- e: dQ = diag(Gamma) dO S^T + (dM * D) K
-    {
-        float dq[8][4];
-        zero_acc<8>(dq);
-        wgemm<8, 4, false, true>(dq, sb + OC_DO, LDD, r0, sb + OC_S, LDD, n128, lane, NoScale());
-        const float ga = Gam[ra], gb = Gam[rb];
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) dq[nt][0] *= ga, dq[nt][1] *= ga, dq[nt][2] *= gb, dq[nt][3] *= gb;
-        wgemm<4, 4, false, true>(dq, sb + OC_M, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale());
-        rowdot(dq, OC_Q, n128, pg0, pg1);
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int col = n128 + 8 * nt + 2 * t4;
-            if (va) atomicAdd(a.dq + rowq_a + col, dq[nt][0]), atomicAdd(a.dq + rowq_a + col + 1, dq[nt][1]);
-            if (vb) atomicAdd(a.dq + rowq_b + col, dq[nt][2]), atomicAdd(a.dq + rowq_b + col + 1, dq[nt][3]);
+                for (int e = 0; e < 4; ++e) dm[mi][nt][e] *= dec(row(mi, e), n64 + 8 * nt + 2 * t4 + (e & 1));
+            store_h(dm[mi], mi, 2, OC_M, LDC, n64, 1.f);   // M is dead
         }
     }
-    // ---- f: dK3 = diag(f) U' dS_next^T (the start of dK)
-    float dk[8][4];
+    __syncthreads();
+    // ---- e: dQ = diag(Gamma) dO S^T + (dM * D) K
     {
-        zero_acc<8>(dk);
-        wgemm<8, 4, false, true>(dk, sb + OC_U, LDD, r0, sb + OC_DS, LDD, n128, lane, NoScale());
-        const float fa = fv[ra], fb = fv[rb];
+        float dq[2][4][4];
+        zero2<4>(dq);
+        wgemm2<8, 2, false, true>(dq, sb + OC_DO, LDD, r0, sb + OC_S, LDD, n128, lane, NoScale2());
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) dk[nt][0] *= fa, dk[nt][1] *= fa, dk[nt][2] *= fb, dk[nt][3] *= fb;
-        float s0 = 0.f, s1 = 0.f;
-        rowdot(dk, OC_K, n128, s0, s1);
-        pg0 -= s0, pg1 -= s1, tot3 += s0 + s1;
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dq[mi][nt][e] *= Gam[row(mi, e)];
+        wgemm2<4, 2, false, true>(dq, sb + OC_M, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale2());
+        rowdot(dq, OC_Q, n128, pg);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi) {
+                const int r = row(mi, 2 * hi);
+                if (c * C + r >= a.T) continue;
+                float *dst = a.dq + (((size_t)b * a.T + c * C + r) * a.Hk + hk) * D + n128 + 2 * t4;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    atomicAdd(dst + 8 * nt, dq[mi][nt][2 * hi]);
+                    atomicAdd(dst + 8 * nt + 1, dq[mi][nt][2 * hi + 1]);
+                }
+            }
+    }
+    // ---- f: dK3 = diag(f) U' dS_next^T (the start of dK)
+    float dk[2][4][4];
+    {
+        zero2<4>(dk);
+        wgemm2<8, 2, false, true>(dk, sb + OC_U, LDD, r0, sb + OC_DS, LDD, n128, lane, NoScale2());
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dk[mi][nt][e] *= fv[row(mi, e)];
+        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        rowdot(dk, OC_K, n128, s);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi) pg[mi][hi] -= s[mi][hi], tot3 += s[mi][hi];
     }
     // ---- g: dW = -dU' S^T, into the dS_next slot once every warp is done with it
     {
-        float dw[8][4];
-        zero_acc<8>(dw);
-        wgemm<8, 4, false, true>(dw, sb + OC_W, LDD, r0, sb + OC_S, LDD, n128, lane, NoScale());
+        float dw[2][4][4];
+        zero2<4>(dw);
+        wgemm2<8, 2, false, true>(dw, sb + OC_W, LDD, r0, sb + OC_S, LDD, n128, lane, NoScale2());
         __syncthreads();
-        store_h(dw, 8, OC_DS, LDD, n128, -1.f);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) store_h(dw[mi], mi, 4, OC_DS, LDD, n128, -1.f);
     }
     __syncthreads();
     // ---- h: dV = diag(beta) T^T dU', and dK1's first part diag(Gamma beta) T^T dW
     {
-        float y[8][4];
-        zero_acc<8>(y);
-        wgemm<4, 4, true, true>(y, sb + OC_T, LDC, r0, sb + OC_W, LDD, n128, lane, NoScale());
-        rowdot(y, OC_V, n128, pb0, pb1);   // rowsum(V * T^T dU')
-        const float ba = beta[ra], bb = beta[rb];
-        const size_t rowv_a = (((size_t)b * a.T + c * C + ra) * a.Hv + h) * D, rowv_b = rowv_a + (size_t)8 * a.Hv * D;
+        float y[2][4][4];
+        zero2<4>(y);
+        wgemm2<4, 2, true, true>(y, sb + OC_T, LDC, r0, sb + OC_W, LDD, n128, lane, NoScale2());
+        rowdot(y, OC_V, n128, pb);   // rowsum(V * T^T dU')
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int col = n128 + 8 * nt + 2 * t4;
-            if (va) *reinterpret_cast<float2 *>(a.dv + rowv_a + col) = make_float2(ba * y[nt][0], ba * y[nt][1]);
-            if (vb) *reinterpret_cast<float2 *>(a.dv + rowv_b + col) = make_float2(bb * y[nt][2], bb * y[nt][3]);
-        }
-        zero_acc<8>(y);
-        wgemm<4, 4, true, true>(y, sb + OC_T, LDC, r0, sb + OC_DS, LDD, n128, lane, NoScale());
-        float s0 = 0.f, s1 = 0.f;
-        rowdot(y, OC_K, n128, s0, s1);   // rowsum(K * T^T dW)
-        const float ga = Gam[ra], gb = Gam[rb];
-        pb0 += ga * s0, pb1 += gb * s1;
-        pg0 += ga * ba * s0, pg1 += gb * bb * s1;   // rowsum(dK1a * K)
+        for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            dk[nt][0] += ga * ba * y[nt][0], dk[nt][1] += ga * ba * y[nt][1];
-            dk[nt][2] += gb * bb * y[nt][2], dk[nt][3] += gb * bb * y[nt][3];
-        }
-    }
-    // ---- i: dT = dU' V^T diag(beta) + dW K^T diag(beta Gamma), into the U' slot
-    {
-        float x1[4][4], x2[4][4];
-        zero_acc<4>(x1);
-        zero_acc<4>(x2);
-        wgemm<8, 2, false, false>(x1, sb + OC_W, LDD, r0, sb + OC_V, LDD, n64, lane, NoScale());
-        wgemm<8, 2, false, false>(x2, sb + OC_DS, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale());
+            for (int hi = 0; hi < 2; ++hi) {
+                const int r = row(mi, 2 * hi);
+                if (c * C + r >= a.T) continue;
+                const float br = beta[r];
+                float *dst = a.dv + (((size_t)b * a.T + c * C + r) * a.Hv + h) * D + n128 + 2 * t4;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                x1[nt][e] = beta[i] * (x1[nt][e] + Gam[i] * x2[nt][e]);
+                for (int nt = 0; nt < 4; ++nt)
+                    *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(br * y[mi][nt][2 * hi], br * y[mi][nt][2 * hi + 1]);
             }
-        store_h(x1, 4, OC_U, LDC, n64, 1.f);   // U' is dead (read in d and f)
+        zero2<4>(y);
+        wgemm2<4, 2, true, true>(y, sb + OC_T, LDC, r0, sb + OC_DS, LDD, n128, lane, NoScale2());
+        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        rowdot(y, OC_K, n128, s);   // rowsum(K * T^T dW)
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi) {
+                const int r = row(mi, 2 * hi);
+                const float gr = Gam[r], gbr = gr * beta[r];
+                pb[mi][hi] += gr * s[mi][hi];
+                pg[mi][hi] += gbr * s[mi][hi];   // rowsum(dK1a * K)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    dk[mi][nt][2 * hi] += gbr * y[mi][nt][2 * hi];
+                    dk[mi][nt][2 * hi + 1] += gbr * y[mi][nt][2 * hi + 1];
+                }
+            }
+    }
+    // ---- i: dT = dU' V^T diag(beta) + dW K^T diag(beta Gamma), into the U' slot (dead after f)
+    {
+        float x1[2][2][4], x2[2][2][4];
+        zero2<2>(x1);
+        zero2<2>(x2);
+        wgemm2<8, 1, false, false>(x1, sb + OC_W, LDD, r0, sb + OC_V, LDD, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(x2, sb + OC_DS, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale2());
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = n64 + 8 * nt + 2 * t4 + (e & 1);
+                    x1[mi][nt][e] = beta[i] * (x1[mi][nt][e] + Gam[i] * x2[mi][nt][e]);
+                }
+            store_h(x1[mi], mi, 2, OC_U, LDC, n64, 1.f);
+        }
     }
     __syncthreads();
     // ---- j: X = T^T dT (into the S^T slot), then dA = strict tril(-X T^T)
     {
-        float x[4][4];
-        zero_acc<4>(x);
-        wgemm<4, 2, true, true>(x, sb + OC_T, LDC, r0, sb + OC_U, LDC, n64, lane, NoScale());
-        store_h(x, 4, OC_S, LDC, n64, 1.f);
+        float x[2][2][4];
+        zero2<2>(x);
+        wgemm2<4, 1, true, true>(x, sb + OC_T, LDC, r0, sb + OC_U, LDC, n64, lane, NoScale2());
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) store_h(x[mi], mi, 2, OC_S, LDC, n64, 1.f);
     }
     __syncthreads();
     {
-        float y[4][4];
-        zero_acc<4>(y);
-        wgemm<4, 2, false, false>(y, sb + OC_S, LDC, r0, sb + OC_T, LDC, n64, lane, NoScale());
-        const float ba = beta[ra], bb = beta[rb];
+        float y[2][2][4];
+        zero2<2>(y);
+        wgemm2<4, 1, false, false>(y, sb + OC_S, LDC, r0, sb + OC_T, LDC, n64, lane, NoScale2());
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = e < 2 ? ra : rb, i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                const float dA = r > i ? -y[nt][e] : 0.f;
-                if (e < 2) pb0 += dA * bm[nt][e];
-                else pb1 += dA * bm[nt][e];
-                y[nt][e] = (e < 2 ? ba : bb) * dA * dec(r, i);   // dB * D
-            }
-        store_h(y, 4, OC_U, LDC, n64, 1.f);   // dT is dead (read for X)
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = row(mi, e), i = n64 + 8 * nt + 2 * t4 + (e & 1);
+                    const float dA = r > i ? -y[mi][nt][e] : 0.f;
+                    pb[mi][e >> 1] += dA * bm[mi][nt][e];
+                    y[mi][nt][e] = beta[r] * dA * dec(r, i);   // dB * D
+                }
+            store_h(y[mi], mi, 2, OC_U, LDC, n64, 1.f);   // dT is dead (read for X)
+        }
     }
     __syncthreads();
     // ---- k: dK1 += (dB * D) K;  dK2 = (dM * D)^T Q + (dB * D)^T K
     {
-        float p[8][4];
-        zero_acc<8>(p);
-        wgemm<4, 4, false, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale());
-        rowdot(p, OC_K, n128, pg0, pg1);
+        float p[2][4][4];
+        zero2<4>(p);
+        wgemm2<4, 2, false, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale2());
+        rowdot(p, OC_K, n128, pg);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dk[nt][e] += p[nt][e];
-        zero_acc<8>(p);
-        wgemm<4, 4, true, true>(p, sb + OC_M, LDC, r0, sb + OC_Q, LDD, n128, lane, NoScale());
-        wgemm<4, 4, true, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale());
-        float s0 = 0.f, s1 = 0.f;
-        rowdot(p, OC_K, n128, s0, s1);
-        pg0 -= s0, pg1 -= s1;
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int col = n128 + 8 * nt + 2 * t4;
-            const float k0 = dk[nt][0] + p[nt][0], k1 = dk[nt][1] + p[nt][1];
-            const float k2 = dk[nt][2] + p[nt][2], k3 = dk[nt][3] + p[nt][3];
-            if (va) atomicAdd(a.dk + rowq_a + col, k0), atomicAdd(a.dk + rowq_a + col + 1, k1);
-            if (vb) atomicAdd(a.dk + rowq_b + col, k2), atomicAdd(a.dk + rowq_b + col + 1, k3);
-        }
+                for (int e = 0; e < 4; ++e) dk[mi][nt][e] += p[mi][nt][e];
+        zero2<4>(p);
+        wgemm2<4, 2, true, true>(p, sb + OC_M, LDC, r0, sb + OC_Q, LDD, n128, lane, NoScale2());
+        wgemm2<4, 2, true, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale2());
+        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        rowdot(p, OC_K, n128, s);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi) {
+                pg[mi][hi] -= s[mi][hi];
+                const int r = row(mi, 2 * hi);
+                if (c * C + r >= a.T) continue;
+                float *dst = a.dk + (((size_t)b * a.T + c * C + r) * a.Hk + hk) * D + n128 + 2 * t4;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    atomicAdd(dst + 8 * nt, dk[mi][nt][2 * hi] + p[mi][nt][2 * hi]);
+                    atomicAdd(dst + 8 * nt + 1, dk[mi][nt][2 * hi + 1] + p[mi][nt][2 * hi + 1]);
+                }
+            }
     }
     // ---- l: row sums over the warps, then dg (reverse cumulative sum) and dbeta
 #pragma unroll
-    for (int o = 1; o < 4; o <<= 1) {
-        pg0 += __shfl_xor_sync(0xffffffffu, pg0, o);
-        pg1 += __shfl_xor_sync(0xffffffffu, pg1, o);
-        pb0 += __shfl_xor_sync(0xffffffffu, pb0, o);
-        pb1 += __shfl_xor_sync(0xffffffffu, pb1, o);
-    }
-    if (t4 == 0) {
-        vec[VDG + 64 * cw + ra] = pg0;
-        vec[VDG + 64 * cw + rb] = pg1;
-        vec[VDB + 64 * cw + ra] = pb0;
-        vec[VDB + 64 * cw + rb] = pb1;
-    }
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                pg[mi][hi] += __shfl_xor_sync(0xffffffffu, pg[mi][hi], o);
+                pb[mi][hi] += __shfl_xor_sync(0xffffffffu, pb[mi][hi], o);
+            }
+            if (t4 == 0) {
+                vec[VDG + 64 * cw + row(mi, 2 * hi)] = pg[mi][hi];
+                vec[VDB + 64 * cw + row(mi, 2 * hi)] = pb[mi][hi];
+            }
+        }
     tot3 = warp_sum(tot3);
     if (lane == 0) vec[VT3 + warp] = tot3;
     __syncthreads();
@@ -613,11 +751,12 @@ __global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
         float t3 = 0.f, ss = 0.f;
 #pragma unroll
         for (int w8 = 0; w8 < 8; ++w8) t3 += vec[VT3 + w8], ss += vec[VSS + w8];
+        auto dgrow = [&](int r) { return ((vec[VDG + r] + vec[VDG + 64 + r]) + vec[VDG + 128 + r]) + vec[VDG + 192 + r]; };
+        auto dbrow = [&](int r) { return ((vec[VDB + r] + vec[VDB + 64 + r]) + vec[VDB + 128 + r]) + vec[VDB + 192 + r]; };
         // rows 63 - lane and 31 - lane: an inclusive scan over the lanes is the reverse sum
         const float extra = t3 + __expf(G[C - 1]) * ss;
         const int rA = 63 - lane, rB = 31 - lane;
-        float x0 = vec[VDG + rA] + vec[VDG + 64 + rA] + (lane == 0 ? extra : 0.f);
-        float x1 = vec[VDG + rB] + vec[VDG + 64 + rB];
+        float x0 = dgrow(rA) + (lane == 0 ? extra : 0.f), x1 = dgrow(rB);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
@@ -627,11 +766,11 @@ __global__ void __launch_bounds__(NT, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
         const size_t base = (size_t)b * a.T + c * C;
         if (c * C + rA < a.T) {
             a.dg[(base + rA) * a.Hv + h] = x0;
-            a.dbeta[(base + rA) * a.Hv + h] = vec[VDB + rA] + vec[VDB + 64 + rA];
+            a.dbeta[(base + rA) * a.Hv + h] = dbrow(rA);
         }
         if (c * C + rB < a.T) {
             a.dg[(base + rB) * a.Hv + h] = x1;
-            a.dbeta[(base + rB) * a.Hv + h] = vec[VDB + rB] + vec[VDB + 64 + rB];
+            a.dbeta[(base + rB) * a.Hv + h] = dbrow(rB);
         }
     }
 }
@@ -667,14 +806,16 @@ cudaError_t launch_bwdc(const BwdArgs &a, void *workspace, cudaStream_t st)
     f.save_s = ws.s, f.save_p = ws.p, f.save_qh = ws.qh, f.save_t = ws.t;
     cudaError_t e = launch_fwd_tc(f, st);
     if (e != cudaSuccess) return e;
+    CUtensorMap mdo;
+    if (!make_map(&mdo, a.dout, a.B, a.T, a.Hv, 64, false, true)) return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(bwdc_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_SCAN);
     if (e != cudaSuccess) return e;
-    bwdc_scan_kernel<<<(unsigned)(a.B * a.Hv), NT, SMEM_SCAN, st>>>(a, ws);
+    bwdc_scan_kernel<<<(unsigned)(a.B * a.Hv), NT, SMEM_SCAN, st>>>(a, ws, mdo);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwdc_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_CHUNK);
     if (e != cudaSuccess) return e;
-    bwdc_chunk_kernel<<<(unsigned)cu, NT, SMEM_CHUNK, st>>>(a, ws);
+    bwdc_chunk_kernel<<<(unsigned)cu, NTC, SMEM_CHUNK, st>>>(a, ws);
     return cudaGetLastError();
 }
 

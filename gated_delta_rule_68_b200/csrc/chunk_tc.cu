@@ -187,6 +187,14 @@ __device__ __forceinline__ void st_chunk8(uint32_t addr, const float *x)
                  "r"(pack_h2(x[2], x[3])), "r"(pack_h2(x[4], x[5])), "r"(pack_h2(x[6], x[7]))
                  : "memory");
 }
+// The same 8 fp16 values into shared memory and to a 16-byte aligned global address.
+__device__ __forceinline__ void st_chunk8_g(uint32_t addr, const float *x, void *gp)
+{
+    const uint4 u = make_uint4(pack_h2(x[0], x[1]), pack_h2(x[2], x[3]), pack_h2(x[4], x[5]), pack_h2(x[6], x[7]));
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+                 : "memory");
+    *reinterpret_cast<uint4 *>(gp) = u;
+}
 __device__ __forceinline__ void st_h1(uint8_t *sm, uint32_t off, float x)
 {
     *reinterpret_cast<__half *>(sm + off) = __float2half_rn(x);
@@ -329,8 +337,9 @@ __device__ __forceinline__ void st_tglobal(__half *tg, int R0, int I0, const flo
 // exactly its own code): q and k rows divided by sqrt(sum of squares + 1e-6) as they are
 // converted, and o rows replaced by o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
 // SAVE (scalar gate, one CTA per unit): the first pass of the chunked backward. Per chunk it
-// also writes the entering state S^T, P, Qh^T and T (unscaled, lower triangle and diagonal
-// blocks) to the caller's buffers as fp16, and stores no o.
+// also writes the entering state S^T, T (unscaled; the lower triangle and diagonal blocks)
+// and the images of the P and Qh^T operand tiles (128-byte swizzled) to the caller's buffers
+// as fp16, and stores no o.
 template <typename TOut, bool NORM, int GATE, bool SCHED, bool SAVE = false>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -1079,6 +1088,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
             for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? __ldcg(h0 + (size_t)dk * D) : 0.f;
             if (GATE == 0) store_s16(gsb);
+            if (SAVE) {   // the state entering chunk 0: row p of S^T, columns 64 hf ..
+                __half *sg = reinterpret_cast<__half *>(a.save_s) + ((size_t)bh * NC * D + p) * D + 64 * hf;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) st_global_h8(sg + 8 * j, S + 8 * j);
+            }
         }
         float gbn[4] = {0.f, 0.f, 0.f, 0.f};
         if (issuer && c1 > c0) {
@@ -1103,24 +1117,20 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     prefetch_l1(reinterpret_cast<const __nv_bfloat16 *>(a.z) +
                                 ((size_t)(tok0 + c * C + r) * a.Hv + h) * D + 32 * k);
             }
-            const size_t save_at = SAVE ? ((size_t)bh * NC + c) * D + p : 0;
-            if (SAVE) {   // the state entering chunk c: row p of S^T, columns 64 hf ..
-                __half *sg = reinterpret_cast<__half *>(a.save_s) + save_at * D + 64 * hf;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) st_global_h8(sg + 8 * j, S + 8 * j);
-            }
             // P and Qh of this chunk, out of tensor memory into the operand tiles
             wait(B_P1, gs & 1);
             tc_fence_after();
             {
                 float v[32];
                 tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
+                if (SAVE) {   // and to global memory: the tile's image, 16 KB per chunk
+                    uint8_t *qg = reinterpret_cast<uint8_t *>(a.save_qh) + ((size_t)bh * NC + c) * 16384;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
-                if (SAVE) {   // row p of Qh^T, tokens 32 hf ..
-                    __half *qg = reinterpret_cast<__half *>(a.save_qh) + save_at * C + 32 * hf;
+                    for (int j = 0; j < 4; ++j)
+                        st_chunk8_g(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j, qg + swz_chunk(p, 4 * hf + j, 0));
+                } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) st_global_h8(qg + 8 * j, v + 8 * j);
+                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
                 }
             }
             wait(B_P, gs & 1);
@@ -1132,12 +1142,14 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 64 * hf), tmem_addr(tb, q4, TM_Y + 64 * hf + 32), v);
+                if (SAVE) {   // and to global memory: the tile's image, 32 KB per chunk
+                    uint8_t *pg = reinterpret_cast<uint8_t *>(a.save_p) + ((size_t)bh * NC + c) * 32768;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
-                if (SAVE) {   // row p of P, columns 64 hf ..
-                    __half *pg = reinterpret_cast<__half *>(a.save_p) + save_at * D + 64 * hf;
+                    for (int j = 0; j < 8; ++j)
+                        st_chunk8_g(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j, pg + swz_chunk(p, j, hf * 16384));
+                } else {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) st_global_h8(pg + 8 * j, v + 8 * j);
+                    for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
                 }
             }
             const float gC = GATE ? 0.f : vec[(gs & 1) * V_SET + V_GC];
@@ -1184,6 +1196,12 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                         w[j] = pack_h2(S[32 * h2 + 2 * j], S[32 * h2 + 2 * j + 1]);
                     }
                     tmem_st16(tmem_addr(tb, q4, TM_S16 + 32 * hf + 16 * h2), w);
+                    if (SAVE && c + 1 < c1) {   // the state entering chunk c + 1, as its fp16 copy
+                        uint4 *sg = reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(a.save_s) +
+                                                              (((size_t)bh * NC + c + 1) * D + p) * D + 64 * hf + 32 * h2);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) sg[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    }
                 }
                 tmem_wait_st();
             } else {   // S <- diag(Gamma_C) S + (P S + R), row dk = 64 hf + i, in two halves of 32

@@ -41,8 +41,9 @@ struct FwdArgs {
     unsigned long long *sched_flags = nullptr;
     float *sched_states = nullptr;
     // tcgen05 kernel, scalar gate: the chunked backward's forward pass. Per (unit, chunk),
-    // fp16: the entering state S^T [Dv][Dk], P [Dk][Dk], Qh^T [Dk][64] and T [64][64] (the
-    // lower triangle; entries above the diagonal blocks are not written). No o is stored.
+    // fp16: the entering state S^T [Dv][Dk], T [64][64] (the lower triangle; entries above
+    // the diagonal blocks are not written), and the images of the P [Dk][Dk] and Qh^T [Dk][64]
+    // operand tiles in the 128-byte swizzle (32 and 16 KB). No o is stored.
     void *save_s = nullptr, *save_p = nullptr, *save_qh = nullptr, *save_t = nullptr;
 };
 
