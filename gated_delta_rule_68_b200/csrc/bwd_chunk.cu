@@ -140,6 +140,11 @@ constexpr uint32_t ID_SP = tcu::idesc_f16(128, 128, false, false, true);   // dS
 
 __device__ unsigned int g_bwdc_timeouts;
 
+// Global -> L2 prefetches: a 16-byte aligned span of a multiple of 16 bytes.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -204,32 +209,28 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
         issue_loads(NC - 1, 0);
         if (NC > 1) issue_loads(NC - 2, 1);
     }
+    // g of a chunk, two values per lane (summed over the warp when needed), loaded one chunk ahead
+    auto load_g = [&](int c, float &g0, float &g1) {
+        const int t0 = c * C + lane, t1 = t0 + 32;
+        g0 = (c >= 0 && t0 < a.T) ? a.g[((size_t)b * a.T + t0) * a.Hv + h] : 0.f;
+        g1 = (c >= 0 && t1 < a.T) ? a.g[((size_t)b * a.T + t1) * a.Hv + h] : 0.f;
+    };
+    auto convert_do = [&](int buf) {   // this thread's 64 bytes of dO to fp16 (rows past T are zeros)
+        uint8_t *d = sm + buf * SC_BUF + SC_DO + tid * 64;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) bf16_to_fp16_16B(d + 16 * k);
+    };
+    float ga, gb;
+    load_g(NC - 1, ga, gb);
+    wait(0, 0);
+    convert_do(0);
     for (int s = 0; s < NC; ++s) {
         const int c = NC - 1 - s, buf = s & 1;
-        // Gamma_C of chunk c: exp of the sum of its g (loads in flight during the wait below)
-        float gsum = 0.f;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int t = c * C + lane + 32 * k;
-            if (t < a.T) gsum += a.g[((size_t)b * a.T + t) * a.Hv + h];
-        }
-        wait(buf, (s >> 1) & 1);
-        {   // this thread's 64 bytes of dO to fp16 (rows past T arrive as zeros)
-            uint8_t *d = sm + buf * SC_BUF + SC_DO + tid * 64;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) bf16_to_fp16_16B(d + 16 * k);
-        }
-        {   // dS_next of chunk c: row p of dS^T, columns 64 hf .., fp16
-            uint4 *dst = reinterpret_cast<uint4 *>(ws.ds + ((size_t)unit * NC + c) * D * D + (size_t)p * D + 64 * hf);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                dst[j] = make_uint4(pack_h2f(dS[8 * j], dS[8 * j + 1]), pack_h2f(dS[8 * j + 2], dS[8 * j + 3]),
-                                    pack_h2f(dS[8 * j + 4], dS[8 * j + 5]), pack_h2f(dS[8 * j + 6], dS[8 * j + 7]));
-        }
-        const float gC = __expf(warp_sum(gsum));
+        const float gC = __expf(warp_sum(ga + gb));   // Gamma_C of chunk c
+        load_g(c - 1, ga, gb);
         fence_proxy_async();
         tc_fence_before();
-        __syncthreads();
+        __syncthreads();   // dO of chunk c converted, the copy of dS^T written
         if (tid == 0) {
             tc_fence_after();
             const uint32_t base = sb + buf * SC_BUF;
@@ -241,6 +242,19 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
             for (int k = 0; k < 8; ++k)
                 mma_ts(tb + TS_D, tb + TS_A + 8 * k, sdesc(base + SC_P + k * 2048, 16384, 1024), ID_SP, true);
             mma_commit(bar(2));
+        }
+        {   // while the products run: dS_next of chunk c (row p of dS^T, columns 64 hf .., as the
+            // fp16 image of a 128-byte swizzled tile) ...
+            uint8_t *dst = reinterpret_cast<uint8_t *>(ws.ds + ((size_t)unit * NC + c) * D * D);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4 *>(dst + swz_chunk(p, j, hf * 16384)) =
+                    make_uint4(pack_h2f(dS[8 * j], dS[8 * j + 1]), pack_h2f(dS[8 * j + 2], dS[8 * j + 3]),
+                               pack_h2f(dS[8 * j + 4], dS[8 * j + 5]), pack_h2f(dS[8 * j + 6], dS[8 * j + 7]));
+        }
+        if (s + 1 < NC) {   // ... and the next chunk's dO
+            wait(buf ^ 1, ((s + 1) >> 1) & 1);
+            convert_do(buf ^ 1);
         }
         wait(2, s & 1);
         tc_fence_after();
@@ -259,8 +273,6 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
             tmem_st16(tmem_addr(tb, q4, TS_A + 32 * hf + 16 * h2), w);
         }
         tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
     }
     {   // dh0 = dS entering chunk 0
         float *dst = a.dh0 + (size_t)unit * D * D + (size_t)(64 * hf) * D + p;
@@ -285,44 +297,60 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
 // product (two m16 blocks, mi = 0, 1) and columns 32 cw .. of the 128-wide ones, 16 cw .. of
 // the 64-wide ones: each fragment loaded from shared memory feeds two to four MMAs.
 constexpr int NTC = 256;
-constexpr uint32_t SZ_DT = C * LDD * 2;     // [64][136] fp16
-constexpr uint32_t SZ_ST = D * LDD * 2;     // [128][136] fp16
-constexpr uint32_t SZ_CT = C * LDC * 2;     // [64][72] fp16
-constexpr uint32_t OC_Q = 0, OC_K = SZ_DT, OC_V = 2 * SZ_DT, OC_DO = 3 * SZ_DT;
-constexpr uint32_t OC_S = 4 * SZ_DT;          // S^T [dv][dk]; later X = T^T dT [64][LDC]
-constexpr uint32_t OC_DS = OC_S + SZ_ST;      // dS_next^T [dv][dk]; later dW [64][LDD]
-constexpr uint32_t OC_T = OC_DS + SZ_ST;      // T [64][LDC]
-constexpr uint32_t OC_M = OC_T + SZ_CT;       // M, then dM * D [64][LDC]
+// Input tiles are 128-byte swizzled images (64-column atoms, 1024-byte aligned), loaded by TMA
+// (q, k, v, dO) and bulk copies (S^T, dS_next^T, T); the tiles the kernel writes itself are
+// plain rows padded to LDD / LDC halves. A tile's "ld" below is its padded row stride in
+// halves, or minus its atom stride in bytes for a swizzled image.
+constexpr uint32_t SZ_DT = C * LDD * 2;     // padded [64][136] fp16
+constexpr uint32_t SZ_CT = C * LDC * 2;     // padded [64][72] fp16
+constexpr int LQ = -8192, LS = -16384, LT = -8192;   // swizzled [64][128], [128][128], [64][64]
+constexpr uint32_t OC_Q = 0, OC_K = 16384, OC_V = 32768, OC_DO = 49152;
+constexpr uint32_t OC_S = 65536;              // S^T [dv][dk]; later X = T^T dT [64][LDC]
+constexpr uint32_t OC_DS = OC_S + 32768;      // dS_next^T [dv][dk]; later dW [64][LDD]
+constexpr uint32_t OC_T = OC_DS + 32768;      // T [64][64]
+constexpr uint32_t OC_M = OC_T + 8192;        // M, then dM * D [64][LDC]
 constexpr uint32_t OC_W = OC_M + SZ_CT;       // W, then dU' [64][LDD]
 constexpr uint32_t OC_U = OC_W + SZ_DT;       // U', then dT, then dB * D [64][LDC]
-constexpr uint32_t OC_VEC = OC_U + SZ_DT;
+constexpr uint32_t OC_DEC = OC_U + SZ_DT;     // D_ri = exp(G_r - G_i) (r >= i, else 0) [64][LDC] fp16
+constexpr uint32_t OC_BM = OC_DEC + SZ_CT;    // Bm = tril(K K^T * D, -1) [64][LDC] fp16
+constexpr uint32_t OC_BAR = OC_BM + SZ_CT;    // two mbarriers: inputs, then S^T and dS_next^T
+constexpr uint32_t OC_VEC = OC_BAR + 16;
 // vectors: G, Gamma, beta, f [64]; per column quarter of the warps, the row sums of dG and dbeta
 // [4][64] each; per warp, sum(dK3 * K) and sum(dS_next * S) [8] each (summed in a fixed order,
 // so that dg and dbeta repeat bit for bit)
 constexpr int VG = 0, VGAM = 64, VBETA = 128, VF = 192, VDG = 256, VDB = 512, VT3 = 768, VSS = 776;
-constexpr uint32_t SMEM_CHUNK = OC_VEC + (VSS + 8) * 4;
+constexpr uint32_t SMEM_CHUNK = OC_VEC + (VSS + 8) * 4 + 1024;   // + alignment of the base
 static_assert(SMEM_CHUNK <= 227 * 1024, "shared memory");
 
+// Byte address of element (row, col) of a tile with the given ld (see above).
+__device__ __forceinline__ uint32_t taddr(uint32_t base, int ld, int row, int col)
+{
+    if (ld > 0) return base + (uint32_t)(row * ld + col) * 2u;
+    return base + (uint32_t)(col >> 6) * (uint32_t)(-ld) + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+           (((uint32_t)((col & 63) >> 3) ^ (uint32_t)(row & 7)) << 4) + (uint32_t)(col & 7) * 2u;
+}
 // acc[2][2 NP][4] += A (rows r0 .. r0 + 31, K = 16 KS) B (columns n0 .. n0 + 16 NP), as wgemm.
 // ascale(af, j, mi) may rescale the A fragment of k-step j, row block mi.
 template <int KS, int NP, bool AT, bool BT, typename AS>
 __device__ __forceinline__ void wgemm2(float (*acc)[2 * NP][4], uint32_t aB, int lda, int r0, uint32_t bB, int ldb,
                                        int n0, int lane, AS ascale)
 {
-#pragma unroll
+#pragma unroll 4
     for (int j = 0; j < KS; ++j) {
         uint32_t af[2][4];
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
-            if (AT) ldsm_t(af[mi], a_tr(aB, lda, r0 + 16 * mi, 16 * j, lane));
-            else ldsm(af[mi], a_rm(aB, lda, r0 + 16 * mi, 16 * j, lane));
+            const int m0 = r0 + 16 * mi, k0 = 16 * j;
+            if (AT) ldsm_t(af[mi], taddr(aB, lda, k0 + (lane & 7) + (lane >> 4) * 8, m0 + ((lane >> 3) & 1) * 8));
+            else ldsm(af[mi], taddr(aB, lda, m0 + (lane & 7) + ((lane >> 3) & 1) * 8, k0 + (lane >> 4) * 8));
             ascale(af[mi], j, mi);
         }
 #pragma unroll
         for (int np = 0; np < NP; ++np) {
             uint32_t bf[4];
-            if (BT) ldsm_t(bf, b_kn(bB, ldb, n0 + 16 * np, 16 * j, lane));
-            else ldsm(bf, b_nk(bB, ldb, n0 + 16 * np, 16 * j, lane));
+            const int nn = n0 + 16 * np, k0 = 16 * j;
+            if (BT) ldsm_t(bf, taddr(bB, ldb, k0 + (lane & 7) + ((lane >> 3) & 1) * 8, nn + (lane >> 4) * 8));
+            else ldsm(bf, taddr(bB, ldb, nn + (lane & 7) + (lane >> 4) * 8, k0 + ((lane >> 3) & 1) * 8));
 #pragma unroll
             for (int mi = 0; mi < 2; ++mi) {
                 mma(acc[mi][2 * np], af[mi], bf[0], bf[1]);
@@ -343,9 +371,16 @@ __device__ __forceinline__ void zero2(float (*acc)[N][4])
         for (int i = 0; i < N; ++i) acc[mi][i][0] = acc[mi][i][1] = acc[mi][i][2] = acc[mi][i][3] = 0.f;
 }
 
-__global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws)
+// pf: the CTA that runs pf launches later on this SM (the resident CTA count) gets its inputs
+// prefetched into L2 by this one; sole: every key head has one value head, so dq and dk rows
+// have one writer and take plain stores.
+__global__ void __launch_bounds__(NTC, 1)
+bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ CUtensorMap map_q,
+                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                  const __grid_constant__ CUtensorMap map_do)
 {
-    extern __shared__ __align__(128) uint8_t sm[];
+    extern __shared__ __align__(1024) uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
     const int rw = warp & 1, cw = warp >> 1, r0 = 32 * rw;
     const int NC = (a.T + C - 1) / C;
@@ -355,52 +390,74 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     float *vec = reinterpret_cast<float *>(sm + OC_VEC);
     const size_t cu = (size_t)unit * NC + c;
 
-    // ---- loads, in two groups: q, k (key head), v, dO (value head) as bf16 with rows past T
-    // zero, and T; then S^T and dS_next^T, which arrive while the Grams, W and U are formed
-    {
-        const __nv_bfloat16 *src[4] = {reinterpret_cast<const __nv_bfloat16 *>(a.q),
-                                       reinterpret_cast<const __nv_bfloat16 *>(a.k),
-                                       reinterpret_cast<const __nv_bfloat16 *>(a.v),
-                                       reinterpret_cast<const __nv_bfloat16 *>(a.dout)};
-        for (int i = tid; i < 4 * C * 16; i += NTC) {
-            const int m = i >> 10, r = (i >> 4) & 63, j = i & 15, t = c * C + r;
-            const bool ok = t < a.T;
-            const int H = m < 2 ? a.Hk : a.Hv, hh = m < 2 ? hk : h;
-            cp_async16(sb + m * SZ_DT + (r * LDD + 8 * j) * 2,
-                       src[m] + (((size_t)b * a.T + (ok ? t : 0)) * H + hh) * D + 8 * j, ok ? 16 : 0);
+    // ---- loads, on two mbarriers: q, k (key head), v, dO (value head) by TMA (bf16, rows past T
+    // zero) and T; then S^T and dS_next^T, which arrive while the Grams, W and U are formed
+    __shared__ int abort_sh;
+    const uint32_t bar0 = sb + OC_BAR, bar1 = bar0 + 8;
+    if (tid == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar1, 1);
+        abort_sh = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int t0 = c * C;
+        mbar_expect_tx(bar0, 4 * 16384 + 8192);
+        tma_load_4d(sb + OC_Q, &map_q, 0, hk, t0, b, bar0);
+        tma_load_4d(sb + OC_Q + 8192, &map_q, 64, hk, t0, b, bar0);
+        tma_load_4d(sb + OC_K, &map_k, 0, hk, t0, b, bar0);
+        tma_load_4d(sb + OC_K + 8192, &map_k, 64, hk, t0, b, bar0);
+        tma_load_4d(sb + OC_V, &map_v, 0, h, t0, b, bar0);
+        tma_load_4d(sb + OC_V + 8192, &map_v, 64, h, t0, b, bar0);
+        tma_load_4d(sb + OC_DO, &map_do, 0, h, t0, b, bar0);
+        tma_load_4d(sb + OC_DO + 8192, &map_do, 64, h, t0, b, bar0);
+        bulk_g2s(sb + OC_T, ws.t + cu * C * C, 8192, bar0);
+        mbar_expect_tx(bar1, 2 * 32768);
+        bulk_g2s(sb + OC_S, ws.s + cu * D * D, 32768, bar1);
+        bulk_g2s(sb + OC_DS, ws.ds + cu * D * D, 32768, bar1);
+    }
+    auto wait = [&](uint32_t bar) {
+        if (*reinterpret_cast<volatile int *>(&abort_sh)) return;
+        if (!mbar_wait_bounded(bar, 0)) {
+            *reinterpret_cast<volatile int *>(&abort_sh) = 1;
+            atomicAdd(&g_bwdc_timeouts, 1u);
         }
-        const __half *Tg = ws.t + cu * C * C;
-        for (int i = tid; i < C * 8; i += NTC) {
-            const int r = i >> 3, j = i & 7;
-            cp_async16(sb + OC_T + (r * LDC + 8 * j) * 2, Tg + r * C + 8 * j, 16);
+    };
+    if (tid < C) {
+        const int t = c * C + tid;
+        const bool ok = t < a.T;
+        vec[VG + tid] = ok ? a.g[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
+        vec[VBETA + tid] = ok ? a.beta[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
+    }
+    {   // the inputs of the CTA pf launches later into L2, while this one computes
+        const long nb = (long)blockIdx.x + pf;
+        if (pf > 0 && nb < (long)gridDim.x) {
+            const int nu = (int)(nb / NC), ncc = (int)(nb % NC);
+            const int n_b = nu / a.Hv, n_h = nu % a.Hv, n_hk = n_h / (a.Hv / a.Hk);
+            const int m = tid >> 6, r = tid & 63, t = ncc * C + r;
+            if (t < a.T) {
+                const void *src = m == 0 ? a.q : m == 1 ? a.k : m == 2 ? a.v : a.dout;
+                const int H = m < 2 ? a.Hk : a.Hv, hh = m < 2 ? n_hk : n_h;
+                prefetch_l2_bulk(reinterpret_cast<const __nv_bfloat16 *>(src) + (((size_t)n_b * a.T + t) * H + hh) * D,
+                                 D * 2);
+            }
+            if (tid == 0) {
+                const size_t ncu = (size_t)nu * NC + ncc;
+                prefetch_l2_bulk(ws.s + ncu * D * D, D * D * 2);
+                prefetch_l2_bulk(ws.ds + ncu * D * D, D * D * 2);
+                prefetch_l2_bulk(ws.t + ncu * C * C, C * C * 2);
+            }
         }
-        cp_async_commit();
-        const __half *S = ws.s + cu * D * D, *dS = ws.ds + cu * D * D;
-        for (int i = tid; i < D * 16; i += NTC) {
-            const int r = i >> 4, j = i & 15;
-            cp_async16(sb + OC_S + (r * LDD + 8 * j) * 2, S + r * D + 8 * j, 16);
-            cp_async16(sb + OC_DS + (r * LDD + 8 * j) * 2, dS + r * D + 8 * j, 16);
-        }
-        cp_async_commit();
-        if (tid < C) {
-            const int t = c * C + tid;
-            const bool ok = t < a.T;
-            vec[VG + tid] = ok ? a.g[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
-            vec[VBETA + tid] = ok ? a.beta[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
-        }
-        cp_async_wait1();
-        for (int i = tid; i < 4 * C * 16; i += NTC) {
-            const int m = i >> 10, r = (i >> 4) & 63, j = i & 15;
-            bf16_to_fp16_16B(sm + m * SZ_DT + (r * LDD + 8 * j) * 2);
-        }
-        // T is lower triangular: clear what the forward left unwritten above the diagonal blocks
-        for (int i = tid; i < C * 8; i += NTC) {
-            const int r = i >> 3, j = i & 7;
-            __half *row = reinterpret_cast<__half *>(sm + OC_T) + r * LDC + 8 * j;
+    }
+    wait(bar0);
+    for (int i = tid; i < 4 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_Q + 16 * i);   // q, k, v, dO to fp16
+    // T is lower triangular: clear what the forward left unwritten above the diagonal blocks
+    for (int i = tid; i < C * 8; i += NTC) {
+        const int r = i >> 3, j = i & 7;
+        __half *row = reinterpret_cast<__half *>(sm + OC_T + tcu::swz_chunk(r, j, 0));
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (8 * j + e > r) row[e] = __float2half(0.f);
-        }
+        for (int e = 0; e < 8; ++e)
+            if (8 * j + e > r) row[e] = __float2half(0.f);
     }
     __syncthreads();
     if (warp == 0) {   // in-chunk prefix G, Gamma = exp(G), f = Gamma_C / Gamma
@@ -425,18 +482,19 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     // this thread's rows: row(mi, hi) = r0 + 16 mi + 8 hi + g8 (accumulator elements 2 hi, 2 hi + 1)
     auto row = [&](int mi, int e) { return r0 + 16 * mi + g8 + 8 * (e >> 1); };
     auto dec = [&](int r, int i) { return r >= i ? __expf(G[r] - G[i]) : 0.f; };
+    // D and Bm, written in a and read back by the same thread (same warp tiles) in d and j
+    __half *decm = reinterpret_cast<__half *>(sm + OC_DEC), *bmm = reinterpret_cast<__half *>(sm + OC_BM);
     // per-row partial sums of this thread, [mi][hi], added to dG / dbeta at the end
     float pg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, tot3 = 0.f;
     auto rowdot = [&](const float (*acc)[4][4], uint32_t tile, int n0, float (*s)[2]) {
-        // sum over this thread's columns of acc * tile (fp16 [64][LDD]) on its rows
-        const __half *tp = reinterpret_cast<const __half *>(sm + tile);
+        // sum over this thread's columns of acc * tile (a swizzled [64][128] input) on its rows
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int col = n0 + 8 * nt + 2 * t4;
-                const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(tp + row(mi, 0) * LDD + col));
-                const float2 y = __half22float2(*reinterpret_cast<const __half2 *>(tp + row(mi, 2) * LDD + col));
+                const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(sm + (taddr(tile, LQ, row(mi, 0), col))));
+                const float2 y = __half22float2(*reinterpret_cast<const __half2 *>(sm + (taddr(tile, LQ, row(mi, 2), col))));
                 s[mi][0] = fmaf(acc[mi][nt][0], x.x, fmaf(acc[mi][nt][1], x.y, s[mi][0]));
                 s[mi][1] = fmaf(acc[mi][nt][2], y.x, fmaf(acc[mi][nt][3], y.y, s[mi][1]));
             }
@@ -462,32 +520,32 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     };
 
     // ---- a: the Grams, M = tril(Q K^T * D) and Bm = tril(K K^T * D, -1)
-    float bm[2][2][4];
     {
         float qk[2][2][4], kk[2][2][4];
         zero2<2>(qk);
         zero2<2>(kk);
-        wgemm2<8, 1, false, false>(qk, sb + OC_Q, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale2());
-        wgemm2<8, 1, false, false>(kk, sb + OC_K, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(qk, sb + OC_Q, LQ, r0, sb + OC_K, LQ, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(kk, sb + OC_K, LQ, r0, sb + OC_K, LQ, n64, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = row(mi, e), i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                    const float d = dec(r, i);
-                    qk[mi][nt][e] *= d;
-                    bm[mi][nt][e] = r > i ? kk[mi][nt][e] * d : 0.f;
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = row(mi, 2 * hi), i = n64 + 8 * nt + 2 * t4;
+                    const float d0 = dec(r, i), d1 = dec(r, i + 1);
+                    *reinterpret_cast<__half2 *>(decm + r * LDC + i) = __floats2half2_rn(d0, d1);
+                    *reinterpret_cast<__half2 *>(bmm + r * LDC + i) =
+                        __floats2half2_rn(r > i ? kk[mi][nt][2 * hi] * d0 : 0.f, r > i + 1 ? kk[mi][nt][2 * hi + 1] * d1 : 0.f);
+                    qk[mi][nt][2 * hi] *= d0;
+                    qk[mi][nt][2 * hi + 1] *= d1;
                 }
             store_h(qk[mi], mi, 2, OC_M, LDC, n64, 1.f);
         }
     }
     // ---- b: W = T diag(beta Gamma) K, U = T diag(beta) V, then U' = U - W S
     {
-        float w[2][4][4], u[2][4][4];
-        zero2<4>(w);
-        zero2<4>(u);
+        float u[2][4][4];
         auto colscale = [&](const float *s1, const float *s2) {
             return [=](uint32_t *af, int j, int) {
                 const int k0 = 16 * j + 2 * t4;
@@ -500,18 +558,22 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
                 hmul_frag(af[3], hi);
             };
         };
-        wgemm2<4, 2, false, true>(w, sb + OC_T, LDC, r0, sb + OC_K, LDD, n128, lane, colscale(beta, Gam));
-        wgemm2<4, 2, false, true>(u, sb + OC_T, LDC, r0, sb + OC_V, LDD, n128, lane, colscale(beta, nullptr));
+        {
+            float w[2][4][4];
+            zero2<4>(w);
+            wgemm2<4, 2, false, true>(w, sb + OC_T, LT, r0, sb + OC_K, LQ, n128, lane, colscale(beta, Gam));
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) store_h(w[mi], mi, 4, OC_W, LDD, n128, 1.f);
-        cp_async_wait_all();   // S^T and dS_next^T
+            for (int mi = 0; mi < 2; ++mi) store_h(w[mi], mi, 4, OC_W, LDD, n128, 1.f);
+        }
+        zero2<4>(u);
+        wgemm2<4, 2, false, true>(u, sb + OC_T, LT, r0, sb + OC_V, LQ, n128, lane, colscale(beta, nullptr));
+        wait(bar1);   // S^T and dS_next^T
         __syncthreads();
         {   // sum(dS_next * S) over the whole state
             float s = 0.f;
-            for (int i = tid; i < D * 16; i += NTC) {
-                const int r = i >> 4, j = i & 15;
-                const __half2 *x = reinterpret_cast<const __half2 *>(sm + OC_S + (r * LDD + 8 * j) * 2);
-                const __half2 *y = reinterpret_cast<const __half2 *>(sm + OC_DS + (r * LDD + 8 * j) * 2);
+            for (int i = tid; i < D * 16; i += NTC) {   // the two images share one layout
+                const __half2 *x = reinterpret_cast<const __half2 *>(sm + OC_S + 16 * i);
+                const __half2 *y = reinterpret_cast<const __half2 *>(sm + OC_DS + 16 * i);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 fx = __half22float2(x[e]), fy = __half22float2(y[e]);
@@ -522,7 +584,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
             if (lane == 0) vec[VSS + warp] = s;
         }
         const __half2 neg = __floats2half2_rn(-1.f, -1.f);
-        wgemm2<8, 2, false, false>(u, sb + OC_W, LDD, r0, sb + OC_S, LDD, n128, lane, [=](uint32_t *af, int, int) {
+        wgemm2<8, 2, false, false>(u, sb + OC_W, LDD, r0, sb + OC_S, LS, n128, lane, [=](uint32_t *af, int, int) {
             hmul_frag(af[0], neg);
             hmul_frag(af[1], neg);
             hmul_frag(af[2], neg);
@@ -536,8 +598,8 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float du[2][4][4];
         zero2<4>(du);
-        wgemm2<4, 2, true, true>(du, sb + OC_M, LDC, r0, sb + OC_DO, LDD, n128, lane, NoScale2());
-        wgemm2<8, 2, false, false>(du, sb + OC_K, LDD, r0, sb + OC_DS, LDD, n128, lane, rowscale(fv));
+        wgemm2<4, 2, true, true>(du, sb + OC_M, LDC, r0, sb + OC_DO, LQ, n128, lane, NoScale2());
+        wgemm2<8, 2, false, false>(du, sb + OC_K, LQ, r0, sb + OC_DS, LS, n128, lane, rowscale(fv));
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) store_h(du[mi], mi, 4, OC_W, LDD, n128, 1.f);   // W is dead
     }
@@ -546,13 +608,13 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float dm[2][2][4];
         zero2<2>(dm);
-        wgemm2<8, 1, false, false>(dm, sb + OC_DO, LDD, r0, sb + OC_U, LDD, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(dm, sb + OC_DO, LQ, r0, sb + OC_U, LDD, n64, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dm[mi][nt][e] *= dec(row(mi, e), n64 + 8 * nt + 2 * t4 + (e & 1));
+                for (int e = 0; e < 4; ++e) dm[mi][nt][e] *= __half2float(decm[row(mi, e) * LDC + n64 + 8 * nt + 2 * t4 + (e & 1)]);
             store_h(dm[mi], mi, 2, OC_M, LDC, n64, 1.f);   // M is dead
         }
     }
@@ -561,14 +623,14 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float dq[2][4][4];
         zero2<4>(dq);
-        wgemm2<8, 2, false, true>(dq, sb + OC_DO, LDD, r0, sb + OC_S, LDD, n128, lane, NoScale2());
+        wgemm2<8, 2, false, true>(dq, sb + OC_DO, LQ, r0, sb + OC_S, LS, n128, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dq[mi][nt][e] *= Gam[row(mi, e)];
-        wgemm2<4, 2, false, true>(dq, sb + OC_M, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale2());
+        wgemm2<4, 2, false, true>(dq, sb + OC_M, LDC, r0, sb + OC_K, LQ, n128, lane, NoScale2());
         rowdot(dq, OC_Q, n128, pg);
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
@@ -579,8 +641,12 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
                 float *dst = a.dq + (((size_t)b * a.T + c * C + r) * a.Hk + hk) * D + n128 + 2 * t4;
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    atomicAdd(dst + 8 * nt, dq[mi][nt][2 * hi]);
-                    atomicAdd(dst + 8 * nt + 1, dq[mi][nt][2 * hi + 1]);
+                    if (sole) {
+                        *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(dq[mi][nt][2 * hi], dq[mi][nt][2 * hi + 1]);
+                    } else {
+                        atomicAdd(dst + 8 * nt, dq[mi][nt][2 * hi]);
+                        atomicAdd(dst + 8 * nt + 1, dq[mi][nt][2 * hi + 1]);
+                    }
                 }
             }
     }
@@ -588,7 +654,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     float dk[2][4][4];
     {
         zero2<4>(dk);
-        wgemm2<8, 2, false, true>(dk, sb + OC_U, LDD, r0, sb + OC_DS, LDD, n128, lane, NoScale2());
+        wgemm2<8, 2, false, true>(dk, sb + OC_U, LDD, r0, sb + OC_DS, LS, n128, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
@@ -606,7 +672,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float dw[2][4][4];
         zero2<4>(dw);
-        wgemm2<8, 2, false, true>(dw, sb + OC_W, LDD, r0, sb + OC_S, LDD, n128, lane, NoScale2());
+        wgemm2<8, 2, false, true>(dw, sb + OC_W, LDD, r0, sb + OC_S, LS, n128, lane, NoScale2());
         __syncthreads();
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) store_h(dw[mi], mi, 4, OC_DS, LDD, n128, -1.f);
@@ -616,7 +682,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float y[2][4][4];
         zero2<4>(y);
-        wgemm2<4, 2, true, true>(y, sb + OC_T, LDC, r0, sb + OC_W, LDD, n128, lane, NoScale2());
+        wgemm2<4, 2, true, true>(y, sb + OC_T, LT, r0, sb + OC_W, LDD, n128, lane, NoScale2());
         rowdot(y, OC_V, n128, pb);   // rowsum(V * T^T dU')
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
@@ -631,7 +697,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
                     *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(br * y[mi][nt][2 * hi], br * y[mi][nt][2 * hi + 1]);
             }
         zero2<4>(y);
-        wgemm2<4, 2, true, true>(y, sb + OC_T, LDC, r0, sb + OC_DS, LDD, n128, lane, NoScale2());
+        wgemm2<4, 2, true, true>(y, sb + OC_T, LT, r0, sb + OC_DS, LDD, n128, lane, NoScale2());
         float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         rowdot(y, OC_K, n128, s);   // rowsum(K * T^T dW)
 #pragma unroll
@@ -654,8 +720,8 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
         float x1[2][2][4], x2[2][2][4];
         zero2<2>(x1);
         zero2<2>(x2);
-        wgemm2<8, 1, false, false>(x1, sb + OC_W, LDD, r0, sb + OC_V, LDD, n64, lane, NoScale2());
-        wgemm2<8, 1, false, false>(x2, sb + OC_DS, LDD, r0, sb + OC_K, LDD, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(x1, sb + OC_W, LDD, r0, sb + OC_V, LQ, n64, lane, NoScale2());
+        wgemm2<8, 1, false, false>(x2, sb + OC_DS, LDD, r0, sb + OC_K, LQ, n64, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
@@ -673,7 +739,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float x[2][2][4];
         zero2<2>(x);
-        wgemm2<4, 1, true, true>(x, sb + OC_T, LDC, r0, sb + OC_U, LDC, n64, lane, NoScale2());
+        wgemm2<4, 1, true, true>(x, sb + OC_T, LT, r0, sb + OC_U, LDC, n64, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) store_h(x[mi], mi, 2, OC_S, LDC, n64, 1.f);
     }
@@ -681,7 +747,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float y[2][2][4];
         zero2<2>(y);
-        wgemm2<4, 1, false, false>(y, sb + OC_S, LDC, r0, sb + OC_T, LDC, n64, lane, NoScale2());
+        wgemm2<4, 1, false, false>(y, sb + OC_S, LDC, r0, sb + OC_T, LT, n64, lane, NoScale2());
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
@@ -690,8 +756,8 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
                 for (int e = 0; e < 4; ++e) {
                     const int r = row(mi, e), i = n64 + 8 * nt + 2 * t4 + (e & 1);
                     const float dA = r > i ? -y[mi][nt][e] : 0.f;
-                    pb[mi][e >> 1] += dA * bm[mi][nt][e];
-                    y[mi][nt][e] = beta[r] * dA * dec(r, i);   // dB * D
+                    pb[mi][e >> 1] += dA * __half2float(bmm[r * LDC + i]);
+                    y[mi][nt][e] = beta[r] * dA * __half2float(decm[r * LDC + i]);   // dB * D
                 }
             store_h(y[mi], mi, 2, OC_U, LDC, n64, 1.f);   // dT is dead (read for X)
         }
@@ -701,7 +767,7 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
     {
         float p[2][4][4];
         zero2<4>(p);
-        wgemm2<4, 2, false, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale2());
+        wgemm2<4, 2, false, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LQ, n128, lane, NoScale2());
         rowdot(p, OC_K, n128, pg);
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
@@ -710,8 +776,8 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dk[mi][nt][e] += p[mi][nt][e];
         zero2<4>(p);
-        wgemm2<4, 2, true, true>(p, sb + OC_M, LDC, r0, sb + OC_Q, LDD, n128, lane, NoScale2());
-        wgemm2<4, 2, true, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LDD, n128, lane, NoScale2());
+        wgemm2<4, 2, true, true>(p, sb + OC_M, LDC, r0, sb + OC_Q, LQ, n128, lane, NoScale2());
+        wgemm2<4, 2, true, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LQ, n128, lane, NoScale2());
         float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         rowdot(p, OC_K, n128, s);
 #pragma unroll
@@ -724,8 +790,13 @@ __global__ void __launch_bounds__(NTC, 1) bwdc_chunk_kernel(BwdArgs a, BwdcWs ws
                 float *dst = a.dk + (((size_t)b * a.T + c * C + r) * a.Hk + hk) * D + n128 + 2 * t4;
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    atomicAdd(dst + 8 * nt, dk[mi][nt][2 * hi] + p[mi][nt][2 * hi]);
-                    atomicAdd(dst + 8 * nt + 1, dk[mi][nt][2 * hi + 1] + p[mi][nt][2 * hi + 1]);
+                    const float k0 = dk[mi][nt][2 * hi] + p[mi][nt][2 * hi], k1 = dk[mi][nt][2 * hi + 1] + p[mi][nt][2 * hi + 1];
+                    if (sole) {
+                        *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(k0, k1);
+                    } else {
+                        atomicAdd(dst + 8 * nt, k0);
+                        atomicAdd(dst + 8 * nt + 1, k1);
+                    }
                 }
             }
     }
@@ -815,7 +886,11 @@ cudaError_t launch_bwdc(const BwdArgs &a, void *workspace, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwdc_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_CHUNK);
     if (e != cudaSuccess) return e;
-    bwdc_chunk_kernel<<<(unsigned)cu, NTC, SMEM_CHUNK, st>>>(a, ws);
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, a.q, a.B, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, a.B, a.T, a.Hk, 64, false, true) ||
+        !make_map(&mv, a.v, a.B, a.T, a.Hv, 64, false, true))
+        return cudaErrorInvalidValue;
+    bwdc_chunk_kernel<<<(unsigned)cu, NTC, SMEM_CHUNK, st>>>(a, ws, sm_count(), a.Hv == a.Hk ? 1 : 0, mq, mk, mv, mdo);
     return cudaGetLastError();
 }
 

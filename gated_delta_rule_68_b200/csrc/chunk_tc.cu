@@ -317,7 +317,8 @@ __device__ __forceinline__ void st_global_h8(void *gp, const float *v)
     u.w = pack_h2(v[6], v[7]);
     *reinterpret_cast<uint4 *>(gp) = u;
 }
-// Block (R0.., I0..) of T (two n8 tiles times s) into the unit's [64][64] fp16 T in global memory.
+// Block (R0.., I0..) of T (two n8 tiles times s) into the chunk's [64][64] fp16 T in global memory,
+// as the image of a 128-byte swizzled tile.
 __device__ __forceinline__ void st_tglobal(__half *tg, int R0, int I0, const float c0[4], const float c1[4], float s,
                                            int lane)
 {
@@ -328,7 +329,8 @@ __device__ __forceinline__ void st_tglobal(__half *tg, int R0, int I0, const flo
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int r = R0 + g + 8 * hh, i = I0 + 8 * nt + 2 * t4;
-            *reinterpret_cast<uint32_t *>(tg + r * 64 + i) = pack_h2(s * c[2 * hh], s * c[2 * hh + 1]);
+            *reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(tg) + swz_off(r, i, 0)) =
+                pack_h2(s * c[2 * hh], s * c[2 * hh + 1]);
         }
     }
 }
@@ -337,9 +339,9 @@ __device__ __forceinline__ void st_tglobal(__half *tg, int R0, int I0, const flo
 // exactly its own code): q and k rows divided by sqrt(sum of squares + 1e-6) as they are
 // converted, and o rows replaced by o / sqrt(mean(o^2) + eps) * weight * SiLU(z).
 // SAVE (scalar gate, one CTA per unit): the first pass of the chunked backward. Per chunk it
-// also writes the entering state S^T, T (unscaled; the lower triangle and diagonal blocks)
-// and the images of the P and Qh^T operand tiles (128-byte swizzled) to the caller's buffers
-// as fp16, and stores no o.
+// also writes, as fp16 images of 128-byte swizzled tiles, the entering state S^T, T
+// (unscaled; the lower triangle and diagonal blocks) and the P and Qh^T operand tiles to the
+// caller's buffers, and stores no o.
 template <typename TOut, bool NORM, int GATE, bool SCHED, bool SAVE = false>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -579,7 +581,7 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                         *reinterpret_cast<uint32_t *>(sm + INV_D + (uint32_t)((wq * 16 + r) * LDT16 + col) * 2u) =
                             pack_h2(x0, x1);
                         *reinterpret_cast<uint32_t *>(sm + OFF_TPP + swz_off(I0 + r, i, 0)) = pack_h2(w0, w1);
-                        if (SAVE) *reinterpret_cast<uint32_t *>(tg + (I0 + r) * C + i) = pack_h2(x0, x1);
+                        if (SAVE) *reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(tg) + swz_off(I0 + r, i, 0)) = pack_h2(x0, x1);
                         if (GATE == 0) {
                             const float u0 = x0 * vc[V_BG + i], u1 = x1 * vc[V_BG + i + 1];
                             *reinterpret_cast<uint32_t *>(sm + OFF_TP + swz_off(I0 + r, i, 0)) = pack_h2(u0, u1);
@@ -1089,9 +1091,9 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             for (int dk = 0; dk < 64; ++dk) S[dk] = h0 ? __ldcg(h0 + (size_t)dk * D) : 0.f;
             if (GATE == 0) store_s16(gsb);
             if (SAVE) {   // the state entering chunk 0: row p of S^T, columns 64 hf ..
-                __half *sg = reinterpret_cast<__half *>(a.save_s) + ((size_t)bh * NC * D + p) * D + 64 * hf;
+                uint8_t *sg = reinterpret_cast<uint8_t *>(a.save_s) + (size_t)bh * NC * (D * D * 2);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_global_h8(sg + 8 * j, S + 8 * j);
+                for (int j = 0; j < 8; ++j) st_global_h8(sg + swz_chunk(p, j, hf * 16384), S + 8 * j);
             }
         }
         float gbn[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1197,10 +1199,11 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     }
                     tmem_st16(tmem_addr(tb, q4, TM_S16 + 32 * hf + 16 * h2), w);
                     if (SAVE && c + 1 < c1) {   // the state entering chunk c + 1, as its fp16 copy
-                        uint4 *sg = reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(a.save_s) +
-                                                              (((size_t)bh * NC + c + 1) * D + p) * D + 64 * hf + 32 * h2);
+                        uint8_t *sg = reinterpret_cast<uint8_t *>(a.save_s) + ((size_t)bh * NC + c + 1) * (D * D * 2);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) sg[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(sg + swz_chunk(p, 4 * h2 + j, hf * 16384)) =
+                                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
                     }
                 }
                 tmem_wait_st();

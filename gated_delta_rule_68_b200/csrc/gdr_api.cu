@@ -343,9 +343,14 @@ int gdr_bwd_chunked(const void *q, const void *k, const void *v, const float *g,
     if (!workspace || workspace_bytes < need)
         return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given%s", need, workspace_bytes,
                     workspace ? "" : " (NULL)");
+    // dq and dk are sums over the value heads of a key head; with one value head per key head
+    // each element has one writer and no zeroing is needed
     const size_t nqk = (size_t)B * T * Hk * Dk * sizeof(float);
-    cudaError_t e = cudaMemsetAsync(dq, 0, nqk, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nqk, s);
+    cudaError_t e = cudaSuccess;
+    if (Hv != Hk) {
+        e = cudaMemsetAsync(dq, 0, nqk, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nqk, s);
+    }
     if (e == cudaSuccess) e = gdr::launch_bwdc(a, workspace, s);
     if (e != cudaSuccess) return fail(GDR_ERR_CUDA, "CUDA launch failed: %s", cudaGetErrorString(e));
     g_launches += 3;

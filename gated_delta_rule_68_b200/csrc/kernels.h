@@ -40,10 +40,10 @@ struct FwdArgs {
     unsigned long long sched_tag = 0;
     unsigned long long *sched_flags = nullptr;
     float *sched_states = nullptr;
-    // tcgen05 kernel, scalar gate: the chunked backward's forward pass. Per (unit, chunk),
-    // fp16: the entering state S^T [Dv][Dk], T [64][64] (the lower triangle; entries above
-    // the diagonal blocks are not written), and the images of the P [Dk][Dk] and Qh^T [Dk][64]
-    // operand tiles in the 128-byte swizzle (32 and 16 KB). No o is stored.
+    // tcgen05 kernel, scalar gate: the chunked backward's forward pass. Per (unit, chunk), the
+    // fp16 images of 128-byte swizzled tiles (64-column atoms): the entering state S^T
+    // [Dv][Dk] and P [Dk][Dk] (32 KB), Qh^T [Dk][64] (16 KB), T [64][64] (8 KB; the lower
+    // triangle, entries above the diagonal blocks are not written). No o is stored.
     void *save_s = nullptr, *save_p = nullptr, *save_qh = nullptr, *save_t = nullptr;
 };
 
@@ -86,8 +86,8 @@ bool bwd_supported(const BwdArgs &a);
 size_t bwd_workspace_size(const BwdArgs &a);
 cudaError_t launch_bwd(const BwdArgs &a, void *ws, cudaStream_t st);
 // Chunked backward on tensor cores (bwd_chunk.cu): scalar gate, bf16 inputs, Dk = Dv = 128.
-// dq and dk are accumulated with atomics and must be zero on entry; dv, dg, dbeta and dh0
-// are written once.
+// With more value heads than key heads dq and dk are accumulated with atomics and must be
+// zero on entry; otherwise they are written once, as are dv, dg, dbeta and dh0.
 bool bwdc_supported(const BwdArgs &a);
 size_t bwdc_workspace_size(const BwdArgs &a);
 cudaError_t launch_bwdc(const BwdArgs &a, void *ws, cudaStream_t st);
