@@ -145,6 +145,12 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes
 {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
+// One TMA box into L2 (no shared-memory destination).
+__device__ __forceinline__ void prefetch_tma_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -429,28 +435,8 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
         vec[VG + tid] = ok ? a.g[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
         vec[VBETA + tid] = ok ? a.beta[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
     }
-    {   // the inputs of the CTA pf launches later into L2, while this one computes
-        const long nb = (long)blockIdx.x + pf;
-        if (pf > 0 && nb < (long)gridDim.x) {
-            const int nu = (int)(nb / NC), ncc = (int)(nb % NC);
-            const int n_b = nu / a.Hv, n_h = nu % a.Hv, n_hk = n_h / (a.Hv / a.Hk);
-            const int m = tid >> 6, r = tid & 63, t = ncc * C + r;
-            if (t < a.T) {
-                const void *src = m == 0 ? a.q : m == 1 ? a.k : m == 2 ? a.v : a.dout;
-                const int H = m < 2 ? a.Hk : a.Hv, hh = m < 2 ? n_hk : n_h;
-                prefetch_l2_bulk(reinterpret_cast<const __nv_bfloat16 *>(src) + (((size_t)n_b * a.T + t) * H + hh) * D,
-                                 D * 2);
-            }
-            if (tid == 0) {
-                const size_t ncu = (size_t)nu * NC + ncc;
-                prefetch_l2_bulk(ws.s + ncu * D * D, D * D * 2);
-                prefetch_l2_bulk(ws.ds + ncu * D * D, D * D * 2);
-                prefetch_l2_bulk(ws.t + ncu * C * C, C * C * 2);
-            }
-        }
-    }
     wait(bar0);
-    for (int i = tid; i < 4 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_Q + 16 * i);   // q, k, v, dO to fp16
+    for (int i = tid; i < 2 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_Q + 16 * i);   // q, k to fp16
     // T is lower triangular: clear what the forward left unwritten above the diagonal blocks
     for (int i = tid; i < C * 8; i += NTC) {
         const int r = i >> 3, j = i & 7;
@@ -565,10 +551,31 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
 #pragma unroll
             for (int mi = 0; mi < 2; ++mi) store_h(w[mi], mi, 4, OC_W, LDD, n128, 1.f);
         }
+        // v and dO to fp16 (v for U, dO from c on), while S^T and dS_next^T arrive
+        for (int i = tid; i < 2 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_V + 16 * i);
+        __syncthreads();
         zero2<4>(u);
         wgemm2<4, 2, false, true>(u, sb + OC_T, LT, r0, sb + OC_V, LQ, n128, lane, colscale(beta, nullptr));
         wait(bar1);   // S^T and dS_next^T
         __syncthreads();
+        if (tid == 0 && pf > 0 && (long)blockIdx.x + pf < (long)gridDim.x) {
+            // the inputs of the CTA pf launches later, into L2 while this one computes (its own
+            // loads have landed, so the two do not compete): eight TMA boxes and three spans
+            const long nbk = (long)blockIdx.x + pf;
+            const int nu = (int)(nbk / NC), ncc = (int)(nbk % NC);
+            const int n_b = nu / a.Hv, n_h = nu % a.Hv, n_hk = n_h / (a.Hv / a.Hk), nt0 = ncc * C;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                prefetch_tma_4d(&map_q, 64 * x, n_hk, nt0, n_b);
+                prefetch_tma_4d(&map_k, 64 * x, n_hk, nt0, n_b);
+                prefetch_tma_4d(&map_v, 64 * x, n_h, nt0, n_b);
+                prefetch_tma_4d(&map_do, 64 * x, n_h, nt0, n_b);
+            }
+            const size_t ncu = (size_t)nu * NC + ncc;
+            prefetch_l2_bulk(ws.s + ncu * D * D, D * D * 2);
+            prefetch_l2_bulk(ws.ds + ncu * D * D, D * D * 2);
+            prefetch_l2_bulk(ws.t + ncu * C * C, C * C * 2);
+        }
         {   // sum(dS_next * S) over the whole state
             float s = 0.f;
             for (int i = tid; i < D * 16; i += NTC) {   // the two images share one layout
