@@ -365,6 +365,57 @@ __device__ __forceinline__ void wgemm2(float (*acc)[2 * NP][4], uint32_t aB, int
         }
     }
 }
+// Two products of the same shape in lockstep (twice the independent MMAs per k-step):
+// acc1 += A1 B1, acc2 += A2 B2. SA: A2 is A1's tile (loaded once, then scaled by each
+// product's ascale); SB: B2 is B1's tile (loaded once).
+template <int KS, int NP, bool AT1, bool BT1, bool AT2, bool BT2, bool SA, bool SB, typename AS1, typename AS2>
+__device__ __forceinline__ void wgemm2_pair(float (*acc1)[2 * NP][4], uint32_t a1, int lda1, uint32_t b1, int ldb1,
+                                            AS1 as1, float (*acc2)[2 * NP][4], uint32_t a2, int lda2, uint32_t b2,
+                                            int ldb2, AS2 as2, int r0, int n0, int lane)
+{
+    auto lda_ = [&](uint32_t *f, uint32_t aB, int lda, bool at, int m0, int k0) {
+        if (at) ldsm_t(f, taddr(aB, lda, k0 + (lane & 7) + (lane >> 4) * 8, m0 + ((lane >> 3) & 1) * 8));
+        else ldsm(f, taddr(aB, lda, m0 + (lane & 7) + ((lane >> 3) & 1) * 8, k0 + (lane >> 4) * 8));
+    };
+    auto ldb_ = [&](uint32_t *f, uint32_t bB, int ldb, bool bt, int nn, int k0) {
+        if (bt) ldsm_t(f, taddr(bB, ldb, k0 + (lane & 7) + ((lane >> 3) & 1) * 8, nn + (lane >> 4) * 8));
+        else ldsm(f, taddr(bB, ldb, nn + (lane & 7) + (lane >> 4) * 8, k0 + ((lane >> 3) & 1) * 8));
+    };
+#pragma unroll 2
+    for (int j = 0; j < KS; ++j) {
+        uint32_t f1[2][4], f2[2][4];
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+            lda_(f1[mi], a1, lda1, AT1, r0 + 16 * mi, 16 * j);
+            if (SA) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f2[mi][e] = f1[mi][e];
+            } else {
+                lda_(f2[mi], a2, lda2, AT2, r0 + 16 * mi, 16 * j);
+            }
+            as1(f1[mi], j, mi);
+            as2(f2[mi], j, mi);
+        }
+#pragma unroll
+        for (int np = 0; np < NP; ++np) {
+            uint32_t g1[4], g2[4];
+            ldb_(g1, b1, ldb1, BT1, n0 + 16 * np, 16 * j);
+            if (SB) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) g2[e] = g1[e];
+            } else {
+                ldb_(g2, b2, ldb2, BT2, n0 + 16 * np, 16 * j);
+            }
+#pragma unroll
+            for (int mi = 0; mi < 2; ++mi) {
+                mma(acc1[mi][2 * np], f1[mi], g1[0], g1[1]);
+                mma(acc2[mi][2 * np], f2[mi], g2[0], g2[1]);
+                mma(acc1[mi][2 * np + 1], f1[mi], g1[2], g1[3]);
+                mma(acc2[mi][2 * np + 1], f2[mi], g2[2], g2[3]);
+            }
+        }
+    }
+}
 struct NoScale2 {
     __device__ __forceinline__ void operator()(uint32_t *, int, int) const {}
 };
@@ -510,8 +561,8 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
         float qk[2][2][4], kk[2][2][4];
         zero2<2>(qk);
         zero2<2>(kk);
-        wgemm2<8, 1, false, false>(qk, sb + OC_Q, LQ, r0, sb + OC_K, LQ, n64, lane, NoScale2());
-        wgemm2<8, 1, false, false>(kk, sb + OC_K, LQ, r0, sb + OC_K, LQ, n64, lane, NoScale2());
+        wgemm2_pair<8, 1, false, false, false, false, false, true>(qk, sb + OC_Q, LQ, sb + OC_K, LQ, NoScale2(), kk,
+                                                                   sb + OC_K, LQ, sb + OC_K, LQ, NoScale2(), r0, n64, lane);
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
@@ -544,18 +595,19 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
                 hmul_frag(af[3], hi);
             };
         };
+        // v and dO to fp16 (v for U, dO from c on)
+        for (int i = tid; i < 2 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_V + 16 * i);
+        __syncthreads();
         {
             float w[2][4][4];
             zero2<4>(w);
-            wgemm2<4, 2, false, true>(w, sb + OC_T, LT, r0, sb + OC_K, LQ, n128, lane, colscale(beta, Gam));
+            zero2<4>(u);
+            wgemm2_pair<4, 2, false, true, false, true, true, false>(w, sb + OC_T, LT, sb + OC_K, LQ, colscale(beta, Gam), u,
+                                                                     sb + OC_T, LT, sb + OC_V, LQ, colscale(beta, nullptr),
+                                                                     r0, n128, lane);
 #pragma unroll
             for (int mi = 0; mi < 2; ++mi) store_h(w[mi], mi, 4, OC_W, LDD, n128, 1.f);
         }
-        // v and dO to fp16 (v for U, dO from c on), while S^T and dS_next^T arrive
-        for (int i = tid; i < 2 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_V + 16 * i);
-        __syncthreads();
-        zero2<4>(u);
-        wgemm2<4, 2, false, true>(u, sb + OC_T, LT, r0, sb + OC_V, LQ, n128, lane, colscale(beta, nullptr));
         wait(bar1);   // S^T and dS_next^T
         __syncthreads();
         if (tid == 0 && pf > 0 && (long)blockIdx.x + pf < (long)gridDim.x) {
@@ -687,9 +739,11 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
     __syncthreads();
     // ---- h: dV = diag(beta) T^T dU', and dK1's first part diag(Gamma beta) T^T dW
     {
-        float y[2][4][4];
+        float y[2][4][4], y2[2][4][4];
         zero2<4>(y);
-        wgemm2<4, 2, true, true>(y, sb + OC_T, LT, r0, sb + OC_W, LDD, n128, lane, NoScale2());
+        zero2<4>(y2);
+        wgemm2_pair<4, 2, true, true, true, true, true, false>(y, sb + OC_T, LT, sb + OC_W, LDD, NoScale2(), y2,
+                                                               sb + OC_T, LT, sb + OC_DS, LDD, NoScale2(), r0, n128, lane);
         rowdot(y, OC_V, n128, pb);   // rowsum(V * T^T dU')
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
@@ -703,10 +757,8 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
                 for (int nt = 0; nt < 4; ++nt)
                     *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(br * y[mi][nt][2 * hi], br * y[mi][nt][2 * hi + 1]);
             }
-        zero2<4>(y);
-        wgemm2<4, 2, true, true>(y, sb + OC_T, LT, r0, sb + OC_DS, LDD, n128, lane, NoScale2());
         float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        rowdot(y, OC_K, n128, s);   // rowsum(K * T^T dW)
+        rowdot(y2, OC_K, n128, s);   // rowsum(K * T^T dW)
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
@@ -717,8 +769,8 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
                 pg[mi][hi] += gbr * s[mi][hi];   // rowsum(dK1a * K)
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    dk[mi][nt][2 * hi] += gbr * y[mi][nt][2 * hi];
-                    dk[mi][nt][2 * hi + 1] += gbr * y[mi][nt][2 * hi + 1];
+                    dk[mi][nt][2 * hi] += gbr * y2[mi][nt][2 * hi];
+                    dk[mi][nt][2 * hi + 1] += gbr * y2[mi][nt][2 * hi + 1];
                 }
             }
     }
@@ -727,8 +779,8 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
         float x1[2][2][4], x2[2][2][4];
         zero2<2>(x1);
         zero2<2>(x2);
-        wgemm2<8, 1, false, false>(x1, sb + OC_W, LDD, r0, sb + OC_V, LQ, n64, lane, NoScale2());
-        wgemm2<8, 1, false, false>(x2, sb + OC_DS, LDD, r0, sb + OC_K, LQ, n64, lane, NoScale2());
+        wgemm2_pair<8, 1, false, false, false, false, false, false>(x1, sb + OC_W, LDD, sb + OC_V, LQ, NoScale2(), x2,
+                                                                    sb + OC_DS, LDD, sb + OC_K, LQ, NoScale2(), r0, n64, lane);
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll

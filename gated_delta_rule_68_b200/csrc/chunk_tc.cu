@@ -187,14 +187,14 @@ __device__ __forceinline__ void st_chunk8(uint32_t addr, const float *x)
                  "r"(pack_h2(x[2], x[3])), "r"(pack_h2(x[4], x[5])), "r"(pack_h2(x[6], x[7]))
                  : "memory");
 }
-// The same 8 fp16 values into shared memory and to a 16-byte aligned global address.
-__device__ __forceinline__ void st_chunk8_g(uint32_t addr, const float *x, void *gp)
+// A shared-memory span to global memory by the bulk-copy engine (both 16-byte aligned, a
+// multiple of 16 bytes), tracked in this thread's bulk groups.
+__device__ __forceinline__ void bulk_s2g(void *gdst, uint32_t ssrc, uint32_t bytes)
 {
-    const uint4 u = make_uint4(pack_h2(x[0], x[1]), pack_h2(x[2], x[3]), pack_h2(x[4], x[5]), pack_h2(x[6], x[7]));
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
                  : "memory");
-    *reinterpret_cast<uint4 *>(gp) = u;
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void st_h1(uint8_t *sm, uint32_t off, float x)
 {
     *reinterpret_cast<__half *>(sm + off) = __float2half_rn(x);
@@ -341,7 +341,8 @@ __device__ __forceinline__ void st_tglobal(__half *tg, int R0, int I0, const flo
 // SAVE (scalar gate, one CTA per unit): the first pass of the chunked backward. Per chunk it
 // also writes, as fp16 images of 128-byte swizzled tiles, the entering state S^T, T
 // (unscaled; the lower triangle and diagonal blocks) and the P and Qh^T operand tiles to the
-// caller's buffers, and stores no o.
+// caller's buffers, and stores no o. P, Qh^T and S^T (staged in the P tile once the products
+// have read it) go out by bulk copies from shared memory, T from the inverse's registers.
 template <typename TOut, bool NORM, int GATE, bool SCHED, bool SAVE = false>
 __global__ void __launch_bounds__(NTH, 1)
 tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -1125,15 +1126,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[32];
                 tmem_ld32(tmem_addr(tb, q4, TM_X + 32 * hf), v);
-                if (SAVE) {   // and to global memory: the tile's image, 16 KB per chunk
-                    uint8_t *qg = reinterpret_cast<uint8_t *>(a.save_qh) + ((size_t)bh * NC + c) * 16384;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        st_chunk8_g(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j, qg + swz_chunk(p, 4 * hf + j, 0));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
-                }
+                for (int j = 0; j < 4; ++j) st_chunk8(sb0 + swz_chunk(p, 4 * hf + j, OFF_QH16), v + 8 * j);
             }
             wait(B_P, gs & 1);
             if (issuer && c + 2 < c1) issue_loads(c + 2, gs + 2);   // chunk c's staging buffer is free
@@ -1144,15 +1138,8 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             {
                 float v[64];
                 tmem_ld32x2(tmem_addr(tb, q4, TM_Y + 64 * hf), tmem_addr(tb, q4, TM_Y + 64 * hf + 32), v);
-                if (SAVE) {   // and to global memory: the tile's image, 32 KB per chunk
-                    uint8_t *pg = reinterpret_cast<uint8_t *>(a.save_p) + ((size_t)bh * NC + c) * 32768;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        st_chunk8_g(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j, pg + swz_chunk(p, j, hf * 16384));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
-                }
+                for (int j = 0; j < 8; ++j) st_chunk8(sb0 + swz_chunk(p, j, OFF_P16 + hf * 16384), v + 8 * j);
             }
             const float gC = GATE ? 0.f : vec[(gs & 1) * V_SET + V_GC];
             tc_fence_before();
@@ -1171,9 +1158,19 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                     mma_ts(tb + TM_O, tb + TM_S16 + 8 * s, sdesc(sb0 + OFF_QH16 + s * 2048, 8192, 1024), ID_O, true);
                 }
                 mma_commit(bar(B_ST));
+                if (SAVE) {   // the finished P and Qh^T tiles, as they are, to the caller's buffers
+                    const size_t cu = (size_t)bh * NC + c;
+                    bulk_s2g(reinterpret_cast<uint8_t *>(a.save_p) + cu * 32768, sb0 + OFF_P16, 32768);
+                    bulk_s2g(reinterpret_cast<uint8_t *>(a.save_qh) + cu * 16384, sb0 + OFF_QH16, 16384);
+                    bulk_commit();
+                }
             }
             wait(B_ST, gs & 1);
             tc_fence_after();
+            if (SAVE) {   // the copies have read P and Qh^T: the P tile holds the state's image next
+                if (issuer) tma_store_wait_read();
+                named_bar_sync(2, GT);
+            }
             // S <- Gamma_C S + (P S + R), and its fp16 copy for the next batch
             if (GATE == 0 && NORM) {
                 // The layer instance's state group is its longer chain: one TMEM wait for all
@@ -1198,15 +1195,23 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
                         w[j] = pack_h2(S[32 * h2 + 2 * j], S[32 * h2 + 2 * j + 1]);
                     }
                     tmem_st16(tmem_addr(tb, q4, TM_S16 + 32 * hf + 16 * h2), w);
-                    if (SAVE && c + 1 < c1) {   // the state entering chunk c + 1, as its fp16 copy
-                        uint8_t *sg = reinterpret_cast<uint8_t *>(a.save_s) + ((size_t)bh * NC + c + 1) * (D * D * 2);
+                    if (SAVE && c + 1 < c1) {   // the state entering chunk c + 1: its image in the P tile
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            *reinterpret_cast<uint4 *>(sg + swz_chunk(p, 4 * h2 + j, hf * 16384)) =
+                            *reinterpret_cast<uint4 *>(sm + swz_chunk(p, 4 * h2 + j, OFF_P16 + hf * 16384)) =
                                 make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
                     }
                 }
                 tmem_wait_st();
+                if (SAVE && c + 1 < c1) {   // ... and from there to the caller's buffer
+                    fence_proxy_async();
+                    named_bar_sync(2, GT);
+                    if (issuer) {
+                        bulk_s2g(reinterpret_cast<uint8_t *>(a.save_s) + ((size_t)bh * NC + c + 1) * (D * D * 2),
+                                 sb0 + OFF_P16, D * D * 2);
+                        bulk_commit();
+                    }
+                }
             } else {   // S <- diag(Gamma_C) S + (P S + R), row dk = 64 hf + i, in two halves of 32
                 const float4 *g4 = reinterpret_cast<const float4 *>(vec + (gs & 1) * KV_SET + KV_GC + 64 * hf);
 #pragma unroll
@@ -1233,6 +1238,10 @@ tc_fwd_kernel(FwdArgs a, const __grid_constant__ CUtensorMap map_q, const __grid
             // columns p - 1 and p).
             const int nvalid = min(C, T - c * C);
             const bool tile = !(a.cu_seqlens && nvalid < C);
+            if (SAVE) {   // the copy has read the state's image before o is written there
+                if (issuer) tma_store_wait_read();
+                named_bar_sync(2, GT);
+            }
             if (NORM && a.z) {
                 // Pass A: fp32 o into the P tile (dead until the next chunk), in the TMA swizzle of
                 // an fp32 o tile. Pass B, a row per 4 threads (row r = 8 warp + lane % 8, columns
