@@ -120,7 +120,9 @@ KERNEL_SOURCES = {
     "fused_fwd_kernel": ("chunk_mma.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
     "bwd_kernel": ("bwd.cu", "common.cuh", "kernels.h"),
     "decode_kernel": ("decode.cu", "common.cuh", "kernels.h"),
-    "bwdc_chunk_kernel": ("bwd_chunk.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
+    "bwdc_chunk_kernel": ("bwd_chunk.cu", "mma_util.cuh", "tc_util.cuh", "common.cuh", "kernels.h"),
+    # the chunked backward's step: its forward pass, scan and chunk kernels together
+    "bwdc_step": ("bwd_chunk.cu", "chunk_tc.cu", "mma_util.cuh", "tc_util.cuh", "common.cuh", "kernels.h"),
 }
 
 
@@ -835,6 +837,43 @@ def run_decode_bench(args, w, wr, rank, world, local, dev):
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, dev)
 
+    # The same steps captured in a CUDA graph and replayed (the entry point allocates nothing
+    # and does not synchronise), at this batch and at a serving batch of 4 rows where launch
+    # overhead shows; outside the timed region.
+    def graph_ms(bw):
+        winp = make_inputs(wr.with_(B=bw, T=args.steps), "cpu")
+        winp = {n: t.to(dev) for n, t in winp.items()}
+        st = winp["h0"].clone()
+        ob = torch.empty((args.steps, bw, w.Hv, w.Dv), dtype=w.torch_dtype, device=dev)
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+
+        def run(strm):
+            for s in range(args.steps):
+                gdr.gdr_decode_step(winp["q"][s], winp["k"][s], winp["v"][s], winp["g"][s], winp["beta"][s], st,
+                                    o=ob[s], stream=strm)
+
+        run(stream)   # eager, warm
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        run(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        eager = t0.elapsed_time(t1) / args.steps
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            run(cap)
+        graph.replay()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return {"batch": bw, "eager_ms_per_step": eager, "graph_ms_per_step": t0.elapsed_time(t1) / args.steps}
+
+    cuda_graph = [graph_ms(w.B), graph_ms(4)] if world == 1 else None
+
     e2e = None
     if not args.no_e2e:   # one token's inputs up, its outputs down, every step
         host = {n: inp_cpu[n][0].pin_memory() for n in ("q", "k", "v", "g", "beta")}
@@ -883,7 +922,7 @@ def run_decode_bench(args, w, wr, rank, world, local, dev):
                      "traffic": traffic, "traffic_kernel": traffic_kernel, "kernel": "gdr_decode_step"},
         "cpu_baseline": decode_oracle_sample(w) if world == 1 and not args.no_cpu_baseline else None,
         "e2e": e2e, "gpu_launches": launches,
-        "launches_per_step": launches / args.steps, "clocks": clk.summary(),
+        "launches_per_step": launches / args.steps, "clocks": clk.summary(), "cuda_graph": cuda_graph,
     }
     print(json.dumps(line), flush=True)
     return 0
