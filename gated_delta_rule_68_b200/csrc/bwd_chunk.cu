@@ -9,11 +9,13 @@
 // and the gradients of the chunk's own inputs depend only on S, dS_next, dO and the
 // chunk's inputs. Three passes:
 //   1. the tcgen05 forward (chunk_tc.cu, its SAVE instance) stores, per chunk, the
-//      entering state S^T, P, Qh^T and T = (I + A)^-1 in fp16;
-//   2. bwdc_scan_kernel: per (batch row, value head), the chunks in reverse; dS^T is
-//      carried in fp32 warp-MMA accumulators and stored per chunk (as dS_next of that
-//      chunk) in fp16; the last one is dh0;
-//   3. bwdc_chunk_kernel: one CTA per (unit, chunk), all chunks at once. With the
+//      entering state S^T, P, Qh^T and T = (I + A)^-1 as fp16 images of 128-byte swizzled
+//      tiles;
+//   2. bwdc_scan_kernel: per (batch row, value head), the chunks in reverse on tcgen05;
+//      dS^T is carried in fp32 registers, its fp16 copy in tensor memory is the products'
+//      A operand, and it is stored per chunk (as dS_next of that chunk); the last is dh0;
+//   3. bwdc_chunk_kernel: one CTA per (unit, chunk), all chunks at once, on the warp-level
+//      MMAs (mma.sync, fp16 operands, fp32 accumulation). With the
 //      in-chunk decays D_ri = exp(G_r - G_i) (r >= i) and f = Gamma_C / Gamma:
 //        W = T diag(beta Gamma) K,  U = T diag(beta) V,  U' = U - W S
 //        dU' = M^T dO + diag(f) K dS_next,       M = tril(Q K^T * D)
@@ -27,7 +29,6 @@
 //        dG = rowsum((dK1 - dK2 - dK3) * K + dQ * Q), and its last row adds
 //             sum(dK3 * K) + Gamma_C sum(dS_next * S); dg = reverse cumulative sum of dG.
 //      Every factor is relative (at most 1), as in the forward.
-// Products are warp-level mma.sync (fp16 operands, fp32 accumulation).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -49,12 +50,6 @@ constexpr int NT = 256;   // 8 warps
 struct BwdcWs {
     __half *s, *p, *qh, *t, *ds;   // S^T [Dv][Dk], P [Dk][Dk], Qh^T [Dk][64], T [64][64], dS_next^T [Dv][Dk]
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_h2f(float x, float y)
 {
@@ -84,40 +79,6 @@ __device__ __forceinline__ void hmul_frag(uint32_t &r, __half2 s)
     __half2 h = *reinterpret_cast<__half2 *>(&r);
     h = __hmul2(h, s);
     r = *reinterpret_cast<uint32_t *>(&h);
-}
-
-// acc[2 NP][4] += A (16 rows from r0, K = 16 KS) B (columns n0 .. n0 + 16 NP).
-// A: row-major [m][k] (AT false) or stored transposed [k][m] (AT true);
-// B: stored [n][k] (BT false) or [k][n] (BT true). ascale(af, j) may rescale the A
-// fragment of k-step j in registers.
-template <int KS, int NP, bool AT, bool BT, typename AS>
-__device__ __forceinline__ void wgemm(float (*acc)[4], uint32_t aB, int lda, int r0, uint32_t bB, int ldb, int n0,
-                                      int lane, AS ascale)
-{
-#pragma unroll
-    for (int j = 0; j < KS; ++j) {
-        uint32_t af[4];
-        if (AT) ldsm_t(af, a_tr(aB, lda, r0, 16 * j, lane));
-        else ldsm(af, a_rm(aB, lda, r0, 16 * j, lane));
-        ascale(af, j);
-#pragma unroll
-        for (int np = 0; np < NP; ++np) {
-            uint32_t bf[4];
-            if (BT) ldsm_t(bf, b_kn(bB, ldb, n0 + 16 * np, 16 * j, lane));
-            else ldsm(bf, b_nk(bB, ldb, n0 + 16 * np, 16 * j, lane));
-            mma(acc[2 * np], af, bf[0], bf[1]);
-            mma(acc[2 * np + 1], af, bf[2], bf[3]);
-        }
-    }
-}
-struct NoScale {
-    __device__ __forceinline__ void operator()(uint32_t *, int) const {}
-};
-template <int N>
-__device__ __forceinline__ void zero_acc(float (*acc)[4])
-{
-#pragma unroll
-    for (int i = 0; i < N; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 }
 
 // ------------------------------------------------------------------ pass 2: the reverse scan
@@ -335,8 +296,11 @@ __device__ __forceinline__ uint32_t taddr(uint32_t base, int ld, int row, int co
     return base + (uint32_t)(col >> 6) * (uint32_t)(-ld) + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
            (((uint32_t)((col & 63) >> 3) ^ (uint32_t)(row & 7)) << 4) + (uint32_t)(col & 7) * 2u;
 }
-// acc[2][2 NP][4] += A (rows r0 .. r0 + 31, K = 16 KS) B (columns n0 .. n0 + 16 NP), as wgemm.
-// ascale(af, j, mi) may rescale the A fragment of k-step j, row block mi.
+// acc[2][2 NP][4] += A (rows r0 .. r0 + 31, K = 16 KS) B (columns n0 .. n0 + 16 NP) on the
+// warp-level MMAs (m16n8k16, fp16 operands, fp32 accumulators in the m16n8 layout).
+// A: [m][k] (AT false) or stored transposed [k][m] (AT true); B: stored [n][k] (BT false) or
+// [k][n] (BT true); each tile by its ld (see taddr). ascale(af, j, mi) may rescale the A
+// fragment of k-step j, row block mi, in registers.
 template <int KS, int NP, bool AT, bool BT, typename AS>
 __device__ __forceinline__ void wgemm2(float (*acc)[2 * NP][4], uint32_t aB, int lda, int r0, uint32_t bB, int ldb,
                                        int n0, int lane, AS ascale)
