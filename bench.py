@@ -120,7 +120,7 @@ KERNEL_SOURCES = {
     "fused_fwd_kernel": ("chunk_mma.cu", "mma_util.cuh", "common.cuh", "kernels.h"),
     "bwd_kernel": ("bwd.cu", "common.cuh", "kernels.h"),
     "decode_kernel": ("decode.cu", "common.cuh", "kernels.h"),
-    "bwdc_chunk_kernel": ("bwd_chunk.cu", "mma_util.cuh", "tc_util.cuh", "common.cuh", "kernels.h"),
+    "bwdc_tc_kernel": ("bwd_chunk.cu", "mma_util.cuh", "tc_util.cuh", "common.cuh", "kernels.h"),
     # the chunked backward's step: its forward pass, scan and chunk kernels together
     "bwdc_step": ("bwd_chunk.cu", "chunk_tc.cu", "mma_util.cuh", "tc_util.cuh", "common.cuh", "kernels.h"),
 }
@@ -510,8 +510,9 @@ def bwd_flops(w):
 def bwdc_flops(w):
     """Tensor-core flops per call of the chunked backward, per (unit, 64-token chunk): the
     forward pass's products (Gram [K; Q] K^T, W and U, R, Qh, Uh, P and the state batch),
-    the reverse scan's dS^T P and dO^T Qh, and the chunk kernel's 6400 m16n8k16 products
-    (Grams, W, U, U', dU', dM, dQ, dK3, dW, T^T dU', T^T dW, dT, T^T dT T^T, the dK terms)."""
+    the reverse scan's dS^T P and dO^T Qh, and the chunk kernel's products (Grams, W, U, U', dU',
+    dM, dQ, dK3, dW, T^T dU', T^T dW, dT, T^T dT T^T, the dK terms: 26.2 MFLOP, 6400 tiles of
+    16 x 8 x 16). Rows and blocks that the tensor-core shapes compute beyond these are not counted."""
     fwd = 5 * 2 * 128 * 64 * 128 + 2 * 128 * 64 * 64 + 2 * 128 * 128 * 128 + 2 * 128 * 64 * 128
     scan = 2 * 128 * 128 * 128 + 2 * 128 * 128 * 64
     chunk = 6400 * 2 * 16 * 8 * 16
@@ -673,7 +674,7 @@ def run_bwd_bench(args, w, wr, rank, world, local, dev):
                     "frac": achieved / tpk, "peak_source": tkind, "algorithmic_flops_per_launch": flops,
                     "traffic": traffic, "traffic_kernel": traffic_kernel,
                     "kernel": "gdr_bwd_chunked step (tc_fwd_kernel storing the chunk maps + bwdc_scan_kernel "
-                              "+ bwdc_chunk_kernel)"}
+                              "+ bwdc_tc_kernel)"}
     else:
         peak = alu_peak_tflops(peak_mhz)
         flops = bwd_flops(w)

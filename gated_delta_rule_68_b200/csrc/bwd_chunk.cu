@@ -14,9 +14,9 @@
 //   2. bwdc_scan_kernel: per (batch row, value head), the chunks in reverse on tcgen05;
 //      dS^T is carried in fp32 registers, its fp16 copy in tensor memory is the products'
 //      A operand, and it is stored per chunk (as dS_next of that chunk); the last is dh0;
-//   3. bwdc_chunk_kernel: one CTA per (unit, chunk), all chunks at once, on the warp-level
-//      MMAs (mma.sync, fp16 operands, fp32 accumulation). With the
-//      in-chunk decays D_ri = exp(G_r - G_i) (r >= i) and f = Gamma_C / Gamma:
+//   3. bwdc_tc_kernel: one CTA per (unit, chunk), all chunks at once, on tcgen05 (fp16
+//      operands, fp32 accumulators in tensor memory). With the in-chunk decays
+//      D_ri = exp(G_r - G_i) (r >= i) and f = Gamma_C / Gamma:
 //        W = T diag(beta Gamma) K,  U = T diag(beta) V,  U' = U - W S
 //        dU' = M^T dO + diag(f) K dS_next,       M = tril(Q K^T * D)
 //        dM = tril(dO U'^T),                     dQ = diag(Gamma) dO S^T + (dM * D) K
@@ -73,12 +73,6 @@ __device__ __forceinline__ float warp_sum(float x)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
-}
-__device__ __forceinline__ void hmul_frag(uint32_t &r, __half2 s)
-{
-    __half2 h = *reinterpret_cast<__half2 *>(&r);
-    h = __hmul2(h, s);
-    r = *reinterpret_cast<uint32_t *>(&h);
 }
 
 // ------------------------------------------------------------------ pass 2: the reverse scan
@@ -260,209 +254,195 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
 }
 
 // ------------------------------------------------------------------ pass 3: per-chunk gradients
-// 8 warps; warp (rw, cw) = (warp & 1, warp >> 1) computes rows 32 rw .. 32 rw + 31 of every
-// product (two m16 blocks, mi = 0, 1) and columns 32 cw .. of the 128-wide ones, 16 cw .. of
-// the 64-wide ones: each fragment loaded from shared memory feeds two to four MMAs.
-constexpr int NTC = 256;
-// Input tiles are 128-byte swizzled images (64-column atoms, 1024-byte aligned), loaded by TMA
-// (q, k, v, dO) and bulk copies (S^T, dS_next^T, T); the tiles the kernel writes itself are
-// plain rows padded to LDD / LDC halves. A tile's "ld" below is its padded row stride in
-// halves, or minus its atom stride in bytes for a swizzled image.
-constexpr uint32_t SZ_DT = C * LDD * 2;     // padded [64][136] fp16
-constexpr uint32_t SZ_CT = C * LDC * 2;     // padded [64][72] fp16
-constexpr int LQ = -8192, LS = -16384, LT = -8192;   // swizzled [64][128], [128][128], [64][64]
-constexpr uint32_t OC_Q = 0, OC_K = 16384, OC_V = 32768, OC_DO = 49152;
-constexpr uint32_t OC_S = 65536;              // S^T [dv][dk]; later X = T^T dT [64][LDC]
-constexpr uint32_t OC_DS = OC_S + 32768;      // dS_next^T [dv][dk]; later dW [64][LDD]
-constexpr uint32_t OC_T = OC_DS + 32768;      // T [64][64]
-constexpr uint32_t OC_M = OC_T + 8192;        // M, then dM * D [64][LDC]
-constexpr uint32_t OC_W = OC_M + SZ_CT;       // W, then dU' [64][LDD]
-constexpr uint32_t OC_U = OC_W + SZ_DT;       // U', then dT, then dB * D [64][LDC]
-constexpr uint32_t OC_DEC = OC_U + SZ_DT;     // D_ri = exp(G_r - G_i) (r >= i, else 0) [64][LDC] fp16
-constexpr uint32_t OC_BM = OC_DEC + SZ_CT;    // Bm = tril(K K^T * D, -1) [64][LDC] fp16
-constexpr uint32_t OC_BAR = OC_BM + SZ_CT;    // two mbarriers: inputs, then S^T and dS_next^T
-constexpr uint32_t OC_VEC = OC_BAR + 16;
-// vectors: G, Gamma, beta, f [64]; per column quarter of the warps, the row sums of dG and dbeta
-// [4][64] each; per warp, sum(dK3 * K) and sum(dS_next * S) [8] each (summed in a fixed order,
-// so that dg and dbeta repeat bit for bit)
-constexpr int VG = 0, VGAM = 64, VBETA = 128, VF = 192, VDG = 256, VDB = 512, VT3 = 768, VSS = 776;
-constexpr uint32_t SMEM_CHUNK = OC_VEC + (VSS + 8) * 4 + 1024;   // + alignment of the base
-static_assert(SMEM_CHUNK <= 227 * 1024, "shared memory");
+// One CTA of 16 warps per (unit, chunk), all chunks at once, every product on tcgen05: M = 128,
+// fp16 operands from shared memory, fp32 accumulators in tensor memory, issued by thread 0.
+// Most products are taken transposed, feature index by token (W^T, U'^T, dU'^T, dV^T,
+// dQ^T, dK^T, ...), so that the 128 features fill the 128 lanes. The token-by-token
+// products (dM, X, Y) fill only lanes 0-63: their A operand's rows 64-127 are whatever
+// the neighbouring tile holds, and those accumulator rows are never read. The two dT terms
+// run as one product of the stacked [dU'; dW] (A, 128 rows) with the stacked [V; K]
+// (B, 128 rows), of which two diagonal 64 x 64 blocks are used.
+// Warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (thread p = its lane there) and
+// columns 16 (w / 4) .. + 15 of each 64-column accumulator.
+constexpr int NTT = 512;
+constexpr uint32_t QKV_AS = 24576;                    // per 64-feature atom x: V, K, Q tiles at 24576 x + 0, 8192, 16384
+constexpr uint32_t O_V = 0, O_K = 8192, O_Q = 16384;  // [64 tokens][64 features] each
+constexpr uint32_t O_DO = 49152;                      // dO [token][dv], atoms 8192 apart
+constexpr uint32_t O_S = 65536;                       // S^T [dv][dk], atoms 16384 apart; later dB * D [r][i]
+constexpr uint32_t O_DS = 98304;                      // dS_next^T [dv][dk]; later fp32 [i][r] hand-over for dT
+constexpr uint32_t O_T = 131072;                      // T [r][i]
+constexpr uint32_t O_TP = 139264, O_TPP = 147456;     // T diag(beta Gamma), T diag(beta); later dU'^T [dv][r]
+constexpr uint32_t O_M = 155648;                      // M [r][i]; later dM * D
+constexpr uint32_t O_W = 163840;                      // W^T [dk][r]; later dT [r][i] and X [m][n]
+constexpr uint32_t O_U = 180224;                      // U'^T [dv][r]; later dW^T [dk][r]
+constexpr uint32_t O_DU = O_TP, O_DW = O_U, O_DMD = O_M, O_DT = O_W, O_X = O_W + 8192, O_DBD = O_S, O_XCH = O_DS;
+constexpr uint32_t O_VEC = 196608;
+// floats: G, Gamma, beta, f [64]; per lane quarter, the row partial sums of dG and dbeta
+// [4][64]; per column quarter, dbeta's dA term [4][64]; per warp, sum(dK3 * K) and
+// sum(dS_next * S) [16]
+constexpr int W_G = 0, W_GAM = 64, W_BETA = 128, W_F = 192, W_DG = 256, W_DB = 512, W_DA = 768, W_T3 = 1024,
+              W_SS = 1040, W_END = 1056;
+constexpr uint32_t O_BAR = O_VEC + W_END * 4;         // mbarriers: two loads, seven product batches, drain
+constexpr int NB_TC = 10;
+constexpr uint32_t SMEM_TC = O_BAR + NB_TC * 8 + 1024;
+static_assert(SMEM_TC <= 227 * 1024, "shared memory");
+static_assert(O_DW > O_DU, "the stacked [dU'; dW] operand needs a positive atom stride");
+// tensor-memory columns (512)
+constexpr uint32_t C_G = 0;     // [K; Q] K^T: KK^T (lanes 0-63, kept for dbeta), QK^T (lanes 64-127)
+constexpr uint32_t C_A = 64;    // W^T, then dM, then the dT stack (128 columns), then X, then dK1b^T
+constexpr uint32_t C_B = 128;   // U'^T, then dW^T, then Y
+constexpr uint32_t C_QA = 192;  // S dO^T
+constexpr uint32_t C_C = 256;   // dSn^T K^T, then dV^T, then K^T (dM * D)^T
+constexpr uint32_t C_D = 320;   // dO^T M, then dK3^T
+constexpr uint32_t C_K1A = 384; // dW^T T
+constexpr uint32_t C_K2 = 448;  // Q^T (dM * D) + K^T (dB * D)
+constexpr uint32_t I_KK = tcu::idesc_f16(128, 64, false, false, false);
+constexpr uint32_t I_MK = tcu::idesc_f16(128, 64, false, true, false);
+constexpr uint32_t I_KM = tcu::idesc_f16(128, 64, false, false, true);
+constexpr uint32_t I_MM = tcu::idesc_f16(128, 64, false, true, true);
+constexpr uint32_t I_KM_NEG = tcu::idesc_f16(128, 64, false, false, true, true);
+constexpr uint32_t I_MM_NEG = tcu::idesc_f16(128, 64, false, true, true, true);
+constexpr uint32_t I_MK_N128 = tcu::idesc_f16(128, 128, false, true, false);
 
-// Byte address of element (row, col) of a tile with the given ld (see above).
-__device__ __forceinline__ uint32_t taddr(uint32_t base, int ld, int row, int col)
+__device__ __forceinline__ void st_h8(uint32_t addr, const float *x)
 {
-    if (ld > 0) return base + (uint32_t)(row * ld + col) * 2u;
-    return base + (uint32_t)(col >> 6) * (uint32_t)(-ld) + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
-           (((uint32_t)((col & 63) >> 3) ^ (uint32_t)(row & 7)) << 4) + (uint32_t)(col & 7) * 2u;
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pack_h2f(x[0], x[1])),
+                 "r"(pack_h2f(x[2], x[3])), "r"(pack_h2f(x[4], x[5])), "r"(pack_h2f(x[6], x[7]))
+                 : "memory");
 }
-// acc[2][2 NP][4] += A (rows r0 .. r0 + 31, K = 16 KS) B (columns n0 .. n0 + 16 NP) on the
-// warp-level MMAs (m16n8k16, fp16 operands, fp32 accumulators in the m16n8 layout).
-// A: [m][k] (AT false) or stored transposed [k][m] (AT true); B: stored [n][k] (BT false) or
-// [k][n] (BT true); each tile by its ld (see taddr). ascale(af, j, mi) may rescale the A
-// fragment of k-step j, row block mi, in registers.
-template <int KS, int NP, bool AT, bool BT, typename AS>
-__device__ __forceinline__ void wgemm2(float (*acc)[2 * NP][4], uint32_t aB, int lda, int r0, uint32_t bB, int ldb,
-                                       int n0, int lane, AS ascale)
+// 16 consecutive fp32 columns of this thread's lane (32x32b shape) at a0 (and a1), one wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t a0, float *v)
 {
-#pragma unroll 4
-    for (int j = 0; j < KS; ++j) {
-        uint32_t af[2][4];
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15])
+                 : "r"(a0)
+                 : "memory");
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-            const int m0 = r0 + 16 * mi, k0 = 16 * j;
-            if (AT) ldsm_t(af[mi], taddr(aB, lda, k0 + (lane & 7) + (lane >> 4) * 8, m0 + ((lane >> 3) & 1) * 8));
-            else ldsm(af[mi], taddr(aB, lda, m0 + (lane & 7) + ((lane >> 3) & 1) * 8, k0 + (lane >> 4) * 8));
-            ascale(af[mi], j, mi);
-        }
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld16x2(uint32_t a0, uint32_t a1, float *v)
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+                 "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(a0), "r"(a1)
+                 : "memory");
 #pragma unroll
-        for (int np = 0; np < NP; ++np) {
-            uint32_t bf[4];
-            const int nn = n0 + 16 * np, k0 = 16 * j;
-            if (BT) ldsm_t(bf, taddr(bB, ldb, k0 + (lane & 7) + ((lane >> 3) & 1) * 8, nn + (lane >> 4) * 8));
-            else ldsm(bf, taddr(bB, ldb, nn + (lane & 7) + (lane >> 4) * 8, k0 + ((lane >> 3) & 1) * 8));
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// One step of a butterfly reduce-scatter over the warp: lanes with bit W set keep the upper
+// W of their first 2W values, the others the lower W, each adding its partner's copy.
+template <int W>
+__device__ __forceinline__ void rs_step(float *x, int lane)
+{
+    const bool up = (lane & W) != 0;
 #pragma unroll
-            for (int mi = 0; mi < 2; ++mi) {
-                mma(acc[mi][2 * np], af[mi], bf[0], bf[1]);
-                mma(acc[mi][2 * np + 1], af[mi], bf[2], bf[3]);
-            }
-        }
+    for (int j = 0; j < W; ++j) {
+        const float send = up ? x[j] : x[j + W];
+        const float keep = up ? x[j + W] : x[j];
+        x[j] = keep + __shfl_xor_sync(0xffffffffu, send, W);
     }
 }
-// Two products of the same shape in lockstep (twice the independent MMAs per k-step):
-// acc1 += A1 B1, acc2 += A2 B2. SA: A2 is A1's tile (loaded once, then scaled by each
-// product's ascale); SB: B2 is B1's tile (loaded once).
-template <int KS, int NP, bool AT1, bool BT1, bool AT2, bool BT2, bool SA, bool SB, typename AS1, typename AS2>
-__device__ __forceinline__ void wgemm2_pair(float (*acc1)[2 * NP][4], uint32_t a1, int lda1, uint32_t b1, int ldb1,
-                                            AS1 as1, float (*acc2)[2 * NP][4], uint32_t a2, int lda2, uint32_t b2,
-                                            int ldb2, AS2 as2, int r0, int n0, int lane)
+// x[16] per lane; returns, in lanes l and l + 16, the sum of x[l % 16] over the warp's 32
+// lanes (16 shuffles, in a fixed order).
+__device__ __forceinline__ float warp_rs16(float *x, int lane)
 {
-    auto lda_ = [&](uint32_t *f, uint32_t aB, int lda, bool at, int m0, int k0) {
-        if (at) ldsm_t(f, taddr(aB, lda, k0 + (lane & 7) + (lane >> 4) * 8, m0 + ((lane >> 3) & 1) * 8));
-        else ldsm(f, taddr(aB, lda, m0 + (lane & 7) + ((lane >> 3) & 1) * 8, k0 + (lane >> 4) * 8));
-    };
-    auto ldb_ = [&](uint32_t *f, uint32_t bB, int ldb, bool bt, int nn, int k0) {
-        if (bt) ldsm_t(f, taddr(bB, ldb, k0 + (lane & 7) + ((lane >> 3) & 1) * 8, nn + (lane >> 4) * 8));
-        else ldsm(f, taddr(bB, ldb, nn + (lane & 7) + (lane >> 4) * 8, k0 + ((lane >> 3) & 1) * 8));
-    };
-#pragma unroll 2
-    for (int j = 0; j < KS; ++j) {
-        uint32_t f1[2][4], f2[2][4];
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-            lda_(f1[mi], a1, lda1, AT1, r0 + 16 * mi, 16 * j);
-            if (SA) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) f2[mi][e] = f1[mi][e];
-            } else {
-                lda_(f2[mi], a2, lda2, AT2, r0 + 16 * mi, 16 * j);
-            }
-            as1(f1[mi], j, mi);
-            as2(f2[mi], j, mi);
-        }
-#pragma unroll
-        for (int np = 0; np < NP; ++np) {
-            uint32_t g1[4], g2[4];
-            ldb_(g1, b1, ldb1, BT1, n0 + 16 * np, 16 * j);
-            if (SB) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) g2[e] = g1[e];
-            } else {
-                ldb_(g2, b2, ldb2, BT2, n0 + 16 * np, 16 * j);
-            }
-#pragma unroll
-            for (int mi = 0; mi < 2; ++mi) {
-                mma(acc1[mi][2 * np], f1[mi], g1[0], g1[1]);
-                mma(acc2[mi][2 * np], f2[mi], g2[0], g2[1]);
-                mma(acc1[mi][2 * np + 1], f1[mi], g1[2], g1[3]);
-                mma(acc2[mi][2 * np + 1], f2[mi], g2[2], g2[3]);
-            }
-        }
-    }
+    rs_step<8>(x, lane);
+    rs_step<4>(x, lane);
+    rs_step<2>(x, lane);
+    rs_step<1>(x, lane);
+    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 16);
 }
-struct NoScale2 {
-    __device__ __forceinline__ void operator()(uint32_t *, int, int) const {}
-};
-template <int N>
-__device__ __forceinline__ void zero2(float (*acc)[N][4])
+__device__ __forceinline__ void prefetch_l2_line(const void *p)
 {
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-        for (int i = 0; i < N; ++i) acc[mi][i][0] = acc[mi][i][1] = acc[mi][i][2] = acc[mi][i][3] = 0.f;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // pf: the CTA that runs pf launches later on this SM (the resident CTA count) gets its inputs
 // prefetched into L2 by this one; sole: every key head has one value head, so dq and dk rows
 // have one writer and take plain stores.
-__global__ void __launch_bounds__(NTC, 1)
-bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ CUtensorMap map_q,
-                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                  const __grid_constant__ CUtensorMap map_do)
+__global__ void __launch_bounds__(NTT, 1)
+bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ CUtensorMap map_q,
+               const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+               const __grid_constant__ CUtensorMap map_do)
 {
+    using namespace tcu;
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
-    const int rw = warp & 1, cw = warp >> 1, r0 = 32 * rw;
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, cq = warp >> 2, p = 32 * q4 + lane;
+    const int col0 = 16 * cq;   // this thread's first column of a 64-column accumulator
     const int NC = (a.T + C - 1) / C;
     const int unit = blockIdx.x / NC, c = blockIdx.x % NC;
     const int b = unit / a.Hv, h = unit % a.Hv, hk = h / (a.Hv / a.Hk);
-    const uint32_t sb = smem_u32(sm);
-    float *vec = reinterpret_cast<float *>(sm + OC_VEC);
     const size_t cu = (size_t)unit * NC + c;
-
-    // ---- loads, on two mbarriers: q, k (key head), v, dO (value head) by TMA (bf16, rows past T
-    // zero) and T; then S^T and dS_next^T, which arrive while the Grams, W and U are formed
+    const int nvalid = min(C, a.T - c * C);
+    float *vec = reinterpret_cast<float *>(sm + O_VEC);
+    auto bar = [&](int i) { return sb + O_BAR + 8 * i; };   // 0, 1: loads; 2-8: products; 9: drain
+    __shared__ uint32_t tmem_sh;
     __shared__ int abort_sh;
-    const uint32_t bar0 = sb + OC_BAR, bar1 = bar0 + 8;
     if (tid == 0) {
-        mbar_init(bar0, 1);
-        mbar_init(bar1, 1);
+        for (int i = 0; i < NB_TC; ++i) mbar_init(bar(i), 1);
         abort_sh = 0;
     }
+    if (warp == 0) tmem_alloc(smem_u32(&tmem_sh), 512);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = tmem_sh;
     if (tid == 0) {
         const int t0 = c * C;
-        mbar_expect_tx(bar0, 4 * 16384 + 8192);
-        tma_load_4d(sb + OC_Q, &map_q, 0, hk, t0, b, bar0);
-        tma_load_4d(sb + OC_Q + 8192, &map_q, 64, hk, t0, b, bar0);
-        tma_load_4d(sb + OC_K, &map_k, 0, hk, t0, b, bar0);
-        tma_load_4d(sb + OC_K + 8192, &map_k, 64, hk, t0, b, bar0);
-        tma_load_4d(sb + OC_V, &map_v, 0, h, t0, b, bar0);
-        tma_load_4d(sb + OC_V + 8192, &map_v, 64, h, t0, b, bar0);
-        tma_load_4d(sb + OC_DO, &map_do, 0, h, t0, b, bar0);
-        tma_load_4d(sb + OC_DO + 8192, &map_do, 64, h, t0, b, bar0);
-        bulk_g2s(sb + OC_T, ws.t + cu * C * C, 8192, bar0);
-        mbar_expect_tx(bar1, 2 * 32768);
-        bulk_g2s(sb + OC_S, ws.s + cu * D * D, 32768, bar1);
-        bulk_g2s(sb + OC_DS, ws.ds + cu * D * D, 32768, bar1);
+        mbar_expect_tx(bar(0), 8 * 8192 + 8192);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sb + O_V + x * QKV_AS, &map_v, 64 * x, h, t0, b, bar(0));
+            tma_load_4d(sb + O_K + x * QKV_AS, &map_k, 64 * x, hk, t0, b, bar(0));
+            tma_load_4d(sb + O_Q + x * QKV_AS, &map_q, 64 * x, hk, t0, b, bar(0));
+            tma_load_4d(sb + O_DO + x * 8192, &map_do, 64 * x, h, t0, b, bar(0));
+        }
+        bulk_g2s(sb + O_T, ws.t + cu * C * C, 8192, bar(0));
+        mbar_expect_tx(bar(1), 2 * 32768);
+        bulk_g2s(sb + O_S, ws.s + cu * D * D, 32768, bar(1));
+        bulk_g2s(sb + O_DS, ws.ds + cu * D * D, 32768, bar(1));
     }
-    auto wait = [&](uint32_t bar) {
+    auto wait = [&](int i) {
         if (*reinterpret_cast<volatile int *>(&abort_sh)) return;
-        if (!mbar_wait_bounded(bar, 0)) {
+        if (!mbar_wait_bounded(bar(i), 0)) {
             *reinterpret_cast<volatile int *>(&abort_sh) = 1;
             atomicAdd(&g_bwdc_timeouts, 1u);
         }
     };
-    if (tid < C) {
-        const int t = c * C + tid;
+    // Every product batch: the operand tiles written by all threads are made visible to the
+    // tensor core, the tensor-memory reads of the previous epilogue are ordered before it.
+    auto to_issue = [&]() {
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+    if (tid >= 64 && tid < 64 + C) {   // (not the warp that issues the copies)
+        const int t = c * C + tid - 64;
         const bool ok = t < a.T;
-        vec[VG + tid] = ok ? a.g[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
-        vec[VBETA + tid] = ok ? a.beta[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
-    }
-    wait(bar0);
-    for (int i = tid; i < 2 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_Q + 16 * i);   // q, k to fp16
-    // T is lower triangular: clear what the forward left unwritten above the diagonal blocks
-    for (int i = tid; i < C * 8; i += NTC) {
-        const int r = i >> 3, j = i & 7;
-        __half *row = reinterpret_cast<__half *>(sm + OC_T + tcu::swz_chunk(r, j, 0));
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if (8 * j + e > r) row[e] = __float2half(0.f);
+        vec[W_G + tid - 64] = ok ? a.g[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
+        vec[W_BETA + tid - 64] = ok ? a.beta[((size_t)b * a.T + t) * a.Hv + h] : 0.f;
     }
     __syncthreads();
-    if (warp == 0) {   // in-chunk prefix G, Gamma = exp(G), f = Gamma_C / Gamma
-        float x0 = vec[VG + lane], x1 = vec[VG + 32 + lane];
+    if (warp == 2) {   // in-chunk prefix G, Gamma = exp(G), f = Gamma_C / Gamma
+        float x0 = vec[W_G + lane], x1 = vec[W_G + 32 + lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
@@ -470,116 +450,95 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
         }
         x1 += __shfl_sync(0xffffffffu, x0, 31);
         const float GL = __shfl_sync(0xffffffffu, x1, 31);
-        vec[VG + lane] = x0;
-        vec[VG + 32 + lane] = x1;
-        vec[VGAM + lane] = __expf(x0);
-        vec[VGAM + 32 + lane] = __expf(x1);
-        vec[VF + lane] = __expf(GL - x0);
-        vec[VF + 32 + lane] = __expf(GL - x1);
+        vec[W_G + lane] = x0;
+        vec[W_G + 32 + lane] = x1;
+        vec[W_GAM + lane] = __expf(x0);
+        vec[W_GAM + 32 + lane] = __expf(x1);
+        vec[W_F + lane] = __expf(GL - x0);
+        vec[W_F + 32 + lane] = __expf(GL - x1);
     }
     __syncthreads();
-
-    const float *G = vec + VG, *Gam = vec + VGAM, *beta = vec + VBETA, *fv = vec + VF;
-    // this thread's rows: row(mi, hi) = r0 + 16 mi + 8 hi + g8 (accumulator elements 2 hi, 2 hi + 1)
-    auto row = [&](int mi, int e) { return r0 + 16 * mi + g8 + 8 * (e >> 1); };
-    auto dec = [&](int r, int i) { return r >= i ? __expf(G[r] - G[i]) : 0.f; };
-    // D and Bm, written in a and read back by the same thread (same warp tiles) in d and j
-    __half *decm = reinterpret_cast<__half *>(sm + OC_DEC), *bmm = reinterpret_cast<__half *>(sm + OC_BM);
-    // per-row partial sums of this thread, [mi][hi], added to dG / dbeta at the end
-    float pg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, tot3 = 0.f;
-    auto rowdot = [&](const float (*acc)[4][4], uint32_t tile, int n0, float (*s)[2]) {
-        // sum over this thread's columns of acc * tile (a swizzled [64][128] input) on its rows
+    const float *G = vec + W_G, *Gam = vec + W_GAM, *beta = vec + W_BETA, *fv = vec + W_F;
+    // Element (token col0 + j, feature p) of the V, K and Q tiles: byte offset pbase + (j / 8) 1024
+    // + xo[j % 8] from the tile's first atom (the 128-byte swizzle of swz_off, with col0 a multiple
+    // of 16).
+    const uint32_t pbase = (uint32_t)(p >> 6) * QKV_AS + (uint32_t)cq * 2048u + (uint32_t)(p & 7) * 2u;
+    uint32_t xo[8];
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int col = n0 + 8 * nt + 2 * t4;
-                const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(sm + (taddr(tile, LQ, row(mi, 0), col))));
-                const float2 y = __half22float2(*reinterpret_cast<const __half2 *>(sm + (taddr(tile, LQ, row(mi, 2), col))));
-                s[mi][0] = fmaf(acc[mi][nt][0], x.x, fmaf(acc[mi][nt][1], x.y, s[mi][0]));
-                s[mi][1] = fmaf(acc[mi][nt][2], y.x, fmaf(acc[mi][nt][3], y.y, s[mi][1]));
-            }
-    };
-    auto store_h = [&](const float (*acc)[4], int mi, int ntn, uint32_t tile, int ld, int n0, float sc) {
-        __half *tp = reinterpret_cast<__half *>(sm + tile);
-        for (int nt = 0; nt < ntn; ++nt) {
-            const int col = n0 + 8 * nt + 2 * t4;
-            *reinterpret_cast<uint32_t *>(tp + row(mi, 0) * ld + col) = pack_h2f(sc * acc[nt][0], sc * acc[nt][1]);
-            *reinterpret_cast<uint32_t *>(tp + row(mi, 2) * ld + col) = pack_h2f(sc * acc[nt][2], sc * acc[nt][3]);
-        }
-    };
-    const int n128 = 32 * cw, n64 = 16 * cw;   // this warp's columns of 128- and 64-wide outputs
-    // per-row scalings of A fragments (rows g8 and g8 + 8 of block mi)
-    auto rowscale = [&](const float *v) {
-        return [=](uint32_t *af, int, int mi) {
-            const __half2 sa = __float2half2_rn(v[r0 + 16 * mi + g8]), sb2 = __float2half2_rn(v[r0 + 16 * mi + g8 + 8]);
-            hmul_frag(af[0], sa);
-            hmul_frag(af[1], sb2);
-            hmul_frag(af[2], sa);
-            hmul_frag(af[3], sb2);
-        };
+    for (int k = 0; k < 8; ++k) xo[k] = (uint32_t)k * 128u + ((((uint32_t)(p & 63) >> 3) ^ (uint32_t)k) << 4);
+    auto colrd = [&](uint32_t tile, int j) {
+        return __half2float(*reinterpret_cast<const __half *>(sm + tile + pbase + (uint32_t)(j >> 3) * 1024u + xo[j & 7]));
     };
 
-    // ---- a: the Grams, M = tril(Q K^T * D) and Bm = tril(K K^T * D, -1)
+    // ---- inputs to fp16 in place (V, K, Q, dO: 4096 16-byte words, four loads in flight);
+    // T's entries above the diagonal blocks cleared (the forward leaves them unwritten), and
+    // T' = T diag(beta Gamma), T'' = T diag(beta)
+    wait(0);
+#pragma unroll
+    for (int j0 = 0; j0 < 8; j0 += 4) {
+        uint4 u[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[j] = reinterpret_cast<const uint4 *>(sm)[tid + NTT * (j0 + j)];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) reinterpret_cast<uint4 *>(sm)[tid + NTT * (j0 + j)] = bf16x8_to_f16x8(u[j]);
+    }
     {
-        float qk[2][2][4], kk[2][2][4];
-        zero2<2>(qk);
-        zero2<2>(kk);
-        wgemm2_pair<8, 1, false, false, false, false, false, true>(qk, sb + OC_Q, LQ, sb + OC_K, LQ, NoScale2(), kk,
-                                                                   sb + OC_K, LQ, sb + OC_K, LQ, NoScale2(), r0, n64, lane);
+        const int r = tid >> 3, j = tid & 7;
+        uint4 u = *reinterpret_cast<const uint4 *>(sm + swz_chunk(r, j, O_T));
+        __half2 *hh = reinterpret_cast<__half2 *>(&u);
+        float x[8], y[8];
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(hh[k]);
+            x[2 * k] = 8 * j + 2 * k > r ? 0.f : f.x;
+            x[2 * k + 1] = 8 * j + 2 * k + 1 > r ? 0.f : f.y;
+        }
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+        for (int k = 0; k < 8; ++k) y[k] = x[k] * beta[8 * j + k];
+        st_h8(sb + swz_chunk(r, j, O_TPP), y);
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int r = row(mi, 2 * hi), i = n64 + 8 * nt + 2 * t4;
-                    const float d0 = dec(r, i), d1 = dec(r, i + 1);
-                    *reinterpret_cast<__half2 *>(decm + r * LDC + i) = __floats2half2_rn(d0, d1);
-                    *reinterpret_cast<__half2 *>(bmm + r * LDC + i) =
-                        __floats2half2_rn(r > i ? kk[mi][nt][2 * hi] * d0 : 0.f, r > i + 1 ? kk[mi][nt][2 * hi + 1] * d1 : 0.f);
-                    qk[mi][nt][2 * hi] *= d0;
-                    qk[mi][nt][2 * hi + 1] *= d1;
-                }
-            store_h(qk[mi], mi, 2, OC_M, LDC, n64, 1.f);
+        for (int k = 0; k < 8; ++k) y[k] *= Gam[8 * j + k];
+        st_h8(sb + swz_chunk(r, j, O_TP), y);
+        st_h8(sb + swz_chunk(r, j, O_T), x);
+    }
+    to_issue();
+    // ---- batch 1: [K; Q] K^T, W^T = K^T T'^T, U^T = V^T T''^T; then (once S and dS_next have
+    // landed) S dO^T and dS_next^T K^T
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t ko = (s >> 2) * QKV_AS + (s & 3) * 32;
+            mma_ss(tb + C_G, sdesc(sb + O_K + ko, 16, 1024), sdesc(sb + O_K + ko, 16, 1024), I_KK, s > 0);
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_A, sdesc(sb + O_K + s * 2048, QKV_AS, 1024), sdesc(sb + O_TP + s * 32, 16, 1024), I_MK, s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_B, sdesc(sb + O_V + s * 2048, QKV_AS, 1024), sdesc(sb + O_TPP + s * 32, 16, 1024), I_MK, s > 0);
+        mma_commit(bar(2));
+    }
+    wait(1);
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_ss(tb + C_QA, sdesc(sb + O_S + s * 2048, 16384, 1024),
+                   sdesc(sb + O_DO + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), I_MK, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t ko = (s >> 2) * 16384 + (s & 3) * 32;
+            mma_ss(tb + C_C, sdesc(sb + O_DS + ko, 16, 1024), sdesc(sb + O_K + (s >> 2) * QKV_AS + (s & 3) * 32, 16, 1024),
+                   I_KK, s > 0);
         }
     }
-    // ---- b: W = T diag(beta Gamma) K, U = T diag(beta) V, then U' = U - W S
-    {
-        float u[2][4][4];
-        auto colscale = [&](const float *s1, const float *s2) {
-            return [=](uint32_t *af, int j, int) {
-                const int k0 = 16 * j + 2 * t4;
-                const __half2 lo = __floats2half2_rn(s1[k0] * (s2 ? s2[k0] : 1.f), s1[k0 + 1] * (s2 ? s2[k0 + 1] : 1.f));
-                const __half2 hi =
-                    __floats2half2_rn(s1[k0 + 8] * (s2 ? s2[k0 + 8] : 1.f), s1[k0 + 9] * (s2 ? s2[k0 + 9] : 1.f));
-                hmul_frag(af[0], lo);
-                hmul_frag(af[1], lo);
-                hmul_frag(af[2], hi);
-                hmul_frag(af[3], hi);
-            };
-        };
-        // v and dO to fp16 (v for U, dO from c on)
-        for (int i = tid; i < 2 * C * 16; i += NTC) bf16_to_fp16_16B(sm + OC_V + 16 * i);
-        __syncthreads();
-        {
-            float w[2][4][4];
-            zero2<4>(w);
-            zero2<4>(u);
-            wgemm2_pair<4, 2, false, true, false, true, true, false>(w, sb + OC_T, LT, sb + OC_K, LQ, colscale(beta, Gam), u,
-                                                                     sb + OC_T, LT, sb + OC_V, LQ, colscale(beta, nullptr),
-                                                                     r0, n128, lane);
-#pragma unroll
-            for (int mi = 0; mi < 2; ++mi) store_h(w[mi], mi, 4, OC_W, LDD, n128, 1.f);
-        }
-        wait(bar1);   // S^T and dS_next^T
-        __syncthreads();
-        if (tid == 0 && pf > 0 && (long)blockIdx.x + pf < (long)gridDim.x) {
-            // the inputs of the CTA pf launches later, into L2 while this one computes (its own
-            // loads have landed, so the two do not compete): eight TMA boxes and three spans
-            const long nbk = (long)blockIdx.x + pf;
-            const int nu = (int)(nbk / NC), ncc = (int)(nbk % NC);
-            const int n_b = nu / a.Hv, n_h = nu % a.Hv, n_hk = n_h / (a.Hv / a.Hk), nt0 = ncc * C;
+    const long nbk = (long)blockIdx.x + pf;
+    if (pf > 0 && nbk < (long)gridDim.x && warp == 1) {
+        // the inputs of the CTA pf launches later, into L2 while this one computes (its own
+        // loads have landed, so the two do not compete)
+        const int nu = (int)(nbk / NC), ncc = (int)(nbk % NC);
+        const int n_b = nu / a.Hv, n_h = nu % a.Hv, n_hk = n_h / (a.Hv / a.Hk), nt0 = ncc * C;
+        if (lane == 0) {
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 prefetch_tma_4d(&map_q, 64 * x, n_hk, nt0, n_b);
@@ -592,262 +551,309 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
             prefetch_l2_bulk(ws.ds + ncu * D * D, D * D * 2);
             prefetch_l2_bulk(ws.t + ncu * C * C, C * C * 2);
         }
-        {   // sum(dS_next * S) over the whole state
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int t = nt0 + lane + 32 * e;
+            if (t < a.T) {
+                const size_t ix = ((size_t)n_b * a.T + t) * a.Hv + n_h;
+                prefetch_l2_line(a.g + ix);
+                prefetch_l2_line(a.beta + ix);
+            }
+        }
+    }
+    {   // sum(dS_next * S) over the whole state, while the products run
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // the two images share one layout
+            const int i = tid + NTT * k;
+            const uint4 ux = *reinterpret_cast<const uint4 *>(sm + O_S + 16 * i);
+            const uint4 uy = *reinterpret_cast<const uint4 *>(sm + O_DS + 16 * i);
+            const __half2 *x = reinterpret_cast<const __half2 *>(&ux), *y = reinterpret_cast<const __half2 *>(&uy);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fx = __half22float2(x[e]), fy = __half22float2(y[e]);
+                s = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, s));
+            }
+        }
+        s = warp_sum(s);
+        if (lane == 0) vec[W_SS + warp] = s;
+    }
+    // ---- epilogue 1: M = tril(Q K^T * D) (lanes 64-127), W^T
+    wait(2);
+    tc_fence_after();
+    {
+        float v[16];
+        if (p >= 64) {
+            tmem_ld16(tmem_addr(tb, q4, C_G + col0), v);
+            const int r = p - 64;
+            const float gr = G[r];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = col0 + j <= r ? v[j] * __expf(gr - G[col0 + j]) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(r, 2 * cq + jj, O_M), v + 8 * jj);
+        }
+        tmem_ld16(tmem_addr(tb, q4, C_A + col0), v);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_W), v + 8 * jj);
+    }
+    to_issue();
+    // ---- batch 2: U'^T = U^T - S^T W^T, dO^T M
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_ss(tb + C_B, sdesc(sb + O_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                   sdesc(sb + O_W + s * 2048, 8192, 1024), I_KM_NEG, true);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_D, sdesc(sb + O_DO + s * 2048, 8192, 1024), sdesc(sb + O_M + s * 2048, 8192, 1024), I_MM, s > 0);
+        mma_commit(bar(3));
+    }
+    // ---- epilogue 2: U'^T; dU'^T = dO^T M + (dS_next^T K^T) diag(f)
+    wait(3);
+    tc_fence_after();
+    {
+        float v[32];
+        tmem_ld16(tmem_addr(tb, q4, C_B + col0), v);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_U), v + 8 * jj);
+        tmem_ld16x2(tmem_addr(tb, q4, C_D + col0), tmem_addr(tb, q4, C_C + col0), v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = fmaf(fv[col0 + j], v[16 + j], v[j]);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_DU), v + 8 * jj);
+    }
+    to_issue();
+    // ---- batch 3: dM = dO U'^T (lanes 0-63), dK3^T = dS_next U'^T, dW^T = -S dU'^T, dV^T = dU'^T T
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_ss(tb + C_A, sdesc(sb + O_DO + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024),
+                   sdesc(sb + O_U + s * 2048, 8192, 1024), I_KM, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_ss(tb + C_D, sdesc(sb + O_DS + s * 2048, 16384, 1024), sdesc(sb + O_U + s * 2048, 8192, 1024), I_MM, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_ss(tb + C_B, sdesc(sb + O_S + s * 2048, 16384, 1024), sdesc(sb + O_DU + s * 2048, 8192, 1024), I_MM_NEG,
+                   s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_C, sdesc(sb + O_DU + s * 32, 16, 1024), sdesc(sb + O_T + s * 2048, 8192, 1024), I_KM, s > 0);
+        mma_commit(bar(4));
+    }
+    // ---- epilogue 3: dM * D (lanes 0-63), dW^T; dV and rowsum(V * T^T dU') once batch 4 is issued
+    wait(4);
+    tc_fence_after();
+    float dv[16];
+    {
+        float v[16];
+        if (p < 64) {
+            tmem_ld16(tmem_addr(tb, q4, C_A + col0), v);
+            const float gr = G[p];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = col0 + j <= p ? v[j] * __expf(gr - G[col0 + j]) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_DMD), v + 8 * jj);
+        }
+        tmem_ld16(tmem_addr(tb, q4, C_B + col0), v);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_DW), v + 8 * jj);
+        tmem_ld16(tmem_addr(tb, q4, C_C + col0), dv);   // (T^T dU')^T [dv = p][i]
+    }
+    to_issue();
+    // ---- batch 4: dQb^T = K^T (dM * D)^T, dK2^T = Q^T (dM * D), dK1a^T = dW^T T, and the dT stack
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_C, sdesc(sb + O_K + s * 2048, QKV_AS, 1024), sdesc(sb + O_DMD + s * 32, 16, 1024), I_MK, s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_K2, sdesc(sb + O_Q + s * 2048, QKV_AS, 1024), sdesc(sb + O_DMD + s * 2048, 8192, 1024), I_MM,
+                   s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_ss(tb + C_K1A, sdesc(sb + O_DW + s * 32, 16, 1024), sdesc(sb + O_T + s * 2048, 8192, 1024), I_KM, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_ss(tb + C_A, sdesc(sb + O_DU + s * 2048, O_DW - O_DU, 1024),
+                   sdesc(sb + O_V + (s >> 2) * QKV_AS + (s & 3) * 32, 16, 1024), I_MK_N128, s > 0);
+        mma_commit(bar(5));
+    }
+    {
+        float *dst = a.dv + (((size_t)b * a.T + c * C + col0) * a.Hv + h) * D + p;
+        const size_t stride = (size_t)a.Hv * D;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int i = col0 + j;
+            if (i < nvalid) dst[j * stride] = beta[i] * dv[j];
+            dv[j] *= colrd(O_V, j);
+        }
+        const float s = warp_rs16(dv, lane);
+        if (lane < 16) vec[W_DB + 64 * q4 + col0 + lane] = s;
+    }
+    // dQ = diag(Gamma) dO S^T + (dM * D) K (from the two accumulators, which no later batch
+    // overwrites) and rowsum(dQ * Q)
+    auto dq_out = [&]() {
+        float v[32];
+        tmem_ld16x2(tmem_addr(tb, q4, C_QA + col0), tmem_addr(tb, q4, C_C + col0), v);
+        float *dst = a.dq + (((size_t)b * a.T + c * C + col0) * a.Hk + hk) * D + p;
+        const size_t stride = (size_t)a.Hk * D;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int r = col0 + j;
+            const float x = fmaf(Gam[r], v[j], v[16 + j]);
+            if (r < nvalid) {
+                if (sole) dst[j * stride] = x;
+                else atomicAdd(dst + j * stride, x);
+            }
+            v[j] = x * colrd(O_Q, j);
+        }
+        const float s = warp_rs16(v, lane);
+        if (lane < 16) vec[W_DG + 64 * q4 + col0 + lane] = s;
+    };
+    // ---- epilogue 4: dT = (dU' V^T + dW K^T diag(Gamma)) diag(beta). The dW K^T block sits on
+    // lanes 64-127, columns 64-127 of the stack, and goes to the dU' V^T block's threads through
+    // shared memory. From here the token-by-token chain (X, Y, dA, dB) runs on the warps of
+    // lanes 0-63 alone, synchronised among themselves (named barrier 1), while the others write
+    // their dQ; the chain's warps write theirs once batch 7 is issued.
+    wait(5);
+    tc_fence_after();
+    float *xch = reinterpret_cast<float *>(sm + O_XCH);   // [i][r]
+    if (p >= 64) {
+        float v[16];
+        tmem_ld16(tmem_addr(tb, q4, C_A + 64 + col0), v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xch[(col0 + j) * C + (p - 64)] = Gam[col0 + j] * v[j];
+    }
+    tc_fence_before();
+    __syncthreads();
+    // the chain: fence the written tiles and tensor-memory reads, then sync its 8 warps
+    auto chain_sync = [&]() {
+        fence_proxy_async();
+        tc_fence_before();
+        named_bar_sync(1, NTT / 2);
+        tc_fence_after();
+    };
+    if (p < 64) {
+        {
+            float v[16];
+            tmem_ld16(tmem_addr(tb, q4, C_A + col0), v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = beta[col0 + j] * (v[j] + xch[(col0 + j) * C + p]);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_DT), v + 8 * jj);
+        }
+        chain_sync();
+        // ---- batch 5: X = T^T dT (lanes 0-63)
+        if (tid == 0) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_ss(tb + C_A, sdesc(sb + O_T + s * 2048, 8192, 1024), sdesc(sb + O_DT + s * 2048, 8192, 1024), I_MM,
+                       s > 0);
+            mma_commit(bar(6));
+        }
+        wait(6);
+        tc_fence_after();
+        {
+            float v[16];
+            tmem_ld16(tmem_addr(tb, q4, C_A + col0), v);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_X), v + 8 * jj);
+        }
+        chain_sync();
+        // ---- batch 6: Y = X T^T (lanes 0-63)
+        if (tid == 0) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_ss(tb + C_B, sdesc(sb + O_X + s * 32, 16, 1024), sdesc(sb + O_T + s * 32, 16, 1024), I_KK, s > 0);
+            mma_commit(bar(7));
+        }
+        // ---- epilogue 6: dA = strict tril(-Y), rowsum(dA * tril(K K^T * D, -1)), dB * D = diag(beta) dA * D
+        wait(7);
+        tc_fence_after();
+        {
+            float v[32];
+            tmem_ld16x2(tmem_addr(tb, q4, C_B + col0), tmem_addr(tb, q4, C_G + col0), v);
+            const float gr = G[p], br = beta[p];
             float s = 0.f;
-            for (int i = tid; i < D * 16; i += NTC) {   // the two images share one layout
-                const __half2 *x = reinterpret_cast<const __half2 *>(sm + OC_S + 16 * i);
-                const __half2 *y = reinterpret_cast<const __half2 *>(sm + OC_DS + 16 * i);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 fx = __half22float2(x[e]), fy = __half22float2(y[e]);
-                    s = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, s));
-                }
+            for (int j = 0; j < 16; ++j) {
+                const int i = col0 + j;
+                const float d = i < p ? __expf(gr - G[i]) : 0.f;
+                const float dA = -v[j];
+                s = fmaf(dA * d, v[16 + j], s);
+                v[j] = br * dA * d;
             }
-            s = warp_sum(s);
-            if (lane == 0) vec[VSS + warp] = s;
+            vec[W_DA + 64 * cq + p] = s;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) st_h8(sb + swz_chunk(p, 2 * cq + jj, O_DBD), v + 8 * jj);
         }
-        const __half2 neg = __floats2half2_rn(-1.f, -1.f);
-        wgemm2<8, 2, false, false>(u, sb + OC_W, LDD, r0, sb + OC_S, LS, n128, lane, [=](uint32_t *af, int, int) {
-            hmul_frag(af[0], neg);
-            hmul_frag(af[1], neg);
-            hmul_frag(af[2], neg);
-            hmul_frag(af[3], neg);
-        });
+        chain_sync();
+        // ---- batch 7: dK1b^T = K^T (dB * D)^T, dK2^T += K^T (dB * D)
+        if (tid == 0) {
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) store_h(u[mi], mi, 4, OC_U, LDD, n128, 1.f);
-    }
-    __syncthreads();
-    // ---- c: dU' = M^T dO + diag(f) K dS_next
-    {
-        float du[2][4][4];
-        zero2<4>(du);
-        wgemm2<4, 2, true, true>(du, sb + OC_M, LDC, r0, sb + OC_DO, LQ, n128, lane, NoScale2());
-        wgemm2<8, 2, false, false>(du, sb + OC_K, LQ, r0, sb + OC_DS, LS, n128, lane, rowscale(fv));
+            for (int s = 0; s < 4; ++s)
+                mma_ss(tb + C_A, sdesc(sb + O_K + s * 2048, QKV_AS, 1024), sdesc(sb + O_DBD + s * 32, 16, 1024), I_MK,
+                       s > 0);
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) store_h(du[mi], mi, 4, OC_W, LDD, n128, 1.f);   // W is dead
-    }
-    __syncthreads();
-    // ---- d: dM = tril(dO U'^T), stored as dM * D
-    {
-        float dm[2][2][4];
-        zero2<2>(dm);
-        wgemm2<8, 1, false, false>(dm, sb + OC_DO, LQ, r0, sb + OC_U, LDD, n64, lane, NoScale2());
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dm[mi][nt][e] *= __half2float(decm[row(mi, e) * LDC + n64 + 8 * nt + 2 * t4 + (e & 1)]);
-            store_h(dm[mi], mi, 2, OC_M, LDC, n64, 1.f);   // M is dead
+            for (int s = 0; s < 4; ++s)
+                mma_ss(tb + C_K2, sdesc(sb + O_K + s * 2048, QKV_AS, 1024), sdesc(sb + O_DBD + s * 2048, 8192, 1024),
+                       I_MM, true);
+            mma_commit(bar(8));
         }
     }
-    __syncthreads();
-    // ---- e: dQ = diag(Gamma) dO S^T + (dM * D) K
+    dq_out();
+    // ---- epilogue 7: dK = diag(f) dK3 + diag(Gamma beta) T^T dW + dK1b + dK2, with the row sums
+    // of dG, dbeta and the total sum(dK3 * K)
+    wait(8);
+    tc_fence_after();
     {
-        float dq[2][4][4];
-        zero2<4>(dq);
-        wgemm2<8, 2, false, true>(dq, sb + OC_DO, LQ, r0, sb + OC_S, LS, n128, lane, NoScale2());
+        float v[32], kd[16], gs[16], kv[16], t3 = 0.f;
+        tmem_ld16x2(tmem_addr(tb, q4, C_D + col0), tmem_addr(tb, q4, C_K1A + col0), v);
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dq[mi][nt][e] *= Gam[row(mi, e)];
-        wgemm2<4, 2, false, true>(dq, sb + OC_M, LDC, r0, sb + OC_K, LQ, n128, lane, NoScale2());
-        rowdot(dq, OC_Q, n128, pg);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                const int r = row(mi, 2 * hi);
-                if (c * C + r >= a.T) continue;
-                float *dst = a.dq + (((size_t)b * a.T + c * C + r) * a.Hk + hk) * D + n128 + 2 * t4;
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    if (sole) {
-                        *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(dq[mi][nt][2 * hi], dq[mi][nt][2 * hi + 1]);
-                    } else {
-                        atomicAdd(dst + 8 * nt, dq[mi][nt][2 * hi]);
-                        atomicAdd(dst + 8 * nt + 1, dq[mi][nt][2 * hi + 1]);
-                    }
-                }
-            }
-    }
-    // ---- f: dK3 = diag(f) U' dS_next^T (the start of dK)
-    float dk[2][4][4];
-    {
-        zero2<4>(dk);
-        wgemm2<8, 2, false, true>(dk, sb + OC_U, LDD, r0, sb + OC_DS, LS, n128, lane, NoScale2());
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dk[mi][nt][e] *= fv[row(mi, e)];
-        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        rowdot(dk, OC_K, n128, s);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) pg[mi][hi] -= s[mi][hi], tot3 += s[mi][hi];
-    }
-    // ---- g: dW = -dU' S^T, into the dS_next slot once every warp is done with it
-    {
-        float dw[2][4][4];
-        zero2<4>(dw);
-        wgemm2<8, 2, false, true>(dw, sb + OC_W, LDD, r0, sb + OC_S, LS, n128, lane, NoScale2());
-        __syncthreads();
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) store_h(dw[mi], mi, 4, OC_DS, LDD, n128, -1.f);
-    }
-    __syncthreads();
-    // ---- h: dV = diag(beta) T^T dU', and dK1's first part diag(Gamma beta) T^T dW
-    {
-        float y[2][4][4], y2[2][4][4];
-        zero2<4>(y);
-        zero2<4>(y2);
-        wgemm2_pair<4, 2, true, true, true, true, true, false>(y, sb + OC_T, LT, sb + OC_W, LDD, NoScale2(), y2,
-                                                               sb + OC_T, LT, sb + OC_DS, LDD, NoScale2(), r0, n128, lane);
-        rowdot(y, OC_V, n128, pb);   // rowsum(V * T^T dU')
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                const int r = row(mi, 2 * hi);
-                if (c * C + r >= a.T) continue;
-                const float br = beta[r];
-                float *dst = a.dv + (((size_t)b * a.T + c * C + r) * a.Hv + h) * D + n128 + 2 * t4;
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-                    *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(br * y[mi][nt][2 * hi], br * y[mi][nt][2 * hi + 1]);
-            }
-        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        rowdot(y2, OC_K, n128, s);   // rowsum(K * T^T dW)
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                const int r = row(mi, 2 * hi);
-                const float gr = Gam[r], gbr = gr * beta[r];
-                pb[mi][hi] += gr * s[mi][hi];
-                pg[mi][hi] += gbr * s[mi][hi];   // rowsum(dK1a * K)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    dk[mi][nt][2 * hi] += gbr * y2[mi][nt][2 * hi];
-                    dk[mi][nt][2 * hi + 1] += gbr * y2[mi][nt][2 * hi + 1];
-                }
-            }
-    }
-    // ---- i: dT = dU' V^T diag(beta) + dW K^T diag(beta Gamma), into the U' slot (dead after f)
-    {
-        float x1[2][2][4], x2[2][2][4];
-        zero2<2>(x1);
-        zero2<2>(x2);
-        wgemm2_pair<8, 1, false, false, false, false, false, false>(x1, sb + OC_W, LDD, sb + OC_V, LQ, NoScale2(), x2,
-                                                                    sb + OC_DS, LDD, sb + OC_K, LQ, NoScale2(), r0, n64, lane);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                    x1[mi][nt][e] = beta[i] * (x1[mi][nt][e] + Gam[i] * x2[mi][nt][e]);
-                }
-            store_h(x1[mi], mi, 2, OC_U, LDC, n64, 1.f);
+        for (int j = 0; j < 16; ++j) {
+            const int i = col0 + j;
+            kv[j] = colrd(O_K, j);
+            const float k3 = fv[i] * v[j], k1 = Gam[i] * beta[i] * v[16 + j];
+            kd[j] = k3 + k1;
+            gs[j] = kv[j] * (k1 - k3);
+            t3 = fmaf(k3, kv[j], t3);
+            v[j] = Gam[i] * kv[j] * v[16 + j];   // K * T^T dW, for dbeta
         }
-    }
-    __syncthreads();
-    // ---- j: X = T^T dT (into the S^T slot), then dA = strict tril(-X T^T)
-    {
-        float x[2][2][4];
-        zero2<2>(x);
-        wgemm2<4, 1, true, true>(x, sb + OC_T, LT, r0, sb + OC_U, LDC, n64, lane, NoScale2());
+        const float sb_ = warp_rs16(v, lane);
+        if (lane < 16) vec[W_DB + 64 * q4 + col0 + lane] += sb_;
+        tmem_ld16x2(tmem_addr(tb, q4, C_A + col0), tmem_addr(tb, q4, C_K2 + col0), v);
+        float *dst = a.dk + (((size_t)b * a.T + c * C + col0) * a.Hk + hk) * D + p;
+        const size_t stride = (size_t)a.Hk * D;
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) store_h(x[mi], mi, 2, OC_S, LDC, n64, 1.f);
-    }
-    __syncthreads();
-    {
-        float y[2][2][4];
-        zero2<2>(y);
-        wgemm2<4, 1, false, false>(y, sb + OC_S, LDC, r0, sb + OC_T, LT, n64, lane, NoScale2());
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = row(mi, e), i = n64 + 8 * nt + 2 * t4 + (e & 1);
-                    const float dA = r > i ? -y[mi][nt][e] : 0.f;
-                    pb[mi][e >> 1] += dA * __half2float(bmm[r * LDC + i]);
-                    y[mi][nt][e] = beta[r] * dA * __half2float(decm[r * LDC + i]);   // dB * D
-                }
-            store_h(y[mi], mi, 2, OC_U, LDC, n64, 1.f);   // dT is dead (read for X)
-        }
-    }
-    __syncthreads();
-    // ---- k: dK1 += (dB * D) K;  dK2 = (dM * D)^T Q + (dB * D)^T K
-    {
-        float p[2][4][4];
-        zero2<4>(p);
-        wgemm2<4, 2, false, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LQ, n128, lane, NoScale2());
-        rowdot(p, OC_K, n128, pg);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dk[mi][nt][e] += p[mi][nt][e];
-        zero2<4>(p);
-        wgemm2<4, 2, true, true>(p, sb + OC_M, LDC, r0, sb + OC_Q, LQ, n128, lane, NoScale2());
-        wgemm2<4, 2, true, true>(p, sb + OC_U, LDC, r0, sb + OC_K, LQ, n128, lane, NoScale2());
-        float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        rowdot(p, OC_K, n128, s);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                pg[mi][hi] -= s[mi][hi];
-                const int r = row(mi, 2 * hi);
-                if (c * C + r >= a.T) continue;
-                float *dst = a.dk + (((size_t)b * a.T + c * C + r) * a.Hk + hk) * D + n128 + 2 * t4;
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const float k0 = dk[mi][nt][2 * hi] + p[mi][nt][2 * hi], k1 = dk[mi][nt][2 * hi + 1] + p[mi][nt][2 * hi + 1];
-                    if (sole) {
-                        *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(k0, k1);
-                    } else {
-                        atomicAdd(dst + 8 * nt, k0);
-                        atomicAdd(dst + 8 * nt + 1, k1);
-                    }
-                }
-            }
-    }
-    // ---- l: row sums over the warps, then dg (reverse cumulative sum) and dbeta
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-#pragma unroll
-            for (int o = 1; o < 4; o <<= 1) {
-                pg[mi][hi] += __shfl_xor_sync(0xffffffffu, pg[mi][hi], o);
-                pb[mi][hi] += __shfl_xor_sync(0xffffffffu, pb[mi][hi], o);
-            }
-            if (t4 == 0) {
-                vec[VDG + 64 * cw + row(mi, 2 * hi)] = pg[mi][hi];
-                vec[VDB + 64 * cw + row(mi, 2 * hi)] = pb[mi][hi];
+        for (int j = 0; j < 16; ++j) {
+            const int i = col0 + j;
+            const float x = kd[j] + v[j] + v[16 + j];
+            gs[j] = fmaf(kv[j], v[j] - v[16 + j], gs[j]);
+            if (i < nvalid) {
+                if (sole) dst[j * stride] = x;
+                else atomicAdd(dst + j * stride, x);
             }
         }
-    tot3 = warp_sum(tot3);
-    if (lane == 0) vec[VT3 + warp] = tot3;
+        const float sg = warp_rs16(gs, lane);
+        if (lane < 16) vec[W_DG + 64 * q4 + col0 + lane] += sg;
+        t3 = warp_sum(t3);
+        if (lane == 0) vec[W_T3 + warp] = t3;
+    }
+    tc_fence_before();
     __syncthreads();
+    // ---- dg (reverse cumulative sum of the row sums of dG) and dbeta
     if (warp == 0) {
         float t3 = 0.f, ss = 0.f;
 #pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) t3 += vec[VT3 + w8], ss += vec[VSS + w8];
-        auto dgrow = [&](int r) { return ((vec[VDG + r] + vec[VDG + 64 + r]) + vec[VDG + 128 + r]) + vec[VDG + 192 + r]; };
-        auto dbrow = [&](int r) { return ((vec[VDB + r] + vec[VDB + 64 + r]) + vec[VDB + 128 + r]) + vec[VDB + 192 + r]; };
-        // rows 63 - lane and 31 - lane: an inclusive scan over the lanes is the reverse sum
+        for (int w = 0; w < NTT / 32; ++w) t3 += vec[W_T3 + w], ss += vec[W_SS + w];
+        auto dgrow = [&](int r) {
+            return ((vec[W_DG + r] + vec[W_DG + 64 + r]) + vec[W_DG + 128 + r]) + vec[W_DG + 192 + r];
+        };
+        auto dbrow = [&](int r) {
+            return (((vec[W_DB + r] + vec[W_DB + 64 + r]) + vec[W_DB + 128 + r]) + vec[W_DB + 192 + r]) +
+                   (((vec[W_DA + r] + vec[W_DA + 64 + r]) + vec[W_DA + 128 + r]) + vec[W_DA + 192 + r]);
+        };
         const float extra = t3 + __expf(G[C - 1]) * ss;
         const int rA = 63 - lane, rB = 31 - lane;
         float x0 = dgrow(rA) + (lane == 0 ? extra : 0.f), x1 = dgrow(rB);
@@ -858,14 +864,25 @@ bwdc_chunk_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant_
         }
         x1 += __shfl_sync(0xffffffffu, x0, 31);
         const size_t base = (size_t)b * a.T + c * C;
-        if (c * C + rA < a.T) {
+        if (rA < nvalid) {
             a.dg[(base + rA) * a.Hv + h] = x0;
             a.dbeta[(base + rA) * a.Hv + h] = dbrow(rA);
         }
-        if (c * C + rB < a.T) {
+        if (rB < nvalid) {
             a.dg[(base + rB) * a.Hv + h] = x1;
             a.dbeta[(base + rB) * a.Hv + h] = dbrow(rB);
         }
+    }
+    if (tid == 0) {   // every product this thread issued has completed before the memory is freed
+        tc_fence_after();
+        mma_commit(bar(9));
+        mbar_wait_bounded(bar(9), 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tb, 512);
     }
 }
 
@@ -907,13 +924,13 @@ cudaError_t launch_bwdc(const BwdArgs &a, void *workspace, cudaStream_t st)
     bwdc_scan_kernel<<<(unsigned)(a.B * a.Hv), NT, SMEM_SCAN, st>>>(a, ws, mdo);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwdc_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_CHUNK);
+    e = cudaFuncSetAttribute(bwdc_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, a.B, a.T, a.Hk, 64, false, true) || !make_map(&mk, a.k, a.B, a.T, a.Hk, 64, false, true) ||
         !make_map(&mv, a.v, a.B, a.T, a.Hv, 64, false, true))
         return cudaErrorInvalidValue;
-    bwdc_chunk_kernel<<<(unsigned)cu, NTC, SMEM_CHUNK, st>>>(a, ws, sm_count(), a.Hv == a.Hk ? 1 : 0, mq, mk, mv, mdo);
+    bwdc_tc_kernel<<<(unsigned)cu, NTT, SMEM_TC, st>>>(a, ws, sm_count(), a.Hv == a.Hk ? 1 : 0, mq, mk, mv, mdo);
     return cudaGetLastError();
 }
 
