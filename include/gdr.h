@@ -130,12 +130,14 @@ GDR_API int gdr_bwd(const void *q, const void *k, const void *v, const float *g,
  * in the workspace; a reverse scan over the chunks carries the state gradient
  * dS <- Gamma_C dS + P^T dS + Qh^T dout, the transposed chunk map, and stores it per
  * chunk; then every chunk forms its own gradients from its entering state, the
- * gradient of the state it leaves, dout and its inputs, all chunks at once. The
- * products take fp16 operands with fp32 accumulation (the forward's precision), so
- * results are of the forward's accuracy class (about 1e-3 relative), not fp32:
- * gdr_bwd is the fp32 path. q, k, v, dout and the states must stay inside the fp16
- * range. dq and dk are sums over CTAs (atomics), so they are repeatable to
- * rounding only.
+ * gradient of the state it leaves, dout and its inputs, all chunks at once. All
+ * three passes run their products on the tcgen05 tensor cores with fp16 operands
+ * and fp32 accumulation (the forward's precision), so results are of the
+ * forward's accuracy class (about 1e-3 relative), not fp32: gdr_bwd is the fp32
+ * path. q, k, v, dout and the states must stay inside the fp16 range. dv, dg,
+ * dbeta and dh0 repeat bit for bit; so do dq and dk when Hv == Hk (one writer per
+ * row). With grouped value heads dq and dk are sums over the value heads' work
+ * (atomics), repeatable to rounding only.
  *
  * workspace: device buffer of at least gdr_bwd_chunked_workspace_size(...) bytes
  * (B * Hv * ceil(T / 64) * 120 KiB), owned by the caller; two calls that overlap

@@ -96,6 +96,17 @@ def test_repeatable():
         assert rel_err(a[n], b[n].double().cpu().numpy()) <= 1e-5, n
 
 
+def test_repeatable_with_one_value_head_per_key_head():
+    """With Hv == Hk every dq and dk row has one writer (plain stores, no atomics): every
+    gradient repeats bit for bit, ragged last chunk included."""
+    w = WORKLOADS["gdn_bf16"].with_(B=2, T=200, Hk=2, Hv=2, seed=917)
+    inp, do, dhT, a = run(w, 7)
+    b = gdr.gdr_bwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do, dhT)
+    torch.cuda.synchronize()
+    for n in NAMES:
+        assert torch.equal(a[n], b[n]), n
+
+
 def test_rejects_the_per_channel_gate():
     w = WORKLOADS["gdn_bf16"].with_(B=1, T=16, Hk=1, Hv=1, gate="channel", seed=916)
     inp = make_inputs(w, DEV)
