@@ -100,7 +100,8 @@ def gdr_kernel_launches() -> int:
 
 
 def gdr_fused_error_counts():
-    """(load_timeouts, range_errors) of the fused kernel on the current device; see include/gdr.h."""
+    """(load_timeouts, range_errors) of the tensor-core chunked forward and backward kernels on the
+    current device; see include/gdr.h."""
     t, r = ctypes.c_uint(0), ctypes.c_uint(0)
     lib().gdr_fused_error_counts(ctypes.byref(t), ctypes.byref(r))
     return int(t.value), int(r.value)

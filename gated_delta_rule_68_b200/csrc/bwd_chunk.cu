@@ -94,6 +94,15 @@ constexpr uint32_t ID_SQ = tcu::idesc_f16(128, 128, false, true, false);   // dO
 constexpr uint32_t ID_SP = tcu::idesc_f16(128, 128, false, false, true);   // dS^T P
 
 __device__ unsigned int g_bwdc_timeouts;
+// Work whose gradients came out inf or NaN: scan units (their dh0) and chunk CTAs (their dq,
+// dk, dv, dg, dbeta). An fp16 operand that overflowed (an input, a stored chunk map, the
+// state gradient's copy or a tile formed from them) leaves every product it enters
+// non-finite, and every product reaches a gradient, so checking the gradients finds it.
+// Threads fold x * 0 (0 for finite x, NaN otherwise): the scan over the dh0 values it
+// stores, the chunk kernel over the row sums of dq * q, dk * k and dv * v that its epilogues
+// form (every stored element enters one, and a non-finite term never cancels: inf * 0 and
+// inf - inf are NaN) and over dg and dbeta.
+__device__ unsigned int g_bwdc_range_errors;
 
 // Global -> L2 prefetches: a 16-byte aligned span of a multiple of 16 bytes.
 __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes)
@@ -124,10 +133,11 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
     const int NC = (a.T + C - 1) / C;
     auto bar = [&](int i) { return sb + SC_BAR + 8 * i; };   // 0, 1: loads; 2: products; 3: drain
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + SC_BAR + 32);
-    __shared__ int abort_sh;
+    __shared__ int abort_sh, range_sh;
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) mbar_init(bar(i), 1);
         abort_sh = 0;
+        range_sh = 0;
     }
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
     tc_fence_before();
@@ -237,8 +247,13 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
     }
     {   // dh0 = dS entering chunk 0
         float *dst = a.dh0 + (size_t)unit * D * D + (size_t)(64 * hf) * D + p;
+        float nf = 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) dst[(size_t)i * D] = dS[i];
+        for (int i = 0; i < 64; ++i) {
+            dst[(size_t)i * D] = dS[i];
+            nf = fmaf(dS[i], 0.f, nf);
+        }
+        if (nf != 0.f) range_sh = 1;
     }
     if (tid == 0) {   // every product this thread issued has completed before the memory is freed
         tc_fence_after();
@@ -251,6 +266,7 @@ __global__ void __launch_bounds__(NT, 1) bwdc_scan_kernel(BwdArgs a, BwdcWs ws, 
         tc_fence_after();
         tmem_dealloc(tb, 256);
     }
+    if (tid == 0 && range_sh) atomicAdd(&g_bwdc_range_errors, 1u);
 }
 
 // ------------------------------------------------------------------ pass 3: per-chunk gradients
@@ -394,11 +410,13 @@ bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ C
     float *vec = reinterpret_cast<float *>(sm + O_VEC);
     auto bar = [&](int i) { return sb + O_BAR + 8 * i; };   // 0, 1: loads; 2-8: products; 9: drain
     __shared__ uint32_t tmem_sh;
-    __shared__ int abort_sh;
+    __shared__ int abort_sh, range_sh;
     if (tid == 0) {
         for (int i = 0; i < NB_TC; ++i) mbar_init(bar(i), 1);
         abort_sh = 0;
+        range_sh = 0;
     }
+    float nf = 0.f;   // x * 0 folded over the gradients this thread stores (NaN if one is not finite)
     if (warp == 0) tmem_alloc(smem_u32(&tmem_sh), 512);
     tc_fence_before();
     __syncthreads();
@@ -690,6 +708,7 @@ bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ C
         }
         const float s = warp_rs16(dv, lane);
         if (lane < 16) vec[W_DB + 64 * q4 + col0 + lane] = s;
+        nf = fmaf(s, 0.f, nf);
     }
     // dQ = diag(Gamma) dO S^T + (dM * D) K (from the two accumulators, which no later batch
     // overwrites) and rowsum(dQ * Q)
@@ -710,6 +729,7 @@ bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ C
         }
         const float s = warp_rs16(v, lane);
         if (lane < 16) vec[W_DG + 64 * q4 + col0 + lane] = s;
+        nf = fmaf(s, 0.f, nf);
     };
     // ---- epilogue 4: dT = (dU' V^T + dW K^T diag(Gamma)) diag(beta). The dW K^T block sits on
     // lanes 64-127, columns 64-127 of the stack, and goes to the dU' V^T block's threads through
@@ -837,6 +857,7 @@ bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ C
         }
         const float sg = warp_rs16(gs, lane);
         if (lane < 16) vec[W_DG + 64 * q4 + col0 + lane] += sg;
+        nf = fmaf(sg, 0.f, fmaf(sb_, 0.f, nf));
         t3 = warp_sum(t3);
         if (lane == 0) vec[W_T3 + warp] = t3;
     }
@@ -867,12 +888,15 @@ bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ C
         if (rA < nvalid) {
             a.dg[(base + rA) * a.Hv + h] = x0;
             a.dbeta[(base + rA) * a.Hv + h] = dbrow(rA);
+            nf = fmaf(x0, 0.f, fmaf(dbrow(rA), 0.f, nf));
         }
         if (rB < nvalid) {
             a.dg[(base + rB) * a.Hv + h] = x1;
             a.dbeta[(base + rB) * a.Hv + h] = dbrow(rB);
+            nf = fmaf(x1, 0.f, fmaf(dbrow(rB), 0.f, nf));
         }
     }
+    if (nf != 0.f) range_sh = 1;
     if (tid == 0) {   // every product this thread issued has completed before the memory is freed
         tc_fence_after();
         mma_commit(bar(9));
@@ -884,9 +908,20 @@ bwdc_tc_kernel(BwdArgs a, BwdcWs ws, int pf, int sole, const __grid_constant__ C
         tc_fence_after();
         tmem_dealloc(tb, 512);
     }
+    if (tid == 0 && range_sh) atomicAdd(&g_bwdc_range_errors, 1u);
 }
 
 }  // namespace
+
+unsigned int bwdc_error_counts(unsigned int *timeouts, unsigned int *range_errors)
+{
+    unsigned int t = 0, r = 0;
+    cudaMemcpyFromSymbol(&t, g_bwdc_timeouts, sizeof(t));
+    cudaMemcpyFromSymbol(&r, g_bwdc_range_errors, sizeof(r));
+    if (timeouts) *timeouts = t;
+    if (range_errors) *range_errors = r;
+    return t + r;
+}
 
 bool bwdc_supported(const BwdArgs &a)
 {

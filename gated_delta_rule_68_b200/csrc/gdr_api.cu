@@ -64,6 +64,11 @@ namespace gdr {
 int set_failure(int status, const char *msg) { return fail(status, "%s", msg); }
 }  // namespace gdr
 
+namespace gdr {
+// Device-side failure counts of the chunked backward (bwd_chunk.cu).
+unsigned int bwdc_error_counts(unsigned int *timeouts, unsigned int *range_errors);
+}  // namespace gdr
+
 extern "C" {
 
 int gdr_version(void) { return 300; }
@@ -78,6 +83,10 @@ unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *r
     gdr::fused_error_counts(&t, &r);
     t += gdr::tc_error_count();
     r += gdr::tc_range_error_count();
+    unsigned int bt = 0, br = 0;
+    gdr::bwdc_error_counts(&bt, &br);
+    t += bt;
+    r += br;
     if (load_timeouts) *load_timeouts = t;
     if (range_errors) *range_errors = r;
     return t + r;

@@ -168,6 +168,11 @@ GDR_API int gdr_bwd_chunked(const void *q, const void *k, const void *v, const f
  *                  state, A, M, the inverse, W, U, P, Qh), since a product
  *                  of an inf operand is never finite, or when an input was
  *                  inf or NaN; that unit's o and hT are not valid.
+ * The chunked backward (gdr_bwd_chunked) adds its own: load_timeouts counts its
+ * waits that gave up, range_errors its reverse-scan units whose dh0 and its
+ * (unit, chunk) work items whose dq, dk, dv, dg or dbeta came out inf or NaN (an
+ * fp16 operand that overflowed: an input, a stored chunk map, the state
+ * gradient's copy or a tile formed from them); those gradients are not valid.
  * Reads device memory, so it waits for prior work on the default stream.
  */
 GDR_API unsigned int gdr_fused_error_counts(unsigned int *load_timeouts, unsigned int *range_errors);

@@ -31,6 +31,13 @@ def test_header_declares_the_binding_exports():
     assert set(declared_symbols()) == set(gdr.EXPORTS)
 
 
+def test_library_resolves_every_symbol_at_load(L):
+    """Binding every symbol at load time (RTLD_NOW) fails on any reference the library leaves
+    undefined, such as an internal function declared with the wrong linkage, which a lazy load
+    would only reveal at its first call."""
+    ctypes.CDLL(gdr.LIB_PATH, mode=os.RTLD_NOW | os.RTLD_LOCAL)
+
+
 def test_library_exports_every_declared_symbol(L):
     for name in declared_symbols():
         assert hasattr(L, name), name

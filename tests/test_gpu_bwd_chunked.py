@@ -36,7 +36,9 @@ def run(w, seed, with_dhT=True):
 
 
 def check(w, seed, with_dhT=True):
+    before = gdr.gdr_fused_error_counts()
     inp, do, dhT, got = run(w, seed, with_dhT)
+    assert gdr.gdr_fused_error_counts() == before, "wait timeouts or range errors counted"
     ref = oracle.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do, dhT)
     for n in NAMES:
         err = rel_err(got[n], ref[n])
@@ -105,6 +107,26 @@ def test_repeatable_with_one_value_head_per_key_head():
     torch.cuda.synchronize()
     for n in NAMES:
         assert torch.equal(a[n], b[n]), n
+
+
+def test_fp16_overflow_is_counted():
+    """dout beyond the fp16 range (bf16 holds it) overflows the fp16 operands: the non-finite
+    gradients are counted as range errors, one per reverse-scan unit (its dh0) and one per
+    chunk work item, while the same inputs at unit scale count none."""
+    w = WORKLOADS["gdn_bf16"].with_(B=1, T=128, Hk=1, Hv=1, seed=918)
+    inp = make_inputs(w, DEV)
+    do, dhT = upstream(w, 8)
+    t0, r0 = gdr.gdr_fused_error_counts()
+    gdr.gdr_bwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do, dhT)
+    torch.cuda.synchronize()
+    assert gdr.gdr_fused_error_counts() == (t0, r0)
+    big = (do.float() * 3.0e4).to(torch.bfloat16)   # |x| up to about 1.2e5 > 65504
+    got = gdr.gdr_bwd_chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], big, dhT)
+    torch.cuda.synchronize()
+    t1, r1 = gdr.gdr_fused_error_counts()
+    assert t1 == t0
+    assert r1 - r0 == 1 + 2, (r0, r1)   # the unit's scan and its two chunks
+    assert not torch.isfinite(got["dh0"]).all()
 
 
 def test_rejects_the_per_channel_gate():
