@@ -52,3 +52,28 @@ def test_decode_oracle_sample_is_bounded():
     w = WORKLOADS["decode_bf16"].with_(Dk=16, Dv=16)
     cpu = bench.decode_oracle_sample(w, target_s=0.5)
     assert cpu["kind"] == "oracle" and cpu["value"] > 0 and cpu["seconds"] < 5.0
+
+
+def test_forward_roofline_bytes_match_the_hand_derived_table():
+    """The roofline denominators: algorithmic bytes per call (per step for decode) against the
+    table derived by hand for the five workloads (q and k once per key head, v and o once
+    per value head, g, beta, and h0 and hT once; decode: the state read and written once)."""
+    expect_mb = {"gdn_bf16": 287.3, "gva_gdn_bf16": 568.3, "kda_bf16": 1623.2, "decode_bf16": 1619.1}
+    for name, mb in expect_mb.items():
+        assert bench.algorithmic_bytes(WORKLOADS[name]) / 1e6 == pytest.approx(mb, abs=0.05), name
+    # nanochat GDN spelled out: 8 x 2048 tokens, 16 heads of 128, bf16 tensors, fp32 g/beta/states
+    n = 8 * 2048 * 16
+    by_hand = 4 * n * 128 * 2 + 2 * n * 4 + 2 * 8 * 16 * 128 * 128 * 4
+    assert bench.algorithmic_bytes(WORKLOADS["gdn_bf16"]) == by_hand
+
+
+def test_chunked_backward_tensor_flops_by_hand():
+    """Per (unit, 64-token chunk): the forward pass's products (Gram 128x64x128, W and U
+    128x64x64 each, R 128x128x64, Qh two 128x64x64, Uh 128x64x64, P 128x128x64, the state
+    batch 128x128x128 and 128x64x128), the scan's two (128x128x128, 128x128x64) and the chunk
+    kernel's 26.2 Mflop; 4096 chunk units on the nanochat shape."""
+    fwd = 2 * (128 * 64 * 128 + 2 * 128 * 64 * 64 + 128 * 128 * 64 + 2 * 128 * 64 * 64 + 128 * 64 * 64
+               + 128 * 128 * 64 + 128 * 128 * 128 + 128 * 64 * 128)
+    scan = 2 * (128 * 128 * 128 + 128 * 128 * 64)
+    chunk = 6400 * 2 * 16 * 8 * 16
+    assert bench.bwdc_flops(WORKLOADS["gdn_bwd_bf16"]) == 4096 * (fwd + scan + chunk)
